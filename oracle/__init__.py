@@ -1,0 +1,203 @@
+"""Float64 CPU oracle for the Hyena long-convolution operator.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  The
+CUDA product path never imports it, and the two share no code.
+
+The arithmetic lives in ``hyena_oracle.c`` (plain C, float64, a textbook
+radix-2 FFT and the direct O(L^2) sums); this module only compiles it with
+gcc and marshals numpy arrays through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hyena_oracle.c")
+_SO = os.path.join(_HERE, "_build", "libhyena_oracle.so")
+
+ROUTE_DIRECT = 0
+ROUTE_FFT = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/_build/libhyena_oracle.so``."""
+    if (not force and os.path.exists(_SO)
+            and os.path.getmtime(_SO) >= os.path.getmtime(_SRC)):
+        return _SO
+    os.makedirs(os.path.dirname(_SO), exist_ok=True)
+    tmp = _SO + f".tmp{os.getpid()}"
+    # -ffp-contract=off: no fused multiply-adds, every product is rounded
+    # to float64 exactly as written.
+    cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math",
+           "-fPIC", "-shared", "-o", tmp, _SRC, "-lm", "-lpthread"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, _SO)
+    return _SO
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    dp = ctypes.POINTER(ctypes.c_double)
+    i, l, d = ctypes.c_int, ctypes.c_long, ctypes.c_double
+    sigs = {
+        "oracle_filter_gen": [dp, dp, dp, dp, dp, i, i, i, i, i, d, i, dp],
+        "oracle_filter_gen_2d": [dp, dp, dp, dp, dp, i, i, i, i, i, i, d, i, dp],
+        "oracle_fft": [dp, dp, l, i],
+        "oracle_rfft_pad2": [dp, l, l, dp, dp],
+        "oracle_rfft2_pad2": [dp, l, l, l, dp, dp],
+        "oracle_conv": [dp, dp, l, i, dp],
+        "oracle_conv2": [dp, dp, l, l, i, dp],
+        "oracle_hyena_forward": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
+        "oracle_hyena_forward_2d": [dp, dp, dp, dp, l, l, l, l, l, i, i, dp],
+    }
+    for name, args in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _check(rc: int, name: str) -> None:
+    if rc != 0:
+        raise RuntimeError(f"{name} failed with status {rc}")
+
+
+def default_threads() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+def _route(route) -> int:
+    return {"direct": ROUTE_DIRECT, "fft": ROUTE_FFT}[route] if isinstance(route, str) else int(route)
+
+
+def filter_gen(W1, W2, W3, Wout, alpha, N, D, L, n_bands=8, width=64,
+               decay_div=64.0, threads=None) -> np.ndarray:
+    """Implicit filters h[N][D][L] (float64)."""
+    W1, W2, W3, Wout, alpha = map(_f64, (W1, W2, W3, Wout, alpha))
+    assert W1.shape == (width, 1 + 2 * n_bands) and Wout.shape == (N * D, width)
+    assert alpha.shape == (D,)
+    h = np.empty((N, D, L), dtype=np.float64)
+    rc = _load().oracle_filter_gen(_ptr(W1), _ptr(W2), _ptr(W3), _ptr(Wout),
+                                   _ptr(alpha), N, D, L, n_bands, width,
+                                   float(decay_div), threads or default_threads(),
+                                   _ptr(h))
+    _check(rc, "oracle_filter_gen")
+    return h
+
+
+def filter_gen_2d(W1, W2, W3, Wout, alpha, N, C, H, W, n_bands=8, width=64,
+                  decay_div=64.0, threads=None) -> np.ndarray:
+    """Implicit 2-D filters h[N][C][H][W] (float64)."""
+    W1, W2, W3, Wout, alpha = map(_f64, (W1, W2, W3, Wout, alpha))
+    assert W1.shape == (width, 2 + 4 * n_bands) and Wout.shape == (N * C, width)
+    assert alpha.shape == (C,)
+    h = np.empty((N, C, H, W), dtype=np.float64)
+    rc = _load().oracle_filter_gen_2d(_ptr(W1), _ptr(W2), _ptr(W3), _ptr(Wout),
+                                      _ptr(alpha), N, C, H, W, n_bands, width,
+                                      float(decay_div),
+                                      threads or default_threads(), _ptr(h))
+    _check(rc, "oracle_filter_gen_2d")
+    return h
+
+
+def fft(x, sign: int = -1) -> np.ndarray:
+    """Unnormalised DFT of a power-of-two length complex vector."""
+    x = np.asarray(x, dtype=np.complex128)
+    re, im = _f64(x.real).copy(), _f64(x.imag).copy()
+    _check(_load().oracle_fft(_ptr(re), _ptr(im), re.size, sign), "oracle_fft")
+    return re + 1j * im
+
+
+def rfft_pad2(h) -> np.ndarray:
+    """Bins 0..L of the DFT of each row of h[..., L] zero-padded to 2L."""
+    h = _f64(h)
+    L = h.shape[-1]
+    rows = h.size // L
+    re = np.empty(rows * (L + 1)); im = np.empty(rows * (L + 1))
+    _check(_load().oracle_rfft_pad2(_ptr(h), rows, L, _ptr(re), _ptr(im)),
+           "oracle_rfft_pad2")
+    return (re + 1j * im).reshape(h.shape[:-1] + (L + 1,))
+
+
+def rfft2_pad2(h) -> np.ndarray:
+    """2-D DFT of each h[..., H, W] zero-padded to 2H x 2W, columns 0..W."""
+    h = _f64(h)
+    H, W = h.shape[-2:]
+    rows = h.size // (H * W)
+    n = rows * 2 * H * (W + 1)
+    re = np.empty(n); im = np.empty(n)
+    _check(_load().oracle_rfft2_pad2(_ptr(h), rows, H, W, _ptr(re), _ptr(im)),
+           "oracle_rfft2_pad2")
+    return (re + 1j * im).reshape(h.shape[:-2] + (2 * H, W + 1))
+
+
+def conv(h, u, route="direct") -> np.ndarray:
+    """Causal convolution of one sequence: y[t] = sum_{s<=t} h[s] u[t-s]."""
+    h, u = _f64(h), _f64(u)
+    assert h.shape == u.shape and h.ndim == 1
+    y = np.empty_like(u)
+    _check(_load().oracle_conv(_ptr(h), _ptr(u), u.size, _route(route), _ptr(y)),
+           "oracle_conv")
+    return y
+
+
+def conv2(h, u, route="direct") -> np.ndarray:
+    """Causal (first-quadrant) 2-D convolution of one image."""
+    h, u = _f64(h), _f64(u)
+    assert h.shape == u.shape and h.ndim == 2
+    y = np.empty_like(u)
+    _check(_load().oracle_conv2(_ptr(h), _ptr(u), u.shape[0], u.shape[1],
+                                _route(route), _ptr(y)), "oracle_conv2")
+    return y
+
+
+def hyena_forward(v, x, h, bias, route="fft", threads=None) -> np.ndarray:
+    """y = z_N of the order-N recurrence.
+
+    v [B][D][L], x [N][B][D][L] (x_1..x_N stacked), h [N][D][L], bias [N][D].
+    """
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    B, D, L = v.shape
+    N = h.shape[0]
+    assert x.shape == (N, B, D, L) and h.shape == (N, D, L) and bias.shape == (N, D)
+    y = np.empty_like(v)
+    rc = _load().oracle_hyena_forward(_ptr(v), _ptr(x), _ptr(h), _ptr(bias),
+                                      B, D, L, N, _route(route),
+                                      threads or default_threads(), _ptr(y))
+    _check(rc, "oracle_hyena_forward")
+    return y
+
+
+def hyena_forward_2d(v, x, h, bias, route="fft", threads=None) -> np.ndarray:
+    """2-D recurrence: v [B][C][H][W], x [N][B][C][H][W], h [N][C][H][W],
+    bias [N][C] -> y [B][C][H][W]."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    B, C, H, W = v.shape
+    N = h.shape[0]
+    assert x.shape == (N, B, C, H, W) and h.shape == (N, C, H, W)
+    assert bias.shape == (N, C)
+    y = np.empty_like(v)
+    rc = _load().oracle_hyena_forward_2d(_ptr(v), _ptr(x), _ptr(h), _ptr(bias),
+                                         B, C, H, W, N, _route(route),
+                                         threads or default_threads(), _ptr(y))
+    _check(rc, "oracle_hyena_forward_2d")
+    return y

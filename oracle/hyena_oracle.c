@@ -1,0 +1,667 @@
+/*
+ * hyena_oracle.c -- plain float64 CPU oracle for the Hyena long-convolution
+ * operator (filter generation, causal long convolution, order-N gated
+ * recurrence, and the 2-D variant).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product (CUDA)
+ * path never links, loads or calls it, and the two share no code, header,
+ * table or constant generator.
+ *
+ * Sources (page title, section):
+ *  - "Hyena Hierarchy: Towards Larger Convolutional Language Models",
+ *    abstract: the operator interleaves implicitly parametrised long
+ *    convolutions with data-controlled (multiplicative) gating.  This file
+ *    reads that as the order-N recurrence
+ *        z_0 = v,   z_n = x_n * (h_n (*) z_{n-1} + b_n * z_{n-1}),   y = z_N
+ *    with (*) a per-channel causal convolution over the whole sequence and
+ *    b_n a per-channel bias (skip) term.
+ *  - "Long Context Language Models and their Biological Applications with
+ *    Eric Nguyen - #690", 4:29 (an MLP parametrises the filter), 5:48 (the
+ *    filter is as long as the input: a global convolution), 6:27 (the
+ *    convolution theorem: FFT both, multiply elementwise, transform back).
+ *  - "Native Multi-Dimensional Subquadratic Operators via Input Dependent
+ *    Long Convolutions", Methodology, "Native ND Convolution" (N-D FFT on the
+ *    grid) and "Handling Boundaries" (non-circular convolution by zero
+ *    padding to double the grid before the FFT).
+ *
+ * Readings where the pages are silent (the pages give no formulas):
+ *  - conv(h, u)[t] = sum_{s=0..t} h[s] u[t-s]: h[0] is the zero-lag tap,
+ *    no flip, no centring; the result is causal.
+ *  - The filter network: features phi(i) = [t, sin(2 pi k t), cos(2 pi k t)
+ *    for k = 1..K], t = i/L; three bias-free Linear+sin layers of the given
+ *    width; one bias-free linear head to N*D outputs; filter n, channel d is
+ *    head row n*D + d; times the window exp(-alpha_d * t * L / decay_div).
+ *  - 2-D: features [ty, tx, sin/cos(2 pi k ty) for k = 1..K,
+ *    sin/cos(2 pi k tx) for k = 1..K], ty = iy/H, tx = ix/W; the same FFN;
+ *    separable window exp(-alpha_c ty H / div) * exp(-alpha_c tx W / div).
+ *
+ * Every routine is written for clarity, not speed: loops in the order of the
+ * definition, a textbook iterative radix-2 FFT whose twiddles are taken
+ * from cos/sin of each angle in float64, no blocking, no fusion.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_PI 3.14159265358979323846
+
+enum { ORACLE_OK = 0, ORACLE_EBADARG = -1, ORACLE_ENOMEM = -2 };
+enum { ROUTE_DIRECT = 0, ROUTE_FFT = 1 };
+
+static int is_pow2(long n) { return n > 0 && (n & (n - 1)) == 0; }
+
+static long next_pow2(long n)
+{
+    long p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+/* ------------------------------------------------------------------ */
+/* Filter network (TWIML #690, 4:29: an MLP parametrises the filter).  */
+/* ------------------------------------------------------------------ */
+
+/* out[r] = sum_c W[r][c] * in[c]   (W row-major [rows][cols]) */
+static void matvec(const double *W, int rows, int cols, const double *in,
+                   double *out)
+{
+    for (int r = 0; r < rows; ++r) {
+        double s = 0.0;
+        for (int c = 0; c < cols; ++c) s += W[(long)r * cols + c] * in[c];
+        out[r] = s;
+    }
+}
+
+/* The FFN: three Linear+sin layers then a linear head. */
+static void ffn(const double *W1, const double *W2, const double *W3,
+                const double *Wout, int n_in, int width, int n_out,
+                const double *phi, double *a1, double *a2, double *a3,
+                double *o)
+{
+    matvec(W1, width, n_in, phi, a1);
+    for (int j = 0; j < width; ++j) a1[j] = sin(a1[j]);
+    matvec(W2, width, width, a1, a2);
+    for (int j = 0; j < width; ++j) a2[j] = sin(a2[j]);
+    matvec(W3, width, width, a2, a3);
+    for (int j = 0; j < width; ++j) a3[j] = sin(a3[j]);
+    matvec(Wout, n_out, width, a3, o);
+}
+
+typedef struct {
+    const double *W1, *W2, *W3, *Wout, *alpha;
+    int N, D, L, n_bands, width;
+    double decay_div;
+    double *h;
+    int i0, i1; /* positions handled by this worker */
+    int status;
+} fg_job;
+
+static void *filter_gen_worker(void *arg)
+{
+    fg_job *j = (fg_job *)arg;
+    const int n_in = 1 + 2 * j->n_bands;
+    const int n_out = j->N * j->D;
+    double *phi = malloc(sizeof(double) * n_in);
+    double *a1 = malloc(sizeof(double) * j->width);
+    double *a2 = malloc(sizeof(double) * j->width);
+    double *a3 = malloc(sizeof(double) * j->width);
+    double *o = malloc(sizeof(double) * n_out);
+    if (!phi || !a1 || !a2 || !a3 || !o) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (int i = j->i0; i < j->i1; ++i) {
+        const double t = (double)i / (double)j->L;
+        phi[0] = t;
+        for (int k = 1; k <= j->n_bands; ++k) {
+            phi[2 * k - 1] = sin(2.0 * ORACLE_PI * k * t);
+            phi[2 * k] = cos(2.0 * ORACLE_PI * k * t);
+        }
+        ffn(j->W1, j->W2, j->W3, j->Wout, n_in, j->width, n_out, phi, a1, a2,
+            a3, o);
+        for (int n = 0; n < j->N; ++n)
+            for (int d = 0; d < j->D; ++d) {
+                const double window =
+                    exp(-j->alpha[d] * t * (double)j->L / j->decay_div);
+                j->h[((long)n * j->D + d) * j->L + i] = o[n * j->D + d] * window;
+            }
+    }
+    j->status = ORACLE_OK;
+done:
+    free(phi); free(a1); free(a2); free(a3); free(o);
+    return NULL;
+}
+
+/* h[N][D][L] from the FFN weights (W1 [width][1+2K], W2, W3 [width][width],
+ * Wout [N*D][width], all row-major [out][in]) and the decay rates alpha[D]. */
+int oracle_filter_gen(const double *W1, const double *W2, const double *W3,
+                      const double *Wout, const double *alpha, int N, int D,
+                      int L, int n_bands, int width, double decay_div,
+                      int nthreads, double *h)
+{
+    if (!W1 || !W2 || !W3 || !Wout || !alpha || !h || N < 1 || D < 1 ||
+        L < 1 || n_bands < 0 || width < 1 || !(decay_div > 0.0))
+        return ORACLE_EBADARG;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > L) nthreads = L;
+    fg_job *jobs = calloc(nthreads, sizeof(fg_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        fg_job j = {W1, W2, W3, Wout, alpha, N, D, L, n_bands, width,
+                    decay_div, h, (int)((long)L * k / nthreads),
+                    (int)((long)L * (k + 1) / nthreads), 0};
+        jobs[k] = j;
+        pthread_create(&tid[k], NULL, filter_gen_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}
+
+typedef struct {
+    const double *W1, *W2, *W3, *Wout, *alpha;
+    int N, C, H, W, n_bands, width;
+    double decay_div;
+    double *h;
+    int p0, p1; /* flattened grid positions handled by this worker */
+    int status;
+} fg2_job;
+
+static void *filter_gen_2d_worker(void *arg)
+{
+    fg2_job *j = (fg2_job *)arg;
+    const int n_in = 2 + 4 * j->n_bands;
+    const int n_out = j->N * j->C;
+    const long HW = (long)j->H * j->W;
+    double *phi = malloc(sizeof(double) * n_in);
+    double *a1 = malloc(sizeof(double) * j->width);
+    double *a2 = malloc(sizeof(double) * j->width);
+    double *a3 = malloc(sizeof(double) * j->width);
+    double *o = malloc(sizeof(double) * n_out);
+    if (!phi || !a1 || !a2 || !a3 || !o) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (int p = j->p0; p < j->p1; ++p) {
+        const int iy = p / j->W, ix = p % j->W;
+        const double ty = (double)iy / (double)j->H;
+        const double tx = (double)ix / (double)j->W;
+        phi[0] = ty;
+        phi[1] = tx;
+        for (int k = 1; k <= j->n_bands; ++k) {
+            phi[2 * k] = sin(2.0 * ORACLE_PI * k * ty);
+            phi[2 * k + 1] = cos(2.0 * ORACLE_PI * k * ty);
+        }
+        for (int k = 1; k <= j->n_bands; ++k) {
+            phi[2 * j->n_bands + 2 * k] = sin(2.0 * ORACLE_PI * k * tx);
+            phi[2 * j->n_bands + 2 * k + 1] = cos(2.0 * ORACLE_PI * k * tx);
+        }
+        ffn(j->W1, j->W2, j->W3, j->Wout, n_in, j->width, n_out, phi, a1, a2,
+            a3, o);
+        for (int n = 0; n < j->N; ++n)
+            for (int c = 0; c < j->C; ++c) {
+                const double window =
+                    exp(-j->alpha[c] * ty * (double)j->H / j->decay_div) *
+                    exp(-j->alpha[c] * tx * (double)j->W / j->decay_div);
+                j->h[((long)n * j->C + c) * HW + p] = o[n * j->C + c] * window;
+            }
+    }
+    j->status = ORACLE_OK;
+done:
+    free(phi); free(a1); free(a2); free(a3); free(o);
+    return NULL;
+}
+
+/* h[N][C][H][W] from the FFN weights (W1 [width][2+4K]) and alpha[C]. */
+int oracle_filter_gen_2d(const double *W1, const double *W2, const double *W3,
+                         const double *Wout, const double *alpha, int N, int C,
+                         int H, int W, int n_bands, int width,
+                         double decay_div, int nthreads, double *h)
+{
+    if (!W1 || !W2 || !W3 || !Wout || !alpha || !h || N < 1 || C < 1 ||
+        H < 1 || W < 1 || n_bands < 0 || width < 1 || !(decay_div > 0.0))
+        return ORACLE_EBADARG;
+    const int HW = H * W;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > HW) nthreads = HW;
+    fg2_job *jobs = calloc(nthreads, sizeof(fg2_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        fg2_job j = {W1, W2, W3, Wout, alpha, N, C, H, W, n_bands, width,
+                     decay_div, h, (int)((long)HW * k / nthreads),
+                     (int)((long)HW * (k + 1) / nthreads), 0};
+        jobs[k] = j;
+        pthread_create(&tid[k], NULL, filter_gen_2d_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
+/* Naive iterative radix-2 FFT (TWIML #690, 6:27: the FFT route).      */
+/* ------------------------------------------------------------------ */
+
+/* In place, unnormalised: X[k] = sum_j x[j] exp(sign * 2 pi i j k / n).
+ * sign = -1 is the forward transform.  n must be a power of two. */
+static void fft_radix2(double *re, double *im, long n, int sign)
+{
+    /* bit-reversal permutation */
+    for (long i = 1, j = 0; i < n; ++i) {
+        long bit = n >> 1;
+        for (; j & bit; bit >>= 1) j ^= bit;
+        j ^= bit;
+        if (i < j) {
+            double t = re[i]; re[i] = re[j]; re[j] = t;
+            t = im[i]; im[i] = im[j]; im[j] = t;
+        }
+    }
+    /* log2(n) butterfly stages; the twiddle of each butterfly comes from
+     * cos/sin of its own angle */
+    for (long len = 2; len <= n; len <<= 1) {
+        const long half = len / 2;
+        for (long k = 0; k < half; ++k) {
+            const double ang = sign * 2.0 * ORACLE_PI * (double)k / (double)len;
+            const double wr = cos(ang), wi = sin(ang);
+            for (long s = 0; s < n; s += len) {
+                const long a = s + k, b = a + half;
+                const double tr = wr * re[b] - wi * im[b];
+                const double ti = wr * im[b] + wi * re[b];
+                re[b] = re[a] - tr;
+                im[b] = im[a] - ti;
+                re[a] += tr;
+                im[a] += ti;
+            }
+        }
+    }
+}
+
+/* Exposed for the oracle's own pins (closed forms, Parseval). */
+int oracle_fft(double *re, double *im, long n, int sign)
+{
+    if (!re || !im || !is_pow2(n) || (sign != 1 && sign != -1))
+        return ORACLE_EBADARG;
+    fft_radix2(re, im, n, sign);
+    return ORACLE_OK;
+}
+
+/* Spectrum of each row of h[rows][L] zero-padded to P = 2L (Handling
+ * Boundaries: pad to double the grid).  Keeps bins 0..L of the P-point DFT:
+ * out_re/out_im [rows][L+1].  P must be a power of two. */
+int oracle_rfft_pad2(const double *h, long rows, long L, double *out_re,
+                     double *out_im)
+{
+    const long P = 2 * L;
+    if (!h || !out_re || !out_im || rows < 0 || L < 1 || !is_pow2(P))
+        return ORACLE_EBADARG;
+    double *re = malloc(sizeof(double) * P), *im = malloc(sizeof(double) * P);
+    if (!re || !im) { free(re); free(im); return ORACLE_ENOMEM; }
+    for (long r = 0; r < rows; ++r) {
+        for (long t = 0; t < P; ++t) {
+            re[t] = t < L ? h[r * L + t] : 0.0;
+            im[t] = 0.0;
+        }
+        fft_radix2(re, im, P, -1);
+        for (long k = 0; k <= L; ++k) {
+            out_re[r * (L + 1) + k] = re[k];
+            out_im[r * (L + 1) + k] = im[k];
+        }
+    }
+    free(re); free(im);
+    return ORACLE_OK;
+}
+
+/* 2-D spectrum of each h[rows][H][W] zero-padded to 2H x 2W; keeps
+ * columns 0..W of every one of the 2H rows: out [rows][2H][W+1]. */
+int oracle_rfft2_pad2(const double *h, long rows, long H, long W,
+                      double *out_re, double *out_im)
+{
+    const long PH = 2 * H, PW = 2 * W;
+    if (!h || !out_re || !out_im || rows < 0 || H < 1 || W < 1 ||
+        !is_pow2(PH) || !is_pow2(PW))
+        return ORACLE_EBADARG;
+    double *re = malloc(sizeof(double) * PH * PW);
+    double *im = malloc(sizeof(double) * PH * PW);
+    double *cr = malloc(sizeof(double) * PH), *ci = malloc(sizeof(double) * PH);
+    if (!re || !im || !cr || !ci) {
+        free(re); free(im); free(cr); free(ci);
+        return ORACLE_ENOMEM;
+    }
+    for (long r = 0; r < rows; ++r) {
+        for (long y = 0; y < PH; ++y)
+            for (long x = 0; x < PW; ++x) {
+                re[y * PW + x] = (y < H && x < W) ? h[(r * H + y) * W + x] : 0.0;
+                im[y * PW + x] = 0.0;
+            }
+        for (long y = 0; y < PH; ++y) fft_radix2(re + y * PW, im + y * PW, PW, -1);
+        for (long x = 0; x < PW; ++x) {
+            for (long y = 0; y < PH; ++y) { cr[y] = re[y * PW + x]; ci[y] = im[y * PW + x]; }
+            fft_radix2(cr, ci, PH, -1);
+            for (long y = 0; y < PH; ++y) { re[y * PW + x] = cr[y]; im[y * PW + x] = ci[y]; }
+        }
+        for (long y = 0; y < PH; ++y)
+            for (long x = 0; x <= W; ++x) {
+                out_re[(r * PH + y) * (W + 1) + x] = re[y * PW + x];
+                out_im[(r * PH + y) * (W + 1) + x] = im[y * PW + x];
+            }
+    }
+    free(re); free(im); free(cr); free(ci);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Causal long convolution, two independent routes.                   */
+/* ------------------------------------------------------------------ */
+
+/* The definition: y[t] = sum_{s=0..t} h[s] u[t-s]. */
+static void conv_direct(const double *h, const double *u, long L, double *y)
+{
+    for (long t = 0; t < L; ++t) {
+        double s = 0.0;
+        for (long k = 0; k <= t; ++k) s += h[k] * u[t - k];
+        y[t] = s;
+    }
+}
+
+typedef struct { double *hr, *hi, *ur, *ui; long P; } fft_scratch;
+
+static int scratch_alloc(fft_scratch *s, long P)
+{
+    s->P = P;
+    s->hr = malloc(sizeof(double) * P); s->hi = malloc(sizeof(double) * P);
+    s->ur = malloc(sizeof(double) * P); s->ui = malloc(sizeof(double) * P);
+    return (s->hr && s->hi && s->ur && s->ui) ? ORACLE_OK : ORACLE_ENOMEM;
+}
+
+static void scratch_free(fft_scratch *s)
+{
+    free(s->hr); free(s->hi); free(s->ur); free(s->ui);
+}
+
+/* The convolution theorem route: zero-pad h and u to P >= 2L (a power of
+ * two, so no wrap-around reaches t < L), DFT both, multiply, inverse DFT,
+ * scale by 1/P, keep t < L. */
+static void conv_fft(const double *h, const double *u, long L, double *y,
+                     fft_scratch *s)
+{
+    const long P = s->P;
+    for (long t = 0; t < P; ++t) {
+        s->hr[t] = t < L ? h[t] : 0.0; s->hi[t] = 0.0;
+        s->ur[t] = t < L ? u[t] : 0.0; s->ui[t] = 0.0;
+    }
+    fft_radix2(s->hr, s->hi, P, -1);
+    fft_radix2(s->ur, s->ui, P, -1);
+    for (long k = 0; k < P; ++k) {
+        const double re = s->hr[k] * s->ur[k] - s->hi[k] * s->ui[k];
+        const double im = s->hr[k] * s->ui[k] + s->hi[k] * s->ur[k];
+        s->ur[k] = re;
+        s->ui[k] = im;
+    }
+    fft_radix2(s->ur, s->ui, P, +1);
+    for (long t = 0; t < L; ++t) y[t] = s->ur[t] / (double)P;
+}
+
+int oracle_conv(const double *h, const double *u, long L, int route, double *y)
+{
+    if (!h || !u || !y || L < 1) return ORACLE_EBADARG;
+    if (route == ROUTE_DIRECT) {
+        conv_direct(h, u, L, y);
+        return ORACLE_OK;
+    }
+    if (route != ROUTE_FFT) return ORACLE_EBADARG;
+    fft_scratch s;
+    if (scratch_alloc(&s, next_pow2(2 * L)) != ORACLE_OK) {
+        scratch_free(&s);
+        return ORACLE_ENOMEM;
+    }
+    conv_fft(h, u, L, y, &s);
+    scratch_free(&s);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* The order-N Hyena recurrence, 1-D.                                  */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const double *v, *x, *h, *bias;
+    long B, D, L, N;
+    int route;
+    double *y;
+    long s0, step; /* sequences s0, s0 + step, ... (s = b*D + d) */
+    int status;
+} fwd_job;
+
+static void *forward_worker(void *arg)
+{
+    fwd_job *j = (fwd_job *)arg;
+    const long L = j->L, BDL = j->B * j->D * L;
+    double *z = malloc(sizeof(double) * L), *c = malloc(sizeof(double) * L);
+    fft_scratch s = {0};
+    if (!z || !c || (j->route == ROUTE_FFT &&
+                     scratch_alloc(&s, next_pow2(2 * L)) != ORACLE_OK)) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (long seq = j->s0; seq < j->B * j->D; seq += j->step) {
+        const long d = seq % j->D;
+        memcpy(z, j->v + seq * L, sizeof(double) * L); /* z_0 = v */
+        for (long n = 0; n < j->N; ++n) {
+            const double *hn = j->h + (n * j->D + d) * L;
+            const double *xn = j->x + n * BDL + seq * L;
+            const double bn = j->bias[n * j->D + d];
+            if (j->route == ROUTE_DIRECT) conv_direct(hn, z, L, c);
+            else conv_fft(hn, z, L, c, &s);
+            /* z_n = x_n * (h_n (*) z_{n-1} + b_n z_{n-1}) */
+            for (long t = 0; t < L; ++t) z[t] = xn[t] * (c[t] + bn * z[t]);
+        }
+        memcpy(j->y + seq * L, z, sizeof(double) * L); /* y = z_N */
+    }
+    j->status = ORACLE_OK;
+done:
+    free(z); free(c);
+    if (j->route == ROUTE_FFT) scratch_free(&s);
+    return NULL;
+}
+
+/* v [B][D][L], x [N][B][D][L], h [N][D][L], bias [N][D] -> y [B][D][L]. */
+int oracle_hyena_forward(const double *v, const double *x, const double *h,
+                         const double *bias, long B, long D, long L, long N,
+                         int route, int nthreads, double *y)
+{
+    if (!v || !x || !h || !bias || !y || B < 1 || D < 1 || L < 1 || N < 1 ||
+        (route != ROUTE_DIRECT && route != ROUTE_FFT))
+        return ORACLE_EBADARG;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > B * D) nthreads = (int)(B * D);
+    fwd_job *jobs = calloc(nthreads, sizeof(fwd_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        fwd_job j = {v, x, h, bias, B, D, L, N, route, y, k, nthreads, 0};
+        jobs[k] = j;
+        pthread_create(&tid[k], NULL, forward_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
+/* 2-D: linear convolution on the grid (Native ND Convolution;         */
+/* Handling Boundaries: zero-pad to double the grid).                  */
+/* ------------------------------------------------------------------ */
+
+/* The definition: y[p][q] = sum_{i<=p, j<=q} h[i][j] u[p-i][q-j]. */
+static void conv2_direct(const double *h, const double *u, long H, long W,
+                         double *y)
+{
+    for (long p = 0; p < H; ++p)
+        for (long q = 0; q < W; ++q) {
+            double s = 0.0;
+            for (long i = 0; i <= p; ++i)
+                for (long j = 0; j <= q; ++j)
+                    s += h[i * W + j] * u[(p - i) * W + (q - j)];
+            y[p * W + q] = s;
+        }
+}
+
+typedef struct {
+    double *hr, *hi, *ur, *ui, *cr, *ci;
+    long PH, PW;
+} fft2_scratch;
+
+static int scratch2_alloc(fft2_scratch *s, long PH, long PW)
+{
+    s->PH = PH; s->PW = PW;
+    s->hr = malloc(sizeof(double) * PH * PW); s->hi = malloc(sizeof(double) * PH * PW);
+    s->ur = malloc(sizeof(double) * PH * PW); s->ui = malloc(sizeof(double) * PH * PW);
+    s->cr = malloc(sizeof(double) * PH); s->ci = malloc(sizeof(double) * PH);
+    return (s->hr && s->hi && s->ur && s->ui && s->cr && s->ci) ? ORACLE_OK
+                                                               : ORACLE_ENOMEM;
+}
+
+static void scratch2_free(fft2_scratch *s)
+{
+    free(s->hr); free(s->hi); free(s->ur); free(s->ui); free(s->cr); free(s->ci);
+}
+
+/* 2-D DFT of a PH x PW row-major grid: every row, then every column. */
+static void fft2(double *re, double *im, fft2_scratch *s, int sign)
+{
+    const long PH = s->PH, PW = s->PW;
+    for (long y = 0; y < PH; ++y) fft_radix2(re + y * PW, im + y * PW, PW, sign);
+    for (long x = 0; x < PW; ++x) {
+        for (long y = 0; y < PH; ++y) { s->cr[y] = re[y * PW + x]; s->ci[y] = im[y * PW + x]; }
+        fft_radix2(s->cr, s->ci, PH, sign);
+        for (long y = 0; y < PH; ++y) { re[y * PW + x] = s->cr[y]; im[y * PW + x] = s->ci[y]; }
+    }
+}
+
+static void conv2_fft(const double *h, const double *u, long H, long W,
+                      double *y, fft2_scratch *s)
+{
+    const long PH = s->PH, PW = s->PW;
+    for (long r = 0; r < PH; ++r)
+        for (long q = 0; q < PW; ++q) {
+            const int in = r < H && q < W;
+            s->hr[r * PW + q] = in ? h[r * W + q] : 0.0; s->hi[r * PW + q] = 0.0;
+            s->ur[r * PW + q] = in ? u[r * W + q] : 0.0; s->ui[r * PW + q] = 0.0;
+        }
+    fft2(s->hr, s->hi, s, -1);
+    fft2(s->ur, s->ui, s, -1);
+    for (long k = 0; k < PH * PW; ++k) {
+        const double re = s->hr[k] * s->ur[k] - s->hi[k] * s->ui[k];
+        const double im = s->hr[k] * s->ui[k] + s->hi[k] * s->ur[k];
+        s->ur[k] = re;
+        s->ui[k] = im;
+    }
+    fft2(s->ur, s->ui, s, +1);
+    for (long r = 0; r < H; ++r)
+        for (long q = 0; q < W; ++q)
+            y[r * W + q] = s->ur[r * PW + q] / (double)(PH * PW);
+}
+
+int oracle_conv2(const double *h, const double *u, long H, long W, int route,
+                 double *y)
+{
+    if (!h || !u || !y || H < 1 || W < 1) return ORACLE_EBADARG;
+    if (route == ROUTE_DIRECT) {
+        conv2_direct(h, u, H, W, y);
+        return ORACLE_OK;
+    }
+    if (route != ROUTE_FFT) return ORACLE_EBADARG;
+    fft2_scratch s;
+    if (scratch2_alloc(&s, next_pow2(2 * H), next_pow2(2 * W)) != ORACLE_OK) {
+        scratch2_free(&s);
+        return ORACLE_ENOMEM;
+    }
+    conv2_fft(h, u, H, W, y, &s);
+    scratch2_free(&s);
+    return ORACLE_OK;
+}
+
+typedef struct {
+    const double *v, *x, *h, *bias;
+    long B, C, H, W, N;
+    int route;
+    double *y;
+    long s0, step; /* images s0, s0 + step, ... (s = b*C + c) */
+    int status;
+} fwd2_job;
+
+static void *forward_2d_worker(void *arg)
+{
+    fwd2_job *j = (fwd2_job *)arg;
+    const long HW = j->H * j->W, BCHW = j->B * j->C * HW;
+    double *z = malloc(sizeof(double) * HW), *c = malloc(sizeof(double) * HW);
+    fft2_scratch s = {0};
+    if (!z || !c || (j->route == ROUTE_FFT &&
+                     scratch2_alloc(&s, next_pow2(2 * j->H),
+                                    next_pow2(2 * j->W)) != ORACLE_OK)) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (long img = j->s0; img < j->B * j->C; img += j->step) {
+        const long ch = img % j->C;
+        memcpy(z, j->v + img * HW, sizeof(double) * HW);
+        for (long n = 0; n < j->N; ++n) {
+            const double *hn = j->h + (n * j->C + ch) * HW;
+            const double *xn = j->x + n * BCHW + img * HW;
+            const double bn = j->bias[n * j->C + ch];
+            if (j->route == ROUTE_DIRECT) conv2_direct(hn, z, j->H, j->W, c);
+            else conv2_fft(hn, z, j->H, j->W, c, &s);
+            for (long p = 0; p < HW; ++p) z[p] = xn[p] * (c[p] + bn * z[p]);
+        }
+        memcpy(j->y + img * HW, z, sizeof(double) * HW);
+    }
+    j->status = ORACLE_OK;
+done:
+    free(z); free(c);
+    if (j->route == ROUTE_FFT) scratch2_free(&s);
+    return NULL;
+}
+
+/* v [B][C][H][W], x [N][B][C][H][W], h [N][C][H][W], bias [N][C]
+ * -> y [B][C][H][W]. */
+int oracle_hyena_forward_2d(const double *v, const double *x, const double *h,
+                            const double *bias, long B, long C, long H, long W,
+                            long N, int route, int nthreads, double *y)
+{
+    if (!v || !x || !h || !bias || !y || B < 1 || C < 1 || H < 1 || W < 1 ||
+        N < 1 || (route != ROUTE_DIRECT && route != ROUTE_FFT))
+        return ORACLE_EBADARG;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > B * C) nthreads = (int)(B * C);
+    fwd2_job *jobs = calloc(nthreads, sizeof(fwd2_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        fwd2_job j = {v, x, h, bias, B, C, H, W, N, route, y, k, nthreads, 0};
+        jobs[k] = j;
+        pthread_create(&tid[k], NULL, forward_2d_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}
