@@ -1,0 +1,388 @@
+"""Benchmark of the Hyena FFT-conv + gate path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c1] [--impl reference]
+
+One step = one pass of the whole path over one batch of synthetic input:
+implicit filter generation (hyena_filter_gen), the filter spectra
+(hyena_filter_rfft, computed once and shared by the whole batch) and the
+fused order-N forward (hyena_fftconv_gate_forward).  The metric is
+channel-positions per second (B * D * L per step).  Device time comes from
+CUDA events on the launching stream; L2 is flushed (a 256 MB write) before
+every timed step, outside the timed events.  Under torchrun every rank runs
+the same workload on its own GPU (the channel-sequences are independent, so
+the ranks share no data: weak scaling) and rank 0 prints one JSON line with
+the max time over ranks.
+
+--impl reference times the float64 CPU oracle on the host cores on a
+bounded sample of the same workload (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from subquadratic_sequence_b200 import synth  # noqa: E402
+
+METRIC = "Hyena FFT-conv+gate fwd: channel-positions/s and % of B200 HBM roofline"
+UNIT = "channel-positions/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def describe(wl: synth.Workload) -> dict:
+    return {"workload": f"{wl.name}: order-{wl.N} Hyena 1-D operator, B={wl.B}, D={wl.D}, "
+                        f"L={wl.L}, {wl.io} storage, fp32 compute",
+            "N": wl.N, "B": wl.B, "D": wl.D, "L": wl.L, "io": wl.io,
+            "filters": f"implicit FFN (3 sine layers of width {synth.WIDTH}, {synth.N_BANDS} bands) "
+                       "x exponential decay, regenerated every step",
+            "l2": "flushed (256 MB write) before every timed step"}
+
+
+def alg_bytes_forward(wl: synth.Workload) -> int:
+    """Algorithmic HBM bytes of one fused forward: v, x_1..x_N, y plus the
+    N*D packed spectra (L complex64 slots each)."""
+    return (wl.N + 2) * wl.B * wl.D * wl.L * wl.io_bytes + wl.N * wl.D * wl.L * 8
+
+
+def peaks() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "subquadratic_sequence_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` on `workload` from the committed ncu
+    summary, if it was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)[f"{kernel}@{workload}"]
+    except Exception:
+        return None
+    return rec["dram_bytes_per_launch"] if rec.get("source_hash") == kernel_source_hash() else None
+
+
+# ----------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1])); mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ GPU arm
+
+def run_gpu(args, wl: synth.Workload) -> dict | None:
+    import torch
+    import torch.distributed as dist
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the path has no CPU fallback)")
+    from subquadratic_sequence_b200 import hyena
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    inp = synth.make_inputs(wl)
+    io = torch.bfloat16 if wl.io == "bf16" else torch.float32
+
+    def to_dev(a, dtype=torch.float32):
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda().to(dtype)
+
+    v = to_dev(inp["v"], io)
+    xs = [to_dev(x, io) for x in inp["x"]]
+    b = to_dev(inp["b"])
+    W = [to_dev(inp[k]) for k in ("W1", "W2", "W3", "Wout", "alpha")]
+    h = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.float32)
+    H = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.complex64)
+    y = torch.empty_like(v)
+    flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hyena.hyena_filter_gen(*W, wl.N, wl.D, wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                               decay_div=synth.DECAY_DIV, out=h)
+        hyena.hyena_filter_rfft(h, out=H)
+        hyena.hyena_fftconv_gate_forward(v, xs, b, H=H, out=y)
+
+    launches_per_step = 3
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed steps (device time; L2 flushed before each, outside the events)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    gpu_uuid = str(torch.cuda.get_device_properties(local).uuid)
+    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+    with ClockSampler(gpu_id) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        wall = time.perf_counter() - t_wall
+        # keep sampling clocks over the same work when the timed region was
+        # shorter than a few samples
+        t_end = time.perf_counter() + max(0.0, 1.5 - wall)
+        while time.perf_counter() < t_end:
+            for _ in range(20):
+                flush.zero_()
+                step()
+            torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(bb) for a, bb in ev]
+    total_ms = max_over_ranks(sum(step_ms))
+
+    # ---- the dominant kernel alone: the fused forward, per launch
+    fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(max(args.steps, 10))]
+    hyena.hyena_filter_gen(*W, wl.N, wl.D, wl.L, out=h)
+    hyena.hyena_filter_rfft(h, out=H)
+    for i in range(len(fev)):
+        flush.zero_()
+        fev[i][0].record(stream)
+        hyena.hyena_fftconv_gate_forward(v, xs, b, H=H, out=y)
+        fev[i][1].record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = max_over_ranks(statistics.mean(a.elapsed_time(bb) for a, bb in fev))
+
+    # ---- end to end through the C ABI with host buffers: H2D of the step's
+    # inputs from pinned memory, the step, D2H of the result
+    hv = torch.from_numpy(np.ascontiguousarray(inp["v"], np.float32)).to(io).pin_memory()
+    hxs = [torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(io).pin_memory() for x in inp["x"]]
+    hb = torch.from_numpy(inp["b"]).pin_memory()
+    hW = [torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
+          for k in ("W1", "W2", "W3", "Wout", "alpha")]
+    hy_out = torch.empty(y.shape, dtype=io).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in [hv, *hxs, hb, *hW])
+    d2h = hy_out.numel() * hy_out.element_size()
+    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        eev[i][0].record(stream)
+        v.copy_(hv, non_blocking=True)
+        for xd, xh in zip(xs, hxs):
+            xd.copy_(xh, non_blocking=True)
+        b.copy_(hb, non_blocking=True)
+        for wd, wh in zip(W, hW):
+            wd.copy_(wh, non_blocking=True)
+        step()
+        hy_out.copy_(y, non_blocking=True)
+        eev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(bb) for a, bb in eev))
+
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    positions = wl.positions * world
+    value = positions * args.steps / (total_ms / 1e3)
+    peak, peak_kind = peaks()
+    achieved = alg_bytes_forward(wl) / (fwd_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": describe(wl),
+        "roofline": {"bound": "hbm", "kernel": "fused1d_kernel (hyena_fftconv_gate_forward)",
+                     "achieved": achieved, "peak": peak, "peak_source": peak_kind,
+                     "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": ncu_traffic("fused1d_kernel", wl.name),
+                     "alg_bytes_per_launch": alg_bytes_forward(wl), "ms_per_launch": fwd_ms},
+        "forward_only": {"value": wl.positions * world / (fwd_ms / 1e3), "unit": UNIT},
+        "e2e": {"value": positions * args.steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
+    return line
+
+
+# ------------------------------------------------------- oracle (CPU)
+
+def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: int) -> float:
+    """Seconds the oracle takes for the whole path (filter generation for the
+    sampled channels, then the order-N forward by its FFT route) on all B
+    batch elements of the sampled channels."""
+    import oracle
+    rows = np.concatenate([n * wl.D + channels for n in range(wl.N)])
+    t0 = time.perf_counter()
+    h = oracle.filter_gen(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
+                          wl.N, len(channels), wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                          decay_div=synth.DECAY_DIV, threads=threads)
+    v = inp["v"][:, channels].astype(np.float64)
+    x = np.stack([xx[:, channels] for xx in inp["x"]]).astype(np.float64)
+    oracle.hyena_forward(v, x, h, inp["b"][:, channels].astype(np.float64), route="fft",
+                         threads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl: synth.Workload, budget_s: float = 15.0, inp: dict | None = None) -> dict:
+    import oracle
+    inp = inp or synth.make_inputs(wl)
+    threads = oracle.default_threads()
+    rng = np.random.default_rng(0)
+    n = max(1, min(wl.D, threads))
+    t = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
+    # grow the sample to about budget_s of CPU work
+    n2 = int(min(wl.D, max(n, n * budget_s / max(t, 1e-3))))
+    if n2 > n:
+        n = n2
+        t = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
+    positions = wl.B * n * wl.L
+    return {"value": positions / t, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {wl.D} channels x all {wl.B} batch elements x L={wl.L} "
+                      f"(filter generation + order-{wl.N} forward, float64 FFT route), {t:.1f} s"}
+
+
+def run_reference(args, wl: synth.Workload) -> dict | None:
+    """The reference arm: the float64 CPU oracle, each step a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import oracle
+    inp = synth.make_inputs(wl)
+    threads = oracle.default_threads()
+    rng = np.random.default_rng(0)
+    n = max(1, min(wl.D, threads))
+    probe = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
+    # size each step so that warm-up + timed steps end within ~2 minutes
+    per_step_budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(min(wl.D, max(1, n * per_step_budget / max(probe, 1e-3))))
+    chans = [np.sort(rng.choice(wl.D, n, replace=False)) for _ in range(args.steps + args.warmup)]
+    for i in range(args.warmup):
+        oracle_sample(wl, inp, chans[i], threads)
+    total = sum(oracle_sample(wl, inp, chans[args.warmup + i], threads) for i in range(args.steps))
+    positions = wl.B * n * wl.L
+    value = positions * args.steps / total
+    sample = (f"{n} of {wl.D} channels x all {wl.B} batch elements x L={wl.L} per step "
+              f"(filter generation + order-{wl.N} forward, float64 FFT route)")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": describe(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="c1", choices=[k for k, w in synth.WORKLOADS.items()
+                                                         if w.kind == "1d" and w.L <= 16384])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("bench.py: at least 3 warm-up steps are required")
+    wl = synth.WORKLOADS[args.workload]
+    line = run_reference(args, wl) if args.impl == "reference" else run_gpu(args, wl)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

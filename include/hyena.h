@@ -1,0 +1,165 @@
+/*
+ * hyena.h -- C ABI of the B200 (sm_100a) Hyena long-convolution library.
+ *
+ * The operator ("Hyena Hierarchy: Towards Larger Convolutional Language
+ * Models", abstract: implicitly parametrised long convolutions interleaved
+ * with data-controlled gating), read as the order-N recurrence, per batch
+ * element b and channel d:
+ *
+ *     z_0 = v,   z_n = x_n * (h_n (*) z_{n-1} + b_n * z_{n-1}),   y = z_N
+ *
+ * where (*) is the causal linear convolution over the whole sequence,
+ *     (h (*) u)[t] = sum_{s=0..t} h[s] u[t-s],
+ * computed through the convolution theorem ("Long Context Language Models
+ * and their Biological Applications with Eric Nguyen - #690", 6:27) on a
+ * grid zero-padded to twice its size ("Native Multi-Dimensional
+ * Subquadratic Operators via Input Dependent Long Convolutions", Handling
+ * Boundaries), and b_n is a per-channel bias (skip) term.
+ *
+ * Conventions for every entry point:
+ *  - All array arguments are DEVICE pointers unless stated otherwise; the
+ *    caller allocates and owns every buffer and the stream.  The library
+ *    never allocates device memory and never synchronises the stream.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  A returned HYENA_OK means the work was
+ *    enqueued; kernel faults surface on the stream like any CUDA error.
+ *  - Arrays are dense, row-major, C order, the last index fastest.
+ *    Complex arrays hold interleaved (re, im) float pairs (complex64).
+ *  - Argument errors are detected on the host before anything is enqueued
+ *    and return HYENA_ERR_INVALID_ARG (or HYENA_ERR_UNSUPPORTED for valid
+ *    but unimplemented shapes); the GPU is not touched.  A failed launch
+ *    returns HYENA_ERR_CUDA; hyena_last_cuda_error() then gives the
+ *    cudaError_t value (per calling thread).
+ *  - The only global state is per-device kernel attributes (the shared
+ *    memory opt-in), set on first use.  Calls are otherwise reentrant.
+ *  - v, x_n and y (the activations) may be float32 or bf16 (io); filters,
+ *    spectra, biases and filter-network weights are always float32.  All
+ *    arithmetic is float32; bf16 outputs are rounded to nearest even.
+ */
+#ifndef HYENA_B200_H
+#define HYENA_B200_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define HYENA_API __attribute__((visibility("default")))
+#else
+#define HYENA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HYENA_OK = 0,
+    HYENA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misalignment, aliasing */
+    HYENA_ERR_UNSUPPORTED = 2,  /* valid arguments this build does not implement */
+    HYENA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+    HYENA_ERR_CUDA = 4          /* a CUDA call or launch failed */
+} hyena_status_t;
+
+typedef enum { HYENA_F32 = 0, HYENA_BF16 = 1 } hyena_dtype_t;
+
+/* Largest order N accepted by the forward calls. */
+#define HYENA_MAX_ORDER 16
+/* Largest 1-D length L (a power of two) accepted by the forward calls. */
+#define HYENA_MAX_LEN (1 << 22)
+
+/* The implicit filter network ("Long Context Language Models ... #690",
+ * 4:29: an MLP parametrises the filter).  Reading adopted here: positional
+ * features
+ *   1-D: phi(i) = [t, sin(2 pi k t), cos(2 pi k t) for k = 1..n_bands],
+ *        t = i/L, so n_in = 1 + 2 n_bands;
+ *   2-D: phi(iy, ix) = [ty, tx, sin/cos(2 pi k ty) for k = 1..n_bands,
+ *        sin/cos(2 pi k tx) for k = 1..n_bands], ty = iy/H, tx = ix/W,
+ *        so n_in = 2 + 4 n_bands;
+ * three bias-free layers a1 = sin(W1 phi), a2 = sin(W2 a1), a3 = sin(W3 a2)
+ * of `width` units, a bias-free head o = Wout a3 with N*D outputs, and the
+ * window exp(-alpha_d * i / decay_div) (2-D: exp(-alpha_c (iy+ix)/decay_div)).
+ * Filter n of channel d is head row n*D + d.
+ * All weight arrays are device float32, row-major [out][in]:
+ *   W1 [width][n_in], W2 [width][width], W3 [width][width],
+ *   Wout [N*D][width], alpha [D].
+ * Limits: 1 <= width <= 64, 0 <= n_bands <= 16, decay_div > 0. */
+typedef struct {
+    const float* W1;
+    const float* W2;
+    const float* W3;
+    const float* Wout;
+    const float* alpha;
+    int n_bands;
+    int width;
+    float decay_div;
+} hyena_ffn_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+HYENA_API const char* hyena_status_string(hyena_status_t status);
+
+/* cudaError_t of the last HYENA_ERR_CUDA returned on this thread (0 if
+ * none). */
+HYENA_API int hyena_last_cuda_error(void);
+
+/* ---------------------------------------------------------------- 1-D */
+
+/* Implicit filters h [N][D][L] float32 from the filter network (see
+ * hyena_ffn_t).  Any L >= 1.  ffn is a HOST pointer to the struct; the
+ * arrays it names are device pointers. */
+HYENA_API hyena_status_t hyena_filter_gen(const hyena_ffn_t* ffn, int N, int D, int L,
+                                float* h, void* stream);
+
+/* Filter spectra H [N][D][L] complex64 in the PACKED real-DFT layout: for
+ * each h[n][d] zero-padded to 2L ("Handling Boundaries": pad to double the
+ * grid so the product of spectra is a linear, non-circular convolution),
+ * its 2L-point DFT X has L+1 distinct bins X[0..L]; X[0] and X[L] are real,
+ * so they share slot 0 as (X[0], X[L]) and slot k holds X[k] for
+ * 1 <= k < L.  Rows are L * 8 bytes (16-byte aligned rows).
+ * h is [N][D][L] float32.  L is a power of two, 16 <= L <= 16384.
+ * Alignment: h 8 bytes, H 16 bytes.  H must not overlap h.
+ * The spectrum depends only on the filters: compute it once and reuse it
+ * for every batch and every call. */
+HYENA_API hyena_status_t hyena_filter_rfft(const float* h, int N, int D, int L,
+                                 float* H, void* stream);
+
+/* Bytes of workspace hyena_fftconv_gate_forward needs for these sizes
+ * (0 when none).  spectrum_given = 1 when the caller passes the cached
+ * spectrum H; 0 when it passes the filters h and the spectrum is computed
+ * into the workspace first.  Returns (size_t)-1 for invalid sizes. */
+HYENA_API size_t hyena_fftconv_workspace_size(int B, int D, int L, int N,
+                                    hyena_dtype_t io, int spectrum_given);
+
+/* The fused order-N forward (the recurrence above) over B*D
+ * channel-sequences of length L, one launch for all N orders:
+ *   v      [B][D][L] io            input z_0
+ *   x      HOST array of N device pointers, each [B][D][L] io (x_1..x_N)
+ *   h      [N][D][L] float32 filters, or NULL when H is given
+ *   H      [N][D][L] packed complex64 spectra (hyena_filter_rfft), or NULL
+ *          when h is given; H wins when both are given
+ *   bias   [N][D] float32 (b_n)
+ *   y      [B][D][L] io output z_N; must not overlap any input or the
+ *          workspace
+ *   workspace / ws_bytes: device scratch of at least
+ *          hyena_fftconv_workspace_size(...) bytes, 256-byte aligned
+ *          (NULL / 0 when that size is 0)
+ * L is a power of two, 16 <= L <= 16384 in this build; 1 <= N <=
+ * HYENA_MAX_ORDER.  Alignment: v, x_n, y, H 16 bytes; h 8; bias 4.
+ * Returns HYENA_ERR_WORKSPACE if the workspace is too small. */
+HYENA_API hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x,
+                                          const float* h, const float* H,
+                                          const float* bias, int B, int D,
+                                          int L, int N, hyena_dtype_t io,
+                                          void* y, void* workspace,
+                                          size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- 2-D */
+
+/* Implicit 2-D filters h [N][C][H][W] float32 (features and window as in
+ * hyena_ffn_t, 2-D form; D = C).  Any H, W >= 1. */
+HYENA_API hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C,
+                                   int H, int W, float* h, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYENA_B200_H */

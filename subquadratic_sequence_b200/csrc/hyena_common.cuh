@@ -1,0 +1,256 @@
+// hyena_common.cuh -- register-level building blocks shared by the CUDA
+// kernels of the Hyena long-convolution path: complex arithmetic on float2,
+// compile-time twiddle multiplies, and an unrolled in-register DFT of a
+// power-of-two size R <= 32.
+//
+// The FFT route follows the convolution theorem as stated in "Long Context
+// Language Models and their Biological Applications with Eric Nguyen -
+// #690" (6:27): transform, multiply elementwise, transform back.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <type_traits>
+#include <utility>
+
+namespace hyena {
+
+// ------------------------------------------------------------------ utils
+
+template <typename F, int... Is>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>)
+{
+    (f(std::integral_constant<int, Is>{}), ...);
+}
+
+// Calls f(std::integral_constant<int, i>) for i = 0 .. N-1, fully unrolled.
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F&& f)
+{
+    static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+__host__ __device__ constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n / 2); }
+
+__host__ __device__ constexpr int bitrev(int i, int bits)
+{
+    int r = 0;
+    for (int b = 0; b < bits; ++b) r |= ((i >> b) & 1) << (bits - 1 - b);
+    return r;
+}
+
+// ---------------------------------------------------------------- complex
+
+__device__ __forceinline__ float2 cadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+__device__ __forceinline__ float2 csub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+__device__ __forceinline__ float2 cconj(float2 a) { return make_float2(a.x, -a.y); }
+__device__ __forceinline__ float2 cmul(float2 a, float2 b)
+{
+    return make_float2(fmaf(a.x, b.x, -a.y * b.y), fmaf(a.x, b.y, a.y * b.x));
+}
+// a * conj(b)
+__device__ __forceinline__ float2 cmulc(float2 a, float2 b)
+{
+    return make_float2(fmaf(a.x, b.x, a.y * b.y), fmaf(a.y, b.x, -a.x * b.y));
+}
+__device__ __forceinline__ float2 mul_i(float2 a) { return make_float2(-a.y, a.x); }   // a * i
+__device__ __forceinline__ float2 mul_mi(float2 a) { return make_float2(a.y, -a.x); }  // a * (-i)
+
+// ------------------------------------------------------ constant twiddles
+
+// cos(pi k / 32), k = 0..16 (first quadrant of the 64th roots of unity).
+__host__ __device__ constexpr float cos64_q1(int k)
+{
+    constexpr float t[17] = {
+        1.0f,
+        0.995184726672196886245f,
+        0.980785280403230449126f,
+        0.956940335732208864936f,
+        0.923879532511286756128f,
+        0.881921264348355029713f,
+        0.831469612302545237079f,
+        0.773010453362736960811f,
+        0.707106781186547524401f,
+        0.634393284163645498215f,
+        0.555570233019602224743f,
+        0.471396736825997648556f,
+        0.382683432365089771728f,
+        0.290284677254462367636f,
+        0.195090322016128267848f,
+        0.0980171403295606019942f,
+        0.0f};
+    return t[k];
+}
+
+// cos(2 pi q / 64) for any integer q.
+__host__ __device__ constexpr float cos64(int q)
+{
+    q = ((q % 64) + 64) % 64;
+    return q <= 16 ? cos64_q1(q)
+         : q <= 32 ? -cos64_q1(32 - q)
+         : q <= 48 ? -cos64_q1(q - 32)
+                   : cos64_q1(64 - q);
+}
+__host__ __device__ constexpr float sin64(int q) { return cos64(q - 16); }
+
+// a * exp(SIGN * 2 pi i Q / 64), specialised for the trivial angles.
+template <int Q, int SIGN>
+__device__ __forceinline__ float2 mul_w64(float2 a)
+{
+    constexpr int q = ((Q % 64) + 64) % 64;
+    if constexpr (q == 0) {
+        return a;
+    } else if constexpr (q == 32) {
+        return make_float2(-a.x, -a.y);
+    } else if constexpr (q == 16) {
+        return SIGN > 0 ? mul_i(a) : mul_mi(a);
+    } else if constexpr (q == 48) {
+        return SIGN > 0 ? mul_mi(a) : mul_i(a);
+    } else if constexpr (q % 16 == 8) {
+        // |cos| = |sin| = 1/sqrt(2): two adds and two multiplies
+        constexpr float c = cos64(q);
+        constexpr float s = SIGN * sin64(q);
+        constexpr float r = 0.707106781186547524401f;
+        constexpr float sc = c > 0 ? 1.0f : -1.0f;
+        constexpr float ss = s > 0 ? 1.0f : -1.0f;
+        return make_float2(r * (sc * a.x - ss * a.y), r * (ss * a.x + sc * a.y));
+    } else {
+        constexpr float c = cos64(q);
+        constexpr float s = SIGN * sin64(q);
+        return make_float2(fmaf(a.x, c, -a.y * s), fmaf(a.x, s, a.y * c));
+    }
+}
+
+// 0.0f that depends on `dep`: x - x is not folded under IEEE rules (it is
+// NaN for x = inf or NaN), so values computed from it cannot be scheduled
+// before `dep` exists.  Used to keep data-independent twiddle arithmetic
+// next to the data it multiplies instead of hoisted (and held in registers)
+// across whole FFT passes.
+__device__ __forceinline__ float zero_after(float dep) { return dep - dep; }
+
+// exp(SIGN * i * pi * num / den) with an exactly representable ratio.
+template <int SIGN>
+__device__ __forceinline__ float2 expi_pi(float ratio)
+{
+    float s, c;
+    sincospif(ratio, &s, &c);
+    return make_float2(c, SIGN * s);
+}
+
+// ----------------------------------------------------- in-register DFT
+
+// Unnormalised DFT of R complex values held in registers a[0..R-1]:
+//   X[k] = sum_j a[j] exp(SIGN 2 pi i j k / R),  natural order in and out.
+// Radix-2 decimation in frequency, fully unrolled, constant twiddles.
+//  ZERO_HI : a[R/2 .. R-1] are known to be zero (zero-padded input).
+//  HALF_OUT: only X[0 .. R/2-1] are needed; the others are left undefined.
+template <int R, int SIGN, bool ZERO_HI = false, bool HALF_OUT = false>
+__device__ __forceinline__ void dft(float2* a)
+{
+    static_assert(R >= 1 && R <= 32 && (R & (R - 1)) == 0, "radix");
+    if constexpr (R == 1) {
+        return;
+    } else {
+        constexpr int LOGR = ilog2(R);
+        static_for<LOGR>([&](auto st) {
+            constexpr int stage = decltype(st)::value;
+            constexpr int HALF = R >> (stage + 1);   // butterfly span
+            constexpr int TW = 64 / (2 * HALF);      // w_{2 HALF} = w64^TW
+            static_for<R / (2 * HALF)>([&](auto sb) {
+                constexpr int s = decltype(sb)::value * 2 * HALF;
+                static_for<HALF>([&](auto kk) {
+                    constexpr int k = decltype(kk)::value;
+                    if constexpr (ZERO_HI && stage == 0) {
+                        a[s + k + HALF] = mul_w64<k * TW, SIGN>(a[s + k]);
+                    } else if constexpr (HALF_OUT && HALF == 1) {
+                        a[s + k] = cadd(a[s + k], a[s + k + HALF]);
+                    } else {
+                        const float2 u = a[s + k], v = a[s + k + HALF];
+                        a[s + k] = cadd(u, v);
+                        a[s + k + HALF] = mul_w64<k * TW, SIGN>(csub(u, v));
+                    }
+                });
+            });
+        });
+        // the outputs sit in bit-reversed order: rename registers
+        float2 t[R];
+        static_for<R>([&](auto ii) {
+            constexpr int i = decltype(ii)::value;
+            if constexpr (!HALF_OUT || i < R / 2) t[i] = a[bitrev(i, LOGR)];
+        });
+        static_for<R>([&](auto ii) {
+            constexpr int i = decltype(ii)::value;
+            if constexpr (!HALF_OUT || i < R / 2) a[i] = t[i];
+        });
+    }
+}
+
+// a[r] *= w^r for r = 1..R-1 (w^0 = 1); powers by recurrence.
+template <int R>
+__device__ __forceinline__ void apply_twiddle_powers(float2* a, float2 w)
+{
+    if constexpr (R > 1) {
+        float2 wr = w;
+        static_for<R - 1>([&](auto ii) {
+            constexpr int r = decltype(ii)::value + 1;
+            a[r] = cmul(a[r], wr);
+            if constexpr (r < R - 1) wr = cmul(wr, w);
+        });
+    }
+}
+
+// ---------------------------------------------------------------- I/O
+
+// Storage types of v, x_n and y.  Two consecutive real samples are moved
+// as one element (one float2, or one bf16 pair).
+template <typename IO> struct IoPair;
+template <> struct IoPair<float> {
+    using T = float2;
+    static __device__ __forceinline__ float2 load_smem(const T* p) { return *p; }
+    static __device__ __forceinline__ float2 load(const T* p) { return __ldg(p); }
+    static __device__ __forceinline__ void store(T* p, float2 v) { *p = v; }
+};
+template <> struct IoPair<__nv_bfloat16> {
+    using T = __nv_bfloat162;
+    static __device__ __forceinline__ float2 load_smem(const T* p) { return __bfloat1622float2(*p); }
+    static __device__ __forceinline__ float2 load(const T* p)
+    {
+        return __bfloat1622float2(__ldg(p));
+    }
+    static __device__ __forceinline__ void store(T* p, float2 v)
+    {
+        *p = __floats2bfloat162_rn(v.x, v.y);  // round to nearest even
+    }
+};
+
+// ------------------------------------------------------- async copies
+
+// 16-byte global -> shared copy that completes asynchronously (no register
+// staging); cp_async_wait_all() blocks until this thread's copies landed.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+// Cooperative copy of `bytes` (a multiple of 16, both ends 16-byte
+// aligned) by `nthreads` threads; thread `t` issues every nthreads-th chunk.
+__device__ __forceinline__ void cp_async_row(void* smem_dst, const void* gmem_src, int bytes, int t,
+                                             int nthreads)
+{
+    char* d = static_cast<char*>(smem_dst);
+    const char* s = static_cast<const char*>(gmem_src);
+    for (int i = t * 16; i < bytes; i += nthreads * 16) cp_async16(d + i, s + i);
+}
+
+// Shared-memory index with one float2 of padding per 16: strided Stockham
+// writes then hit distinct banks.
+__device__ __forceinline__ int pad16(int i) { return i + (i >> 4); }
+__host__ __device__ constexpr int padded_size(int n) { return n + n / 16; }
+
+}  // namespace hyena

@@ -1,0 +1,175 @@
+"""Thin ctypes binding of ``libhyena_b200.so`` (the C ABI in include/hyena.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Tensors are torch CUDA tensors used as device memory; the work is
+enqueued on the current torch stream unless a stream is given.  There is no
+fallback: if the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+HYENA_OK = 0
+HYENA_ERR_INVALID_ARG = 1
+HYENA_ERR_UNSUPPORTED = 2
+HYENA_ERR_WORKSPACE = 3
+HYENA_ERR_CUDA = 4
+HYENA_F32 = 0
+HYENA_BF16 = 1
+HYENA_MAX_ORDER = 16
+
+
+class HyenaError(RuntimeError):
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn}: {message}")
+        self.status = status
+
+
+class hyena_ffn_t(ctypes.Structure):
+    _fields_ = [("W1", ctypes.c_void_p), ("W2", ctypes.c_void_p), ("W3", ctypes.c_void_p),
+                ("Wout", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("n_bands", ctypes.c_int), ("width", ctypes.c_int), ("decay_div", ctypes.c_float)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_build.LIB):
+        raise ImportError(
+            f"{_build.LIB} is missing: build the CUDA library first "
+            "(python -m subquadratic_sequence_b200.build)")
+    lib = ctypes.CDLL(_build.LIB)
+    vp, i, sz, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    ffn_p = ctypes.POINTER(hyena_ffn_t)
+    sigs = {
+        "hyena_status_string": ([i], ctypes.c_char_p),
+        "hyena_last_cuda_error": ([], i),
+        "hyena_filter_gen": ([ffn_p, i, i, i, vp, vp], i),
+        "hyena_filter_gen_2d": ([ffn_p, i, i, i, i, vp, vp], i),
+        "hyena_filter_rfft": ([vp, i, i, i, vp, vp], i),
+        "hyena_fftconv_workspace_size": ([i, i, i, i, i, i], sz),
+        "hyena_fftconv_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp, vp,
+                                        sz, vp], i),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(status: int) -> str:
+    return LIB.hyena_status_string(status).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != HYENA_OK:
+        msg = status_string(status)
+        if status == HYENA_ERR_CUDA:
+            msg += f" (cudaError {LIB.hyena_last_cuda_error()})"
+        raise HyenaError(fn, status, msg)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, dtype, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def io_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return HYENA_F32
+    if t.dtype == torch.bfloat16:
+        return HYENA_BF16
+    raise TypeError(f"activations must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ffn(W1, W2, W3, Wout, alpha, n_bands, width, decay_div) -> hyena_ffn_t:
+    f32 = torch.float32
+    return hyena_ffn_t(_dev(W1, f32, "W1"), _dev(W2, f32, "W2"), _dev(W3, f32, "W3"),
+                       _dev(Wout, f32, "Wout"), _dev(alpha, f32, "alpha"),
+                       n_bands, width, float(decay_div))
+
+
+def hyena_filter_gen(W1, W2, W3, Wout, alpha, N: int, D: int, L: int, *, n_bands: int = 8,
+                     width: int = 64, decay_div: float = 64.0, out=None, stream=None):
+    """Implicit filters h [N][D][L] float32."""
+    f = _ffn(W1, W2, W3, Wout, alpha, n_bands, width, decay_div)
+    if out is None:
+        out = torch.empty((N, D, L), device=W1.device, dtype=torch.float32)
+    _check("hyena_filter_gen", LIB.hyena_filter_gen(
+        ctypes.byref(f), N, D, L, ctypes.c_void_p(_dev(out, torch.float32, "h")), _stream(stream)))
+    return out
+
+
+def hyena_filter_gen_2d(W1, W2, W3, Wout, alpha, N: int, C: int, H: int, W: int, *,
+                        n_bands: int = 8, width: int = 64, decay_div: float = 64.0, out=None,
+                        stream=None):
+    """Implicit 2-D filters h [N][C][H][W] float32."""
+    f = _ffn(W1, W2, W3, Wout, alpha, n_bands, width, decay_div)
+    if out is None:
+        out = torch.empty((N, C, H, W), device=W1.device, dtype=torch.float32)
+    _check("hyena_filter_gen_2d", LIB.hyena_filter_gen_2d(
+        ctypes.byref(f), N, C, H, W, ctypes.c_void_p(_dev(out, torch.float32, "h")),
+        _stream(stream)))
+    return out
+
+
+def hyena_filter_rfft(h: torch.Tensor, *, out=None, stream=None):
+    """Packed spectra [N][D][L] complex64 (slot 0 = (bin 0, bin L)) of the
+    filters h [N][D][L] zero-padded to 2L."""
+    N, D, L = h.shape
+    if out is None:
+        out = torch.empty((N, D, L), device=h.device, dtype=torch.complex64)
+    _check("hyena_filter_rfft", LIB.hyena_filter_rfft(
+        ctypes.c_void_p(_dev(h, torch.float32, "h")), N, D, L,
+        ctypes.c_void_p(_dev(out, torch.complex64, "H")), _stream(stream)))
+    return out
+
+
+def hyena_fftconv_workspace_size(B: int, D: int, L: int, N: int, io: int,
+                                 spectrum_given: bool) -> int:
+    n = LIB.hyena_fftconv_workspace_size(B, D, L, N, io, int(bool(spectrum_given)))
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv_workspace_size", HYENA_ERR_INVALID_ARG, "invalid sizes")
+    return n
+
+
+def hyena_fftconv_gate_forward(v: torch.Tensor, xs, bias: torch.Tensor, *, H=None, h=None,
+                               out=None, workspace=None, stream=None):
+    """y = z_N of the order-N recurrence for v [B][D][L] (float32 or bf16),
+    xs = [x_1 .. x_N] (same shape and dtype), bias [N][D] float32 and either
+    the packed spectra H [N][D][L] complex64 or the filters h [N][D][L]."""
+    B, D, L = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    Hp = ctypes.c_void_p(_dev(H, torch.complex64, "H")) if H is not None else None
+    hp = ctypes.c_void_p(_dev(h, torch.float32, "h")) if h is not None else None
+    ws_need = hyena_fftconv_workspace_size(B, D, L, N, io, H is not None)
+    if ws_need and workspace is None:
+        workspace = torch.empty(ws_need, device=v.device, dtype=torch.uint8)
+    wp = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+    wn = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("hyena_fftconv_gate_forward", LIB.hyena_fftconv_gate_forward(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, hp, Hp,
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), wp, wn, _stream(stream)))
+    return out

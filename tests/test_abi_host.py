@@ -1,0 +1,162 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol
+that include/hyena.h declares, and rejects bad arguments on the host before
+anything is enqueued.
+
+Every call below that passes placeholder device addresses is built to fail
+validation (a null, misaligned, aliased, oversized or unsupported argument),
+so none of them can reach a kernel launch on any machine.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from subquadratic_sequence_b200 import build as hbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+F32, BF16 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hbuild.build()
+    from subquadratic_sequence_b200 import hyena
+    return hyena.LIB
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"HYENA_API[^;(]*?\b(hyena_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for required in ("hyena_filter_gen", "hyena_filter_rfft", "hyena_fftconv_gate_forward",
+                     "hyena_fftconv_workspace_size", "hyena_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.hyena_status_string(s)
+    assert b"unknown" in lib.hyena_status_string(99)
+
+
+def test_workspace_size(lib):
+    from subquadratic_sequence_b200 import hyena
+    B, D, L, N = 8, 768, 2048, 2
+    assert hyena.hyena_fftconv_workspace_size(B, D, L, N, BF16, True) == 0
+    need = hyena.hyena_fftconv_workspace_size(B, D, L, N, BF16, False)
+    assert need >= N * D * L * 8 and need % 256 == 0
+    bad = ctypes.c_size_t(-1).value
+    assert lib.hyena_fftconv_workspace_size(B, D, 1000, N, F32, 1) == bad
+    assert lib.hyena_fftconv_workspace_size(B, D, L, 0, F32, 1) == bad
+    assert lib.hyena_fftconv_workspace_size(B, D, L, N, 7, 1) == bad
+
+
+# placeholder device addresses (never dereferenced: every call fails validation)
+A = 0x7F0000000000          # 256-byte aligned
+BIG = 1 << 30
+
+
+def P(k):
+    return ctypes.c_void_p(A + k * BIG)
+
+
+def fwd(lib, v=P(0), xs=(P(1), P(2)), h=None, H=P(3), bias=P(4), B=2, D=3, L=64, N=None,
+        io=F32, y=P(5), ws=None, wsb=0):
+    N = len(xs) if N is None else N
+    arr = (ctypes.c_void_p * max(len(xs), 1))(*[x.value if x is not None else None for x in xs])
+    xp = None if xs is None else arr
+    return lib.hyena_fftconv_gate_forward(v, xp, h, H, bias, B, D, L, N, io, y, ws, wsb, None)
+
+
+def test_forward_rejects_bad_arguments(lib):
+    assert fwd(lib, v=None) == INVALID
+    assert fwd(lib, y=None) == INVALID
+    assert fwd(lib, bias=None) == INVALID
+    assert fwd(lib, H=None, h=None) == INVALID
+    assert fwd(lib, xs=(P(1), None)) == INVALID
+    assert fwd(lib, B=0) == INVALID
+    assert fwd(lib, D=-1) == INVALID
+    assert fwd(lib, L=0) == INVALID
+    assert fwd(lib, N=0) == INVALID
+    assert fwd(lib, io=5) == INVALID
+    # valid but not implemented
+    assert fwd(lib, L=1000) == UNSUPPORTED
+    assert fwd(lib, L=8) == UNSUPPORTED
+    assert fwd(lib, L=1 << 23) == UNSUPPORTED
+    xs17 = tuple(P(10 + i) for i in range(17))
+    assert fwd(lib, xs=xs17) == UNSUPPORTED
+    # misalignment
+    assert fwd(lib, v=ctypes.c_void_p(A + 8)) == INVALID
+    assert fwd(lib, y=ctypes.c_void_p(A + 5 * BIG + 4)) == INVALID
+    assert fwd(lib, xs=(P(1), ctypes.c_void_p(A + 2 * BIG + 8))) == INVALID
+    assert fwd(lib, H=ctypes.c_void_p(A + 3 * BIG + 8)) == INVALID
+    assert fwd(lib, bias=ctypes.c_void_p(A + 4 * BIG + 2)) == INVALID
+    # aliasing: y overlapping an input
+    assert fwd(lib, y=P(0)) == INVALID
+    assert fwd(lib, y=ctypes.c_void_p(A + 2 * BIG + 256)) == INVALID
+    assert fwd(lib, y=P(3)) == INVALID
+    # filters instead of spectra need a workspace
+    assert fwd(lib, H=None, h=P(3)) == WORKSPACE
+    assert fwd(lib, H=None, h=P(3), ws=P(6), wsb=16) == WORKSPACE
+    assert fwd(lib, H=None, h=P(3), ws=ctypes.c_void_p(A + 6 * BIG + 16), wsb=1 << 20) == WORKSPACE
+    # workspace overlapping y
+    assert fwd(lib, H=None, h=P(3), ws=P(5), wsb=1 << 20) == INVALID
+
+
+def test_filter_rfft_rejects_bad_arguments(lib):
+    r = lib.hyena_filter_rfft
+    assert r(None, 2, 3, 64, P(1), None) == INVALID
+    assert r(P(0), 2, 3, 64, None, None) == INVALID
+    assert r(P(0), 0, 3, 64, P(1), None) == INVALID
+    assert r(P(0), 2, 3, 0, P(1), None) == INVALID
+    assert r(P(0), 2, 3, 48, P(1), None) == UNSUPPORTED
+    assert r(P(0), 2, 3, 1 << 15, P(1), None) == UNSUPPORTED
+    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + BIG + 8), None) == INVALID
+    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + 256), None) == INVALID   # H overlaps h
+
+
+def _ffn(lib, **kw):
+    from subquadratic_sequence_b200.hyena import hyena_ffn_t
+    f = dict(W1=A, W2=A + BIG, W3=A + 2 * BIG, Wout=A + 3 * BIG, alpha=A + 4 * BIG,
+             n_bands=8, width=64, decay_div=64.0)
+    f.update(kw)
+    return hyena_ffn_t(**f)
+
+
+def test_filter_gen_rejects_bad_arguments(lib):
+    g = lib.hyena_filter_gen
+    assert g(None, 2, 3, 64, P(5), None) == INVALID
+    assert g(ctypes.byref(_ffn(lib, W2=None)), 2, 3, 64, P(5), None) == INVALID
+    assert g(ctypes.byref(_ffn(lib, width=0)), 2, 3, 64, P(5), None) == INVALID
+    assert g(ctypes.byref(_ffn(lib, width=65)), 2, 3, 64, P(5), None) == UNSUPPORTED
+    assert g(ctypes.byref(_ffn(lib, n_bands=17)), 2, 3, 64, P(5), None) == UNSUPPORTED
+    assert g(ctypes.byref(_ffn(lib, decay_div=0.0)), 2, 3, 64, P(5), None) == INVALID
+    assert g(ctypes.byref(_ffn(lib)), 2, 3, 0, P(5), None) == INVALID
+    assert g(ctypes.byref(_ffn(lib)), 2, 3, 64, None, None) == INVALID
+    assert g(ctypes.byref(_ffn(lib, alpha=A + 4 * BIG + 2)), 2, 3, 64, P(5), None) == INVALID
+    g2 = lib.hyena_filter_gen_2d
+    assert g2(ctypes.byref(_ffn(lib)), 2, 3, 0, 8, P(5), None) == INVALID
+    assert g2(ctypes.byref(_ffn(lib, width=100)), 2, 3, 8, 8, P(5), None) == UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from subquadratic_sequence_b200 import hyena
+    v = torch.zeros(1, 1, 16)
+    with pytest.raises(TypeError):
+        hyena.hyena_fftconv_gate_forward(v, [v], torch.zeros(1, 1), H=torch.zeros(1, 1, 16, dtype=torch.complex64))
