@@ -63,7 +63,7 @@ typedef enum { HYENA_F32 = 0, HYENA_BF16 = 1 } hyena_dtype_t;
 
 /* Largest order N accepted by the forward calls. */
 #define HYENA_MAX_ORDER 16
-/* Largest 1-D length L (a power of two) accepted by the forward calls. */
+/* Largest 1-D length L (a power of two) accepted by the 1-D calls. */
 #define HYENA_MAX_LEN (1 << 22)
 
 /* The implicit filter network ("Long Context Language Models ... #690",
@@ -114,12 +114,16 @@ HYENA_API hyena_status_t hyena_filter_gen(const hyena_ffn_t* ffn, int N, int D, 
  * its 2L-point DFT X has L+1 distinct bins X[0..L]; X[0] and X[L] are real,
  * so they share slot 0 as (X[0], X[L]) and slot k holds X[k] for
  * 1 <= k < L.  Rows are L * 8 bytes (16-byte aligned rows).
- * h is [N][D][L] float32.  L is a power of two, 16 <= L <= 16384.
- * Alignment: h 8 bytes, H 16 bytes.  H must not overlap h.
- * The spectrum depends only on the filters: compute it once and reuse it
- * for every batch and every call. */
+ * h is [N][D][L] float32.  L is a power of two, 16 <= L <= HYENA_MAX_LEN.
+ * workspace: device scratch of hyena_filter_rfft_workspace_size(N, D, L)
+ * bytes, 256-byte aligned (0 -- NULL allowed -- for L <= 16384).
+ * Alignment: h 16 bytes, H 16 bytes.  H must not overlap h or the
+ * workspace.  The spectrum depends only on the filters: compute it once
+ * and reuse it for every batch and every call. */
+HYENA_API size_t hyena_filter_rfft_workspace_size(int N, int D, int L);
 HYENA_API hyena_status_t hyena_filter_rfft(const float* h, int N, int D, int L,
-                                 float* H, void* stream);
+                                           float* H, void* workspace, size_t ws_bytes,
+                                           void* stream);
 
 /* Bytes of workspace hyena_fftconv_gate_forward needs for these sizes
  * (0 when none).  spectrum_given = 1 when the caller passes the cached
@@ -129,7 +133,7 @@ HYENA_API size_t hyena_fftconv_workspace_size(int B, int D, int L, int N,
                                     hyena_dtype_t io, int spectrum_given);
 
 /* The fused order-N forward (the recurrence above) over B*D
- * channel-sequences of length L, one launch for all N orders:
+ * channel-sequences of length L:
  *   v      [B][D][L] io            input z_0
  *   x      HOST array of N device pointers, each [B][D][L] io (x_1..x_N)
  *   h      [N][D][L] float32 filters, or NULL when H is given
@@ -140,9 +144,12 @@ HYENA_API size_t hyena_fftconv_workspace_size(int B, int D, int L, int N,
  *          workspace
  *   workspace / ws_bytes: device scratch of at least
  *          hyena_fftconv_workspace_size(...) bytes, 256-byte aligned
- *          (NULL / 0 when that size is 0)
- * L is a power of two, 16 <= L <= 16384 in this build; 1 <= N <=
- * HYENA_MAX_ORDER.  Alignment: v, x_n, y, H 16 bytes; h 8; bias 4.
+ *          (NULL / 0 when that size is 0); it must not overlap any input.
+ * L is a power of two, 16 <= L <= HYENA_MAX_LEN; 1 <= N <= HYENA_MAX_ORDER.
+ * For L <= 16384 one launch runs all N orders with each sequence on one
+ * SM; longer sequences take a four-step FFT through the workspace, 2N + 1
+ * launches per wave of sequences (one wave's scratch stays in L2).
+ * Alignment: v, x_n, y, h, H 16 bytes; bias 4.
  * Returns HYENA_ERR_WORKSPACE if the workspace is too small. */
 HYENA_API hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x,
                                           const float* h, const float* H,

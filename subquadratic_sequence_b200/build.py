@@ -39,18 +39,37 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ into one shared library (if stale)."""
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(os.path.dirname(LIB), exist_ok=True)
-    tmp = LIB + f".tmp{os.getpid()}"
+def _compile(src: str, obj: str, verbose: bool) -> str:
     cmd = [nvcc(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-           "-shared", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+           "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    subprocess.check_call(cmd)
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{r.stdout}{r.stderr}")
+    return r.stdout + r.stderr
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every .cu under csrc/ (one translation unit per kernel
+    family, in parallel) and link them into one shared library, if stale."""
+    if not force and up_to_date():
+        return LIB
+    from concurrent.futures import ThreadPoolExecutor
+
+    objdir = os.path.join(PKG, "lib", "_obj")
+    os.makedirs(objdir, exist_ok=True)
+    srcs = sources()
+    objs = [os.path.join(objdir, os.path.basename(s)[:-3] + f".{os.getpid()}.o") for s in srcs]
+    with ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
+        logs = list(ex.map(lambda so: _compile(so[0], so[1], verbose), zip(srcs, objs)))
+    if verbose:
+        print("".join(logs))
+    tmp = LIB + f".tmp{os.getpid()}"
+    subprocess.check_call([nvcc(), *ARCH_FLAGS, "-shared", "-o", tmp, *objs])
+    for o in objs:
+        os.remove(o)
     os.replace(tmp, LIB)
     return LIB
 

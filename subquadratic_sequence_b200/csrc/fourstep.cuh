@@ -1,0 +1,380 @@
+// fourstep.cuh -- the Hyena forward for sequences too long for one SM
+// (L > 16384), and the filter spectra at those lengths.
+//
+// Same operator and same real-FFT packing as fused1d.cuh: the 2L-point real
+// FFT of the zero-padded sequence is an M = L point complex FFT of
+// z[m] = u[2m] + i u[2m+1].  Here that FFT is split four-step, M = M1 * M2:
+//   n = n2 + M2 n1,  k = k1 + M1 k2,
+//   Z[k1 + M1 k2] = sum_n2 W_M2^{n2 k2} W_M^{n2 k1} sum_n1 z[n2 + M2 n1] W_M1^{n1 k1}
+// and its inverse the same way backwards.  One order of the recurrence is
+// two launches:
+//   row kernel    per pair of rows (k1, M1 - k1): the M2-point row FFTs,
+//                 the real split + bias-folded spectral multiply + inverse
+//                 re-pack (bin k pairs with bin M - k, which sits in row
+//                 M1 - k1), the inverse row FFTs and their twiddle;
+//   column kernel per block of columns n2: the inverse M1-point column
+//                 FFTs, the crop (n1 < M1/2 is the first L outputs), the
+//                 gate by x_n, and -- unless this was the last order -- the
+//                 next order's forward column FFTs and twiddle.
+// The first order starts with a column kernel that reads v.  The scratch
+// (one M-point complex array per sequence) is read and written in place;
+// sequences go through in waves small enough for the wave's scratch to stay
+// resident in L2.
+#pragma once
+
+#include "hyena_common.cuh"
+
+namespace hyena {
+
+__host__ __device__ constexpr int ipow16(int p) { return p <= 0 ? 1 : 16 * ipow16(p - 1); }
+
+// Shared-memory buffer stride (float2) that is >= padded_size(n) and
+// congruent to `mod16` modulo 16: neighbouring buffers then start on
+// different banks.
+__host__ __device__ constexpr int stride_mod16(int n, int mod16)
+{
+    const int p = padded_size(n);
+    return p + ((mod16 - p % 16) + 16) % 16;
+}
+
+// One S = 2^LOG2S point FFT held in a padded shared buffer and transformed
+// by T = S/16 threads (16 values each), Stockham DIT, natural order in and
+// out.  Several transforms run side by side in a CTA; every pass ends in a
+// __syncthreads() of the whole CTA.  On return a[r] holds X[t + r S/16].
+template <int LOG2S>
+struct SmemFft {
+    static_assert(LOG2S >= 4, "S >= 16");
+    static constexpr int S = 1 << LOG2S;
+    static constexpr int T = S / 16;
+    static constexpr int R0 = (LOG2S % 4 == 0) ? 16 : (1 << (LOG2S % 4));  // first pass radix
+    static constexpr int NP = (LOG2S + 3) / 4;                             // passes
+
+    // PADDED_IN: the input sits at buf[pad16(i)] (else at buf[i]).
+    template <int SIGN, bool PADDED_IN>
+    static __device__ __forceinline__ void run(float2* buf, float2* a, int t)
+    {
+        static_for<NP>([&](auto pp) {
+            constexpr int p = decltype(pp)::value;
+            constexpr int R = p == 0 ? R0 : 16;
+            constexpr int NS = p == 0 ? 1 : R0 * ipow16(p - 1);
+            constexpr int C = 16 / R;
+            constexpr bool LAST = p == NP - 1;
+            static_for<C>([&](auto cc) {
+                constexpr int c = decltype(cc)::value;
+                const int j = t + c * T;
+                static_for<R>([&](auto rr) {
+                    constexpr int r = decltype(rr)::value;
+                    const int i = j + r * (S / R);
+                    a[c * R + r] = buf[(p == 0 && !PADDED_IN) ? i : pad16(i)];
+                });
+            });
+            __syncthreads();
+            float dep = zero_after(a[0].x);
+            static_for<C>([&](auto cc) {
+                constexpr int c = decltype(cc)::value;
+                const int j = t + c * T;
+                const int jm = j % NS;
+                float2* ar = a + c * R;
+                if constexpr (p > 0)
+                    apply_twiddle_powers<R>(ar, expi_pi<SIGN>(2.0f * (float)jm / (float)(NS * R) + dep));
+                dft<R, SIGN>(ar);
+                if constexpr (!LAST) {
+                    const int base = (j / NS) * NS * R + jm;
+                    static_for<R>([&](auto rr) {
+                        constexpr int r = decltype(rr)::value;
+                        buf[pad16(base + r * NS)] = ar[r];
+                    });
+                }
+                dep = zero_after(ar[R - 1].x);
+            });
+            if constexpr (!LAST) __syncthreads();
+        });
+    }
+};
+
+struct FourStepArgs {
+    const void* v;                 // [B][D][L] io (first column kernel)
+    const void* x[kMaxOrder];    // x_1..x_N, [B][D][L] io
+    void* y;                       // [B][D][L] io
+    const float2* H;               // [N][D][L] packed spectra (row kernel, conv mode)
+    const float* bias;             // [N][D]
+    float2* S;                     // scratch [wave][M1][M2] complex
+    float2* Hout;                  // [rows][L] packed spectra (row kernel, spectrum mode)
+    int B, D;
+    int q0;                        // first sequence of the wave (channel-major index)
+    int n;                         // order handled by this launch
+    int n_last;                    // N - 1
+};
+
+template <int LOG2M1, int LOG2M2>
+struct FourStep {
+    static constexpr int M1 = 1 << LOG2M1, M2 = 1 << LOG2M2, M = M1 * M2;
+    using F1 = SmemFft<LOG2M1>;
+    using F2 = SmemFft<LOG2M2>;
+    // row kernel: U units (row pairs) per CTA
+    static constexpr int U = F2::T >= 128 ? 2 : 4;
+    static constexpr int ROWS = 2 * U;
+    static constexpr int ROW_THREADS = ROWS * F2::T;
+    static constexpr int ROW_STRIDE = stride_mod16(M2, 2);
+    static constexpr size_t ROW_SMEM = sizeof(float2) * ROWS * ROW_STRIDE;
+    static constexpr int ROW_CTAS_PER_SEQ = (M1 / 2) / U;
+    // column kernel: TC consecutive columns per CTA, column index fastest
+    // across threads so every global access is a TC-element run
+    static constexpr int TC = (512 / F1::T) > 16 ? 16 : ((512 / F1::T) < 4 ? 4 : 512 / F1::T);
+    static constexpr int COL_THREADS = TC * F1::T;
+    static constexpr int COL_STRIDE = stride_mod16(M1, 16 / TC);
+    static constexpr size_t COL_SMEM = sizeof(float2) * TC * COL_STRIDE;
+    static constexpr int COL_CTAS_PER_SEQ = M2 / TC;
+    static_assert(ROW_THREADS <= 1024 && COL_THREADS <= 1024, "block size");
+    static_assert(ROW_SMEM <= 227 * 1024 && COL_SMEM <= 227 * 1024, "shared memory");
+    static_assert(M2 % TC == 0 && (M1 / 2) % U == 0, "tiling");
+
+    // row of the CTA's row slot rr (units u: rows u and M1 - u; unit 0:
+    // rows 0 and M1/2)
+    static __device__ __forceinline__ int row_of(int ublk, int rr)
+    {
+        const int u = ublk * U + rr / 2;
+        if (u == 0) return (rr & 1) ? M1 / 2 : 0;
+        return (rr & 1) ? M1 - u : u;
+    }
+};
+
+// The real split + bias-folded spectral multiply + inverse re-pack of one
+// bin pair (k, Mtot - k), as in fused1d.cuh (scale 1/(2P) included).
+template <int MTOT>
+__device__ __forceinline__ void spectral_pair(float2& z1, float2& z2, float2 h1, float2 h2,
+                                              float2 w, float bias)
+{
+    constexpr float s = 1.0f / (4.0f * (float)MTOT);
+    const float2 bc = cconj(z2);
+    const float2 S = cadd(z1, bc);
+    const float2 Tw = cmul(w, csub(z1, bc));
+    const float2 X1 = make_float2(S.x + Tw.y, S.y - Tw.x);
+    const float2 X2 = make_float2(S.x - Tw.y, -(S.y + Tw.x));
+    const float2 G1 = make_float2((h1.x + bias) * s, h1.y * s);
+    const float2 G2 = make_float2((h2.x + bias) * s, h2.y * s);
+    const float2 Y1 = cmul(X1, G1);
+    const float2 Y2 = cmul(X2, G2);
+    const float2 U = make_float2(Y1.x + Y2.x, Y1.y - Y2.y);
+    const float2 V = cmulc(make_float2(Y1.x - Y2.x, Y1.y + Y2.y), w);
+    z1 = make_float2(U.x - V.y, U.y + V.x);
+    z2 = make_float2(U.x + V.y, V.x - U.y);
+}
+
+// The real split alone: packed spectrum bins k and Mtot - k from Z[k], Z[Mtot - k].
+__device__ __forceinline__ void real_split(float2 z1, float2 z2, float2 w, float2& X1, float2& X2)
+{
+    const float2 bc = cconj(z2);
+    const float2 S = cadd(z1, bc);
+    const float2 Tw = cmul(w, csub(z1, bc));
+    X1 = make_float2(0.5f * (S.x + Tw.y), 0.5f * (S.y - Tw.x));
+    X2 = make_float2(0.5f * (S.x - Tw.y), -0.5f * (S.y + Tw.x));
+}
+
+// Row kernel.  SPECTRUM = false: one order of the forward (conv mode);
+// SPECTRUM = true: forward row FFTs + real split written to Hout in the
+// packed layout (filter spectra).
+template <int LOG2M1, int LOG2M2, bool SPECTRUM>
+__global__ void __launch_bounds__(FourStep<LOG2M1, LOG2M2>::ROW_THREADS)
+fourstep_row_kernel(FourStepArgs a)
+{
+    using FS = FourStep<LOG2M1, LOG2M2>;
+    constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, U = FS::U, T2 = FS::F2::T;
+    constexpr int RS = FS::ROW_STRIDE;
+    extern __shared__ __align__(16) float2 smem_fs[];
+
+    const int qi = blockIdx.x / FS::ROW_CTAS_PER_SEQ;        // sequence within the wave
+    const int ublk = blockIdx.x % FS::ROW_CTAS_PER_SEQ;
+    const int q = a.q0 + qi;                                 // channel-major index
+    const int d = SPECTRUM ? 0 : q / a.B;
+    float2* Sq = a.S + (size_t)qi * M;
+    const int tid = threadIdx.x;
+
+#pragma unroll 1
+    for (int rr = 0; rr < FS::ROWS; ++rr)
+        cp_async_row(smem_fs + rr * RS, Sq + (size_t)FS::row_of(ublk, rr) * M2, M2 * 8, tid,
+                     FS::ROW_THREADS);
+    cp_async_wait_all();
+    __syncthreads();
+
+    const int row = tid / T2, t = tid % T2;
+    float2* rb = smem_fs + row * RS;
+    float2 reg[16];
+    FS::F2::template run<-1, false>(rb, reg, t);
+    static_for<16>([&](auto rr) {
+        constexpr int r = decltype(rr)::value;
+        rb[pad16(t + r * (M2 / 16))] = reg[r];
+    });
+    __syncthreads();
+
+    // bin pairs: thread p -> (row pair up = p % U, k2 = p / U), so adjacent
+    // threads touch adjacent spectrum slots (k1 consecutive)
+    if constexpr (SPECTRUM) {
+        float2* Ho = a.Hout + (size_t)q * M;
+#pragma unroll 1
+        for (int p = tid; p < U * M2; p += FS::ROW_THREADS) {
+            const int up = p % U, k2 = p / U, u = ublk * U + up;
+            float2* r0 = smem_fs + (2 * up) * RS;
+            float2* r1 = smem_fs + (2 * up + 1) * RS;
+            float2 X1, X2;
+            if (u != 0) {
+                const int k = u + M1 * k2;
+                real_split(r0[pad16(k2)], r1[pad16(M2 - 1 - k2)], expi_pi<-1>((float)k / (float)M), X1, X2);
+                Ho[k] = X1;
+                Ho[M - k] = X2;
+            } else if (k2 < M2 / 2) {
+                const int k = M1 / 2 + M1 * k2;     // row M1/2 with itself, reversed
+                real_split(r1[pad16(k2)], r1[pad16(M2 - 1 - k2)], expi_pi<-1>((float)k / (float)M), X1, X2);
+                Ho[k] = X1;
+                Ho[M - k] = X2;
+                if (k2 > 0) {                        // row 0: k2 with M2 - k2
+                    const int k0 = M1 * k2;
+                    real_split(r0[pad16(k2)], r0[pad16(M2 - k2)], expi_pi<-1>((float)k0 / (float)M), X1, X2);
+                    Ho[k0] = X1;
+                    Ho[M - k0] = X2;
+                } else {                             // bins 0 and M (slot 0), and M/2
+                    const float2 z = r0[0];
+                    Ho[0] = make_float2(z.x + z.y, z.x - z.y);
+                    const float2 zh = r0[pad16(M2 / 2)];
+                    real_split(zh, zh, make_float2(0.0f, -1.0f), X1, X2);
+                    Ho[M / 2] = X1;
+                }
+            }
+        }
+        return;
+    } else {
+        const float bias = __ldg(a.bias + a.n * a.D + d);
+        const float2* Hr = a.H + ((size_t)a.n * a.D + d) * M;
+#pragma unroll 1
+        for (int p = tid; p < U * M2; p += FS::ROW_THREADS) {
+            const int up = p % U, k2 = p / U, u = ublk * U + up;
+            float2* r0 = smem_fs + (2 * up) * RS;
+            float2* r1 = smem_fs + (2 * up + 1) * RS;
+            if (u != 0) {
+                const int k = u + M1 * k2;           // partner M - k: row M1 - u, slot M2 - 1 - k2
+                float2 z1 = r0[pad16(k2)], z2 = r1[pad16(M2 - 1 - k2)];
+                spectral_pair<M>(z1, z2, __ldg(Hr + k), __ldg(Hr + (M - k)),
+                                 expi_pi<-1>((float)k / (float)M), bias);
+                r0[pad16(k2)] = z1;
+                r1[pad16(M2 - 1 - k2)] = z2;
+            } else if (k2 < M2 / 2) {
+                {
+                    const int k = M1 / 2 + M1 * k2;
+                    float2 z1 = r1[pad16(k2)], z2 = r1[pad16(M2 - 1 - k2)];
+                    spectral_pair<M>(z1, z2, __ldg(Hr + k), __ldg(Hr + (M - k)),
+                                     expi_pi<-1>((float)k / (float)M), bias);
+                    r1[pad16(k2)] = z1;
+                    r1[pad16(M2 - 1 - k2)] = z2;
+                }
+                if (k2 > 0) {
+                    const int k = M1 * k2;
+                    float2 z1 = r0[pad16(k2)], z2 = r0[pad16(M2 - k2)];
+                    spectral_pair<M>(z1, z2, __ldg(Hr + k), __ldg(Hr + (M - k)),
+                                     expi_pi<-1>((float)k / (float)M), bias);
+                    r0[pad16(k2)] = z1;
+                    r0[pad16(M2 - k2)] = z2;
+                } else {
+                    const float2 h0 = __ldg(Hr);
+                    float2 z1 = r0[0], z2 = z1;
+                    spectral_pair<M>(z1, z2, make_float2(h0.x, 0.0f), make_float2(h0.y, 0.0f),
+                                     make_float2(1.0f, 0.0f), bias);
+                    r0[0] = z1;
+                    const float2 hm = __ldg(Hr + M / 2);
+                    float2 w1 = r0[pad16(M2 / 2)], w2 = w1;
+                    spectral_pair<M>(w1, w2, hm, hm, make_float2(0.0f, -1.0f), bias);
+                    r0[pad16(M2 / 2)] = w1;
+                }
+            }
+        }
+        __syncthreads();
+
+        FS::F2::template run<+1, true>(rb, reg, t);
+        // B[k1][n2] *= exp(+2 pi i n2 k1 / M), n2 = t + r M2/16
+        const int k1 = FS::row_of(ublk, row);
+        float2 w = expi_pi<+1>(2.0f * (float)((t * k1) % M) / (float)M);
+        const float2 step = expi_pi<+1>(2.0f * (float)((k1 * (M2 / 16)) % M) / (float)M);
+        static_for<16>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            Sq[(size_t)k1 * M2 + t + r * (M2 / 16)] = cmul(reg[r], w);
+            if constexpr (r < 15) w = cmul(w, step);
+        });
+    }
+}
+
+// Column kernel.  MODE 0: the first order's forward columns from v (or, for
+// the spectrum, from h); MODE 1: inverse columns, gate, next order's forward
+// columns; MODE 2: inverse columns, gate, store y.
+template <int LOG2M1, int LOG2M2, typename IO, int MODE>
+__global__ void __launch_bounds__(FourStep<LOG2M1, LOG2M2>::COL_THREADS)
+fourstep_col_kernel(FourStepArgs a)
+{
+    using FS = FourStep<LOG2M1, LOG2M2>;
+    using IOP = IoPair<IO>;
+    using PT = typename IOP::T;
+    constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, TC = FS::TC;
+    extern __shared__ __align__(16) float2 smem_fs[];
+
+    const int qi = blockIdx.x / FS::COL_CTAS_PER_SEQ;
+    const int c0 = (blockIdx.x % FS::COL_CTAS_PER_SEQ) * TC;
+    const int q = a.q0 + qi;
+    const int d = q / a.B, b = q % a.B;
+    const size_t seq = (size_t)b * a.D + d;                  // (spectrum: a.B = 1, a.D = rows)
+    float2* Sq = a.S + (size_t)qi * M;
+    const int tid = threadIdx.x;
+    const int c = tid % TC, t = tid / TC;
+    const int n2 = c0 + c;
+    float2* buf = smem_fs + c * FS::COL_STRIDE;
+    float2 reg[16];
+
+    if constexpr (MODE == 0) {
+        const PT* vp = reinterpret_cast<const PT*>(a.v) + seq * (M / 2);
+        static_for<8>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            reg[r] = IOP::load(vp + n2 + (size_t)M2 * (t + r * (M1 / 16)));
+        });
+    } else {
+        static_for<16>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            const int k1 = t + r * (M1 / 16);
+            buf[pad16(k1)] = Sq[(size_t)k1 * M2 + n2];
+        });
+        __syncthreads();
+        FS::F1::template run<+1, true>(buf, reg, t);
+        // crop (n1 = t + r M1/16 < M1/2 <=> r < 8) and gate
+        const void* xn = a.x[0];
+#pragma unroll
+        for (int i = 1; i < kMaxOrder; ++i)
+            if (i == a.n) xn = a.x[i];
+        const PT* xp = reinterpret_cast<const PT*>(xn) + seq * (M / 2);
+        static_for<8>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            const float2 xv = IOP::load(xp + n2 + (size_t)M2 * (t + r * (M1 / 16)));
+            reg[r] = make_float2(reg[r].x * xv.x, reg[r].y * xv.y);
+        });
+        if constexpr (MODE == 2) {
+            PT* yp = reinterpret_cast<PT*>(a.y) + seq * (M / 2);
+            static_for<8>([&](auto rr) {
+                constexpr int r = decltype(rr)::value;
+                IOP::store(yp + n2 + (size_t)M2 * (t + r * (M1 / 16)), reg[r]);
+            });
+            return;
+        }
+    }
+    // forward column FFT of z (n1 < M1/2), zero-padded, then the four-step
+    // twiddle exp(-2 pi i n2 k1 / M)
+    static_for<16>([&](auto rr) {
+        constexpr int r = decltype(rr)::value;
+        buf[pad16(t + r * (M1 / 16))] = r < 8 ? reg[r] : make_float2(0.0f, 0.0f);
+    });
+    __syncthreads();
+    FS::F1::template run<-1, true>(buf, reg, t);
+    float2 w = expi_pi<-1>(2.0f * (float)((n2 * t) % M) / (float)M);
+    const float2 step = expi_pi<-1>(2.0f * (float)((n2 * (M1 / 16)) % M) / (float)M);
+    static_for<16>([&](auto rr) {
+        constexpr int r = decltype(rr)::value;
+        Sq[(size_t)(t + r * (M1 / 16)) * M2 + n2] = cmul(reg[r], w);
+        if constexpr (r < 15) w = cmul(w, step);
+    });
+}
+
+}  // namespace hyena

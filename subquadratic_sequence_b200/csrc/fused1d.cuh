@@ -59,8 +59,6 @@ HYENA_PLAN1D(13, 32, 16, 32, 1, 16)
 HYENA_PLAN1D(14, 32, 16, 8, 8, 16)
 #undef HYENA_PLAN1D
 
-constexpr int kMaxOrder = 16;
-
 struct Fused1dArgs {
     const void* v;                 // [B][D][L] io
     const void* x[kMaxOrder];      // N pointers, each [B][D][L] io

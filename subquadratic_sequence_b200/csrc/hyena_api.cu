@@ -1,23 +1,14 @@
 // hyena_api.cu -- the extern "C" entry points declared in include/hyena.h:
-// argument validation on the host, kernel selection and launch.
+// argument validation on the host, then the dispatchers of launch.cuh.
 #include <stdint.h>
 
-#include "filter_gen.cuh"
-#include "fused1d.cuh"
-#include "hyena.h"
+#include "launch.cuh"
 
 using namespace hyena;
 
 namespace {
 
 thread_local int g_last_cuda_error = 0;
-
-hyena_status_t from_cuda(cudaError_t e)
-{
-    if (e == cudaSuccess) return HYENA_OK;
-    g_last_cuda_error = (int)e;
-    return HYENA_ERR_CUDA;
-}
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
@@ -37,80 +28,22 @@ int exact_log2(long n)
     return k;
 }
 
-constexpr int kMinLog2 = 4;    // L >= 16
-constexpr int kMaxLog2Fused = 14;  // single-CTA path: L <= 16384
-
 size_t io_bytes(hyena_dtype_t io) { return io == HYENA_BF16 ? 2 : 4; }
 
-// ------------------------------------------------------------ launchers
+size_t scratch_bytes(long nseq, long L) { return sizeof(float2) * (size_t)wave_seqs(nseq, L) * L; }
 
-template <typename K>
-cudaError_t allow_smem(K kernel, size_t bytes)
+// spectra of rows filters: single-CTA kernel or four-step (scratch needed)
+hyena_status_t spectra(int log2m, const float* h, int rows, float2* H, float2* scratch,
+                       cudaStream_t st)
 {
-    if (bytes <= 48 * 1024) return cudaSuccess;
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-}
-
-template <int LOG2M, typename IO>
-hyena_status_t launch_fused(const Fused1dArgs& args, cudaStream_t st)
-{
-    using F = Fft1d<LOG2M>;
-    auto kernel = fused1d_kernel<LOG2M, IO>;
-    cudaError_t e = allow_smem(kernel, F::SMEM_BYTES);
-    if (e != cudaSuccess) return from_cuda(e);
-    const long BD = (long)args.B * args.D;
-    const unsigned grid = (unsigned)((BD + F::G - 1) / F::G);
-    kernel<<<grid, F::THREADS, F::SMEM_BYTES, st>>>(args);
-    return from_cuda(cudaGetLastError());
-}
-
-template <int LOG2M>
-hyena_status_t launch_rfft(const Rfft1dArgs& args, cudaStream_t st)
-{
-    using F = Fft1d<LOG2M>;
-    auto kernel = rfft1d_kernel<LOG2M>;
-    cudaError_t e = allow_smem(kernel, F::SMEM_BYTES_FFT);
-    if (e != cudaSuccess) return from_cuda(e);
-    const unsigned grid = (unsigned)((args.rows + F::G - 1) / F::G);
-    kernel<<<grid, F::THREADS, F::SMEM_BYTES_FFT, st>>>(args);
-    return from_cuda(cudaGetLastError());
-}
-
-template <typename IO>
-hyena_status_t dispatch_fused(int log2m, const Fused1dArgs& a, cudaStream_t st)
-{
-    switch (log2m) {
-    case 4: return launch_fused<4, IO>(a, st);
-    case 5: return launch_fused<5, IO>(a, st);
-    case 6: return launch_fused<6, IO>(a, st);
-    case 7: return launch_fused<7, IO>(a, st);
-    case 8: return launch_fused<8, IO>(a, st);
-    case 9: return launch_fused<9, IO>(a, st);
-    case 10: return launch_fused<10, IO>(a, st);
-    case 11: return launch_fused<11, IO>(a, st);
-    case 12: return launch_fused<12, IO>(a, st);
-    case 13: return launch_fused<13, IO>(a, st);
-    case 14: return launch_fused<14, IO>(a, st);
-    default: return HYENA_ERR_UNSUPPORTED;
+    if (log2m <= kMaxLog2Fused) {
+        Rfft1dArgs ra;
+        ra.h = h;
+        ra.H = H;
+        ra.rows = rows;
+        return dispatch_rfft(log2m, ra, st);
     }
-}
-
-hyena_status_t dispatch_rfft(int log2m, const Rfft1dArgs& a, cudaStream_t st)
-{
-    switch (log2m) {
-    case 4: return launch_rfft<4>(a, st);
-    case 5: return launch_rfft<5>(a, st);
-    case 6: return launch_rfft<6>(a, st);
-    case 7: return launch_rfft<7>(a, st);
-    case 8: return launch_rfft<8>(a, st);
-    case 9: return launch_rfft<9>(a, st);
-    case 10: return launch_rfft<10>(a, st);
-    case 11: return launch_rfft<11>(a, st);
-    case 12: return launch_rfft<12>(a, st);
-    case 13: return launch_rfft<13>(a, st);
-    case 14: return launch_rfft<14>(a, st);
-    default: return HYENA_ERR_UNSUPPORTED;
-    }
+    return dispatch_fourstep_rfft(log2m, h, rows, H, scratch, st);
 }
 
 // Validates a 1-D length: INVALID_ARG for L < 1, UNSUPPORTED outside the
@@ -135,8 +68,8 @@ hyena_status_t check_ffn(const hyena_ffn_t* f)
     return HYENA_OK;
 }
 
-hyena_status_t launch_filter_gen(const hyena_ffn_t* f, int rows, int D, long npos, int L, int Hh,
-                                 int Ww, bool two_d, float* h, cudaStream_t st)
+hyena_status_t filter_gen(const hyena_ffn_t* f, int rows, int D, long npos, int L, int Hh,
+                          int Ww, bool two_d, float* h, cudaStream_t st)
 {
     FilterGenArgs a;
     a.W1 = f->W1; a.W2 = f->W2; a.W3 = f->W3; a.Wout = f->Wout; a.alpha = f->alpha;
@@ -148,17 +81,7 @@ hyena_status_t launch_filter_gen(const hyena_ffn_t* f, int rows, int D, long npo
     a.n_bands = f->n_bands;
     a.inv_div = 1.0f / f->decay_div;
     a.h = h;
-    const unsigned grid = (unsigned)((npos + kFgTile - 1) / kFgTile);
-    cudaError_t e;
-    if (two_d) {
-        e = allow_smem(filter_gen_kernel<true>, kFgSmemBytes);
-        if (e == cudaSuccess) filter_gen_kernel<true><<<grid, kFgThreads, kFgSmemBytes, st>>>(a);
-    } else {
-        e = allow_smem(filter_gen_kernel<false>, kFgSmemBytes);
-        if (e == cudaSuccess) filter_gen_kernel<false><<<grid, kFgThreads, kFgSmemBytes, st>>>(a);
-    }
-    if (e != cudaSuccess) return from_cuda(e);
-    return from_cuda(cudaGetLastError());
+    return launch_filter_gen(a, two_d, npos, st);
 }
 
 // packed spectrum: L complex slots per filter (bins 0 and L share slot 0)
@@ -167,6 +90,15 @@ size_t spectrum_bytes(long N, long D, long L) { return sizeof(float2) * N * D * 
 size_t round_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
 }  // namespace
+
+namespace hyena {
+hyena_status_t from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess) return HYENA_OK;
+    g_last_cuda_error = (int)e;
+    return HYENA_ERR_CUDA;
+}
+}  // namespace hyena
 
 extern "C" {
 
@@ -190,7 +122,7 @@ hyena_status_t hyena_filter_gen(const hyena_ffn_t* ffn, int N, int D, int L, flo
     if (s != HYENA_OK) return s;
     if (!h || N < 1 || D < 1 || L < 1 || !aligned(h, 4)) return HYENA_ERR_INVALID_ARG;
     if ((long)N * D > (1L << 30) || (long)N * D * (long)L > (1L << 40)) return HYENA_ERR_UNSUPPORTED;
-    return launch_filter_gen(ffn, N * D, D, L, L, 0, 0, false, h, (cudaStream_t)stream);
+    return filter_gen(ffn, N * D, D, L, L, 0, 0, false, h, (cudaStream_t)stream);
 }
 
 hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C, int H, int W, float* h,
@@ -200,24 +132,35 @@ hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C, int H, 
     if (s != HYENA_OK) return s;
     if (!h || N < 1 || C < 1 || H < 1 || W < 1 || !aligned(h, 4)) return HYENA_ERR_INVALID_ARG;
     if ((long)H * W > (1L << 30) || (long)N * C * (long)H * W > (1L << 40)) return HYENA_ERR_UNSUPPORTED;
-    return launch_filter_gen(ffn, N * C, C, (long)H * W, 0, H, W, true, h, (cudaStream_t)stream);
+    return filter_gen(ffn, N * C, C, (long)H * W, 0, H, W, true, h, (cudaStream_t)stream);
 }
 
-hyena_status_t hyena_filter_rfft(const float* h, int N, int D, int L, float* H, void* stream)
+size_t hyena_filter_rfft_workspace_size(int N, int D, int L)
+{
+    int log2m = 0;
+    if (N < 1 || D < 1 || check_len(L, kMaxLog2, &log2m) != HYENA_OK) return (size_t)-1;
+    return log2m <= kMaxLog2Fused ? 0 : round_up(scratch_bytes((long)N * D, L), 256);
+}
+
+hyena_status_t hyena_filter_rfft(const float* h, int N, int D, int L, float* H, void* workspace,
+                                 size_t ws_bytes, void* stream)
 {
     if (!h || !H || N < 1 || D < 1) return HYENA_ERR_INVALID_ARG;
     int log2m = 0;
-    hyena_status_t s = check_len(L, kMaxLog2Fused, &log2m);
+    hyena_status_t s = check_len(L, kMaxLog2, &log2m);
     if (s != HYENA_OK) return s;
-    if (!aligned(h, 8) || !aligned(H, 16)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(h, 16) || !aligned(H, 16)) return HYENA_ERR_INVALID_ARG;
     if ((long)N * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
-    if (overlap(h, sizeof(float) * N * D * (size_t)L, H, spectrum_bytes(N, D, L)))
-        return HYENA_ERR_INVALID_ARG;
-    Rfft1dArgs a;
-    a.h = h;
-    a.H = reinterpret_cast<float2*>(H);
-    a.rows = N * D;
-    return dispatch_rfft(log2m, a, (cudaStream_t)stream);
+    const size_t spec = spectrum_bytes(N, D, L);
+    if (overlap(h, sizeof(float) * N * D * (size_t)L, H, spec)) return HYENA_ERR_INVALID_ARG;
+    const size_t need = log2m <= kMaxLog2Fused ? 0 : round_up(scratch_bytes((long)N * D, L), 256);
+    if (need > 0) {
+        if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+        if (overlap(workspace, need, H, spec) || overlap(workspace, need, h, sizeof(float) * N * D * (size_t)L))
+            return HYENA_ERR_INVALID_ARG;
+    }
+    return spectra(log2m, h, N * D, reinterpret_cast<float2*>(H), reinterpret_cast<float2*>(workspace),
+                   (cudaStream_t)stream);
 }
 
 size_t hyena_fftconv_workspace_size(int B, int D, int L, int N, hyena_dtype_t io,
@@ -226,8 +169,13 @@ size_t hyena_fftconv_workspace_size(int B, int D, int L, int N, hyena_dtype_t io
     int log2m = 0;
     if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || (io != HYENA_F32 && io != HYENA_BF16))
         return (size_t)-1;
-    if (check_len(L, kMaxLog2Fused, &log2m) != HYENA_OK) return (size_t)-1;
-    return spectrum_given ? 0 : round_up(spectrum_bytes(N, D, L), 256);
+    if (check_len(L, kMaxLog2, &log2m) != HYENA_OK) return (size_t)-1;
+    size_t need = spectrum_given ? 0 : round_up(spectrum_bytes(N, D, L), 256);
+    if (log2m > kMaxLog2Fused) {
+        const long nseq = (long)B * D > (long)N * D ? (long)B * D : (long)N * D;
+        need += round_up(scratch_bytes(nseq, L), 256);
+    }
+    return need;
 }
 
 hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, const float* h,
@@ -240,17 +188,17 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
     if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
     if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
     int log2m = 0;
-    hyena_status_t s = check_len(L, kMaxLog2Fused, &log2m);
+    hyena_status_t s = check_len(L, kMaxLog2, &log2m);
     if (s != HYENA_OK) return s;
     if ((long)B * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
     for (int n = 0; n < N; ++n)
         if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
     if (!aligned(v, 16) || !aligned(y, 16) || !aligned(bias, 4)) return HYENA_ERR_INVALID_ARG;
-    if ((H && !aligned(H, 16)) || (!H && !aligned(h, 8))) return HYENA_ERR_INVALID_ARG;
+    if ((H && !aligned(H, 16)) || (!H && !aligned(h, 16))) return HYENA_ERR_INVALID_ARG;
 
     const size_t act = (size_t)B * D * L * io_bytes(io);
     const size_t spec = spectrum_bytes(N, D, L);
-    const size_t need = H ? 0 : round_up(spec, 256);
+    const size_t need = hyena_fftconv_workspace_size(B, D, L, N, io, H != nullptr);
     if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256)))
         return HYENA_ERR_WORKSPACE;
     // y must not overlap anything it is computed from
@@ -260,22 +208,39 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
         (need > 0 && overlap(y, act, workspace, need)))
         return HYENA_ERR_INVALID_ARG;
     for (int n = 0; n < N; ++n)
-        if (overlap(y, act, x[n], act)) return HYENA_ERR_INVALID_ARG;
-    if (!H && overlap(h, sizeof(float) * N * D * (size_t)L, workspace, need))
+        if (overlap(y, act, x[n], act) || (need > 0 && overlap(workspace, need, x[n], act)))
+            return HYENA_ERR_INVALID_ARG;
+    if (need > 0 && (overlap(workspace, need, v, act) || (H && overlap(workspace, need, H, spec)) ||
+                     (!H && overlap(h, sizeof(float) * N * D * (size_t)L, workspace, need))))
         return HYENA_ERR_INVALID_ARG;
 
     cudaStream_t st = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
     const float2* spectrum = reinterpret_cast<const float2*>(H);
+    float2* scratch = nullptr;
     if (!H) {
-        Rfft1dArgs ra;
-        ra.h = h;
-        ra.H = reinterpret_cast<float2*>(workspace);
-        ra.rows = N * D;
-        s = dispatch_rfft(log2m, ra, st);
+        float2* Hw = reinterpret_cast<float2*>(ws);
+        ws += round_up(spec, 256);
+        if (log2m > kMaxLog2Fused) scratch = reinterpret_cast<float2*>(ws);
+        s = spectra(log2m, h, N * D, Hw, scratch, st);
         if (s != HYENA_OK) return s;
-        spectrum = ra.H;
+        spectrum = Hw;
+    } else if (log2m > kMaxLog2Fused) {
+        scratch = reinterpret_cast<float2*>(ws);
     }
-    Fused1dArgs a;
+    if (log2m <= kMaxLog2Fused) {
+        Fused1dArgs a;
+        a.v = v;
+        for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
+        a.y = y;
+        a.H = spectrum;
+        a.bias = bias;
+        a.B = B;
+        a.D = D;
+        a.N = N;
+        return io == HYENA_BF16 ? dispatch_fused_bf16(log2m, a, st) : dispatch_fused_f32(log2m, a, st);
+    }
+    FourStepArgs a = {};
     a.v = v;
     for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
     a.y = y;
@@ -283,9 +248,8 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
     a.bias = bias;
     a.B = B;
     a.D = D;
-    a.N = N;
-    return io == HYENA_BF16 ? dispatch_fused<__nv_bfloat16>(log2m, a, st)
-                            : dispatch_fused<float>(log2m, a, st);
+    return io == HYENA_BF16 ? dispatch_fourstep_bf16(log2m, a, N, scratch, st)
+                            : dispatch_fourstep_f32(log2m, a, N, scratch, st);
 }
 
 }  // extern "C"

@@ -17,6 +17,9 @@
 
 namespace hyena {
 
+// Largest order N (number of long convolutions) one forward call accepts.
+constexpr int kMaxOrder = 16;
+
 // ------------------------------------------------------------------ utils
 
 template <typename F, int... Is>

@@ -1,0 +1,61 @@
+// launch.cuh -- internal (not exported) launch helpers shared by the
+// library's translation units.  Each kernel family is instantiated and
+// launched in its own .cu file so the library compiles in parallel;
+// hyena_api.cu validates arguments and calls these dispatchers.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "filter_gen.cuh"
+#include "fourstep.cuh"
+#include "fused1d.cuh"
+#include "hyena.h"
+
+namespace hyena {
+
+constexpr int kMinLog2 = 4;        // L >= 16
+constexpr int kMaxLog2Fused = 14;  // single-CTA path: L <= 16384
+constexpr int kMaxLog2 = 22;       // four-step path: L <= 2^22
+// the scratch of one wave of long sequences stays under this (L2 resident)
+constexpr size_t kWaveScratchBytes = 64u << 20;
+
+// Maps a CUDA error to a status and records it for hyena_last_cuda_error().
+hyena_status_t from_cuda(cudaError_t e);
+
+// Opts a kernel in to more than 48 KB of dynamic shared memory.
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes)
+{
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <typename K, typename A>
+hyena_status_t launch(K kernel, unsigned grid, int threads, size_t smem, cudaStream_t st, const A& a)
+{
+    cudaError_t e = allow_smem(kernel, smem);
+    if (e != cudaSuccess) return from_cuda(e);
+    kernel<<<grid, threads, smem, st>>>(a);
+    return from_cuda(cudaGetLastError());
+}
+
+// sequences per wave of the four-step path (scratch = wave * L complex)
+inline long wave_seqs(long nseq, long L)
+{
+    long per = (long)(kWaveScratchBytes / (sizeof(float2) * (size_t)L));
+    if (per < 1) per = 1;
+    return nseq < per ? nseq : per;
+}
+
+hyena_status_t dispatch_fused_f32(int log2m, const Fused1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_fused_bf16(int log2m, const Fused1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_rfft(int log2m, const Rfft1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_fourstep_f32(int log2m, const FourStepArgs& a, int N, float2* scratch,
+                                     cudaStream_t st);
+hyena_status_t dispatch_fourstep_bf16(int log2m, const FourStepArgs& a, int N, float2* scratch,
+                                      cudaStream_t st);
+hyena_status_t dispatch_fourstep_rfft(int log2m, const float* h, int rows, float2* H,
+                                      float2* scratch, cudaStream_t st);
+hyena_status_t launch_filter_gen(const FilterGenArgs& a, bool two_d, long npos, cudaStream_t st);
+
+}  // namespace hyena

@@ -49,7 +49,8 @@ def _load() -> ctypes.CDLL:
         "hyena_last_cuda_error": ([], i),
         "hyena_filter_gen": ([ffn_p, i, i, i, vp, vp], i),
         "hyena_filter_gen_2d": ([ffn_p, i, i, i, i, vp, vp], i),
-        "hyena_filter_rfft": ([vp, i, i, i, vp, vp], i),
+        "hyena_filter_rfft_workspace_size": ([i, i, i], sz),
+        "hyena_filter_rfft": ([vp, i, i, i, vp, vp, sz, vp], i),
         "hyena_fftconv_workspace_size": ([i, i, i, i, i, i], sz),
         "hyena_fftconv_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp, vp,
                                         sz, vp], i),
@@ -130,15 +131,27 @@ def hyena_filter_gen_2d(W1, W2, W3, Wout, alpha, N: int, C: int, H: int, W: int,
     return out
 
 
-def hyena_filter_rfft(h: torch.Tensor, *, out=None, stream=None):
+def hyena_filter_rfft_workspace_size(N: int, D: int, L: int) -> int:
+    n = LIB.hyena_filter_rfft_workspace_size(N, D, L)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_filter_rfft_workspace_size", HYENA_ERR_INVALID_ARG, "invalid sizes")
+    return n
+
+
+def hyena_filter_rfft(h: torch.Tensor, *, out=None, workspace=None, stream=None):
     """Packed spectra [N][D][L] complex64 (slot 0 = (bin 0, bin L)) of the
     filters h [N][D][L] zero-padded to 2L."""
     N, D, L = h.shape
     if out is None:
         out = torch.empty((N, D, L), device=h.device, dtype=torch.complex64)
+    need = hyena_filter_rfft_workspace_size(N, D, L)
+    if need and workspace is None:
+        workspace = torch.empty(need, device=h.device, dtype=torch.uint8)
+    wp = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+    wn = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("hyena_filter_rfft", LIB.hyena_filter_rfft(
         ctypes.c_void_p(_dev(h, torch.float32, "h")), N, D, L,
-        ctypes.c_void_p(_dev(out, torch.complex64, "H")), _stream(stream)))
+        ctypes.c_void_p(_dev(out, torch.complex64, "H")), wp, wn, _stream(stream)))
     return out
 
 

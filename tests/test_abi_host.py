@@ -98,6 +98,8 @@ def test_forward_rejects_bad_arguments(lib):
     assert fwd(lib, L=1000) == UNSUPPORTED
     assert fwd(lib, L=8) == UNSUPPORTED
     assert fwd(lib, L=1 << 23) == UNSUPPORTED
+    # long sequences need a workspace even with the spectrum given
+    assert fwd(lib, L=1 << 16) == WORKSPACE
     xs17 = tuple(P(10 + i) for i in range(17))
     assert fwd(lib, xs=xs17) == UNSUPPORTED
     # misalignment
@@ -120,14 +122,25 @@ def test_forward_rejects_bad_arguments(lib):
 
 def test_filter_rfft_rejects_bad_arguments(lib):
     r = lib.hyena_filter_rfft
-    assert r(None, 2, 3, 64, P(1), None) == INVALID
-    assert r(P(0), 2, 3, 64, None, None) == INVALID
-    assert r(P(0), 0, 3, 64, P(1), None) == INVALID
-    assert r(P(0), 2, 3, 0, P(1), None) == INVALID
-    assert r(P(0), 2, 3, 48, P(1), None) == UNSUPPORTED
-    assert r(P(0), 2, 3, 1 << 15, P(1), None) == UNSUPPORTED
-    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + BIG + 8), None) == INVALID
-    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + 256), None) == INVALID   # H overlaps h
+    assert r(None, 2, 3, 64, P(1), None, 0, None) == INVALID
+    assert r(P(0), 2, 3, 64, None, None, 0, None) == INVALID
+    assert r(P(0), 0, 3, 64, P(1), None, 0, None) == INVALID
+    assert r(P(0), 2, 3, 0, P(1), None, 0, None) == INVALID
+    assert r(P(0), 2, 3, 48, P(1), None, 0, None) == UNSUPPORTED
+    assert r(P(0), 2, 3, 1 << 23, P(1), None, 0, None) == UNSUPPORTED
+    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + BIG + 8), None, 0, None) == INVALID
+    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + 256), None, 0, None) == INVALID   # H overlaps h
+    # long filters need a workspace
+    assert r(P(0), 2, 3, 1 << 16, P(1), None, 0, None) == WORKSPACE
+    assert r(P(0), 2, 3, 1 << 16, P(1), P(2), 1024, None) == WORKSPACE
+    assert r(P(0), 2, 3, 1 << 16, P(1), P(1), 1 << 26, None) == INVALID        # workspace overlaps H
+
+
+def test_rfft_workspace_size(lib):
+    assert lib.hyena_filter_rfft_workspace_size(2, 3, 1 << 14) == 0
+    n = lib.hyena_filter_rfft_workspace_size(2, 3, 1 << 16)
+    assert n >= 6 * (1 << 16) * 8 and n % 256 == 0
+    assert lib.hyena_filter_rfft_workspace_size(2, 3, 100) == ctypes.c_size_t(-1).value
 
 
 def _ffn(lib, **kw):

@@ -74,7 +74,8 @@ def test_filter_gen_2d_matches_oracle(hy, N, C, H, W):
     assert rel_max_err(got, ref) <= 2e-5
 
 
-@pytest.mark.parametrize("L", [16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384])
+@pytest.mark.parametrize("L", [16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384,
+                               32768, 65536, 262144])
 def test_rfft_matches_oracle(hy, L):
     rng = np.random.default_rng(L)
     h = (rng.standard_normal((2, 3, L)) * np.exp(-np.arange(L) / (L / 4))).astype(np.float32)
@@ -90,6 +91,9 @@ FWD_CASES = [(3, 5, L, 2, "f32") for L in (16, 32, 64, 128, 256, 512, 1024, 2048
 FWD_CASES += [(3, 5, L, 2, "bf16") for L in (16, 256, 2048, 8192)]
 FWD_CASES += [(2, 7, 2048, 1, "f32"), (2, 7, 2048, 3, "f32"), (1, 3, 256, 16, "f32"),
               (1, 1, 4096, 2, "f32"), (5, 1, 1024, 2, "f32"), (4, 33, 1024, 2, "bf16")]
+# four-step path (L > 16384)
+FWD_CASES += [(1, 3, 32768, 2, "f32"), (2, 2, 65536, 2, "f32"), (1, 2, 131072, 3, "f32"),
+              (1, 2, 65536, 2, "bf16"), (1, 1, 262144, 1, "f32")]
 
 
 @pytest.mark.parametrize("B,D,L,N,io", FWD_CASES)
@@ -170,20 +174,33 @@ def test_c0_end_to_end(hy):
 
 
 def _sampled_full_size(hy, name, n_samples, seed):
+    """The whole workload on the GPU (filter generation, spectra, forward);
+    the oracle on n_samples seeded (b, d) rows plus the first and last,
+    its filters generated for just those channels."""
     wl = synth.WORKLOADS[name]
     inp = synth.make_inputs(wl)
     h = gpu_filters(inp, wl)
     H = hy.hyena_filter_rfft(h)
+    del h
     y = hy.hyena_fftconv_gate_forward(dev(inp["v"], wl.io), [dev(x, wl.io) for x in inp["x"]],
                                       dev(inp["b"]), H=H)
     torch.cuda.synchronize()
+    del H
     rng = np.random.default_rng(seed)
     seqs = [(int(rng.integers(wl.B)), int(rng.integers(wl.D))) for _ in range(n_samples)]
     seqs += [(0, 0), (wl.B - 1, wl.D - 1)]
-    y = y.float()
-    got = np.stack([y[bi, di].cpu().numpy() for (bi, di) in seqs]).astype(np.float64)
-    ref = oracle_forward(inp, oracle_filters(inp, wl), seqs=seqs)
-    return assert_close(got, ref, wl.io, name)
+    got = np.stack([y[bi, di].float().cpu().numpy() for (bi, di) in seqs]).astype(np.float64)
+    del y
+    refs = []
+    for (bi, di) in seqs:
+        rows = [n * wl.D + di for n in range(wl.N)]
+        hd = oracle.filter_gen(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][[di]],
+                               wl.N, 1, wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                               decay_div=synth.DECAY_DIV)
+        v = inp["v"][bi:bi + 1, di:di + 1].astype(np.float64)
+        x = np.stack([xx[bi:bi + 1, di:di + 1] for xx in inp["x"]]).astype(np.float64)
+        refs.append(oracle.hyena_forward(v, x, hd, inp["b"][:, di:di + 1].astype(np.float64))[0, 0])
+    return assert_close(got, np.stack(refs), wl.io, name)
 
 
 def test_c1_full_size_sampled(hy):
@@ -196,3 +213,29 @@ def test_c1_full_size_sampled(hy):
 def test_c2_full_size_sampled(hy, name):
     """Order-3, B=2, D=768, L=8192 / 16384, fp32."""
     _sampled_full_size(hy, name, 16, seed=2)
+
+
+@pytest.mark.parametrize("name", ["c3_64k", "c3_256k", "c3_1m"])
+def test_c3_full_size_sampled(hy, name):
+    """Order-2, B=1, D=256, L = 64k / 256k / 1M, fp32: the four-step path."""
+    _sampled_full_size(hy, name, 4 if name != "c3_1m" else 2, seed=3)
+
+
+def test_long_forward_from_filters(hy):
+    # the workspace then holds the spectra and the four-step scratch
+    wl, inp = random_problem(1, 3, 65536, 2, seed=12)
+    h32 = oracle_filters(inp, wl).astype(np.float32)
+    a = run_forward(hy, inp, wl, h32, use_h=False)
+    b = run_forward(hy, inp, wl, h32, use_h=True)
+    assert np.array_equal(a, b)
+
+
+def test_long_wave_boundaries(hy):
+    # more sequences than one wave of the four-step scratch holds at 1M
+    # (8 per 64 MB wave): 10 sequences span two waves
+    wl, inp = random_problem(2, 5, 1 << 20, 1, seed=13)
+    h32 = (np.random.default_rng(1).standard_normal((1, 5, 1 << 20))
+           * np.exp(-np.arange(1 << 20) / 300.0)).astype(np.float32)
+    got = run_forward(hy, inp, wl, h32)
+    ref = oracle_forward(inp, h32.astype(np.float64), seqs=[(0, 0), (1, 4), (0, 3)])
+    assert_close(got[[0, 1, 0], [0, 4, 3]], ref, "f32", "waves")
