@@ -64,25 +64,33 @@ def peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# source files that define each kernel measured by ncu (the traffic figure
+# is dropped as soon as any of them changes)
+KERNEL_SOURCES = {
+    "fused1d_kernel": ["fused1d.cuh", "hyena_common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "subquadratic_sequence_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str, workload: str):
-    """Per-launch DRAM bytes of `kernel` on `workload` from the committed ncu
-    summary, if it was taken on the current kernel sources; else None."""
+    """Per-launch DRAM bytes (read + write) of `kernel` on `workload` from
+    profiles/traffic.json, if it was captured on the current sources of that
+    kernel; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)[f"{kernel}@{workload}"]
     except Exception:
         return None
-    return rec["dram_bytes_per_launch"] if rec.get("source_hash") == kernel_source_hash() else None
+    return rec["dram_bytes_per_launch"] if rec.get("source_hash") == kernel_source_hash(kernel) else None
 
 
 # ----------------------------------------------------------- clocks

@@ -305,6 +305,40 @@ struct Fft1d {
         });
     }
 
+    // Visit the bin pairs (k, M - k) of the RL folded layout (the real-FFT
+    // split): f(i1, i2, k, kind, w) with registers i1 (bin k) and i2 (bin
+    // M - k) and w = exp(-i pi k / M); kind 0 = a pair, 1 = bins 0 and M
+    // (both in register i1 = i2), 2 = bin M/2 alone (i1 = i2).
+    template <typename F>
+    static __device__ __forceinline__ void for_each_pair(int t, F&& f)
+    {
+        constexpr int R = P::RL, NCOL = M / R;
+        static_for<E / (2 * R)>([&](auto cc) {
+            constexpr int c = decltype(cc)::value;
+            const int u = t + c * T;
+            if (u != 0) {
+                const float2 wb = expi_pi<-1>((float)u / (float)M);
+                static_for<R>([&](auto rr) {
+                    constexpr int r = decltype(rr)::value;
+                    f((2 * c) * R + r, (2 * c + 1) * R + R - 1 - r, u + r * NCOL, 0,
+                      mul_w64<r * 32 / R, -1>(wb));
+                });
+            } else {
+                f(0, 0, 0, 1, make_float2(1.0f, 0.0f));
+                static_for<R / 2 - 1>([&](auto rr) {
+                    constexpr int r = decltype(rr)::value + 1;
+                    f(r, R - r, r * NCOL, 0, mul_w64<r * 32 / R, -1>(make_float2(1.0f, 0.0f)));
+                });
+                f(R / 2, R / 2, M / 2, 2, make_float2(0.0f, -1.0f));
+                const float2 wb = expi_pi<-1>(1.0f / (float)(2 * R));
+                static_for<R / 2>([&](auto rr) {
+                    constexpr int r = decltype(rr)::value;
+                    f(R + r, 2 * R - 1 - r, NCOL / 2 + r * NCOL, 0, mul_w64<r * 32 / R, -1>(wb));
+                });
+            }
+        });
+    }
+
     // Visit the data positions m = j + r M/RF (r < RF/2) of the RF folded
     // layout: f(register index, m).
     template <typename F>

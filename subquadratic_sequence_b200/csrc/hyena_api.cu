@@ -121,7 +121,8 @@ hyena_status_t hyena_filter_gen(const hyena_ffn_t* ffn, int N, int D, int L, flo
     hyena_status_t s = check_ffn(ffn);
     if (s != HYENA_OK) return s;
     if (!h || N < 1 || D < 1 || L < 1 || !aligned(h, 4)) return HYENA_ERR_INVALID_ARG;
-    if ((long)N * D > (1L << 30) || (long)N * D * (long)L > (1L << 40)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)N * D > 65535L * kFgRowTile || (long)N * D * (long)L > (1L << 40))
+        return HYENA_ERR_UNSUPPORTED;
     return filter_gen(ffn, N * D, D, L, L, 0, 0, false, h, (cudaStream_t)stream);
 }
 
@@ -131,7 +132,9 @@ hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C, int H, 
     hyena_status_t s = check_ffn(ffn);
     if (s != HYENA_OK) return s;
     if (!h || N < 1 || C < 1 || H < 1 || W < 1 || !aligned(h, 4)) return HYENA_ERR_INVALID_ARG;
-    if ((long)H * W > (1L << 30) || (long)N * C * (long)H * W > (1L << 40)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)H * W > (1L << 30) || (long)N * C > 65535L * kFgRowTile ||
+        (long)N * C * (long)H * W > (1L << 40))
+        return HYENA_ERR_UNSUPPORTED;
     return filter_gen(ffn, N * C, C, (long)H * W, 0, H, W, true, h, (cudaStream_t)stream);
 }
 

@@ -31,7 +31,7 @@ cudaError_t allow_smem(K kernel, size_t bytes)
 }
 
 template <typename K, typename A>
-hyena_status_t launch(K kernel, unsigned grid, int threads, size_t smem, cudaStream_t st, const A& a)
+hyena_status_t launch(K kernel, dim3 grid, int threads, size_t smem, cudaStream_t st, const A& a)
 {
     cudaError_t e = allow_smem(kernel, smem);
     if (e != cudaSuccess) return from_cuda(e);
