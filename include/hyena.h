@@ -158,6 +158,33 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* c
                                           void* y, void* workspace,
                                           size_t ws_bytes, void* stream);
 
+/* Size of the scratch array built into the library for
+ * hyena_fftconv_gate_forward_noalloc (16 MB on every device that loads the
+ * library, held until the process exits). */
+#define HYENA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* hyena_fftconv_gate_forward without a workspace, for callers that cannot
+ * allocate device memory: hosts that plan all device memory at start-up
+ * and hand a kernel only its inputs and outputs, and code where a
+ * cudaMalloc would synchronise the device or is not allowed.  The pages
+ * have no counterpart; this is an interface choice of this library.
+ * Same arguments and results as hyena_fftconv_gate_forward with the cached
+ * spectrum H (no h, no workspace).  Sequences longer than 16384 use a
+ * scratch array inside the library instead of a workspace:
+ *  - its device address is looked up (cudaGetSymbolAddress) on the first
+ *    call on each device; make that first call before any stream capture;
+ *  - one sequence's scratch, 8 L bytes, must fit it: L <= 2^21, else
+ *    HYENA_ERR_WORKSPACE;
+ *  - all calls on a device share it and it keeps the last call's contents
+ *    (nothing in it needs to start at zero); calls that overlap on the GPU
+ *    (other streams, other host threads) race on it, so order them.
+ * Allocates nothing (no cudaMalloc, no cudaFree). */
+HYENA_API hyena_status_t hyena_fftconv_gate_forward_noalloc(const void* v, const void* const* x,
+                                                            const float* H, const float* bias,
+                                                            int B, int D, int L, int N,
+                                                            hyena_dtype_t io, void* y,
+                                                            void* stream);
+
 /* ---------------------------------------------------------------- 2-D */
 
 /* Implicit 2-D filters h [N][C][H][W] float32 (features and window as in

@@ -54,6 +54,8 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv_workspace_size": ([i, i, i, i, i, i], sz),
         "hyena_fftconv_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp, vp,
                                         sz, vp], i),
+        "hyena_fftconv_gate_forward_noalloc": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp,
+                                                vp], i),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -186,3 +188,22 @@ def hyena_fftconv_gate_forward(v: torch.Tensor, xs, bias: torch.Tensor, *, H=Non
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
         ctypes.c_void_p(_dev(out, v.dtype, "y")), wp, wn, _stream(stream)))
     return out
+
+
+def hyena_fftconv_gate_forward_noalloc(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor, *,
+                                       out=None, stream=None):
+    """The forward without a workspace, for callers that cannot allocate
+    device memory: long sequences use the library's built-in 16 MB scratch
+    (shared by all calls on a device; order calls that could overlap)."""
+    B, D, L = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    _check("hyena_fftconv_gate_forward_noalloc", LIB.hyena_fftconv_gate_forward_noalloc(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), _stream(stream)))
+    return out
+
