@@ -192,6 +192,45 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_noalloc(const void* v, const
 HYENA_API hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C,
                                    int H, int W, float* h, void* stream);
 
+/* 2-D filter spectra Hs [N][C][2H][W] complex64 in the PACKED real 2-D DFT
+ * layout, for filters h [N][C][H][W] (offsets 0..H-1 x 0..W-1) zero-padded
+ * to 2H x 2W ("Handling Boundaries"; "Native ND Convolution": the N-D FFT):
+ * with X[ky][kx] the 2H x 2W DFT (kx = 0..W distinct bins),
+ *   slot [ky][kx] = X[ky][kx]                 for 1 <= kx < W,
+ *   slot [ky][0]  = F[ky], the 2H-point DFT over y of the complex column
+ *                   c[y] = R_y[0] + i R_y[W],
+ * where R_y[k] is the 2W-point DFT of row y (R_y[0], R_y[W] are real), so
+ *   X[ky][0] = (F[ky] + conj F[-ky]) / 2,  X[ky][W] = (F[ky] - conj F[-ky]) / (2i).
+ * H and W are powers of two in [16, 1024].  Alignment 16 bytes; Hs must
+ * not overlap h.  No workspace. */
+HYENA_API hyena_status_t hyena_filter_rfft2d(const float* h, int N, int C, int H, int W,
+                                             float* Hs, void* stream);
+
+/* Bytes of workspace hyena_fftconv2d_gate_forward needs (the spectra when
+ * spectrum_given = 0, plus the scratch of one wave of images);
+ * (size_t)-1 for invalid sizes. */
+HYENA_API size_t hyena_fftconv2d_workspace_size(int B, int C, int H, int W, int N,
+                                                hyena_dtype_t io, int spectrum_given);
+
+/* The order-N 2-D forward, per image (b, c):
+ *   z_0 = v,  z_n = x_n * (h_n (*) z_{n-1} + b_n z_{n-1}),  y = z_N
+ * with (*) the linear 2-D convolution
+ *   (h (*) u)[p][q] = sum_{i <= p, j <= q} h[i][j] u[p-i][q-j]
+ * computed on the grid zero-padded to 2H x 2W and cropped to H x W.
+ *   v, x_n, y [B][C][H][W] io; h [N][C][H][W] float32 or Hs [N][C][2H][W]
+ *   (hyena_filter_rfft2d; wins when both are given); bias [N][C];
+ *   x is a HOST array of N device pointers.
+ * workspace: hyena_fftconv2d_workspace_size(...) bytes, 256-byte aligned.
+ * H, W powers of two in [16, 1024]; 1 <= N <= HYENA_MAX_ORDER.
+ * Alignment: v, x_n, y, h, Hs 16 bytes; bias 4.  y must not overlap any
+ * input or the workspace. */
+HYENA_API hyena_status_t hyena_fftconv2d_gate_forward(const void* v, const void* const* x,
+                                                      const float* h, const float* Hs,
+                                                      const float* bias, int B, int C, int H,
+                                                      int W, int N, hyena_dtype_t io, void* y,
+                                                      void* workspace, size_t ws_bytes,
+                                                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -40,7 +40,7 @@ struct Fft2dArgs {
     const float2* Hs;              // [N][C][2H][W] packed 2-D spectra (column kernel)
     const float* bias;             // [N][C]
     float2* S;                     // scratch [wave][H][W] complex (conv) / spectra (filters)
-    int B, C, H;                   // W is a template parameter
+    int B, C, H, W;
     int q0;                        // first image of the wave (channel-major index)
     int nq;                        // images in the wave
     int n;                         // order handled by this launch
@@ -71,10 +71,13 @@ struct Fft2dRows {
     using F = Fft1d<LOG2W>;
     static constexpr int W = 1 << LOG2W;
 
-    // forward row FFT of the registers and split into a packed row
-    static __device__ __forceinline__ void forward_split(float2* a, float2* sm, float2* row, int t)
+    // forward row FFT of the registers (every thread: the passes hold
+    // barriers) and, if `store`, the split into a packed row
+    static __device__ __forceinline__ void forward_split(float2* a, float2* sm, float2* row, int t,
+                                                         bool store)
     {
         F::forward(a, sm, t);
+        if (!store) return;
         F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
             if (kind == 1) {
                 const float2 z = a[i1];
@@ -151,14 +154,7 @@ fft2d_row_kernel(Fft2dArgs a)
         }
         const PT* vp = reinterpret_cast<const PT*>(a.v) + (img * a.H + yrow) * (W / 2);
         F::for_each_io(t, [&](int i, int m) { arr[i] = IOP::load(vp + m); });
-        // every thread runs the FFT (barriers); only active rows store
-        float2 dummy[1];
-        (void)dummy;
-        if (active) {
-            R::forward_split(arr, sm, row, t);
-        } else {
-            F::forward(arr, sm, t);
-        }
+        R::forward_split(arr, sm, row, t, active);
     } else {
         const int c = q / a.B, b = q % a.B;
         const size_t img = (size_t)b * a.C + c;
@@ -180,11 +176,7 @@ fft2d_row_kernel(Fft2dArgs a)
                 F::for_each_io(t, [&](int i, int m) { IOP::store(yp + m, arr[i]); });
             }
         } else {
-            if (active) {
-                R::forward_split(arr, sm, row, t);
-            } else {
-                F::forward(arr, sm, t);
-            }
+            R::forward_split(arr, sm, row, t, active);
         }
     }
 }
@@ -204,14 +196,15 @@ struct Fft2dCols {
 // multiply with the packed 2-D filter spectrum and the bias, inverse column
 // FFTs, rows y < H back to the scratch.  SPECTRUM = true: forward column
 // FFTs of rows y < H of the packed spectra, all 2H rows written back.
-template <int LOG2H2, int LOG2W, bool SPECTRUM>
+template <int LOG2H2, bool SPECTRUM>
 __global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS)
 fft2d_col_kernel(Fft2dArgs a)
 {
     using CL = Fft2dCols<LOG2H2>;
     using FC = typename CL::FC;
-    constexpr int H2 = CL::H2, TC = CL::TC, W = 1 << LOG2W, HH = H2 / 2;
-    constexpr int CTAS_PER_IMG = W / TC;
+    constexpr int H2 = CL::H2, TC = CL::TC, HH = H2 / 2;
+    const int W = a.W;
+    const int CTAS_PER_IMG = W / TC;
     extern __shared__ __align__(16) float2 smem_c2[];
 
     const int qi = blockIdx.x / CTAS_PER_IMG;

@@ -10,14 +10,18 @@
 // decay window exp(-alpha_d i / div) (2-D: exp(-alpha_c (iy + ix) / div)
 // as the product of the two axis windows).
 //
-// One CTA takes a tile of 64 consecutive positions and up to 128 head rows
-// (a 2-D grid: position tiles x row tiles).  All 256 threads evaluate the
-// three sine layers -- four threads per position, 16 output units each, so
-// every thread runs 16 independent accumulation chains -- with weights and
-// activations in shared memory; then the head runs as a 64-position x
-// 128-row x 64 product out of shared memory and h is written coalesced
-// along the position.  The layers are recomputed by every row tile of a
-// position tile: 64 x 9.3k multiply-adds, cheaper than a scratch round trip.
+// Three launches, no recomputation:
+//  layers: all threads of a CTA evaluate the three sine layers for 16
+//          positions (16 threads per position, 4 output units each, weights
+//          broadcast from shared memory) and stash a3 [64][positions] in
+//          the LAST 64 rows of h (they are outputs too, written last);
+//  head:   h[r][p] = (sum_j Wout[r][j] a3[j][p]) * window for the rows
+//          before the stash, as 128-row x 64-position tiles out of shared
+//          memory, written coalesced along the position;
+//  tail:   the head for the 64 stash rows: each CTA loads its own
+//          position tile of a3 into shared memory before overwriting it.
+// With fewer than 64 head rows the layers are evaluated inside the head
+// kernel instead (one launch).
 #pragma once
 
 #include "hyena_common.cuh"
@@ -38,43 +42,73 @@ struct FilterGenArgs {
     float* h;                      // [rows][positions]
 };
 
-constexpr int kFgTile = 64;        // positions per CTA
+constexpr int kFgTile = 64;        // positions per head CTA
 constexpr int kFgRowTile = 128;    // head rows per CTA
 constexpr int kFgThreads = 256;
+constexpr int kFgLayerPos = 16;    // positions per layers CTA (16 threads each)
 constexpr int kFgAS = kFgTile + 1; // activation row stride
 constexpr int kFgOS = kFfnWidth + 1;
-// weight row strides: odd, so the four units a position's threads read at
-// once (rows 4 jj + q, q < 4) sit on four different banks
+// weight row strides: odd, so the units the threads of one position read
+// at once sit on different banks
 constexpr int kFgW1S = kFfnMaxIn + 1;
 constexpr int kFgWS = kFfnWidth + 1;
-// dynamic shared memory (floats): W1 [64][67], W2, W3 [64][65], two
-// activation buffers [64][65]; the head's Wout tile [128][65] reuses the
-// weight region
 constexpr int kFgWRegion = kFfnWidth * kFgW1S + 2 * kFfnWidth * kFgWS;
+// layers kernel shared memory (floats): weights + two activation buffers
+constexpr size_t kFgLayerSmemBytes = sizeof(float) * (kFgWRegion + 2 * kFfnWidth * (kFgLayerPos + 1));
+// head kernel shared memory (floats): Wout tile [128][65] + a3 tile [64][65]
+constexpr size_t kFgHeadSmemBytes = sizeof(float) * (kFgRowTile * kFgOS + kFfnWidth * kFgAS);
+// single-launch path (few rows): weights + Wout tile + two activation tiles
+constexpr size_t kFgFusedSmemBytes = sizeof(float) * (kFgWRegion + 2 * kFfnWidth * kFgAS);
 static_assert(kFgRowTile * kFgOS <= kFgWRegion, "Wout tile fits the weight region");
-constexpr size_t kFgSmemBytes = sizeof(float) * (kFgWRegion + 2 * kFfnWidth * kFgAS);
 
+// Positional features of position `pos` in the canonical slots (1-D:
+// [t, (sin, cos) band 1..16]; 2-D: [ty, tx, (sin, cos) y-band 1..16,
+// (sin, cos) x-band 1..16]).
 template <bool TWO_D>
-__global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
+__device__ __forceinline__ void features(const FilterGenArgs& a, long pos, float* phi)
 {
-    extern __shared__ __align__(16) float fg_smem[];
-    float* sW1 = fg_smem;                                   // [64][67]
-    float* sW2 = sW1 + kFfnWidth * kFgW1S;                  // [64][65]
-    float* sW3 = sW2 + kFfnWidth * kFgWS;                   // [64][65]
-    float* sOut = fg_smem;                                  // [128][65], after the layers
-    float* sA = fg_smem + kFgWRegion;                       // [64][65]  a1, a3
-    float* sB = sA + kFfnWidth * kFgAS;                     // [64][65]  a2
+#pragma unroll
+    for (int c = 0; c < kFfnMaxIn; ++c) phi[c] = 0.0f;
+    if constexpr (!TWO_D) {
+        const int i = (int)pos;
+        phi[0] = (float)i / (float)a.L;
+#pragma unroll
+        for (int k = 1; k <= 16; ++k) {
+            if (k > a.n_bands) break;
+            // angle 2 pi k i / L reduced exactly: 2 pi ((k i) mod L) / L
+            const int qk = (int)(((long)k * i) % a.L);
+            float sn, cs;
+            sincospif(2.0f * (float)qk / (float)a.L, &sn, &cs);
+            phi[2 * k - 1] = sn;
+            phi[2 * k] = cs;
+        }
+    } else {
+        const int iy = (int)(pos / a.Ww), ix = (int)(pos % a.Ww);
+        phi[0] = (float)iy / (float)a.Hh;
+        phi[1] = (float)ix / (float)a.Ww;
+#pragma unroll
+        for (int k = 1; k <= 16; ++k) {
+            if (k > a.n_bands) break;
+            float sn, cs;
+            const int qy = (int)(((long)k * iy) % a.Hh);
+            sincospif(2.0f * (float)qy / (float)a.Hh, &sn, &cs);
+            phi[2 * k] = sn;
+            phi[2 * k + 1] = cs;
+            const int qx = (int)(((long)k * ix) % a.Ww);
+            sincospif(2.0f * (float)qx / (float)a.Ww, &sn, &cs);
+            phi[2 + 2 * 16 + 2 * (k - 1)] = sn;
+            phi[2 + 2 * 16 + 2 * (k - 1) + 1] = cs;
+        }
+    }
+}
 
+// Stage W1 (canonical feature slots), W2, W3 into shared memory, zero
+// padded to 64 units (sin(0) = 0: padded units contribute nothing).
+template <bool TWO_D>
+__device__ __forceinline__ void stage_weights(const FilterGenArgs& a, float* sW1, float* sW2, float* sW3)
+{
     const int tid = threadIdx.x;
-    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
-    const long p0 = (long)blockIdx.x * kFgTile;
-    const int r0 = blockIdx.y * kFgRowTile;
-
-    // W1's columns go to a canonical layout in which every feature has a
-    // fixed slot: 1-D [t, (sin, cos) band 1..16]; 2-D [ty, tx, (sin, cos)
-    // y-band 1..16, (sin, cos) x-band 1..16].  Units beyond `width` are
-    // zero: sin(0) = 0, so they contribute nothing.
-    for (int e = tid; e < kFfnWidth * kFfnMaxIn; e += kFgThreads) {
+    for (int e = tid; e < kFfnWidth * kFfnMaxIn; e += blockDim.x) {
         const int r = e / kFfnMaxIn, c = e % kFfnMaxIn;
         int src = -1;
         if constexpr (!TWO_D) {
@@ -86,63 +120,38 @@ __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
         }
         sW1[r * kFgW1S + c] = (r < a.width && src >= 0) ? __ldg(a.W1 + r * a.n_in + src) : 0.0f;
     }
-    for (int e = tid; e < kFfnWidth * kFfnWidth; e += kFgThreads) {
+    for (int e = tid; e < kFfnWidth * kFfnWidth; e += blockDim.x) {
         const int r = e / kFfnWidth, c = e % kFfnWidth;
         const bool in = r < a.width && c < a.width;
         sW2[r * kFgWS + c] = in ? __ldg(a.W2 + r * a.width + c) : 0.0f;
         sW3[r * kFgWS + c] = in ? __ldg(a.W3 + r * a.width + c) : 0.0f;
     }
+}
 
-    // ---- three sine layers: thread (p, q) computes units 4 jj + q
-    // (jj < 16) of position p0 + p
-    const int p = tid / 4, q = tid % 4;
+// The three sine layers for position p of a tile: UPT = 64 / TPP output
+// units per thread, TPP threads per position (thread q of the position owns
+// units TPP * jj + q).  a1 and a3 end up in sA[j * AS + p], a2 in sB.
+template <bool TWO_D, int TPP, int AS>
+__device__ __forceinline__ void sine_layers(const FilterGenArgs& a, long pos, int p, int q,
+                                            const float* sW1, const float* sW2, const float* sW3,
+                                            float* sA, float* sB)
+{
+    constexpr int UPT = kFfnWidth / TPP;
+    constexpr int NIN = TWO_D ? kFfnMaxIn : 33;        // 1-D features use slots < 33
     {
-        const long pos = min(p0 + p, npos - 1);
         float phi[kFfnMaxIn];
+        features<TWO_D>(a, pos, phi);
+        __syncthreads();                                   // weights staged by all threads
+        float acc[UPT];
 #pragma unroll
-        for (int c = 0; c < kFfnMaxIn; ++c) phi[c] = 0.0f;
-        if constexpr (!TWO_D) {
-            const int i = (int)pos;
-            phi[0] = (float)i / (float)a.L;
+        for (int jj = 0; jj < UPT; ++jj) acc[jj] = 0.0f;
 #pragma unroll
-            for (int k = 1; k <= (kFfnMaxIn - 1) / 2; ++k) {
-                if (k > a.n_bands) break;
-                // angle 2 pi k i / L reduced exactly: 2 pi ((k i) mod L) / L
-                const int qk = (int)(((long)k * i) % a.L);
-                float sn, cs;
-                sincospif(2.0f * (float)qk / (float)a.L, &sn, &cs);
-                phi[2 * k - 1] = sn;
-                phi[2 * k] = cs;
-            }
-        } else {
-            const int iy = (int)(pos / a.Ww), ix = (int)(pos % a.Ww);
-            phi[0] = (float)iy / (float)a.Hh;
-            phi[1] = (float)ix / (float)a.Ww;
+        for (int c = 0; c < NIN; ++c)
 #pragma unroll
-            for (int k = 1; k <= (kFfnMaxIn - 2) / 4; ++k) {
-                if (k > a.n_bands) break;
-                float sn, cs;
-                const int qy = (int)(((long)k * iy) % a.Hh);
-                sincospif(2.0f * (float)qy / (float)a.Hh, &sn, &cs);
-                phi[2 * k] = sn;
-                phi[2 * k + 1] = cs;
-                const int qx = (int)(((long)k * ix) % a.Ww);
-                sincospif(2.0f * (float)qx / (float)a.Ww, &sn, &cs);
-                phi[2 + 2 * 16 + 2 * (k - 1)] = sn;
-                phi[2 + 2 * 16 + 2 * (k - 1) + 1] = cs;
-            }
-        }
-        __syncthreads();                                   // weights staged
-        float acc[16];
+            for (int jj = 0; jj < UPT; ++jj)
+                acc[jj] = fmaf(sW1[(TPP * jj + q) * kFgW1S + c], phi[c], acc[jj]);
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.0f;
-#pragma unroll
-        for (int c = 0; c < kFfnMaxIn; ++c)
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj)
-                acc[jj] = fmaf(sW1[(4 * jj + q) * kFgW1S + c], phi[c], acc[jj]);
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) sA[(4 * jj + q) * kFgAS + p] = sinf(acc[jj]);
+        for (int jj = 0; jj < UPT; ++jj) sA[(TPP * jj + q) * AS + p] = sinf(acc[jj]);
     }
     __syncthreads();
 #pragma unroll 1
@@ -150,29 +159,35 @@ __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
         const float* Wl = layer == 0 ? sW2 : sW3;
         const float* in = layer == 0 ? sA : sB;
         float* out = layer == 0 ? sB : sA;
-        float acc[16];
+        float acc[UPT];
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.0f;
+        for (int jj = 0; jj < UPT; ++jj) acc[jj] = 0.0f;
 #pragma unroll 8
         for (int c = 0; c < kFfnWidth; ++c) {
-            const float x = in[c * kFgAS + p];
+            const float x = in[c * AS + p];
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) acc[jj] = fmaf(Wl[(4 * jj + q) * kFgWS + c], x, acc[jj]);
+            for (int jj = 0; jj < UPT; ++jj) acc[jj] = fmaf(Wl[(TPP * jj + q) * kFgWS + c], x, acc[jj]);
         }
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) out[(4 * jj + q) * kFgAS + p] = sinf(acc[jj]);
+        for (int jj = 0; jj < UPT; ++jj) out[(TPP * jj + q) * AS + p] = sinf(acc[jj]);
         __syncthreads();
     }
+}
 
-    // ---- head: out[r][p] = sum_j Wout[r][j] a3[j][p], times the window.
-    // Thread (ty, tx) of a 16 x 16 grid computes rows ty + 16 i (i < 8) and
-    // positions tx + 16 k (k < 4).
+// Head for rows r0 .. r0+127 (< r_end) and positions p0 .. p0+63 from the
+// a3 tile in sA [64][kFgAS] and the Wout tile staged into sOut.
+template <bool TWO_D>
+__device__ __forceinline__ void head_tile(const FilterGenArgs& a, long npos, long p0, int r0, int r_end,
+                                          float* sOut, const float* sA)
+{
+    const int tid = threadIdx.x;
     for (int e = tid; e < kFgRowTile * kFfnWidth; e += kFgThreads) {
         const int r = e / kFfnWidth, j = e % kFfnWidth;
-        sOut[r * kFgOS + j] = (r0 + r < a.rows && j < a.width)
+        sOut[r * kFgOS + j] = (r0 + r < r_end && j < a.width)
                                   ? __ldg(a.Wout + (long)(r0 + r) * a.width + j) : 0.0f;
     }
     __syncthreads();
+    // thread (ty, tx) of a 16 x 16 grid: rows ty + 16 i (i < 8), positions tx + 16 k (k < 4)
     const int tx = tid % 16, ty = tid / 16;
     float acc[8][4];
 #pragma unroll
@@ -194,7 +209,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int r = r0 + ty + 16 * i;
-        if (r >= a.rows) continue;
+        if (r >= r_end) continue;
         const float al = __ldg(a.alpha + r % a.D);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -206,6 +221,75 @@ __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
             a.h[(long)r * npos + pos] = acc[i][k] * expf(-al * dist * a.inv_div);
         }
     }
+}
+
+// Layers kernel: a3 of 16 positions into the stash rows (the last 64 rows
+// of h), a3[j][pos] at h[(rows - 64 + j) * npos + pos].
+template <bool TWO_D>
+__global__ void __launch_bounds__(kFgThreads) filter_layers_kernel(FilterGenArgs a)
+{
+    extern __shared__ __align__(16) float fg_smem[];
+    constexpr int AS = kFgLayerPos + 1;
+    float* sW1 = fg_smem;
+    float* sW2 = sW1 + kFfnWidth * kFgW1S;
+    float* sW3 = sW2 + kFfnWidth * kFgWS;
+    float* sA = fg_smem + kFgWRegion;
+    float* sB = sA + kFfnWidth * AS;
+    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long p0 = (long)blockIdx.x * kFgLayerPos;
+    const int p = threadIdx.x / 16, q = threadIdx.x % 16;
+    stage_weights<TWO_D>(a, sW1, sW2, sW3);
+    sine_layers<TWO_D, 16, AS>(a, min(p0 + p, npos - 1), p, q, sW1, sW2, sW3, sA, sB);
+    // stash a3 (coalesced along the position)
+    float* stash = a.h + (long)(a.rows - kFfnWidth) * npos;
+    for (int e = threadIdx.x; e < kFfnWidth * kFgLayerPos; e += kFgThreads) {
+        const int j = e / kFgLayerPos, pp = e % kFgLayerPos;
+        if (p0 + pp < npos) stash[(long)j * npos + p0 + pp] = sA[j * AS + pp];
+    }
+}
+
+// Head kernel.  TAIL = false: rows 0 .. rows-65 (grid.y over 128-row
+// tiles); TAIL = true: the 64 stash rows, each CTA reading its own tile of
+// a3 before overwriting it.
+template <bool TWO_D, bool TAIL>
+__global__ void __launch_bounds__(kFgThreads) filter_head_kernel(FilterGenArgs a)
+{
+    extern __shared__ __align__(16) float fg_smem[];
+    float* sOut = fg_smem;                                   // [128][65]
+    float* sA = fg_smem + kFgRowTile * kFgOS;                // [64][65]
+    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long p0 = (long)blockIdx.x * kFgTile;
+    const int stash_row = a.rows - kFfnWidth;
+    const float* stash = a.h + (long)stash_row * npos;
+    for (int e = threadIdx.x; e < kFfnWidth * kFgTile; e += kFgThreads) {
+        const int j = e / kFgTile, pp = e % kFgTile;
+        sA[j * kFgAS + pp] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
+    }
+    if constexpr (TAIL) {
+        head_tile<TWO_D>(a, npos, p0, stash_row, a.rows, sOut, sA);   // stages Wout, syncs
+    } else {
+        head_tile<TWO_D>(a, npos, p0, blockIdx.y * kFgRowTile, stash_row, sOut, sA);
+    }
+}
+
+// Single launch for few rows (< 64 + 1): every CTA evaluates the layers of
+// its 64 positions, then the head for all rows.
+template <bool TWO_D>
+__global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
+{
+    extern __shared__ __align__(16) float fg_smem[];
+    float* sW1 = fg_smem;
+    float* sW2 = sW1 + kFfnWidth * kFgW1S;
+    float* sW3 = sW2 + kFfnWidth * kFgWS;
+    float* sOut = fg_smem;                                   // after the layers
+    float* sA = fg_smem + kFgWRegion;
+    float* sB = sA + kFfnWidth * kFgAS;
+    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long p0 = (long)blockIdx.x * kFgTile;
+    const int p = threadIdx.x / 4, q = threadIdx.x % 4;
+    stage_weights<TWO_D>(a, sW1, sW2, sW3);
+    sine_layers<TWO_D, 4, kFgAS>(a, min(p0 + p, npos - 1), p, q, sW1, sW2, sW3, sA, sB);
+    head_tile<TWO_D>(a, npos, p0, 0, a.rows, sOut, sA);
 }
 
 }  // namespace hyena
