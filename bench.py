@@ -41,6 +41,13 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 def describe(wl: synth.Workload) -> dict:
+    if wl.kind == "2d":
+        return {"workload": f"{wl.name}: order-{wl.N} Hyena 2-D operator, B={wl.B}, C={wl.D}, "
+                            f"{wl.H}x{wl.W} grid (padded to {2 * wl.H}x{2 * wl.W}), {wl.io} storage, fp32 compute",
+                "N": wl.N, "B": wl.B, "C": wl.D, "H": wl.H, "W": wl.W, "io": wl.io,
+                "filters": f"implicit FFN over (y/H, x/W) (3 sine layers of width {synth.WIDTH}, "
+                           f"{synth.N_BANDS} bands per axis) x separable decay, regenerated every step",
+                "l2": "flushed (256 MB write) before every timed step"}
     return {"workload": f"{wl.name}: order-{wl.N} Hyena 1-D operator, B={wl.B}, D={wl.D}, "
                         f"L={wl.L}, {wl.io} storage, fp32 compute",
             "N": wl.N, "B": wl.B, "D": wl.D, "L": wl.L, "io": wl.io,
@@ -50,13 +57,15 @@ def describe(wl: synth.Workload) -> dict:
 
 
 def alg_bytes_forward(wl: synth.Workload) -> int:
-    """Algorithmic HBM bytes of one fused forward: v, x_1..x_N, y plus the
-    N*D packed spectra (L complex64 slots each)."""
+    """Algorithmic HBM bytes of one forward call: v, x_1..x_N, y plus the
+    N*D packed spectra (L complex64 slots each; 2H x W for the 2-D grid)."""
+    if wl.kind == "2d":
+        return (wl.N + 2) * wl.positions * wl.io_bytes + wl.N * wl.D * 2 * wl.H * wl.W * 8
     return (wl.N + 2) * wl.B * wl.D * wl.L * wl.io_bytes + wl.N * wl.D * wl.L * 8
 
 
 def long_path(wl: synth.Workload) -> bool:
-    return wl.L > 16384
+    return wl.kind == "1d" and wl.L > 16384
 
 
 def waves(nseq: int, L: int) -> int:
@@ -65,17 +74,27 @@ def waves(nseq: int, L: int) -> int:
 
 
 def launches_forward(wl: synth.Workload) -> int:
-    """Kernel launches of one hyena_fftconv_gate_forward call."""
+    """Kernel launches of one forward call."""
+    if wl.kind == "2d":
+        return waves(wl.B * wl.D, wl.H * wl.W) * (1 + 2 * wl.N)
     return waves(wl.B * wl.D, wl.L) * (1 + 2 * wl.N) if long_path(wl) else 1
 
 
 def launches_rfft(wl: synth.Workload) -> int:
+    if wl.kind == "2d":
+        return 2
     return waves(wl.N * wl.D, wl.L) * 2 if long_path(wl) else 1
+
+
+def launches_filter_gen(wl: synth.Workload) -> int:
+    return 3 if wl.N * wl.D > 64 else 1
 
 
 def forward_kernel(wl: synth.Workload) -> str:
     """The timed unit of the roofline: the forward call (one fused kernel,
     or the 2N+1 four-step kernels of each wave)."""
+    if wl.kind == "2d":
+        return "fft2d_row_kernel+fft2d_col_kernel (hyena_fftconv2d_gate_forward, all launches)"
     if long_path(wl):
         return "fourstep_row_kernel+fourstep_col_kernel (hyena_fftconv_gate_forward, all launches)"
     return "fused1d_kernel (hyena_fftconv_gate_forward)"
@@ -176,33 +195,63 @@ class ClockSampler:
 
 # ------------------------------------------------------------ GPU arm
 
+class Ranks:
+    """One process per GPU (torchrun environment).  The ranks run the same
+    workload on their own data (weak scaling) and meet only to line up the
+    timed region (barriers) and to take the max time over ranks."""
+
+    def __init__(self, backend: str):
+        import torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        if backend == "nccl":
+            torch.cuda.set_device(self.local)
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"device_id": torch.device("cuda", self.local)} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        import torch
+        import torch.distributed as dist
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+def throughput(positions_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job channel-positions per second: the units all ranks processed
+    over the slowest rank's time."""
+    return positions_per_rank * world * steps / (total_ms / 1e3)
+
+
 def run_gpu(args, wl: synth.Workload) -> dict | None:
     import torch
-    import torch.distributed as dist
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py: no CUDA device (the path has no CPU fallback)")
     from subquadratic_sequence_b200 import hyena
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl")
+    world, rank, local = ranks.world, ranks.rank, ranks.local
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     inp = synth.make_inputs(wl)
     io = torch.bfloat16 if wl.io == "bf16" else torch.float32
@@ -214,27 +263,42 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     xs = [to_dev(x, io) for x in inp["x"]]
     b = to_dev(inp["b"])
     W = [to_dev(inp[k]) for k in ("W1", "W2", "W3", "Wout", "alpha")]
-    h = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.float32)
-    H = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.complex64)
     y = torch.empty_like(v)
     flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
     stream = torch.cuda.current_stream()
-    # workspaces (four-step scratch for L > 16384), allocated once
-    ws_rfft_n = hyena.hyena_filter_rfft_workspace_size(wl.N, wl.D, wl.L)
-    ws_fwd_n = hyena.hyena_fftconv_workspace_size(wl.B, wl.D, wl.L, wl.N, hyena.io_dtype(v), True)
-    ws_rfft = torch.empty(ws_rfft_n, device="cuda", dtype=torch.uint8) if ws_rfft_n else None
-    ws_fwd = torch.empty(ws_fwd_n, device="cuda", dtype=torch.uint8) if ws_fwd_n else None
+    if wl.kind == "2d":
+        h = torch.empty((wl.N, wl.D, wl.H, wl.W), device="cuda", dtype=torch.float32)
+        H = torch.empty((wl.N, wl.D, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
+        ws_n = hyena.hyena_fftconv2d_workspace_size(wl.B, wl.D, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
+        ws_fwd = torch.empty(ws_n, device="cuda", dtype=torch.uint8)
 
-    def forward():
-        hyena.hyena_fftconv_gate_forward(v, xs, b, H=H, out=y, workspace=ws_fwd)
+        def forward():
+            hyena.hyena_fftconv2d_gate_forward(v, xs, b, Hs=H, out=y, workspace=ws_fwd)
 
-    def step():
-        hyena.hyena_filter_gen(*W, wl.N, wl.D, wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
-                               decay_div=synth.DECAY_DIV, out=h)
-        hyena.hyena_filter_rfft(h, out=H, workspace=ws_rfft)
-        forward()
+        def step():
+            hyena.hyena_filter_gen_2d(*W, wl.N, wl.D, wl.H, wl.W, n_bands=synth.N_BANDS,
+                                      width=synth.WIDTH, decay_div=synth.DECAY_DIV, out=h)
+            hyena.hyena_filter_rfft2d(h, out=H)
+            forward()
+    else:
+        h = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.float32)
+        H = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.complex64)
+        # workspaces (four-step scratch for L > 16384), allocated once
+        ws_rfft_n = hyena.hyena_filter_rfft_workspace_size(wl.N, wl.D, wl.L)
+        ws_fwd_n = hyena.hyena_fftconv_workspace_size(wl.B, wl.D, wl.L, wl.N, hyena.io_dtype(v), True)
+        ws_rfft = torch.empty(ws_rfft_n, device="cuda", dtype=torch.uint8) if ws_rfft_n else None
+        ws_fwd = torch.empty(ws_fwd_n, device="cuda", dtype=torch.uint8) if ws_fwd_n else None
 
-    launches_per_step = 1 + launches_rfft(wl) + launches_forward(wl)
+        def forward():
+            hyena.hyena_fftconv_gate_forward(v, xs, b, H=H, out=y, workspace=ws_fwd)
+
+        def step():
+            hyena.hyena_filter_gen(*W, wl.N, wl.D, wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                   decay_div=synth.DECAY_DIV, out=h)
+            hyena.hyena_filter_rfft(h, out=H, workspace=ws_rfft)
+            forward()
+
+    launches_per_step = launches_filter_gen(wl) + launches_rfft(wl) + launches_forward(wl)
 
     # ---- warm-up
     for _ in range(args.warmup):
@@ -308,14 +372,12 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(bb) for a, bb in eev))
 
-    if world > 1:
-        barrier()
-        dist.destroy_process_group()
+    ranks.close()
     if rank != 0:
         return None
 
     positions = wl.positions * world
-    value = positions * args.steps / (total_ms / 1e3)
+    value = throughput(wl.positions, world, args.steps, total_ms)
     peak, peak_kind = peaks()
     achieved = alg_bytes_forward(wl) / (fwd_ms / 1e3) / 1e9
     line = {
@@ -412,8 +474,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="c1", choices=[k for k, w in synth.WORKLOADS.items()
-                                                         if w.kind == "1d"])
+    ap.add_argument("--workload", default="c1", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
