@@ -18,8 +18,8 @@
 //  head:   h[r][p] = (sum_j Wout[r][j] a3[j][p]) * window for the rows
 //          before the stash, as 128-row x 64-position tiles out of shared
 //          memory, written coalesced along the position;
-//  tail:   the head for the 64 stash rows: each CTA loads its own
-//          position tile of a3 into shared memory before overwriting it.
+//  tail:   the head for the 64 stash rows, 16 positions per CTA: each CTA
+//          loads its own tile of a3 into shared memory before overwriting it.
 // With fewer than 64 head rows the layers are evaluated inside the head
 // kernel instead (one launch).
 #pragma once
@@ -55,8 +55,14 @@ constexpr int kFgWS = kFfnWidth + 1;
 constexpr int kFgWRegion = kFfnWidth * kFgW1S + 2 * kFfnWidth * kFgWS;
 // layers kernel shared memory (floats): weights + two activation buffers
 constexpr size_t kFgLayerSmemBytes = sizeof(float) * (kFgWRegion + 2 * kFfnWidth * (kFgLayerPos + 1));
-// head kernel shared memory (floats): Wout tile [128][65] + a3 tile [64][65]
-constexpr size_t kFgHeadSmemBytes = sizeof(float) * (kFgRowTile * kFgOS + kFfnWidth * kFgAS);
+// head kernel shared memory (floats): the Wout tile transposed [64][132]
+// and the a3 tile [64][68]; rows 16-byte aligned for 128-bit loads
+constexpr int kFgWTS = kFgRowTile + 4;
+constexpr int kFgA4S = kFgTile + 4;
+constexpr size_t kFgHeadSmemBytes = sizeof(float) * (kFfnWidth * kFgWTS + kFfnWidth * kFgA4S);
+// tail kernel: 16 positions x the 64 stash rows per CTA
+constexpr int kFgTailPos = 16;
+constexpr size_t kFgTailSmemBytes = sizeof(float) * (kFfnWidth * kFgOS + kFfnWidth * (kFgTailPos + 1));
 // single-launch path (few rows): weights + Wout tile + two activation tiles
 constexpr size_t kFgFusedSmemBytes = sizeof(float) * (kFgWRegion + 2 * kFfnWidth * kFgAS);
 static_assert(kFgRowTile * kFgOS <= kFgWRegion, "Wout tile fits the weight region");
@@ -248,27 +254,109 @@ __global__ void __launch_bounds__(kFgThreads) filter_layers_kernel(FilterGenArgs
     }
 }
 
-// Head kernel.  TAIL = false: rows 0 .. rows-65 (grid.y over 128-row
-// tiles); TAIL = true: the 64 stash rows, each CTA reading its own tile of
-// a3 before overwriting it.
-template <bool TWO_D, bool TAIL>
+// Head kernel: rows 0 .. rows-65 as 128-row x 64-position tiles (grid.y
+// over row tiles).  Thread (ty, tx) computes rows 8 ty + i (i < 8) and
+// positions 4 tx + k (k < 4): per unit j one 128-bit load of 4 a3 values and
+// two of 8 Wout values for 32 multiply-adds.
+template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_head_kernel(FilterGenArgs a)
 {
     extern __shared__ __align__(16) float fg_smem[];
-    float* sOut = fg_smem;                                   // [128][65]
-    float* sA = fg_smem + kFgRowTile * kFgOS;                // [64][65]
+    float* sWT = fg_smem;                                   // [64][132]: Wout tile, transposed
+    float* sA = fg_smem + kFfnWidth * kFgWTS;               // [64][68]:  a3 tile
     const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
     const long p0 = (long)blockIdx.x * kFgTile;
+    const int r0 = blockIdx.y * kFgRowTile;
     const int stash_row = a.rows - kFfnWidth;
     const float* stash = a.h + (long)stash_row * npos;
-    for (int e = threadIdx.x; e < kFfnWidth * kFgTile; e += kFgThreads) {
+    const int tid = threadIdx.x;
+    for (int e = tid; e < kFfnWidth * kFgTile; e += kFgThreads) {
         const int j = e / kFgTile, pp = e % kFgTile;
-        sA[j * kFgAS + pp] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
+        sA[j * kFgA4S + pp] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
     }
-    if constexpr (TAIL) {
-        head_tile<TWO_D>(a, npos, p0, stash_row, a.rows, sOut, sA);   // stages Wout, syncs
-    } else {
-        head_tile<TWO_D>(a, npos, p0, blockIdx.y * kFgRowTile, stash_row, sOut, sA);
+    for (int e = tid; e < kFgRowTile * kFfnWidth; e += kFgThreads) {
+        const int r = e / kFfnWidth, j = e % kFfnWidth;
+        sWT[j * kFgWTS + r] = (r0 + r < stash_row && j < a.width)
+                                  ? __ldg(a.Wout + (long)(r0 + r) * a.width + j) : 0.0f;
+    }
+    __syncthreads();
+    const int tx = tid % 16, ty = tid / 16;
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[i][k] = 0.0f;
+#pragma unroll 4
+    for (int j = 0; j < kFfnWidth; ++j) {
+        const float4 x4 = *reinterpret_cast<const float4*>(sA + j * kFgA4S + 4 * tx);
+        const float4 w0 = *reinterpret_cast<const float4*>(sWT + j * kFgWTS + 8 * ty);
+        const float4 w1 = *reinterpret_cast<const float4*>(sWT + j * kFgWTS + 8 * ty + 4);
+        const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const float x[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[i][k] = fmaf(w[i], x[k], acc[i][k]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = r0 + 8 * ty + i;
+        if (r >= stash_row) continue;
+        const float al = __ldg(a.alpha + r % a.D);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const long pos = p0 + 4 * tx + k;
+            if (pos >= npos) continue;
+            float dist;   // the window's argument: i (1-D) or iy + ix (2-D)
+            if constexpr (!TWO_D) dist = (float)pos;
+            else dist = (float)(pos / a.Ww) + (float)(pos % a.Ww);
+            a.h[(long)r * npos + pos] = acc[i][k] * expf(-al * dist * a.inv_div);
+        }
+    }
+}
+
+// Tail kernel: the 64 stash rows for 16 positions per CTA; each CTA reads
+// its own 64 x 16 tile of a3 before overwriting exactly that tile.
+template <bool TWO_D>
+__global__ void __launch_bounds__(kFgThreads) filter_tail_kernel(FilterGenArgs a)
+{
+    extern __shared__ __align__(16) float fg_smem[];
+    constexpr int AS = kFgTailPos + 1;
+    float* sW = fg_smem;                                    // [64][65]: Wout stash rows
+    float* sA = fg_smem + kFfnWidth * kFgOS;                // [64][17]: a3 tile
+    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long p0 = (long)blockIdx.x * kFgTailPos;
+    const int stash_row = a.rows - kFfnWidth;
+    float* stash = a.h + (long)stash_row * npos;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < kFfnWidth * kFgTailPos; e += kFgThreads) {
+        const int j = e / kFgTailPos, pp = e % kFgTailPos;
+        sA[j * AS + pp] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
+    }
+    for (int e = tid; e < kFfnWidth * kFfnWidth; e += kFgThreads) {
+        const int r = e / kFfnWidth, j = e % kFfnWidth;
+        sW[r * kFgOS + j] = j < a.width ? __ldg(a.Wout + (long)(stash_row + r) * a.width + j) : 0.0f;
+    }
+    __syncthreads();
+    // thread (ty, tx): rows ty + 16 i (i < 4), position tx
+    const int tx = tid % 16, ty = tid / 16;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 8
+    for (int j = 0; j < kFfnWidth; ++j) {
+        const float x = sA[j * AS + tx];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = fmaf(sW[(ty + 16 * i) * kFgOS + j], x, acc[i]);
+    }
+    const long pos = p0 + tx;
+    if (pos >= npos) return;
+    float dist;
+    if constexpr (!TWO_D) dist = (float)pos;
+    else dist = (float)(pos / a.Ww) + (float)(pos % a.Ww);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = stash_row + ty + 16 * i;
+        const float al = __ldg(a.alpha + r % a.D);
+        stash[(long)(ty + 16 * i) * npos + pos] = acc[i] * expf(-al * dist * a.inv_div);
     }
 }
 

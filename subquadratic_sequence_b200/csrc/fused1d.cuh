@@ -84,7 +84,10 @@ struct Fft1d {
     static constexpr int M = 1 << LOG2M;
     static constexpr int E = P::E;
     static constexpr int T = M / E;                    // threads per sequence
-    static constexpr int G = T >= 128 ? 1 : 128 / T;   // sequences per CTA
+    // sequences per CTA: up to 384 threads, one CTA per SM at 168 registers,
+    // so every warp of the SM runs the same pass at the same time and they
+    // share the instruction fetch (the unrolled passes are large)
+    static constexpr int G = T >= 128 ? (T == 128 ? 3 : 1) : 384 / T;
     static constexpr int THREADS = G * T;
     // exchange buffer, float2; even, so every buffer starts 16-byte aligned
     static constexpr int SMEM_SEQ = (padded_size(M) + 1) & ~1;
@@ -96,9 +99,9 @@ struct Fft1d {
     static constexpr int STAGE_SEQ = H_IN_EXCHANGE ? M / 2 : M;  // staging buffer, float2
     static constexpr size_t SMEM_BYTES = sizeof(float2) * G * (SMEM_SEQ + STAGE_SEQ);
     static constexpr size_t SMEM_BYTES_FFT = sizeof(float2) * G * SMEM_SEQ;
-    // resident CTAs per SM the register budget is sized for: three
-    // 128-thread CTAs (168 registers per thread), else one
-    static constexpr int MIN_BLOCKS = THREADS <= 128 ? 3 : 1;
+    // resident CTAs per SM the register budget is sized for: 168 registers
+    // per thread (384 threads per SM) where that allows a CTA at all
+    static constexpr int MIN_BLOCKS = THREADS * 168 <= 65536 ? 65536 / (THREADS * 168) : 1;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
     static_assert((SMEM_SEQ * sizeof(float2)) % 16 == 0 && (STAGE_SEQ * sizeof(float2)) % 16 == 0,
                   "cp.async targets must be 16-byte aligned");

@@ -14,11 +14,12 @@ hyena_status_t filter_gen_launches(const FilterGenArgs& a, long npos, cudaStream
                               kFgLayerSmemBytes, st, a);
     const int head_rows = a.rows - kFfnWidth;
     if (s == HYENA_OK)
-        s = launch(filter_head_kernel<TWO_D, false>,
+        s = launch(filter_head_kernel<TWO_D>,
                    dim3(ptiles, (unsigned)((head_rows + kFgRowTile - 1) / kFgRowTile)), kFgThreads,
                    kFgHeadSmemBytes, st, a);
     if (s == HYENA_OK)
-        s = launch(filter_head_kernel<TWO_D, true>, dim3(ptiles), kFgThreads, kFgHeadSmemBytes, st, a);
+        s = launch(filter_tail_kernel<TWO_D>, dim3((unsigned)((npos + kFgTailPos - 1) / kFgTailPos)),
+                   kFgThreads, kFgTailSmemBytes, st, a);
     return s;
 }
 
