@@ -10,18 +10,24 @@
 // decay window exp(-alpha_d i / div) (2-D: exp(-alpha_c (iy + ix) / div)
 // as the product of the two axis windows).
 //
-// Three launches, no recomputation:
-//  layers: all threads of a CTA evaluate the three sine layers for 16
-//          positions (16 threads per position, 4 output units each, weights
-//          broadcast from shared memory) and stash a3 [64][positions] in
-//          the LAST 64 rows of h (they are outputs too, written last);
+// Every stage is a small dense product evaluated as a register-tiled SIMT
+// GEMM out of shared memory (each thread owns a 4 x 4 or 8 x 4 block of
+// outputs: one 128-bit load of weights and one of activations per 16 or 32
+// multiply-adds).  Three launches, no recomputation:
+//  layers: a persistent kernel (weights staged once per CTA) evaluates the
+//          three sine layers for tiles of positions and stashes
+//          a3 [64][positions] in the LAST 64 rows of h (they are outputs
+//          too, written last);
 //  head:   h[r][p] = (sum_j Wout[r][j] a3[j][p]) * window for the rows
-//          before the stash, as 128-row x 64-position tiles out of shared
-//          memory, written coalesced along the position;
-//  tail:   the head for the 64 stash rows, 16 positions per CTA: each CTA
-//          loads its own tile of a3 into shared memory before overwriting it.
-// With fewer than 64 head rows the layers are evaluated inside the head
-// kernel instead (one launch).
+//          before the stash, as 128-row x 64-position tiles;
+//  tail:   the head for the 64 stash rows, 64 positions per CTA: each CTA
+//          loads its own tile of a3 into shared memory before overwriting
+//          exactly that tile.
+// With at most 64 rows the layers are evaluated inside the head kernel
+// instead (one launch).  The sine is the hardware approximation __sinf:
+// the arguments are sums of 17 to 66 products of N(0, 1/fan_in) weights
+// with values in [-1, 1], so they stay within a few units of zero, where
+// its absolute error is below 1e-6.
 #pragma once
 
 #include "hyena_common.cuh"
@@ -40,344 +46,428 @@ struct FilterGenArgs {
     int n_bands;
     float inv_div;                 // 1 / decay_div
     float* h;                      // [rows][positions]
+    int vec;                       // positions % 4 == 0 and h 16-byte aligned: 128-bit h access
 };
 
-constexpr int kFgTile = 64;        // positions per head CTA
-constexpr int kFgRowTile = 128;    // head rows per CTA
-constexpr int kFgThreads = 256;
-constexpr int kFgLayerPos = 16;    // positions per layers CTA (16 threads each)
-constexpr int kFgAS = kFgTile + 1; // activation row stride
-constexpr int kFgOS = kFfnWidth + 1;
-// weight row strides: odd, so the units the threads of one position read
-// at once sit on different banks
-constexpr int kFgW1S = kFfnMaxIn + 1;
-constexpr int kFgWS = kFfnWidth + 1;
-constexpr int kFgWRegion = kFfnWidth * kFgW1S + 2 * kFfnWidth * kFgWS;
-// layers kernel shared memory (floats): weights + two activation buffers
-constexpr size_t kFgLayerSmemBytes = sizeof(float) * (kFgWRegion + 2 * kFfnWidth * (kFgLayerPos + 1));
-// head kernel shared memory (floats): the Wout tile transposed [64][132]
-// and the a3 tile [64][68]; rows 16-byte aligned for 128-bit loads
-constexpr int kFgWTS = kFgRowTile + 4;
-constexpr int kFgA4S = kFgTile + 4;
-constexpr size_t kFgHeadSmemBytes = sizeof(float) * (kFfnWidth * kFgWTS + kFfnWidth * kFgA4S);
-// tail kernel: 16 positions x the 64 stash rows per CTA
-constexpr int kFgTailPos = 16;
-constexpr size_t kFgTailSmemBytes = sizeof(float) * (kFfnWidth * kFgOS + kFfnWidth * (kFgTailPos + 1));
-// single-launch path (few rows): weights + Wout tile + two activation tiles
-constexpr size_t kFgFusedSmemBytes = sizeof(float) * (kFgWRegion + 2 * kFfnWidth * kFgAS);
-static_assert(kFgRowTile * kFgOS <= kFgWRegion, "Wout tile fits the weight region");
+constexpr int kFgThreads = 256;     // a 16 x 16 thread grid
+constexpr int kFgTile = 64;         // positions per head / tail / layers tile
+constexpr int kFgRowTile = 128;     // head rows per CTA
+constexpr int kFgSmallTile = 16;    // positions per layers tile for short filters
+// shared-memory row strides (floats): multiples of 4, so every row starts
+// 16-byte aligned for 128-bit loads
+constexpr int kFgUS = kFfnWidth + 4;     // [input][unit] weight rows, [unit][pos] tiles of 64
+constexpr int kFgRS = kFgRowTile + 4;    // [unit][row] Wout tile of the head
+// transposed W1 (canonical feature slots), W2, W3: [input][unit]
+constexpr int kFgWRegion = (kFfnMaxIn + 2 * kFfnWidth) * kFgUS;
 
-// Positional features of position `pos` in the canonical slots (1-D:
-// [t, (sin, cos) band 1..16]; 2-D: [ty, tx, (sin, cos) y-band 1..16,
-// (sin, cos) x-band 1..16]).
-template <bool TWO_D>
-__device__ __forceinline__ void features(const FilterGenArgs& a, long pos, float* phi)
+template <int PT>
+struct LayerTile {
+    static constexpr int AS = PT + 4;                    // activation row stride
+    static constexpr int PPT = PT / 16;                  // positions per thread
+    // weights + features/a2 [66][AS] + a1/a3 [64][AS]
+    static constexpr size_t SMEM = sizeof(float) * (kFgWRegion + (kFfnMaxIn + kFfnWidth) * AS);
+};
+constexpr size_t kFgHeadSmemBytes = sizeof(float) * (kFfnWidth * kFgRS + kFfnWidth * kFgUS);
+constexpr size_t kFgTailSmemBytes = sizeof(float) * 2 * kFfnWidth * kFgUS;
+// single launch (rows <= 64): layers tile of 64 positions, then the head;
+// the Wout rows reuse the weight region
+constexpr size_t kFgFusedSmemBytes = LayerTile<kFgTile>::SMEM;
+static_assert(kFfnWidth * kFgUS <= kFgWRegion, "Wout rows fit the weight region");
+
+// Positional features of the tile's positions p0 .. p0+PT-1 into sX[slot][p]
+// (1-D slots: [t, (sin, cos) band 1..16]; 2-D: [ty, tx, (sin, cos) y-band
+// 1..16, (sin, cos) x-band 1..16]); bands above n_bands and positions past
+// the end are zero.
+template <bool TWO_D, int PT>
+__device__ __forceinline__ void features_tile(const FilterGenArgs& a, long npos, long p0, float* sX)
 {
-#pragma unroll
-    for (int c = 0; c < kFfnMaxIn; ++c) phi[c] = 0.0f;
+    constexpr int AS = LayerTile<PT>::AS;
+    const int tid = threadIdx.x;
     if constexpr (!TWO_D) {
-        const int i = (int)pos;
-        phi[0] = (float)i / (float)a.L;
-#pragma unroll
-        for (int k = 1; k <= 16; ++k) {
-            if (k > a.n_bands) break;
-            // angle 2 pi k i / L reduced exactly: 2 pi ((k i) mod L) / L
-            const int qk = (int)(((long)k * i) % a.L);
-            float sn, cs;
-            sincospif(2.0f * (float)qk / (float)a.L, &sn, &cs);
-            phi[2 * k - 1] = sn;
-            phi[2 * k] = cs;
+        for (int e = tid; e < 17 * PT; e += kFgThreads) {
+            const int k = e / PT, p = e % PT;
+            const long pos = p0 + p;
+            const int i = (int)pos;
+            if (k == 0) {
+                sX[p] = pos < npos ? (float)i / (float)a.L : 0.0f;
+            } else {
+                float sn = 0.0f, cs = 0.0f;
+                if (k <= a.n_bands && pos < npos) {
+                    // angle 2 pi k i / L reduced exactly: 2 pi ((k i) mod L) / L
+                    const int qk = (int)(((long)k * i) % a.L);
+                    sincospif(2.0f * (float)qk / (float)a.L, &sn, &cs);
+                }
+                sX[(2 * k - 1) * AS + p] = sn;
+                sX[(2 * k) * AS + p] = cs;
+            }
         }
     } else {
-        const int iy = (int)(pos / a.Ww), ix = (int)(pos % a.Ww);
-        phi[0] = (float)iy / (float)a.Hh;
-        phi[1] = (float)ix / (float)a.Ww;
-#pragma unroll
-        for (int k = 1; k <= 16; ++k) {
-            if (k > a.n_bands) break;
-            float sn, cs;
-            const int qy = (int)(((long)k * iy) % a.Hh);
-            sincospif(2.0f * (float)qy / (float)a.Hh, &sn, &cs);
-            phi[2 * k] = sn;
-            phi[2 * k + 1] = cs;
-            const int qx = (int)(((long)k * ix) % a.Ww);
-            sincospif(2.0f * (float)qx / (float)a.Ww, &sn, &cs);
-            phi[2 + 2 * 16 + 2 * (k - 1)] = sn;
-            phi[2 + 2 * 16 + 2 * (k - 1) + 1] = cs;
+        constexpr int XB = 2 + 2 * 16;                  // slot of the first x-band feature
+        for (int e = tid; e < 33 * PT; e += kFgThreads) {
+            const int k = e / PT, p = e % PT;
+            const long pos = p0 + p;
+            const int iy = (int)(pos / a.Ww), ix = (int)(pos % a.Ww);
+            if (k == 0) {
+                sX[p] = pos < npos ? (float)iy / (float)a.Hh : 0.0f;
+                sX[AS + p] = pos < npos ? (float)ix / (float)a.Ww : 0.0f;
+            } else {
+                const int band = (k - 1) % 16 + 1;
+                const bool xaxis = k > 16;
+                float sn = 0.0f, cs = 0.0f;
+                if (band <= a.n_bands && pos < npos) {
+                    const int n = xaxis ? a.Ww : a.Hh, c = xaxis ? ix : iy;
+                    const int qk = (int)(((long)band * c) % n);
+                    sincospif(2.0f * (float)qk / (float)n, &sn, &cs);
+                }
+                const int slot = xaxis ? XB + 2 * (band - 1) : 2 * band;
+                sX[slot * AS + p] = sn;
+                sX[(slot + 1) * AS + p] = cs;
+            }
         }
     }
 }
 
-// Stage W1 (canonical feature slots), W2, W3 into shared memory, zero
-// padded to 64 units (sin(0) = 0: padded units contribute nothing).
+// Stage W1 (canonical feature slots), W2, W3 transposed into shared memory
+// as [input][unit], zero padded to 64 units (sin(0) = 0: padded units
+// contribute nothing).  All loads of a matrix are issued before its stores.
 template <bool TWO_D>
-__device__ __forceinline__ void stage_weights(const FilterGenArgs& a, float* sW1, float* sW2, float* sW3)
+__device__ __forceinline__ void stage_weights(const FilterGenArgs& a, float* sW)
 {
+    constexpr int NIN = TWO_D ? kFfnMaxIn : 33;
     const int tid = threadIdx.x;
-    for (int e = tid; e < kFfnWidth * kFfnMaxIn; e += blockDim.x) {
-        const int r = e / kFfnMaxIn, c = e % kFfnMaxIn;
-        int src = -1;
-        if constexpr (!TWO_D) {
-            src = c < a.n_in ? c : -1;
-        } else {
-            constexpr int XB = 2 + 2 * 16;   // slot of the first x-band feature
-            if (c < 2 + 2 * a.n_bands) src = c;
-            else if (c >= XB && c < XB + 2 * a.n_bands) src = 2 + 2 * a.n_bands + (c - XB);
-        }
-        sW1[r * kFgW1S + c] = (r < a.width && src >= 0) ? __ldg(a.W1 + r * a.n_in + src) : 0.0f;
-    }
-    for (int e = tid; e < kFfnWidth * kFfnWidth; e += blockDim.x) {
-        const int r = e / kFfnWidth, c = e % kFfnWidth;
-        const bool in = r < a.width && c < a.width;
-        sW2[r * kFgWS + c] = in ? __ldg(a.W2 + r * a.width + c) : 0.0f;
-        sW3[r * kFgWS + c] = in ? __ldg(a.W3 + r * a.width + c) : 0.0f;
-    }
-}
-
-// The three sine layers for position p of a tile: UPT = 64 / TPP output
-// units per thread, TPP threads per position (thread q of the position owns
-// units TPP * jj + q).  a1 and a3 end up in sA[j * AS + p], a2 in sB.
-template <bool TWO_D, int TPP, int AS>
-__device__ __forceinline__ void sine_layers(const FilterGenArgs& a, long pos, int p, int q,
-                                            const float* sW1, const float* sW2, const float* sW3,
-                                            float* sA, float* sB)
-{
-    constexpr int UPT = kFfnWidth / TPP;
-    constexpr int NIN = TWO_D ? kFfnMaxIn : 33;        // 1-D features use slots < 33
+    float* sW1 = sW;
+    float* sW2 = sW + kFfnMaxIn * kFgUS;
+    float* sW3 = sW2 + kFfnWidth * kFgUS;
     {
-        float phi[kFfnMaxIn];
-        features<TWO_D>(a, pos, phi);
-        __syncthreads();                                   // weights staged by all threads
-        float acc[UPT];
+        constexpr int PER = (kFfnWidth * NIN + kFgThreads - 1) / kFgThreads;
+        float v[PER];
 #pragma unroll
-        for (int jj = 0; jj < UPT; ++jj) acc[jj] = 0.0f;
-#pragma unroll
-        for (int c = 0; c < NIN; ++c)
-#pragma unroll
-            for (int jj = 0; jj < UPT; ++jj)
-                acc[jj] = fmaf(sW1[(TPP * jj + q) * kFgW1S + c], phi[c], acc[jj]);
-#pragma unroll
-        for (int jj = 0; jj < UPT; ++jj) sA[(TPP * jj + q) * AS + p] = sinf(acc[jj]);
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int layer = 0; layer < 2; ++layer) {
-        const float* Wl = layer == 0 ? sW2 : sW3;
-        const float* in = layer == 0 ? sA : sB;
-        float* out = layer == 0 ? sB : sA;
-        float acc[UPT];
-#pragma unroll
-        for (int jj = 0; jj < UPT; ++jj) acc[jj] = 0.0f;
-#pragma unroll 8
-        for (int c = 0; c < kFfnWidth; ++c) {
-            const float x = in[c * AS + p];
-#pragma unroll
-            for (int jj = 0; jj < UPT; ++jj) acc[jj] = fmaf(Wl[(TPP * jj + q) * kFgWS + c], x, acc[jj]);
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads;
+            const int u = e / NIN, c = e % NIN;
+            int src = -1;
+            if constexpr (!TWO_D) {
+                src = c < a.n_in ? c : -1;
+            } else {
+                constexpr int XB = 2 + 2 * 16;
+                if (c < 2 + 2 * a.n_bands) src = c;
+                else if (c >= XB && c < XB + 2 * a.n_bands) src = 2 + 2 * a.n_bands + (c - XB);
+            }
+            v[i] = (e < kFfnWidth * NIN && u < a.width && src >= 0) ? __ldg(a.W1 + u * a.n_in + src) : 0.0f;
         }
 #pragma unroll
-        for (int jj = 0; jj < UPT; ++jj) out[(TPP * jj + q) * AS + p] = sinf(acc[jj]);
-        __syncthreads();
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads;
+            if (e < kFfnWidth * NIN) sW1[(e % NIN) * kFgUS + e / NIN] = v[i];
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        const float* W = m == 0 ? a.W2 : a.W3;
+        float* dst = m == 0 ? sW2 : sW3;
+        constexpr int PER = kFfnWidth * kFfnWidth / kFgThreads;
+        float v[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads;
+            const int u = e / kFfnWidth, c = e % kFfnWidth;
+            v[i] = (u < a.width && c < a.width) ? __ldg(W + u * a.width + c) : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads;
+            dst[(e % kFfnWidth) * kFgUS + e / kFfnWidth] = v[i];
+        }
     }
 }
 
-// Head for rows r0 .. r0+127 (< r_end) and positions p0 .. p0+63 from the
-// a3 tile in sA [64][kFgAS] and the Wout tile staged into sOut.
+// out[u][p] = sin(sum_c W[u][c] in[c][p]) for 64 units and the PT positions
+// of a tile; thread (ty, tx) owns units 4 ty .. 4 ty + 3 and positions
+// PPT tx .. PPT tx + PPT - 1.  WT is [input][unit] (stride kFgUS).
+template <int PT, int K>
+__device__ __forceinline__ void sine_layer(const float* WT, const float* in, float* out)
+{
+    constexpr int AS = LayerTile<PT>::AS, PPT = LayerTile<PT>::PPT;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[4][PPT];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int k = 0; k < PPT; ++k) acc[i][k] = 0.0f;
+#pragma unroll 11
+    for (int c = 0; c < K; ++c) {
+        const float4 w = *reinterpret_cast<const float4*>(WT + c * kFgUS + 4 * ty);
+        float x[PPT];
+        if constexpr (PPT == 4) {
+            const float4 x4 = *reinterpret_cast<const float4*>(in + c * AS + 4 * tx);
+            x[0] = x4.x; x[1] = x4.y; x[2] = x4.z; x[3] = x4.w;
+        } else {
+            x[0] = in[c * AS + tx];
+        }
+        const float wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < PPT; ++k) acc[i][k] = fmaf(wv[i], x[k], acc[i][k]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if constexpr (PPT == 4) {
+            *reinterpret_cast<float4*>(out + (4 * ty + i) * AS + 4 * tx) =
+                make_float4(__sinf(acc[i][0]), __sinf(acc[i][1]), __sinf(acc[i][2]), __sinf(acc[i][3]));
+        } else {
+            out[(4 * ty + i) * AS + tx] = __sinf(acc[i][0]);
+        }
+    }
+}
+
+// The three sine layers of one tile: features into sX, a1 into sY, a2 into
+// sX, a3 into sY.  Ends with a barrier (a3 visible to the whole CTA).
+template <bool TWO_D, int PT>
+__device__ __forceinline__ void layers_tile(const FilterGenArgs& a, long npos, long p0, const float* sW,
+                                            float* sX, float* sY)
+{
+    constexpr int NIN = TWO_D ? kFfnMaxIn : 33;
+    features_tile<TWO_D, PT>(a, npos, p0, sX);
+    __syncthreads();
+    sine_layer<PT, NIN>(sW, sX, sY);
+    __syncthreads();
+    sine_layer<PT, kFfnWidth>(sW + kFfnMaxIn * kFgUS, sY, sX);
+    __syncthreads();
+    sine_layer<PT, kFfnWidth>(sW + (kFfnMaxIn + kFfnWidth) * kFgUS, sX, sY);
+    __syncthreads();
+}
+
+// The decay window of row r (alpha index r % D) at position pos: the
+// argument is i (1-D) or iy + ix (2-D).
 template <bool TWO_D>
-__device__ __forceinline__ void head_tile(const FilterGenArgs& a, long npos, long p0, int r0, int r_end,
-                                          float* sOut, const float* sA)
+__device__ __forceinline__ float window(const FilterGenArgs& a, float al, long pos)
+{
+    float dist;
+    if constexpr (!TWO_D) dist = (float)pos;
+    else dist = (float)(pos / a.Ww) + (float)(pos % a.Ww);
+    return expf(-al * dist * a.inv_div);
+}
+
+// Load a [64][64] tile of a3 (positions p0 .. p0+63 of the stash rows) into
+// sA [64][kFgUS]; positions past the end read as zero.
+__device__ __forceinline__ void load_a3_tile(const FilterGenArgs& a, long npos, long p0, const float* stash,
+                                             float* sA)
 {
     const int tid = threadIdx.x;
-    for (int e = tid; e < kFgRowTile * kFfnWidth; e += kFgThreads) {
-        const int r = e / kFfnWidth, j = e % kFfnWidth;
-        sOut[r * kFgOS + j] = (r0 + r < r_end && j < a.width)
-                                  ? __ldg(a.Wout + (long)(r0 + r) * a.width + j) : 0.0f;
-    }
-    __syncthreads();
-    // thread (ty, tx) of a 16 x 16 grid: rows ty + 16 i (i < 8), positions tx + 16 k (k < 4)
-    const int tx = tid % 16, ty = tid / 16;
-    float acc[8][4];
+    if (a.vec) {
+        float4 v[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + i * kFgThreads, j = e / 16, q = e % 16;
+            const long pos = p0 + 4 * q;
+            v[i] = pos < npos ? *reinterpret_cast<const float4*>(stash + (long)j * npos + pos)
+                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + i * kFgThreads, j = e / 16, q = e % 16;
+            *reinterpret_cast<float4*>(sA + j * kFgUS + 4 * q) = v[i];
+        }
+    } else {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int e = tid + i * kFgThreads, j = e / 64, pp = e % 64;
+            v[i] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int e = tid + i * kFgThreads;
+            sA[(e / 64) * kFgUS + e % 64] = v[i];
+        }
+    }
+}
+
+// Stage rows r0 .. r0 + NR - 1 (< r_end) of Wout transposed into
+// sWT [64][RS] (zero past r_end and past the width).
+template <int NR, int RS>
+__device__ __forceinline__ void load_wout_tile(const FilterGenArgs& a, int r0, int r_end, float* sWT)
+{
+    constexpr int PER = NR * kFfnWidth / kFgThreads;
+    const int tid = threadIdx.x;
+    float v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = tid + i * kFgThreads, r = e / kFfnWidth, j = e % kFfnWidth;
+        v[i] = (r0 + r < r_end && j < a.width) ? __ldg(a.Wout + (long)(r0 + r) * a.width + j) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = tid + i * kFgThreads;
+        sWT[(e % kFfnWidth) * RS + e / kFfnWidth] = v[i];
+    }
+}
+
+// h[r][p] = (sum_j Wout[r][j] a3[j][p]) * window for rows r0 + RT ty + i
+// (i < RT, r < r_end) and positions p0 + 4 tx + k (k < 4) from sWT
+// [64][RS] and sA [64][kFgUS]; alpha of the thread's rows is passed in.
+template <bool TWO_D, int RT, int RS>
+__device__ __forceinline__ void head_block(const FilterGenArgs& a, long npos, long p0, int r0, int r_end,
+                                           const float* sWT, const float* sA, const float* al)
+{
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[RT][4];
+#pragma unroll
+    for (int i = 0; i < RT; ++i)
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[i][k] = 0.0f;
-#pragma unroll 4
+#pragma unroll 8
     for (int j = 0; j < kFfnWidth; ++j) {
-        float w[8], x[4];
+        const float4 x4 = *reinterpret_cast<const float4*>(sA + j * kFgUS + 4 * tx);
+        float w[RT];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = sOut[(ty + 16 * i) * kFgOS + j];
+        for (int i = 0; i < RT; i += 4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(sWT + j * RS + RT * ty + i);
+            w[i] = w4.x; w[i + 1] = w4.y; w[i + 2] = w4.z; w[i + 3] = w4.w;
+        }
+        const float x[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) x[k] = sA[j * kFgAS + tx + 16 * k];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < RT; ++i)
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[i][k] = fmaf(w[i], x[k], acc[i][k]);
     }
+    const long pos0 = p0 + 4 * tx;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int r = r0 + ty + 16 * i;
+    for (int i = 0; i < RT; ++i) {
+        const int r = r0 + RT * ty + i;
         if (r >= r_end) continue;
-        const float al = __ldg(a.alpha + r % a.D);
+        float* hr = a.h + (long)r * npos;
+        if (a.vec) {
+            if (pos0 < npos)
+                *reinterpret_cast<float4*>(hr + pos0) =
+                    make_float4(acc[i][0] * window<TWO_D>(a, al[i], pos0),
+                                acc[i][1] * window<TWO_D>(a, al[i], pos0 + 1),
+                                acc[i][2] * window<TWO_D>(a, al[i], pos0 + 2),
+                                acc[i][3] * window<TWO_D>(a, al[i], pos0 + 3));
+        } else {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const long pos = p0 + tx + 16 * k;
-            if (pos >= npos) continue;
-            float dist;   // the window's argument: i (1-D) or iy + ix (2-D)
-            if constexpr (!TWO_D) dist = (float)pos;
-            else dist = (float)(pos / a.Ww) + (float)(pos % a.Ww);
-            a.h[(long)r * npos + pos] = acc[i][k] * expf(-al * dist * a.inv_div);
+            for (int k = 0; k < 4; ++k)
+                if (pos0 + k < npos) hr[pos0 + k] = acc[i][k] * window<TWO_D>(a, al[i], pos0 + k);
         }
     }
 }
 
-// Layers kernel: a3 of 16 positions into the stash rows (the last 64 rows
-// of h), a3[j][pos] at h[(rows - 64 + j) * npos + pos].
-template <bool TWO_D>
+// alpha of rows r0 + RT ty + i (loaded before the products so the loads
+// overlap them)
+template <int RT>
+__device__ __forceinline__ void load_alpha(const FilterGenArgs& a, int r0, int r_end, float* al)
+{
+    const int ty = threadIdx.x / 16;
+#pragma unroll
+    for (int i = 0; i < RT; ++i) {
+        const int r = r0 + RT * ty + i;
+        al[i] = r < r_end ? __ldg(a.alpha + r % a.D) : 0.0f;
+    }
+}
+
+// Layers kernel (persistent over position tiles of PT): a3 into the stash
+// rows (the last 64 rows of h), a3[j][pos] at h[(rows - 64 + j) * npos + pos].
+template <bool TWO_D, int PT>
 __global__ void __launch_bounds__(kFgThreads) filter_layers_kernel(FilterGenArgs a)
 {
+    using LT = LayerTile<PT>;
+    constexpr int AS = LT::AS, PPT = LT::PPT;
     extern __shared__ __align__(16) float fg_smem[];
-    constexpr int AS = kFgLayerPos + 1;
-    float* sW1 = fg_smem;
-    float* sW2 = sW1 + kFfnWidth * kFgW1S;
-    float* sW3 = sW2 + kFfnWidth * kFgWS;
-    float* sA = fg_smem + kFgWRegion;
-    float* sB = sA + kFfnWidth * AS;
+    float* sW = fg_smem;
+    float* sX = fg_smem + kFgWRegion;
+    float* sY = sX + kFfnMaxIn * AS;
     const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
-    const long p0 = (long)blockIdx.x * kFgLayerPos;
-    const int p = threadIdx.x / 16, q = threadIdx.x % 16;
-    stage_weights<TWO_D>(a, sW1, sW2, sW3);
-    sine_layers<TWO_D, 16, AS>(a, min(p0 + p, npos - 1), p, q, sW1, sW2, sW3, sA, sB);
-    // stash a3 (coalesced along the position)
+    const long ntiles = (npos + PT - 1) / PT;
     float* stash = a.h + (long)(a.rows - kFfnWidth) * npos;
-    for (int e = threadIdx.x; e < kFfnWidth * kFgLayerPos; e += kFgThreads) {
-        const int j = e / kFgLayerPos, pp = e % kFgLayerPos;
-        if (p0 + pp < npos) stash[(long)j * npos + p0 + pp] = sA[j * AS + pp];
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    stage_weights<TWO_D>(a, sW);
+    for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const long p0 = tile * PT;
+        layers_tile<TWO_D, PT>(a, npos, p0, sW, sX, sY);   // ends with a barrier
+        // stash a3: thread (ty, tx) stores its own 4 units x PPT positions
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int u = 4 * ty + i;
+            const long pos = p0 + PPT * tx;
+            float* dst = stash + (long)u * npos;
+            if constexpr (PPT == 4) {
+                if (a.vec) {
+                    if (pos < npos)
+                        *reinterpret_cast<float4*>(dst + pos) = *reinterpret_cast<const float4*>(sY + u * AS + 4 * tx);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (pos + k < npos) dst[pos + k] = sY[u * AS + 4 * tx + k];
+                }
+            } else {
+                if (pos < npos) dst[pos] = sY[u * AS + tx];
+            }
+        }
+        __syncthreads();                                     // sX / sY reused by the next tile
     }
 }
 
 // Head kernel: rows 0 .. rows-65 as 128-row x 64-position tiles (grid.y
-// over row tiles).  Thread (ty, tx) computes rows 8 ty + i (i < 8) and
-// positions 4 tx + k (k < 4): per unit j one 128-bit load of 4 a3 values and
-// two of 8 Wout values for 32 multiply-adds.
+// over row tiles), thread (ty, tx) owning rows 8 ty + i (i < 8) and
+// positions 4 tx + k (k < 4).
 template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_head_kernel(FilterGenArgs a)
 {
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][132]: Wout tile, transposed
-    float* sA = fg_smem + kFfnWidth * kFgWTS;               // [64][68]:  a3 tile
+    float* sA = fg_smem + kFfnWidth * kFgRS;                // [64][68]:  a3 tile
     const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
     const long p0 = (long)blockIdx.x * kFgTile;
     const int r0 = blockIdx.y * kFgRowTile;
     const int stash_row = a.rows - kFfnWidth;
-    const float* stash = a.h + (long)stash_row * npos;
-    const int tid = threadIdx.x;
-    for (int e = tid; e < kFfnWidth * kFgTile; e += kFgThreads) {
-        const int j = e / kFgTile, pp = e % kFgTile;
-        sA[j * kFgA4S + pp] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
-    }
-    for (int e = tid; e < kFgRowTile * kFfnWidth; e += kFgThreads) {
-        const int r = e / kFfnWidth, j = e % kFfnWidth;
-        sWT[j * kFgWTS + r] = (r0 + r < stash_row && j < a.width)
-                                  ? __ldg(a.Wout + (long)(r0 + r) * a.width + j) : 0.0f;
-    }
+    float al[8];
+    load_alpha<8>(a, r0, stash_row, al);
+    load_a3_tile(a, npos, p0, a.h + (long)stash_row * npos, sA);
+    load_wout_tile<kFgRowTile, kFgRS>(a, r0, stash_row, sWT);
     __syncthreads();
-    const int tx = tid % 16, ty = tid / 16;
-    float acc[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[i][k] = 0.0f;
-#pragma unroll 4
-    for (int j = 0; j < kFfnWidth; ++j) {
-        const float4 x4 = *reinterpret_cast<const float4*>(sA + j * kFgA4S + 4 * tx);
-        const float4 w0 = *reinterpret_cast<const float4*>(sWT + j * kFgWTS + 8 * ty);
-        const float4 w1 = *reinterpret_cast<const float4*>(sWT + j * kFgWTS + 8 * ty + 4);
-        const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        const float x[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[i][k] = fmaf(w[i], x[k], acc[i][k]);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int r = r0 + 8 * ty + i;
-        if (r >= stash_row) continue;
-        const float al = __ldg(a.alpha + r % a.D);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const long pos = p0 + 4 * tx + k;
-            if (pos >= npos) continue;
-            float dist;   // the window's argument: i (1-D) or iy + ix (2-D)
-            if constexpr (!TWO_D) dist = (float)pos;
-            else dist = (float)(pos / a.Ww) + (float)(pos % a.Ww);
-            a.h[(long)r * npos + pos] = acc[i][k] * expf(-al * dist * a.inv_div);
-        }
-    }
+    head_block<TWO_D, 8, kFgRS>(a, npos, p0, r0, stash_row, sWT, sA, al);
 }
 
-// Tail kernel: the 64 stash rows for 16 positions per CTA; each CTA reads
-// its own 64 x 16 tile of a3 before overwriting exactly that tile.
+// Tail kernel: the 64 stash rows for 64 positions per CTA; each CTA reads
+// its own 64 x 64 tile of a3 before overwriting exactly that tile.
 template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_tail_kernel(FilterGenArgs a)
 {
     extern __shared__ __align__(16) float fg_smem[];
-    constexpr int AS = kFgTailPos + 1;
-    float* sW = fg_smem;                                    // [64][65]: Wout stash rows
-    float* sA = fg_smem + kFfnWidth * kFgOS;                // [64][17]: a3 tile
+    float* sWT = fg_smem;                                   // [64][68]: Wout stash rows, transposed
+    float* sA = fg_smem + kFfnWidth * kFgUS;                // [64][68]: a3 tile
     const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
-    const long p0 = (long)blockIdx.x * kFgTailPos;
+    const long p0 = (long)blockIdx.x * kFgTile;
     const int stash_row = a.rows - kFfnWidth;
-    float* stash = a.h + (long)stash_row * npos;
-    const int tid = threadIdx.x;
-    for (int e = tid; e < kFfnWidth * kFgTailPos; e += kFgThreads) {
-        const int j = e / kFgTailPos, pp = e % kFgTailPos;
-        sA[j * AS + pp] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
-    }
-    for (int e = tid; e < kFfnWidth * kFfnWidth; e += kFgThreads) {
-        const int r = e / kFfnWidth, j = e % kFfnWidth;
-        sW[r * kFgOS + j] = j < a.width ? __ldg(a.Wout + (long)(stash_row + r) * a.width + j) : 0.0f;
-    }
+    float al[4];
+    load_alpha<4>(a, stash_row, a.rows, al);
+    load_a3_tile(a, npos, p0, a.h + (long)stash_row * npos, sA);
+    load_wout_tile<kFfnWidth, kFgUS>(a, stash_row, a.rows, sWT);
     __syncthreads();
-    // thread (ty, tx): rows ty + 16 i (i < 4), position tx
-    const int tx = tid % 16, ty = tid / 16;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 8
-    for (int j = 0; j < kFfnWidth; ++j) {
-        const float x = sA[j * AS + tx];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] = fmaf(sW[(ty + 16 * i) * kFgOS + j], x, acc[i]);
-    }
-    const long pos = p0 + tx;
-    if (pos >= npos) return;
-    float dist;
-    if constexpr (!TWO_D) dist = (float)pos;
-    else dist = (float)(pos / a.Ww) + (float)(pos % a.Ww);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = stash_row + ty + 16 * i;
-        const float al = __ldg(a.alpha + r % a.D);
-        stash[(long)(ty + 16 * i) * npos + pos] = acc[i] * expf(-al * dist * a.inv_div);
-    }
+    head_block<TWO_D, 4, kFgUS>(a, npos, p0, stash_row, a.rows, sWT, sA, al);
 }
 
-// Single launch for few rows (< 64 + 1): every CTA evaluates the layers of
-// its 64 positions, then the head for all rows.
+// Single launch for at most 64 rows: every CTA evaluates the layers of its
+// 64 positions, then the head for all rows from shared memory.
 template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
 {
+    using LT = LayerTile<kFgTile>;
     extern __shared__ __align__(16) float fg_smem[];
-    float* sW1 = fg_smem;
-    float* sW2 = sW1 + kFfnWidth * kFgW1S;
-    float* sW3 = sW2 + kFfnWidth * kFgWS;
-    float* sOut = fg_smem;                                   // after the layers
-    float* sA = fg_smem + kFgWRegion;
-    float* sB = sA + kFfnWidth * kFgAS;
+    float* sW = fg_smem;
+    float* sX = fg_smem + kFgWRegion;
+    float* sY = sX + kFfnMaxIn * LT::AS;
     const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
     const long p0 = (long)blockIdx.x * kFgTile;
-    const int p = threadIdx.x / 4, q = threadIdx.x % 4;
-    stage_weights<TWO_D>(a, sW1, sW2, sW3);
-    sine_layers<TWO_D, 4, kFgAS>(a, min(p0 + p, npos - 1), p, q, sW1, sW2, sW3, sA, sB);
-    head_tile<TWO_D>(a, npos, p0, 0, a.rows, sOut, sA);
+    float al[4];
+    load_alpha<4>(a, 0, a.rows, al);
+    stage_weights<TWO_D>(a, sW);
+    layers_tile<TWO_D, kFgTile>(a, npos, p0, sW, sX, sY);  // ends with a barrier
+    load_wout_tile<kFfnWidth, kFgUS>(a, 0, a.rows, sW);   // the weights are no longer read
+    __syncthreads();
+    static_assert(LT::AS == kFgUS, "a3 tile stride");
+    head_block<TWO_D, 4, kFgUS>(a, npos, p0, 0, a.rows, sW, sY, al);
 }
 
 }  // namespace hyena

@@ -130,9 +130,11 @@ struct Fft1d {
                 constexpr int h = decltype(hh)::value;
                 float2* ar = a + (2 * c + h) * R;
                 dft<R, SIGN, ZERO_HI>(ar);
+                const int pj = pad16(j[h] * R);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    sm[pad16(j[h] * R + r)] = ar[r];
+                    // j R + r with R a multiple of 16: pad16(j R) + r + r / 16
+                    sm[R % 16 == 0 ? pj + r + r / 16 : pad16(j[h] * R + r)] = ar[r];
                 });
             });
         });
@@ -150,9 +152,10 @@ struct Fft1d {
             static_for<C>([&](auto cc) {
                 constexpr int c = decltype(cc)::value;
                 const int j = t + c * T;
+                const int pj = pad16(j);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    a[c * R + r] = sm[pad16(j + r * (M / R))];
+                    a[c * R + r] = sm[pad16_at<M / R>(j, pj, r)];
                 });
             });
             __syncthreads();
@@ -165,9 +168,10 @@ struct Fft1d {
                 apply_twiddle_powers<R>(ar, expi_pi<SIGN>(2.0f * (float)jm / (float)(NS * R) + dep));
                 dft<R, SIGN>(ar);
                 const int base = (j / NS) * NS * R + jm;
+                const int pb = pad16(base);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    sm[pad16(base + r * NS)] = ar[r];
+                    sm[pad16_at<NS>(base, pb, r)] = ar[r];
                 });
                 dep = zero_after(ar[R - 1].x);
             });
@@ -185,9 +189,10 @@ struct Fft1d {
             unit_cols<R>(t + c * T, j[0], j[1]);
             static_for<2>([&](auto hh) {
                 constexpr int h = decltype(hh)::value;
+                const int pj = pad16(j[h]);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    a[(2 * c + h) * R + r] = sm[pad16(j[h] + r * (M / R))];
+                    a[(2 * c + h) * R + r] = sm[pad16_at<M / R>(j[h], pj, r)];
                 });
             });
         });

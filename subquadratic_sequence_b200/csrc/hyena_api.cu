@@ -82,6 +82,7 @@ hyena_status_t filter_gen(const hyena_ffn_t* f, int rows, int D, long npos, int 
     a.n_bands = f->n_bands;
     a.inv_div = 1.0f / f->decay_div;
     a.h = h;
+    a.vec = (npos % 4 == 0 && aligned(h, 16)) ? 1 : 0;
     return launch_filter_gen(a, two_d, npos, st);
 }
 

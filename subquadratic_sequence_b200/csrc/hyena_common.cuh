@@ -256,4 +256,14 @@ __device__ __forceinline__ void cp_async_row(void* smem_dst, const void* gmem_sr
 __device__ __forceinline__ int pad16(int i) { return i + (i >> 4); }
 __host__ __device__ constexpr int padded_size(int n) { return n + n / 16; }
 
+// pad16(i + r * S) given pi = pad16(i), for a compile-time stride S: when S
+// is a multiple of 16 the padding of the offset is a constant, so the whole
+// index is pi plus an immediate.
+template <int S>
+__device__ __forceinline__ int pad16_at(int i, int pi, int r)
+{
+    if constexpr (S % 16 == 0) return pi + r * (S + S / 16);
+    else return pad16(i + r * S);
+}
+
 }  // namespace hyena

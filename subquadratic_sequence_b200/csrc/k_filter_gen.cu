@@ -3,23 +3,40 @@
 
 namespace hyena {
 
+namespace {
+
+// The layers kernel is persistent: at most `per_sm` CTAs per SM, each
+// staging the weights once and walking position tiles.
+template <bool TWO_D, int PT>
+hyena_status_t launch_layers(const FilterGenArgs& a, long npos, int sms, int per_sm, cudaStream_t st)
+{
+    const long tiles = (npos + PT - 1) / PT;
+    const long cap = (long)sms * per_sm;
+    return launch(filter_layers_kernel<TWO_D, PT>, dim3((unsigned)(tiles < cap ? tiles : cap)), kFgThreads,
+                  LayerTile<PT>::SMEM, st, a);
+}
+
+}  // namespace
+
 template <bool TWO_D>
 hyena_status_t filter_gen_launches(const FilterGenArgs& a, long npos, cudaStream_t st)
 {
     const unsigned ptiles = (unsigned)((npos + kFgTile - 1) / kFgTile);
-    if (a.rows < kFfnWidth + 1)
+    if (a.rows <= kFfnWidth)
         return launch(filter_gen_kernel<TWO_D>, dim3(ptiles), kFgThreads, kFgFusedSmemBytes, st, a);
-    hyena_status_t s = launch(filter_layers_kernel<TWO_D>,
-                              dim3((unsigned)((npos + kFgLayerPos - 1) / kFgLayerPos)), kFgThreads,
-                              kFgLayerSmemBytes, st, a);
+    int sms = 0;
+    hyena_status_t s = sm_count(&sms);
+    if (s != HYENA_OK) return s;
+    // short filters: 16-position tiles, so that every SM gets work
+    s = (long)ptiles >= 2L * sms ? launch_layers<TWO_D, kFgTile>(a, npos, sms, 2, st)
+                                 : launch_layers<TWO_D, kFgSmallTile>(a, npos, sms, 3, st);
     const int head_rows = a.rows - kFfnWidth;
-    if (s == HYENA_OK)
+    if (s == HYENA_OK && head_rows > 0)
         s = launch(filter_head_kernel<TWO_D>,
                    dim3(ptiles, (unsigned)((head_rows + kFgRowTile - 1) / kFgRowTile)), kFgThreads,
                    kFgHeadSmemBytes, st, a);
     if (s == HYENA_OK)
-        s = launch(filter_tail_kernel<TWO_D>, dim3((unsigned)((npos + kFgTailPos - 1) / kFgTailPos)),
-                   kFgThreads, kFgTailSmemBytes, st, a);
+        s = launch(filter_tail_kernel<TWO_D>, dim3(ptiles), kFgThreads, kFgTailSmemBytes, st, a);
     return s;
 }
 

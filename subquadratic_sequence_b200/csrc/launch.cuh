@@ -39,6 +39,16 @@ hyena_status_t launch(K kernel, dim3 grid, int threads, size_t smem, cudaStream_
     return from_cuda(cudaGetLastError());
 }
 
+// Number of SMs of the current device.
+inline hyena_status_t sm_count(int* n)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess && *n < 1) *n = 1;
+    return from_cuda(e);
+}
+
 // sequences per wave of the four-step path (scratch = wave * L complex)
 inline long wave_seqs(long nseq, long L)
 {
