@@ -185,10 +185,17 @@ template <int LOG2H2>
 struct Fft2dCols {
     using FC = SmemFft<LOG2H2>;
     static constexpr int H2 = 1 << LOG2H2;             // 2H
-    static constexpr int TC = (512 / FC::T) > 16 ? 16 : ((512 / FC::T) < 4 ? 4 : 512 / FC::T);
+    // TC columns per CTA (column index fastest across threads: every global
+    // access is a TC-element run); about 256 threads
+    static constexpr int TC = (256 / FC::T) > 16 ? 16 : ((256 / FC::T) < 4 ? 4 : 256 / FC::T);
     static constexpr int THREADS = TC * FC::T;
     static constexpr int STRIDE = stride_mod16(H2, 16 / TC);
     static constexpr size_t SMEM = sizeof(float2) * TC * STRIDE;
+    // resident CTAs per SM: up to three, as shared memory allows and with at
+    // least 80 registers per thread
+    static constexpr int BY_SMEM = 3 * SMEM <= 227 * 1024 ? 3 : (2 * SMEM <= 227 * 1024 ? 2 : 1);
+    static constexpr int BY_REGS = 65536 / (THREADS * 80) < 1 ? 1 : 65536 / (THREADS * 80);
+    static constexpr int MIN_BLOCKS = BY_SMEM < BY_REGS ? BY_SMEM : BY_REGS;
     static_assert(THREADS <= 1024 && SMEM <= 227 * 1024, "column kernel geometry");
 };
 
@@ -197,7 +204,7 @@ struct Fft2dCols {
 // FFTs, rows y < H back to the scratch.  SPECTRUM = true: forward column
 // FFTs of rows y < H of the packed spectra, all 2H rows written back.
 template <int LOG2H2, bool SPECTRUM>
-__global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS)
+__global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS, Fft2dCols<LOG2H2>::MIN_BLOCKS)
 fft2d_col_kernel(Fft2dArgs a)
 {
     using CL = Fft2dCols<LOG2H2>;
@@ -217,11 +224,12 @@ fft2d_col_kernel(Fft2dArgs a)
     // rows of this image's column kx: scratch [H][W] or spectra [2H][W]
     float2* col = SPECTRUM ? a.S + (size_t)q * H2 * W + kx : a.S + (size_t)qi * HH * W + kx;
     float2 reg[16];
+    const int pt = pad16(t);
 
     static_for<16>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
         const int y = t + r * (H2 / 16);
-        buf[pad16(y)] = r < 8 ? col[(size_t)y * W] : make_float2(0.0f, 0.0f);
+        buf[pad16_at<H2 / 16>(t, pt, r)] = r < 8 ? col[(size_t)y * W] : make_float2(0.0f, 0.0f);
     });
     __syncthreads();
     FC::template run<-1, true>(buf, reg, t);
@@ -234,7 +242,7 @@ fft2d_col_kernel(Fft2dArgs a)
     } else {
         static_for<16>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            buf[pad16(t + r * (H2 / 16))] = reg[r];
+            buf[pad16_at<H2 / 16>(t, pt, r)] = reg[r];
         });
         __syncthreads();
         // spectral multiply by (H + b) / (2H)
@@ -247,7 +255,8 @@ fft2d_col_kernel(Fft2dArgs a)
                 constexpr int r = decltype(rr)::value;
                 const int ky = t + r * (H2 / 16);
                 const float2 hv = __ldg(Hc + (size_t)ky * W);
-                buf[pad16(ky)] = cmul(buf[pad16(ky)], make_float2((hv.x + bias) * s, hv.y * s));
+                const int pk = pad16_at<H2 / 16>(t, pt, r);
+                buf[pk] = cmul(buf[pk], make_float2((hv.x + bias) * s, hv.y * s));
             });
         } else {
             // slot 0 = (bin-0 column) + i (bin-W column): separate both

@@ -67,8 +67,10 @@ struct LayerTile {
     // weights + features/a2 [66][AS] + a1/a3 [64][AS]
     static constexpr size_t SMEM = sizeof(float) * (kFgWRegion + (kFfnMaxIn + kFfnWidth) * AS);
 };
-constexpr size_t kFgHeadSmemBytes = sizeof(float) * (kFfnWidth * kFgRS + kFfnWidth * kFgUS);
+template <int NG>
+constexpr size_t fg_head_smem_bytes() { return sizeof(float) * (kFfnWidth * kFgRS + kFfnWidth * (64 * NG + 4)); }
 constexpr size_t kFgTailSmemBytes = sizeof(float) * 2 * kFfnWidth * kFgUS;
+constexpr size_t kFgTail16SmemBytes = sizeof(float) * kFfnWidth * (kFgUS + kFgSmallTile + 4);
 // single launch (rows <= 64): layers tile of 64 positions, then the head;
 // the Wout rows reuse the weight region
 constexpr size_t kFgFusedSmemBytes = LayerTile<kFgTile>::SMEM;
@@ -106,7 +108,7 @@ __device__ __forceinline__ void features_tile(const FilterGenArgs& a, long npos,
         for (int e = tid; e < 33 * PT; e += kFgThreads) {
             const int k = e / PT, p = e % PT;
             const long pos = p0 + p;
-            const int iy = (int)(pos / a.Ww), ix = (int)(pos % a.Ww);
+            const int ip = (int)pos, iy = ip / a.Ww, ix = ip - iy * a.Ww;   // positions < 2^30
             if (k == 0) {
                 sX[p] = pos < npos ? (float)iy / (float)a.Hh : 0.0f;
                 sX[AS + p] = pos < npos ? (float)ix / (float)a.Ww : 0.0f;
@@ -238,48 +240,54 @@ __device__ __forceinline__ void layers_tile(const FilterGenArgs& a, long npos, l
     __syncthreads();
 }
 
-// The decay window of row r (alpha index r % D) at position pos: the
-// argument is i (1-D) or iy + ix (2-D).
+// The argument of the decay window at position pos: i (1-D) or iy + ix
+// (2-D; positions are below 2^30).
 template <bool TWO_D>
-__device__ __forceinline__ float window(const FilterGenArgs& a, float al, long pos)
+__device__ __forceinline__ float window_dist(const FilterGenArgs& a, long pos)
 {
-    float dist;
-    if constexpr (!TWO_D) dist = (float)pos;
-    else dist = (float)(pos / a.Ww) + (float)(pos % a.Ww);
-    return expf(-al * dist * a.inv_div);
+    if constexpr (!TWO_D) {
+        return (float)pos;
+    } else {
+        const int ip = (int)pos, iy = ip / a.Ww;
+        return (float)(iy + (ip - iy * a.Ww));
+    }
 }
 
-// Load a [64][64] tile of a3 (positions p0 .. p0+63 of the stash rows) into
-// sA [64][kFgUS]; positions past the end read as zero.
+// Load a [64][64 NG] tile of a3 (positions p0 .. p0 + 64 NG - 1 of the
+// stash rows) into sA [64][64 NG + 4]; positions past the end read as zero.
+template <int NG>
 __device__ __forceinline__ void load_a3_tile(const FilterGenArgs& a, long npos, long p0, const float* stash,
                                              float* sA)
 {
+    constexpr int PT = 64 * NG, AS = PT + 4;
     const int tid = threadIdx.x;
     if (a.vec) {
-        float4 v[4];
+        constexpr int PER = kFfnWidth * PT / 4 / kFgThreads;
+        float4 v[PER];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int e = tid + i * kFgThreads, j = e / 16, q = e % 16;
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads, j = e / (PT / 4), q = e % (PT / 4);
             const long pos = p0 + 4 * q;
             v[i] = pos < npos ? *reinterpret_cast<const float4*>(stash + (long)j * npos + pos)
                               : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int e = tid + i * kFgThreads, j = e / 16, q = e % 16;
-            *reinterpret_cast<float4*>(sA + j * kFgUS + 4 * q) = v[i];
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads, j = e / (PT / 4), q = e % (PT / 4);
+            *reinterpret_cast<float4*>(sA + j * AS + 4 * q) = v[i];
         }
     } else {
-        float v[16];
+        constexpr int PER = kFfnWidth * PT / kFgThreads;
+        float v[PER];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int e = tid + i * kFgThreads, j = e / 64, pp = e % 64;
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads, j = e / PT, pp = e % PT;
             v[i] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < PER; ++i) {
             const int e = tid + i * kFgThreads;
-            sA[(e / 64) * kFgUS + e % 64] = v[i];
+            sA[(e / PT) * AS + e % PT] = v[i];
         }
     }
 }
@@ -305,50 +313,61 @@ __device__ __forceinline__ void load_wout_tile(const FilterGenArgs& a, int r0, i
 }
 
 // h[r][p] = (sum_j Wout[r][j] a3[j][p]) * window for rows r0 + RT ty + i
-// (i < RT, r < r_end) and positions p0 + 4 tx + k (k < 4) from sWT
-// [64][RS] and sA [64][kFgUS]; alpha of the thread's rows is passed in.
-template <bool TWO_D, int RT, int RS>
+// (i < RT, r < r_end) and positions p0 + 64 g + 4 tx + k (g < NG, k < 4)
+// from sWT [64][RS] and sA [64][64 NG + 4] (each 128-bit load of a3 is then
+// contiguous across the 16 tx); alpha of the thread's rows is passed in.
+template <bool TWO_D, int RT, int RS, int NG>
 __device__ __forceinline__ void head_block(const FilterGenArgs& a, long npos, long p0, int r0, int r_end,
                                            const float* sWT, const float* sA, const float* al)
 {
+    constexpr int AS = 64 * NG + 4;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-    float acc[RT][4];
+    float acc[RT][4 * NG];
 #pragma unroll
     for (int i = 0; i < RT; ++i)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) acc[i][k] = 0.0f;
+        for (int k = 0; k < 4 * NG; ++k) acc[i][k] = 0.0f;
 #pragma unroll 8
     for (int j = 0; j < kFfnWidth; ++j) {
-        const float4 x4 = *reinterpret_cast<const float4*>(sA + j * kFgUS + 4 * tx);
-        float w[RT];
+        float x[4 * NG], w[RT];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            const float4 x4 = *reinterpret_cast<const float4*>(sA + j * AS + 64 * g + 4 * tx);
+            x[4 * g] = x4.x; x[4 * g + 1] = x4.y; x[4 * g + 2] = x4.z; x[4 * g + 3] = x4.w;
+        }
 #pragma unroll
         for (int i = 0; i < RT; i += 4) {
             const float4 w4 = *reinterpret_cast<const float4*>(sWT + j * RS + RT * ty + i);
             w[i] = w4.x; w[i + 1] = w4.y; w[i + 2] = w4.z; w[i + 3] = w4.w;
         }
-        const float x[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
         for (int i = 0; i < RT; ++i)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc[i][k] = fmaf(w[i], x[k], acc[i][k]);
+            for (int k = 0; k < 4 * NG; ++k) acc[i][k] = fmaf(w[i], x[k], acc[i][k]);
     }
-    const long pos0 = p0 + 4 * tx;
 #pragma unroll
-    for (int i = 0; i < RT; ++i) {
-        const int r = r0 + RT * ty + i;
-        if (r >= r_end) continue;
-        float* hr = a.h + (long)r * npos;
-        if (a.vec) {
-            if (pos0 < npos)
-                *reinterpret_cast<float4*>(hr + pos0) =
-                    make_float4(acc[i][0] * window<TWO_D>(a, al[i], pos0),
-                                acc[i][1] * window<TWO_D>(a, al[i], pos0 + 1),
-                                acc[i][2] * window<TWO_D>(a, al[i], pos0 + 2),
-                                acc[i][3] * window<TWO_D>(a, al[i], pos0 + 3));
-        } else {
+    for (int g = 0; g < NG; ++g) {
+        const long pos0 = p0 + 64 * g + 4 * tx;
+        float dist[4];   // window arguments of the group's 4 positions
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                if (pos0 + k < npos) hr[pos0 + k] = acc[i][k] * window<TWO_D>(a, al[i], pos0 + k);
+        for (int k = 0; k < 4; ++k) dist[k] = window_dist<TWO_D>(a, pos0 + k);
+#pragma unroll
+        for (int i = 0; i < RT; ++i) {
+            const int r = r0 + RT * ty + i;
+            if (r >= r_end) continue;
+            float* hr = a.h + (long)r * npos;
+            const float c = -al[i] * a.inv_div;
+            const float* v = acc[i] + 4 * g;
+            if (a.vec) {
+                if (pos0 < npos)
+                    *reinterpret_cast<float4*>(hr + pos0) =
+                        make_float4(v[0] * expf(c * dist[0]), v[1] * expf(c * dist[1]),
+                                    v[2] * expf(c * dist[2]), v[3] * expf(c * dist[3]));
+            } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (pos0 + k < npos) hr[pos0 + k] = v[k] * expf(c * dist[k]);
+            }
         }
     }
 }
@@ -408,25 +427,25 @@ __global__ void __launch_bounds__(kFgThreads) filter_layers_kernel(FilterGenArgs
     }
 }
 
-// Head kernel: rows 0 .. rows-65 as 128-row x 64-position tiles (grid.y
+// Head kernel: rows 0 .. rows-65 as 128-row x 64 NG-position tiles (grid.y
 // over row tiles), thread (ty, tx) owning rows 8 ty + i (i < 8) and
-// positions 4 tx + k (k < 4).
-template <bool TWO_D>
-__global__ void __launch_bounds__(kFgThreads) filter_head_kernel(FilterGenArgs a)
+// positions 64 g + 4 tx + k (g < NG, k < 4).
+template <bool TWO_D, int NG>
+__global__ void __launch_bounds__(kFgThreads, NG == 1 ? 3 : 2) filter_head_kernel(FilterGenArgs a)
 {
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][132]: Wout tile, transposed
-    float* sA = fg_smem + kFfnWidth * kFgRS;                // [64][68]:  a3 tile
+    float* sA = fg_smem + kFfnWidth * kFgRS;                // [64][64 NG + 4]: a3 tile
     const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
-    const long p0 = (long)blockIdx.x * kFgTile;
+    const long p0 = (long)blockIdx.x * (64 * NG);
     const int r0 = blockIdx.y * kFgRowTile;
     const int stash_row = a.rows - kFfnWidth;
     float al[8];
     load_alpha<8>(a, r0, stash_row, al);
-    load_a3_tile(a, npos, p0, a.h + (long)stash_row * npos, sA);
+    load_a3_tile<NG>(a, npos, p0, a.h + (long)stash_row * npos, sA);
     load_wout_tile<kFgRowTile, kFgRS>(a, r0, stash_row, sWT);
     __syncthreads();
-    head_block<TWO_D, 8, kFgRS>(a, npos, p0, r0, stash_row, sWT, sA, al);
+    head_block<TWO_D, 8, kFgRS, NG>(a, npos, p0, r0, stash_row, sWT, sA, al);
 }
 
 // Tail kernel: the 64 stash rows for 64 positions per CTA; each CTA reads
@@ -442,10 +461,60 @@ __global__ void __launch_bounds__(kFgThreads) filter_tail_kernel(FilterGenArgs a
     const int stash_row = a.rows - kFfnWidth;
     float al[4];
     load_alpha<4>(a, stash_row, a.rows, al);
-    load_a3_tile(a, npos, p0, a.h + (long)stash_row * npos, sA);
+    load_a3_tile<1>(a, npos, p0, a.h + (long)stash_row * npos, sA);
     load_wout_tile<kFfnWidth, kFgUS>(a, stash_row, a.rows, sWT);
     __syncthreads();
-    head_block<TWO_D, 4, kFgUS>(a, npos, p0, stash_row, a.rows, sWT, sA, al);
+    head_block<TWO_D, 4, kFgUS, 1>(a, npos, p0, stash_row, a.rows, sWT, sA, al);
+}
+
+// Tail kernel for short filters: 16 positions per CTA (more CTAs), thread
+// (ty, tx) owning stash rows 4 ty + i (i < 4) at position tx.
+template <bool TWO_D>
+__global__ void __launch_bounds__(kFgThreads) filter_tail16_kernel(FilterGenArgs a)
+{
+    constexpr int PT = kFgSmallTile, AS = PT + 4;
+    extern __shared__ __align__(16) float fg_smem[];
+    float* sWT = fg_smem;                                   // [64][68]: Wout stash rows, transposed
+    float* sA = fg_smem + kFfnWidth * kFgUS;                // [64][20]: a3 tile
+    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long p0 = (long)blockIdx.x * PT;
+    const int stash_row = a.rows - kFfnWidth;
+    float* stash = a.h + (long)stash_row * npos;
+    const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+    float al[4];
+    load_alpha<4>(a, stash_row, a.rows, al);
+    {
+        constexpr int PER = kFfnWidth * PT / kFgThreads;
+        float v[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads, j = e / PT, pp = e % PT;
+            v[i] = p0 + pp < npos ? stash[(long)j * npos + p0 + pp] : 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int e = tid + i * kFgThreads;
+            sA[(e / PT) * AS + e % PT] = v[i];
+        }
+    }
+    load_wout_tile<kFfnWidth, kFgUS>(a, stash_row, a.rows, sWT);
+    __syncthreads();
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 8
+    for (int j = 0; j < kFfnWidth; ++j) {
+        const float4 w = *reinterpret_cast<const float4*>(sWT + j * kFgUS + 4 * ty);
+        const float x = sA[j * AS + tx];
+        acc[0] = fmaf(w.x, x, acc[0]);
+        acc[1] = fmaf(w.y, x, acc[1]);
+        acc[2] = fmaf(w.z, x, acc[2]);
+        acc[3] = fmaf(w.w, x, acc[3]);
+    }
+    const long pos = p0 + tx;
+    if (pos >= npos) return;
+    const float dist = window_dist<TWO_D>(a, pos);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        stash[(long)(4 * ty + i) * npos + pos] = acc[i] * expf(-al[i] * a.inv_div * dist);
 }
 
 // Single launch for at most 64 rows: every CTA evaluates the layers of its
@@ -467,7 +536,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
     load_wout_tile<kFfnWidth, kFgUS>(a, 0, a.rows, sW);   // the weights are no longer read
     __syncthreads();
     static_assert(LT::AS == kFgUS, "a3 tile stride");
-    head_block<TWO_D, 4, kFgUS>(a, npos, p0, 0, a.rows, sW, sY, al);
+    head_block<TWO_D, 4, kFgUS, 1>(a, npos, p0, 0, a.rows, sW, sY, al);
 }
 
 }  // namespace hyena

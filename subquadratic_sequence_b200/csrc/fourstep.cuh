@@ -62,10 +62,10 @@ struct SmemFft {
             static_for<C>([&](auto cc) {
                 constexpr int c = decltype(cc)::value;
                 const int j = t + c * T;
+                const int pj = pad16(j);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    const int i = j + r * (S / R);
-                    a[c * R + r] = buf[(p == 0 && !PADDED_IN) ? i : pad16(i)];
+                    a[c * R + r] = buf[(p == 0 && !PADDED_IN) ? j + r * (S / R) : pad16_at<S / R>(j, pj, r)];
                 });
             });
             __syncthreads();
@@ -80,9 +80,10 @@ struct SmemFft {
                 dft<R, SIGN>(ar);
                 if constexpr (!LAST) {
                     const int base = (j / NS) * NS * R + jm;
+                    const int pb = pad16(base);
                     static_for<R>([&](auto rr) {
                         constexpr int r = decltype(rr)::value;
-                        buf[pad16(base + r * NS)] = ar[r];
+                        buf[pad16_at<NS>(base, pb, r)] = ar[r];
                     });
                 }
                 dep = zero_after(ar[R - 1].x);
@@ -128,6 +129,49 @@ struct FourStep {
     static_assert(ROW_THREADS <= 1024 && COL_THREADS <= 1024, "block size");
     static_assert(ROW_SMEM <= 227 * 1024 && COL_SMEM <= 227 * 1024, "shared memory");
     static_assert(M2 % TC == 0 && (M1 / 2) % U == 0, "tiling");
+
+    // Bin pairs (k, M - k) of the real split over the CTA's row pairs, in
+    // shared memory after the forward row FFTs (row slot 2 up holds row u,
+    // slot 2 up + 1 row M1 - u; unit 0: rows 0 and M1/2).  Thread tid takes
+    // unit up = tid % U and k2 = tid / U + it M2/8 (it < 8), so adjacent
+    // threads touch adjacent spectrum slots (k1 consecutive), and the
+    // split's twiddle exp(-i pi k / M) of iteration it is that of it = 0
+    // times exp(-i pi it / 8).  f(kind, p1, p2, k, w): kind 0 = bins k
+    // (*p1) and M - k (*p2); 1 = bins 0 and M (slot 0, p1 == p2); 2 = bin
+    // M/2 alone (p1 == p2).
+    template <typename Fn>
+    static __device__ __forceinline__ void for_each_pair(float2* smem, int ublk, int tid, Fn&& f)
+    {
+        constexpr int RS = ROW_STRIDE, KSTEP = ROW_THREADS / U, ITER = U * M2 / ROW_THREADS;
+        static_assert(ITER == 8 && ITER * KSTEP == M2, "pair iteration");
+        const int up = tid % U, k20 = tid / U, u = ublk * U + up;
+        float2* r0 = smem + (2 * up) * RS;
+        float2* r1 = smem + (2 * up + 1) * RS;
+        if (u != 0) {
+            const int k0 = u + M1 * k20;                    // partner M - k: row M1 - u, slot M2 - 1 - k2
+            const float2 w0 = expi_pi<-1>((float)k0 / (float)M);
+            static_for<ITER>([&](auto ii) {
+                constexpr int it = decltype(ii)::value;
+                const int k2 = k20 + it * KSTEP;
+                f(0, r0 + pad16(k2), r1 + pad16(M2 - 1 - k2), k0 + it * KSTEP * M1, mul_w64<4 * it, -1>(w0));
+            });
+        } else {
+            // row M1/2 pairs with itself reversed; row 0 pairs k2 with M2 - k2
+            const float2 wh0 = expi_pi<-1>((float)(M1 / 2 + M1 * k20) / (float)M);
+            const float2 wz0 = expi_pi<-1>((float)(M1 * k20) / (float)M);
+            static_for<ITER / 2>([&](auto ii) {
+                constexpr int it = decltype(ii)::value;
+                const int k2 = k20 + it * KSTEP;             // < M2 / 2
+                f(0, r1 + pad16(k2), r1 + pad16(M2 - 1 - k2), M1 / 2 + M1 * k2, mul_w64<4 * it, -1>(wh0));
+                if (k2 > 0) {
+                    f(0, r0 + pad16(k2), r0 + pad16(M2 - k2), M1 * k2, mul_w64<4 * it, -1>(wz0));
+                } else {
+                    f(1, r0, r0, 0, make_float2(1.0f, 0.0f));
+                    f(2, r0 + pad16(M2 / 2), r0 + pad16(M2 / 2), M / 2, make_float2(0.0f, -1.0f));
+                }
+            });
+        }
+    }
 
     // row of the CTA's row slot rr (units u: rows u and M1 - u; unit 0:
     // rows 0 and M1/2)
@@ -201,91 +245,41 @@ fourstep_row_kernel(FourStepArgs a)
     float2* rb = smem_fs + row * RS;
     float2 reg[16];
     FS::F2::template run<-1, false>(rb, reg, t);
+    const int pt = pad16(t);
     static_for<16>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
-        rb[pad16(t + r * (M2 / 16))] = reg[r];
+        rb[pad16_at<M2 / 16>(t, pt, r)] = reg[r];
     });
     __syncthreads();
 
-    // bin pairs: thread p -> (row pair up = p % U, k2 = p / U), so adjacent
-    // threads touch adjacent spectrum slots (k1 consecutive)
     if constexpr (SPECTRUM) {
         float2* Ho = a.Hout + (size_t)q * M;
-#pragma unroll 1
-        for (int p = tid; p < U * M2; p += FS::ROW_THREADS) {
-            const int up = p % U, k2 = p / U, u = ublk * U + up;
-            float2* r0 = smem_fs + (2 * up) * RS;
-            float2* r1 = smem_fs + (2 * up + 1) * RS;
-            float2 X1, X2;
-            if (u != 0) {
-                const int k = u + M1 * k2;
-                real_split(r0[pad16(k2)], r1[pad16(M2 - 1 - k2)], expi_pi<-1>((float)k / (float)M), X1, X2);
+        FS::for_each_pair(smem_fs, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2 w) {
+            if (kind == 1) {                                    // bins 0 and M share slot 0
+                const float2 z = *p1;
+                Ho[0] = make_float2(z.x + z.y, z.x - z.y);
+            } else {
+                float2 X1, X2;
+                real_split(*p1, *p2, w, X1, X2);
                 Ho[k] = X1;
-                Ho[M - k] = X2;
-            } else if (k2 < M2 / 2) {
-                const int k = M1 / 2 + M1 * k2;     // row M1/2 with itself, reversed
-                real_split(r1[pad16(k2)], r1[pad16(M2 - 1 - k2)], expi_pi<-1>((float)k / (float)M), X1, X2);
-                Ho[k] = X1;
-                Ho[M - k] = X2;
-                if (k2 > 0) {                        // row 0: k2 with M2 - k2
-                    const int k0 = M1 * k2;
-                    real_split(r0[pad16(k2)], r0[pad16(M2 - k2)], expi_pi<-1>((float)k0 / (float)M), X1, X2);
-                    Ho[k0] = X1;
-                    Ho[M - k0] = X2;
-                } else {                             // bins 0 and M (slot 0), and M/2
-                    const float2 z = r0[0];
-                    Ho[0] = make_float2(z.x + z.y, z.x - z.y);
-                    const float2 zh = r0[pad16(M2 / 2)];
-                    real_split(zh, zh, make_float2(0.0f, -1.0f), X1, X2);
-                    Ho[M / 2] = X1;
-                }
+                if (kind == 0) Ho[M - k] = X2;
             }
-        }
+        });
         return;
     } else {
         const float bias = __ldg(a.bias + a.n * a.D + d);
         const float2* Hr = a.H + ((size_t)a.n * a.D + d) * M;
-#pragma unroll 1
-        for (int p = tid; p < U * M2; p += FS::ROW_THREADS) {
-            const int up = p % U, k2 = p / U, u = ublk * U + up;
-            float2* r0 = smem_fs + (2 * up) * RS;
-            float2* r1 = smem_fs + (2 * up + 1) * RS;
-            if (u != 0) {
-                const int k = u + M1 * k2;           // partner M - k: row M1 - u, slot M2 - 1 - k2
-                float2 z1 = r0[pad16(k2)], z2 = r1[pad16(M2 - 1 - k2)];
-                spectral_pair<M>(z1, z2, __ldg(Hr + k), __ldg(Hr + (M - k)),
-                                 expi_pi<-1>((float)k / (float)M), bias);
-                r0[pad16(k2)] = z1;
-                r1[pad16(M2 - 1 - k2)] = z2;
-            } else if (k2 < M2 / 2) {
-                {
-                    const int k = M1 / 2 + M1 * k2;
-                    float2 z1 = r1[pad16(k2)], z2 = r1[pad16(M2 - 1 - k2)];
-                    spectral_pair<M>(z1, z2, __ldg(Hr + k), __ldg(Hr + (M - k)),
-                                     expi_pi<-1>((float)k / (float)M), bias);
-                    r1[pad16(k2)] = z1;
-                    r1[pad16(M2 - 1 - k2)] = z2;
-                }
-                if (k2 > 0) {
-                    const int k = M1 * k2;
-                    float2 z1 = r0[pad16(k2)], z2 = r0[pad16(M2 - k2)];
-                    spectral_pair<M>(z1, z2, __ldg(Hr + k), __ldg(Hr + (M - k)),
-                                     expi_pi<-1>((float)k / (float)M), bias);
-                    r0[pad16(k2)] = z1;
-                    r0[pad16(M2 - k2)] = z2;
-                } else {
-                    const float2 h0 = __ldg(Hr);
-                    float2 z1 = r0[0], z2 = z1;
-                    spectral_pair<M>(z1, z2, make_float2(h0.x, 0.0f), make_float2(h0.y, 0.0f),
-                                     make_float2(1.0f, 0.0f), bias);
-                    r0[0] = z1;
-                    const float2 hm = __ldg(Hr + M / 2);
-                    float2 w1 = r0[pad16(M2 / 2)], w2 = w1;
-                    spectral_pair<M>(w1, w2, hm, hm, make_float2(0.0f, -1.0f), bias);
-                    r0[pad16(M2 / 2)] = w1;
-                }
+        FS::for_each_pair(smem_fs, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2 w) {
+            float2 z1 = *p1, z2 = *p2;
+            if (kind == 1) {                                    // slot 0 holds (bin 0, bin M), both real
+                const float2 h0 = __ldg(Hr);
+                spectral_pair<M>(z1, z2, make_float2(h0.x, 0.0f), make_float2(h0.y, 0.0f), w, bias);
+            } else {
+                spectral_pair<M>(z1, z2, __ldg(Hr + k), __ldg(Hr + (M - k)), w, bias);
             }
-        }
+            *p1 = z1;
+            if (kind == 0) *p2 = z2;
+        });
         __syncthreads();
 
         FS::F2::template run<+1, true>(rb, reg, t);
@@ -333,10 +327,11 @@ fourstep_col_kernel(FourStepArgs a)
             reg[r] = IOP::load(vp + n2 + (size_t)M2 * (t + r * (M1 / 16)));
         });
     } else {
+        const int pt = pad16(t);
         static_for<16>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             const int k1 = t + r * (M1 / 16);
-            buf[pad16(k1)] = Sq[(size_t)k1 * M2 + n2];
+            buf[pad16_at<M1 / 16>(t, pt, r)] = Sq[(size_t)k1 * M2 + n2];
         });
         __syncthreads();
         FS::F1::template run<+1, true>(buf, reg, t);
@@ -362,10 +357,13 @@ fourstep_col_kernel(FourStepArgs a)
     }
     // forward column FFT of z (n1 < M1/2), zero-padded, then the four-step
     // twiddle exp(-2 pi i n2 k1 / M)
-    static_for<16>([&](auto rr) {
-        constexpr int r = decltype(rr)::value;
-        buf[pad16(t + r * (M1 / 16))] = r < 8 ? reg[r] : make_float2(0.0f, 0.0f);
-    });
+    {
+        const int pt = pad16(t);
+        static_for<16>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            buf[pad16_at<M1 / 16>(t, pt, r)] = r < 8 ? reg[r] : make_float2(0.0f, 0.0f);
+        });
+    }
     __syncthreads();
     FS::F1::template run<-1, true>(buf, reg, t);
     float2 w = expi_pi<-1>(2.0f * (float)((n2 * t) % M) / (float)M);

@@ -31,12 +31,21 @@ hyena_status_t filter_gen_launches(const FilterGenArgs& a, long npos, cudaStream
     s = (long)ptiles >= 2L * sms ? launch_layers<TWO_D, kFgTile>(a, npos, sms, 2, st)
                                  : launch_layers<TWO_D, kFgSmallTile>(a, npos, sms, 3, st);
     const int head_rows = a.rows - kFfnWidth;
+    const unsigned rtiles = (unsigned)((head_rows + kFgRowTile - 1) / kFgRowTile);
+    const unsigned ptiles2 = (unsigned)((npos + 127) / 128);
+    // 128-position tiles (8 x 8 outputs per thread) once they fill every SM twice
     if (s == HYENA_OK && head_rows > 0)
-        s = launch(filter_head_kernel<TWO_D>,
-                   dim3(ptiles, (unsigned)((head_rows + kFgRowTile - 1) / kFgRowTile)), kFgThreads,
-                   kFgHeadSmemBytes, st, a);
+        s = (long)ptiles2 * rtiles >= 2L * sms
+                ? launch(filter_head_kernel<TWO_D, 2>, dim3(ptiles2, rtiles), kFgThreads,
+                         fg_head_smem_bytes<2>(), st, a)
+                : launch(filter_head_kernel<TWO_D, 1>, dim3(ptiles, rtiles), kFgThreads,
+                         fg_head_smem_bytes<1>(), st, a);
+    // the tail in 16-position tiles unless 64-position tiles fill every SM
     if (s == HYENA_OK)
-        s = launch(filter_tail_kernel<TWO_D>, dim3(ptiles), kFgThreads, kFgTailSmemBytes, st, a);
+        s = (long)ptiles >= sms
+                ? launch(filter_tail_kernel<TWO_D>, dim3(ptiles), kFgThreads, kFgTailSmemBytes, st, a)
+                : launch(filter_tail16_kernel<TWO_D>, dim3((unsigned)((npos + kFgSmallTile - 1) / kFgSmallTile)),
+                         kFgThreads, kFgTail16SmemBytes, st, a);
     return s;
 }
 

@@ -56,7 +56,10 @@ def oracle_forward(inp, h, seqs=None, route="fft"):
 
 # ------------------------------------------------------------- filters
 
-@pytest.mark.parametrize("N,D,L", [(2, 64, 1024), (2, 768, 2048), (3, 5, 100), (1, 1, 1), (2, 3, 65536)])
+# covers the single-launch path (N*D <= 64), the 64- and 128-position head
+# tiles, and lengths that are not a multiple of 4 (scalar h access)
+@pytest.mark.parametrize("N,D,L", [(2, 64, 1024), (2, 768, 2048), (3, 5, 100), (1, 1, 1), (2, 3, 65536),
+                                   (3, 100, 5001), (2, 256, 65536), (2, 256, 65535)])
 def test_filter_gen_matches_oracle(hy, N, D, L):
     wl, inp = random_problem(1, D, L, N, seed=11 + L)
     got = host(gpu_filters(inp, wl))
@@ -64,7 +67,7 @@ def test_filter_gen_matches_oracle(hy, N, D, L):
     assert rel_max_err(got, ref) <= 2e-5
 
 
-@pytest.mark.parametrize("N,C,H,W", [(2, 4, 16, 32), (1, 3, 7, 5), (2, 128, 256, 256)])
+@pytest.mark.parametrize("N,C,H,W", [(2, 4, 16, 32), (1, 3, 7, 5), (2, 128, 256, 256), (2, 128, 255, 257)])
 def test_filter_gen_2d_matches_oracle(hy, N, C, H, W):
     wl = synth.Workload("c", "2d", N=N, B=1, D=C, H=H, W=W, seed=7 + H)
     inp = synth.make_inputs(wl)
