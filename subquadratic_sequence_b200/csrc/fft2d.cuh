@@ -124,6 +124,7 @@ template <int LOG2W, typename IO, int MODE>
 __global__ void __launch_bounds__(Fft1d<LOG2W>::THREADS)
 fft2d_row_kernel(Fft2dArgs a)
 {
+    grid_dependency_begin();
     using R = Fft2dRows<LOG2W>;
     using F = typename R::F;
     using IOP = IoPair<IO>;
@@ -207,6 +208,7 @@ template <int LOG2H2, bool SPECTRUM>
 __global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS, Fft2dCols<LOG2H2>::MIN_BLOCKS)
 fft2d_col_kernel(Fft2dArgs a)
 {
+    grid_dependency_begin();
     using CL = Fft2dCols<LOG2H2>;
     using FC = typename CL::FC;
     constexpr int H2 = CL::H2, TC = CL::TC, HH = H2 / 2;

@@ -390,6 +390,7 @@ __device__ __forceinline__ void load_alpha(const FilterGenArgs& a, int r0, int r
 template <bool TWO_D, int PT>
 __global__ void __launch_bounds__(kFgThreads) filter_layers_kernel(FilterGenArgs a)
 {
+    grid_dependency_begin();
     using LT = LayerTile<PT>;
     constexpr int AS = LT::AS, PPT = LT::PPT;
     extern __shared__ __align__(16) float fg_smem[];
@@ -433,6 +434,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_layers_kernel(FilterGenArgs
 template <bool TWO_D, int NG>
 __global__ void __launch_bounds__(kFgThreads, NG == 1 ? 3 : 2) filter_head_kernel(FilterGenArgs a)
 {
+    grid_dependency_begin();
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][132]: Wout tile, transposed
     float* sA = fg_smem + kFfnWidth * kFgRS;                // [64][64 NG + 4]: a3 tile
@@ -453,6 +455,7 @@ __global__ void __launch_bounds__(kFgThreads, NG == 1 ? 3 : 2) filter_head_kerne
 template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_tail_kernel(FilterGenArgs a)
 {
+    grid_dependency_begin();
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][68]: Wout stash rows, transposed
     float* sA = fg_smem + kFfnWidth * kFgUS;                // [64][68]: a3 tile
@@ -472,6 +475,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_tail_kernel(FilterGenArgs a
 template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_tail16_kernel(FilterGenArgs a)
 {
+    grid_dependency_begin();
     constexpr int PT = kFgSmallTile, AS = PT + 4;
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][68]: Wout stash rows, transposed
@@ -522,6 +526,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_tail16_kernel(FilterGenArgs
 template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
 {
+    grid_dependency_begin();
     using LT = LayerTile<kFgTile>;
     extern __shared__ __align__(16) float fg_smem[];
     float* sW = fg_smem;

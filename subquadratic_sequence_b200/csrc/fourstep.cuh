@@ -222,6 +222,7 @@ template <int LOG2M1, int LOG2M2, bool SPECTRUM>
 __global__ void __launch_bounds__(FourStep<LOG2M1, LOG2M2>::ROW_THREADS)
 fourstep_row_kernel(FourStepArgs a)
 {
+    grid_dependency_begin();
     using FS = FourStep<LOG2M1, LOG2M2>;
     constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, U = FS::U, T2 = FS::F2::T;
     constexpr int RS = FS::ROW_STRIDE;
@@ -302,6 +303,7 @@ template <int LOG2M1, int LOG2M2, typename IO, int MODE>
 __global__ void __launch_bounds__(FourStep<LOG2M1, LOG2M2>::COL_THREADS)
 fourstep_col_kernel(FourStepArgs a)
 {
+    grid_dependency_begin();
     using FS = FourStep<LOG2M1, LOG2M2>;
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;

@@ -376,6 +376,7 @@ template <int LOG2M, typename IO>
 __global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS, Fft1d<LOG2M>::MIN_BLOCKS)
 fused1d_kernel(Fused1dArgs args)
 {
+    grid_dependency_begin();
     using F = Fft1d<LOG2M>;
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;
@@ -454,6 +455,7 @@ template <int LOG2M>
 __global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS)
 rfft1d_kernel(Rfft1dArgs args)
 {
+    grid_dependency_begin();
     using F = Fft1d<LOG2M>;
     constexpr int M = F::M, E = F::E, T = F::T, R = F::P::RL, NCOL = M / R;
     extern __shared__ __align__(16) float2 smem_dyn[];

@@ -204,6 +204,20 @@ __device__ __forceinline__ void apply_twiddle_powers(float2* a, float2 w)
     }
 }
 
+// ------------------------------------------- programmatic dependent launch
+
+// Every kernel of the library is launched with programmatic stream
+// serialisation.  At entry it lets the next kernel in the stream begin
+// launching (its CTAs are placed as this grid's CTAs drain, once all of them
+// have started), then waits until the previous kernel in the stream has
+// completed and its memory operations are visible, before touching global
+// memory.  This hides the launch gap between dependent kernels.
+__device__ __forceinline__ void grid_dependency_begin()
+{
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+
 // ---------------------------------------------------------------- I/O
 
 // Storage types of v, x_n and y.  Two consecutive real samples are moved

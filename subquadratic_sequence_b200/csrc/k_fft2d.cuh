@@ -27,7 +27,7 @@ hyena_status_t launch_rows2d(const Fft2dArgs& a, cudaStream_t st)
     using F = Fft1d<LOG2W>;
     const long rows = (long)a.nq * a.H;
     return launch(fft2d_row_kernel<LOG2W, IO, MODE>, (unsigned)((rows + F::G - 1) / F::G), F::THREADS,
-                  F::SMEM_BYTES_FFT, st, a);
+                  F::SMEM_BYTES_FFT, st, a, false);
 }
 
 // the order-N 2-D forward over B*C images, wave by wave

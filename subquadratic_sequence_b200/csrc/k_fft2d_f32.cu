@@ -9,8 +9,8 @@ hyena_status_t launch_cols2d_n(bool spectrum, const Fft2dArgs& a, cudaStream_t s
 {
     using CL = Fft2dCols<LOG2H2>;
     const unsigned grid = (unsigned)((long)a.nq * (a.W / CL::TC));
-    return spectrum ? launch(fft2d_col_kernel<LOG2H2, true>, grid, CL::THREADS, CL::SMEM, st, a)
-                    : launch(fft2d_col_kernel<LOG2H2, false>, grid, CL::THREADS, CL::SMEM, st, a);
+    return spectrum ? launch(fft2d_col_kernel<LOG2H2, true>, grid, CL::THREADS, CL::SMEM, st, a, false)
+                    : launch(fft2d_col_kernel<LOG2H2, false>, grid, CL::THREADS, CL::SMEM, st, a, false);
 }
 
 hyena_status_t launch_cols2d(int log2h, bool spectrum, const Fft2dArgs& a, cudaStream_t st)

@@ -30,13 +30,27 @@ cudaError_t allow_smem(K kernel, size_t bytes)
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <typename K, typename A>
-hyena_status_t launch(K kernel, dim3 grid, int threads, size_t smem, cudaStream_t st, const A& a)
+// Launches a kernel (every kernel starts with grid_dependency_begin()).
+// With `pdl` it is launched with programmatic stream serialisation, so its
+// CTAs may be placed while the previous kernel drains; the 2-D FFT kernels
+// measured slower that way and are launched plainly.
+template <typename A>
+hyena_status_t launch(void (*kernel)(A), dim3 grid, int threads, size_t smem, cudaStream_t st, const A& a,
+                      bool pdl = true)
 {
     cudaError_t e = allow_smem(kernel, smem);
     if (e != cudaSuccess) return from_cuda(e);
-    kernel<<<grid, threads, smem, st>>>(a);
-    return from_cuda(cudaGetLastError());
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return from_cuda(cudaLaunchKernelEx(&cfg, kernel, a));
 }
 
 // Number of SMs of the current device.
