@@ -59,6 +59,7 @@ def _load():
         "oracle_conv2": [dp, dp, l, l, i, dp],
         "oracle_hyena_forward": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
         "oracle_hyena_forward_2d": [dp, dp, dp, dp, l, l, l, l, l, i, i, dp],
+        "oracle_hyena_backward": [dp, dp, dp, dp, dp, l, l, l, l, i, i, dp, dp, dp, dp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -201,3 +202,23 @@ def hyena_forward_2d(v, x, h, bias, route="fft", threads=None) -> np.ndarray:
                                          threads or default_threads(), _ptr(y))
     _check(rc, "oracle_hyena_forward_2d")
     return y
+
+
+def hyena_backward(v, x, h, bias, dy, route="fft", threads=None):
+    """Gradients of a scalar loss with dL/dy = dy through the order-N
+    recurrence: returns (dv [B][D][L], dx [N][B][D][L], dh [N][D][L],
+    dbias [N][D]); dh and dbias are summed over the batch."""
+    v, x, h, bias, dy = map(_f64, (v, x, h, bias, dy))
+    B, D, L = v.shape
+    N = h.shape[0]
+    assert x.shape == (N, B, D, L) and h.shape == (N, D, L) and bias.shape == (N, D)
+    assert dy.shape == v.shape
+    dv = np.empty_like(v)
+    dx = np.empty_like(x)
+    dh = np.empty_like(h)
+    db = np.empty_like(bias)
+    rc = _load().oracle_hyena_backward(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), _ptr(dy),
+                                       B, D, L, N, _route(route), threads or default_threads(),
+                                       _ptr(dv), _ptr(dx), _ptr(dh), _ptr(db))
+    _check(rc, "oracle_hyena_backward")
+    return dv, dx, dh, db

@@ -504,6 +504,172 @@ int oracle_hyena_forward(const double *v, const double *x, const double *h,
 }
 
 /* ------------------------------------------------------------------ */
+/* The backward pass of the 1-D recurrence: the exact adjoint.          */
+/* ------------------------------------------------------------------ */
+/*
+ * The pages give no training formulas; the gradient of a composition is
+ * fixed by the chain rule.  With c_n = h_n (*) z_{n-1} + b_n z_{n-1} and
+ * z_n = x_n c_n, and g = dL/dz_n flowing back from g = dy at n = N:
+ *     dx_n          = g * c_n
+ *     e             = g * x_n                       (dL/dc_n)
+ *     dh_n[d][s]   += sum_t e[t] z_{n-1}[t - s]     (s = 0..L-1, t >= s)
+ *     db_n[d]      += sum_t e[t] z_{n-1}[t]
+ *     dz_{n-1}[u]   = sum_{t >= u} h_n[t - u] e[t] + b_n e[u]
+ * and dv = dz_0.  dh and db are summed over the batch.
+ */
+
+/* Adjoint of the causal convolution with respect to its signal:
+ * out[u] = sum_{t=u..L-1} h[t-u] e[t]. */
+static void corr_direct(const double *h, const double *e, long L, double *out)
+{
+    for (long u = 0; u < L; ++u) {
+        double s = 0.0;
+        for (long t = u; t < L; ++t) s += h[t - u] * e[t];
+        out[u] = s;
+    }
+}
+
+/* Lagged products: out[s] = sum_{t=s..L-1} e[t] z[t-s]. */
+static void lagged_direct(const double *e, const double *z, long L, double *out)
+{
+    for (long s = 0; s < L; ++s) {
+        double acc = 0.0;
+        for (long t = s; t < L; ++t) acc += e[t] * z[t - s];
+        out[s] = acc;
+    }
+}
+
+/* out[s] = sum_t a[t + s] b[t] for s = 0..L-1 through the DFT of both
+ * zero-padded to P >= 2L: IDFT(A conj(B)) / P at s.  Both corr_direct
+ * (a = e, b = h) and lagged_direct (a = e, b = z) have this form. */
+static void corr_fft(const double *a, const double *b, long L, double *out,
+                     fft_scratch *s)
+{
+    const long P = s->P;
+    for (long t = 0; t < P; ++t) {
+        s->hr[t] = t < L ? b[t] : 0.0; s->hi[t] = 0.0;
+        s->ur[t] = t < L ? a[t] : 0.0; s->ui[t] = 0.0;
+    }
+    fft_radix2(s->hr, s->hi, P, -1);
+    fft_radix2(s->ur, s->ui, P, -1);
+    for (long k = 0; k < P; ++k) {
+        /* A conj(B) */
+        const double re = s->ur[k] * s->hr[k] + s->ui[k] * s->hi[k];
+        const double im = s->ui[k] * s->hr[k] - s->ur[k] * s->hi[k];
+        s->ur[k] = re;
+        s->ui[k] = im;
+    }
+    fft_radix2(s->ur, s->ui, P, +1);
+    for (long t = 0; t < L; ++t) out[t] = s->ur[t] / (double)P;
+}
+
+typedef struct {
+    const double *v, *x, *h, *bias, *dy;
+    long B, D, L, N;
+    int route;
+    double *dv, *dx, *dh, *dbias;
+    long d0, step; /* channels d0, d0 + step, ... (dh, db summed over b here) */
+    int status;
+} bwd_job;
+
+static void *backward_worker(void *arg)
+{
+    bwd_job *j = (bwd_job *)arg;
+    const long L = j->L, N = j->N, D = j->D, BDL = j->B * D * L;
+    /* z[n] = z_n for n = 0..N-1, c[n] = c_{n+1}; g, e, tmp: length L */
+    double *z = malloc(sizeof(double) * N * L), *c = malloc(sizeof(double) * N * L);
+    double *g = malloc(sizeof(double) * L), *e = malloc(sizeof(double) * L);
+    double *tmp = malloc(sizeof(double) * L);
+    fft_scratch s = {0};
+    if (!z || !c || !g || !e || !tmp ||
+        (j->route == ROUTE_FFT && scratch_alloc(&s, next_pow2(2 * L)) != ORACLE_OK)) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (long d = j->d0; d < D; d += j->step) {
+        for (long n = 0; n < N; ++n) {
+            memset(j->dh + (n * D + d) * L, 0, sizeof(double) * L);
+            j->dbias[n * D + d] = 0.0;
+        }
+        for (long b = 0; b < j->B; ++b) {
+            const long seq = b * D + d;
+            /* forward, keeping z_{n-1} and c_n */
+            memcpy(z, j->v + seq * L, sizeof(double) * L);
+            for (long n = 0; n < N; ++n) {
+                const double *hn = j->h + (n * D + d) * L;
+                const double *xn = j->x + n * BDL + seq * L;
+                const double bn = j->bias[n * D + d];
+                double *zn = z + n * L, *cn = c + n * L;
+                if (j->route == ROUTE_DIRECT) conv_direct(hn, zn, L, cn);
+                else conv_fft(hn, zn, L, cn, &s);
+                for (long t = 0; t < L; ++t) cn[t] += bn * zn[t];
+                if (n + 1 < N)
+                    for (long t = 0; t < L; ++t) z[(n + 1) * L + t] = xn[t] * cn[t];
+            }
+            /* backward */
+            memcpy(g, j->dy + seq * L, sizeof(double) * L);
+            for (long n = N - 1; n >= 0; --n) {
+                const double *hn = j->h + (n * D + d) * L;
+                const double *xn = j->x + n * BDL + seq * L;
+                const double bn = j->bias[n * D + d];
+                const double *zn = z + n * L, *cn = c + n * L;
+                double *dxn = j->dx + n * BDL + seq * L;
+                double *dhn = j->dh + (n * D + d) * L;
+                for (long t = 0; t < L; ++t) {
+                    dxn[t] = g[t] * cn[t];
+                    e[t] = g[t] * xn[t];
+                }
+                if (j->route == ROUTE_DIRECT) lagged_direct(e, zn, L, tmp);
+                else corr_fft(e, zn, L, tmp, &s);
+                for (long t = 0; t < L; ++t) dhn[t] += tmp[t];
+                double db = 0.0;
+                for (long t = 0; t < L; ++t) db += e[t] * zn[t];
+                j->dbias[n * D + d] += db;
+                if (j->route == ROUTE_DIRECT) corr_direct(hn, e, L, tmp);
+                else corr_fft(e, hn, L, tmp, &s);
+                for (long t = 0; t < L; ++t) g[t] = tmp[t] + bn * e[t];
+            }
+            memcpy(j->dv + seq * L, g, sizeof(double) * L); /* dv = dz_0 */
+        }
+    }
+    j->status = ORACLE_OK;
+done:
+    free(z); free(c); free(g); free(e); free(tmp);
+    if (j->route == ROUTE_FFT) scratch_free(&s);
+    return NULL;
+}
+
+/* Gradients of a scalar loss with dL/dy = dy [B][D][L]: dv [B][D][L],
+ * dx [N][B][D][L], dh [N][D][L] and dbias [N][D] (both summed over the
+ * batch).  Inputs as oracle_hyena_forward. */
+int oracle_hyena_backward(const double *v, const double *x, const double *h,
+                          const double *bias, const double *dy, long B, long D,
+                          long L, long N, int route, int nthreads, double *dv,
+                          double *dx, double *dh, double *dbias)
+{
+    if (!v || !x || !h || !bias || !dy || !dv || !dx || !dh || !dbias || B < 1 ||
+        D < 1 || L < 1 || N < 1 || (route != ROUTE_DIRECT && route != ROUTE_FFT))
+        return ORACLE_EBADARG;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > D) nthreads = (int)D;
+    bwd_job *jobs = calloc(nthreads, sizeof(bwd_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        bwd_job j = {v, x, h, bias, dy, B, D, L, N, route, dv, dx, dh, dbias, k, nthreads, 0};
+        jobs[k] = j;
+        pthread_create(&tid[k], NULL, backward_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
 /* 2-D: linear convolution on the grid (Native ND Convolution;         */
 /* Handling Boundaries: zero-pad to double the grid).                  */
 /* ------------------------------------------------------------------ */

@@ -1,0 +1,95 @@
+"""Pins of the oracle's backward pass (the exact adjoint of the recurrence).
+
+The pages give no training formulas; the gradient of the forward is fixed by
+calculus.  Each test checks ``oracle.hyena_backward`` against something it
+does not share code with: central finite differences of the (separately
+pinned) oracle forward, a closed form for a delta filter written out with
+numpy, and identities of the definitions.  A wrong sign, a transposed lag
+(t - s vs s - t) or a dropped bias term fails at least one of them.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def problem(B, D, L, N, seed):
+    r = np.random.default_rng(seed)
+    v = r.standard_normal((B, D, L))
+    x = r.standard_normal((N, B, D, L))
+    h = r.standard_normal((N, D, L)) * np.exp(-np.arange(L) / 4.0)
+    b = r.standard_normal((N, D))
+    dy = r.standard_normal((B, D, L))
+    return v, x, h, b, dy
+
+
+def rel_err(a, b):
+    return float(np.max(np.abs(np.asarray(a) - np.asarray(b))) / max(np.max(np.abs(b)), 1e-300))
+
+
+@pytest.mark.parametrize("N", [1, 2, 3])
+def test_backward_matches_finite_differences(N):
+    # loss = sum(dy * y); every gradient against a central difference of the
+    # oracle forward (direct route), step 1e-6: truncation ~1e-12, rounding ~1e-10
+    v, x, h, b, dy = problem(2, 2, 7, N, seed=N)
+    dv, dx, dh, db = oracle.hyena_backward(v, x, h, b, dy, route="direct")
+
+    def loss(v_, x_, h_, b_):
+        return float(np.sum(dy * oracle.hyena_forward(v_, x_, h_, b_, route="direct")))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name
+
+
+@pytest.mark.parametrize("route", ["direct", "fft"])
+def test_backward_delta_filter_closed_form(route):
+    # N = 1, h = delta_0: y = x (1 + b) v, so
+    # dv = dy x (1+b), dx = dy (1+b) v, db = sum_b sum_t dy x v,
+    # dh[s] = sum_b sum_t dy[t] x[t] v[t - s]
+    B, D, L = 3, 2, 12
+    v, x, _, b, dy = problem(B, D, L, 1, seed=11)
+    h = np.zeros((1, D, L))
+    h[:, :, 0] = 1.0
+    dv, dx, dh, db = oracle.hyena_backward(v, x, h, b, dy, route=route)
+    gain = (1.0 + b[0])[None, :, None]
+    assert rel_err(dv, dy * x[0] * gain) < 1e-13
+    assert rel_err(dx[0], dy * gain * v) < 1e-13
+    assert rel_err(db[0], np.sum(dy * x[0] * v, axis=(0, 2))) < 1e-13
+    want = np.zeros((D, L))
+    e = dy * x[0]
+    for s in range(L):
+        want[:, s] = np.sum(e[:, :, s:] * v[:, :, :L - s], axis=(0, 2))
+    assert rel_err(dh[0], want) < 1e-13
+
+
+def test_backward_routes_agree():
+    v, x, h, b, dy = problem(2, 3, 100, 3, seed=5)
+    a = oracle.hyena_backward(v, x, h, b, dy, route="direct")
+    f = oracle.hyena_backward(v, x, h, b, dy, route="fft")
+    for ga, gf in zip(a, f):
+        assert rel_err(gf, ga) < 1e-12
+
+
+def test_backward_bias_gradient_is_the_lag0_filter_gradient():
+    # db_n[d] and dh_n[d][0] are the same sum over (b, t) of dL/dc_n z_{n-1}
+    v, x, h, b, dy = problem(2, 4, 64, 2, seed=6)
+    _, _, dh, db = oracle.hyena_backward(v, x, h, b, dy)
+    assert rel_err(db, dh[:, :, 0]) < 1e-13
+
+
+def test_backward_linear_in_dy_and_threads_agree():
+    v, x, h, b, dy = problem(2, 3, 32, 2, seed=7)
+    g1 = oracle.hyena_backward(v, x, h, b, dy, threads=1)
+    g2 = oracle.hyena_backward(v, x, h, b, 2.5 * dy, threads=3)
+    for a, c in zip(g1, g2):
+        assert rel_err(c, 2.5 * a) < 1e-13
