@@ -64,6 +64,15 @@ def alg_bytes_forward(wl: synth.Workload) -> int:
     return (wl.N + 2) * wl.B * wl.D * wl.L * wl.io_bytes + wl.N * wl.D * wl.L * 8
 
 
+def alg_bytes_backward(wl: synth.Workload) -> int:
+    """Bytes the backward must move at least: v, x_1..x_N and dy in, dv and
+    dx_1..dx_N out (storage type), the spectra H in (complex64), dh and
+    dbias out (float32)."""
+    io = 2 if wl.io == "bf16" else 4
+    act = wl.B * wl.D * wl.L * io
+    return (2 * wl.N + 3) * act + wl.N * wl.D * wl.L * (8 + 4) + wl.N * wl.D * 4
+
+
 def long_path(wl: synth.Workload) -> bool:
     return wl.kind == "1d" and wl.L > 16384
 
@@ -372,6 +381,32 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(bb) for a, bb in eev))
 
+    # ---- the backward pass (1-D, L <= 16384): one call per timed repetition
+    bwd = None
+    if wl.kind == "1d" and not long_path(wl):
+        dy = to_dev(synth.make_output_grad(wl), io)
+        ws_b = torch.empty(hyena.hyena_fftconv_backward_workspace_size(wl.D, wl.L, wl.N),
+                           device="cuda", dtype=torch.uint8)
+
+        def backward():
+            hyena.hyena_fftconv_gate_backward(v, xs, b, H, dy, workspace=ws_b)
+
+        for _ in range(3):
+            backward()
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(max(args.steps // 5, 5))]
+        for i in range(len(bev)):
+            flush.zero_()
+            bev[i][0].record(stream)
+            backward()
+            bev[i][1].record(stream)
+        torch.cuda.synchronize()
+        bwd_ms = max_over_ranks(statistics.mean(a.elapsed_time(bb) for a, bb in bev))
+        bwd = {"kernel": "backward1d_kernel (hyena_fftconv_gate_backward)", "ms_per_call": bwd_ms,
+               "value": wl.positions * world / (bwd_ms / 1e3), "unit": UNIT,
+               "alg_bytes_per_call": alg_bytes_backward(wl),
+               "achieved_gbs": alg_bytes_backward(wl) / (bwd_ms / 1e3) / 1e9}
+
     ranks.close()
     if rank != 0:
         return None
@@ -396,6 +431,9 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
+    if bwd is not None:
+        bwd["frac"] = bwd["achieved_gbs"] / peak
+        line["backward"] = bwd
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     return line

@@ -185,6 +185,36 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_noalloc(const void* v, const
                                                             hyena_dtype_t io, void* y,
                                                             void* stream);
 
+/* The backward pass of the order-N forward, for training: the gradients of
+ * a scalar loss whose gradient with respect to y is dy.  The pages give
+ * the forward only; the gradient is the exact adjoint (chain rule) of the
+ * recurrence above, with g = dL/dz_n running back from dy:
+ *   dx_n = g * c_n,   e = g * x_n,   (c_n = h_n (*) z_{n-1} + b_n z_{n-1})
+ *   dh_n[d][s] = sum_b sum_t e[t] z_{n-1}[t-s],   db_n[d] = dh_n[d][0],
+ *   dz_{n-1}[u] = sum_{t>=u} h_n[t-u] e[t] + b_n e[u],   dv = dz_0.
+ * Arguments as hyena_fftconv_gate_forward with the cached spectrum H, plus
+ *   dy     [B][D][L] io             gradient of the loss with respect to y
+ *   dv     [B][D][L] io             out
+ *   dx     HOST array of N device pointers, each [B][D][L] io, out
+ *   dh     [N][D][L] float32 out    summed over the batch
+ *   dbias  [N][D] float32 out       summed over the batch
+ *   workspace / ws_bytes: device scratch of at least
+ *          hyena_fftconv_backward_workspace_size(D, L, N) bytes (20 N D L),
+ *          256-byte aligned; nothing in it needs to start at zero.
+ * L is a power of two, 16 <= L <= 16384 (HYENA_ERR_UNSUPPORTED above);
+ * 1 <= N <= HYENA_MAX_ORDER.  One launch: a group of threads owns a
+ * channel and walks its B sequences (the forward again, then the orders
+ * backwards), so dh and dbias need no atomics and are deterministic.
+ * Alignment: v, x_n, dy, dv, dx_n, H, dh 16 bytes; bias, dbias 4.  Outputs
+ * must not overlap each other, any input or the workspace. */
+HYENA_API size_t hyena_fftconv_backward_workspace_size(int D, int L, int N);
+HYENA_API hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x,
+                                                     const float* H, const float* bias,
+                                                     const void* dy, int B, int D, int L, int N,
+                                                     hyena_dtype_t io, void* dv, void* const* dx,
+                                                     float* dh, float* dbias, void* workspace,
+                                                     size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- 2-D */
 
 /* Implicit 2-D filters h [N][C][H][W] float32 (features and window as in

@@ -1,0 +1,218 @@
+// backward1d.cuh -- the backward pass of the single-CTA 1-D path (L <= 16384).
+//
+// The pages describe the forward only; its gradient follows from the chain
+// rule.  With c_n = h_n (*) z_{n-1} + b_n z_{n-1} and z_n = x_n c_n, and
+// g = dL/dz_n flowing back from g = dy at n = N:
+//     dx_n        = g * c_n
+//     e           = g * x_n                         (dL/dc_n)
+//     dh_n[s]    += sum_t e[t] z_{n-1}[t - s]       (summed over the batch)
+//     db_n       += sum_t e[t] z_{n-1}[t]  =  dh_n[0]
+//     dz_{n-1}    = corr(h_n, e) + b_n e,   corr(h, e)[u] = sum_{t>=u} h[t-u] e[t]
+// and dv = dz_0.  On the 2L-point grid (zero-padded, "Native
+// Multi-Dimensional Subquadratic Operators via Input Dependent Long
+// Convolutions", Handling Boundaries) both sums are correlations:
+//     DFT(dz_{n-1}) = (conj(H_n) + b_n) DFT(e)          (first L outputs)
+//     DFT(dh_n)     = sum_b DFT(e) conj(DFT(z_{n-1}))   (first L lags)
+//
+// One CTA group (T threads, the same FFT machinery and layouts as the fused
+// forward) owns one channel d and walks its B sequences:
+//   A. the forward again, saving Z_n = DFT(z_n) and c_{n+1} to the
+//      workspace in register order (each thread reads back what it wrote);
+//   B. for n = N..1: dx_n and e from g; E = DFT(e); accumulate E conj(Z)
+//      into the channel's dh spectrum (only this group touches it, so a
+//      plain read-modify-write); g = inverse of (conj(H_n) + b_n) E.
+// After the last sequence the group turns each accumulated spectrum into
+// dh_n (inverse real FFT, first L lags) and db_n = dh_n[0].
+#pragma once
+
+#include "fused1d.cuh"
+
+namespace hyena {
+
+struct Backward1dArgs {
+    const void* v;                 // [B][D][L] io
+    const void* x[kMaxOrder];      // x_1..x_N, [B][D][L] io
+    const void* dy;                // [B][D][L] io
+    const float2* H;               // [N][D][L] packed filter spectra
+    const float* bias;             // [N][D]
+    void* dv;                      // [B][D][L] io
+    void* dx[kMaxOrder];           // [B][D][L] io each
+    float* dh;                     // [N][D][L]
+    float* dbias;                  // [N][D]
+    float2* acc;                   // workspace [N][D][L]: accumulated dh spectra (packed)
+    float2* wz;                    // workspace [D][N][L]: Z_n in register order
+    float2* wc;                    // workspace [D][N][L/2]: c_{n+1} in register order
+    int B, D, N;
+};
+
+template <int LOG2M, typename IO>
+__global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS, Fft1d<LOG2M>::MIN_BLOCKS)
+backward1d_kernel(Backward1dArgs args)
+{
+    grid_dependency_begin();
+    using F = Fft1d<LOG2M>;
+    using IOP = IoPair<IO>;
+    using PT = typename IOP::T;
+    constexpr int M = F::M, E = F::E, T = F::T, RF = F::P::RF;
+    extern __shared__ __align__(16) float2 smem_dyn[];
+
+    const int g = threadIdx.x / T, t = threadIdx.x % T;
+    const int d_raw = blockIdx.x * F::G + g;
+    const bool active = d_raw < args.D;      // inactive groups compute but write nothing
+    const int d = active ? d_raw : args.D - 1;
+    const int D = args.D, N = args.N;
+    float2* sm = smem_dyn + g * F::SMEM_SEQ;
+    float2* stage = smem_dyn + F::G * F::SMEM_SEQ + g * F::STAGE_SEQ;
+    float2* wz = args.wz + (size_t)d * N * M;
+    float2* wc = args.wc + (size_t)d * N * (M / 2);
+    // index of io register i among the thread's E/2 io registers
+    auto io_slot = [](int i) { return (i / RF) * (RF / 2) + i % RF; };
+    // x_{n+1} (0-based n) with constant indices into the parameter array
+    auto x_of = [&](int n) {
+        const void* p = args.x[0];
+#pragma unroll
+        for (int i = 1; i < kMaxOrder; ++i)
+            if (i == n) p = args.x[i];
+        return reinterpret_cast<const PT*>(p);
+    };
+    // H_n into shared memory (into the exchange buffer at the largest size,
+    // once the forward FFT has finished with it); returns the staged row
+    auto stage_h_before = [&](int n) {
+        if constexpr (!F::H_IN_EXCHANGE)
+            cp_async_row(stage, args.H + ((size_t)n * D + d) * M, M * 8, t, T);
+    };
+    auto stage_h_after = [&](int n) -> const float2* {
+        if constexpr (F::H_IN_EXCHANGE) {
+            cp_async_row(sm, args.H + ((size_t)n * D + d) * M, M * 8, t, T);
+            cp_async_wait_all();
+            __syncthreads();
+            return sm;
+        } else {
+            cp_async_wait_all();
+            __syncthreads();
+            return stage;
+        }
+    };
+
+    float2 a[E];
+    for (int b = 0; b < args.B; ++b) {
+        const size_t seq = (size_t)b * D + d;
+        // ---------------------------------------------- A. forward again
+        {
+            const PT* vp = reinterpret_cast<const PT*>(args.v) + seq * (M / 2);
+            F::for_each_io(t, [&](int i, int m) { a[i] = IOP::load(vp + m); });
+        }
+        for (int n = 0; n < N; ++n) {
+            const float bias = __ldg(args.bias + n * D + d);
+            stage_h_before(n);
+            F::forward(a, sm, t);
+            if (active)
+                static_for<E>([&](auto ii) {
+                    constexpr int i = decltype(ii)::value;
+                    wz[(size_t)n * M + i * T + t] = a[i];
+                });
+            const float2* Hs = stage_h_after(n);
+            F::spectral(a, Hs, bias, t);
+            __syncthreads();                                  // H_n consumed
+            F::inverse(a, sm, t);
+            const PT* xp = x_of(n) + seq * (M / 2);
+            F::for_each_io(t, [&](int i, int m) {
+                if (active) wc[(size_t)n * (M / 2) + io_slot(i) * T + t] = a[i];
+                if (n + 1 < N) {
+                    const float2 xv = IOP::load(xp + m);
+                    a[i] = make_float2(a[i].x * xv.x, a[i].y * xv.y);
+                }
+            });
+        }
+        // ---------------------------------------------- B. backward
+        {
+            const PT* gp = reinterpret_cast<const PT*>(args.dy) + seq * (M / 2);
+            F::for_each_io(t, [&](int i, int m) { a[i] = IOP::load(gp + m); });
+        }
+        for (int n = N - 1; n >= 0; --n) {
+            const float bias = __ldg(args.bias + n * D + d);
+            {
+                // dx_n = g c_n, e = g x_n  (g in the io registers)
+                const PT* xp = x_of(n) + seq * (M / 2);
+                void* dxn = args.dx[0];
+#pragma unroll
+                for (int i = 1; i < kMaxOrder; ++i)
+                    if (i == n) dxn = args.dx[i];
+                PT* dxp = reinterpret_cast<PT*>(dxn) + seq * (M / 2);
+                F::for_each_io(t, [&](int i, int m) {
+                    const float2 c = wc[(size_t)n * (M / 2) + io_slot(i) * T + t];
+                    const float2 xv = IOP::load(xp + m);
+                    if (active) IOP::store(dxp + m, make_float2(a[i].x * c.x, a[i].y * c.y));
+                    a[i] = make_float2(a[i].x * xv.x, a[i].y * xv.y);
+                });
+            }
+            stage_h_before(n);
+            F::forward(a, sm, t);                            // a = DFT(e), packed
+            // dh spectrum: acc[k] (+)= E[k] conj(Z_{n-1}[k]) over the 2L-point bins
+            if (active) {
+                float2* acc = args.acc + ((size_t)n * D + d) * M;
+                const float2* zr = wz + (size_t)n * M;
+                const bool first = b == 0;
+                F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
+                    const float2 e1 = a[i1], e2 = a[i2];
+                    const float2 z1 = zr[i1 * T + t], z2 = zr[i2 * T + t];
+                    if (kind == 1) {
+                        // slot 0: bins 0 and M, both real
+                        const float2 p = make_float2((e1.x + e1.y) * (z1.x + z1.y),
+                                                     (e1.x - e1.y) * (z1.x - z1.y));
+                        acc[0] = first ? p : cadd(acc[0], p);
+                    } else {
+                        float2 E1, E2, Z1, Z2;
+                        split_pair(e1, e2, w, E1, E2);
+                        split_pair(z1, z2, w, Z1, Z2);
+                        const float2 p1 = cmulc(E1, Z1);
+                        acc[k] = first ? p1 : cadd(acc[k], p1);
+                        if (kind == 0) {
+                            const float2 p2 = cmulc(E2, Z2);
+                            acc[M - k] = first ? p2 : cadd(acc[M - k], p2);
+                        }
+                    }
+                });
+            }
+            const float2* Hs = stage_h_after(n);
+            F::template spectral<true>(a, Hs, bias, t);      // (conj(H_n) + b_n) E, re-packed
+            __syncthreads();                                  // H_n consumed
+            F::inverse(a, sm, t);                            // io registers: g = dz_{n-1}
+        }
+        if (active) {
+            PT* dvp = reinterpret_cast<PT*>(args.dv) + seq * (M / 2);
+            F::for_each_io(t, [&](int i, int m) { IOP::store(dvp + m, a[i]); });
+        }
+    }
+    // ------------------------------------------ dh_n and db_n of channel d
+    constexpr float s = 1.0f / (2.0f * (float)M);           // 1/P of the inverse DFT
+    for (int n = 0; n < N; ++n) {
+        const float2* acc = args.acc + ((size_t)n * D + d) * M;
+        F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
+            float2 z1, z2;
+            if (kind == 1) {
+                const float2 p = acc[0];
+                unsplit_pair(make_float2(p.x, 0.0f), make_float2(p.y, 0.0f), w, s, z1, z2);
+                a[i1] = z1;
+            } else if (kind == 2) {
+                const float2 y = acc[k];
+                unsplit_pair(y, y, w, s, z1, z2);
+                a[i1] = z1;
+            } else {
+                unsplit_pair(acc[k], acc[M - k], w, s, z1, z2);
+                a[i1] = z1;
+                a[i2] = z2;
+            }
+        });
+        F::inverse(a, sm, t);
+        if (active) {
+            float2* dhp = reinterpret_cast<float2*>(args.dh + ((size_t)n * D + d) * M);
+            F::for_each_io(t, [&](int i, int m) {
+                dhp[m] = a[i];
+                if (m == 0) args.dbias[n * D + d] = a[i].x;   // db_n = dh_n[0]
+            });
+        }
+    }
+}
+
+}  // namespace hyena

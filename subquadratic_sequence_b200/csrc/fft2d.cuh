@@ -46,26 +46,6 @@ struct Fft2dArgs {
     int n;                         // order handled by this launch
 };
 
-// The real split of one bin pair: X[k], X[M-k] from Z[k], Z[M-k].
-__device__ __forceinline__ void split_pair(float2 z1, float2 z2, float2 w, float2& X1, float2& X2)
-{
-    const float2 bc = cconj(z2);
-    const float2 S = cadd(z1, bc);
-    const float2 Tw = cmul(w, csub(z1, bc));
-    X1 = make_float2(0.5f * (S.x + Tw.y), 0.5f * (S.y - Tw.x));
-    X2 = make_float2(0.5f * (S.x - Tw.y), -0.5f * (S.y + Tw.x));
-}
-
-// The inverse re-pack of one bin pair (scale s): Z'[k], Z'[M-k] from Y[k], Y[M-k].
-__device__ __forceinline__ void unsplit_pair(float2 y1, float2 y2, float2 w, float s, float2& z1,
-                                             float2& z2)
-{
-    const float2 U = make_float2(y1.x + y2.x, y1.y - y2.y);                 // Y1 + conj Y2
-    const float2 V = cmulc(make_float2(y1.x - y2.x, y1.y + y2.y), w);        // conj(w)(Y1 - conj Y2)
-    z1 = make_float2(s * (U.x - V.y), s * (U.y + V.x));                     // U + i V
-    z2 = make_float2(s * (U.x + V.y), s * (V.x - U.y));                     // conj(U - i V)
-}
-
 template <int LOG2W>
 struct Fft2dRows {
     using F = Fft1d<LOG2W>;

@@ -74,6 +74,29 @@ struct Rfft1dArgs {
     int rows;
 };
 
+// The real split of one bin pair: the 2M-point spectrum bins X[k] and
+// X[M-k] of a real sequence from the M-point transform Z of its packed form
+// (Z[k], Z[M-k]); w = exp(-i pi k / M).
+__device__ __forceinline__ void split_pair(float2 z1, float2 z2, float2 w, float2& X1, float2& X2)
+{
+    const float2 bc = cconj(z2);
+    const float2 S = cadd(z1, bc);
+    const float2 Tw = cmul(w, csub(z1, bc));
+    X1 = make_float2(0.5f * (S.x + Tw.y), 0.5f * (S.y - Tw.x));
+    X2 = make_float2(0.5f * (S.x - Tw.y), -0.5f * (S.y + Tw.x));
+}
+
+// The inverse re-pack of one bin pair (scale s): the M-point inverse
+// transform input Z'[k], Z'[M-k] from the spectrum bins Y[k], Y[M-k].
+__device__ __forceinline__ void unsplit_pair(float2 y1, float2 y2, float2 w, float s, float2& z1,
+                                             float2& z2)
+{
+    const float2 U = make_float2(y1.x + y2.x, y1.y - y2.y);                 // Y1 + conj Y2
+    const float2 V = cmulc(make_float2(y1.x - y2.x, y1.y + y2.y), w);        // conj(w)(Y1 - conj Y2)
+    z1 = make_float2(s * (U.x - V.y), s * (U.y + V.x));                     // U + i V
+    z2 = make_float2(s * (U.x + V.y), s * (V.x - U.y));                     // conj(U - i V)
+}
+
 // Packed spectrum of a real length-L filter zero-padded to 2L: M = L
 // complex slots; slot k (1 <= k < L) holds DFT bin k, slot 0 holds
 // (bin 0, bin L), both real.  Rows are L * 8 bytes, so 16-byte aligned.
@@ -257,9 +280,12 @@ struct Fft1d {
     }
 
     // Spectral step on the RL folded layout for one order; Hs is the
-    // packed spectrum row staged in shared memory.
+    // packed spectrum row staged in shared memory.  CONJ: multiply by
+    // conj(H) + b instead (the adjoint, used by the backward pass).
+    template <bool CONJ = false>
     static __device__ __forceinline__ void spectral(float2* a, const float2* Hs, float bias, int t)
     {
+        auto hv = [&](int k) { return CONJ ? cconj(Hs[k]) : Hs[k]; };
         constexpr int R = P::RL, NCOL = M / R;
         static_for<E / (2 * R)>([&](auto cc) {
             constexpr int c = decltype(cc)::value;
@@ -277,7 +303,7 @@ struct Fft1d {
                     const int k = j0 + r * NCOL + __float2int_rz(dep);
                     float2 w = mul_w64<r * 32 / R, -1>(wb);
                     w.x += dep;
-                    pair(a0[r], a1[R - 1 - r], Hs[k], Hs[M - k], w, bias);
+                    pair(a0[r], a1[R - 1 - r], hv(k), hv(M - k), w, bias);
                     dep = zero_after(a0[r].x);
                 });
             } else {
@@ -293,12 +319,12 @@ struct Fft1d {
                 }
                 static_for<R / 2 - 1>([&](auto rr) {
                     constexpr int r = decltype(rr)::value + 1;
-                    pair(a0[r], a0[R - r], Hs[r * NCOL], Hs[M - r * NCOL],
+                    pair(a0[r], a0[R - r], hv(r * NCOL), hv(M - r * NCOL),
                          mul_w64<r * 32 / R, -1>(make_float2(1.0f, 0.0f)), bias);
                 });
                 {
                     float2 z1 = a0[R / 2], z2 = a0[R / 2];
-                    const float2 hm = Hs[M / 2];
+                    const float2 hm = hv(M / 2);
                     pair(z1, z2, hm, hm, make_float2(0.0f, -1.0f), bias);
                     a0[R / 2] = z1;
                 }
@@ -307,7 +333,7 @@ struct Fft1d {
                 static_for<R / 2>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
                     const int k = NCOL / 2 + r * NCOL;
-                    pair(a1[r], a1[R - 1 - r], Hs[k], Hs[M - k], mul_w64<r * 32 / R, -1>(wb), bias);
+                    pair(a1[r], a1[R - 1 - r], hv(k), hv(M - k), mul_w64<r * 32 / R, -1>(wb), bias);
                 });
             }
         });

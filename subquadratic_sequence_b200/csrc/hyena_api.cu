@@ -257,6 +257,83 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
                             : dispatch_fourstep_f32(log2m, a, N, scratch, st);
 }
 
+size_t hyena_fftconv_backward_workspace_size(int D, int L, int N)
+{
+    int log2m = 0;
+    if (D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2Fused, &log2m) != HYENA_OK)
+        return (size_t)-1;
+    const size_t spec = sizeof(float2) * (size_t)N * D * L;
+    return round_up(spec, 256) * 2 + round_up(spec / 2, 256);   // acc, wz, wc
+}
+
+hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, const float* H,
+                                           const float* bias, const void* dy, int B, int D, int L,
+                                           int N, hyena_dtype_t io, void* dv, void* const* dx,
+                                           float* dh, float* dbias, void* workspace, size_t ws_bytes,
+                                           void* stream)
+{
+    if (!v || !x || !H || !bias || !dy || !dv || !dx || !dh || !dbias) return HYENA_ERR_INVALID_ARG;
+    if (B < 1 || D < 1 || N < 1 || L < 1) return HYENA_ERR_INVALID_ARG;
+    if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
+    int log2m = 0;
+    hyena_status_t s = check_len(L, kMaxLog2Fused, &log2m);
+    if (s != HYENA_OK) return s;
+    if ((long)B * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    for (int n = 0; n < N; ++n)
+        if (!x[n] || !dx[n] || !aligned(x[n], 16) || !aligned(dx[n], 16)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(v, 16) || !aligned(dy, 16) || !aligned(dv, 16) || !aligned(H, 16) || !aligned(dh, 16) ||
+        !aligned(bias, 4) || !aligned(dbias, 4))
+        return HYENA_ERR_INVALID_ARG;
+    const size_t need = hyena_fftconv_backward_workspace_size(D, L, N);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+
+    // every output against every input, the other outputs and the workspace
+    const size_t act = (size_t)B * D * L * io_bytes(io);
+    struct Range { const void* p; size_t n; };
+    Range in[kMaxOrder + 5], out[kMaxOrder + 3];
+    int ni = 0, no = 0;
+    in[ni++] = {v, act};
+    in[ni++] = {dy, act};
+    in[ni++] = {H, spectrum_bytes(N, D, L)};
+    in[ni++] = {bias, sizeof(float) * N * D};
+    in[ni++] = {workspace, need};
+    for (int n = 0; n < N; ++n) in[ni++] = {x[n], act};
+    out[no++] = {dv, act};
+    out[no++] = {dh, sizeof(float) * (size_t)N * D * L};
+    out[no++] = {dbias, sizeof(float) * N * D};
+    for (int n = 0; n < N; ++n) out[no++] = {dx[n], act};
+    for (int o = 0; o < no; ++o) {
+        for (int i = 0; i < ni; ++i)
+            if (overlap(out[o].p, out[o].n, in[i].p, in[i].n)) return HYENA_ERR_INVALID_ARG;
+        for (int p = o + 1; p < no; ++p)
+            if (overlap(out[o].p, out[o].n, out[p].p, out[p].n)) return HYENA_ERR_INVALID_ARG;
+    }
+
+    const size_t spec = sizeof(float2) * (size_t)N * D * L;
+    char* ws = static_cast<char*>(workspace);
+    Backward1dArgs a;
+    a.v = v;
+    a.dy = dy;
+    for (int n = 0; n < kMaxOrder; ++n) {
+        a.x[n] = n < N ? x[n] : nullptr;
+        a.dx[n] = n < N ? dx[n] : nullptr;
+    }
+    a.H = reinterpret_cast<const float2*>(H);
+    a.bias = bias;
+    a.dv = dv;
+    a.dh = dh;
+    a.dbias = dbias;
+    a.acc = reinterpret_cast<float2*>(ws);
+    a.wz = reinterpret_cast<float2*>(ws + round_up(spec, 256));
+    a.wc = reinterpret_cast<float2*>(ws + 2 * round_up(spec, 256));
+    a.B = B;
+    a.D = D;
+    a.N = N;
+    cudaStream_t st = (cudaStream_t)stream;
+    return io == HYENA_BF16 ? dispatch_backward_bf16(log2m, a, st) : dispatch_backward_f32(log2m, a, st);
+}
+
 // ------------------------------------------------------------------ 2-D
 
 size_t hyena_fftconv2d_workspace_size(int B, int C, int H, int W, int N, hyena_dtype_t io,

@@ -1,0 +1,37 @@
+// k_backward1d.cuh -- launchers of the 1-D backward pass, included by one
+// .cu file per activation type.
+#pragma once
+
+#include "backward1d.cuh"
+#include "launch.cuh"
+
+namespace hyena {
+
+template <int LOG2M, typename IO>
+hyena_status_t launch_backward(const Backward1dArgs& a, cudaStream_t st)
+{
+    using F = Fft1d<LOG2M>;
+    return launch(backward1d_kernel<LOG2M, IO>, (unsigned)((a.D + F::G - 1) / F::G), F::THREADS,
+                  F::SMEM_BYTES, st, a);
+}
+
+template <typename IO>
+hyena_status_t dispatch_backward(int log2m, const Backward1dArgs& a, cudaStream_t st)
+{
+    switch (log2m) {
+    case 4: return launch_backward<4, IO>(a, st);
+    case 5: return launch_backward<5, IO>(a, st);
+    case 6: return launch_backward<6, IO>(a, st);
+    case 7: return launch_backward<7, IO>(a, st);
+    case 8: return launch_backward<8, IO>(a, st);
+    case 9: return launch_backward<9, IO>(a, st);
+    case 10: return launch_backward<10, IO>(a, st);
+    case 11: return launch_backward<11, IO>(a, st);
+    case 12: return launch_backward<12, IO>(a, st);
+    case 13: return launch_backward<13, IO>(a, st);
+    case 14: return launch_backward<14, IO>(a, st);
+    default: return HYENA_ERR_UNSUPPORTED;
+    }
+}
+
+}  // namespace hyena

@@ -56,6 +56,9 @@ def _load() -> ctypes.CDLL:
                                         sz, vp], i),
         "hyena_fftconv_gate_forward_noalloc": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp,
                                                 vp], i),
+        "hyena_fftconv_backward_workspace_size": ([i, i, i], sz),
+        "hyena_fftconv_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp,
+                                         ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_filter_rfft2d": ([vp, i, i, i, i, vp, vp], i),
         "hyena_fftconv2d_workspace_size": ([i, i, i, i, i, i, i], sz),
         "hyena_fftconv2d_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
@@ -213,6 +216,39 @@ def hyena_fftconv_gate_forward_noalloc(v: torch.Tensor, xs, bias: torch.Tensor, 
 
 
 # ------------------------------------------------------------------ 2-D
+
+def hyena_fftconv_backward_workspace_size(D: int, L: int, N: int) -> int:
+    n = LIB.hyena_fftconv_backward_workspace_size(D, L, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv_backward_workspace_size", HYENA_ERR_INVALID_ARG, "invalid sizes")
+    return n
+
+
+def hyena_fftconv_gate_backward(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor,
+                                dy: torch.Tensor, *, workspace=None, stream=None):
+    """Gradients of a loss with dL/dy = dy through the order-N forward:
+    returns (dv [B][D][L], [dx_1..dx_N], dh [N][D][L] float32, dbias [N][D]
+    float32); v, x_n, dy float32 or bf16, H the packed spectra, L <= 16384."""
+    B, D, L = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty((N, D, L), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, D), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(hyena_fftconv_backward_workspace_size(D, L, N), device=v.device,
+                                dtype=torch.uint8)
+    _check("hyena_fftconv_gate_backward", LIB.hyena_fftconv_gate_backward(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+        B, D, L, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+        ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db
+
 
 def hyena_filter_rfft2d(h: torch.Tensor, *, out=None, stream=None):
     """Packed 2-D spectra [N][C][2H][W] complex64 of the filters h

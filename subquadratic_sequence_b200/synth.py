@@ -120,3 +120,12 @@ def make_inputs(wl: Workload) -> dict:
     W1, W2, W3, Wout = _weights(rng, n_in, WIDTH, wl.N * wl.D)
     alpha = np.linspace(0.3, 1.5, wl.D).astype(np.float32)
     return dict(v=v, x=x, b=b, W1=W1, W2=W2, W3=W3, Wout=Wout, alpha=alpha)
+
+
+def make_output_grad(wl: Workload) -> np.ndarray:
+    """The upstream gradient dL/dy for the backward pass: i.i.d. N(0, 1) of
+    the activation shape (bf16-rounded for bf16 storage), from its own
+    stream (seed + 1) so the forward inputs are unchanged."""
+    rng = np.random.default_rng(wl.seed + 1)
+    shape = (wl.B, wl.D, wl.L) if wl.kind == "1d" else (wl.B, wl.D, wl.H, wl.W)
+    return _activation(rng, shape, wl.io)

@@ -120,6 +120,46 @@ def test_forward_rejects_bad_arguments(lib):
     assert fwd(lib, H=None, h=P(3), ws=P(5), wsb=1 << 20) == INVALID
 
 
+def bwd(lib, v=P(0), xs=(P(1), P(2)), H=P(3), bias=P(4), dy=P(5), B=2, D=3, L=64, N=None,
+        io=F32, dv=P(6), dxs=(P(7), P(8)), dh=P(9), db=P(10), ws=P(11), wsb=1 << 24):
+    N = len(xs) if N is None else N
+    xa = (ctypes.c_void_p * max(len(xs), 1))(*[x.value if x is not None else None for x in xs])
+    da = (ctypes.c_void_p * max(len(dxs), 1))(*[x.value if x is not None else None for x in dxs])
+    return lib.hyena_fftconv_gate_backward(v, xa, H, bias, dy, B, D, L, N, io, dv, da, dh, db,
+                                           ws, wsb, None)
+
+
+def test_backward_rejects_bad_arguments(lib):
+    lib.hyena_fftconv_backward_workspace_size.restype = ctypes.c_size_t
+    lib.hyena_fftconv_backward_workspace_size.argtypes = [ctypes.c_int] * 3
+    need = lib.hyena_fftconv_backward_workspace_size(3, 64, 2)
+    assert need >= 20 * 2 * 3 * 64
+    assert lib.hyena_fftconv_backward_workspace_size(3, 1 << 15, 2) == ctypes.c_size_t(-1).value
+    assert lib.hyena_fftconv_backward_workspace_size(0, 64, 2) == ctypes.c_size_t(-1).value
+    for k in ("v", "H", "bias", "dy", "dv", "dh", "db"):
+        assert bwd(lib, **{k: None}) == INVALID, k
+    assert bwd(lib, xs=(P(1), None)) == INVALID
+    assert bwd(lib, dxs=(P(7), None)) == INVALID
+    assert bwd(lib, B=0) == INVALID
+    assert bwd(lib, io=3) == INVALID
+    # only the single-CTA lengths
+    assert bwd(lib, L=1 << 15) == UNSUPPORTED
+    assert bwd(lib, L=100) == UNSUPPORTED
+    # workspace: missing, short, misaligned
+    assert bwd(lib, ws=None) == WORKSPACE
+    assert bwd(lib, wsb=need - 1) == WORKSPACE
+    assert bwd(lib, ws=ctypes.c_void_p(A + 11 * BIG + 16)) == WORKSPACE
+    # misalignment of an output
+    assert bwd(lib, dh=ctypes.c_void_p(A + 9 * BIG + 4)) == INVALID
+    assert bwd(lib, dxs=(P(7), ctypes.c_void_p(A + 8 * BIG + 8))) == INVALID
+    # outputs overlapping inputs, each other, the workspace
+    assert bwd(lib, dv=P(0)) == INVALID
+    assert bwd(lib, dh=P(3)) == INVALID
+    assert bwd(lib, db=ctypes.c_void_p(A + 6 * BIG + 64)) == INVALID
+    assert bwd(lib, dxs=(P(7), P(7))) == INVALID
+    assert bwd(lib, dxs=(P(11), P(8))) == INVALID
+
+
 def test_filter_rfft_rejects_bad_arguments(lib):
     r = lib.hyena_filter_rfft
     assert r(None, 2, 3, 64, P(1), None, 0, None) == INVALID

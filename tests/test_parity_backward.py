@@ -1,0 +1,100 @@
+"""GPU parity of the 1-D backward pass against the float64 oracle (-m gpu).
+
+The oracle's backward is pinned to finite differences of its forward
+(tests/test_oracle_backward_pins.py).  Tolerances: dv and dx_n as the
+forward's output (1e-4 of the maximum for float32 storage, 2e-2 for bf16);
+dh and dbias, accumulated in float32 from float32 intermediates, 1e-4 of
+their maximum for both storage types.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from subquadratic_sequence_b200 import synth
+from tests.gpu_helpers import assert_close, dev, host, random_problem, rel_max_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hy():
+    from subquadratic_sequence_b200 import hyena
+    assert torch.cuda.is_available()
+    return hyena
+
+
+def filters(wl, seed):
+    """Seeded decaying filters (float32), the shape the filter network gives."""
+    r = np.random.default_rng(seed)
+    decay = np.exp(-np.arange(wl.L) * np.linspace(0.3, 1.5, wl.D)[:, None] / 64.0)
+    return (r.standard_normal((wl.N, wl.D, wl.L)) * 0.2 * decay).astype(np.float32)
+
+
+def run(hy, wl, inp, h32, dy):
+    io = wl.io
+    H = hy.hyena_filter_rfft(dev(h32))
+    dv, dxs, dh, db = hy.hyena_fftconv_gate_backward(
+        dev(inp["v"], io), [dev(x, io) for x in inp["x"]], dev(inp["b"]), H, dev(dy, io))
+    torch.cuda.synchronize()
+    return host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+
+
+def check(got, ref, io, name):
+    dv, dx, dh, db = got
+    rdv, rdx, rdh, rdb = ref
+    assert_close(dv, rdv, io, f"{name} dv")
+    assert_close(dx, rdx, io, f"{name} dx")
+    assert rel_max_err(dh, rdh) <= 1e-4, f"{name} dh {rel_max_err(dh, rdh):.3e}"
+    assert rel_max_err(db, rdb) <= 1e-4, f"{name} db {rel_max_err(db, rdb):.3e}"
+
+
+CASES = [
+    (1, 1, 16, 1, "f32"), (2, 3, 64, 2, "f32"), (3, 5, 256, 3, "f32"), (2, 7, 1024, 2, "bf16"),
+    (2, 13, 2048, 2, "f32"),        # 13 channels: a partly idle CTA at L = 2048 (6 per CTA)
+    (1, 4, 4096, 4, "f32"), (2, 3, 8192, 2, "f32"), (1, 2, 16384, 2, "f32"), (3, 2, 512, 16, "f32"),
+    (8, 6, 2048, 2, "bf16"),
+]
+
+
+@pytest.mark.parametrize("B,D,L,N,io", CASES)
+def test_backward_matches_oracle(hy, B, D, L, N, io):
+    wl, inp = random_problem(B, D, L, N, seed=300 + L + N, io=io)
+    h32 = filters(wl, seed=L + N)
+    dy = synth.make_output_grad(wl)
+    got = run(hy, wl, inp, h32, dy)
+    ref = oracle.hyena_backward(inp["v"], np.stack(inp["x"]), h32, inp["b"], dy)
+    check(got, ref, io, f"B{B} D{D} L{L} N{N} {io}")
+
+
+def test_backward_c1_full_size(hy):
+    """Order-2, B=8, D=768, L=2048, bf16 storage: every output compared."""
+    wl = synth.WORKLOADS["c1"]
+    inp = synth.make_inputs(wl)
+    h32 = filters(wl, seed=1)
+    dy = synth.make_output_grad(wl)
+    got = run(hy, wl, inp, h32, dy)
+    ref = oracle.hyena_backward(inp["v"], np.stack(inp["x"]), h32, inp["b"], dy)
+    check(got, ref, wl.io, "c1")
+
+
+def test_backward_is_deterministic(hy):
+    wl, inp = random_problem(4, 6, 1024, 2, seed=9)
+    h32 = filters(wl, seed=9)
+    dy = synth.make_output_grad(wl)
+    a = run(hy, wl, inp, h32, dy)
+    b = run(hy, wl, inp, h32, dy)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_backward_of_delta_filters_is_the_closed_form(hy):
+    # h = delta_0, N = 1: dv = dy x (1+b), dx = dy (1+b) v
+    wl, inp = random_problem(2, 3, 512, 1, seed=4)
+    h32 = np.zeros((1, 3, 512), np.float32)
+    h32[:, :, 0] = 1.0
+    dy = synth.make_output_grad(wl)
+    dv, dx, _, _ = run(hy, wl, inp, h32, dy)
+    gain = (1.0 + inp["b"][0].astype(np.float64))[None, :, None]
+    assert rel_max_err(dv, dy * inp["x"][0] * gain) <= 1e-5
+    assert rel_max_err(dx[0], dy * gain * inp["v"]) <= 1e-5
