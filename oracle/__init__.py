@@ -60,6 +60,7 @@ def _load():
         "oracle_hyena_forward": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
         "oracle_hyena_forward_2d": [dp, dp, dp, dp, l, l, l, l, l, i, i, dp],
         "oracle_hyena_backward": [dp, dp, dp, dp, dp, l, l, l, l, i, i, dp, dp, dp, dp],
+        "oracle_filter_gen_film": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, d, i, dp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -222,3 +223,32 @@ def hyena_backward(v, x, h, bias, dy, route="fft", threads=None):
                                        _ptr(dv), _ptr(dx), _ptr(dh), _ptr(db))
     _check(rc, "oracle_hyena_backward")
     return dv, dx, dh, db
+
+
+def filter_gen_film(W1, W2, W3, Wout, omega, gamma, beta, window, gaussian, N, D, L, n_bands=8,
+                    width=64, decay_div=64.0, threads=None) -> np.ndarray:
+    """Per-sample (input-dependent) filters h [B][N][D][L]: the sine layers
+    modulated by the sample's FiLM vectors, a_l = sin(omega_l (gamma_bl
+    W_l a_(l-1) + beta_bl)); omega [3][width], gamma and beta [B][3][width];
+    window [D] is alpha (exponential decay) or sigma (Gaussian)."""
+    W1, W2, W3, Wout, omega, gamma, beta, window = map(
+        _f64, (W1, W2, W3, Wout, omega, gamma, beta, window))
+    B = gamma.shape[0]
+    assert omega.shape == (3, width) and gamma.shape == (B, 3, width) and beta.shape == gamma.shape
+    assert window.shape == (D,)
+    h = np.empty((B, N, D, L))
+    rc = _load().oracle_filter_gen_film(_ptr(W1), _ptr(W2), _ptr(W3), _ptr(Wout), _ptr(omega),
+                                        _ptr(gamma), _ptr(beta), _ptr(window), int(bool(gaussian)),
+                                        B, N, D, L, n_bands, width, float(decay_div),
+                                        threads or default_threads(), _ptr(h))
+    _check(rc, "oracle_filter_gen_film")
+    return h
+
+
+def hyena_forward_per_sample(v, x, h, bias, route="fft", threads=None) -> np.ndarray:
+    """The forward with a filter set per sample, h [B][N][D][L]: the
+    recurrence of :func:`hyena_forward` applied to each sample with its own
+    filters."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    return np.concatenate([hyena_forward(v[b:b + 1], x[:, b:b + 1], h[b], bias, route, threads)
+                           for b in range(v.shape[0])])

@@ -165,6 +165,111 @@ int oracle_filter_gen(const double *W1, const double *W2, const double *W3,
     return st;
 }
 
+/* ------------------------------------------------------------------ */
+/* Input-dependent filters ("Native Multi-Dimensional Subquadratic       */
+/* Operators via Input Dependent Long Convolutions": Input-Dependent     */
+/* Kernels via Registers and FiLM; Kernel Parameterization).             */
+/* ------------------------------------------------------------------ */
+/*
+ * Per sample b the sine layers are modulated feature-wise (FiLM) by the
+ * sample's control vectors, and each hidden unit has its own frequency:
+ *     a_l = sin(omega_l * (gamma_{b,l} * (W_l a_{l-1}) + beta_{b,l})),
+ * l = 1..3, then o = Wout a_3; the filter is o times a window: the
+ * exponential decay exp(-alpha_d t L / div) of the shared filters, or the
+ * Gaussian exp(-t^2 / (2 sigma_d^2)), t = i/L.  The control vectors come
+ * from the sample (the pages derive them from register tokens); here they
+ * are inputs.  omega = 1, gamma = 1, beta = 0 with the exponential window
+ * is the shared filter of oracle_filter_gen.
+ */
+typedef struct {
+    const double *W1, *W2, *W3, *Wout, *omega, *gamma, *beta, *win;
+    int gaussian, B, N, D, L, n_bands, width;
+    double decay_div;
+    double *h;
+    int i0, i1;
+    int status;
+} fgf_job;
+
+/* a[j] = sin(om[j] * (g[j] * a[j] + be[j])) */
+static void film_sin(double *a, int width, const double *om, const double *g, const double *be)
+{
+    for (int j = 0; j < width; ++j) a[j] = sin(om[j] * (g[j] * a[j] + be[j]));
+}
+
+static void *filter_gen_film_worker(void *arg)
+{
+    fgf_job *j = (fgf_job *)arg;
+    const int n_in = 1 + 2 * j->n_bands, w = j->width, n_out = j->N * j->D;
+    double *phi = malloc(sizeof(double) * n_in);
+    double *a1 = malloc(sizeof(double) * w), *a2 = malloc(sizeof(double) * w);
+    double *a3 = malloc(sizeof(double) * w), *o = malloc(sizeof(double) * n_out);
+    if (!phi || !a1 || !a2 || !a3 || !o) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (int b = 0; b < j->B; ++b) {
+        const double *g = j->gamma + (long)b * 3 * w, *be = j->beta + (long)b * 3 * w;
+        for (int i = j->i0; i < j->i1; ++i) {
+            const double t = (double)i / (double)j->L;
+            phi[0] = t;
+            for (int k = 1; k <= j->n_bands; ++k) {
+                phi[2 * k - 1] = sin(2.0 * ORACLE_PI * k * t);
+                phi[2 * k] = cos(2.0 * ORACLE_PI * k * t);
+            }
+            matvec(j->W1, w, n_in, phi, a1);
+            film_sin(a1, w, j->omega, g, be);
+            matvec(j->W2, w, w, a1, a2);
+            film_sin(a2, w, j->omega + w, g + w, be + w);
+            matvec(j->W3, w, w, a2, a3);
+            film_sin(a3, w, j->omega + 2 * w, g + 2 * w, be + 2 * w);
+            matvec(j->Wout, n_out, w, a3, o);
+            for (int n = 0; n < j->N; ++n)
+                for (int d = 0; d < j->D; ++d) {
+                    const double window =
+                        j->gaussian ? exp(-t * t / (2.0 * j->win[d] * j->win[d]))
+                                    : exp(-j->win[d] * t * (double)j->L / j->decay_div);
+                    j->h[(((long)b * j->N + n) * j->D + d) * j->L + i] = o[n * j->D + d] * window;
+                }
+        }
+    }
+    j->status = ORACLE_OK;
+done:
+    free(phi); free(a1); free(a2); free(a3); free(o);
+    return NULL;
+}
+
+/* h[B][N][D][L]: per-sample filters.  omega [3][width], gamma and beta
+ * [B][3][width]; win [D] is alpha (gaussian = 0) or sigma (gaussian = 1). */
+int oracle_filter_gen_film(const double *W1, const double *W2, const double *W3,
+                           const double *Wout, const double *omega, const double *gamma,
+                           const double *beta, const double *win, int gaussian, int B, int N,
+                           int D, int L, int n_bands, int width, double decay_div,
+                           int nthreads, double *h)
+{
+    if (!W1 || !W2 || !W3 || !Wout || !omega || !gamma || !beta || !win || !h || B < 1 ||
+        N < 1 || D < 1 || L < 1 || n_bands < 0 || width < 1 || !(decay_div > 0.0))
+        return ORACLE_EBADARG;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > L) nthreads = L;
+    fgf_job *jobs = calloc(nthreads, sizeof(fgf_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        fgf_job j = {W1, W2, W3, Wout, omega, gamma, beta, win, gaussian, B, N, D, L, n_bands,
+                     width, decay_div, h, (int)((long)L * k / nthreads),
+                     (int)((long)L * (k + 1) / nthreads), 0};
+        jobs[k] = j;
+        pthread_create(&tid[k], NULL, filter_gen_film_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}
+
 typedef struct {
     const double *W1, *W2, *W3, *Wout, *alpha;
     int N, C, H, W, n_bands, width;

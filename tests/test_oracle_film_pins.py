@@ -1,0 +1,107 @@
+"""Pins of the oracle's input-dependent filters (FiLM-modulated sine layers,
+per-unit frequencies, Gaussian window) and of its per-sample forward.
+
+Each test ties the oracle to something outside the routine under test: the
+separately pinned shared-filter generator and forward, or an identity of the
+sine (sin(x + pi) = -sin(x), sin(c * x / c) = sin(x)) that fails if FiLM
+modulates the wrong layer, the wrong side of the product, or a sample's
+filters leak into another sample's.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+W, N, D, L = 64, 2, 3, 48
+
+
+def net(seed=0):
+    r = np.random.default_rng(seed)
+    return dict(W1=r.standard_normal((W, 17)) / np.sqrt(17), W2=r.standard_normal((W, W)) / 8,
+                W3=r.standard_normal((W, W)) / 8, Wout=r.standard_normal((N * D, W)) / 8)
+
+
+def film(n, omega, gamma, beta, window, gaussian=False):
+    return oracle.filter_gen_film(n["W1"], n["W2"], n["W3"], n["Wout"], omega, gamma, beta, window,
+                                  gaussian, N, D, L)
+
+
+ALPHA = np.linspace(0.3, 1.5, D)
+
+
+def test_identity_modulation_is_the_shared_filter():
+    n = net()
+    B = 3
+    h = film(n, np.ones((3, W)), np.ones((B, 3, W)), np.zeros((B, 3, W)), ALPHA)
+    ref = oracle.filter_gen(n["W1"], n["W2"], n["W3"], n["Wout"], ALPHA, N, D, L)
+    for b in range(B):
+        assert np.array_equal(h[b], ref)
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2])
+def test_gamma_scales_the_pre_activation_of_its_layer(layer):
+    # gamma_l = c is the same as W_l scaled by c
+    n = net(1)
+    c = 1.7
+    g = np.ones((1, 3, W))
+    g[0, layer] = c
+    a = film(n, np.ones((3, W)), g, np.zeros((1, 3, W)), ALPHA)
+    n2 = dict(n)
+    key = ("W1", "W2", "W3")[layer]
+    n2[key] = n[key] * c
+    b = film(n2, np.ones((3, W)), np.ones((1, 3, W)), np.zeros((1, 3, W)), ALPHA)
+    assert np.max(np.abs(a - b)) < 1e-12 * np.max(np.abs(b))
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2])
+def test_beta_pi_flips_the_sign_of_the_filter(layer):
+    # sin(x + pi) = -sin(x), and every later layer is odd in its input
+    n = net(2)
+    be = np.zeros((1, 3, W))
+    be[0, layer] = np.pi
+    a = film(n, np.ones((3, W)), np.ones((1, 3, W)), be, ALPHA)
+    b = film(n, np.ones((3, W)), np.ones((1, 3, W)), np.zeros((1, 3, W)), ALPHA)
+    assert np.max(np.abs(a + b)) < 1e-12 * np.max(np.abs(b))
+
+
+def test_omega_and_gamma_cancel():
+    # sin(c * (x / c)) = sin(x), per unit
+    n = net(3)
+    om = np.random.default_rng(4).uniform(0.5, 3.0, (3, W))
+    a = film(n, om, 1.0 / om[None], np.zeros((1, 3, W)), ALPHA)
+    b = film(n, np.ones((3, W)), np.ones((1, 3, W)), np.zeros((1, 3, W)), ALPHA)
+    assert np.max(np.abs(a - b)) < 1e-12 * np.max(np.abs(b))
+
+
+def test_gaussian_window_ratio():
+    # the two windows differ only in the window: the ratio of the filters is
+    # exp(-t^2 / (2 sigma^2)) / exp(-alpha t L / 64) at every position
+    n = net(5)
+    sigma = np.array([0.1, 0.25, 0.6])
+    r = np.random.default_rng(6)
+    g, be = r.uniform(0.5, 1.5, (1, 3, W)), r.normal(0, 0.3, (1, 3, W))
+    hg = film(n, np.ones((3, W)), g, be, sigma, gaussian=True)
+    he = film(n, np.ones((3, W)), g, be, ALPHA)
+    t = np.arange(L) / L
+    want = np.exp(-t[None, :] ** 2 / (2 * sigma[:, None] ** 2)) / np.exp(-ALPHA[:, None] * t[None, :] * L / 64.0)
+    np.testing.assert_allclose(hg[0], he[0] * want[None], rtol=1e-12, atol=1e-300)
+
+
+def test_samples_do_not_mix():
+    n = net(7)
+    r = np.random.default_rng(8)
+    g, be = r.uniform(0.5, 1.5, (3, 3, W)), r.normal(0, 0.3, (3, 3, W))
+    h = film(n, np.ones((3, W)), g, be, ALPHA)
+    perm = [2, 0, 1]
+    hp = film(n, np.ones((3, W)), g[perm], be[perm], ALPHA)
+    assert np.array_equal(hp, h[perm])
+    assert np.max(np.abs(h[0] - h[1])) > 1e-3
+
+
+def test_per_sample_forward_with_shared_filters_is_the_forward():
+    r = np.random.default_rng(9)
+    B = 3
+    v, x = r.standard_normal((B, D, L)), r.standard_normal((N, B, D, L))
+    h, bias = r.standard_normal((N, D, L)) * 0.3, r.standard_normal((N, D))
+    hp = np.broadcast_to(h, (B, N, D, L))
+    assert np.array_equal(oracle.hyena_forward_per_sample(v, x, hp, bias), oracle.hyena_forward(v, x, h, bias))
