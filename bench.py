@@ -48,11 +48,15 @@ def describe(wl: synth.Workload) -> dict:
                 "filters": f"implicit FFN over (y/H, x/W) (3 sine layers of width {synth.WIDTH}, "
                            f"{synth.N_BANDS} bands per axis) x separable decay, regenerated every step",
                 "l2": "flushed (256 MB write) before every timed step"}
+    filters = (f"implicit FFN (3 sine layers of width {synth.WIDTH}, {synth.N_BANDS} bands) "
+               "x exponential decay, regenerated every step")
+    if wl.film:
+        filters = (f"input-dependent: a filter set per sample, the {synth.WIDTH}-wide sine layers "
+                   "FiLM-modulated per sample, first layer at frequencies 1/2/4/8, Gaussian window; "
+                   "B*N*D filters and spectra regenerated every step")
     return {"workload": f"{wl.name}: order-{wl.N} Hyena 1-D operator, B={wl.B}, D={wl.D}, "
                         f"L={wl.L}, {wl.io} storage, fp32 compute",
-            "N": wl.N, "B": wl.B, "D": wl.D, "L": wl.L, "io": wl.io,
-            "filters": f"implicit FFN (3 sine layers of width {synth.WIDTH}, {synth.N_BANDS} bands) "
-                       "x exponential decay, regenerated every step",
+            "N": wl.N, "B": wl.B, "D": wl.D, "L": wl.L, "io": wl.io, "filters": filters,
             "l2": "flushed (256 MB write) before every timed step"}
 
 
@@ -61,7 +65,8 @@ def alg_bytes_forward(wl: synth.Workload) -> int:
     N*D packed spectra (L complex64 slots each; 2H x W for the 2-D grid)."""
     if wl.kind == "2d":
         return (wl.N + 2) * wl.positions * wl.io_bytes + wl.N * wl.D * 2 * wl.H * wl.W * 8
-    return (wl.N + 2) * wl.B * wl.D * wl.L * wl.io_bytes + wl.N * wl.D * wl.L * 8
+    sets = wl.B if wl.film else 1          # filter spectra per sample, or shared by the batch
+    return (wl.N + 2) * wl.B * wl.D * wl.L * wl.io_bytes + sets * wl.N * wl.D * wl.L * 8
 
 
 def alg_bytes_backward(wl: synth.Workload) -> int:
@@ -92,7 +97,8 @@ def launches_forward(wl: synth.Workload) -> int:
 def launches_rfft(wl: synth.Workload) -> int:
     if wl.kind == "2d":
         return 2
-    return waves(wl.N * wl.D, wl.L) * 2 if long_path(wl) else 1
+    rows = wl.N * wl.D * (wl.B if wl.film else 1)
+    return waves(rows, wl.L) * 2 if long_path(wl) else 1
 
 
 def launches_filter_gen(wl: synth.Workload) -> int:
@@ -289,6 +295,25 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
                                       width=synth.WIDTH, decay_div=synth.DECAY_DIV, out=h)
             hyena.hyena_filter_rfft2d(h, out=H)
             forward()
+    elif wl.film:
+        F = [to_dev(inp[k]) for k in ("omega", "gamma", "beta", "sigma")]
+        h = torch.empty((wl.B, wl.N, wl.D, wl.L), device="cuda", dtype=torch.float32)
+        H = torch.empty((wl.B, wl.N, wl.D, wl.L), device="cuda", dtype=torch.complex64)
+        ws_rfft_n = hyena.hyena_filter_rfft_workspace_size(wl.B * wl.N, wl.D, wl.L)
+        ws_fwd_n = hyena.hyena_fftconv_workspace_size(wl.B, wl.D, wl.L, wl.N, hyena.io_dtype(v), True)
+        ws_rfft = torch.empty(ws_rfft_n, device="cuda", dtype=torch.uint8) if ws_rfft_n else None
+        ws_fwd = torch.empty(max(ws_fwd_n, 1), device="cuda", dtype=torch.uint8)
+
+        def forward():
+            hyena.hyena_fftconv_gate_forward_per_sample(v, xs, b, H, out=y, workspace=ws_fwd)
+
+        def step():
+            hyena.hyena_filter_gen_film(*W, wl.N, wl.D, wl.L, B=wl.B, omega=F[0], gamma=F[1], beta=F[2],
+                                        sigma=F[3], n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                        decay_div=synth.DECAY_DIV, out=h)
+            hyena.hyena_filter_rfft(h.view(wl.B * wl.N, wl.D, wl.L), out=H.view(wl.B * wl.N, wl.D, wl.L),
+                                    workspace=ws_rfft)
+            forward()
     else:
         h = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.complex64)
@@ -361,6 +386,11 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     hb = torch.from_numpy(inp["b"]).pin_memory()
     hW = [torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
           for k in ("W1", "W2", "W3", "Wout", "alpha")]
+    dW = list(W)
+    if wl.film:   # the per-sample control vectors are step inputs as well
+        hW += [torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
+               for k in ("omega", "gamma", "beta", "sigma")]
+        dW += F
     hy_out = torch.empty(y.shape, dtype=io).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in [hv, *hxs, hb, *hW])
     d2h = hy_out.numel() * hy_out.element_size()
@@ -373,7 +403,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
         for xd, xh in zip(xs, hxs):
             xd.copy_(xh, non_blocking=True)
         b.copy_(hb, non_blocking=True)
-        for wd, wh in zip(W, hW):
+        for wd, wh in zip(dW, hW):
             wd.copy_(wh, non_blocking=True)
         step()
         hy_out.copy_(y, non_blocking=True)
@@ -383,7 +413,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
 
     # ---- the backward pass (1-D, L <= 16384): one call per timed repetition
     bwd = None
-    if wl.kind == "1d" and not long_path(wl):
+    if wl.kind == "1d" and not long_path(wl) and not wl.film:
         dy = to_dev(synth.make_output_grad(wl), io)
         ws_b = torch.empty(hyena.hyena_fftconv_backward_workspace_size(wl.D, wl.L, wl.N),
                            device="cuda", dtype=torch.uint8)
@@ -448,11 +478,19 @@ def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: 
     import oracle
     rows = np.concatenate([n * wl.D + channels for n in range(wl.N)])
     t0 = time.perf_counter()
+    v = inp["v"][:, channels].astype(np.float64)
+    x = np.stack([xx[:, channels] for xx in inp["x"]]).astype(np.float64)
+    if wl.film:
+        h = oracle.filter_gen_film(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["omega"],
+                                   inp["gamma"], inp["beta"], inp["sigma"][channels], True, wl.N,
+                                   len(channels), wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                   decay_div=synth.DECAY_DIV, threads=threads)
+        oracle.hyena_forward_per_sample(v, x, h, inp["b"][:, channels].astype(np.float64), route="fft",
+                                        threads=threads)
+        return time.perf_counter() - t0
     h = oracle.filter_gen(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
                           wl.N, len(channels), wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
                           decay_div=synth.DECAY_DIV, threads=threads)
-    v = inp["v"][:, channels].astype(np.float64)
-    x = np.stack([xx[:, channels] for xx in inp["x"]]).astype(np.float64)
     oracle.hyena_forward(v, x, h, inp["b"][:, channels].astype(np.float64), route="fft",
                          threads=threads)
     return time.perf_counter() - t0

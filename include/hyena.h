@@ -108,6 +108,35 @@ HYENA_API int hyena_last_cuda_error(void);
 HYENA_API hyena_status_t hyena_filter_gen(const hyena_ffn_t* ffn, int N, int D, int L,
                                 float* h, void* stream);
 
+/* Input-dependent filters ("Native Multi-Dimensional Subquadratic Operators
+ * via Input Dependent Long Convolutions": Input-Dependent Kernels via
+ * Registers and FiLM; Kernel Parameterization).  Per sample b the three
+ * sine layers of the filter network are modulated feature-wise (FiLM) and
+ * each hidden unit has its own frequency:
+ *     a_l = sin(omega_l * (gamma_bl * (W_l a_(l-1)) + beta_bl)),  l = 1..3,
+ * then the head and a window: the exponential decay of hyena_ffn_t, or,
+ * when sigma is given, the Gaussian exp(-t^2 / (2 sigma_d^2)), t = i/L.
+ * The control vectors gamma, beta of each sample come from the model (the
+ * pages derive them from register tokens); here they are inputs.  All
+ * pointers are device pointers, NULL for the default:
+ *   omega  [3][width]     per-unit frequencies (default 1)
+ *   gamma  [B][3][width]  FiLM scales (default 1)
+ *   beta   [B][3][width]  FiLM shifts (default 0)
+ *   sigma  [D]            Gaussian window widths (default: exponential) */
+typedef struct {
+    const float* omega;
+    const float* gamma;
+    const float* beta;
+    const float* sigma;
+} hyena_film_t;
+
+/* Per-sample filters h [B][N][D][L] float32 (1-D).  With every pointer of
+ * film NULL each sample's filters equal hyena_filter_gen's.  Their spectra
+ * are hyena_filter_rfft of the B*N rows of D filters (N' = B*N); the
+ * forward that uses them is hyena_fftconv_gate_forward_per_sample. */
+HYENA_API hyena_status_t hyena_filter_gen_film(const hyena_ffn_t* ffn, const hyena_film_t* film,
+                                               int B, int N, int D, int L, float* h, void* stream);
+
 /* Filter spectra H [N][D][L] complex64 in the PACKED real-DFT layout: for
  * each h[n][d] zero-padded to 2L ("Handling Boundaries": pad to double the
  * grid so the product of spectra is a linear, non-circular convolution),
@@ -157,6 +186,18 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* c
                                           int L, int N, hyena_dtype_t io,
                                           void* y, void* workspace,
                                           size_t ws_bytes, void* stream);
+
+/* The forward with a filter set per sample (input-dependent filters, see
+ * hyena_filter_gen_film): H [B][N][D][L] packed complex64, the spectra of
+ * sample b's filters at H + b*N*D*L.  Everything else as
+ * hyena_fftconv_gate_forward with the spectrum given (the same workspace
+ * size).  Sequence (b, d) multiplies by sample b's spectra of channel d. */
+HYENA_API hyena_status_t hyena_fftconv_gate_forward_per_sample(const void* v, const void* const* x,
+                                                               const float* H, const float* bias,
+                                                               int B, int D, int L, int N,
+                                                               hyena_dtype_t io, void* y,
+                                                               void* workspace, size_t ws_bytes,
+                                                               void* stream);
 
 /* Size of the scratch array built into the library for
  * hyena_fftconv_gate_forward_noalloc (16 MB on every device that loads the

@@ -45,9 +45,39 @@ struct FilterGenArgs {
     int Hh, Ww;                    // 2-D grid; 0 for 1-D
     int n_bands;
     float inv_div;                 // 1 / decay_div
-    float* h;                      // [rows][positions]
+    float* h;                      // [rows][positions] (per sample with FiLM)
     int vec;                       // positions % 4 == 0 and h 16-byte aligned: 128-bit h access
+    // input-dependent filters (1-D): sample b = blockIdx.z modulates the
+    // sine layers, a_l = sin(omega_l (gamma_bl (W_l a_(l-1)) + beta_bl));
+    // NULL omega / gamma / beta mean 1 / 1 / 0
+    const float *omega;            // [3][width]
+    const float *gamma, *beta;     // [B][3][width]
+    int film;                      // 1: modulate (any of the three given)
+    int gaussian;                  // 1: window exp(-t^2 / (2 sigma^2)), sigma in alpha[]
+    float inv_L2;                  // 1 / L^2
+    long sample_stride;            // floats of h per sample (rows * positions)
 };
+
+// The window of a row is exp(c u): the exponential decay has u = dist
+// (i in 1-D, iy + ix in 2-D) and c = -alpha / div; the Gaussian (1-D) has
+// u = dist^2 and c = -1 / (2 sigma^2 L^2).  par is alpha or sigma.
+__device__ __forceinline__ float window_coeff(const FilterGenArgs& a, float par)
+{
+    return a.gaussian ? -0.5f * a.inv_L2 / (par * par) : -par * a.inv_div;
+}
+__device__ __forceinline__ float window_arg(const FilterGenArgs& a, float dist)
+{
+    return a.gaussian ? dist * dist : dist;
+}
+
+// Offsets the per-sample pointers by the sample of this CTA (blockIdx.z).
+__device__ __forceinline__ void select_sample(FilterGenArgs& a)
+{
+    const int b = blockIdx.z;
+    a.h += (long)b * a.sample_stride;
+    if (a.gamma) a.gamma += (long)b * 3 * a.width;
+    if (a.beta) a.beta += (long)b * 3 * a.width;
+}
 
 constexpr int kFgThreads = 256;     // a 16 x 16 thread grid
 constexpr int kFgTile = 64;         // positions per head / tail / layers tile
@@ -59,13 +89,15 @@ constexpr int kFgUS = kFfnWidth + 4;     // [input][unit] weight rows, [unit][po
 constexpr int kFgRS = kFgRowTile + 4;    // [unit][row] Wout tile of the head
 // transposed W1 (canonical feature slots), W2, W3: [input][unit]
 constexpr int kFgWRegion = (kFfnMaxIn + 2 * kFfnWidth) * kFgUS;
+// FiLM parameters of the three layers: [layer][omega, gamma, beta][unit]
+constexpr int kFgFilm = 3 * 3 * kFfnWidth;
 
 template <int PT>
 struct LayerTile {
     static constexpr int AS = PT + 4;                    // activation row stride
     static constexpr int PPT = PT / 16;                  // positions per thread
-    // weights + features/a2 [66][AS] + a1/a3 [64][AS]
-    static constexpr size_t SMEM = sizeof(float) * (kFgWRegion + (kFfnMaxIn + kFfnWidth) * AS);
+    // weights + features/a2 [66][AS] + a1/a3 [64][AS] + FiLM [3][3][64]
+    static constexpr size_t SMEM = sizeof(float) * (kFgWRegion + (kFfnMaxIn + kFfnWidth) * AS + kFgFilm);
 };
 template <int NG>
 constexpr size_t fg_head_smem_bytes() { return sizeof(float) * (kFfnWidth * kFgRS + kFfnWidth * (64 * NG + 4)); }
@@ -187,7 +219,7 @@ __device__ __forceinline__ void stage_weights(const FilterGenArgs& a, float* sW)
 // of a tile; thread (ty, tx) owns units 4 ty .. 4 ty + 3 and positions
 // PPT tx .. PPT tx + PPT - 1.  WT is [input][unit] (stride kFgUS).
 template <int PT, int K>
-__device__ __forceinline__ void sine_layer(const float* WT, const float* in, float* out)
+__device__ __forceinline__ void sine_layer(const float* WT, const float* in, float* out, const float* film)
 {
     constexpr int AS = LayerTile<PT>::AS, PPT = LayerTile<PT>::PPT;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -212,6 +244,16 @@ __device__ __forceinline__ void sine_layer(const float* WT, const float* in, flo
 #pragma unroll
             for (int k = 0; k < PPT; ++k) acc[i][k] = fmaf(wv[i], x[k], acc[i][k]);
     }
+    if (film) {
+        // feature-wise modulation of this layer: omega (gamma acc + beta)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int u = 4 * ty + i;
+            const float om = film[u], g = film[kFfnWidth + u], be = film[2 * kFfnWidth + u];
+#pragma unroll
+            for (int k = 0; k < PPT; ++k) acc[i][k] = om * fmaf(g, acc[i][k], be);
+        }
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         if constexpr (PPT == 4) {
@@ -223,20 +265,36 @@ __device__ __forceinline__ void sine_layer(const float* WT, const float* in, flo
     }
 }
 
+// Stage the FiLM parameters of this CTA's sample into sF [3][3][64]
+// (omega, gamma, beta per layer; defaults 1, 1, 0).
+__device__ __forceinline__ void stage_film(const FilterGenArgs& a, float* sF)
+{
+    for (int e = threadIdx.x; e < kFgFilm; e += blockDim.x) {
+        const int l = e / (3 * kFfnWidth), kind = (e / kFfnWidth) % 3, u = e % kFfnWidth;
+        float v = kind == 2 ? 0.0f : 1.0f;
+        if (u < a.width) {
+            const float* src = kind == 0 ? a.omega : kind == 1 ? a.gamma : a.beta;
+            if (src) v = __ldg(src + l * a.width + u);
+        }
+        sF[e] = v;
+    }
+}
+
 // The three sine layers of one tile: features into sX, a1 into sY, a2 into
 // sX, a3 into sY.  Ends with a barrier (a3 visible to the whole CTA).
 template <bool TWO_D, int PT>
 __device__ __forceinline__ void layers_tile(const FilterGenArgs& a, long npos, long p0, const float* sW,
-                                            float* sX, float* sY)
+                                            float* sX, float* sY, const float* sF)
 {
     constexpr int NIN = TWO_D ? kFfnMaxIn : 33;
+    const float* f = a.film ? sF : nullptr;
     features_tile<TWO_D, PT>(a, npos, p0, sX);
     __syncthreads();
-    sine_layer<PT, NIN>(sW, sX, sY);
+    sine_layer<PT, NIN>(sW, sX, sY, f);
     __syncthreads();
-    sine_layer<PT, kFfnWidth>(sW + kFfnMaxIn * kFgUS, sY, sX);
+    sine_layer<PT, kFfnWidth>(sW + kFfnMaxIn * kFgUS, sY, sX, f ? f + 3 * kFfnWidth : nullptr);
     __syncthreads();
-    sine_layer<PT, kFfnWidth>(sW + (kFfnMaxIn + kFfnWidth) * kFgUS, sX, sY);
+    sine_layer<PT, kFfnWidth>(sW + (kFfnMaxIn + kFfnWidth) * kFgUS, sX, sY, f ? f + 6 * kFfnWidth : nullptr);
     __syncthreads();
 }
 
@@ -348,32 +406,31 @@ __device__ __forceinline__ void head_block(const FilterGenArgs& a, long npos, lo
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
         const long pos0 = p0 + 64 * g + 4 * tx;
-        float dist[4];   // window arguments of the group's 4 positions
+            float dist[4];   // window arguments of the group's 4 positions
 #pragma unroll
-        for (int k = 0; k < 4; ++k) dist[k] = window_dist<TWO_D>(a, pos0 + k);
+        for (int k = 0; k < 4; ++k) dist[k] = window_arg(a, window_dist<TWO_D>(a, pos0 + k));
 #pragma unroll
         for (int i = 0; i < RT; ++i) {
             const int r = r0 + RT * ty + i;
             if (r >= r_end) continue;
             float* hr = a.h + (long)r * npos;
-            const float c = -al[i] * a.inv_div;
             const float* v = acc[i] + 4 * g;
+            float wv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) wv[k] = v[k] * expf(al[i] * dist[k]);
             if (a.vec) {
-                if (pos0 < npos)
-                    *reinterpret_cast<float4*>(hr + pos0) =
-                        make_float4(v[0] * expf(c * dist[0]), v[1] * expf(c * dist[1]),
-                                    v[2] * expf(c * dist[2]), v[3] * expf(c * dist[3]));
+                if (pos0 < npos) *reinterpret_cast<float4*>(hr + pos0) = make_float4(wv[0], wv[1], wv[2], wv[3]);
             } else {
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    if (pos0 + k < npos) hr[pos0 + k] = v[k] * expf(c * dist[k]);
+                    if (pos0 + k < npos) hr[pos0 + k] = wv[k];
             }
         }
     }
 }
 
-// alpha of rows r0 + RT ty + i (loaded before the products so the loads
-// overlap them)
+// Window coefficients of rows r0 + RT ty + i (loaded before the products
+// so the loads overlap them).
 template <int RT>
 __device__ __forceinline__ void load_alpha(const FilterGenArgs& a, int r0, int r_end, float* al)
 {
@@ -381,7 +438,7 @@ __device__ __forceinline__ void load_alpha(const FilterGenArgs& a, int r0, int r
 #pragma unroll
     for (int i = 0; i < RT; ++i) {
         const int r = r0 + RT * ty + i;
-        al[i] = r < r_end ? __ldg(a.alpha + r % a.D) : 0.0f;
+        al[i] = r < r_end ? window_coeff(a, __ldg(a.alpha + r % a.D)) : 0.0f;
     }
 }
 
@@ -391,20 +448,23 @@ template <bool TWO_D, int PT>
 __global__ void __launch_bounds__(kFgThreads) filter_layers_kernel(FilterGenArgs a)
 {
     grid_dependency_begin();
+    select_sample(a);
     using LT = LayerTile<PT>;
     constexpr int AS = LT::AS, PPT = LT::PPT;
     extern __shared__ __align__(16) float fg_smem[];
     float* sW = fg_smem;
     float* sX = fg_smem + kFgWRegion;
     float* sY = sX + kFfnMaxIn * AS;
+    float* sF = sY + kFfnWidth * AS;
     const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
     const long ntiles = (npos + PT - 1) / PT;
     float* stash = a.h + (long)(a.rows - kFfnWidth) * npos;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
     stage_weights<TWO_D>(a, sW);
+    if (a.film) stage_film(a, sF);
     for (long tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const long p0 = tile * PT;
-        layers_tile<TWO_D, PT>(a, npos, p0, sW, sX, sY);   // ends with a barrier
+        layers_tile<TWO_D, PT>(a, npos, p0, sW, sX, sY, sF);   // ends with a barrier
         // stash a3: thread (ty, tx) stores its own 4 units x PPT positions
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -435,6 +495,7 @@ template <bool TWO_D, int NG>
 __global__ void __launch_bounds__(kFgThreads, NG == 1 ? 3 : 2) filter_head_kernel(FilterGenArgs a)
 {
     grid_dependency_begin();
+    select_sample(a);
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][132]: Wout tile, transposed
     float* sA = fg_smem + kFfnWidth * kFgRS;                // [64][64 NG + 4]: a3 tile
@@ -456,6 +517,7 @@ template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_tail_kernel(FilterGenArgs a)
 {
     grid_dependency_begin();
+    select_sample(a);
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][68]: Wout stash rows, transposed
     float* sA = fg_smem + kFfnWidth * kFgUS;                // [64][68]: a3 tile
@@ -476,6 +538,7 @@ template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_tail16_kernel(FilterGenArgs a)
 {
     grid_dependency_begin();
+    select_sample(a);
     constexpr int PT = kFgSmallTile, AS = PT + 4;
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][68]: Wout stash rows, transposed
@@ -515,10 +578,9 @@ __global__ void __launch_bounds__(kFgThreads) filter_tail16_kernel(FilterGenArgs
     }
     const long pos = p0 + tx;
     if (pos >= npos) return;
-    const float dist = window_dist<TWO_D>(a, pos);
+    const float u = window_arg(a, window_dist<TWO_D>(a, pos));
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        stash[(long)(4 * ty + i) * npos + pos] = acc[i] * expf(-al[i] * a.inv_div * dist);
+    for (int i = 0; i < 4; ++i) stash[(long)(4 * ty + i) * npos + pos] = acc[i] * expf(al[i] * u);
 }
 
 // Single launch for at most 64 rows: every CTA evaluates the layers of its
@@ -527,17 +589,20 @@ template <bool TWO_D>
 __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
 {
     grid_dependency_begin();
+    select_sample(a);
     using LT = LayerTile<kFgTile>;
     extern __shared__ __align__(16) float fg_smem[];
     float* sW = fg_smem;
     float* sX = fg_smem + kFgWRegion;
     float* sY = sX + kFfnMaxIn * LT::AS;
+    float* sF = sY + kFfnWidth * LT::AS;
     const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
     const long p0 = (long)blockIdx.x * kFgTile;
     float al[4];
     load_alpha<4>(a, 0, a.rows, al);
     stage_weights<TWO_D>(a, sW);
-    layers_tile<TWO_D, kFgTile>(a, npos, p0, sW, sX, sY);  // ends with a barrier
+    if (a.film) stage_film(a, sF);
+    layers_tile<TWO_D, kFgTile>(a, npos, p0, sW, sX, sY, sF);  // ends with a barrier
     load_wout_tile<kFfnWidth, kFgUS>(a, 0, a.rows, sW);   // the weights are no longer read
     __syncthreads();
     static_assert(LT::AS == kFgUS, "a3 tile stride");

@@ -98,6 +98,7 @@ struct FourStepArgs {
     const void* x[kMaxOrder];    // x_1..x_N, [B][D][L] io
     void* y;                       // [B][D][L] io
     const float2* H;               // [N][D][L] packed spectra (row kernel, conv mode)
+    size_t H_bstride;              // slots between samples' spectra (0: shared by the batch)
     const float* bias;             // [N][D]
     float2* S;                     // scratch [wave][M1][M2] complex
     float2* Hout;                  // [rows][L] packed spectra (row kernel, spectrum mode)
@@ -269,7 +270,7 @@ fourstep_row_kernel(FourStepArgs a)
         return;
     } else {
         const float bias = __ldg(a.bias + a.n * a.D + d);
-        const float2* Hr = a.H + ((size_t)a.n * a.D + d) * M;
+        const float2* Hr = a.H + (size_t)(q % a.B) * a.H_bstride + ((size_t)a.n * a.D + d) * M;
         FS::for_each_pair(smem_fs, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2 w) {
             float2 z1 = *p1, z2 = *p2;
             if (kind == 1) {                                    // slot 0 holds (bin 0, bin M), both real

@@ -63,9 +63,10 @@ struct Fused1dArgs {
     const void* v;                 // [B][D][L] io
     const void* x[kMaxOrder];      // N pointers, each [B][D][L] io
     void* y;                       // [B][D][L] io
-    const float2* H;               // [N][D][L] packed filter spectra
+    const float2* H;               // [N][D][L] packed filter spectra ([B][N][D][L] per sample)
     const float* bias;             // [N][D]
     int B, D, N;
+    size_t H_bstride;              // slots between samples' spectra (0: shared by the batch)
 };
 
 struct Rfft1dArgs {
@@ -421,9 +422,10 @@ fused1d_kernel(Fused1dArgs args)
     float2* sm = smem_dyn + g * F::SMEM_SEQ;
     float2* stage = smem_dyn + F::G * F::SMEM_SEQ + g * F::STAGE_SEQ;
 
+    const float2* Hb = args.H + (size_t)b * args.H_bstride;    // this sample's spectra
     // H_0 (or x_1) is in flight while v is loaded and transformed
     if constexpr (!F::H_IN_EXCHANGE)
-        cp_async_row(stage, args.H + (size_t)d * M, M * 8, t, T);
+        cp_async_row(stage, Hb + (size_t)d * M, M * 8, t, T);
 
     float2 a[E];
     {
@@ -438,7 +440,7 @@ fused1d_kernel(Fused1dArgs args)
         for (int i = 1; i < kMaxOrder; ++i)
             if (i == n) xn = args.x[i];
         const PT* xg = reinterpret_cast<const PT*>(xn) + seq * (M / 2);
-        const float2* Hg = args.H + ((size_t)n * args.D + d) * M;
+        const float2* Hg = Hb + ((size_t)n * args.D + d) * M;
         const float bias = __ldg(args.bias + n * args.D + d);
         const float2* Hs;
 
@@ -468,7 +470,7 @@ fused1d_kernel(Fused1dArgs args)
         __syncthreads();                                  // x_n consumed
         if constexpr (!F::H_IN_EXCHANGE)
             if (n + 1 < args.N)
-                cp_async_row(stage, args.H + ((size_t)(n + 1) * args.D + d) * M, M * 8, t, T);
+                cp_async_row(stage, Hb + ((size_t)(n + 1) * args.D + d) * M, M * 8, t, T);
     }
     if (active) {
         PT* yp = reinterpret_cast<PT*>(args.y) + seq * (M / 2);

@@ -70,9 +70,10 @@ hyena_status_t check_ffn(const hyena_ffn_t* f)
 }
 
 hyena_status_t filter_gen(const hyena_ffn_t* f, int rows, int D, long npos, int L, int Hh,
-                          int Ww, bool two_d, float* h, cudaStream_t st)
+                          int Ww, bool two_d, float* h, cudaStream_t st,
+                          const hyena_film_t* film = nullptr, int B = 1)
 {
-    FilterGenArgs a;
+    FilterGenArgs a = {};
     a.W1 = f->W1; a.W2 = f->W2; a.W3 = f->W3; a.Wout = f->Wout; a.alpha = f->alpha;
     a.n_in = two_d ? 2 + 4 * f->n_bands : 1 + 2 * f->n_bands;
     a.width = f->width;
@@ -83,13 +84,29 @@ hyena_status_t filter_gen(const hyena_ffn_t* f, int rows, int D, long npos, int 
     a.inv_div = 1.0f / f->decay_div;
     a.h = h;
     a.vec = (npos % 4 == 0 && aligned(h, 16)) ? 1 : 0;
-    return launch_filter_gen(a, two_d, npos, st);
+    a.sample_stride = (long)rows * npos;
+    a.inv_L2 = L > 0 ? 1.0f / ((float)L * (float)L) : 0.0f;
+    if (film) {
+        a.omega = film->omega;
+        a.gamma = film->gamma;
+        a.beta = film->beta;
+        a.film = (film->omega || film->gamma || film->beta) ? 1 : 0;
+        if (film->sigma) {
+            a.gaussian = 1;
+            a.alpha = film->sigma;                 // the per-channel window parameter
+        }
+    }
+    return launch_filter_gen(a, two_d, npos, B, st);
 }
 
 // packed spectrum: L complex slots per filter (bins 0 and L share slot 0)
 size_t spectrum_bytes(long N, long D, long L) { return sizeof(float2) * N * D * L; }
 
 size_t round_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
+
+hyena_status_t forward_impl(const void* v, const void* const* x, const float* h, const float* H,
+                            bool per_sample, const float* bias, int B, int D, int L, int N,
+                            hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes, void* stream);
 
 }  // namespace
 
@@ -126,6 +143,20 @@ hyena_status_t hyena_filter_gen(const hyena_ffn_t* ffn, int N, int D, int L, flo
     if ((long)N * D > 65535L * kFgRowTile || (long)N * D * (long)L > (1L << 40))
         return HYENA_ERR_UNSUPPORTED;
     return filter_gen(ffn, N * D, D, L, L, 0, 0, false, h, (cudaStream_t)stream);
+}
+
+hyena_status_t hyena_filter_gen_film(const hyena_ffn_t* ffn, const hyena_film_t* film, int B, int N,
+                                     int D, int L, float* h, void* stream)
+{
+    hyena_status_t s = check_ffn(ffn);
+    if (s != HYENA_OK) return s;
+    if (!film || !h || B < 1 || N < 1 || D < 1 || L < 1 || !aligned(h, 4)) return HYENA_ERR_INVALID_ARG;
+    const void* p[4] = {film->omega, film->gamma, film->beta, film->sigma};
+    for (const void* q : p)
+        if (q && !aligned(q, 4)) return HYENA_ERR_INVALID_ARG;
+    if (B > 65535 || (long)N * D > 65535L * kFgRowTile || (long)B * N * D * (long)L > (1L << 40))
+        return HYENA_ERR_UNSUPPORTED;
+    return filter_gen(ffn, N * D, D, L, L, 0, 0, false, h, (cudaStream_t)stream, film, B);
 }
 
 hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C, int H, int W, float* h,
@@ -188,6 +219,27 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
                                           int N, hyena_dtype_t io, void* y, void* workspace,
                                           size_t ws_bytes, void* stream)
 {
+    return forward_impl(v, x, h, H, false, bias, B, D, L, N, io, y, workspace, ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv_gate_forward_per_sample(const void* v, const void* const* x,
+                                                     const float* H, const float* bias, int B, int D,
+                                                     int L, int N, hyena_dtype_t io, void* y,
+                                                     void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!H) return HYENA_ERR_INVALID_ARG;
+    return forward_impl(v, x, nullptr, H, true, bias, B, D, L, N, io, y, workspace, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// The forward; per_sample: H holds B spectrum sets [B][N][D][L].
+hyena_status_t forward_impl(const void* v, const void* const* x, const float* h, const float* H,
+                            bool per_sample, const float* bias, int B, int D, int L, int N,
+                            hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes, void* stream)
+{
     if (!v || !x || !y || !bias || (!h && !H)) return HYENA_ERR_INVALID_ARG;
     if (B < 1 || D < 1 || N < 1 || L < 1) return HYENA_ERR_INVALID_ARG;
     if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
@@ -202,7 +254,7 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
     if ((H && !aligned(H, 16)) || (!H && !aligned(h, 16))) return HYENA_ERR_INVALID_ARG;
 
     const size_t act = (size_t)B * D * L * io_bytes(io);
-    const size_t spec = spectrum_bytes(N, D, L);
+    const size_t spec = spectrum_bytes(N, D, L) * (per_sample ? (size_t)B : 1);
     const size_t need = hyena_fftconv_workspace_size(B, D, L, N, io, H != nullptr);
     if (need > 0 && (!workspace || ws_bytes < need || !aligned(workspace, 256)))
         return HYENA_ERR_WORKSPACE;
@@ -234,7 +286,7 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
         scratch = reinterpret_cast<float2*>(ws);
     }
     if (log2m <= kMaxLog2Fused) {
-        Fused1dArgs a;
+        Fused1dArgs a = {};
         a.v = v;
         for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
         a.y = y;
@@ -243,6 +295,7 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
         a.B = B;
         a.D = D;
         a.N = N;
+        a.H_bstride = per_sample ? (size_t)N * D * L : 0;
         return io == HYENA_BF16 ? dispatch_fused_bf16(log2m, a, st) : dispatch_fused_f32(log2m, a, st);
     }
     FourStepArgs a = {};
@@ -250,12 +303,17 @@ hyena_status_t hyena_fftconv_gate_forward(const void* v, const void* const* x, c
     for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
     a.y = y;
     a.H = spectrum;
+    a.H_bstride = per_sample ? (size_t)N * D * L : 0;
     a.bias = bias;
     a.B = B;
     a.D = D;
     return io == HYENA_BF16 ? dispatch_fourstep_bf16(log2m, a, N, scratch, st)
                             : dispatch_fourstep_f32(log2m, a, N, scratch, st);
 }
+
+}  // namespace
+
+extern "C" {
 
 size_t hyena_fftconv_backward_workspace_size(int D, int L, int N)
 {

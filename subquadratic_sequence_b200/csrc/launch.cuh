@@ -81,7 +81,7 @@ hyena_status_t dispatch_fourstep_bf16(int log2m, const FourStepArgs& a, int N, f
                                       cudaStream_t st);
 hyena_status_t dispatch_fourstep_rfft(int log2m, const float* h, int rows, float2* H,
                                       float2* scratch, cudaStream_t st);
-hyena_status_t launch_filter_gen(const FilterGenArgs& a, bool two_d, long npos, cudaStream_t st);
+hyena_status_t launch_filter_gen(const FilterGenArgs& a, bool two_d, long npos, int B, cudaStream_t st);
 hyena_status_t dispatch_backward_f32(int log2m, const Backward1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_backward_bf16(int log2m, const Backward1dArgs& a, cudaStream_t st);
 

@@ -147,7 +147,7 @@ extern "C" hyena_status_t hyena_fftconv_gate_forward_noalloc(const void* v, cons
 
     cudaStream_t st = (cudaStream_t)stream;
     if (log2m <= kMaxLog2Fused) {       // no scratch at these lengths
-        Fused1dArgs a;
+        Fused1dArgs a = {};
         a.v = v;
         for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
         a.y = y;

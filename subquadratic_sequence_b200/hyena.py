@@ -36,6 +36,11 @@ class hyena_ffn_t(ctypes.Structure):
                 ("n_bands", ctypes.c_int), ("width", ctypes.c_int), ("decay_div", ctypes.c_float)]
 
 
+class hyena_film_t(ctypes.Structure):
+    _fields_ = [("omega", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("sigma", ctypes.c_void_p)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(_build.LIB):
         raise ImportError(
@@ -49,6 +54,9 @@ def _load() -> ctypes.CDLL:
         "hyena_last_cuda_error": ([], i),
         "hyena_filter_gen": ([ffn_p, i, i, i, vp, vp], i),
         "hyena_filter_gen_2d": ([ffn_p, i, i, i, i, vp, vp], i),
+        "hyena_filter_gen_film": ([ffn_p, ctypes.POINTER(hyena_film_t), i, i, i, i, vp, vp], i),
+        "hyena_fftconv_gate_forward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp,
+                                                   sz, vp], i),
         "hyena_filter_rfft_workspace_size": ([i, i, i], sz),
         "hyena_filter_rfft": ([vp, i, i, i, vp, vp, sz, vp], i),
         "hyena_fftconv_workspace_size": ([i, i, i, i, i, i], sz),
@@ -124,6 +132,44 @@ def hyena_filter_gen(W1, W2, W3, Wout, alpha, N: int, D: int, L: int, *, n_bands
         out = torch.empty((N, D, L), device=W1.device, dtype=torch.float32)
     _check("hyena_filter_gen", LIB.hyena_filter_gen(
         ctypes.byref(f), N, D, L, ctypes.c_void_p(_dev(out, torch.float32, "h")), _stream(stream)))
+    return out
+
+
+def hyena_filter_gen_film(W1, W2, W3, Wout, alpha, N: int, D: int, L: int, *, B: int, omega=None,
+                          gamma=None, beta=None, sigma=None, n_bands: int = 8, width: int = 64,
+                          decay_div: float = 64.0, out=None, stream=None):
+    """Per-sample (input-dependent) filters h [B][N][D][L] float32: the sine
+    layers modulated by FiLM, a_l = sin(omega_l (gamma_bl W_l a_(l-1) +
+    beta_bl)); omega [3][width], gamma / beta [B][3][width], sigma [D] (the
+    Gaussian window; None keeps the exponential decay of alpha)."""
+    f = _ffn(W1, W2, W3, Wout, alpha, n_bands, width, decay_div)
+    opt = lambda t, name: ctypes.c_void_p(_dev(t, torch.float32, name)) if t is not None else None
+    film = hyena_film_t(opt(omega, "omega"), opt(gamma, "gamma"), opt(beta, "beta"), opt(sigma, "sigma"))
+    if out is None:
+        out = torch.empty((B, N, D, L), device=W1.device, dtype=torch.float32)
+    _check("hyena_filter_gen_film", LIB.hyena_filter_gen_film(
+        ctypes.byref(f), ctypes.byref(film), B, N, D, L, ctypes.c_void_p(_dev(out, torch.float32, "h")),
+        _stream(stream)))
+    return out
+
+
+def hyena_fftconv_gate_forward_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor, *,
+                                          out=None, workspace=None, stream=None):
+    """The forward with per-sample spectra H [B][N][D][L] complex64."""
+    B, D, L = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    need = hyena_fftconv_workspace_size(B, D, L, N, io, True)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=v.device, dtype=torch.uint8)
+    _check("hyena_fftconv_gate_forward_per_sample", LIB.hyena_fftconv_gate_forward_per_sample(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
 
 

@@ -41,6 +41,7 @@ class Workload:
     W: int = 0       # grid width (2-D)
     io: str = "f32"  # storage type of v, x_n, y: "f32" or "bf16"
     seed: int = 0
+    film: bool = False  # input-dependent (per-sample, FiLM-modulated) filters
 
     @property
     def positions(self) -> int:
@@ -73,6 +74,9 @@ WORKLOADS = {
     "c3_1m": Workload("c3_1m", "1d", N=2, B=1, D=256, L=1048576, io="f32", seed=_seed(3, 2)),
     # order-2 2-D operator on a 256x256 grid, B=2, C=128
     "c4": Workload("c4", "2d", N=2, B=2, D=128, H=256, W=256, io="f32", seed=_seed(4)),
+    # c1 with input-dependent filters: a filter set per sample (FiLM-modulated
+    # sine layers, multi-frequency first layer, Gaussian window)
+    "c1_film": Workload("c1_film", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), film=True),
 }
 
 
@@ -119,7 +123,25 @@ def make_inputs(wl: Workload) -> dict:
     n_in = 1 + 2 * N_BANDS if wl.kind == "1d" else 2 + 4 * N_BANDS
     W1, W2, W3, Wout = _weights(rng, n_in, WIDTH, wl.N * wl.D)
     alpha = np.linspace(0.3, 1.5, wl.D).astype(np.float32)
-    return dict(v=v, x=x, b=b, W1=W1, W2=W2, W3=W3, Wout=Wout, alpha=alpha)
+    out = dict(v=v, x=x, b=b, W1=W1, W2=W2, W3=W3, Wout=Wout, alpha=alpha)
+    if wl.film:
+        out.update(make_film(wl))
+    return out
+
+
+def make_film(wl: Workload) -> dict:
+    """FiLM inputs of an input-dependent workload, from their own stream
+    (seed + 2): per-sample scales gamma = 1 + 0.1 N(0, 1) and shifts
+    beta = 0.1 N(0, 1) [B][3][64]; per-unit frequencies omega [3][64] with
+    the first layer in four blocks of 16 units at 1, 2, 4, 8 and the other
+    layers at 1; Gaussian window widths sigma = linspace(0.05, 0.5, D)."""
+    rng = np.random.default_rng(wl.seed + 2)
+    gamma = (1.0 + 0.1 * rng.standard_normal((wl.B, 3, WIDTH))).astype(np.float32)
+    beta = (0.1 * rng.standard_normal((wl.B, 3, WIDTH))).astype(np.float32)
+    omega = np.ones((3, WIDTH), np.float32)
+    omega[0] = np.repeat(np.array([1.0, 2.0, 4.0, 8.0], np.float32), WIDTH // 4)
+    sigma = np.linspace(0.05, 0.5, wl.D).astype(np.float32)
+    return dict(gamma=gamma, beta=beta, omega=omega, sigma=sigma)
 
 
 def make_output_grad(wl: Workload) -> np.ndarray:
