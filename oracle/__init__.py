@@ -61,6 +61,9 @@ def _load():
         "oracle_hyena_forward_2d": [dp, dp, dp, dp, l, l, l, l, l, i, i, dp],
         "oracle_hyena_backward": [dp, dp, dp, dp, dp, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_filter_gen_film": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, d, i, dp],
+        "oracle_cconv": [dp, dp, l, i, dp],
+        "oracle_rfft_circ": [dp, l, l, dp, dp],
+        "oracle_hyena_forward_circular": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -252,3 +255,34 @@ def hyena_forward_per_sample(v, x, h, bias, route="fft", threads=None) -> np.nda
     v, x, h, bias = map(_f64, (v, x, h, bias))
     return np.concatenate([hyena_forward(v[b:b + 1], x[:, b:b + 1], h[b], bias, route, threads)
                            for b in range(v.shape[0])])
+
+
+def cconv(h, u, route="direct") -> np.ndarray:
+    """Circular convolution y[t] = sum_s h[s] u[(t - s) mod L]."""
+    h, u = _f64(h), _f64(u)
+    y = np.empty_like(u)
+    _check(_load().oracle_cconv(_ptr(h), _ptr(u), u.shape[-1], _route(route), _ptr(y)), "oracle_cconv")
+    return y
+
+
+def rfft_circ(h) -> np.ndarray:
+    """L-point spectrum (no padding) of each row of h [..., L]: bins 0..L/2."""
+    h = _f64(h)
+    L = h.shape[-1]
+    rows = h.size // L
+    re = np.empty(h.shape[:-1] + (L // 2 + 1,))
+    im = np.empty_like(re)
+    _check(_load().oracle_rfft_circ(_ptr(h), rows, L, _ptr(re), _ptr(im)), "oracle_rfft_circ")
+    return re + 1j * im
+
+
+def hyena_forward_circular(v, x, h, bias, route="fft", threads=None) -> np.ndarray:
+    """The recurrence with circular convolutions of length L."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    B, D, L = v.shape
+    N = h.shape[0]
+    y = np.empty_like(v)
+    rc = _load().oracle_hyena_forward_circular(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), B, D, L, N,
+                                               _route(route), threads or default_threads(), _ptr(y))
+    _check(rc, "oracle_hyena_forward_circular")
+    return y

@@ -537,6 +537,78 @@ int oracle_conv(const double *h, const double *u, long L, int route, double *y)
 }
 
 /* ------------------------------------------------------------------ */
+/* Circular convolution ("Native Multi-Dimensional Subquadratic         */
+/* Operators ...", Handling Boundaries: circular convolutions for        */
+/* periodic systems, the alternative to zero padding).                   */
+/* ------------------------------------------------------------------ */
+
+/* The definition: y[t] = sum_{s=0..L-1} h[s] u[(t - s) mod L]. */
+static void cconv_direct(const double *h, const double *u, long L, double *y)
+{
+    for (long t = 0; t < L; ++t) {
+        double s = 0.0;
+        for (long k = 0; k < L; ++k) s += h[k] * u[((t - k) % L + L) % L];
+        y[t] = s;
+    }
+}
+
+/* The convolution theorem at exactly L points (no padding; L a power of
+ * two): DFT both, multiply, inverse DFT, scale by 1/L. */
+static void cconv_fft(const double *h, const double *u, long L, double *y, fft_scratch *s)
+{
+    for (long t = 0; t < L; ++t) {
+        s->hr[t] = h[t]; s->hi[t] = 0.0;
+        s->ur[t] = u[t]; s->ui[t] = 0.0;
+    }
+    fft_radix2(s->hr, s->hi, L, -1);
+    fft_radix2(s->ur, s->ui, L, -1);
+    for (long k = 0; k < L; ++k) {
+        const double re = s->hr[k] * s->ur[k] - s->hi[k] * s->ui[k];
+        const double im = s->hr[k] * s->ui[k] + s->hi[k] * s->ur[k];
+        s->ur[k] = re;
+        s->ui[k] = im;
+    }
+    fft_radix2(s->ur, s->ui, L, +1);
+    for (long t = 0; t < L; ++t) y[t] = s->ur[t] / (double)L;
+}
+
+int oracle_cconv(const double *h, const double *u, long L, int route, double *y)
+{
+    if (!h || !u || !y || L < 1) return ORACLE_EBADARG;
+    if (route == ROUTE_DIRECT) {
+        cconv_direct(h, u, L, y);
+        return ORACLE_OK;
+    }
+    if (route != ROUTE_FFT || !is_pow2(L)) return ORACLE_EBADARG;
+    fft_scratch s;
+    if (scratch_alloc(&s, L) != ORACLE_OK) {
+        scratch_free(&s);
+        return ORACLE_ENOMEM;
+    }
+    cconv_fft(h, u, L, y, &s);
+    scratch_free(&s);
+    return ORACLE_OK;
+}
+
+/* L-point spectrum of each row of h[rows][L] (no padding): bins 0..L/2. */
+int oracle_rfft_circ(const double *h, long rows, long L, double *out_re, double *out_im)
+{
+    if (!h || !out_re || !out_im || rows < 0 || L < 2 || !is_pow2(L)) return ORACLE_EBADARG;
+    double *re = malloc(sizeof(double) * L), *im = malloc(sizeof(double) * L);
+    if (!re || !im) { free(re); free(im); return ORACLE_ENOMEM; }
+    for (long r = 0; r < rows; ++r) {
+        for (long t = 0; t < L; ++t) { re[t] = h[r * L + t]; im[t] = 0.0; }
+        fft_radix2(re, im, L, -1);
+        for (long k = 0; k <= L / 2; ++k) {
+            out_re[r * (L / 2 + 1) + k] = re[k];
+            out_im[r * (L / 2 + 1) + k] = im[k];
+        }
+    }
+    free(re); free(im);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* The order-N Hyena recurrence, 1-D.                                  */
 /* ------------------------------------------------------------------ */
 
@@ -547,6 +619,7 @@ typedef struct {
     double *y;
     long s0, step; /* sequences s0, s0 + step, ... (s = b*D + d) */
     int status;
+    int circular;  /* 1: circular convolution of length L instead of causal */
 } fwd_job;
 
 static void *forward_worker(void *arg)
@@ -556,7 +629,7 @@ static void *forward_worker(void *arg)
     double *z = malloc(sizeof(double) * L), *c = malloc(sizeof(double) * L);
     fft_scratch s = {0};
     if (!z || !c || (j->route == ROUTE_FFT &&
-                     scratch_alloc(&s, next_pow2(2 * L)) != ORACLE_OK)) {
+                     scratch_alloc(&s, j->circular ? L : next_pow2(2 * L)) != ORACLE_OK)) {
         j->status = ORACLE_ENOMEM;
         goto done;
     }
@@ -567,8 +640,13 @@ static void *forward_worker(void *arg)
             const double *hn = j->h + (n * j->D + d) * L;
             const double *xn = j->x + n * BDL + seq * L;
             const double bn = j->bias[n * j->D + d];
-            if (j->route == ROUTE_DIRECT) conv_direct(hn, z, L, c);
-            else conv_fft(hn, z, L, c, &s);
+            if (j->circular) {
+                if (j->route == ROUTE_DIRECT) cconv_direct(hn, z, L, c);
+                else cconv_fft(hn, z, L, c, &s);
+            } else {
+                if (j->route == ROUTE_DIRECT) conv_direct(hn, z, L, c);
+                else conv_fft(hn, z, L, c, &s);
+            }
             /* z_n = x_n * (h_n (*) z_{n-1} + b_n z_{n-1}) */
             for (long t = 0; t < L; ++t) z[t] = xn[t] * (c[t] + bn * z[t]);
         }
@@ -581,10 +659,31 @@ done:
     return NULL;
 }
 
+static int forward_any(const double *v, const double *x, const double *h, const double *bias,
+                       long B, long D, long L, long N, int route, int nthreads, int circular,
+                       double *y);
+
 /* v [B][D][L], x [N][B][D][L], h [N][D][L], bias [N][D] -> y [B][D][L]. */
 int oracle_hyena_forward(const double *v, const double *x, const double *h,
                          const double *bias, long B, long D, long L, long N,
                          int route, int nthreads, double *y)
+{
+    return forward_any(v, x, h, bias, B, D, L, N, route, nthreads, 0, y);
+}
+
+/* The same recurrence with circular convolutions of length L (L a power of
+ * two for the FFT route). */
+int oracle_hyena_forward_circular(const double *v, const double *x, const double *h,
+                                  const double *bias, long B, long D, long L, long N,
+                                  int route, int nthreads, double *y)
+{
+    if (route == ROUTE_FFT && !is_pow2(L)) return ORACLE_EBADARG;
+    return forward_any(v, x, h, bias, B, D, L, N, route, nthreads, 1, y);
+}
+
+static int forward_any(const double *v, const double *x, const double *h, const double *bias,
+                       long B, long D, long L, long N, int route, int nthreads, int circular,
+                       double *y)
 {
     if (!v || !x || !h || !bias || !y || B < 1 || D < 1 || L < 1 || N < 1 ||
         (route != ROUTE_DIRECT && route != ROUTE_FFT))
@@ -595,7 +694,7 @@ int oracle_hyena_forward(const double *v, const double *x, const double *h,
     pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
     if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
     for (int k = 0; k < nthreads; ++k) {
-        fwd_job j = {v, x, h, bias, B, D, L, N, route, y, k, nthreads, 0};
+        fwd_job j = {v, x, h, bias, B, D, L, N, route, y, k, nthreads, 0, circular};
         jobs[k] = j;
         pthread_create(&tid[k], NULL, forward_worker, &jobs[k]);
     }

@@ -1,0 +1,71 @@
+"""Pins of the oracle's circular mode (convolution of length L without
+padding; "Native Multi-Dimensional Subquadratic Operators via Input
+Dependent Long Convolutions", Handling Boundaries).
+
+Against numpy's FFT (a library routine), np.roll (the closed form of a
+shift filter), and the separately pinned causal oracle: the circular
+recurrence on sequences zero-padded to 2L is the causal recurrence.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def rel_err(a, b):
+    return float(np.max(np.abs(np.asarray(a) - np.asarray(b))) / max(np.max(np.abs(b)), 1e-300))
+
+
+@pytest.mark.parametrize("L", [1, 2, 5, 16, 64])
+def test_cconv_direct_is_numpy(L):
+    r = np.random.default_rng(L)
+    h, u = r.standard_normal(L), r.standard_normal(L)
+    ref = np.real(np.fft.ifft(np.fft.fft(h) * np.fft.fft(u)))
+    assert rel_err(oracle.cconv(h, u, "direct"), ref) < 1e-12
+
+
+@pytest.mark.parametrize("L", [2, 16, 1024])
+def test_cconv_fft_equals_direct(L):
+    r = np.random.default_rng(L + 1)
+    h, u = r.standard_normal(L), r.standard_normal(L)
+    assert rel_err(oracle.cconv(h, u, "fft"), oracle.cconv(h, u, "direct")) < 1e-12
+
+
+@pytest.mark.parametrize("k", [0, 1, 7, 15])
+def test_cconv_shift_filter_is_a_rotation(k):
+    L = 16
+    u = np.random.default_rng(k).standard_normal(L)
+    h = np.zeros(L)
+    h[k] = 1.0
+    assert np.array_equal(oracle.cconv(h, u, "direct"), np.roll(u, k))
+
+
+def test_rfft_circ_is_numpy():
+    h = np.random.default_rng(3).standard_normal((3, 64))
+    assert rel_err(oracle.rfft_circ(h), np.fft.rfft(h)) < 1e-13
+
+
+@pytest.mark.parametrize("route", ["direct", "fft"])
+def test_circular_on_padded_sequences_is_the_causal_recurrence(route):
+    # zero-padded to 2L (filters and inputs), the circular recurrence's first
+    # L outputs are the causal recurrence's
+    r = np.random.default_rng(4)
+    B, D, L, N = 2, 3, 32, 3
+    v, x = r.standard_normal((B, D, L)), r.standard_normal((N, B, D, L))
+    h, b = r.standard_normal((N, D, L)), r.standard_normal((N, D))
+    pad = lambda a: np.concatenate([a, np.zeros_like(a)], axis=-1)
+    yc = oracle.hyena_forward_circular(pad(v), pad(x), pad(h), b, route=route)
+    assert rel_err(yc[..., :L], oracle.hyena_forward(v, x, h, b, route="direct")) < 1e-12
+    assert np.max(np.abs(yc[..., L:])) == 0.0
+
+
+def test_circular_forward_routes_agree_and_wrap():
+    r = np.random.default_rng(5)
+    B, D, L, N = 2, 2, 64, 2
+    v, x = r.standard_normal((B, D, L)), r.standard_normal((N, B, D, L))
+    h, b = r.standard_normal((N, D, L)), r.standard_normal((N, D))
+    yd = oracle.hyena_forward_circular(v, x, h, b, route="direct")
+    yf = oracle.hyena_forward_circular(v, x, h, b, route="fft")
+    assert rel_err(yf, yd) < 1e-12
+    # and it differs from the causal one (the wrap-around terms)
+    assert rel_err(yd, oracle.hyena_forward(v, x, h, b, route="direct")) > 1e-3
