@@ -199,6 +199,25 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_per_sample(const void* v, co
                                                                void* workspace, size_t ws_bytes,
                                                                void* stream);
 
+/* Circular mode ("Native Multi-Dimensional Subquadratic Operators via Input
+ * Dependent Long Convolutions", Handling Boundaries: circular convolutions
+ * for periodic systems, the alternative to zero padding).  The same
+ * recurrence with every convolution circular of length L:
+ *     (h (*) u)[t] = sum_{s=0..L-1} h[s] u[(t - s) mod L].
+ * L is a power of two, 32 <= L <= 16384 (one launch, each sequence on one
+ * SM); other L return HYENA_ERR_UNSUPPORTED.
+ * hyena_filter_rfft_circular: H [N][D][L/2] complex64, the L-point DFT X of
+ * each filter without padding, packed like hyena_filter_rfft's spectra:
+ * slot 0 = (X[0], X[L/2]) (both real), slot k = X[k] for 1 <= k < L/2.
+ * hyena_fftconv_gate_forward_circular: v, x_n, y [B][D][L] io, H as above,
+ * bias [N][D]; no workspace.  Alignment: h, H, v, x_n, y 16 bytes; bias 4. */
+HYENA_API hyena_status_t hyena_filter_rfft_circular(const float* h, int N, int D, int L, float* H,
+                                                    void* stream);
+HYENA_API hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* const* x,
+                                                             const float* H, const float* bias, int B,
+                                                             int D, int L, int N, hyena_dtype_t io,
+                                                             void* y, void* stream);
+
 /* Size of the scratch array built into the library for
  * hyena_fftconv_gate_forward_noalloc (16 MB on every device that loads the
  * library, held until the process exits). */

@@ -102,7 +102,13 @@ __device__ __forceinline__ void unsplit_pair(float2 y1, float2 y2, float2 w, flo
 // complex slots; slot k (1 <= k < L) holds DFT bin k, slot 0 holds
 // (bin 0, bin L), both real.  Rows are L * 8 bytes, so 16-byte aligned.
 
-template <int LOG2M>
+// PAD = true: the causal (linear) convolution; the real sequence of length
+// L = M is zero-padded to 2M, so only half the packed inputs are non-zero
+// and only half the outputs are kept.  PAD = false: the circular
+// convolution of a real sequence of length 2M ("Handling Boundaries":
+// circular convolutions for periodic systems), all packed inputs and
+// outputs used.
+template <int LOG2M, bool PAD = true>
 struct Fft1d {
     using P = Plan1d<LOG2M>;
     static constexpr int M = 1 << LOG2M;
@@ -121,6 +127,9 @@ struct Fft1d {
     // holds x_n (at most M/2 float2).
     static constexpr bool H_IN_EXCHANGE = sizeof(float2) * G * (SMEM_SEQ + M) > 227 * 1024;
     static constexpr int STAGE_SEQ = H_IN_EXCHANGE ? M / 2 : M;  // staging buffer, float2
+    // packed pairs of real samples per sequence: L/2 = M/2 (causal), M (circular)
+    static constexpr int SEQ = PAD ? M / 2 : M;
+    static_assert(PAD || !H_IN_EXCHANGE, "circular mode needs the x staging buffer of M pairs");
     static constexpr size_t SMEM_BYTES = sizeof(float2) * G * (SMEM_SEQ + STAGE_SEQ);
     static constexpr size_t SMEM_BYTES_FFT = sizeof(float2) * G * SMEM_SEQ;
     // resident CTAs per SM the register budget is sized for: 168 registers
@@ -241,7 +250,7 @@ struct Fft1d {
     // folded layout.
     static __device__ __forceinline__ void forward(float2* a, float2* sm, int t)
     {
-        pass_first<P::RF, -1, true>(a, sm, t);
+        pass_first<P::RF, -1, PAD>(a, sm, t);
         pass_mid<P::RM1, P::RF, -1>(a, sm, t);
         pass_mid<P::RM2, P::RF * P::RM1, -1>(a, sm, t);
         pass_last<P::RL, -1, false>(a, sm, t);
@@ -254,7 +263,7 @@ struct Fft1d {
         pass_first<P::RL, +1, false>(a, sm, t);
         pass_mid<P::RM2, P::RL, +1>(a, sm, t);
         pass_mid<P::RM1, P::RL * P::RM2, +1>(a, sm, t);
-        pass_last<P::RF, +1, true>(a, sm, t);
+        pass_last<P::RF, +1, PAD>(a, sm, t);
     }
 
     // One pair (k, M-k) of the real-FFT split, the spectral multiply with
@@ -386,7 +395,7 @@ struct Fft1d {
             unit_cols<R>(t + c * T, j[0], j[1]);
             static_for<2>([&](auto hh) {
                 constexpr int h = decltype(hh)::value;
-                static_for<R / 2>([&](auto rr) {
+                static_for<PAD ? R / 2 : R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
                     f((2 * c + h) * R + r, j[h] + r * (M / R));
                 });
@@ -399,16 +408,19 @@ struct Fft1d {
 // Shared memory per sequence: the padded exchange buffer of the FFT passes
 // and a staging buffer that receives H_n (during the forward FFT) and then
 // x_n (during the inverse FFT) through asynchronous copies.
-template <int LOG2M, typename IO>
-__global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS, Fft1d<LOG2M>::MIN_BLOCKS)
+// PER_SAMPLE: a spectrum set per sample (input-dependent filters), at
+// H + b * H_bstride; otherwise one set shared by the batch.
+template <int LOG2M, typename IO, bool PAD = true, bool PER_SAMPLE = false>
+__global__ void __launch_bounds__(Fft1d<LOG2M, PAD>::THREADS, Fft1d<LOG2M, PAD>::MIN_BLOCKS)
 fused1d_kernel(Fused1dArgs args)
 {
     grid_dependency_begin();
-    using F = Fft1d<LOG2M>;
+    using F = Fft1d<LOG2M, PAD>;
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;
     constexpr int M = F::M, E = F::E, T = F::T;
-    constexpr int X_BYTES = M * (int)sizeof(PT) / 2;    // one sequence of x_n
+    constexpr int SEQ = F::SEQ;                          // pairs of samples per sequence
+    constexpr int X_BYTES = SEQ * (int)sizeof(PT);       // one sequence of x_n
     extern __shared__ __align__(16) float2 smem_dyn[];
 
     const int g = threadIdx.x / T, t = threadIdx.x % T;
@@ -422,14 +434,14 @@ fused1d_kernel(Fused1dArgs args)
     float2* sm = smem_dyn + g * F::SMEM_SEQ;
     float2* stage = smem_dyn + F::G * F::SMEM_SEQ + g * F::STAGE_SEQ;
 
-    const float2* Hb = args.H + (size_t)b * args.H_bstride;    // this sample's spectra
+    const float2* Hb = PER_SAMPLE ? args.H + (size_t)b * args.H_bstride : args.H;   // this sample's spectra
     // H_0 (or x_1) is in flight while v is loaded and transformed
     if constexpr (!F::H_IN_EXCHANGE)
         cp_async_row(stage, Hb + (size_t)d * M, M * 8, t, T);
 
     float2 a[E];
     {
-        const PT* vp = reinterpret_cast<const PT*>(args.v) + seq * (M / 2);
+        const PT* vp = reinterpret_cast<const PT*>(args.v) + seq * SEQ;
         F::for_each_io(t, [&](int i, int m) { a[i] = IOP::load(vp + m); });
     }
     for (int n = 0; n < args.N; ++n) {
@@ -439,7 +451,7 @@ fused1d_kernel(Fused1dArgs args)
 #pragma unroll
         for (int i = 1; i < kMaxOrder; ++i)
             if (i == n) xn = args.x[i];
-        const PT* xg = reinterpret_cast<const PT*>(xn) + seq * (M / 2);
+        const PT* xg = reinterpret_cast<const PT*>(xn) + seq * SEQ;
         const float2* Hg = Hb + ((size_t)n * args.D + d) * M;
         const float bias = __ldg(args.bias + n * args.D + d);
         const float2* Hs;
@@ -473,18 +485,19 @@ fused1d_kernel(Fused1dArgs args)
                 cp_async_row(stage, Hb + ((size_t)(n + 1) * args.D + d) * M, M * 8, t, T);
     }
     if (active) {
-        PT* yp = reinterpret_cast<PT*>(args.y) + seq * (M / 2);
+        PT* yp = reinterpret_cast<PT*>(args.y) + seq * SEQ;
         F::for_each_io(t, [&](int i, int m) { IOP::store(yp + m, a[i]); });
     }
 }
 
-// Filter spectra in the packed layout: the DFT of h[row] zero-padded to 2L.
-template <int LOG2M>
-__global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS)
+// Filter spectra in the packed layout: the DFT of h[row] zero-padded to 2L
+// (PAD), or of the unpadded row of length 2M (circular).
+template <int LOG2M, bool PAD = true>
+__global__ void __launch_bounds__(Fft1d<LOG2M, PAD>::THREADS)
 rfft1d_kernel(Rfft1dArgs args)
 {
     grid_dependency_begin();
-    using F = Fft1d<LOG2M>;
+    using F = Fft1d<LOG2M, PAD>;
     constexpr int M = F::M, E = F::E, T = F::T, R = F::P::RL, NCOL = M / R;
     extern __shared__ __align__(16) float2 smem_dyn[];
 
@@ -496,7 +509,7 @@ rfft1d_kernel(Rfft1dArgs args)
 
     float2 a[E];
     {
-        const float2* hp = reinterpret_cast<const float2*>(args.h) + row * (M / 2);
+        const float2* hp = reinterpret_cast<const float2*>(args.h) + row * F::SEQ;
         F::for_each_io(t, [&](int i, int m) { a[i] = __ldg(hp + m); });
     }
     F::forward(a, sm, t);

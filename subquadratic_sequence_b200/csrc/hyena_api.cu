@@ -2,6 +2,7 @@
 // argument validation on the host, then the dispatchers of launch.cuh.
 #include <stdint.h>
 
+#include "k_circular.cuh"
 #include "k_fft2d.cuh"
 #include "launch.cuh"
 
@@ -314,6 +315,55 @@ hyena_status_t forward_impl(const void* v, const void* const* x, const float* h,
 }  // namespace
 
 extern "C" {
+
+hyena_status_t hyena_filter_rfft_circular(const float* h, int N, int D, int L, float* H, void* stream)
+{
+    if (!h || !H || N < 1 || D < 1 || L < 1) return HYENA_ERR_INVALID_ARG;
+    const int k = exact_log2(L);
+    if (k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1) return HYENA_ERR_UNSUPPORTED;
+    if (!aligned(h, 16) || !aligned(H, 16)) return HYENA_ERR_INVALID_ARG;
+    if ((long)N * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    if (overlap(h, sizeof(float) * (size_t)N * D * L, H, sizeof(float2) * (size_t)N * D * (L / 2)))
+        return HYENA_ERR_INVALID_ARG;
+    Rfft1dArgs ra;
+    ra.h = h;
+    ra.H = reinterpret_cast<float2*>(H);
+    ra.rows = N * D;
+    return dispatch_rfft_circ(k - 1, ra, (cudaStream_t)stream);
+}
+
+hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* const* x, const float* H,
+                                                   const float* bias, int B, int D, int L, int N,
+                                                   hyena_dtype_t io, void* y, void* stream)
+{
+    if (!v || !x || !H || !bias || !y) return HYENA_ERR_INVALID_ARG;
+    if (B < 1 || D < 1 || N < 1 || L < 1) return HYENA_ERR_INVALID_ARG;
+    if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_ORDER || (long)B * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    const int k = exact_log2(L);
+    if (k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1) return HYENA_ERR_UNSUPPORTED;
+    for (int n = 0; n < N; ++n)
+        if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(v, 16) || !aligned(y, 16) || !aligned(H, 16) || !aligned(bias, 4))
+        return HYENA_ERR_INVALID_ARG;
+    const size_t act = (size_t)B * D * L * io_bytes(io);
+    if (overlap(y, act, v, act) || overlap(y, act, H, sizeof(float2) * (size_t)N * D * (L / 2)) ||
+        overlap(y, act, bias, sizeof(float) * N * D))
+        return HYENA_ERR_INVALID_ARG;
+    for (int n = 0; n < N; ++n)
+        if (overlap(y, act, x[n], act)) return HYENA_ERR_INVALID_ARG;
+    Fused1dArgs a = {};
+    a.v = v;
+    for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
+    a.y = y;
+    a.H = reinterpret_cast<const float2*>(H);
+    a.bias = bias;
+    a.B = B;
+    a.D = D;
+    a.N = N;
+    cudaStream_t st = (cudaStream_t)stream;
+    return io == HYENA_BF16 ? dispatch_fused_circ_bf16(k - 1, a, st) : dispatch_fused_circ_f32(k - 1, a, st);
+}
 
 size_t hyena_fftconv_backward_workspace_size(int D, int L, int N)
 {

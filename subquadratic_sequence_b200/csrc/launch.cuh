@@ -74,6 +74,8 @@ inline long wave_seqs(long nseq, long L)
 
 hyena_status_t dispatch_fused_f32(int log2m, const Fused1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_fused_bf16(int log2m, const Fused1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_fused_ps_f32(int log2m, const Fused1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_fused_ps_bf16(int log2m, const Fused1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_rfft(int log2m, const Rfft1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_fourstep_f32(int log2m, const FourStepArgs& a, int N, float2* scratch,
                                      cudaStream_t st);

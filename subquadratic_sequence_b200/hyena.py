@@ -67,6 +67,8 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv_backward_workspace_size": ([i, i, i], sz),
         "hyena_fftconv_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp,
                                          ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
+        "hyena_filter_rfft_circular": ([vp, i, i, i, vp, vp], i),
+        "hyena_fftconv_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp], i),
         "hyena_filter_rfft2d": ([vp, i, i, i, i, vp, vp], i),
         "hyena_fftconv2d_workspace_size": ([i, i, i, i, i, i, i], sz),
         "hyena_fftconv2d_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
@@ -294,6 +296,33 @@ def hyena_fftconv_gate_backward(v: torch.Tensor, xs, bias: torch.Tensor, H: torc
         ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return dv, dxs, dh, db
+
+
+def hyena_filter_rfft_circular(h: torch.Tensor, *, out=None, stream=None):
+    """Circular-mode spectra H [N][D][L/2] complex64 of filters h [N][D][L]
+    (the L-point DFT without padding, packed: slot 0 = (bin 0, bin L/2))."""
+    N, D, L = h.shape
+    if out is None:
+        out = torch.empty((N, D, L // 2), device=h.device, dtype=torch.complex64)
+    _check("hyena_filter_rfft_circular", LIB.hyena_filter_rfft_circular(
+        ctypes.c_void_p(_dev(h, torch.float32, "h")), N, D, L,
+        ctypes.c_void_p(_dev(out, torch.complex64, "H")), _stream(stream)))
+    return out
+
+
+def hyena_fftconv_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor, *,
+                                        out=None, stream=None):
+    """The order-N forward with circular convolutions of length L."""
+    B, D, L = v.shape
+    N = len(xs)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    _check("hyena_fftconv_gate_forward_circular", LIB.hyena_fftconv_gate_forward_circular(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io_dtype(v),
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), _stream(stream)))
+    return out
 
 
 def hyena_filter_rfft2d(h: torch.Tensor, *, out=None, stream=None):

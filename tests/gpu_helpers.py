@@ -32,7 +32,10 @@ def unpack_spectrum(Hp: np.ndarray) -> np.ndarray:
 
 
 def rel_max_err(got, ref) -> float:
-    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    """max |got - ref| / max |ref|, in complex128 when either side is complex."""
+    cplx = np.iscomplexobj(got) or np.iscomplexobj(ref)
+    dt = np.complex128 if cplx else np.float64
+    got, ref = np.asarray(got, dt), np.asarray(ref, dt)
     return float(np.max(np.abs(got - ref)) / np.max(np.abs(ref)))
 
 

@@ -160,6 +160,20 @@ def test_backward_rejects_bad_arguments(lib):
     assert bwd(lib, dxs=(P(11), P(8))) == INVALID
 
 
+def test_circular_rejects_bad_arguments(lib):
+    xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
+    f = lib.hyena_fftconv_gate_forward_circular
+    assert f(P(0), xs, P(3), P(4), 2, 3, 16, 2, F32, P(5), None) == UNSUPPORTED   # L < 32
+    assert f(P(0), xs, P(3), P(4), 2, 3, 1 << 15, 2, F32, P(5), None) == UNSUPPORTED
+    assert f(P(0), xs, P(3), P(4), 2, 3, 96, 2, F32, P(5), None) == UNSUPPORTED   # not a power of two
+    assert f(None, xs, P(3), P(4), 2, 3, 64, 2, F32, P(5), None) == INVALID
+    assert f(P(0), xs, P(3), P(4), 2, 3, 64, 2, F32, P(0), None) == INVALID       # y aliases v
+    r = lib.hyena_filter_rfft_circular
+    assert r(P(0), 2, 3, 16, P(1), None) == UNSUPPORTED
+    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + BIG + 8), None) == INVALID
+    assert r(P(0), 2, 3, 64, P(0), None) == INVALID                               # H overlaps h
+
+
 def test_filter_rfft_rejects_bad_arguments(lib):
     r = lib.hyena_filter_rfft
     assert r(None, 2, 3, 64, P(1), None, 0, None) == INVALID
