@@ -21,8 +21,10 @@
 //   B. for n = N..1: dx_n and e from g; E = DFT(e); accumulate E conj(Z)
 //      into the channel's dh spectrum (only this group touches it, so a
 //      plain read-modify-write); g = inverse of (conj(H_n) + b_n) E.
-// After the last sequence the group turns each accumulated spectrum into
-// dh_n (inverse real FFT, first L lags) and db_n = dh_n[0].
+// Both phases run through one copy of the FFT code (a step loop), which
+// halves the kernel's instruction footprint.  A second launch turns each
+// accumulated spectrum into dh_n (inverse real FFT, first L lags) and
+// db_n = dh_n[0].
 #pragma once
 
 #include "fused1d.cuh"
@@ -67,104 +69,78 @@ backward1d_kernel(Backward1dArgs args)
     float2* wc = args.wc + (size_t)d * N * (M / 2);
     // index of io register i among the thread's E/2 io registers
     auto io_slot = [](int i) { return (i / RF) * (RF / 2) + i % RF; };
-    // x_{n+1} (0-based n) with constant indices into the parameter array
-    auto x_of = [&](int n) {
-        const void* p = args.x[0];
+    auto pick = [](const void* const* arr, int n) {
+        const void* p = arr[0];
 #pragma unroll
         for (int i = 1; i < kMaxOrder; ++i)
-            if (i == n) p = args.x[i];
-        return reinterpret_cast<const PT*>(p);
-    };
-    // H_n into shared memory (into the exchange buffer at the largest size,
-    // once the forward FFT has finished with it); returns the staged row
-    auto stage_h_before = [&](int n) {
-        if constexpr (!F::H_IN_EXCHANGE)
-            cp_async_row(stage, args.H + ((size_t)n * D + d) * M, M * 8, t, T);
-    };
-    auto stage_h_after = [&](int n) -> const float2* {
-        if constexpr (F::H_IN_EXCHANGE) {
-            cp_async_row(sm, args.H + ((size_t)n * D + d) * M, M * 8, t, T);
-            cp_async_wait_all();
-            __syncthreads();
-            return sm;
-        } else {
-            cp_async_wait_all();
-            __syncthreads();
-            return stage;
-        }
+            if (i == n) p = arr[i];
+        return p;
     };
 
     float2 a[E];
     for (int b = 0; b < args.B; ++b) {
         const size_t seq = (size_t)b * D + d;
-        // ---------------------------------------------- A. forward again
         {
             const PT* vp = reinterpret_cast<const PT*>(args.v) + seq * (M / 2);
             F::for_each_io(t, [&](int i, int m) { a[i] = IOP::load(vp + m); });
         }
-        for (int n = 0; n < N; ++n) {
+        // One step per order, forwards (A) and then backwards (B), through a
+        // single FFT code path:
+        //   A_n: a = z_n;  save Z_n = DFT(z_n);  c_{n+1} = inverse((H_n + b_n) Z_n),
+        //        saved; a = x_{n+1} c_{n+1} (after the last order: a = dy)
+        //   B_n: a = g;  dx_{n+1} = g c_{n+1};  a = e = g x_{n+1};  E = DFT(e);
+        //        dh spectrum += E conj(Z_n);  a = g = inverse((conj H_n + b_n) E)
+        for (int s = 0; s < 2 * N; ++s) {
+            const bool back = s >= N;
+            const int n = back ? 2 * N - 1 - s : s;
             const float bias = __ldg(args.bias + n * D + d);
-            stage_h_before(n);
-            F::forward(a, sm, t);
-            if (active)
-                static_for<E>([&](auto ii) {
-                    constexpr int i = decltype(ii)::value;
-                    wz[(size_t)n * M + i * T + t] = a[i];
-                });
-            const float2* Hs = stage_h_after(n);
-            F::spectral(a, Hs, bias, t);
-            __syncthreads();                                  // H_n consumed
-            F::inverse(a, sm, t);
-            const PT* xp = x_of(n) + seq * (M / 2);
-            F::for_each_io(t, [&](int i, int m) {
-                if (active) wc[(size_t)n * (M / 2) + io_slot(i) * T + t] = a[i];
-                if (n + 1 < N) {
-                    const float2 xv = IOP::load(xp + m);
-                    a[i] = make_float2(a[i].x * xv.x, a[i].y * xv.y);
-                }
-            });
-        }
-        // ---------------------------------------------- B. backward
-        {
-            const PT* gp = reinterpret_cast<const PT*>(args.dy) + seq * (M / 2);
-            F::for_each_io(t, [&](int i, int m) { a[i] = IOP::load(gp + m); });
-        }
-        for (int n = N - 1; n >= 0; --n) {
-            const float bias = __ldg(args.bias + n * D + d);
-            {
-                // dx_n = g c_n, e = g x_n  (g in the io registers)
-                const PT* xp = x_of(n) + seq * (M / 2);
-                void* dxn = args.dx[0];
-#pragma unroll
-                for (int i = 1; i < kMaxOrder; ++i)
-                    if (i == n) dxn = args.dx[i];
-                PT* dxp = reinterpret_cast<PT*>(dxn) + seq * (M / 2);
+            const PT* xp = reinterpret_cast<const PT*>(pick(args.x, n)) + seq * (M / 2);
+            float2* wcn = wc + (size_t)n * (M / 2);
+            if (back) {
+                PT* dxp = reinterpret_cast<PT*>(const_cast<void*>(pick(reinterpret_cast<const void* const*>(args.dx), n)))
+                          + seq * (M / 2);
+                // all loads first, then the stores: one latency, not one per value
+                float2 c[E / 2], xv[E / 2];
                 F::for_each_io(t, [&](int i, int m) {
-                    const float2 c = wc[(size_t)n * (M / 2) + io_slot(i) * T + t];
-                    const float2 xv = IOP::load(xp + m);
-                    if (active) IOP::store(dxp + m, make_float2(a[i].x * c.x, a[i].y * c.y));
-                    a[i] = make_float2(a[i].x * xv.x, a[i].y * xv.y);
+                    c[io_slot(i)] = wcn[io_slot(i) * T + t];
+                    xv[io_slot(i)] = IOP::load(xp + m);
+                });
+                F::for_each_io(t, [&](int i, int m) {
+                    const int k = io_slot(i);
+                    if (active) IOP::store(dxp + m, make_float2(a[i].x * c[k].x, a[i].y * c[k].y));
+                    a[i] = make_float2(a[i].x * xv[k].x, a[i].y * xv[k].y);
                 });
             }
-            stage_h_before(n);
-            F::forward(a, sm, t);                            // a = DFT(e), packed
-            // dh spectrum: acc[k] (+)= E[k] conj(Z_{n-1}[k]) over the 2L-point bins
-            if (active) {
+            if constexpr (!F::H_IN_EXCHANGE)
+                cp_async_row(stage, args.H + ((size_t)n * D + d) * M, M * 8, t, T);
+            F::forward(a, sm, t);
+            if (!back) {
+                if (active)
+                    static_for<E>([&](auto ii) {
+                        constexpr int i = decltype(ii)::value;
+                        wz[(size_t)n * M + i * T + t] = a[i];
+                    });
+            } else if (active) {
+                // dh spectrum: acc[k] (+)= E[k] conj(Z_n[k]) over the 2L-point bins
                 float2* acc = args.acc + ((size_t)n * D + d) * M;
                 const float2* zr = wz + (size_t)n * M;
                 const bool first = b == 0;
+                float2 z[E];
+                static_for<E>([&](auto ii) {
+                    constexpr int i = decltype(ii)::value;
+                    z[i] = zr[i * T + t];
+                });
                 F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
                     const float2 e1 = a[i1], e2 = a[i2];
-                    const float2 z1 = zr[i1 * T + t], z2 = zr[i2 * T + t];
                     if (kind == 1) {
                         // slot 0: bins 0 and M, both real
-                        const float2 p = make_float2((e1.x + e1.y) * (z1.x + z1.y),
-                                                     (e1.x - e1.y) * (z1.x - z1.y));
+                        const float2 p = make_float2((e1.x + e1.y) * (z[i1].x + z[i1].y),
+                                                     (e1.x - e1.y) * (z[i1].x - z[i1].y));
                         acc[0] = first ? p : cadd(acc[0], p);
                     } else {
                         float2 E1, E2, Z1, Z2;
                         split_pair(e1, e2, w, E1, E2);
-                        split_pair(z1, z2, w, Z1, Z2);
+                        split_pair(z[i1], z[i2], w, Z1, Z2);
                         const float2 p1 = cmulc(E1, Z1);
                         acc[k] = first ? p1 : cadd(acc[k], p1);
                         if (kind == 0) {
@@ -174,44 +150,80 @@ backward1d_kernel(Backward1dArgs args)
                     }
                 });
             }
-            const float2* Hs = stage_h_after(n);
-            F::template spectral<true>(a, Hs, bias, t);      // (conj(H_n) + b_n) E, re-packed
+            const float2* Hs = stage;
+            if constexpr (F::H_IN_EXCHANGE) {
+                cp_async_row(sm, args.H + ((size_t)n * D + d) * M, M * 8, t, T);
+                Hs = sm;
+            }
+            cp_async_wait_all();
+            __syncthreads();                                  // H_n visible
+            F::template spectral<false, true>(a, Hs, bias, t, back ? -1.0f : 1.0f);
             __syncthreads();                                  // H_n consumed
-            F::inverse(a, sm, t);                            // io registers: g = dz_{n-1}
+            F::inverse(a, sm, t);
+            if (!back) {
+                // a = c_{n+1}: save it, then z_{n+1} = x_{n+1} c_{n+1}, or g = dy
+                const PT* gp = reinterpret_cast<const PT*>(args.dy) + seq * (M / 2);
+                F::for_each_io(t, [&](int i, int m) {
+                    if (active) wcn[io_slot(i) * T + t] = a[i];
+                    if (n + 1 < N) {
+                        const float2 x = IOP::load(xp + m);
+                        a[i] = make_float2(a[i].x * x.x, a[i].y * x.y);
+                    } else {
+                        a[i] = IOP::load(gp + m);
+                    }
+                });
+            }
         }
         if (active) {
             PT* dvp = reinterpret_cast<PT*>(args.dv) + seq * (M / 2);
             F::for_each_io(t, [&](int i, int m) { IOP::store(dvp + m, a[i]); });
         }
     }
-    // ------------------------------------------ dh_n and db_n of channel d
+}
+
+// dh_n[d] and db_n[d] from the accumulated spectra: one group per row
+// (n, d): the inverse real FFT of the packed spectrum (scale 1/P), the
+// first L lags, and db = dh[0].
+template <int LOG2M>
+__global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS)
+dh_finalize_kernel(Backward1dArgs args)
+{
+    grid_dependency_begin();
+    using F = Fft1d<LOG2M>;
+    constexpr int M = F::M, E = F::E, T = F::T;
+    extern __shared__ __align__(16) float2 smem_dyn[];
+    const int g = threadIdx.x / T, t = threadIdx.x % T;
+    const int rows = args.N * args.D;
+    const int row_raw = blockIdx.x * F::G + g;
+    const bool active = row_raw < rows;
+    const int row = active ? row_raw : rows - 1;
+    float2* sm = smem_dyn + g * F::SMEM_SEQ;
+    const float2* acc = args.acc + (size_t)row * M;
     constexpr float s = 1.0f / (2.0f * (float)M);           // 1/P of the inverse DFT
-    for (int n = 0; n < N; ++n) {
-        const float2* acc = args.acc + ((size_t)n * D + d) * M;
-        F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
-            float2 z1, z2;
-            if (kind == 1) {
-                const float2 p = acc[0];
-                unsplit_pair(make_float2(p.x, 0.0f), make_float2(p.y, 0.0f), w, s, z1, z2);
-                a[i1] = z1;
-            } else if (kind == 2) {
-                const float2 y = acc[k];
-                unsplit_pair(y, y, w, s, z1, z2);
-                a[i1] = z1;
-            } else {
-                unsplit_pair(acc[k], acc[M - k], w, s, z1, z2);
-                a[i1] = z1;
-                a[i2] = z2;
-            }
-        });
-        F::inverse(a, sm, t);
-        if (active) {
-            float2* dhp = reinterpret_cast<float2*>(args.dh + ((size_t)n * D + d) * M);
-            F::for_each_io(t, [&](int i, int m) {
-                dhp[m] = a[i];
-                if (m == 0) args.dbias[n * D + d] = a[i].x;   // db_n = dh_n[0]
-            });
+    float2 a[E];
+    F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
+        float2 z1, z2;
+        if (kind == 1) {
+            const float2 p = acc[0];
+            unsplit_pair(make_float2(p.x, 0.0f), make_float2(p.y, 0.0f), w, s, z1, z2);
+            a[i1] = z1;
+        } else if (kind == 2) {
+            const float2 y = acc[k];
+            unsplit_pair(y, y, w, s, z1, z2);
+            a[i1] = z1;
+        } else {
+            unsplit_pair(acc[k], acc[M - k], w, s, z1, z2);
+            a[i1] = z1;
+            a[i2] = z2;
         }
+    });
+    F::inverse(a, sm, t);
+    if (active) {
+        float2* dhp = reinterpret_cast<float2*>(args.dh + (size_t)row * M);
+        F::for_each_io(t, [&](int i, int m) {
+            dhp[m] = a[i];
+            if (m == 0) args.dbias[row] = a[i].x;             // db_n = dh_n[0]
+        });
     }
 }
 

@@ -292,10 +292,18 @@ struct Fft1d {
     // Spectral step on the RL folded layout for one order; Hs is the
     // packed spectrum row staged in shared memory.  CONJ: multiply by
     // conj(H) + b instead (the adjoint, used by the backward pass).
-    template <bool CONJ = false>
-    static __device__ __forceinline__ void spectral(float2* a, const float2* Hs, float bias, int t)
+    template <bool CONJ = false, bool SIGNED = false>
+    static __device__ __forceinline__ void spectral(float2* a, const float2* Hs, float bias, int t,
+                                                    float him = 1.0f)
     {
-        auto hv = [&](int k) { return CONJ ? cconj(Hs[k]) : Hs[k]; };
+        // SIGNED: the imaginary part of H times him (+1: H, -1: conj(H)),
+        // chosen at run time
+        auto hv = [&](int k) {
+            float2 h = Hs[k];
+            if (CONJ) h.y = -h.y;
+            if (SIGNED) h.y *= him;
+            return h;
+        };
         constexpr int R = P::RL, NCOL = M / R;
         static_for<E / (2 * R)>([&](auto cc) {
             constexpr int c = decltype(cc)::value;

@@ -11,8 +11,12 @@ template <int LOG2M, typename IO>
 hyena_status_t launch_backward(const Backward1dArgs& a, cudaStream_t st)
 {
     using F = Fft1d<LOG2M>;
-    return launch(backward1d_kernel<LOG2M, IO>, (unsigned)((a.D + F::G - 1) / F::G), F::THREADS,
-                  F::SMEM_BYTES, st, a);
+    hyena_status_t s = launch(backward1d_kernel<LOG2M, IO>, (unsigned)((a.D + F::G - 1) / F::G),
+                              F::THREADS, F::SMEM_BYTES, st, a);
+    if (s != HYENA_OK) return s;
+    const int rows = a.N * a.D;
+    return launch(dh_finalize_kernel<LOG2M>, (unsigned)((rows + F::G - 1) / F::G), F::THREADS,
+                  F::SMEM_BYTES_FFT, st, a);
 }
 
 template <typename IO>
