@@ -262,9 +262,10 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_noalloc(const void* v, const
  *          hyena_fftconv_backward_workspace_size(D, L, N) bytes (20 N D L),
  *          256-byte aligned; nothing in it needs to start at zero.
  * L is a power of two, 16 <= L <= 16384 (HYENA_ERR_UNSUPPORTED above);
- * 1 <= N <= HYENA_MAX_ORDER.  One launch: a group of threads owns a
+ * 1 <= N <= HYENA_MAX_ORDER.  Two launches: a group of threads owns a
  * channel and walks its B sequences (the forward again, then the orders
- * backwards), so dh and dbias need no atomics and are deterministic.
+ * backwards), accumulating the channel's dh spectra, so dh and dbias need
+ * no atomics and are deterministic; a second launch inverts those spectra. 
  * Alignment: v, x_n, dy, dv, dx_n, H, dh 16 bytes; bias, dbias 4.  Outputs
  * must not overlap each other, any input or the workspace. */
 HYENA_API size_t hyena_fftconv_backward_workspace_size(int D, int L, int N);
