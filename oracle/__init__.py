@@ -62,6 +62,7 @@ def _load():
         "oracle_hyena_backward": [dp, dp, dp, dp, dp, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_filter_gen_film": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, d, i, dp],
         "oracle_cconv": [dp, dp, l, i, dp],
+        "oracle_filter_gen_film_2d": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, i, d, i, dp],
         "oracle_rfft_circ": [dp, l, l, dp, dp],
         "oracle_hyena_forward_circular": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
     }
@@ -286,3 +287,27 @@ def hyena_forward_circular(v, x, h, bias, route="fft", threads=None) -> np.ndarr
                                                _route(route), threads or default_threads(), _ptr(y))
     _check(rc, "oracle_hyena_forward_circular")
     return y
+
+
+def filter_gen_film_2d(W1, W2, W3, Wout, omega, gamma, beta, window, gaussian, N, C, H, W, n_bands=8,
+                       width=64, decay_div=64.0, threads=None) -> np.ndarray:
+    """Per-sample 2-D filters h [B][N][C][H][W]: the FiLM-modulated sine
+    layers on the 2-D features; window [C] is alpha (separable exponential
+    decay) or sigma (Gaussian exp(-(ty^2 + tx^2) / (2 sigma^2)))."""
+    W1, W2, W3, Wout, omega, gamma, beta, window = map(
+        _f64, (W1, W2, W3, Wout, omega, gamma, beta, window))
+    B = gamma.shape[0]
+    h = np.empty((B, N, C, H, W))
+    rc = _load().oracle_filter_gen_film_2d(_ptr(W1), _ptr(W2), _ptr(W3), _ptr(Wout), _ptr(omega),
+                                           _ptr(gamma), _ptr(beta), _ptr(window), int(bool(gaussian)),
+                                           B, N, C, H, W, n_bands, width, float(decay_div),
+                                           threads or default_threads(), _ptr(h))
+    _check(rc, "oracle_filter_gen_film_2d")
+    return h
+
+
+def hyena_forward_2d_per_sample(v, x, h, bias, route="fft", threads=None) -> np.ndarray:
+    """The 2-D forward with a filter set per sample, h [B][N][C][H][W]."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    return np.concatenate([hyena_forward_2d(v[b:b + 1], x[:, b:b + 1], h[b], bias, route, threads)
+                           for b in range(v.shape[0])])

@@ -324,6 +324,100 @@ done:
     return NULL;
 }
 
+/* Input-dependent 2-D filters: the FiLM-modulated sine layers of
+ * oracle_filter_gen_film on the 2-D features, h[B][N][C][H][W]; the
+ * window is the separable exponential decay of oracle_filter_gen_2d
+ * (gaussian = 0, win = alpha) or the Gaussian exp(-(ty^2 + tx^2) /
+ * (2 sigma_c^2)) (gaussian = 1, win = sigma). */
+typedef struct {
+    const double *W1, *W2, *W3, *Wout, *omega, *gamma, *beta, *win;
+    int gaussian, B, N, C, H, W, n_bands, width;
+    double decay_div;
+    double *h;
+    int p0, p1;
+    int status;
+} fgf2_job;
+
+static void *filter_gen_film_2d_worker(void *arg)
+{
+    fgf2_job *j = (fgf2_job *)arg;
+    const int n_in = 2 + 4 * j->n_bands, w = j->width, n_out = j->N * j->C;
+    const long HW = (long)j->H * j->W;
+    double *phi = malloc(sizeof(double) * n_in);
+    double *a1 = malloc(sizeof(double) * w), *a2 = malloc(sizeof(double) * w);
+    double *a3 = malloc(sizeof(double) * w), *o = malloc(sizeof(double) * n_out);
+    if (!phi || !a1 || !a2 || !a3 || !o) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (int b = 0; b < j->B; ++b) {
+        const double *g = j->gamma + (long)b * 3 * w, *be = j->beta + (long)b * 3 * w;
+        for (int p = j->p0; p < j->p1; ++p) {
+            const int iy = p / j->W, ix = p % j->W;
+            const double ty = (double)iy / (double)j->H, tx = (double)ix / (double)j->W;
+            phi[0] = ty;
+            phi[1] = tx;
+            for (int k = 1; k <= j->n_bands; ++k) {
+                phi[2 * k] = sin(2.0 * ORACLE_PI * k * ty);
+                phi[2 * k + 1] = cos(2.0 * ORACLE_PI * k * ty);
+                phi[2 * j->n_bands + 2 * k] = sin(2.0 * ORACLE_PI * k * tx);
+                phi[2 * j->n_bands + 2 * k + 1] = cos(2.0 * ORACLE_PI * k * tx);
+            }
+            matvec(j->W1, w, n_in, phi, a1);
+            film_sin(a1, w, j->omega, g, be);
+            matvec(j->W2, w, w, a1, a2);
+            film_sin(a2, w, j->omega + w, g + w, be + w);
+            matvec(j->W3, w, w, a2, a3);
+            film_sin(a3, w, j->omega + 2 * w, g + 2 * w, be + 2 * w);
+            matvec(j->Wout, n_out, w, a3, o);
+            for (int n = 0; n < j->N; ++n)
+                for (int c = 0; c < j->C; ++c) {
+                    const double s = j->win[c];
+                    const double window =
+                        j->gaussian ? exp(-(ty * ty + tx * tx) / (2.0 * s * s))
+                                    : exp(-s * ty * (double)j->H / j->decay_div) *
+                                          exp(-s * tx * (double)j->W / j->decay_div);
+                    j->h[(((long)b * j->N + n) * j->C + c) * HW + p] = o[n * j->C + c] * window;
+                }
+        }
+    }
+    j->status = ORACLE_OK;
+done:
+    free(phi); free(a1); free(a2); free(a3); free(o);
+    return NULL;
+}
+
+int oracle_filter_gen_film_2d(const double *W1, const double *W2, const double *W3,
+                              const double *Wout, const double *omega, const double *gamma,
+                              const double *beta, const double *win, int gaussian, int B, int N,
+                              int C, int H, int W, int n_bands, int width, double decay_div,
+                              int nthreads, double *h)
+{
+    if (!W1 || !W2 || !W3 || !Wout || !omega || !gamma || !beta || !win || !h || B < 1 ||
+        N < 1 || C < 1 || H < 1 || W < 1 || n_bands < 0 || width < 1 || !(decay_div > 0.0))
+        return ORACLE_EBADARG;
+    const int HW = H * W;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > HW) nthreads = HW;
+    fgf2_job *jobs = calloc(nthreads, sizeof(fgf2_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        fgf2_job j = {W1, W2, W3, Wout, omega, gamma, beta, win, gaussian, B, N, C, H, W, n_bands,
+                      width, decay_div, h, (int)((long)HW * k / nthreads),
+                      (int)((long)HW * (k + 1) / nthreads), 0};
+        jobs[k] = j;
+        pthread_create(&tid[k], NULL, filter_gen_film_2d_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}
+
 /* h[N][C][H][W] from the FFN weights (W1 [width][2+4K]) and alpha[C]. */
 int oracle_filter_gen_2d(const double *W1, const double *W2, const double *W3,
                          const double *Wout, const double *alpha, int N, int C,

@@ -105,3 +105,61 @@ def test_per_sample_forward_with_shared_filters_is_the_forward():
     h, bias = r.standard_normal((N, D, L)) * 0.3, r.standard_normal((N, D))
     hp = np.broadcast_to(h, (B, N, D, L))
     assert np.array_equal(oracle.hyena_forward_per_sample(v, x, hp, bias), oracle.hyena_forward(v, x, h, bias))
+
+
+# ------------------------------------------------------------------ 2-D
+
+H2, W2 = 12, 10
+
+
+def film2(n, omega, gamma, beta, window, gaussian=False):
+    return oracle.filter_gen_film_2d(n["W1"], n["W2"], n["W3"], n["Wout"], omega, gamma, beta, window,
+                                     gaussian, N, D, H2, W2)
+
+
+def net2(seed=0):
+    r = np.random.default_rng(seed)
+    return dict(W1=r.standard_normal((W, 34)) / np.sqrt(34), W2=r.standard_normal((W, W)) / 8,
+                W3=r.standard_normal((W, W)) / 8, Wout=r.standard_normal((N * D, W)) / 8)
+
+
+def test_2d_identity_modulation_is_the_shared_filter():
+    n = net2()
+    B = 2
+    h = film2(n, np.ones((3, W)), np.ones((B, 3, W)), np.zeros((B, 3, W)), ALPHA)
+    ref = oracle.filter_gen_2d(n["W1"], n["W2"], n["W3"], n["Wout"], ALPHA, N, D, H2, W2)
+    for b in range(B):
+        assert np.array_equal(h[b], ref)
+
+
+@pytest.mark.parametrize("layer", [0, 2])
+def test_2d_beta_pi_flips_the_sign(layer):
+    n = net2(1)
+    be = np.zeros((1, 3, W))
+    be[0, layer] = np.pi
+    a = film2(n, np.ones((3, W)), np.ones((1, 3, W)), be, ALPHA)
+    b = film2(n, np.ones((3, W)), np.ones((1, 3, W)), np.zeros((1, 3, W)), ALPHA)
+    assert np.max(np.abs(a + b)) < 1e-12 * np.max(np.abs(b))
+
+
+def test_2d_gaussian_window_ratio():
+    n = net2(2)
+    sigma = np.array([0.1, 0.3, 0.7])
+    r = np.random.default_rng(3)
+    g, be = r.uniform(0.5, 1.5, (1, 3, W)), r.normal(0, 0.3, (1, 3, W))
+    hg = film2(n, np.ones((3, W)), g, be, sigma, gaussian=True)
+    he = film2(n, np.ones((3, W)), g, be, ALPHA)
+    ty = (np.arange(H2) / H2)[:, None]
+    tx = (np.arange(W2) / W2)[None, :]
+    gauss = np.exp(-(ty ** 2 + tx ** 2)[None] / (2 * sigma[:, None, None] ** 2))
+    expo = np.exp(-ALPHA[:, None, None] * (np.arange(H2)[:, None] + np.arange(W2)[None, :])[None] / 64.0)
+    np.testing.assert_allclose(hg[0], he[0] * (gauss / expo)[None], rtol=1e-12, atol=1e-300)
+
+
+def test_2d_per_sample_forward_with_shared_filters_is_the_forward():
+    r = np.random.default_rng(9)
+    B = 2
+    v, x = r.standard_normal((B, D, 8, 8)), r.standard_normal((N, B, D, 8, 8))
+    h, bias = r.standard_normal((N, D, 8, 8)) * 0.3, r.standard_normal((N, D))
+    hp = np.broadcast_to(h, (B, N, D, 8, 8))
+    assert np.array_equal(oracle.hyena_forward_2d_per_sample(v, x, hp, bias), oracle.hyena_forward_2d(v, x, h, bias))
