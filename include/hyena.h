@@ -283,6 +283,16 @@ HYENA_API hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* 
 HYENA_API hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C,
                                    int H, int W, float* h, void* stream);
 
+/* Input-dependent 2-D filters h [B][N][C][H][W] float32: the FiLM
+ * modulation of hyena_filter_gen_film on the 2-D filter network; with
+ * film->sigma the window is the Gaussian exp(-(ty^2 + tx^2) /
+ * (2 sigma_c^2)), ty = iy/H, tx = ix/W, else the separable decay of
+ * hyena_filter_gen_2d.  Their spectra are hyena_filter_rfft2d of the B*N
+ * rows of C filters; the forward is hyena_fftconv2d_gate_forward_per_sample. */
+HYENA_API hyena_status_t hyena_filter_gen_film_2d(const hyena_ffn_t* ffn, const hyena_film_t* film,
+                                                  int B, int N, int C, int H, int W, float* h,
+                                                  void* stream);
+
 /* 2-D filter spectra Hs [N][C][2H][W] complex64 in the PACKED real 2-D DFT
  * layout, for filters h [N][C][H][W] (offsets 0..H-1 x 0..W-1) zero-padded
  * to 2H x 2W ("Handling Boundaries"; "Native ND Convolution": the N-D FFT):
@@ -321,6 +331,16 @@ HYENA_API hyena_status_t hyena_fftconv2d_gate_forward(const void* v, const void*
                                                       int W, int N, hyena_dtype_t io, void* y,
                                                       void* workspace, size_t ws_bytes,
                                                       void* stream);
+
+/* The 2-D forward with a spectrum set per sample: Hs [B][N][C][2H][W]
+ * (hyena_filter_rfft2d of per-sample filters); otherwise as
+ * hyena_fftconv2d_gate_forward with the spectrum given. */
+HYENA_API hyena_status_t hyena_fftconv2d_gate_forward_per_sample(const void* v, const void* const* x,
+                                                                 const float* Hs, const float* bias,
+                                                                 int B, int C, int H, int W, int N,
+                                                                 hyena_dtype_t io, void* y,
+                                                                 void* workspace, size_t ws_bytes,
+                                                                 void* stream);
 
 #ifdef __cplusplus
 }

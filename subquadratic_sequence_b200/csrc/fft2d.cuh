@@ -44,6 +44,7 @@ struct Fft2dArgs {
     int q0;                        // first image of the wave (channel-major index)
     int nq;                        // images in the wave
     int n;                         // order handled by this launch
+    size_t Hs_bstride;             // slots between samples' spectra (0: shared by the batch)
 };
 
 template <int LOG2W>
@@ -230,7 +231,7 @@ fft2d_col_kernel(Fft2dArgs a)
         // spectral multiply by (H + b) / (2H)
         const int c = q / a.B;
         const float bias = __ldg(a.bias + a.n * a.C + c);
-        const float2* Hc = a.Hs + ((size_t)a.n * a.C + c) * H2 * W + kx;
+        const float2* Hc = a.Hs + (size_t)(q % a.B) * a.Hs_bstride + ((size_t)a.n * a.C + c) * H2 * W + kx;
         constexpr float s = 1.0f / (float)H2;
         if (kx != 0) {
             static_for<16>([&](auto rr) {

@@ -54,20 +54,16 @@ struct FilterGenArgs {
     const float *gamma, *beta;     // [B][3][width]
     int film;                      // 1: modulate (any of the three given)
     int gaussian;                  // 1: window exp(-t^2 / (2 sigma^2)), sigma in alpha[]
-    float inv_L2;                  // 1 / L^2
+    float inv_L, inv_H, inv_W;     // 1/L (1-D), 1/H and 1/W (2-D): t = i/L, ty = iy/H, tx = ix/W
     long sample_stride;            // floats of h per sample (rows * positions)
 };
 
-// The window of a row is exp(c u): the exponential decay has u = dist
-// (i in 1-D, iy + ix in 2-D) and c = -alpha / div; the Gaussian (1-D) has
-// u = dist^2 and c = -1 / (2 sigma^2 L^2).  par is alpha or sigma.
+// The window of a row is exp(c u): the exponential decay has u = i (1-D)
+// or iy + ix (2-D) and c = -alpha / div; the Gaussian has u = t^2 (1-D) or
+// ty^2 + tx^2 (2-D) and c = -1 / (2 sigma^2).  par is alpha or sigma.
 __device__ __forceinline__ float window_coeff(const FilterGenArgs& a, float par)
 {
-    return a.gaussian ? -0.5f * a.inv_L2 / (par * par) : -par * a.inv_div;
-}
-__device__ __forceinline__ float window_arg(const FilterGenArgs& a, float dist)
-{
-    return a.gaussian ? dist * dist : dist;
+    return a.gaussian ? -0.5f / (par * par) : -par * a.inv_div;
 }
 
 // Offsets the per-sample pointers by the sample of this CTA (blockIdx.z).
@@ -298,16 +294,23 @@ __device__ __forceinline__ void layers_tile(const FilterGenArgs& a, long npos, l
     __syncthreads();
 }
 
-// The argument of the decay window at position pos: i (1-D) or iy + ix
-// (2-D; positions are below 2^30).
+// The window's argument u at position pos (positions are below 2^30).
 template <bool TWO_D>
-__device__ __forceinline__ float window_dist(const FilterGenArgs& a, long pos)
+__device__ __forceinline__ float window_u(const FilterGenArgs& a, long pos)
 {
     if constexpr (!TWO_D) {
+        if (a.gaussian) {
+            const float t = (float)pos * a.inv_L;
+            return t * t;
+        }
         return (float)pos;
     } else {
-        const int ip = (int)pos, iy = ip / a.Ww;
-        return (float)(iy + (ip - iy * a.Ww));
+        const int ip = (int)pos, iy = ip / a.Ww, ix = ip - iy * a.Ww;
+        if (a.gaussian) {
+            const float ty = (float)iy * a.inv_H, tx = (float)ix * a.inv_W;
+            return ty * ty + tx * tx;
+        }
+        return (float)(iy + ix);
     }
 }
 
@@ -408,7 +411,7 @@ __device__ __forceinline__ void head_block(const FilterGenArgs& a, long npos, lo
         const long pos0 = p0 + 64 * g + 4 * tx;
             float dist[4];   // window arguments of the group's 4 positions
 #pragma unroll
-        for (int k = 0; k < 4; ++k) dist[k] = window_arg(a, window_dist<TWO_D>(a, pos0 + k));
+        for (int k = 0; k < 4; ++k) dist[k] = window_u<TWO_D>(a, pos0 + k);
 #pragma unroll
         for (int i = 0; i < RT; ++i) {
             const int r = r0 + RT * ty + i;
@@ -578,7 +581,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_tail16_kernel(FilterGenArgs
     }
     const long pos = p0 + tx;
     if (pos >= npos) return;
-    const float u = window_arg(a, window_dist<TWO_D>(a, pos));
+    const float u = window_u<TWO_D>(a, pos);
 #pragma unroll
     for (int i = 0; i < 4; ++i) stash[(long)(4 * ty + i) * npos + pos] = acc[i] * expf(al[i] * u);
 }

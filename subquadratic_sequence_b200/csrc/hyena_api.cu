@@ -86,7 +86,9 @@ hyena_status_t filter_gen(const hyena_ffn_t* f, int rows, int D, long npos, int 
     a.h = h;
     a.vec = (npos % 4 == 0 && aligned(h, 16)) ? 1 : 0;
     a.sample_stride = (long)rows * npos;
-    a.inv_L2 = L > 0 ? 1.0f / ((float)L * (float)L) : 0.0f;
+    a.inv_L = L > 0 ? 1.0f / (float)L : 0.0f;
+    a.inv_H = Hh > 0 ? 1.0f / (float)Hh : 0.0f;
+    a.inv_W = Ww > 0 ? 1.0f / (float)Ww : 0.0f;
     if (film) {
         a.omega = film->omega;
         a.gamma = film->gamma;
@@ -108,6 +110,9 @@ size_t round_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 hyena_status_t forward_impl(const void* v, const void* const* x, const float* h, const float* H,
                             bool per_sample, const float* bias, int B, int D, int L, int N,
                             hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes, void* stream);
+hyena_status_t forward2d_impl(const void* v, const void* const* x, const float* h, const float* Hs,
+                              bool per_sample, const float* bias, int B, int C, int H, int W, int N,
+                              hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes, void* stream);
 
 }  // namespace
 
@@ -158,6 +163,22 @@ hyena_status_t hyena_filter_gen_film(const hyena_ffn_t* ffn, const hyena_film_t*
     if (B > 65535 || (long)N * D > 65535L * kFgRowTile || (long)B * N * D * (long)L > (1L << 40))
         return HYENA_ERR_UNSUPPORTED;
     return filter_gen(ffn, N * D, D, L, L, 0, 0, false, h, (cudaStream_t)stream, film, B);
+}
+
+hyena_status_t hyena_filter_gen_film_2d(const hyena_ffn_t* ffn, const hyena_film_t* film, int B, int N,
+                                        int C, int H, int W, float* h, void* stream)
+{
+    hyena_status_t s = check_ffn(ffn);
+    if (s != HYENA_OK) return s;
+    if (!film || !h || B < 1 || N < 1 || C < 1 || H < 1 || W < 1 || !aligned(h, 4))
+        return HYENA_ERR_INVALID_ARG;
+    const void* p[4] = {film->omega, film->gamma, film->beta, film->sigma};
+    for (const void* q : p)
+        if (q && !aligned(q, 4)) return HYENA_ERR_INVALID_ARG;
+    if (B > 65535 || (long)H * W > (1L << 30) || (long)N * C > 65535L * kFgRowTile ||
+        (long)B * N * C * (long)H * W > (1L << 40))
+        return HYENA_ERR_UNSUPPORTED;
+    return filter_gen(ffn, N * C, C, (long)H * W, 0, H, W, true, h, (cudaStream_t)stream, film, B);
 }
 
 hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C, int H, int W, float* h,
@@ -481,6 +502,26 @@ hyena_status_t hyena_fftconv2d_gate_forward(const void* v, const void* const* x,
                                             int W, int N, hyena_dtype_t io, void* y, void* workspace,
                                             size_t ws_bytes, void* stream)
 {
+    return forward2d_impl(v, x, h, Hs, false, bias, B, C, H, W, N, io, y, workspace, ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv2d_gate_forward_per_sample(const void* v, const void* const* x, const float* Hs,
+                                                       const float* bias, int B, int C, int H, int W, int N,
+                                                       hyena_dtype_t io, void* y, void* workspace,
+                                                       size_t ws_bytes, void* stream)
+{
+    if (!Hs) return HYENA_ERR_INVALID_ARG;
+    return forward2d_impl(v, x, nullptr, Hs, true, bias, B, C, H, W, N, io, y, workspace, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+hyena_status_t forward2d_impl(const void* v, const void* const* x, const float* h, const float* Hs,
+                              bool per_sample, const float* bias, int B, int C, int H, int W, int N,
+                              hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes, void* stream)
+{
     if (!v || !x || !y || !bias || (!h && !Hs)) return HYENA_ERR_INVALID_ARG;
     if (B < 1 || C < 1 || N < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
     if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
@@ -495,7 +536,7 @@ hyena_status_t hyena_fftconv2d_gate_forward(const void* v, const void* const* x,
     if ((Hs && !aligned(Hs, 16)) || (!Hs && !aligned(h, 16))) return HYENA_ERR_INVALID_ARG;
 
     const size_t act = (size_t)B * C * H * W * io_bytes(io);
-    const size_t spec = sizeof(float2) * (size_t)N * C * 2 * H * W;
+    const size_t spec = sizeof(float2) * (size_t)N * C * 2 * H * W * (per_sample ? (size_t)B : 1);
     const size_t filt = sizeof(float) * (size_t)N * C * H * W;
     const size_t need = hyena_fftconv2d_workspace_size(B, C, H, W, N, io, Hs != nullptr);
     if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
@@ -530,6 +571,7 @@ hyena_status_t hyena_fftconv2d_gate_forward(const void* v, const void* const* x,
     for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
     a.y = y;
     a.Hs = spectrum;
+    a.Hs_bstride = per_sample ? (size_t)N * C * 2 * H * W : 0;
     a.bias = bias;
     a.B = B;
     a.C = C;
@@ -539,5 +581,9 @@ hyena_status_t hyena_fftconv2d_gate_forward(const void* v, const void* const* x,
     return io == HYENA_BF16 ? dispatch_fft2d_bf16(lw, lh, a, N, scratch, st)
                             : dispatch_fft2d_f32(lw, lh, a, N, scratch, st);
 }
+
+}  // namespace
+
+extern "C" {
 
 }  // extern "C"

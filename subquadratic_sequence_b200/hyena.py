@@ -70,6 +70,9 @@ def _load() -> ctypes.CDLL:
         "hyena_filter_rfft_circular": ([vp, i, i, i, vp, vp], i),
         "hyena_fftconv_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp], i),
         "hyena_filter_rfft2d": ([vp, i, i, i, i, vp, vp], i),
+        "hyena_filter_gen_film_2d": ([ffn_p, ctypes.POINTER(hyena_film_t), i, i, i, i, i, vp, vp], i),
+        "hyena_fftconv2d_gate_forward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, vp, vp,
+                                                     sz, vp], i),
         "hyena_fftconv2d_workspace_size": ([i, i, i, i, i, i, i], sz),
         "hyena_fftconv2d_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
                                           vp, sz, vp], i),
@@ -364,6 +367,42 @@ def hyena_fftconv2d_gate_forward(v: torch.Tensor, xs, bias: torch.Tensor, *, Hs=
     hp = ctypes.c_void_p(_dev(h, torch.float32, "h")) if h is not None else None
     _check("hyena_fftconv2d_gate_forward", LIB.hyena_fftconv2d_gate_forward(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, hp, Hp,
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, H, W, N, io,
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def hyena_filter_gen_film_2d(W1, W2, W3, Wout, alpha, N: int, C: int, H: int, W: int, *, B: int,
+                             omega=None, gamma=None, beta=None, sigma=None, n_bands: int = 8,
+                             width: int = 64, decay_div: float = 64.0, out=None, stream=None):
+    """Per-sample 2-D filters h [B][N][C][H][W] float32 (FiLM-modulated; the
+    Gaussian window when sigma [C] is given)."""
+    f = _ffn(W1, W2, W3, Wout, alpha, n_bands, width, decay_div)
+    opt = lambda t, name: ctypes.c_void_p(_dev(t, torch.float32, name)) if t is not None else None
+    film = hyena_film_t(opt(omega, "omega"), opt(gamma, "gamma"), opt(beta, "beta"), opt(sigma, "sigma"))
+    if out is None:
+        out = torch.empty((B, N, C, H, W), device=W1.device, dtype=torch.float32)
+    _check("hyena_filter_gen_film_2d", LIB.hyena_filter_gen_film_2d(
+        ctypes.byref(f), ctypes.byref(film), B, N, C, H, W, ctypes.c_void_p(_dev(out, torch.float32, "h")),
+        _stream(stream)))
+    return out
+
+
+def hyena_fftconv2d_gate_forward_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor, *,
+                                            out=None, workspace=None, stream=None):
+    """The 2-D forward with per-sample spectra Hs [B][N][C][2H][W] complex64."""
+    B, C, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    need = hyena_fftconv2d_workspace_size(B, C, H, W, N, io, True)
+    if workspace is None:
+        workspace = torch.empty(need, device=v.device, dtype=torch.uint8)
+    _check("hyena_fftconv2d_gate_forward_per_sample", LIB.hyena_fftconv2d_gate_forward_per_sample(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, H, W, N, io,
         ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
