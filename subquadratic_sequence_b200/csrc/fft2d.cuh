@@ -174,9 +174,10 @@ struct Fft2dCols {
     static constexpr int STRIDE = stride_mod16(H2, 16 / TC);
     static constexpr size_t SMEM = sizeof(float2) * TC * STRIDE;
     // resident CTAs per SM: up to three, as shared memory allows and with at
-    // least 80 registers per thread
+    // least 80 registers per thread (120 with 32 values per thread)
+    static constexpr int REGS = FC::V == 32 ? 120 : 80;
     static constexpr int BY_SMEM = 3 * SMEM <= 227 * 1024 ? 3 : (2 * SMEM <= 227 * 1024 ? 2 : 1);
-    static constexpr int BY_REGS = 65536 / (THREADS * 80) < 1 ? 1 : 65536 / (THREADS * 80);
+    static constexpr int BY_REGS = 65536 / (THREADS * REGS) < 1 ? 1 : 65536 / (THREADS * REGS);
     static constexpr int MIN_BLOCKS = BY_SMEM < BY_REGS ? BY_SMEM : BY_REGS;
     static_assert(THREADS <= 1024 && SMEM <= 227 * 1024, "column kernel geometry");
 };
@@ -192,7 +193,7 @@ fft2d_col_kernel(Fft2dArgs a)
     grid_dependency_begin();
     using CL = Fft2dCols<LOG2H2>;
     using FC = typename CL::FC;
-    constexpr int H2 = CL::H2, TC = CL::TC, HH = H2 / 2;
+    constexpr int H2 = CL::H2, TC = CL::TC, HH = H2 / 2, V = FC::V;
     const int W = a.W;
     const int CTAS_PER_IMG = W / TC;
     extern __shared__ __align__(16) float2 smem_c2[];
@@ -206,26 +207,26 @@ fft2d_col_kernel(Fft2dArgs a)
     float2* buf = smem_c2 + cc * CL::STRIDE;
     // rows of this image's column kx: scratch [H][W] or spectra [2H][W]
     float2* col = SPECTRUM ? a.S + (size_t)q * H2 * W + kx : a.S + (size_t)qi * HH * W + kx;
-    float2 reg[16];
+    float2 reg[V];
     const int pt = pad16(t);
 
-    static_for<16>([&](auto rr) {
+    static_for<V>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
-        const int y = t + r * (H2 / 16);
-        buf[pad16_at<H2 / 16>(t, pt, r)] = r < 8 ? col[(size_t)y * W] : make_float2(0.0f, 0.0f);
+        const int y = t + r * (H2 / V);
+        buf[pad16_at<H2 / V>(t, pt, r)] = r < V / 2 ? col[(size_t)y * W] : make_float2(0.0f, 0.0f);
     });
     __syncthreads();
     FC::template run<-1, true>(buf, reg, t);
     if constexpr (SPECTRUM) {
-        static_for<16>([&](auto rr) {
+        static_for<V>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            col[(size_t)(t + r * (H2 / 16)) * W] = reg[r];
+            col[(size_t)(t + r * (H2 / V)) * W] = reg[r];
         });
         return;
     } else {
-        static_for<16>([&](auto rr) {
+        static_for<V>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            buf[pad16_at<H2 / 16>(t, pt, r)] = reg[r];
+            buf[pad16_at<H2 / V>(t, pt, r)] = reg[r];
         });
         __syncthreads();
         // spectral multiply by (H + b) / (2H)
@@ -234,20 +235,20 @@ fft2d_col_kernel(Fft2dArgs a)
         const float2* Hc = a.Hs + (size_t)(q % a.B) * a.Hs_bstride + ((size_t)a.n * a.C + c) * H2 * W + kx;
         constexpr float s = 1.0f / (float)H2;
         if (kx != 0) {
-            static_for<16>([&](auto rr) {
+            static_for<V>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
-                const int ky = t + r * (H2 / 16);
+                const int ky = t + r * (H2 / V);
                 const float2 hv = __ldg(Hc + (size_t)ky * W);
-                const int pk = pad16_at<H2 / 16>(t, pt, r);
+                const int pk = pad16_at<H2 / V>(t, pt, r);
                 buf[pk] = cmul(buf[pk], make_float2((hv.x + bias) * s, hv.y * s));
             });
         } else {
             // slot 0 = (bin-0 column) + i (bin-W column): separate both
             // through the pair (ky, 2H - ky), multiply each by its own
             // filter column, and re-pack
-            static_for<16>([&](auto rr) {
+            static_for<V>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
-                const int ky = t + r * (H2 / 16);
+                const int ky = t + r * (H2 / V);
                 if (ky <= HH) {
                     const int kn = (H2 - ky) % H2;
                     const float2 c1 = buf[pad16(ky)], c2 = buf[pad16(kn)];
@@ -267,9 +268,9 @@ fft2d_col_kernel(Fft2dArgs a)
         }
         __syncthreads();
         FC::template run<+1, true>(buf, reg, t);
-        static_for<8>([&](auto rr) {
+        static_for<V / 2>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            col[(size_t)(t + r * (H2 / 16)) * W] = reg[r];
+            col[(size_t)(t + r * (H2 / V)) * W] = reg[r];
         });
     }
 }

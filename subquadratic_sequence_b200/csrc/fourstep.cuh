@@ -38,16 +38,20 @@ __host__ __device__ constexpr int stride_mod16(int n, int mod16)
 }
 
 // One S = 2^LOG2S point FFT held in a padded shared buffer and transformed
-// by T = S/16 threads (16 values each), Stockham DIT, natural order in and
-// out.  Several transforms run side by side in a CTA; every pass ends in a
-// __syncthreads() of the whole CTA.  On return a[r] holds X[t + r S/16].
+// by T = S/V threads (V values each), Stockham DIT, natural order in and
+// out.  V = 32 for S = 512 and 1024 (two passes: radix S/32, then 32),
+// else 16 (passes of radix 16 after a first pass of S / 16^(NP-1)).  Several
+// transforms run side by side in a CTA; every pass ends in a
+// __syncthreads() of the whole CTA.  On return a[r] holds X[t + r S/V].
 template <int LOG2S>
 struct SmemFft {
     static_assert(LOG2S >= 4, "S >= 16");
     static constexpr int S = 1 << LOG2S;
-    static constexpr int T = S / 16;
-    static constexpr int R0 = (LOG2S % 4 == 0) ? 16 : (1 << (LOG2S % 4));  // first pass radix
-    static constexpr int NP = (LOG2S + 3) / 4;                             // passes
+    static constexpr int V = (LOG2S == 9 || LOG2S == 10) ? 32 : 16;          // values per thread
+    static constexpr int T = S / V;
+    static constexpr int NP = V == 32 ? 2 : (LOG2S + 3) / 4;                 // passes
+    static constexpr int R0 = V == 32 ? S / 32
+                            : (LOG2S % 4 == 0) ? 16 : (1 << (LOG2S % 4));   // first pass radix
 
     // PADDED_IN: the input sits at buf[pad16(i)] (else at buf[i]).
     template <int SIGN, bool PADDED_IN>
@@ -55,9 +59,9 @@ struct SmemFft {
     {
         static_for<NP>([&](auto pp) {
             constexpr int p = decltype(pp)::value;
-            constexpr int R = p == 0 ? R0 : 16;
-            constexpr int NS = p == 0 ? 1 : R0 * ipow16(p - 1);
-            constexpr int C = 16 / R;
+            constexpr int R = p == 0 ? R0 : V;
+            constexpr int NS = p == 0 ? 1 : (V == 32 ? R0 : R0 * ipow16(p - 1));
+            constexpr int C = V / R;
             constexpr bool LAST = p == NP - 1;
             static_for<C>([&](auto cc) {
                 constexpr int c = decltype(cc)::value;
@@ -134,17 +138,18 @@ struct FourStep {
     // Bin pairs (k, M - k) of the real split over the CTA's row pairs, in
     // shared memory after the forward row FFTs (row slot 2 up holds row u,
     // slot 2 up + 1 row M1 - u; unit 0: rows 0 and M1/2).  Thread tid takes
-    // unit up = tid % U and k2 = tid / U + it M2/8 (it < 8), so adjacent
+    // unit up = tid % U and k2 = tid / U + it KSTEP (it < ITER), so adjacent
     // threads touch adjacent spectrum slots (k1 consecutive), and the
     // split's twiddle exp(-i pi k / M) of iteration it is that of it = 0
-    // times exp(-i pi it / 8).  f(kind, p1, p2, k, w): kind 0 = bins k
+    // times exp(-i pi it / ITER).  f(kind, p1, p2, k, w): kind 0 = bins k
     // (*p1) and M - k (*p2); 1 = bins 0 and M (slot 0, p1 == p2); 2 = bin
     // M/2 alone (p1 == p2).
     template <typename Fn>
     static __device__ __forceinline__ void for_each_pair(float2* smem, int ublk, int tid, Fn&& f)
     {
         constexpr int RS = ROW_STRIDE, KSTEP = ROW_THREADS / U, ITER = U * M2 / ROW_THREADS;
-        static_assert(ITER == 8 && ITER * KSTEP == M2, "pair iteration");
+        constexpr int Q = 32 / ITER;          // exp(-i pi it / ITER) = W_64^(Q it)
+        static_assert(ITER * KSTEP == M2 && 32 % ITER == 0, "pair iteration");
         const int up = tid % U, k20 = tid / U, u = ublk * U + up;
         float2* r0 = smem + (2 * up) * RS;
         float2* r1 = smem + (2 * up + 1) * RS;
@@ -154,7 +159,7 @@ struct FourStep {
             static_for<ITER>([&](auto ii) {
                 constexpr int it = decltype(ii)::value;
                 const int k2 = k20 + it * KSTEP;
-                f(0, r0 + pad16(k2), r1 + pad16(M2 - 1 - k2), k0 + it * KSTEP * M1, mul_w64<4 * it, -1>(w0));
+                f(0, r0 + pad16(k2), r1 + pad16(M2 - 1 - k2), k0 + it * KSTEP * M1, mul_w64<Q * it, -1>(w0));
             });
         } else {
             // row M1/2 pairs with itself reversed; row 0 pairs k2 with M2 - k2
@@ -163,9 +168,9 @@ struct FourStep {
             static_for<ITER / 2>([&](auto ii) {
                 constexpr int it = decltype(ii)::value;
                 const int k2 = k20 + it * KSTEP;             // < M2 / 2
-                f(0, r1 + pad16(k2), r1 + pad16(M2 - 1 - k2), M1 / 2 + M1 * k2, mul_w64<4 * it, -1>(wh0));
+                f(0, r1 + pad16(k2), r1 + pad16(M2 - 1 - k2), M1 / 2 + M1 * k2, mul_w64<Q * it, -1>(wh0));
                 if (k2 > 0) {
-                    f(0, r0 + pad16(k2), r0 + pad16(M2 - k2), M1 * k2, mul_w64<4 * it, -1>(wz0));
+                    f(0, r0 + pad16(k2), r0 + pad16(M2 - k2), M1 * k2, mul_w64<Q * it, -1>(wz0));
                 } else {
                     f(1, r0, r0, 0, make_float2(1.0f, 0.0f));
                     f(2, r0 + pad16(M2 / 2), r0 + pad16(M2 / 2), M / 2, make_float2(0.0f, -1.0f));
@@ -225,7 +230,7 @@ fourstep_row_kernel(FourStepArgs a)
 {
     grid_dependency_begin();
     using FS = FourStep<LOG2M1, LOG2M2>;
-    constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, U = FS::U, T2 = FS::F2::T;
+    constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, U = FS::U, T2 = FS::F2::T, V2 = FS::F2::V;
     constexpr int RS = FS::ROW_STRIDE;
     extern __shared__ __align__(16) float2 smem_fs[];
 
@@ -245,12 +250,12 @@ fourstep_row_kernel(FourStepArgs a)
 
     const int row = tid / T2, t = tid % T2;
     float2* rb = smem_fs + row * RS;
-    float2 reg[16];
+    float2 reg[V2];
     FS::F2::template run<-1, false>(rb, reg, t);
     const int pt = pad16(t);
-    static_for<16>([&](auto rr) {
+    static_for<V2>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
-        rb[pad16_at<M2 / 16>(t, pt, r)] = reg[r];
+        rb[pad16_at<M2 / V2>(t, pt, r)] = reg[r];
     });
     __syncthreads();
 
@@ -285,14 +290,14 @@ fourstep_row_kernel(FourStepArgs a)
         __syncthreads();
 
         FS::F2::template run<+1, true>(rb, reg, t);
-        // B[k1][n2] *= exp(+2 pi i n2 k1 / M), n2 = t + r M2/16
+        // B[k1][n2] *= exp(+2 pi i n2 k1 / M), n2 = t + r M2/V2
         const int k1 = FS::row_of(ublk, row);
         float2 w = expi_pi<+1>(2.0f * (float)((t * k1) % M) / (float)M);
-        const float2 step = expi_pi<+1>(2.0f * (float)((k1 * (M2 / 16)) % M) / (float)M);
-        static_for<16>([&](auto rr) {
+        const float2 step = expi_pi<+1>(2.0f * (float)((k1 * (M2 / V2)) % M) / (float)M);
+        static_for<V2>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            Sq[(size_t)k1 * M2 + t + r * (M2 / 16)] = cmul(reg[r], w);
-            if constexpr (r < 15) w = cmul(w, step);
+            Sq[(size_t)k1 * M2 + t + r * (M2 / V2)] = cmul(reg[r], w);
+            if constexpr (r < V2 - 1) w = cmul(w, step);
         });
     }
 }
@@ -308,7 +313,7 @@ fourstep_col_kernel(FourStepArgs a)
     using FS = FourStep<LOG2M1, LOG2M2>;
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;
-    constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, TC = FS::TC;
+    constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, TC = FS::TC, V1 = FS::F1::V;
     extern __shared__ __align__(16) float2 smem_fs[];
 
     const int qi = blockIdx.x / FS::COL_CTAS_PER_SEQ;
@@ -321,39 +326,39 @@ fourstep_col_kernel(FourStepArgs a)
     const int c = tid % TC, t = tid / TC;
     const int n2 = c0 + c;
     float2* buf = smem_fs + c * FS::COL_STRIDE;
-    float2 reg[16];
+    float2 reg[V1];
 
     if constexpr (MODE == 0) {
         const PT* vp = reinterpret_cast<const PT*>(a.v) + seq * (M / 2);
-        static_for<8>([&](auto rr) {
+        static_for<V1 / 2>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            reg[r] = IOP::load(vp + n2 + (size_t)M2 * (t + r * (M1 / 16)));
+            reg[r] = IOP::load(vp + n2 + (size_t)M2 * (t + r * (M1 / V1)));
         });
     } else {
         const int pt = pad16(t);
-        static_for<16>([&](auto rr) {
+        static_for<V1>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            const int k1 = t + r * (M1 / 16);
-            buf[pad16_at<M1 / 16>(t, pt, r)] = Sq[(size_t)k1 * M2 + n2];
+            const int k1 = t + r * (M1 / V1);
+            buf[pad16_at<M1 / V1>(t, pt, r)] = Sq[(size_t)k1 * M2 + n2];
         });
         __syncthreads();
         FS::F1::template run<+1, true>(buf, reg, t);
-        // crop (n1 = t + r M1/16 < M1/2 <=> r < 8) and gate
+        // crop (n1 = t + r M1/V1 < M1/2 <=> r < V1/2) and gate
         const void* xn = a.x[0];
 #pragma unroll
         for (int i = 1; i < kMaxOrder; ++i)
             if (i == a.n) xn = a.x[i];
         const PT* xp = reinterpret_cast<const PT*>(xn) + seq * (M / 2);
-        static_for<8>([&](auto rr) {
+        static_for<V1 / 2>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            const float2 xv = IOP::load(xp + n2 + (size_t)M2 * (t + r * (M1 / 16)));
+            const float2 xv = IOP::load(xp + n2 + (size_t)M2 * (t + r * (M1 / V1)));
             reg[r] = make_float2(reg[r].x * xv.x, reg[r].y * xv.y);
         });
         if constexpr (MODE == 2) {
             PT* yp = reinterpret_cast<PT*>(a.y) + seq * (M / 2);
-            static_for<8>([&](auto rr) {
+            static_for<V1 / 2>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
-                IOP::store(yp + n2 + (size_t)M2 * (t + r * (M1 / 16)), reg[r]);
+                IOP::store(yp + n2 + (size_t)M2 * (t + r * (M1 / V1)), reg[r]);
             });
             return;
         }
@@ -362,19 +367,19 @@ fourstep_col_kernel(FourStepArgs a)
     // twiddle exp(-2 pi i n2 k1 / M)
     {
         const int pt = pad16(t);
-        static_for<16>([&](auto rr) {
+        static_for<V1>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            buf[pad16_at<M1 / 16>(t, pt, r)] = r < 8 ? reg[r] : make_float2(0.0f, 0.0f);
+            buf[pad16_at<M1 / V1>(t, pt, r)] = r < V1 / 2 ? reg[r] : make_float2(0.0f, 0.0f);
         });
     }
     __syncthreads();
     FS::F1::template run<-1, true>(buf, reg, t);
     float2 w = expi_pi<-1>(2.0f * (float)((n2 * t) % M) / (float)M);
-    const float2 step = expi_pi<-1>(2.0f * (float)((n2 * (M1 / 16)) % M) / (float)M);
-    static_for<16>([&](auto rr) {
+    const float2 step = expi_pi<-1>(2.0f * (float)((n2 * (M1 / V1)) % M) / (float)M);
+    static_for<V1>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
-        Sq[(size_t)(t + r * (M1 / 16)) * M2 + n2] = cmul(reg[r], w);
-        if constexpr (r < 15) w = cmul(w, step);
+        Sq[(size_t)(t + r * (M1 / V1)) * M2 + n2] = cmul(reg[r], w);
+        if constexpr (r < V1 - 1) w = cmul(w, step);
     });
 }
 
