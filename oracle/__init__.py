@@ -62,6 +62,8 @@ def _load():
         "oracle_hyena_backward": [dp, dp, dp, dp, dp, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_filter_gen_film": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, d, i, dp],
         "oracle_cconv": [dp, dp, l, i, dp],
+        "oracle_conv3": [dp, dp, l, l, l, i, dp],
+        "oracle_hyena_forward_3d": [dp, dp, dp, dp, l, l, l, l, l, l, i, dp],
         "oracle_filter_gen_film_2d": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, i, d, i, dp],
         "oracle_rfft_circ": [dp, l, l, dp, dp],
         "oracle_hyena_forward_circular": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
@@ -311,3 +313,24 @@ def hyena_forward_2d_per_sample(v, x, h, bias, route="fft", threads=None) -> np.
     v, x, h, bias = map(_f64, (v, x, h, bias))
     return np.concatenate([hyena_forward_2d(v[b:b + 1], x[:, b:b + 1], h[b], bias, route, threads)
                            for b in range(v.shape[0])])
+
+
+def conv3(h, u, route="direct") -> np.ndarray:
+    """3-D linear convolution on offsets 0..Z-1 x 0..H-1 x 0..W-1, cropped."""
+    h, u = _f64(h), _f64(u)
+    Z, H, W = u.shape
+    y = np.empty_like(u)
+    _check(_load().oracle_conv3(_ptr(h), _ptr(u), Z, H, W, _route(route), _ptr(y)), "oracle_conv3")
+    return y
+
+
+def hyena_forward_3d(v, x, h, bias, route="fft") -> np.ndarray:
+    """The recurrence with 3-D convolutions: v [B][C][Z][H][W], x [N][B][C][Z][H][W],
+    h [N][C][Z][H][W], bias [N][C] -> y [B][C][Z][H][W]."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    B, C, Z, H, W = v.shape
+    N = h.shape[0]
+    y = np.empty_like(v)
+    _check(_load().oracle_hyena_forward_3d(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), B, C, Z, H, W, N,
+                                           _route(route), _ptr(y)), "oracle_hyena_forward_3d")
+    return y

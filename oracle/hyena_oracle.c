@@ -1129,3 +1129,116 @@ int oracle_hyena_forward_2d(const double *v, const double *x, const double *h,
     free(jobs); free(tid);
     return st;
 }
+
+/* ------------------------------------------------------------------ */
+/* 3-D: linear convolution on a volume (Native ND Convolution;          */
+/* Handling Boundaries: zero-pad to double the grid).                  */
+/* ------------------------------------------------------------------ */
+
+/* The definition: y[p][q][r] = sum_{i<=p, j<=q, k<=r} h[i][j][k] u[p-i][q-j][r-k]. */
+static void conv3_direct(const double *h, const double *u, long Z, long H, long W, double *y)
+{
+    for (long p = 0; p < Z; ++p)
+        for (long q = 0; q < H; ++q)
+            for (long r = 0; r < W; ++r) {
+                double s = 0.0;
+                for (long i = 0; i <= p; ++i)
+                    for (long j = 0; j <= q; ++j)
+                        for (long k = 0; k <= r; ++k)
+                            s += h[(i * H + j) * W + k] * u[((p - i) * H + (q - j)) * W + (r - k)];
+                y[(p * H + q) * W + r] = s;
+            }
+}
+
+/* 3-D DFT of a PZ x PH x PW grid: along x for every (z, y), then along y,
+ * then along z, each by the radix-2 routine on a gathered line. */
+static int fft3(double *re, double *im, long PZ, long PH, long PW, int sign)
+{
+    const long n = PZ > PH ? (PZ > PW ? PZ : PW) : (PH > PW ? PH : PW);
+    double *lr = malloc(sizeof(double) * n), *li = malloc(sizeof(double) * n);
+    if (!lr || !li) { free(lr); free(li); return ORACLE_ENOMEM; }
+    for (long z = 0; z < PZ; ++z)
+        for (long y = 0; y < PH; ++y) fft_radix2(re + (z * PH + y) * PW, im + (z * PH + y) * PW, PW, sign);
+    for (long z = 0; z < PZ; ++z)
+        for (long x = 0; x < PW; ++x) {
+            for (long y = 0; y < PH; ++y) { lr[y] = re[(z * PH + y) * PW + x]; li[y] = im[(z * PH + y) * PW + x]; }
+            fft_radix2(lr, li, PH, sign);
+            for (long y = 0; y < PH; ++y) { re[(z * PH + y) * PW + x] = lr[y]; im[(z * PH + y) * PW + x] = li[y]; }
+        }
+    for (long y = 0; y < PH; ++y)
+        for (long x = 0; x < PW; ++x) {
+            for (long z = 0; z < PZ; ++z) { lr[z] = re[(z * PH + y) * PW + x]; li[z] = im[(z * PH + y) * PW + x]; }
+            fft_radix2(lr, li, PZ, sign);
+            for (long z = 0; z < PZ; ++z) { re[(z * PH + y) * PW + x] = lr[z]; im[(z * PH + y) * PW + x] = li[z]; }
+        }
+    free(lr); free(li);
+    return ORACLE_OK;
+}
+
+/* The convolution theorem on the grid padded to 2Z x 2H x 2W (powers of two). */
+static int conv3_fft(const double *h, const double *u, long Z, long H, long W, double *y)
+{
+    const long PZ = 2 * Z, PH = 2 * H, PW = 2 * W, P = PZ * PH * PW;
+    double *hr = calloc(P, sizeof(double)), *hi = calloc(P, sizeof(double));
+    double *ur = calloc(P, sizeof(double)), *ui = calloc(P, sizeof(double));
+    int st = ORACLE_ENOMEM;
+    if (!hr || !hi || !ur || !ui) goto out;
+    for (long z = 0; z < Z; ++z)
+        for (long q = 0; q < H; ++q)
+            for (long r = 0; r < W; ++r) {
+                hr[(z * PH + q) * PW + r] = h[(z * H + q) * W + r];
+                ur[(z * PH + q) * PW + r] = u[(z * H + q) * W + r];
+            }
+    if ((st = fft3(hr, hi, PZ, PH, PW, -1)) != ORACLE_OK) goto out;
+    if ((st = fft3(ur, ui, PZ, PH, PW, -1)) != ORACLE_OK) goto out;
+    for (long k = 0; k < P; ++k) {
+        const double re = hr[k] * ur[k] - hi[k] * ui[k], im = hr[k] * ui[k] + hi[k] * ur[k];
+        ur[k] = re;
+        ui[k] = im;
+    }
+    if ((st = fft3(ur, ui, PZ, PH, PW, +1)) != ORACLE_OK) goto out;
+    for (long z = 0; z < Z; ++z)
+        for (long q = 0; q < H; ++q)
+            for (long r = 0; r < W; ++r) y[(z * H + q) * W + r] = ur[(z * PH + q) * PW + r] / (double)P;
+out:
+    free(hr); free(hi); free(ur); free(ui);
+    return st;
+}
+
+int oracle_conv3(const double *h, const double *u, long Z, long H, long W, int route, double *y)
+{
+    if (!h || !u || !y || Z < 1 || H < 1 || W < 1) return ORACLE_EBADARG;
+    if (route == ROUTE_DIRECT) {
+        conv3_direct(h, u, Z, H, W, y);
+        return ORACLE_OK;
+    }
+    if (route != ROUTE_FFT || !is_pow2(Z) || !is_pow2(H) || !is_pow2(W)) return ORACLE_EBADARG;
+    return conv3_fft(h, u, Z, H, W, y);
+}
+
+/* v [B][C][Z][H][W], x [N][B][C][Z][H][W], h [N][C][Z][H][W], bias [N][C]
+ * -> y [B][C][Z][H][W]: the recurrence with 3-D convolutions (one thread;
+ * the 3-D tests are small). */
+int oracle_hyena_forward_3d(const double *v, const double *x, const double *h, const double *bias,
+                            long B, long C, long Z, long H, long W, long N, int route, double *y)
+{
+    if (!v || !x || !h || !bias || !y || B < 1 || C < 1 || Z < 1 || H < 1 || W < 1 || N < 1)
+        return ORACLE_EBADARG;
+    const long V = Z * H * W, BCV = B * C * V;
+    double *z = malloc(sizeof(double) * V), *c = malloc(sizeof(double) * V);
+    if (!z || !c) { free(z); free(c); return ORACLE_ENOMEM; }
+    int st = ORACLE_OK;
+    for (long img = 0; img < B * C && st == ORACLE_OK; ++img) {
+        const long ch = img % C;
+        memcpy(z, v + img * V, sizeof(double) * V);
+        for (long n = 0; n < N && st == ORACLE_OK; ++n) {
+            const double *hn = h + (n * C + ch) * V, *xn = x + n * BCV + img * V;
+            const double bn = bias[n * C + ch];
+            st = oracle_conv3(hn, z, Z, H, W, route, c);
+            for (long t = 0; t < V; ++t) z[t] = xn[t] * (c[t] + bn * z[t]);
+        }
+        memcpy(y + img * V, z, sizeof(double) * V);
+    }
+    free(z); free(c);
+    return st;
+}

@@ -377,3 +377,47 @@ def test_filter_gen_threads_do_not_change_results():
     a = oracle.filter_gen(W1, W2, W3, Wout, alpha, N, D, L, width=width, threads=1)
     b = oracle.filter_gen(W1, W2, W3, Wout, alpha, N, D, L, width=width, threads=5)
     assert np.array_equal(a, b)
+
+
+# --------------------------------------------------------------------- 3-D
+
+@pytest.mark.parametrize("Z,H,W", [(1, 1, 1), (2, 3, 4), (4, 8, 4)])
+def test_conv3_direct_is_scipy(Z, H, W):
+    r = rng(Z * 100 + H * 10 + W)
+    h, u = r.standard_normal((Z, H, W)), r.standard_normal((Z, H, W))
+    ref = scipy.signal.convolve(h, u, method="direct")[:Z, :H, :W]
+    assert rel_err(oracle.conv3(h, u, "direct"), ref) < 1e-12
+
+
+@pytest.mark.parametrize("Z,H,W", [(2, 2, 2), (4, 8, 4), (8, 4, 16)])
+def test_conv3_fft_equals_direct(Z, H, W):
+    r = rng(Z + H + W)
+    h, u = r.standard_normal((Z, H, W)), r.standard_normal((Z, H, W))
+    assert rel_err(oracle.conv3(h, u, "fft"), oracle.conv3(h, u, "direct")) < 1e-12
+
+
+def test_conv3_separable_reduces_to_2d_and_1d():
+    # h[i][j][k] = f[i] g[j][k]: conv3 = (1-D along z) of (2-D in each plane)
+    r = rng(7)
+    Z, H, W = 4, 8, 8
+    f, g, u = r.standard_normal(Z), r.standard_normal((H, W)), r.standard_normal((Z, H, W))
+    h = f[:, None, None] * g[None]
+    planes = np.stack([oracle.conv2(g, u[z], "direct") for z in range(Z)])
+    ref = np.stack([[[oracle.conv(f, planes[:, q, rr], "direct")[p] for rr in range(W)]
+                     for q in range(H)] for p in range(Z)])
+    assert rel_err(oracle.conv3(h, u, "direct"), ref) < 1e-12
+
+
+@pytest.mark.parametrize("route", ["direct", "fft"])
+def test_forward_3d_delta_filter_and_routes(route):
+    r = rng(8)
+    B, C, Z, H, W, N = 2, 2, 4, 4, 8, 2
+    v, x = r.standard_normal((B, C, Z, H, W)), r.standard_normal((N, B, C, Z, H, W))
+    b = r.standard_normal((N, C))
+    h = np.zeros((N, C, Z, H, W))
+    h[:, :, 0, 0, 0] = 1.0
+    want = v * np.prod(x * (1.0 + b)[:, None, :, None, None, None], axis=0)
+    assert rel_err(oracle.hyena_forward_3d(v, x, h, b, route=route), want) < 1e-12
+    h = r.standard_normal((N, C, Z, H, W))
+    assert rel_err(oracle.hyena_forward_3d(v, x, h, b, route="fft"),
+                   oracle.hyena_forward_3d(v, x, h, b, route="direct")) < 1e-12
