@@ -342,6 +342,50 @@ HYENA_API hyena_status_t hyena_fftconv2d_gate_forward_per_sample(const void* v, 
                                                                  void* workspace, size_t ws_bytes,
                                                                  void* stream);
 
+/* ---------------------------------------------------------------- 3-D */
+
+/* 3-D filter spectra Hs [N][C][2Z][2H][W] complex64, for filters h
+ * [N][C][Z][H][W] float32 (offsets 0..Z-1 x 0..H-1 x 0..W-1) zero-padded
+ * to 2Z x 2H x 2W ("Native Multi-Dimensional Subquadratic Operators via
+ * Input Dependent Long Convolutions": Native ND Convolution, Handling
+ * Boundaries).  The packing extends the 2-D one by the 2Z-point DFT over
+ * z of every slot: with X[kz][ky][kx] the 3-D DFT,
+ *   slot [kz][ky][kx] = X[kz][ky][kx]          for 1 <= kx < W,
+ *   slot [kz][ky][0]  = A = X0 + i XW,  X0 = X[.][.][0], XW = X[.][.][W],
+ * so X0 = (A + conj A') / 2 and XW = (A - conj A') / (2i) with A' the slot
+ * at (-kz, -ky).  Z, H, W powers of two in [16, 256]; N*C*Z*H <= 2^30.
+ * Alignment 16 bytes; Hs must not overlap h.  No workspace. */
+HYENA_API hyena_status_t hyena_filter_rfft3d(const float* h, int N, int C, int Z, int H, int W,
+                                             float* Hs, void* stream);
+
+/* Bytes of workspace hyena_fftconv3d_gate_forward needs (the spectra when
+ * spectrum_given = 0, plus the scratch of one wave of volumes: Z planes of
+ * 2H x W complex slots each); (size_t)-1 for invalid sizes. */
+HYENA_API size_t hyena_fftconv3d_workspace_size(int B, int C, int Z, int H, int W, int N,
+                                                hyena_dtype_t io, int spectrum_given);
+
+/* The order-N 3-D forward, per volume (b, c):
+ *   z_0 = v,  z_n = x_n * (h_n (*) z_{n-1} + b_n z_{n-1}),  y = z_N
+ * with (*) the linear 3-D convolution
+ *   (h (*) u)[p][q][r] = sum_{i <= p, j <= q, k <= r} h[i][j][k] u[p-i][q-j][r-k]
+ * computed on the volume zero-padded to 2Z x 2H x 2W and cropped.
+ *   v, x_n, y [B][C][Z][H][W] io; h [N][C][Z][H][W] float32 or Hs
+ *   [N][C][2Z][2H][W] (hyena_filter_rfft3d; wins when both are given);
+ *   bias [N][C]; x is a HOST array of N device pointers.
+ * workspace: hyena_fftconv3d_workspace_size(...) bytes, 256-byte aligned.
+ * Z, H, W powers of two in [16, 256]; 1 <= N <= HYENA_MAX_ORDER.
+ * Alignment: v, x_n, y, h, Hs 16 bytes; bias 4.  y must not overlap any
+ * input or the workspace.  Per volume and order: forward rows, forward
+ * columns, the z transform with the spectral multiply and its inverse,
+ * inverse columns, inverse rows with the gate (fused with the next
+ * order's forward rows). */
+HYENA_API hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void* const* x,
+                                                      const float* h, const float* Hs,
+                                                      const float* bias, int B, int C, int Z,
+                                                      int H, int W, int N, hyena_dtype_t io,
+                                                      void* y, void* workspace, size_t ws_bytes,
+                                                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -45,7 +45,21 @@ struct Fft2dArgs {
     int nq;                        // images in the wave
     int n;                         // order handled by this launch
     size_t Hs_bstride;             // slots between samples' spectra (0: shared by the batch)
+    // 3-D volumes [Z][Hp][W] as Z planes per image (0 for 2-D grids): the
+    // row kernel then sees H = Z * Hp rows per image and keeps every plane
+    // at a pitch of 2 Hp rows in the scratch (and of 2 Z planes per filter
+    // in the spectra)
+    int zp, Hp;
 };
+
+// Scratch row of row index yrow of image qi (2-D: [H][W] per image; 3-D:
+// plane z = yrow / Hp at a pitch of 2 Hp rows).
+__device__ __forceinline__ float2* scratch_row(const Fft2dArgs& a, int qi, int yrow)
+{
+    if (a.zp == 0) return a.S + ((size_t)qi * a.H + yrow) * a.W;
+    const int z = yrow / a.Hp, y = yrow - z * a.Hp;
+    return a.S + (((size_t)qi * a.zp + z) * 2 * a.Hp + y) * a.W;
+}
 
 template <int LOG2W>
 struct Fft2dRows {
@@ -129,10 +143,15 @@ fft2d_row_kernel(Fft2dArgs a)
         if constexpr (MODE == 0) {
             const int c = q / a.B, b = q % a.B;
             img = (size_t)b * a.C + c;
-            row = a.S + ((size_t)qi * a.H + yrow) * W;
+            row = scratch_row(a, qi, yrow);
         } else {
             img = (size_t)q;                                  // filter row n*C + c
-            row = a.S + ((size_t)q * 2 * a.H + yrow) * W;
+            if (a.zp == 0) {
+                row = a.S + ((size_t)q * 2 * a.H + yrow) * W;
+            } else {                                          // plane z of [2Z][2Hp][W]
+                const int z = yrow / a.Hp, y = yrow - z * a.Hp;
+                row = a.S + (((size_t)q * 2 * a.zp + z) * 2 * a.Hp + y) * W;
+            }
         }
         const PT* vp = reinterpret_cast<const PT*>(a.v) + (img * a.H + yrow) * (W / 2);
         F::for_each_io(t, [&](int i, int m) { arr[i] = IOP::load(vp + m); });
@@ -140,7 +159,7 @@ fft2d_row_kernel(Fft2dArgs a)
     } else {
         const int c = q / a.B, b = q % a.B;
         const size_t img = (size_t)b * a.C + c;
-        float2* row = a.S + ((size_t)qi * a.H + yrow) * W;
+        float2* row = scratch_row(a, qi, yrow);
         R::unsplit_inverse(arr, sm, row, t);
         const void* xn = a.x[0];
 #pragma unroll
@@ -182,14 +201,18 @@ struct Fft2dCols {
     static_assert(THREADS <= 1024 && SMEM <= 227 * 1024, "column kernel geometry");
 };
 
-// Column kernel.  SPECTRUM = false: column FFTs of the scratch, spectral
-// multiply with the packed 2-D filter spectrum and the bias, inverse column
-// FFTs, rows y < H back to the scratch.  SPECTRUM = true: forward column
-// FFTs of rows y < H of the packed spectra, all 2H rows written back.
-template <int LOG2H2, bool SPECTRUM>
+// Column kernel.  MODE 0: column FFTs of the scratch, spectral multiply
+// with the packed 2-D filter spectrum and the bias, inverse column FFTs,
+// rows y < H back to the scratch.  MODE 1: forward column FFTs of rows
+// y < H of each plane (the packed spectra, or 3-D scratch planes), all 2H
+// rows written back; with zp, plane q of the filter spectra is plane
+// q % zp of filter q / zp at a pitch of 2 zp planes.  MODE 2 (3-D): inverse
+// column FFTs of all 2H rows of each plane, rows y < H written back.
+template <int LOG2H2, int MODE>
 __global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS, Fft2dCols<LOG2H2>::MIN_BLOCKS)
 fft2d_col_kernel(Fft2dArgs a)
 {
+    constexpr bool SPECTRUM = MODE == 1;
     grid_dependency_begin();
     using CL = Fft2dCols<LOG2H2>;
     using FC = typename CL::FC;
@@ -205,11 +228,26 @@ fft2d_col_kernel(Fft2dArgs a)
     const int cc = tid % TC, t = tid / TC;
     const int kx = kx0 + cc;
     float2* buf = smem_c2 + cc * CL::STRIDE;
-    // rows of this image's column kx: scratch [H][W] or spectra [2H][W]
-    float2* col = SPECTRUM ? a.S + (size_t)q * H2 * W + kx : a.S + (size_t)qi * HH * W + kx;
+    // rows of this image's column kx: scratch [H][W] or planes [2H][W]
+    const size_t pq = (MODE == 1 && a.zp) ? (size_t)(q / a.zp) * 2 * a.zp + q % a.zp : (size_t)q;
+    float2* col = MODE != 0 ? a.S + pq * H2 * W + kx : a.S + (size_t)qi * HH * W + kx;
     float2 reg[V];
     const int pt = pad16(t);
 
+    if constexpr (MODE == 2) {
+        // inverse column FFT of all 2H rows, rows y < H back
+        static_for<V>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            buf[pad16_at<H2 / V>(t, pt, r)] = col[(size_t)(t + r * (H2 / V)) * W];
+        });
+        __syncthreads();
+        FC::template run<+1, true>(buf, reg, t);
+        static_for<V / 2>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            col[(size_t)(t + r * (H2 / V)) * W] = reg[r];
+        });
+        return;
+    }
     static_for<V>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
         const int y = t + r * (H2 / V);

@@ -4,6 +4,7 @@
 
 #include "k_circular.cuh"
 #include "k_fft2d.cuh"
+#include "k_fft3d.cuh"
 #include "launch.cuh"
 
 using namespace hyena;
@@ -585,5 +586,122 @@ hyena_status_t forward2d_impl(const void* v, const void* const* x, const float* 
 }  // namespace
 
 extern "C" {
+
+}  // extern "C"
+
+namespace {
+
+bool dims3d_ok(int Z, int H, int W, int& lz, int& lh, int& lw)
+{
+    lz = exact_log2(Z);
+    lh = exact_log2(H);
+    lw = exact_log2(W);
+    return lz >= kMinLog2_3d && lz <= kMaxLog2_3d && lh >= kMinLog2_3d && lh <= kMaxLog2_3d &&
+           lw >= kMinLog2_3d && lw <= kMaxLog2_3d;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hyena_fftconv3d_workspace_size(int B, int C, int Z, int H, int W, int N, hyena_dtype_t io,
+                                      int spectrum_given)
+{
+    if (B < 1 || C < 1 || N < 1 || N > HYENA_MAX_ORDER || (io != HYENA_F32 && io != HYENA_BF16))
+        return (size_t)-1;
+    int lz, lh, lw;
+    if (!dims3d_ok(Z, H, W, lz, lh, lw)) return (size_t)-1;
+    const size_t vol2 = (size_t)Z * 2 * H * W;                  // slots of one scratch volume
+    size_t need = spectrum_given ? 0 : round_up(sizeof(float2) * (size_t)N * C * 2 * vol2, 256);
+    return need + round_up(sizeof(float2) * (size_t)wave_images_3d((long)B * C, Z, H, W) * vol2, 256);
+}
+
+hyena_status_t hyena_filter_rfft3d(const float* h, int N, int C, int Z, int H, int W, float* Hs, void* stream)
+{
+    if (!h || !Hs || N < 1 || C < 1 || Z < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
+    int lz, lh, lw;
+    if (!dims3d_ok(Z, H, W, lz, lh, lw)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)N * C * Z * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    if (!aligned(h, 16) || !aligned(Hs, 16)) return HYENA_ERR_INVALID_ARG;
+    if (overlap(h, sizeof(float) * (size_t)N * C * Z * H * W, Hs,
+                sizeof(float2) * (size_t)N * C * 4 * Z * H * W))
+        return HYENA_ERR_INVALID_ARG;
+    Fft2dArgs a = {};
+    a.v = h;
+    a.S = reinterpret_cast<float2*>(Hs);
+    a.B = 1;
+    a.C = N * C;
+    a.W = W;
+    a.nq = N * C;
+    a.zp = Z;
+    a.Hp = H;
+    return dispatch_rfft3d(lw, lh, lz, a, (cudaStream_t)stream);
+}
+
+hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void* const* x, const float* h,
+                                            const float* Hs, const float* bias, int B, int C, int Z,
+                                            int H, int W, int N, hyena_dtype_t io, void* y,
+                                            void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!v || !x || !y || !bias || (!h && !Hs)) return HYENA_ERR_INVALID_ARG;
+    if (B < 1 || C < 1 || N < 1 || Z < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
+    if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
+    int lz, lh, lw;
+    if (!dims3d_ok(Z, H, W, lz, lh, lw)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)B * C > (1L << 20) || (long)N * C * Z * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    for (int n = 0; n < N; ++n)
+        if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(v, 16) || !aligned(y, 16) || !aligned(bias, 4)) return HYENA_ERR_INVALID_ARG;
+    if ((Hs && !aligned(Hs, 16)) || (!Hs && !aligned(h, 16))) return HYENA_ERR_INVALID_ARG;
+
+    const size_t vol = (size_t)Z * H * W;
+    const size_t act = (size_t)B * C * vol * io_bytes(io);
+    const size_t spec = sizeof(float2) * (size_t)N * C * 4 * vol;
+    const size_t filt = sizeof(float) * (size_t)N * C * vol;
+    const size_t need = hyena_fftconv3d_workspace_size(B, C, Z, H, W, N, io, Hs != nullptr);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+    if (overlap(y, act, v, act) || overlap(y, act, bias, sizeof(float) * N * C) ||
+        (Hs && overlap(y, act, Hs, spec)) || (!Hs && overlap(y, act, h, filt)) ||
+        overlap(y, act, workspace, need) || overlap(workspace, need, v, act) ||
+        (Hs && overlap(workspace, need, Hs, spec)) || (!Hs && overlap(workspace, need, h, filt)))
+        return HYENA_ERR_INVALID_ARG;
+    for (int n = 0; n < N; ++n)
+        if (overlap(y, act, x[n], act) || overlap(workspace, need, x[n], act))
+            return HYENA_ERR_INVALID_ARG;
+
+    cudaStream_t st = (cudaStream_t)stream;
+    char* ws = static_cast<char*>(workspace);
+    const float2* spectrum = reinterpret_cast<const float2*>(Hs);
+    if (!Hs) {
+        Fft2dArgs sa = {};
+        sa.v = h;
+        sa.S = reinterpret_cast<float2*>(ws);
+        sa.B = 1;
+        sa.C = N * C;
+        sa.W = W;
+        sa.nq = N * C;
+        sa.zp = Z;
+        sa.Hp = H;
+        hyena_status_t s = dispatch_rfft3d(lw, lh, lz, sa, st);
+        if (s != HYENA_OK) return s;
+        spectrum = sa.S;
+        ws += round_up(spec, 256);
+    }
+    Fft2dArgs a = {};
+    a.v = v;
+    for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
+    a.y = y;
+    a.Hs = spectrum;
+    a.bias = bias;
+    a.B = B;
+    a.C = C;
+    a.W = W;
+    a.zp = Z;
+    a.Hp = H;
+    float2* scratch = reinterpret_cast<float2*>(ws);
+    return io == HYENA_BF16 ? dispatch_fft3d_bf16(lw, lh, lz, a, N, scratch, st)
+                            : dispatch_fft3d_f32(lw, lh, lz, a, N, scratch, st);
+}
 
 }  // extern "C"

@@ -19,7 +19,7 @@ inline long wave_images(long nimg, long H, long W)
 }
 
 // column launches (one 2H-point column FFT per slot column)
-hyena_status_t launch_cols2d(int log2h, bool spectrum, const Fft2dArgs& a, cudaStream_t st);
+hyena_status_t launch_cols2d(int log2h, int mode, const Fft2dArgs& a, cudaStream_t st);
 
 template <int LOG2W, typename IO, int MODE>
 hyena_status_t launch_rows2d(const Fft2dArgs& a, cudaStream_t st)
@@ -43,7 +43,7 @@ hyena_status_t run_fft2d(Fft2dArgs a, int N, int log2h, float2* scratch, cudaStr
         hyena_status_t s = launch_rows2d<LOG2W, IO, 0>(a, st);
         for (int n = 0; n < N && s == HYENA_OK; ++n) {
             a.n = n;
-            s = launch_cols2d(log2h, false, a, st);
+            s = launch_cols2d(log2h, 0, a, st);
             if (s != HYENA_OK) break;
             s = n + 1 < N ? launch_rows2d<LOG2W, IO, 1>(a, st) : launch_rows2d<LOG2W, IO, 2>(a, st);
         }

@@ -76,6 +76,10 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv2d_workspace_size": ([i, i, i, i, i, i, i], sz),
         "hyena_fftconv2d_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
                                           vp, sz, vp], i),
+        "hyena_filter_rfft3d": ([vp, i, i, i, i, i, vp, vp], i),
+        "hyena_fftconv3d_workspace_size": ([i, i, i, i, i, i, i, i], sz),
+        "hyena_fftconv3d_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, i,
+                                          vp, vp, sz, vp], i),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -404,6 +408,51 @@ def hyena_fftconv2d_gate_forward_per_sample(v: torch.Tensor, xs, bias: torch.Ten
     _check("hyena_fftconv2d_gate_forward_per_sample", LIB.hyena_fftconv2d_gate_forward_per_sample(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, H, W, N, io,
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def hyena_filter_rfft3d(h: torch.Tensor, *, out=None, stream=None):
+    """Packed 3-D spectra [N][C][2Z][2H][W] complex64 of the filters h
+    [N][C][Z][H][W] zero-padded to 2Z x 2H x 2W (slot [kz][ky][0] holds
+    the bin-0 + i bin-W pair)."""
+    N, C, Z, H, W = h.shape
+    if out is None:
+        out = torch.empty((N, C, 2 * Z, 2 * H, W), device=h.device, dtype=torch.complex64)
+    _check("hyena_filter_rfft3d", LIB.hyena_filter_rfft3d(
+        ctypes.c_void_p(_dev(h, torch.float32, "h")), N, C, Z, H, W,
+        ctypes.c_void_p(_dev(out, torch.complex64, "Hs")), _stream(stream)))
+    return out
+
+
+def hyena_fftconv3d_workspace_size(B: int, C: int, Z: int, H: int, W: int, N: int, io: int,
+                                   spectrum_given: bool) -> int:
+    n = LIB.hyena_fftconv3d_workspace_size(B, C, Z, H, W, N, io, int(bool(spectrum_given)))
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv3d_workspace_size", HYENA_ERR_INVALID_ARG, "invalid sizes")
+    return n
+
+
+def hyena_fftconv3d_gate_forward(v: torch.Tensor, xs, bias: torch.Tensor, *, Hs=None, h=None,
+                                 out=None, workspace=None, stream=None):
+    """3-D order-N forward: v, x_n [B][C][Z][H][W] (float32 or bf16), bias
+    [N][C], and the packed spectra Hs [N][C][2Z][2H][W] or the filters h
+    [N][C][Z][H][W]."""
+    B, C, Z, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    need = hyena_fftconv3d_workspace_size(B, C, Z, H, W, N, io, Hs is not None)
+    if workspace is None:
+        workspace = torch.empty(need, device=v.device, dtype=torch.uint8)
+    Hp = ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")) if Hs is not None else None
+    hp = ctypes.c_void_p(_dev(h, torch.float32, "h")) if h is not None else None
+    _check("hyena_fftconv3d_gate_forward", LIB.hyena_fftconv3d_gate_forward(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, hp, Hp,
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, Z, H, W, N, io,
         ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out

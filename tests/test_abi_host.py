@@ -227,3 +227,37 @@ def test_binding_refuses_cpu_tensors():
     v = torch.zeros(1, 1, 16)
     with pytest.raises(TypeError):
         hyena.hyena_fftconv_gate_forward(v, [v], torch.zeros(1, 1), H=torch.zeros(1, 1, 16, dtype=torch.complex64))
+
+
+def test_3d_rejects_bad_arguments(lib):
+    from subquadratic_sequence_b200 import hyena
+    ws = lib.hyena_fftconv3d_workspace_size
+    n = ws(2, 3, 16, 32, 64, 2, F32, 1)
+    assert n >= 2 * 3 * 16 * 64 * 64 * 8 and n % 256 == 0
+    assert ws(2, 3, 16, 32, 64, 2, F32, 0) >= n + 2 * 3 * 32 * 64 * 64 * 8
+    assert ws(2, 3, 8, 32, 64, 2, F32, 1) == ctypes.c_size_t(-1).value           # Z < 16
+    assert ws(2, 3, 16, 512, 64, 2, F32, 1) == ctypes.c_size_t(-1).value         # H > 256
+    assert ws(2, 3, 16, 32, 48, 2, F32, 1) == ctypes.c_size_t(-1).value          # W not a power of two
+    with pytest.raises(hyena.HyenaError):
+        hyena.hyena_fftconv3d_workspace_size(2, 3, 16, 16, 16, 17, F32, True)
+
+    r = lib.hyena_filter_rfft3d
+    assert r(None, 2, 3, 16, 16, 16, P(1), None) == INVALID
+    assert r(P(0), 2, 3, 16, 16, 24, P(1), None) == UNSUPPORTED
+    assert r(P(0), 2, 3, 512, 16, 16, P(1), None) == UNSUPPORTED
+    assert r(P(0), 2, 3, 16, 16, 16, ctypes.c_void_p(A + BIG + 8), None) == INVALID
+    assert r(P(0), 2, 3, 16, 16, 16, P(0), None) == INVALID                       # Hs overlaps h
+
+    f = lib.hyena_fftconv3d_gate_forward
+    xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
+    need = ws(2, 3, 16, 16, 16, 2, F32, 1)
+    args = lambda **k: [k.get("v", P(0)), k.get("xs", xs), None, k.get("Hs", P(3)), P(4), 2, 3,
+                        k.get("Z", 16), 16, 16, 2, k.get("io", F32), k.get("y", P(5)),
+                        k.get("wsp", P(6)), k.get("nb", need), None]
+    assert f(*args(v=None)) == INVALID
+    assert f(*args(io=7)) == INVALID
+    assert f(*args(Z=32 + 1)) == UNSUPPORTED
+    assert f(*args(y=P(0))) == INVALID                                           # y aliases v
+    assert f(*args(nb=need - 256)) == WORKSPACE
+    assert f(*args(wsp=ctypes.c_void_p(A + BIG + 16))) == WORKSPACE              # misaligned
+    assert f(*args(xs=(ctypes.c_void_p * 2)(P(1).value, None))) == INVALID
