@@ -41,6 +41,13 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 def describe(wl: synth.Workload) -> dict:
+    if wl.kind == "3d":
+        return {"workload": f"{wl.name}: order-{wl.N} Hyena 3-D operator, B={wl.B}, C={wl.D}, "
+                            f"{wl.Z}x{wl.H}x{wl.W} volumes (padded to {2 * wl.Z}x{2 * wl.H}x{2 * wl.W}), "
+                            f"{wl.io} storage, fp32 compute",
+                "N": wl.N, "B": wl.B, "C": wl.D, "Z": wl.Z, "H": wl.H, "W": wl.W, "io": wl.io,
+                "filters": "given (seeded decaying random volumes); their 3-D spectra recomputed every step",
+                "l2": "flushed (256 MB write) before every timed step"}
     if wl.kind == "2d":
         return {"workload": f"{wl.name}: order-{wl.N} Hyena 2-D operator, B={wl.B}, C={wl.D}, "
                             f"{wl.H}x{wl.W} grid (padded to {2 * wl.H}x{2 * wl.W}), {wl.io} storage, fp32 compute",
@@ -62,7 +69,10 @@ def describe(wl: synth.Workload) -> dict:
 
 def alg_bytes_forward(wl: synth.Workload) -> int:
     """Algorithmic HBM bytes of one forward call: v, x_1..x_N, y plus the
-    N*D packed spectra (L complex64 slots each; 2H x W for the 2-D grid)."""
+    N*D packed spectra (L complex64 slots each; 2H x W for the 2-D grid,
+    2Z x 2H x W for the 3-D volume)."""
+    if wl.kind == "3d":
+        return (wl.N + 2) * wl.positions * wl.io_bytes + wl.N * wl.D * 4 * wl.Z * wl.H * wl.W * 8
     if wl.kind == "2d":
         return (wl.N + 2) * wl.positions * wl.io_bytes + wl.N * wl.D * 2 * wl.H * wl.W * 8
     sets = wl.B if wl.film else 1          # filter spectra per sample, or shared by the batch
@@ -89,12 +99,18 @@ def waves(nseq: int, L: int) -> int:
 
 def launches_forward(wl: synth.Workload) -> int:
     """Kernel launches of one forward call."""
+    if wl.kind == "3d":
+        # per wave: rows, columns, then per order z, inverse columns, rows
+        # (and forward columns before every order but the first)
+        return waves(wl.B * wl.D, 2 * wl.Z * wl.H * wl.W) * (4 * wl.N + 1)
     if wl.kind == "2d":
         return waves(wl.B * wl.D, wl.H * wl.W) * (1 + 2 * wl.N)
     return waves(wl.B * wl.D, wl.L) * (1 + 2 * wl.N) if long_path(wl) else 1
 
 
 def launches_rfft(wl: synth.Workload) -> int:
+    if wl.kind == "3d":
+        return 3
     if wl.kind == "2d":
         return 2
     rows = wl.N * wl.D * (wl.B if wl.film else 1)
@@ -102,12 +118,16 @@ def launches_rfft(wl: synth.Workload) -> int:
 
 
 def launches_filter_gen(wl: synth.Workload) -> int:
+    if wl.kind == "3d":
+        return 0
     return 3 if wl.N * wl.D > 64 else 1
 
 
 def forward_kernel(wl: synth.Workload) -> str:
     """The timed unit of the roofline: the forward call (one fused kernel,
     or the 2N+1 four-step kernels of each wave)."""
+    if wl.kind == "3d":
+        return "fft2d_row_kernel+fft2d_col_kernel+fft3d_z_kernel (hyena_fftconv3d_gate_forward, all launches)"
     if wl.kind == "2d":
         return "fft2d_row_kernel+fft2d_col_kernel (hyena_fftconv2d_gate_forward, all launches)"
     if long_path(wl):
@@ -277,11 +297,24 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     v = to_dev(inp["v"], io)
     xs = [to_dev(x, io) for x in inp["x"]]
     b = to_dev(inp["b"])
-    W = [to_dev(inp[k]) for k in ("W1", "W2", "W3", "Wout", "alpha")]
+    wkeys = ("h",) if wl.kind == "3d" else ("W1", "W2", "W3", "Wout", "alpha")
+    W = [to_dev(inp[k]) for k in wkeys]
     y = torch.empty_like(v)
     flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
     stream = torch.cuda.current_stream()
-    if wl.kind == "2d":
+    if wl.kind == "3d":
+        h = W[0]
+        H = torch.empty((wl.N, wl.D, 2 * wl.Z, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
+        ws_n = hyena.hyena_fftconv3d_workspace_size(wl.B, wl.D, wl.Z, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
+        ws_fwd = torch.empty(ws_n, device="cuda", dtype=torch.uint8)
+
+        def forward():
+            hyena.hyena_fftconv3d_gate_forward(v, xs, b, Hs=H, out=y, workspace=ws_fwd)
+
+        def step():
+            hyena.hyena_filter_rfft3d(h, out=H)
+            forward()
+    elif wl.kind == "2d":
         h = torch.empty((wl.N, wl.D, wl.H, wl.W), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.N, wl.D, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
         ws_n = hyena.hyena_fftconv2d_workspace_size(wl.B, wl.D, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
@@ -384,8 +417,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     hv = torch.from_numpy(np.ascontiguousarray(inp["v"], np.float32)).to(io).pin_memory()
     hxs = [torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(io).pin_memory() for x in inp["x"]]
     hb = torch.from_numpy(inp["b"]).pin_memory()
-    hW = [torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
-          for k in ("W1", "W2", "W3", "Wout", "alpha")]
+    hW = [torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory() for k in wkeys]
     dW = list(W)
     if wl.film:   # the per-sample control vectors are step inputs as well
         hW += [torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
@@ -480,6 +512,16 @@ def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: 
     t0 = time.perf_counter()
     v = inp["v"][:, channels].astype(np.float64)
     x = np.stack([xx[:, channels] for xx in inp["x"]]).astype(np.float64)
+    bias = inp["b"][:, channels].astype(np.float64)
+    if wl.kind == "3d":
+        oracle.hyena_forward_3d(v, x, inp["h"][:, channels].astype(np.float64), bias, route="fft")
+        return time.perf_counter() - t0
+    if wl.kind == "2d":
+        h = oracle.filter_gen_2d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
+                                 wl.N, len(channels), wl.H, wl.W, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                 decay_div=synth.DECAY_DIV, threads=threads)
+        oracle.hyena_forward_2d(v, x, h, bias, route="fft", threads=threads)
+        return time.perf_counter() - t0
     if wl.film:
         h = oracle.filter_gen_film(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["omega"],
                                    inp["gamma"], inp["beta"], inp["sigma"][channels], True, wl.N,
@@ -496,22 +538,37 @@ def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: 
     return time.perf_counter() - t0
 
 
+def extent(wl: synth.Workload) -> str:
+    if wl.kind == "3d":
+        return f"{wl.Z}x{wl.H}x{wl.W}"
+    if wl.kind == "2d":
+        return f"{wl.H}x{wl.W}"
+    return f"L={wl.L}"
+
+
+def stages(wl: synth.Workload) -> str:
+    if wl.kind == "3d":
+        return f"3-D spectra + order-{wl.N} forward, one thread"
+    return f"filter generation + order-{wl.N} forward"
+
+
 def cpu_baseline(wl: synth.Workload, budget_s: float = 15.0, inp: dict | None = None) -> dict:
     import oracle
     inp = inp or synth.make_inputs(wl)
     threads = oracle.default_threads()
     rng = np.random.default_rng(0)
-    n = max(1, min(wl.D, threads))
+    n = 1 if wl.kind == "3d" else max(1, min(wl.D, threads))   # the 3-D oracle runs on one thread
     t = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
     # grow the sample to about budget_s of CPU work
     n2 = int(min(wl.D, max(n, n * budget_s / max(t, 1e-3))))
     if n2 > n:
         n = n2
         t = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
-    positions = wl.B * n * wl.L
-    return {"value": positions / t, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n} of {wl.D} channels x all {wl.B} batch elements x L={wl.L} "
-                      f"(filter generation + order-{wl.N} forward, float64 FFT route), {t:.1f} s"}
+    positions = wl.B * n * wl.per_channel
+    cores = 1 if wl.kind == "3d" else threads
+    return {"value": positions / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {wl.D} channels x all {wl.B} batch elements x {extent(wl)} "
+                      f"({stages(wl)}, float64 FFT route), {t:.1f} s"}
 
 
 def run_reference(args, wl: synth.Workload) -> dict | None:
@@ -523,7 +580,7 @@ def run_reference(args, wl: synth.Workload) -> dict | None:
     inp = synth.make_inputs(wl)
     threads = oracle.default_threads()
     rng = np.random.default_rng(0)
-    n = max(1, min(wl.D, threads))
+    n = 1 if wl.kind == "3d" else max(1, min(wl.D, threads))   # the 3-D oracle runs on one thread
     probe = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
     # size each step so that warm-up + timed steps end within ~2 minutes
     per_step_budget = 120.0 / max(1, args.steps + args.warmup)
@@ -532,10 +589,11 @@ def run_reference(args, wl: synth.Workload) -> dict | None:
     for i in range(args.warmup):
         oracle_sample(wl, inp, chans[i], threads)
     total = sum(oracle_sample(wl, inp, chans[args.warmup + i], threads) for i in range(args.steps))
-    positions = wl.B * n * wl.L
+    positions = wl.B * n * wl.per_channel
     value = positions * args.steps / total
-    sample = (f"{n} of {wl.D} channels x all {wl.B} batch elements x L={wl.L} per step "
-              f"(filter generation + order-{wl.N} forward, float64 FFT route)")
+    sample = (f"{n} of {wl.D} channels x all {wl.B} batch elements x {extent(wl)} per step "
+              f"({stages(wl)}, float64 FFT route)")
+    threads = 1 if wl.kind == "3d" else threads
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

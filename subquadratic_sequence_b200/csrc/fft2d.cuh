@@ -248,13 +248,12 @@ fft2d_col_kernel(Fft2dArgs a)
         });
         return;
     }
-    static_for<V>([&](auto rr) {
+    static_for<V / 2>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
-        const int y = t + r * (H2 / V);
-        buf[pad16_at<H2 / V>(t, pt, r)] = r < V / 2 ? col[(size_t)y * W] : make_float2(0.0f, 0.0f);
+        buf[pad16_at<H2 / V>(t, pt, r)] = col[(size_t)(t + r * (H2 / V)) * W];
     });
     __syncthreads();
-    FC::template run<-1, true>(buf, reg, t);
+    FC::template run<-1, true, true>(buf, reg, t);
     if constexpr (SPECTRUM) {
         static_for<V>([&](auto rr) {
             constexpr int r = decltype(rr)::value;

@@ -32,107 +32,141 @@ struct Fft3dZ {
     static constexpr int THREADS = TC * FZ::T;
     static constexpr int STRIDE = stride_mod16(Z2, 16 / (TC > 16 ? 16 : TC));
     static constexpr size_t SMEM = sizeof(float2) * TC * STRIDE;
+    // resident CTAs per SM the register budget aims at: 96 registers a
+    // thread (128 for one-warp CTAs; no cap with 32 values a thread)
+    static constexpr int REGS = THREADS < 64 ? 128 : 96;
+    static constexpr int MIN_BLOCKS = FZ::V == 32 ? 1 : 65536 / (THREADS * REGS);
     static_assert(THREADS <= 1024 && SMEM <= 227 * 1024, "z kernel geometry");
 };
 
-// z kernel.  MODE 0 (forward): per image qi of the wave, CTAs over
-// (ky, block of TC slots kx) take the z transform of kx != 0, multiply,
-// and transform back (planes z < Z kept); then one CTA per pair u in
-// [0, H] takes slot 0 of rows ky = u and 2H - u together.  MODE 1
-// (spectra): forward z transform of every slot of the filters' planes
-// z < Z, all 2Z planes written.
+// z kernel.  MODE 0 (forward): CTAs per channel of the wave over (ky,
+// block of TC slots kx) hold the channel's filter column (the 2Z spectrum
+// values of their slots, bias and scale folded in) in registers and apply
+// it to every volume of that channel in the wave: z transform, multiply,
+// inverse, planes z < Z kept.  kx = 0 is left to the pair CTAs: each takes
+// TC/2 pairs u in [0, H], slot 0 of rows ky = u (column 2j) and 2H - u
+// (column 2j + 1).  MODE 1 (spectra): forward z transform of every slot of
+// the filters' planes z < Z, all 2Z planes written.
 template <int LOG2Z2, int MODE>
-__global__ void __launch_bounds__(Fft3dZ<LOG2Z2>::THREADS)
+__global__ void __launch_bounds__(Fft3dZ<LOG2Z2>::THREADS, Fft3dZ<LOG2Z2>::MIN_BLOCKS)
 fft3d_z_kernel(Fft2dArgs a)
 {
     grid_dependency_begin();
     using ZL = Fft3dZ<LOG2Z2>;
     using FZ = typename ZL::FZ;
-    constexpr int Z2 = ZL::Z2, TC = ZL::TC, ZH = Z2 / 2, V = FZ::V;
+    constexpr int Z2 = ZL::Z2, TC = ZL::TC, ZH = Z2 / 2, V = FZ::V, NP = TC / 2;
     const int W = a.W, H2 = 2 * a.Hp;
     const int kxb = W / TC;                               // slot blocks per row
-    const long reg_per_img = (long)H2 * kxb;              // regular CTAs per image
+    const long reg_per = (long)H2 * kxb;                  // regular CTAs per image / channel
     extern __shared__ __align__(16) float2 smem_z[];
     const int tid = threadIdx.x;
     const int cc = tid % TC, t = tid / TC;
     float2* buf = smem_z + cc * ZL::STRIDE;
     const int pt = pad16(t);
     const size_t plane = (size_t)H2 * W;                  // slots per plane
+    const long blk = blockIdx.x;
     float2 reg[V];
 
-    // which image and which columns this CTA takes
-    const long blk = blockIdx.x;
-    const bool pair_cta = MODE == 0 && blk >= (long)a.nq * reg_per_img;
-    int qi, ky, kx;
-    if (!pair_cta) {
-        qi = (int)(blk / reg_per_img);
-        const long rem = blk % reg_per_img;
-        ky = (int)(rem / kxb);
-        kx = (int)(rem % kxb) * TC + cc;
-    } else {
-        const long pb = blk - (long)a.nq * reg_per_img;
-        qi = (int)(pb / (a.Hp + 1));
-        const int u = (int)(pb % (a.Hp + 1));
-        // columns 0 and 1: slot 0 of rows u and 2H - u (one row when they coincide)
-        ky = cc == 0 ? u : (H2 - u) % H2;
-        kx = 0;
-    }
-    const int q = a.q0 + qi;
-    const size_t zplanes = MODE == 1 ? (size_t)2 * a.zp : (size_t)a.zp;   // planes allocated per image
-    float2* colp = a.S + (size_t)qi * zplanes * plane + (size_t)ky * W + kx;
-    // a CTA column that writes: regular columns kx != 0 (all in MODE 1),
-    // and the pair CTA's first two columns (the second only if distinct)
-    const bool self_pair = pair_cta && (ky == (H2 - ky) % H2);
-    const bool live = !pair_cta ? (MODE == 1 || kx != 0) : (cc == 0 || (cc == 1 && !(ky == 0 || 2 * ky == H2)));
-
-    // forward z transform of planes z < Z (zero beyond)
-    static_for<V>([&](auto rr) {
-        constexpr int r = decltype(rr)::value;
-        const int z = t + r * (Z2 / V);
-        buf[pad16_at<Z2 / V>(t, pt, r)] = (r < V / 2 && (live || pair_cta)) ? colp[(size_t)z * plane]
-                                                                             : make_float2(0.0f, 0.0f);
-    });
-    __syncthreads();
-    FZ::template run<-1, true>(buf, reg, t);
-    if constexpr (MODE == 1) {
-        if (live)
-            static_for<V>([&](auto rr) {
-                constexpr int r = decltype(rr)::value;
-                colp[(size_t)(t + r * (Z2 / V)) * plane] = reg[r];
-            });
-        return;
-    } else {
-        static_for<V>([&](auto rr) {
+    // planes z < Z of a slot column into the buffer (the upper half is
+    // zero padding, which the forward transform does not read)
+    auto load_col = [&](const float2* colp) {
+        static_for<V / 2>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            buf[pad16_at<Z2 / V>(t, pt, r)] = reg[r];
+            buf[pad16_at<Z2 / V>(t, pt, r)] = colp[(size_t)(t + r * (Z2 / V)) * plane];
         });
         __syncthreads();
-        const int c = q / a.B;
+    };
+
+    if constexpr (MODE == 1) {
+        const int qi = (int)(blk / reg_per);
+        const long rem = blk % reg_per;
+        const int ky = (int)(rem / kxb), kx = (int)(rem % kxb) * TC + cc;
+        float2* colp = a.S + (size_t)qi * 2 * a.zp * plane + (size_t)ky * W + kx;
+        load_col(colp);
+        FZ::template run<-1, true, true>(buf, reg, t);
+        static_for<V>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            colp[(size_t)(t + r * (Z2 / V)) * plane] = reg[r];
+        });
+        return;
+    } else {
+        const int cfirst = a.q0 / a.B;
+        const int nch = (a.q0 + a.nq - 1) / a.B - cfirst + 1;
+        const bool pair_cta = blk >= (long)nch * reg_per;
+        const int npair = (a.Hp + 1 + NP - 1) / NP;       // pair CTAs per channel
+        int ci, ky, kx;
+        bool live;
+        int u = 0;
+        if (!pair_cta) {
+            ci = (int)(blk / reg_per);
+            const long rem = blk % reg_per;
+            ky = (int)(rem / kxb);
+            kx = (int)(rem % kxb) * TC + cc;
+            live = kx != 0;
+        } else {
+            const long pb = blk - (long)nch * reg_per;
+            ci = (int)(pb / npair);
+            u = (int)(pb % npair) * NP + cc / 2;          // this column's pair
+            const bool valid = u <= a.Hp;
+            const int uu = valid ? u : a.Hp;
+            const bool self = uu == 0 || uu == a.Hp;      // rows u and 2H - u coincide
+            ky = (cc % 2 == 0) ? uu : (H2 - uu) % H2;
+            kx = 0;
+            live = valid && (cc % 2 == 0 || !self);
+        }
+        const int c = cfirst + ci;
+        const int qa = max(a.q0, c * a.B), qb = min(a.q0 + a.nq, (c + 1) * a.B);
         const float bias = __ldg(a.bias + a.n * a.C + c);
         const float2* Hn = a.Hs + ((size_t)a.n * a.C + c) * Z2 * plane;   // [2Z][2H][W]
         const float s = 1.0f / ((float)Z2 * (float)H2);
         if (!pair_cta) {
-            if (live)
+            // the filter column, (H + b) / (2Z 2H), in register order
+            float2 hv[V];
+            static_for<V>([&](auto rr) {
+                constexpr int r = decltype(rr)::value;
+                const float2 h = __ldg(Hn + (size_t)(t + r * (Z2 / V)) * plane + (size_t)ky * W + kx);
+                hv[r] = make_float2((h.x + bias) * s, h.y * s);
+            });
+            for (int q = qa; q < qb; ++q) {
+                float2* colp = a.S + (size_t)(q - a.q0) * a.zp * plane + (size_t)ky * W + kx;
+                load_col(colp);
+                FZ::template run<-1, true, true>(buf, reg, t);
                 static_for<V>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    const int kz = t + r * (Z2 / V);
-                    const float2 hv = __ldg(Hn + (size_t)kz * plane + (size_t)ky * W + kx);
-                    const int pk = pad16_at<Z2 / V>(t, pt, r);
-                    buf[pk] = cmul(buf[pk], make_float2((hv.x + bias) * s, hv.y * s));
+                    buf[pad16_at<Z2 / V>(t, pt, r)] = cmul(reg[r], hv[r]);
                 });
+                __syncthreads();
+                FZ::template run<+1, true>(buf, reg, t);
+                if (live)
+                    static_for<V / 2>([&](auto rr) {
+                        constexpr int r = decltype(rr)::value;
+                        colp[(size_t)(t + r * (Z2 / V)) * plane] = reg[r];
+                    });
+            }
         } else {
-            // slot 0: column 0 (row u) pairs with column 1 (row 2H - u, or
-            // itself when u = 0 or H) at kz' = -kz
-            float2* bA = smem_z;                                // column 0
-            float2* bB = self_pair ? smem_z : smem_z + ZL::STRIDE;
-            const int u = ky;                                   // the first column's row (cc == 0 threads)
-            const int u2 = (H2 - u) % H2;
-            const int nkz = self_pair ? ZH + 1 : Z2;
-            if (cc == 0) {
-                for (int kz = t; kz < nkz; kz += FZ::T) {
+            const int u0 = (int)((blk - (long)nch * reg_per) % npair) * NP;
+            for (int q = qa; q < qb; ++q) {
+                float2* colp = a.S + (size_t)(q - a.q0) * a.zp * plane + (size_t)ky * W;
+                load_col(colp);
+                FZ::template run<-1, true, true>(buf, reg, t);
+                static_for<V>([&](auto rr) {
+                    constexpr int r = decltype(rr)::value;
+                    buf[pad16_at<Z2 / V>(t, pt, r)] = reg[r];
+                });
+                __syncthreads();
+                // slot 0 of pair j: column 2j (row u) with column 2j + 1
+                // (row 2H - u, or column 2j itself when u = 0 or H) at kz' = -kz
+                for (int e = tid; e < NP * Z2; e += ZL::THREADS) {
+                    const int j = e / Z2, kz = e % Z2;
+                    const int uj = u0 + j;
+                    const bool self = uj == 0 || uj == a.Hp;
+                    if (uj > a.Hp || (self && kz > ZH)) continue;
+                    const int u2 = (H2 - uj) % H2;
+                    float2* bA = smem_z + (2 * j) * ZL::STRIDE;
+                    float2* bB = self ? bA : smem_z + (2 * j + 1) * ZL::STRIDE;
                     const int kz2 = (Z2 - kz) % Z2;
                     const float2 A = bA[pad16(kz)], Bp = bB[pad16(kz2)];
-                    const float2 p1 = __ldg(Hn + (size_t)kz * plane + (size_t)u * W);
+                    const float2 p1 = __ldg(Hn + (size_t)kz * plane + (size_t)uj * W);
                     const float2 p2 = __ldg(Hn + (size_t)kz2 * plane + (size_t)u2 * W);
                     // X0 = (A + conj B')/2, XW = (A - conj B')/(2i); the filter likewise
                     const float2 x0 = make_float2(0.5f * (A.x + Bp.x), 0.5f * (A.y - Bp.y));
@@ -141,21 +175,18 @@ fft3d_z_kernel(Fft2dArgs a)
                     const float2 hw = make_float2(0.5f * (p1.y + p2.y) + bias, -0.5f * (p1.x - p2.x));
                     const float2 y0 = cmul(x0, h0), yw = cmul(xw, hw);
                     // (kz, u): Y0 + i YW;  (-kz, 2H - u): conj(Y0) + i conj(YW)
-                    const float2 nA = make_float2(s * (y0.x - yw.y), s * (y0.y + yw.x));
-                    const float2 nB = make_float2(s * (y0.x + yw.y), s * (yw.x - y0.y));
-                    if (self_pair && kz2 < kz) continue;        // handled from the partner
-                    if (!(self_pair && kz2 == kz)) bB[pad16(kz2)] = nB;
-                    bA[pad16(kz)] = nA;
+                    bA[pad16(kz)] = make_float2(s * (y0.x - yw.y), s * (y0.y + yw.x));
+                    if (!(self && kz2 == kz)) bB[pad16(kz2)] = make_float2(s * (y0.x + yw.y), s * (yw.x - y0.y));
                 }
+                __syncthreads();
+                FZ::template run<+1, true>(buf, reg, t);
+                if (live)
+                    static_for<V / 2>([&](auto rr) {
+                        constexpr int r = decltype(rr)::value;
+                        colp[(size_t)(t + r * (Z2 / V)) * plane] = reg[r];
+                    });
             }
         }
-        __syncthreads();
-        FZ::template run<+1, true>(buf, reg, t);
-        if (live)
-            static_for<V / 2>([&](auto rr) {
-                constexpr int r = decltype(rr)::value;
-                colp[(size_t)(t + r * (Z2 / V)) * plane] = reg[r];
-            });
     }
 }
 

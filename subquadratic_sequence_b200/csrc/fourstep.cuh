@@ -54,7 +54,11 @@ struct SmemFft {
                             : (LOG2S % 4 == 0) ? 16 : (1 << (LOG2S % 4));   // first pass radix
 
     // PADDED_IN: the input sits at buf[pad16(i)] (else at buf[i]).
-    template <int SIGN, bool PADDED_IN>
+    // ZERO_HI: inputs S/2 .. S-1 are zero (a zero-padded transform): the
+    // first pass neither reads them nor multiplies by them, so the caller
+    // need not write them.  In the first pass thread j < S/R reads inputs
+    // j + r S/R, which lie in the upper half exactly when r >= R/2.
+    template <int SIGN, bool PADDED_IN, bool ZERO_HI = false>
     static __device__ __forceinline__ void run(float2* buf, float2* a, int t)
     {
         static_for<NP>([&](auto pp) {
@@ -69,7 +73,10 @@ struct SmemFft {
                 const int pj = pad16(j);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    a[c * R + r] = buf[(p == 0 && !PADDED_IN) ? j + r * (S / R) : pad16_at<S / R>(j, pj, r)];
+                    if constexpr (ZERO_HI && p == 0 && r >= R / 2)
+                        a[c * R + r] = make_float2(0.0f, 0.0f);
+                    else
+                        a[c * R + r] = buf[(p == 0 && !PADDED_IN) ? j + r * (S / R) : pad16_at<S / R>(j, pj, r)];
                 });
             });
             __syncthreads();
@@ -367,13 +374,13 @@ fourstep_col_kernel(FourStepArgs a)
     // twiddle exp(-2 pi i n2 k1 / M)
     {
         const int pt = pad16(t);
-        static_for<V1>([&](auto rr) {
+        static_for<V1 / 2>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            buf[pad16_at<M1 / V1>(t, pt, r)] = r < V1 / 2 ? reg[r] : make_float2(0.0f, 0.0f);
+            buf[pad16_at<M1 / V1>(t, pt, r)] = reg[r];
         });
     }
     __syncthreads();
-    FS::F1::template run<-1, true>(buf, reg, t);
+    FS::F1::template run<-1, true, true>(buf, reg, t);
     float2 w = expi_pi<-1>(2.0f * (float)((n2 * t) % M) / (float)M);
     const float2 step = expi_pi<-1>(2.0f * (float)((n2 * (M1 / V1)) % M) / (float)M);
     static_for<V1>([&](auto rr) {

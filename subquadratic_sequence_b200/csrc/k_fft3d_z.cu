@@ -7,11 +7,15 @@ template <int LOG2Z2>
 hyena_status_t launch_z3d_n(int mode, const Fft2dArgs& a, cudaStream_t st)
 {
     using ZL = Fft3dZ<LOG2Z2>;
-    const long reg = (long)a.nq * 2 * a.Hp * (a.W / ZL::TC);
+    const long reg = 2L * a.Hp * (a.W / ZL::TC);          // regular CTAs per image or channel
     if (mode == 1)
-        return launch(fft3d_z_kernel<LOG2Z2, 1>, (unsigned)reg, ZL::THREADS, ZL::SMEM, st, a, false);
-    const long pairs = (long)a.nq * (a.Hp + 1);
-    return launch(fft3d_z_kernel<LOG2Z2, 0>, (unsigned)(reg + pairs), ZL::THREADS, ZL::SMEM, st, a, false);
+        return launch(fft3d_z_kernel<LOG2Z2, 1>, (unsigned)(a.nq * reg), ZL::THREADS, ZL::SMEM, st, a, false);
+    // channels the wave touches (images are channel-major), each with its
+    // regular CTAs and its pair CTAs
+    const long nch = (long)(a.q0 + a.nq - 1) / a.B - a.q0 / a.B + 1;
+    const long npair = (a.Hp + 1 + ZL::TC / 2 - 1) / (ZL::TC / 2);
+    return launch(fft3d_z_kernel<LOG2Z2, 0>, (unsigned)(nch * (reg + npair)), ZL::THREADS, ZL::SMEM, st, a,
+                  false);
 }
 
 hyena_status_t launch_z3d(int log2z, int mode, const Fft2dArgs& a, cudaStream_t st)

@@ -32,21 +32,38 @@ DECAY_DIV = 64.0
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str        # "1d" or "2d"
+    kind: str        # "1d", "2d" or "3d"
     N: int           # order (number of long convolutions)
     B: int           # batch
     D: int           # channels (C for the 2-D operator)
     L: int = 0       # sequence length (1-D)
     H: int = 0       # grid height (2-D)
     W: int = 0       # grid width (2-D)
+    Z: int = 0       # volume depth (3-D: volumes [Z][H][W])
     io: str = "f32"  # storage type of v, x_n, y: "f32" or "bf16"
     seed: int = 0
     film: bool = False  # input-dependent (per-sample, FiLM-modulated) filters
 
     @property
+    def per_channel(self) -> int:
+        """Positions of one channel's sequence, grid or volume."""
+        if self.kind == "1d":
+            return self.L
+        return self.H * self.W * (self.Z if self.kind == "3d" else 1)
+
+    @property
+    def shape(self) -> tuple:
+        """Shape of the activations v, x_n, y."""
+        if self.kind == "1d":
+            return (self.B, self.D, self.L)
+        if self.kind == "2d":
+            return (self.B, self.D, self.H, self.W)
+        return (self.B, self.D, self.Z, self.H, self.W)
+
+    @property
     def positions(self) -> int:
-        """Channel-positions per forward call: B*D*L (or B*C*H*W)."""
-        return self.B * self.D * (self.L if self.kind == "1d" else self.H * self.W)
+        """Channel-positions per forward call: B*D*L (B*C*H*W, B*C*Z*H*W)."""
+        return self.B * self.D * self.per_channel
 
     @property
     def io_bytes(self) -> int:
@@ -77,6 +94,9 @@ WORKLOADS = {
     # c1 with input-dependent filters: a filter set per sample (FiLM-modulated
     # sine layers, multi-frequency first layer, Gaussian window)
     "c1_film": Workload("c1_film", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), film=True),
+    # order-2 3-D operator on 64^3 volumes, B=2, C=32, bf16 storage (the
+    # filters are inputs: seeded decaying random volumes)
+    "c5_3d": Workload("c5_3d", "3d", N=2, B=2, D=32, Z=64, H=64, W=64, io="bf16", seed=_seed(5)),
 }
 
 
@@ -116,10 +136,12 @@ def make_inputs(wl: Workload) -> dict:
     ``W3``, ``Wout``, ``alpha`` [D].
     """
     rng = np.random.default_rng(wl.seed)
-    shape = (wl.B, wl.D, wl.L) if wl.kind == "1d" else (wl.B, wl.D, wl.H, wl.W)
+    shape = wl.shape
     v = _activation(rng, shape, wl.io)
     x = [_activation(rng, shape, wl.io) for _ in range(wl.N)]
     b = rng.standard_normal((wl.N, wl.D)).astype(np.float32)
+    if wl.kind == "3d":
+        return dict(v=v, x=x, b=b, h=filters_3d(rng, wl.N, wl.D, wl.Z, wl.H, wl.W))
     n_in = 1 + 2 * N_BANDS if wl.kind == "1d" else 2 + 4 * N_BANDS
     W1, W2, W3, Wout = _weights(rng, n_in, WIDTH, wl.N * wl.D)
     alpha = np.linspace(0.3, 1.5, wl.D).astype(np.float32)
@@ -149,5 +171,15 @@ def make_output_grad(wl: Workload) -> np.ndarray:
     the activation shape (bf16-rounded for bf16 storage), from its own
     stream (seed + 1) so the forward inputs are unchanged."""
     rng = np.random.default_rng(wl.seed + 1)
-    shape = (wl.B, wl.D, wl.L) if wl.kind == "1d" else (wl.B, wl.D, wl.H, wl.W)
-    return _activation(rng, shape, wl.io)
+    return _activation(rng, wl.shape, wl.io)
+
+
+def filters_3d(rng: np.random.Generator, N: int, C: int, Z: int, H: int, W: int) -> np.ndarray:
+    """Seeded 3-D filters [N][C][Z][H][W] float32: N(0, 1) values under a
+    separable exponential envelope exp(-4 (iz/Z + iy/H + ix/W)), scaled by
+    8 / sqrt(Z H W) (long, decaying, O(1) response)."""
+    h = rng.standard_normal((N, C, Z, H, W), dtype=np.float32)
+    h *= np.exp(-np.arange(Z, dtype=np.float32) / (Z / 4))[:, None, None]
+    h *= np.exp(-np.arange(H, dtype=np.float32) / (H / 4))[:, None]
+    h *= np.exp(-np.arange(W, dtype=np.float32) / (W / 4))
+    return (h * np.float32(8.0 / np.sqrt(Z * H * W))).astype(np.float32)
