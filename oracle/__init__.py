@@ -67,6 +67,8 @@ def _load():
         "oracle_filter_gen_film_2d": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, i, d, i, dp],
         "oracle_rfft_circ": [dp, l, l, dp, dp],
         "oracle_hyena_forward_circular": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
+        "oracle_cconv3": [dp, dp, l, l, l, i, dp],
+        "oracle_hyena_forward_circular_nd": [dp, dp, dp, dp, l, l, l, l, l, l, i, dp],
     }
     for name, args in sigs.items():
         fn = getattr(lib, name)
@@ -334,3 +336,29 @@ def hyena_forward_3d(v, x, h, bias, route="fft") -> np.ndarray:
     _check(_load().oracle_hyena_forward_3d(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), B, C, Z, H, W, N,
                                            _route(route), _ptr(y)), "oracle_hyena_forward_3d")
     return y
+
+
+def cconv3(h, u, route="direct") -> np.ndarray:
+    """Circular convolution on a Z x H x W grid (a 2-D grid: Z = 1):
+    y[p][q][r] = sum h[i][j][k] u[(p-i) mod Z][(q-j) mod H][(r-k) mod W]."""
+    h, u = _f64(h), _f64(u)
+    Z, H, W = u.shape
+    y = np.empty_like(u)
+    _check(_load().oracle_cconv3(_ptr(h), _ptr(u), Z, H, W, _route(route), _ptr(y)), "oracle_cconv3")
+    return y
+
+
+def hyena_forward_circular_nd(v, x, h, bias, route="fft") -> np.ndarray:
+    """The recurrence with circular convolutions on 2-D grids or 3-D volumes:
+    v [B][C][(Z)][H][W], x [N][B][C][(Z)][H][W], h [N][C][(Z)][H][W],
+    bias [N][C] -> y of v's shape."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    shape = v.shape
+    B, C = shape[:2]
+    Z, H, W = (1,) + shape[2:] if v.ndim == 4 else shape[2:]
+    N = h.shape[0]
+    y = np.empty_like(v)
+    _check(_load().oracle_hyena_forward_circular_nd(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), B, C, Z, H, W, N,
+                                                    _route(route), _ptr(y)), "oracle_hyena_forward_circular_nd")
+    return y
+

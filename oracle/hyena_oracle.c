@@ -1242,3 +1242,91 @@ int oracle_hyena_forward_3d(const double *v, const double *x, const double *h, c
     free(z); free(c);
     return st;
 }
+
+/* ------------------------------------------------------------------ */
+/* Circular convolution on 2-D grids and 3-D volumes (Handling          */
+/* Boundaries: circular convolutions for periodic physical systems; a   */
+/* 2-D grid is a volume with Z = 1).                                    */
+/* ------------------------------------------------------------------ */
+
+/* The definition: y[p][q][r] = sum_{i,j,k} h[i][j][k]
+ * u[(p-i) mod Z][(q-j) mod H][(r-k) mod W]. */
+static void cconv3_direct(const double *h, const double *u, long Z, long H, long W, double *y)
+{
+    for (long p = 0; p < Z; ++p)
+        for (long q = 0; q < H; ++q)
+            for (long r = 0; r < W; ++r) {
+                double s = 0.0;
+                for (long i = 0; i < Z; ++i)
+                    for (long j = 0; j < H; ++j)
+                        for (long k = 0; k < W; ++k) {
+                            const long a = (p - i + Z) % Z, b = (q - j + H) % H, c = (r - k + W) % W;
+                            s += h[(i * H + j) * W + k] * u[(a * H + b) * W + c];
+                        }
+                y[(p * H + q) * W + r] = s;
+            }
+}
+
+/* The convolution theorem on the Z x H x W grid itself (no padding; powers
+ * of two): 3-D DFT of both, multiply, inverse, scale by 1/(Z H W). */
+static int cconv3_fft(const double *h, const double *u, long Z, long H, long W, double *y)
+{
+    const long P = Z * H * W;
+    double *hr = malloc(sizeof(double) * P), *hi = calloc(P, sizeof(double));
+    double *ur = malloc(sizeof(double) * P), *ui = calloc(P, sizeof(double));
+    int st = ORACLE_ENOMEM;
+    if (!hr || !hi || !ur || !ui) goto out;
+    memcpy(hr, h, sizeof(double) * P);
+    memcpy(ur, u, sizeof(double) * P);
+    if ((st = fft3(hr, hi, Z, H, W, -1)) != ORACLE_OK) goto out;
+    if ((st = fft3(ur, ui, Z, H, W, -1)) != ORACLE_OK) goto out;
+    for (long k = 0; k < P; ++k) {
+        const double re = hr[k] * ur[k] - hi[k] * ui[k], im = hr[k] * ui[k] + hi[k] * ur[k];
+        ur[k] = re;
+        ui[k] = im;
+    }
+    if ((st = fft3(ur, ui, Z, H, W, +1)) != ORACLE_OK) goto out;
+    for (long k = 0; k < P; ++k) y[k] = ur[k] / (double)P;
+out:
+    free(hr); free(hi); free(ur); free(ui);
+    return st;
+}
+
+int oracle_cconv3(const double *h, const double *u, long Z, long H, long W, int route, double *y)
+{
+    if (!h || !u || !y || Z < 1 || H < 1 || W < 1) return ORACLE_EBADARG;
+    if (route == ROUTE_DIRECT) {
+        cconv3_direct(h, u, Z, H, W, y);
+        return ORACLE_OK;
+    }
+    if (route != ROUTE_FFT || !is_pow2(Z) || !is_pow2(H) || !is_pow2(W)) return ORACLE_EBADARG;
+    return cconv3_fft(h, u, Z, H, W, y);
+}
+
+/* v [B][C][Z][H][W], x [N][B][C][Z][H][W], h [N][C][Z][H][W], bias [N][C]
+ * -> y [B][C][Z][H][W]: the recurrence with circular convolutions on the
+ * grid (Z = 1 for 2-D), one thread. */
+int oracle_hyena_forward_circular_nd(const double *v, const double *x, const double *h,
+                                     const double *bias, long B, long C, long Z, long H, long W,
+                                     long N, int route, double *y)
+{
+    if (!v || !x || !h || !bias || !y || B < 1 || C < 1 || Z < 1 || H < 1 || W < 1 || N < 1)
+        return ORACLE_EBADARG;
+    const long V = Z * H * W, BCV = B * C * V;
+    double *z = malloc(sizeof(double) * V), *c = malloc(sizeof(double) * V);
+    if (!z || !c) { free(z); free(c); return ORACLE_ENOMEM; }
+    int st = ORACLE_OK;
+    for (long img = 0; img < B * C && st == ORACLE_OK; ++img) {
+        const long ch = img % C;
+        memcpy(z, v + img * V, sizeof(double) * V);
+        for (long n = 0; n < N && st == ORACLE_OK; ++n) {
+            const double *hn = h + (n * C + ch) * V, *xn = x + n * BCV + img * V;
+            const double bn = bias[n * C + ch];
+            st = oracle_cconv3(hn, z, Z, H, W, route, c);
+            for (long t = 0; t < V; ++t) z[t] = xn[t] * (c[t] + bn * z[t]);
+        }
+        memcpy(y + img * V, z, sizeof(double) * V);
+    }
+    free(z); free(c);
+    return st;
+}

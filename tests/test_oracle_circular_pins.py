@@ -69,3 +69,74 @@ def test_circular_forward_routes_agree_and_wrap():
     assert rel_err(yf, yd) < 1e-12
     # and it differs from the causal one (the wrap-around terms)
     assert rel_err(yd, oracle.hyena_forward(v, x, h, b, route="direct")) > 1e-3
+
+
+# ------------------------------------------------------- 2-D grids and 3-D volumes
+
+@pytest.mark.parametrize("shape", [(1, 1, 5), (1, 6, 4), (3, 4, 5), (4, 8, 8)])
+def test_cconv3_direct_is_numpy(shape):
+    r = np.random.default_rng(sum(shape))
+    h, u = r.standard_normal(shape), r.standard_normal(shape)
+    ref = np.real(np.fft.ifftn(np.fft.fftn(h) * np.fft.fftn(u)))
+    assert rel_err(oracle.cconv3(h, u, "direct"), ref) < 1e-12
+
+
+@pytest.mark.parametrize("shape", [(1, 16, 32), (8, 4, 16), (16, 16, 16)])
+def test_cconv3_fft_equals_direct(shape):
+    r = np.random.default_rng(sum(shape) + 1)
+    h, u = r.standard_normal(shape), r.standard_normal(shape)
+    assert rel_err(oracle.cconv3(h, u, "fft"), oracle.cconv3(h, u, "direct")) < 1e-12
+
+
+@pytest.mark.parametrize("k", [(0, 0, 0), (0, 3, 5), (2, 0, 7), (3, 7, 1)])
+def test_cconv3_shift_filter_is_a_rotation(k):
+    shape = (4, 8, 8)
+    u = np.random.default_rng(sum(k)).standard_normal(shape)
+    h = np.zeros(shape)
+    h[k] = 1.0
+    assert np.array_equal(oracle.cconv3(h, u, "direct"), np.roll(u, k, axis=(0, 1, 2)))
+
+
+def test_cconv3_of_a_line_is_the_1d_circular_convolution():
+    r = np.random.default_rng(9)
+    h, u = r.standard_normal(32), r.standard_normal(32)
+    got = oracle.cconv3(h.reshape(1, 1, 32), u.reshape(1, 1, 32), "fft")[0, 0]
+    assert rel_err(got, oracle.cconv(h, u, "direct")) < 1e-12
+
+
+@pytest.mark.parametrize("route", ["direct", "fft"])
+def test_circular_nd_on_padded_volumes_is_the_linear_recurrence(route):
+    # inputs in the low octant of a grid of twice the size and x zero
+    # outside it: the circular recurrence there is the linear 3-D one
+    # (pinned to scipy), and zero elsewhere
+    B, C, Z, H, W, N = 1, 2, 4, 4, 8, 2
+    r = np.random.default_rng(10)
+    v, x = r.standard_normal((B, C, Z, H, W)), r.standard_normal((N, B, C, Z, H, W))
+    h, b = r.standard_normal((N, C, Z, H, W)), r.standard_normal((N, C))
+    pad = lambda a: np.pad(a, [(0, 0)] * (a.ndim - 3) + [(0, Z), (0, H), (0, W)])
+    got = oracle.hyena_forward_circular_nd(pad(v), pad(x), pad(h), b, route=route)
+    want = oracle.hyena_forward_3d(v, x, h, b, route="direct")
+    assert rel_err(got[..., :Z, :H, :W], want) < 1e-12
+    outside = got.copy()
+    outside[..., :Z, :H, :W] = 0.0
+    assert np.max(np.abs(outside)) == 0.0
+
+
+def test_circular_nd_2d_grid_of_one_row_is_the_1d_circular_recurrence():
+    B, C, W, N = 2, 3, 32, 3
+    r = np.random.default_rng(11)
+    v, x = r.standard_normal((B, C, W)), r.standard_normal((N, B, C, W))
+    h, b = r.standard_normal((N, C, W)), r.standard_normal((N, C))
+    got = oracle.hyena_forward_circular_nd(v[:, :, None], x[:, :, :, None], h[:, :, None], b)[:, :, 0]
+    assert rel_err(got, oracle.hyena_forward_circular(v, x, h, b, route="direct")) < 1e-12
+
+
+def test_circular_nd_routes_agree_and_differ_from_linear():
+    B, C, H, W, N = 1, 2, 16, 16, 2
+    r = np.random.default_rng(12)
+    v, x = r.standard_normal((B, C, H, W)), r.standard_normal((N, B, C, H, W))
+    h, b = r.standard_normal((N, C, H, W)), r.standard_normal((N, C))
+    a = oracle.hyena_forward_circular_nd(v, x, h, b, route="fft")
+    d = oracle.hyena_forward_circular_nd(v, x, h, b, route="direct")
+    assert rel_err(a, d) < 1e-12
+    assert rel_err(a, oracle.hyena_forward_2d(v, x, h, b, route="direct")) > 1e-2
