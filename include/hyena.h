@@ -386,6 +386,34 @@ HYENA_API hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void*
                                                       void* y, void* workspace, size_t ws_bytes,
                                                       void* stream);
 
+/* ------------------------------------------------------- circular 2-D */
+
+/* Circular 2-D filter spectra Hs [N][C][H][W/2] complex64 for filters h
+ * [N][C][H][W] (no padding: "Handling Boundaries", circular convolution
+ * for periodic systems).  The packing of hyena_filter_rfft2d at H x W:
+ * slot [ky][kx] = X[ky][kx] for 1 <= kx < W/2, slot [ky][0] = the H-point
+ * DFT over y of R_y[0] + i R_y[W/2] (R_y the W-point DFT of row y).
+ * H a power of two in [16, 1024], W in [32, 1024].  Alignment 16 bytes;
+ * Hs must not overlap h.  No workspace. */
+HYENA_API hyena_status_t hyena_filter_rfft2d_circular(const float* h, int N, int C, int H, int W,
+                                                      float* Hs, void* stream);
+
+/* Bytes of workspace hyena_fftconv2d_gate_forward_circular needs (one wave
+ * of images, H x W/2 complex slots each); (size_t)-1 for invalid sizes. */
+HYENA_API size_t hyena_fftconv2d_circular_workspace_size(int B, int C, int H, int W);
+
+/* The order-N recurrence with circular 2-D convolutions, per image (b, c):
+ *   z_n = x_n * (h_n (*) z_{n-1} + b_n z_{n-1}),
+ *   (h (*) u)[p][q] = sum_{i, j} h[i][j] u[(p-i) mod H][(q-j) mod W].
+ * v, x_n, y [B][C][H][W] io; Hs from hyena_filter_rfft2d_circular; bias
+ * [N][C]; x a HOST array of N device pointers.  Sizes as for the spectra;
+ * alignment and aliasing as hyena_fftconv2d_gate_forward. */
+HYENA_API hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, const void* const* x,
+                                                               const float* Hs, const float* bias, int B,
+                                                               int C, int H, int W, int N, hyena_dtype_t io,
+                                                               void* y, void* workspace, size_t ws_bytes,
+                                                               void* stream);
+
 #ifdef __cplusplus
 }
 #endif

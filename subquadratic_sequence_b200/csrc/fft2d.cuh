@@ -40,7 +40,8 @@ struct Fft2dArgs {
     const float2* Hs;              // [N][C][2H][W] packed 2-D spectra (column kernel)
     const float* bias;             // [N][C]
     float2* S;                     // scratch [wave][H][W] complex (conv) / spectra (filters)
-    int B, C, H, W;
+    int B, C, H;
+    int W;                         // slots per row: the grid width (padded), half of it (circular)
     int q0;                        // first image of the wave (channel-major index)
     int nq;                        // images in the wave
     int n;                         // order handled by this launch
@@ -53,18 +54,22 @@ struct Fft2dArgs {
 };
 
 // Scratch row of row index yrow of image qi (2-D: [H][W] per image; 3-D:
-// plane z = yrow / Hp at a pitch of 2 Hp rows).
+// plane z = yrow / Hp at a pitch of 2 Hp rows, or Hp rows when circular).
+template <bool PAD>
 __device__ __forceinline__ float2* scratch_row(const Fft2dArgs& a, int qi, int yrow)
 {
     if (a.zp == 0) return a.S + ((size_t)qi * a.H + yrow) * a.W;
     const int z = yrow / a.Hp, y = yrow - z * a.Hp;
-    return a.S + (((size_t)qi * a.zp + z) * 2 * a.Hp + y) * a.W;
+    return a.S + (((size_t)qi * a.zp + z) * (PAD ? 2 : 1) * a.Hp + y) * a.W;
 }
 
-template <int LOG2W>
+// Rows as packed real transforms of 2M points: a row of W = M values
+// zero-padded to 2W (PAD), or of W = 2M values taken whole (circular); M
+// slots per row, slot 0 holding bins 0 and M.
+template <int LOG2M, bool PAD = true>
 struct Fft2dRows {
-    using F = Fft1d<LOG2W>;
-    static constexpr int W = 1 << LOG2W;
+    using F = Fft1d<LOG2M, PAD>;
+    static constexpr int W = 1 << LOG2M;               // slots per row
 
     // forward row FFT of the registers (every thread: the passes hold
     // barriers) and, if `store`, the split into a packed row
@@ -114,17 +119,19 @@ struct Fft2dRows {
 // Row kernel.  MODE 0: forward rows from v into the scratch; 1: un-split,
 // inverse rows, gate, forward rows back into the scratch; 2: un-split,
 // inverse rows, gate, store y; 3: forward rows of the filters h into rows
-// y < H of the packed spectra (S = spectra, C = filter rows).
-template <int LOG2W, typename IO, int MODE>
-__global__ void __launch_bounds__(Fft1d<LOG2W>::THREADS)
+// y < H of the packed spectra (S = spectra, C = filter rows).  PAD: rows
+// zero-padded to twice their width, else circular.
+template <int LOG2M, typename IO, int MODE, bool PAD = true>
+__global__ void __launch_bounds__(Fft1d<LOG2M, PAD>::THREADS)
 fft2d_row_kernel(Fft2dArgs a)
 {
     grid_dependency_begin();
-    using R = Fft2dRows<LOG2W>;
+    using R = Fft2dRows<LOG2M, PAD>;
     using F = typename R::F;
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;
-    constexpr int W = R::W, E = F::E, T = F::T;
+    constexpr int W = R::W, E = F::E, T = F::T, SEQ = F::SEQ;   // slots, -, -, value pairs per row
+    constexpr int RP = PAD ? 2 : 1;                              // spectrum rows (planes) per grid row (plane)
     extern __shared__ __align__(16) float2 smem_r2[];
 
     const int g = threadIdx.x / T, t = threadIdx.x % T;
@@ -143,29 +150,29 @@ fft2d_row_kernel(Fft2dArgs a)
         if constexpr (MODE == 0) {
             const int c = q / a.B, b = q % a.B;
             img = (size_t)b * a.C + c;
-            row = scratch_row(a, qi, yrow);
+            row = scratch_row<PAD>(a, qi, yrow);
         } else {
             img = (size_t)q;                                  // filter row n*C + c
             if (a.zp == 0) {
-                row = a.S + ((size_t)q * 2 * a.H + yrow) * W;
-            } else {                                          // plane z of [2Z][2Hp][W]
+                row = a.S + ((size_t)q * RP * a.H + yrow) * W;
+            } else {                                          // plane z of [RP Z][RP Hp][W]
                 const int z = yrow / a.Hp, y = yrow - z * a.Hp;
-                row = a.S + (((size_t)q * 2 * a.zp + z) * 2 * a.Hp + y) * W;
+                row = a.S + (((size_t)q * RP * a.zp + z) * RP * a.Hp + y) * W;
             }
         }
-        const PT* vp = reinterpret_cast<const PT*>(a.v) + (img * a.H + yrow) * (W / 2);
+        const PT* vp = reinterpret_cast<const PT*>(a.v) + (img * a.H + yrow) * SEQ;
         F::for_each_io(t, [&](int i, int m) { arr[i] = IOP::load(vp + m); });
         R::forward_split(arr, sm, row, t, active);
     } else {
         const int c = q / a.B, b = q % a.B;
         const size_t img = (size_t)b * a.C + c;
-        float2* row = scratch_row(a, qi, yrow);
+        float2* row = scratch_row<PAD>(a, qi, yrow);
         R::unsplit_inverse(arr, sm, row, t);
         const void* xn = a.x[0];
 #pragma unroll
         for (int i = 1; i < kMaxOrder; ++i)
             if (i == a.n) xn = a.x[i];
-        const size_t off = (img * a.H + yrow) * (W / 2);
+        const size_t off = (img * a.H + yrow) * SEQ;
         const PT* xp = reinterpret_cast<const PT*>(xn) + off;
         F::for_each_io(t, [&](int i, int m) {
             const float2 xv = IOP::load(xp + m);
@@ -182,7 +189,7 @@ fft2d_row_kernel(Fft2dArgs a)
     }
 }
 
-template <int LOG2H2>
+template <int LOG2H2, bool PAD = true>
 struct Fft2dCols {
     using FC = SmemFft<LOG2H2>;
     static constexpr int H2 = 1 << LOG2H2;             // 2H
@@ -193,30 +200,35 @@ struct Fft2dCols {
     static constexpr int STRIDE = stride_mod16(H2, 16 / TC);
     static constexpr size_t SMEM = sizeof(float2) * TC * STRIDE;
     // resident CTAs per SM: up to three, as shared memory allows and with at
-    // least 80 registers per thread (120 with 32 values per thread)
-    static constexpr int REGS = FC::V == 32 ? 120 : 80;
+    // least 80 registers per thread (120 with 32 values per thread); more
+    // for circular columns, whose whole column is live in registers
+    static constexpr int REGS = PAD ? (FC::V == 32 ? 120 : 80) : (FC::V == 32 ? 160 : 104);
     static constexpr int BY_SMEM = 3 * SMEM <= 227 * 1024 ? 3 : (2 * SMEM <= 227 * 1024 ? 2 : 1);
     static constexpr int BY_REGS = 65536 / (THREADS * REGS) < 1 ? 1 : 65536 / (THREADS * REGS);
     static constexpr int MIN_BLOCKS = BY_SMEM < BY_REGS ? BY_SMEM : BY_REGS;
     static_assert(THREADS <= 1024 && SMEM <= 227 * 1024, "column kernel geometry");
 };
 
-// Column kernel.  MODE 0: column FFTs of the scratch, spectral multiply
-// with the packed 2-D filter spectrum and the bias, inverse column FFTs,
-// rows y < H back to the scratch.  MODE 1: forward column FFTs of rows
-// y < H of each plane (the packed spectra, or 3-D scratch planes), all 2H
-// rows written back; with zp, plane q of the filter spectra is plane
-// q % zp of filter q / zp at a pitch of 2 zp planes.  MODE 2 (3-D): inverse
-// column FFTs of all 2H rows of each plane, rows y < H written back.
-template <int LOG2H2, int MODE>
-__global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS, Fft2dCols<LOG2H2>::MIN_BLOCKS)
+// Column kernel, columns of H2 = 2H points (PAD: rows y < H, zero-padded)
+// or H2 = H points (circular).  MODE 0: column FFTs of the scratch,
+// spectral multiply with the packed 2-D filter spectrum and the bias,
+// inverse column FFTs, rows y < H back to the scratch.  MODE 1: forward
+// column FFTs of each plane (the packed spectra, or 3-D scratch planes),
+// all H2 rows written back; with zp and PAD, plane q of the filter spectra
+// is plane q % zp of filter q / zp at a pitch of 2 zp planes.  MODE 2
+// (3-D): inverse column FFTs of all H2 rows of each plane, rows y < H
+// written back.
+template <int LOG2H2, int MODE, bool PAD = true>
+__global__ void __launch_bounds__(Fft2dCols<LOG2H2, PAD>::THREADS, Fft2dCols<LOG2H2, PAD>::MIN_BLOCKS)
 fft2d_col_kernel(Fft2dArgs a)
 {
     constexpr bool SPECTRUM = MODE == 1;
     grid_dependency_begin();
-    using CL = Fft2dCols<LOG2H2>;
+    using CL = Fft2dCols<LOG2H2, PAD>;
     using FC = typename CL::FC;
     constexpr int H2 = CL::H2, TC = CL::TC, HH = H2 / 2, V = FC::V;
+    constexpr int ROWS = PAD ? HH : H2;                 // grid rows in a column
+    constexpr int VL = PAD ? V / 2 : V;                 // registers holding grid rows
     const int W = a.W;
     const int CTAS_PER_IMG = W / TC;
     extern __shared__ __align__(16) float2 smem_c2[];
@@ -229,31 +241,31 @@ fft2d_col_kernel(Fft2dArgs a)
     const int kx = kx0 + cc;
     float2* buf = smem_c2 + cc * CL::STRIDE;
     // rows of this image's column kx: scratch [H][W] or planes [2H][W]
-    const size_t pq = (MODE == 1 && a.zp) ? (size_t)(q / a.zp) * 2 * a.zp + q % a.zp : (size_t)q;
-    float2* col = MODE != 0 ? a.S + pq * H2 * W + kx : a.S + (size_t)qi * HH * W + kx;
+    const size_t pq = (MODE == 1 && a.zp && PAD) ? (size_t)(q / a.zp) * 2 * a.zp + q % a.zp : (size_t)q;
+    float2* col = MODE != 0 ? a.S + pq * H2 * W + kx : a.S + (size_t)qi * ROWS * W + kx;
     float2 reg[V];
     const int pt = pad16(t);
 
     if constexpr (MODE == 2) {
-        // inverse column FFT of all 2H rows, rows y < H back
+        // inverse column FFT of all H2 rows, grid rows back
         static_for<V>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             buf[pad16_at<H2 / V>(t, pt, r)] = col[(size_t)(t + r * (H2 / V)) * W];
         });
         __syncthreads();
         FC::template run<+1, true>(buf, reg, t);
-        static_for<V / 2>([&](auto rr) {
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             col[(size_t)(t + r * (H2 / V)) * W] = reg[r];
         });
         return;
     }
-    static_for<V / 2>([&](auto rr) {
+    static_for<VL>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
         buf[pad16_at<H2 / V>(t, pt, r)] = col[(size_t)(t + r * (H2 / V)) * W];
     });
     __syncthreads();
-    FC::template run<-1, true, true>(buf, reg, t);
+    FC::template run<-1, true, PAD>(buf, reg, t);
     if constexpr (SPECTRUM) {
         static_for<V>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
@@ -266,7 +278,7 @@ fft2d_col_kernel(Fft2dArgs a)
             buf[pad16_at<H2 / V>(t, pt, r)] = reg[r];
         });
         __syncthreads();
-        // spectral multiply by (H + b) / (2H)
+        // spectral multiply by (H + b) / H2
         const int c = q / a.B;
         const float bias = __ldg(a.bias + a.n * a.C + c);
         const float2* Hc = a.Hs + (size_t)(q % a.B) * a.Hs_bstride + ((size_t)a.n * a.C + c) * H2 * W + kx;
@@ -305,7 +317,7 @@ fft2d_col_kernel(Fft2dArgs a)
         }
         __syncthreads();
         FC::template run<+1, true>(buf, reg, t);
-        static_for<V / 2>([&](auto rr) {
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             col[(size_t)(t + r * (H2 / V)) * W] = reg[r];
         });

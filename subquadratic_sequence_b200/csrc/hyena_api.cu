@@ -705,3 +705,89 @@ hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void* const* x,
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------- circular 2-D
+
+namespace {
+
+// circular 2-D sizes: W in [32, 1024] (rows of W/2 slots), H in [16, 1024]
+bool dims2d_circ_ok(int H, int W, int& lh, int& lm)
+{
+    lh = exact_log2(H);
+    const int lw = exact_log2(W);
+    lm = lw - 1;
+    return lh >= 4 && lh <= 10 && lw >= 5 && lw <= 10;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hyena_fftconv2d_circular_workspace_size(int B, int C, int H, int W)
+{
+    int lh, lm;
+    if (B < 1 || C < 1 || !dims2d_circ_ok(H, W, lh, lm)) return (size_t)-1;
+    return round_up(sizeof(float2) * (size_t)wave_images((long)B * C, H, W / 2) * H * (W / 2), 256);
+}
+
+hyena_status_t hyena_filter_rfft2d_circular(const float* h, int N, int C, int H, int W, float* Hs, void* stream)
+{
+    if (!h || !Hs || N < 1 || C < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
+    int lh, lm;
+    if (!dims2d_circ_ok(H, W, lh, lm)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)N * C > (1L << 20)) return HYENA_ERR_UNSUPPORTED;
+    if (!aligned(h, 16) || !aligned(Hs, 16)) return HYENA_ERR_INVALID_ARG;
+    if (overlap(h, sizeof(float) * (size_t)N * C * H * W, Hs, sizeof(float2) * (size_t)N * C * H * (W / 2)))
+        return HYENA_ERR_INVALID_ARG;
+    Fft2dArgs a = {};
+    a.v = h;
+    a.S = reinterpret_cast<float2*>(Hs);
+    a.B = 1;
+    a.C = N * C;
+    a.H = H;
+    a.W = W / 2;
+    a.nq = N * C;
+    return dispatch_rfft2d_circ(lm, lh, a, (cudaStream_t)stream);
+}
+
+hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, const void* const* x, const float* Hs,
+                                                     const float* bias, int B, int C, int H, int W, int N,
+                                                     hyena_dtype_t io, void* y, void* workspace,
+                                                     size_t ws_bytes, void* stream)
+{
+    if (!v || !x || !y || !bias || !Hs) return HYENA_ERR_INVALID_ARG;
+    if (B < 1 || C < 1 || N < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
+    if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
+    int lh, lm;
+    if (!dims2d_circ_ok(H, W, lh, lm)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)B * C > (1L << 20) || (long)N * C > (1L << 20)) return HYENA_ERR_UNSUPPORTED;
+    for (int n = 0; n < N; ++n)
+        if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(v, 16) || !aligned(y, 16) || !aligned(bias, 4) || !aligned(Hs, 16)) return HYENA_ERR_INVALID_ARG;
+    const size_t act = (size_t)B * C * H * W * io_bytes(io);
+    const size_t spec = sizeof(float2) * (size_t)N * C * H * (W / 2);
+    const size_t need = hyena_fftconv2d_circular_workspace_size(B, C, H, W);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+    if (overlap(y, act, v, act) || overlap(y, act, bias, sizeof(float) * N * C) || overlap(y, act, Hs, spec) ||
+        overlap(y, act, workspace, need) || overlap(workspace, need, v, act) || overlap(workspace, need, Hs, spec))
+        return HYENA_ERR_INVALID_ARG;
+    for (int n = 0; n < N; ++n)
+        if (overlap(y, act, x[n], act) || overlap(workspace, need, x[n], act)) return HYENA_ERR_INVALID_ARG;
+    Fft2dArgs a = {};
+    a.v = v;
+    for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
+    a.y = y;
+    a.Hs = reinterpret_cast<const float2*>(Hs);
+    a.bias = bias;
+    a.B = B;
+    a.C = C;
+    a.H = H;
+    a.W = W / 2;
+    float2* scratch = static_cast<float2*>(workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    return io == HYENA_BF16 ? dispatch_fft2d_circ_bf16(lm, lh, a, N, scratch, st)
+                            : dispatch_fft2d_circ_f32(lm, lh, a, N, scratch, st);
+}
+
+}  // extern "C"

@@ -18,15 +18,17 @@ inline long wave_images(long nimg, long H, long W)
     return nimg < per ? nimg : per;
 }
 
-// column launches (one 2H-point column FFT per slot column)
+// column launches: one column FFT per slot column, of 2H points (the log2
+// given is log2 H) or, circular, of H points
 hyena_status_t launch_cols2d(int log2h, int mode, const Fft2dArgs& a, cudaStream_t st);
+hyena_status_t launch_cols2d_circ(int log2h, int mode, const Fft2dArgs& a, cudaStream_t st);
 
-template <int LOG2W, typename IO, int MODE>
+template <int LOG2M, typename IO, int MODE, bool PAD = true>
 hyena_status_t launch_rows2d(const Fft2dArgs& a, cudaStream_t st)
 {
-    using F = Fft1d<LOG2W>;
+    using F = Fft1d<LOG2M, PAD>;
     const long rows = (long)a.nq * a.H;
-    return launch(fft2d_row_kernel<LOG2W, IO, MODE>, (unsigned)((rows + F::G - 1) / F::G), F::THREADS,
+    return launch(fft2d_row_kernel<LOG2M, IO, MODE, PAD>, (unsigned)((rows + F::G - 1) / F::G), F::THREADS,
                   F::SMEM_BYTES_FFT, st, a, false);
 }
 
@@ -52,6 +54,44 @@ hyena_status_t run_fft2d(Fft2dArgs a, int N, int log2h, float2* scratch, cudaStr
     return HYENA_OK;
 }
 
+// the order-N circular 2-D forward (rows of W = 2M values, M slots; H-point
+// columns): the same sequence without padding
+template <int LOG2M, typename IO>
+hyena_status_t run_fft2d_circ(Fft2dArgs a, int N, int log2h, float2* scratch, cudaStream_t st)
+{
+    const long nimg = (long)a.B * a.C, per = wave_images(nimg, a.H, a.W);
+    a.S = scratch;
+    for (long q0 = 0; q0 < nimg; q0 += per) {
+        a.q0 = (int)q0;
+        a.nq = (int)(nimg - q0 < per ? nimg - q0 : per);
+        a.n = 0;
+        hyena_status_t s = launch_rows2d<LOG2M, IO, 0, false>(a, st);
+        for (int n = 0; n < N && s == HYENA_OK; ++n) {
+            a.n = n;
+            s = launch_cols2d_circ(log2h, 0, a, st);
+            if (s != HYENA_OK) break;
+            s = n + 1 < N ? launch_rows2d<LOG2M, IO, 1, false>(a, st) : launch_rows2d<LOG2M, IO, 2, false>(a, st);
+        }
+        if (s != HYENA_OK) return s;
+    }
+    return HYENA_OK;
+}
+
+template <typename IO>
+hyena_status_t dispatch_fft2d_circ(int log2m, int log2h, const Fft2dArgs& a, int N, float2* scratch,
+                                   cudaStream_t st)
+{
+    switch (log2m) {
+    case 4: return run_fft2d_circ<4, IO>(a, N, log2h, scratch, st);
+    case 5: return run_fft2d_circ<5, IO>(a, N, log2h, scratch, st);
+    case 6: return run_fft2d_circ<6, IO>(a, N, log2h, scratch, st);
+    case 7: return run_fft2d_circ<7, IO>(a, N, log2h, scratch, st);
+    case 8: return run_fft2d_circ<8, IO>(a, N, log2h, scratch, st);
+    case 9: return run_fft2d_circ<9, IO>(a, N, log2h, scratch, st);
+    default: return HYENA_ERR_UNSUPPORTED;
+    }
+}
+
 template <typename IO>
 hyena_status_t dispatch_fft2d(int log2w, int log2h, const Fft2dArgs& a, int N, float2* scratch,
                               cudaStream_t st)
@@ -73,5 +113,10 @@ hyena_status_t dispatch_fft2d_f32(int log2w, int log2h, const Fft2dArgs& a, int 
 hyena_status_t dispatch_fft2d_bf16(int log2w, int log2h, const Fft2dArgs& a, int N, float2* scratch,
                                    cudaStream_t st);
 hyena_status_t dispatch_rfft2d(int log2w, int log2h, const Fft2dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_fft2d_circ_f32(int log2m, int log2h, const Fft2dArgs& a, int N, float2* scratch,
+                                       cudaStream_t st);
+hyena_status_t dispatch_fft2d_circ_bf16(int log2m, int log2h, const Fft2dArgs& a, int N, float2* scratch,
+                                        cudaStream_t st);
+hyena_status_t dispatch_rfft2d_circ(int log2m, int log2h, const Fft2dArgs& a, cudaStream_t st);
 
 }  // namespace hyena

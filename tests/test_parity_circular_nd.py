@@ -1,0 +1,117 @@
+"""GPU parity of circular mode on 2-D grids (and 3-D volumes) against the
+float64 oracle (run with -m gpu): convolution without padding ("Native
+Multi-Dimensional Subquadratic Operators via Input Dependent Long
+Convolutions", Handling Boundaries: circular convolution for periodic
+systems).  Tolerances as everywhere: 1e-4 (float32 activations), 2e-2
+(bf16) of the oracle's maximum |y|; spectra at 2e-5 of their maximum.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.gpu_helpers import assert_close, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def hy():
+    from subquadratic_sequence_b200 import hyena
+    assert torch.cuda.is_available()
+    return hyena
+
+
+def as_io(a, io):
+    if io == "f32":
+        return a.astype(np.float64)
+    return torch.from_numpy(a).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def decaying(rng, shape):
+    """Seeded random filters with an exponential envelope along every grid axis."""
+    h = rng.standard_normal(shape)
+    for ax, n in enumerate(shape[2:]):
+        env = np.exp(-np.arange(n) / (n / 4)).reshape([-1] + [1] * (len(shape) - 3 - ax))
+        h = h * env
+    return (h / np.sqrt(np.prod(shape[2:])) * 8).astype(np.float32)
+
+
+def problem(B, C, grid, N, seed):
+    rng = np.random.default_rng(seed)
+    shape = (B, C) + tuple(grid)
+    v = rng.standard_normal(shape).astype(np.float32)
+    x = [rng.standard_normal(shape).astype(np.float32) for _ in range(N)]
+    b = rng.standard_normal((N, C)).astype(np.float32)
+    return v, x, b, decaying(rng, (N, C) + tuple(grid))
+
+
+def dft_axis(a, axis):
+    """The oracle's complex DFT (sign -1) along one axis."""
+    return np.apply_along_axis(lambda r: oracle.fft(r, -1), axis, a.astype(np.complex128))
+
+
+def unpack_circ_2d(P):
+    """Packed [..., H, M] -> bins [..., H, M + 1] (M = W/2)."""
+    M = P.shape[-1]
+    out = np.empty(P.shape[:-1] + (M + 1,), np.complex128)
+    out[..., 1:M] = P[..., 1:]
+    A = P[..., 0]
+    Ar = np.conj(np.roll(A[..., ::-1], 1, axis=-1))
+    out[..., 0] = 0.5 * (A + Ar)
+    out[..., M] = (A - Ar) / 2j
+    return out
+
+
+# ------------------------------------------------------------------ 2-D
+
+@pytest.mark.parametrize("H,W", [(16, 32), (32, 64), (64, 16 * 2), (128, 256), (1024, 32), (16, 1024)])
+def test_rfft2d_circular_matches_oracle_dft(hy, H, W):
+    rng = np.random.default_rng(H + 3 * W)
+    h = decaying(rng, (2, 3, H, W))
+    got = unpack_circ_2d(hy.hyena_filter_rfft2d_circular(dev(h)).cpu().numpy().astype(np.complex128))
+    ref = dft_axis(dft_axis(h.astype(np.float64), -1)[..., :W // 2 + 1], -2)
+    assert np.max(np.abs(got - ref)) <= 2e-5 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("B,C,H,W,N,io", [
+    (1, 2, 16, 32, 2, "f32"), (2, 3, 32, 64, 2, "f32"), (1, 2, 64, 32, 3, "f32"), (2, 2, 16, 128, 1, "bf16"),
+    (1, 1, 128, 32, 2, "f32"), (3, 1, 32, 32, 2, "bf16"), (1, 2, 256, 256, 2, "f32"),
+    (1, 1, 1024, 32, 1, "f32"), (1, 1, 16, 1024, 2, "f32"), (1, 1, 512, 512, 1, "bf16"),
+])
+def test_forward_2d_circular_matches_oracle(hy, B, C, H, W, N, io):
+    v, x, b, h = problem(B, C, (H, W), N, seed=H + W + N)
+    Hs = hy.hyena_filter_rfft2d_circular(dev(h))
+    y = host(hy.hyena_fftconv2d_gate_forward_circular(dev(v, io), [dev(xx, io) for xx in x], dev(b), Hs))
+    ref = oracle.hyena_forward_circular_nd(as_io(v, io), np.stack([as_io(xx, io) for xx in x]),
+                                           h.astype(np.float64), b.astype(np.float64))
+    assert_close(y, ref, io, f"circular 2-D B{B} C{C} {H}x{W} N{N} {io}")
+
+
+def test_forward_2d_circular_shift_filters_rotate(hy):
+    # h_1 = delta at (0, 0), h_2 = delta at (5, 30): z_1 = x_1 v (1 + b_1),
+    # y = x_2 (roll(z_1, (5, 30)) + b_2 z_1) -- with wrap-around
+    B, C, H, W, N = 2, 2, 32, 64, 2
+    v, x, b, _ = problem(B, C, (H, W), N, seed=3)
+    h = np.zeros((N, C, H, W), np.float32)
+    h[0, :, 0, 0] = 1.0
+    h[1, :, 5, 30] = 1.0
+    y = host(hy.hyena_fftconv2d_gate_forward_circular(dev(v), [dev(xx) for xx in x], dev(b),
+                                                      hy.hyena_filter_rfft2d_circular(dev(h))))
+    v64, x64, b64 = v.astype(np.float64), [xx.astype(np.float64) for xx in x], b.astype(np.float64)
+    z1 = x64[0] * v64 * (1 + b64[0])[None, :, None, None]
+    ref = x64[1] * (np.roll(z1, (5, 30), axis=(2, 3)) + b64[1][None, :, None, None] * z1)
+    assert_close(y, ref, "f32", "circular 2-D shift filters")
+
+
+def test_forward_2d_circular_on_padded_grids_is_the_linear_forward(hy):
+    # grids zero-padded to 2H x 2W with x zero outside: the circular result
+    # there is the padded (linear) 2-D forward of the GPU's other path
+    B, C, H, W, N = 1, 2, 32, 32, 2
+    v, x, b, h = problem(B, C, (H, W), N, seed=4)
+    pad = lambda a: np.pad(a, [(0, 0)] * (a.ndim - 2) + [(0, H), (0, W)])
+    yc = host(hy.hyena_fftconv2d_gate_forward_circular(dev(pad(v)), [dev(pad(xx)) for xx in x], dev(b),
+                                                       hy.hyena_filter_rfft2d_circular(dev(pad(h)))))
+    yl = host(hy.hyena_fftconv2d_gate_forward(dev(v), [dev(xx) for xx in x], dev(b), h=dev(h)))
+    assert_close(yc[..., :H, :W], yl, "f32", "circular on padded grids")
+    assert np.max(np.abs(yc[..., H:, :])) == 0.0 and np.max(np.abs(yc[..., :, W:])) == 0.0
