@@ -414,6 +414,32 @@ HYENA_API hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, co
                                                                void* y, void* workspace, size_t ws_bytes,
                                                                void* stream);
 
+/* ------------------------------------------------------- circular 3-D */
+
+/* Circular 3-D filter spectra Hs [N][C][Z][H][W/2] complex64 for filters
+ * h [N][C][Z][H][W] (no padding): the circular 2-D packing of every plane
+ * followed by the Z-point DFT over z of every slot; slot [kz][ky][0] holds
+ * A = X0 + i XM (bins 0 and W/2), X0 = (A + conj A') / 2 and
+ * XM = (A - conj A') / (2i), A' the slot at (-kz, -ky).  Z, H powers of two
+ * in [16, 256], W in [32, 256].  Alignment 16 bytes; Hs must not overlap h. */
+HYENA_API hyena_status_t hyena_filter_rfft3d_circular(const float* h, int N, int C, int Z, int H, int W,
+                                                      float* Hs, void* stream);
+
+/* Bytes of workspace hyena_fftconv3d_gate_forward_circular needs (one wave
+ * of volumes, Z x H x W/2 complex slots each); (size_t)-1 for invalid sizes. */
+HYENA_API size_t hyena_fftconv3d_circular_workspace_size(int B, int C, int Z, int H, int W);
+
+/* The order-N recurrence with circular 3-D convolutions, per volume (b, c):
+ *   (h (*) u)[p][q][r] = sum h[i][j][k] u[(p-i) mod Z][(q-j) mod H][(r-k) mod W].
+ * v, x_n, y [B][C][Z][H][W] io; Hs from hyena_filter_rfft3d_circular; bias
+ * [N][C]; x a HOST array of N device pointers.  Sizes as for the spectra;
+ * alignment and aliasing as hyena_fftconv3d_gate_forward. */
+HYENA_API hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, const void* const* x,
+                                                               const float* Hs, const float* bias, int B,
+                                                               int C, int Z, int H, int W, int N,
+                                                               hyena_dtype_t io, void* y, void* workspace,
+                                                               size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,18 +24,21 @@
 
 namespace hyena {
 
-template <int LOG2Z2>
+template <int LOG2Z2, bool PAD = true>
 struct Fft3dZ {
     using FZ = SmemFft<LOG2Z2>;
-    static constexpr int Z2 = 1 << LOG2Z2;              // 2Z
+    static constexpr int Z2 = 1 << LOG2Z2;              // transform length: 2Z (padded) or Z (circular)
     static constexpr int TC = (256 / FZ::T) > 16 ? 16 : ((256 / FZ::T) < 2 ? 2 : 256 / FZ::T);
     static constexpr int THREADS = TC * FZ::T;
     static constexpr int STRIDE = stride_mod16(Z2, 16 / (TC > 16 ? 16 : TC));
     static constexpr size_t SMEM = sizeof(float2) * TC * STRIDE;
     // resident CTAs per SM the register budget aims at: 96 registers a
-    // thread (128 for one-warp CTAs; no cap with 32 values a thread)
-    static constexpr int REGS = THREADS < 64 ? 128 : 96;
-    static constexpr int MIN_BLOCKS = FZ::V == 32 ? 1 : 65536 / (THREADS * REGS);
+    // thread (128 for one-warp CTAs and for circular transforms, whose
+    // whole column is live; no cap with 32 values a thread).  Registers are
+    // allocated per warp.
+    static constexpr int REGS = (THREADS < 64 || !PAD) ? 128 : 96;
+    static constexpr int WARP_THREADS = (THREADS + 31) / 32 * 32;
+    static constexpr int MIN_BLOCKS = FZ::V == 32 ? 1 : 65536 / (WARP_THREADS * REGS);
     static_assert(THREADS <= 1024 && SMEM <= 227 * 1024, "z kernel geometry");
 };
 
@@ -46,16 +49,19 @@ struct Fft3dZ {
 // inverse, planes z < Z kept.  kx = 0 is left to the pair CTAs: each takes
 // TC/2 pairs u in [0, H], slot 0 of rows ky = u (column 2j) and 2H - u
 // (column 2j + 1).  MODE 1 (spectra): forward z transform of every slot of
-// the filters' planes z < Z, all 2Z planes written.
-template <int LOG2Z2, int MODE>
-__global__ void __launch_bounds__(Fft3dZ<LOG2Z2>::THREADS, Fft3dZ<LOG2Z2>::MIN_BLOCKS)
+// the filters' planes z < Z, all 2Z planes written.  Circular (PAD false):
+// Z-point transforms of all Z planes, H rows a plane, nothing cropped.
+template <int LOG2Z2, int MODE, bool PAD = true>
+__global__ void __launch_bounds__(Fft3dZ<LOG2Z2, PAD>::THREADS, Fft3dZ<LOG2Z2, PAD>::MIN_BLOCKS)
 fft3d_z_kernel(Fft2dArgs a)
 {
     grid_dependency_begin();
-    using ZL = Fft3dZ<LOG2Z2>;
+    using ZL = Fft3dZ<LOG2Z2, PAD>;
     using FZ = typename ZL::FZ;
     constexpr int Z2 = ZL::Z2, TC = ZL::TC, ZH = Z2 / 2, V = FZ::V, NP = TC / 2;
-    const int W = a.W, H2 = 2 * a.Hp;
+    constexpr int VL = PAD ? V / 2 : V;                   // registers holding grid planes
+    const int W = a.W, H2 = (PAD ? 2 : 1) * a.Hp;       // slots per row, rows per plane
+    const int UH = H2 / 2;                                // slot-0 pairs u in [0, UH]
     const int kxb = W / TC;                               // slot blocks per row
     const long reg_per = (long)H2 * kxb;                  // regular CTAs per image / channel
     extern __shared__ __align__(16) float2 smem_z[];
@@ -67,10 +73,10 @@ fft3d_z_kernel(Fft2dArgs a)
     const long blk = blockIdx.x;
     float2 reg[V];
 
-    // planes z < Z of a slot column into the buffer (the upper half is
-    // zero padding, which the forward transform does not read)
+    // the grid planes of a slot column into the buffer (padded: the upper
+    // half is zero padding, which the forward transform does not read)
     auto load_col = [&](const float2* colp) {
-        static_for<V / 2>([&](auto rr) {
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             buf[pad16_at<Z2 / V>(t, pt, r)] = colp[(size_t)(t + r * (Z2 / V)) * plane];
         });
@@ -81,9 +87,9 @@ fft3d_z_kernel(Fft2dArgs a)
         const int qi = (int)(blk / reg_per);
         const long rem = blk % reg_per;
         const int ky = (int)(rem / kxb), kx = (int)(rem % kxb) * TC + cc;
-        float2* colp = a.S + (size_t)qi * 2 * a.zp * plane + (size_t)ky * W + kx;
+        float2* colp = a.S + (size_t)qi * Z2 * plane + (size_t)ky * W + kx;
         load_col(colp);
-        FZ::template run<-1, true, true>(buf, reg, t);
+        FZ::template run<-1, true, PAD>(buf, reg, t);
         static_for<V>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             colp[(size_t)(t + r * (Z2 / V)) * plane] = reg[r];
@@ -93,7 +99,7 @@ fft3d_z_kernel(Fft2dArgs a)
         const int cfirst = a.q0 / a.B;
         const int nch = (a.q0 + a.nq - 1) / a.B - cfirst + 1;
         const bool pair_cta = blk >= (long)nch * reg_per;
-        const int npair = (a.Hp + 1 + NP - 1) / NP;       // pair CTAs per channel
+        const int npair = (UH + 1 + NP - 1) / NP;         // pair CTAs per channel
         int ci, ky, kx;
         bool live;
         int u = 0;
@@ -107,9 +113,9 @@ fft3d_z_kernel(Fft2dArgs a)
             const long pb = blk - (long)nch * reg_per;
             ci = (int)(pb / npair);
             u = (int)(pb % npair) * NP + cc / 2;          // this column's pair
-            const bool valid = u <= a.Hp;
-            const int uu = valid ? u : a.Hp;
-            const bool self = uu == 0 || uu == a.Hp;      // rows u and 2H - u coincide
+            const bool valid = u <= UH;
+            const int uu = valid ? u : UH;
+            const bool self = uu == 0 || uu == UH;        // rows u and H2 - u coincide
             ky = (cc % 2 == 0) ? uu : (H2 - uu) % H2;
             kx = 0;
             live = valid && (cc % 2 == 0 || !self);
@@ -130,7 +136,7 @@ fft3d_z_kernel(Fft2dArgs a)
             for (int q = qa; q < qb; ++q) {
                 float2* colp = a.S + (size_t)(q - a.q0) * a.zp * plane + (size_t)ky * W + kx;
                 load_col(colp);
-                FZ::template run<-1, true, true>(buf, reg, t);
+                FZ::template run<-1, true, PAD>(buf, reg, t);
                 static_for<V>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
                     buf[pad16_at<Z2 / V>(t, pt, r)] = cmul(reg[r], hv[r]);
@@ -138,7 +144,7 @@ fft3d_z_kernel(Fft2dArgs a)
                 __syncthreads();
                 FZ::template run<+1, true>(buf, reg, t);
                 if (live)
-                    static_for<V / 2>([&](auto rr) {
+                    static_for<VL>([&](auto rr) {
                         constexpr int r = decltype(rr)::value;
                         colp[(size_t)(t + r * (Z2 / V)) * plane] = reg[r];
                     });
@@ -148,7 +154,7 @@ fft3d_z_kernel(Fft2dArgs a)
             for (int q = qa; q < qb; ++q) {
                 float2* colp = a.S + (size_t)(q - a.q0) * a.zp * plane + (size_t)ky * W;
                 load_col(colp);
-                FZ::template run<-1, true, true>(buf, reg, t);
+                FZ::template run<-1, true, PAD>(buf, reg, t);
                 static_for<V>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
                     buf[pad16_at<Z2 / V>(t, pt, r)] = reg[r];
@@ -159,8 +165,8 @@ fft3d_z_kernel(Fft2dArgs a)
                 for (int e = tid; e < NP * Z2; e += ZL::THREADS) {
                     const int j = e / Z2, kz = e % Z2;
                     const int uj = u0 + j;
-                    const bool self = uj == 0 || uj == a.Hp;
-                    if (uj > a.Hp || (self && kz > ZH)) continue;
+                    const bool self = uj == 0 || uj == UH;
+                    if (uj > UH || (self && kz > ZH)) continue;
                     const int u2 = (H2 - uj) % H2;
                     float2* bA = smem_z + (2 * j) * ZL::STRIDE;
                     float2* bB = self ? bA : smem_z + (2 * j + 1) * ZL::STRIDE;
@@ -181,7 +187,7 @@ fft3d_z_kernel(Fft2dArgs a)
                 __syncthreads();
                 FZ::template run<+1, true>(buf, reg, t);
                 if (live)
-                    static_for<V / 2>([&](auto rr) {
+                    static_for<VL>([&](auto rr) {
                         constexpr int r = decltype(rr)::value;
                         colp[(size_t)(t + r * (Z2 / V)) * plane] = reg[r];
                     });

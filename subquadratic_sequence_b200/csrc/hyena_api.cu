@@ -791,3 +791,96 @@ hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, const void* 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------- circular 3-D
+
+namespace {
+
+// circular 3-D sizes: Z, H in [16, 256], W in [32, 256] (rows of W/2 slots)
+bool dims3d_circ_ok(int Z, int H, int W, int& lz, int& lh, int& lm)
+{
+    lz = exact_log2(Z);
+    lh = exact_log2(H);
+    const int lw = exact_log2(W);
+    lm = lw - 1;
+    return lz >= 4 && lz <= 8 && lh >= 4 && lh <= 8 && lw >= 5 && lw <= 8;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hyena_fftconv3d_circular_workspace_size(int B, int C, int Z, int H, int W)
+{
+    int lz, lh, lm;
+    if (B < 1 || C < 1 || !dims3d_circ_ok(Z, H, W, lz, lh, lm)) return (size_t)-1;
+    const size_t vol = (size_t)Z * H * (W / 2);
+    return round_up(sizeof(float2) * (size_t)wave_images_3d((long)B * C, Z, H, W / 2, false) * vol, 256);
+}
+
+hyena_status_t hyena_filter_rfft3d_circular(const float* h, int N, int C, int Z, int H, int W, float* Hs,
+                                            void* stream)
+{
+    if (!h || !Hs || N < 1 || C < 1 || Z < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
+    int lz, lh, lm;
+    if (!dims3d_circ_ok(Z, H, W, lz, lh, lm)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)N * C * Z * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    if (!aligned(h, 16) || !aligned(Hs, 16)) return HYENA_ERR_INVALID_ARG;
+    const size_t vol = (size_t)Z * H * W;
+    if (overlap(h, sizeof(float) * (size_t)N * C * vol, Hs, sizeof(float2) * (size_t)N * C * (vol / 2)))
+        return HYENA_ERR_INVALID_ARG;
+    Fft2dArgs a = {};
+    a.v = h;
+    a.S = reinterpret_cast<float2*>(Hs);
+    a.B = 1;
+    a.C = N * C;
+    a.W = W / 2;
+    a.nq = N * C;
+    a.zp = Z;
+    a.Hp = H;
+    return dispatch_rfft3d(lm, lh, lz, a, (cudaStream_t)stream, false);
+}
+
+hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, const void* const* x, const float* Hs,
+                                                     const float* bias, int B, int C, int Z, int H, int W,
+                                                     int N, hyena_dtype_t io, void* y, void* workspace,
+                                                     size_t ws_bytes, void* stream)
+{
+    if (!v || !x || !y || !bias || !Hs) return HYENA_ERR_INVALID_ARG;
+    if (B < 1 || C < 1 || N < 1 || Z < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
+    if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
+    int lz, lh, lm;
+    if (!dims3d_circ_ok(Z, H, W, lz, lh, lm)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)B * C > (1L << 20) || (long)N * C * Z * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    for (int n = 0; n < N; ++n)
+        if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(v, 16) || !aligned(y, 16) || !aligned(bias, 4) || !aligned(Hs, 16)) return HYENA_ERR_INVALID_ARG;
+    const size_t vol = (size_t)Z * H * W;
+    const size_t act = (size_t)B * C * vol * io_bytes(io);
+    const size_t spec = sizeof(float2) * (size_t)N * C * (vol / 2);
+    const size_t need = hyena_fftconv3d_circular_workspace_size(B, C, Z, H, W);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+    if (overlap(y, act, v, act) || overlap(y, act, bias, sizeof(float) * N * C) || overlap(y, act, Hs, spec) ||
+        overlap(y, act, workspace, need) || overlap(workspace, need, v, act) || overlap(workspace, need, Hs, spec))
+        return HYENA_ERR_INVALID_ARG;
+    for (int n = 0; n < N; ++n)
+        if (overlap(y, act, x[n], act) || overlap(workspace, need, x[n], act)) return HYENA_ERR_INVALID_ARG;
+    Fft2dArgs a = {};
+    a.v = v;
+    for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
+    a.y = y;
+    a.Hs = reinterpret_cast<const float2*>(Hs);
+    a.bias = bias;
+    a.B = B;
+    a.C = C;
+    a.W = W / 2;
+    a.zp = Z;
+    a.Hp = H;
+    float2* scratch = static_cast<float2*>(workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    return io == HYENA_BF16 ? dispatch_fft3d_bf16(lm, lh, lz, a, N, scratch, st, false)
+                            : dispatch_fft3d_f32(lm, lh, lz, a, N, scratch, st, false);
+}
+
+}  // extern "C"

@@ -78,6 +78,10 @@ def _load() -> ctypes.CDLL:
                                           vp, sz, vp], i),
         "hyena_filter_rfft3d": ([vp, i, i, i, i, i, vp, vp], i),
         "hyena_filter_rfft2d_circular": ([vp, i, i, i, i, vp, vp], i),
+        "hyena_filter_rfft3d_circular": ([vp, i, i, i, i, i, vp, vp], i),
+        "hyena_fftconv3d_circular_workspace_size": ([i, i, i, i, i], sz),
+        "hyena_fftconv3d_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, i, vp, vp,
+                                                   sz, vp], i),
         "hyena_fftconv2d_circular_workspace_size": ([i, i, i, i], sz),
         "hyena_fftconv2d_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, vp, vp,
                                                    sz, vp], i),
@@ -499,6 +503,47 @@ def hyena_fftconv2d_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tenso
     _check("hyena_fftconv2d_gate_forward_circular", LIB.hyena_fftconv2d_gate_forward_circular(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, H, W, N, io,
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def hyena_filter_rfft3d_circular(h: torch.Tensor, *, out=None, stream=None):
+    """Circular 3-D spectra [N][C][Z][H][W/2] complex64 of the filters h
+    [N][C][Z][H][W] (no padding)."""
+    N, C, Z, H, W = h.shape
+    if out is None:
+        out = torch.empty((N, C, Z, H, W // 2), device=h.device, dtype=torch.complex64)
+    _check("hyena_filter_rfft3d_circular", LIB.hyena_filter_rfft3d_circular(
+        ctypes.c_void_p(_dev(h, torch.float32, "h")), N, C, Z, H, W,
+        ctypes.c_void_p(_dev(out, torch.complex64, "Hs")), _stream(stream)))
+    return out
+
+
+def hyena_fftconv3d_circular_workspace_size(B: int, C: int, Z: int, H: int, W: int) -> int:
+    n = LIB.hyena_fftconv3d_circular_workspace_size(B, C, Z, H, W)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv3d_circular_workspace_size", HYENA_ERR_INVALID_ARG, "invalid sizes")
+    return n
+
+
+def hyena_fftconv3d_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor, *,
+                                          out=None, workspace=None, stream=None):
+    """The order-N recurrence with circular 3-D convolutions: v, x_n
+    [B][C][Z][H][W] (float32 or bf16), bias [N][C], Hs from
+    hyena_filter_rfft3d_circular."""
+    B, C, Z, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(hyena_fftconv3d_circular_workspace_size(B, C, Z, H, W), device=v.device,
+                                dtype=torch.uint8)
+    _check("hyena_fftconv3d_gate_forward_circular", LIB.hyena_fftconv3d_gate_forward_circular(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, Z, H, W, N, io,
         ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out

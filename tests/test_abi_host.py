@@ -261,3 +261,36 @@ def test_3d_rejects_bad_arguments(lib):
     assert f(*args(nb=need - 256)) == WORKSPACE
     assert f(*args(wsp=ctypes.c_void_p(A + BIG + 16))) == WORKSPACE              # misaligned
     assert f(*args(xs=(ctypes.c_void_p * 2)(P(1).value, None))) == INVALID
+
+
+def test_circular_nd_rejects_bad_arguments(lib):
+    ws2 = lib.hyena_fftconv2d_circular_workspace_size
+    n = ws2(2, 3, 32, 64)
+    assert n >= 2 * 3 * 32 * 32 * 8 and n % 256 == 0
+    assert ws2(2, 3, 32, 16) == ctypes.c_size_t(-1).value           # W < 32
+    assert ws2(2, 3, 8, 64) == ctypes.c_size_t(-1).value            # H < 16
+    assert ws2(2, 3, 2048, 64) == ctypes.c_size_t(-1).value         # H > 1024
+    r2 = lib.hyena_filter_rfft2d_circular
+    assert r2(None, 2, 3, 32, 64, P(1), None) == INVALID
+    assert r2(P(0), 2, 3, 32, 48, P(1), None) == UNSUPPORTED
+    assert r2(P(0), 2, 3, 32, 64, P(0), None) == INVALID              # Hs overlaps h
+    f2 = lib.hyena_fftconv2d_gate_forward_circular
+    xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
+    need = ws2(2, 3, 32, 64)
+    assert f2(P(0), xs, None, P(4), 2, 3, 32, 64, 2, F32, P(5), P(6), need, None) == INVALID   # no spectra
+    assert f2(P(0), xs, P(3), P(4), 2, 3, 32, 64, 2, F32, P(0), P(6), need, None) == INVALID   # y aliases v
+    assert f2(P(0), xs, P(3), P(4), 2, 3, 32, 64, 2, F32, P(5), P(6), need - 256, None) == WORKSPACE
+    assert f2(P(0), xs, P(3), P(4), 2, 3, 32, 2048, 2, F32, P(5), P(6), need, None) == UNSUPPORTED
+
+    ws3 = lib.hyena_fftconv3d_circular_workspace_size
+    n = ws3(2, 3, 16, 32, 64)
+    assert n >= 2 * 3 * 16 * 32 * 32 * 8 and n % 256 == 0
+    assert ws3(2, 3, 16, 32, 512) == ctypes.c_size_t(-1).value      # W > 256
+    r3 = lib.hyena_filter_rfft3d_circular
+    assert r3(P(0), 2, 3, 16, 16, 16, P(1), None) == UNSUPPORTED       # W < 32
+    assert r3(P(0), 2, 3, 16, 16, 32, P(0), None) == INVALID
+    f3 = lib.hyena_fftconv3d_gate_forward_circular
+    need = ws3(2, 3, 16, 16, 32)
+    assert f3(P(0), xs, P(3), P(4), 2, 3, 16, 16, 32, 2, 7, P(5), P(6), need, None) == INVALID  # io
+    assert f3(P(0), xs, P(3), P(4), 2, 3, 16, 16, 32, 2, F32, P(5), None, need, None) == WORKSPACE
+    assert f3(P(0), xs, P(3), P(4), 2, 3, 16, 16, 32, 17, F32, P(5), P(6), need, None) == UNSUPPORTED

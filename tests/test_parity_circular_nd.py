@@ -115,3 +115,72 @@ def test_forward_2d_circular_on_padded_grids_is_the_linear_forward(hy):
     yl = host(hy.hyena_fftconv2d_gate_forward(dev(v), [dev(xx) for xx in x], dev(b), h=dev(h)))
     assert_close(yc[..., :H, :W], yl, "f32", "circular on padded grids")
     assert np.max(np.abs(yc[..., H:, :])) == 0.0 and np.max(np.abs(yc[..., :, W:])) == 0.0
+
+
+# ------------------------------------------------------------------ 3-D
+
+def unpack_circ_3d(P):
+    """Packed [..., Z, H, M] -> bins [..., Z, H, M + 1] (M = W/2)."""
+    M = P.shape[-1]
+    out = np.empty(P.shape[:-1] + (M + 1,), np.complex128)
+    out[..., 1:M] = P[..., 1:]
+    A = P[..., 0]
+    Ar = np.conj(np.roll(A[..., ::-1, ::-1], (1, 1), axis=(-2, -1)))     # conj A[-kz][-ky]
+    out[..., 0] = 0.5 * (A + Ar)
+    out[..., M] = (A - Ar) / 2j
+    return out
+
+
+@pytest.mark.parametrize("Z,H,W", [(16, 16, 32), (32, 16, 64), (16, 64, 32), (64, 32, 32)])
+def test_rfft3d_circular_matches_oracle_dft(hy, Z, H, W):
+    rng = np.random.default_rng(Z + 5 * H + 7 * W)
+    h = decaying(rng, (2, 2, Z, H, W))
+    got = unpack_circ_3d(hy.hyena_filter_rfft3d_circular(dev(h)).cpu().numpy().astype(np.complex128))
+    ref = dft_axis(dft_axis(dft_axis(h.astype(np.float64), -1)[..., :W // 2 + 1], -2), -3)
+    assert np.max(np.abs(got - ref)) <= 2e-5 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("B,C,Z,H,W,N,io", [
+    (1, 2, 16, 16, 32, 2, "f32"), (2, 1, 16, 32, 64, 2, "f32"), (1, 2, 32, 16, 32, 3, "f32"),
+    (2, 2, 16, 16, 32, 1, "bf16"), (1, 1, 64, 16, 32, 2, "f32"), (1, 1, 16, 64, 32, 2, "bf16"),
+    (1, 1, 256, 16, 32, 1, "f32"), (1, 1, 16, 256, 32, 1, "f32"), (1, 1, 16, 16, 256, 2, "f32"),
+])
+def test_forward_3d_circular_matches_oracle(hy, B, C, Z, H, W, N, io):
+    v, x, b, h = problem(B, C, (Z, H, W), N, seed=Z + H + W + N)
+    Hs = hy.hyena_filter_rfft3d_circular(dev(h))
+    y = host(hy.hyena_fftconv3d_gate_forward_circular(dev(v, io), [dev(xx, io) for xx in x], dev(b), Hs))
+    ref = oracle.hyena_forward_circular_nd(as_io(v, io), np.stack([as_io(xx, io) for xx in x]),
+                                           h.astype(np.float64), b.astype(np.float64))
+    assert_close(y, ref, io, f"circular 3-D B{B} C{C} {Z}x{H}x{W} N{N} {io}")
+
+
+def test_forward_3d_circular_largest_volume_shift_filters(hy):
+    """256^3 volumes, bf16, shift filters with wrap-around: the closed form
+    (np.roll) holds at any size."""
+    B, C, Z, H, W, N = 1, 2, 256, 256, 256, 2
+    rng = np.random.default_rng(8)
+    v = rng.standard_normal((B, C, Z, H, W), dtype=np.float32)
+    x = [rng.standard_normal((B, C, Z, H, W), dtype=np.float32) for _ in range(N)]
+    b = rng.standard_normal((N, C)).astype(np.float32)
+    h = np.zeros((N, C, Z, H, W), np.float32)
+    h[0, :, 0, 0, 0] = 1.0
+    h[1, :, 200, 5, 251] = 1.0
+    y = host(hy.hyena_fftconv3d_gate_forward_circular(dev(v, "bf16"), [dev(xx, "bf16") for xx in x], dev(b),
+                                                      hy.hyena_filter_rfft3d_circular(dev(h))))
+    v64, x64, b64 = as_io(v, "bf16"), [as_io(xx, "bf16") for xx in x], b.astype(np.float64)
+    z1 = x64[0] * v64 * (1 + b64[0])[None, :, None, None, None]
+    ref = x64[1] * (np.roll(z1, (200, 5, 251), axis=(2, 3, 4)) + b64[1][None, :, None, None, None] * z1)
+    assert_close(y, ref, "bf16", "circular 3-D 256^3 shift filters")
+
+
+def test_forward_3d_circular_on_padded_volumes_is_the_linear_forward(hy):
+    B, C, Z, H, W, N = 1, 2, 16, 16, 16, 2
+    v, x, b, h = problem(B, C, (Z, H, W), N, seed=9)
+    pad = lambda a: np.pad(a, [(0, 0)] * (a.ndim - 3) + [(0, Z), (0, H), (0, W)])
+    yc = host(hy.hyena_fftconv3d_gate_forward_circular(dev(pad(v)), [dev(pad(xx)) for xx in x], dev(b),
+                                                       hy.hyena_filter_rfft3d_circular(dev(pad(h)))))
+    yl = host(hy.hyena_fftconv3d_gate_forward(dev(v), [dev(xx) for xx in x], dev(b), h=dev(h)))
+    assert_close(yc[..., :Z, :H, :W], yl, "f32", "circular on padded volumes")
+    outside = yc.copy()
+    outside[..., :Z, :H, :W] = 0.0
+    assert np.max(np.abs(outside)) == 0.0
