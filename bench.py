@@ -22,6 +22,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -41,6 +42,15 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 def describe(wl: synth.Workload) -> dict:
+    d = _describe(wl)
+    if wl.circular:
+        d["workload"] = re.sub(r" \(padded to [^)]*\)", "", d["workload"])
+        d["workload"] += "; circular convolution on the grid itself (periodic boundaries, no padding)"
+        d["circular"] = True
+    return d
+
+
+def _describe(wl: synth.Workload) -> dict:
     if wl.kind == "3d":
         return {"workload": f"{wl.name}: order-{wl.N} Hyena 3-D operator, B={wl.B}, C={wl.D}, "
                             f"{wl.Z}x{wl.H}x{wl.W} volumes (padded to {2 * wl.Z}x{2 * wl.H}x{2 * wl.W}), "
@@ -71,12 +81,15 @@ def alg_bytes_forward(wl: synth.Workload) -> int:
     """Algorithmic HBM bytes of one forward call: v, x_1..x_N, y plus the
     N*D packed spectra (L complex64 slots each; 2H x W for the 2-D grid,
     2Z x 2H x W for the 3-D volume)."""
+    act = (wl.N + 2) * wl.positions * wl.io_bytes
+    if wl.circular:                        # spectra of the grid itself: half a slot per position
+        return act + wl.N * wl.D * wl.per_channel // 2 * 8
     if wl.kind == "3d":
-        return (wl.N + 2) * wl.positions * wl.io_bytes + wl.N * wl.D * 4 * wl.Z * wl.H * wl.W * 8
+        return act + wl.N * wl.D * 4 * wl.Z * wl.H * wl.W * 8
     if wl.kind == "2d":
-        return (wl.N + 2) * wl.positions * wl.io_bytes + wl.N * wl.D * 2 * wl.H * wl.W * 8
+        return act + wl.N * wl.D * 2 * wl.H * wl.W * 8
     sets = wl.B if wl.film else 1          # filter spectra per sample, or shared by the batch
-    return (wl.N + 2) * wl.B * wl.D * wl.L * wl.io_bytes + sets * wl.N * wl.D * wl.L * 8
+    return act + sets * wl.N * wl.D * wl.L * 8
 
 
 def alg_bytes_backward(wl: synth.Workload) -> int:
@@ -99,6 +112,12 @@ def waves(nseq: int, L: int) -> int:
 
 def launches_forward(wl: synth.Workload) -> int:
     """Kernel launches of one forward call."""
+    if wl.circular:
+        if wl.kind == "3d":
+            return waves(wl.B * wl.D, wl.per_channel) * (4 * wl.N + 1)
+        if wl.kind == "2d":
+            return waves(wl.B * wl.D, wl.per_channel // 2) * (1 + 2 * wl.N)
+        return 1
     if wl.kind == "3d":
         # per wave: rows, columns, then per order z, inverse columns, rows
         # (and forward columns before every order but the first)
@@ -109,6 +128,8 @@ def launches_forward(wl: synth.Workload) -> int:
 
 
 def launches_rfft(wl: synth.Workload) -> int:
+    if wl.circular:
+        return {"1d": 1, "2d": 2, "3d": 3}[wl.kind]
     if wl.kind == "3d":
         return 3
     if wl.kind == "2d":
@@ -126,6 +147,12 @@ def launches_filter_gen(wl: synth.Workload) -> int:
 def forward_kernel(wl: synth.Workload) -> str:
     """The timed unit of the roofline: the forward call (one fused kernel,
     or the 2N+1 four-step kernels of each wave)."""
+    if wl.circular:
+        return {"1d": "fused1d_kernel<PAD=false> (hyena_fftconv_gate_forward_circular)",
+                "2d": "fft2d_row_kernel+fft2d_col_kernel<PAD=false> (hyena_fftconv2d_gate_forward_circular, "
+                      "all launches)",
+                "3d": "fft2d_row_kernel+fft2d_col_kernel+fft3d_z_kernel<PAD=false> "
+                      "(hyena_fftconv3d_gate_forward_circular, all launches)"}[wl.kind]
     if wl.kind == "3d":
         return "fft2d_row_kernel+fft2d_col_kernel+fft3d_z_kernel (hyena_fftconv3d_gate_forward, all launches)"
     if wl.kind == "2d":
@@ -302,7 +329,45 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     y = torch.empty_like(v)
     flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
     stream = torch.cuda.current_stream()
-    if wl.kind == "3d":
+    if wl.circular and wl.kind == "3d":
+        h = W[0]
+        H = torch.empty((wl.N, wl.D, wl.Z, wl.H, wl.W // 2), device="cuda", dtype=torch.complex64)
+        ws_fwd = torch.empty(hyena.hyena_fftconv3d_circular_workspace_size(wl.B, wl.D, wl.Z, wl.H, wl.W),
+                             device="cuda", dtype=torch.uint8)
+
+        def forward():
+            hyena.hyena_fftconv3d_gate_forward_circular(v, xs, b, H, out=y, workspace=ws_fwd)
+
+        def step():
+            hyena.hyena_filter_rfft3d_circular(h, out=H)
+            forward()
+    elif wl.circular and wl.kind == "2d":
+        h = torch.empty((wl.N, wl.D, wl.H, wl.W), device="cuda", dtype=torch.float32)
+        H = torch.empty((wl.N, wl.D, wl.H, wl.W // 2), device="cuda", dtype=torch.complex64)
+        ws_fwd = torch.empty(hyena.hyena_fftconv2d_circular_workspace_size(wl.B, wl.D, wl.H, wl.W),
+                             device="cuda", dtype=torch.uint8)
+
+        def forward():
+            hyena.hyena_fftconv2d_gate_forward_circular(v, xs, b, H, out=y, workspace=ws_fwd)
+
+        def step():
+            hyena.hyena_filter_gen_2d(*W, wl.N, wl.D, wl.H, wl.W, n_bands=synth.N_BANDS,
+                                      width=synth.WIDTH, decay_div=synth.DECAY_DIV, out=h)
+            hyena.hyena_filter_rfft2d_circular(h, out=H)
+            forward()
+    elif wl.circular:
+        h = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.float32)
+        H = torch.empty((wl.N, wl.D, wl.L // 2), device="cuda", dtype=torch.complex64)
+
+        def forward():
+            hyena.hyena_fftconv_gate_forward_circular(v, xs, b, H, out=y)
+
+        def step():
+            hyena.hyena_filter_gen(*W, wl.N, wl.D, wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                   decay_div=synth.DECAY_DIV, out=h)
+            hyena.hyena_filter_rfft_circular(h, out=H)
+            forward()
+    elif wl.kind == "3d":
         h = W[0]
         H = torch.empty((wl.N, wl.D, 2 * wl.Z, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
         ws_n = hyena.hyena_fftconv3d_workspace_size(wl.B, wl.D, wl.Z, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
@@ -445,7 +510,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
 
     # ---- the backward pass (1-D, L <= 16384): one call per timed repetition
     bwd = None
-    if wl.kind == "1d" and not long_path(wl) and not wl.film:
+    if wl.kind == "1d" and not long_path(wl) and not wl.film and not wl.circular:
         dy = to_dev(synth.make_output_grad(wl), io)
         ws_b = torch.empty(hyena.hyena_fftconv_backward_workspace_size(wl.D, wl.L, wl.N),
                            device="cuda", dtype=torch.uint8)
@@ -513,6 +578,21 @@ def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: 
     v = inp["v"][:, channels].astype(np.float64)
     x = np.stack([xx[:, channels] for xx in inp["x"]]).astype(np.float64)
     bias = inp["b"][:, channels].astype(np.float64)
+    if wl.circular and wl.kind == "3d":
+        oracle.hyena_forward_circular_nd(v, x, inp["h"][:, channels].astype(np.float64), bias, route="fft")
+        return time.perf_counter() - t0
+    if wl.circular and wl.kind == "2d":
+        h = oracle.filter_gen_2d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
+                                 wl.N, len(channels), wl.H, wl.W, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                 decay_div=synth.DECAY_DIV, threads=threads)
+        oracle.hyena_forward_circular_nd(v, x, h, bias, route="fft")
+        return time.perf_counter() - t0
+    if wl.circular:
+        h = oracle.filter_gen(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
+                              wl.N, len(channels), wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                              decay_div=synth.DECAY_DIV, threads=threads)
+        oracle.hyena_forward_circular(v, x, h, bias, route="fft", threads=threads)
+        return time.perf_counter() - t0
     if wl.kind == "3d":
         oracle.hyena_forward_3d(v, x, inp["h"][:, channels].astype(np.float64), bias, route="fft")
         return time.perf_counter() - t0
@@ -546,9 +626,19 @@ def extent(wl: synth.Workload) -> str:
     return f"L={wl.L}"
 
 
+def one_thread(wl: synth.Workload) -> bool:
+    """The 3-D oracle and the circular 2-D/3-D oracle are single-threaded."""
+    return wl.kind == "3d" or (wl.circular and wl.kind == "2d")
+
+
 def stages(wl: synth.Workload) -> str:
+    circ = "circular " if wl.circular else ""
     if wl.kind == "3d":
-        return f"3-D spectra + order-{wl.N} forward, one thread"
+        return f"3-D spectra + order-{wl.N} {circ}forward, one thread"
+    if one_thread(wl):
+        return f"filter generation (all cores) + order-{wl.N} {circ}forward (one thread)"
+    if wl.circular:
+        return f"filter generation + order-{wl.N} circular forward"
     return f"filter generation + order-{wl.N} forward"
 
 
@@ -557,7 +647,7 @@ def cpu_baseline(wl: synth.Workload, budget_s: float = 15.0, inp: dict | None = 
     inp = inp or synth.make_inputs(wl)
     threads = oracle.default_threads()
     rng = np.random.default_rng(0)
-    n = 1 if wl.kind == "3d" else max(1, min(wl.D, threads))   # the 3-D oracle runs on one thread
+    n = 1 if one_thread(wl) else max(1, min(wl.D, threads))   # the N-D oracles below run on one thread
     t = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
     # grow the sample to about budget_s of CPU work
     n2 = int(min(wl.D, max(n, n * budget_s / max(t, 1e-3))))
@@ -580,7 +670,7 @@ def run_reference(args, wl: synth.Workload) -> dict | None:
     inp = synth.make_inputs(wl)
     threads = oracle.default_threads()
     rng = np.random.default_rng(0)
-    n = 1 if wl.kind == "3d" else max(1, min(wl.D, threads))   # the 3-D oracle runs on one thread
+    n = 1 if one_thread(wl) else max(1, min(wl.D, threads))   # the N-D oracles below run on one thread
     probe = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
     # size each step so that warm-up + timed steps end within ~2 minutes
     per_step_budget = 120.0 / max(1, args.steps + args.warmup)

@@ -43,6 +43,7 @@ class Workload:
     io: str = "f32"  # storage type of v, x_n, y: "f32" or "bf16"
     seed: int = 0
     film: bool = False  # input-dependent (per-sample, FiLM-modulated) filters
+    circular: bool = False  # circular convolution on the grid itself (no padding)
 
     @property
     def per_channel(self) -> int:
@@ -97,6 +98,11 @@ WORKLOADS = {
     # order-2 3-D operator on 64^3 volumes, B=2, C=32, bf16 storage (the
     # filters are inputs: seeded decaying random volumes)
     "c5_3d": Workload("c5_3d", "3d", N=2, B=2, D=32, Z=64, H=64, W=64, io="bf16", seed=_seed(5)),
+    # circular mode (periodic boundaries) at the shapes of c1, c4 and c5_3d
+    "c1_circ": Workload("c1_circ", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), circular=True),
+    "c4_circ": Workload("c4_circ", "2d", N=2, B=2, D=128, H=256, W=256, io="f32", seed=_seed(4), circular=True),
+    "c5_3d_circ": Workload("c5_3d_circ", "3d", N=2, B=2, D=32, Z=64, H=64, W=64, io="bf16", seed=_seed(5),
+                           circular=True),
 }
 
 
