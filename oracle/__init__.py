@@ -68,6 +68,7 @@ def _load():
         "oracle_rfft_circ": [dp, l, l, dp, dp],
         "oracle_hyena_forward_circular": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
         "oracle_cconv3": [dp, dp, l, l, l, i, dp],
+        "oracle_hyena_backward_2d": [dp, dp, dp, dp, dp, l, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_hyena_forward_circular_nd": [dp, dp, dp, dp, l, l, l, l, l, l, i, dp],
     }
     for name, args in sigs.items():
@@ -361,4 +362,21 @@ def hyena_forward_circular_nd(v, x, h, bias, route="fft") -> np.ndarray:
     _check(_load().oracle_hyena_forward_circular_nd(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), B, C, Z, H, W, N,
                                                     _route(route), _ptr(y)), "oracle_hyena_forward_circular_nd")
     return y
+
+
+def hyena_backward_2d(v, x, h, bias, dy, route="fft", threads=None):
+    """Gradients of a scalar loss with dL/dy = dy through the 2-D
+    recurrence: returns (dv [B][C][H][W], dx [N][B][C][H][W], dh
+    [N][C][H][W], dbias [N][C]); dh and dbias are summed over the batch."""
+    v, x, h, bias, dy = map(_f64, (v, x, h, bias, dy))
+    B, C, H, W = v.shape
+    N = h.shape[0]
+    assert x.shape == (N, B, C, H, W) and h.shape == (N, C, H, W) and bias.shape == (N, C)
+    assert dy.shape == v.shape
+    dv, dx, dh, db = np.empty_like(v), np.empty_like(x), np.empty_like(h), np.empty_like(bias)
+    rc = _load().oracle_hyena_backward_2d(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), _ptr(dy), B, C, H, W, N,
+                                          _route(route), threads or default_threads(),
+                                          _ptr(dv), _ptr(dx), _ptr(dh), _ptr(db))
+    _check(rc, "oracle_hyena_backward_2d")
+    return dv, dx, dh, db
 

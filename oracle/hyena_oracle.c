@@ -1330,3 +1330,166 @@ int oracle_hyena_forward_circular_nd(const double *v, const double *x, const dou
     free(z); free(c);
     return st;
 }
+
+/* ------------------------------------------------------------------ */
+/* Backward of the 2-D recurrence (the chain rule, as in 1-D, with the  */
+/* 2-D linear convolution of Native ND Convolution / Handling           */
+/* Boundaries):                                                         */
+/*     dx_n = g c_n,  e = g x_n,                                        */
+/*     dh_n[a][b] += sum_{t,s} e[t][s] z_{n-1}[t-a][s-b],               */
+/*     db_n += sum e z_{n-1} = dh_n[0][0],                              */
+/*     g <- sum_{t>=u, s>=w} h_n[t-u][s-w] e[t][s] + b_n e,  dv = g.    */
+/* ------------------------------------------------------------------ */
+
+/* Adjoint of the 2-D convolution with respect to its signal:
+ * out[u][w] = sum_{t>=u, s>=w} h[t-u][s-w] e[t][s]. */
+static void corr2_direct(const double *h, const double *e, long H, long W, double *out)
+{
+    for (long u = 0; u < H; ++u)
+        for (long w = 0; w < W; ++w) {
+            double acc = 0.0;
+            for (long t = u; t < H; ++t)
+                for (long s = w; s < W; ++s) acc += h[(t - u) * W + (s - w)] * e[t * W + s];
+            out[u * W + w] = acc;
+        }
+}
+
+/* Lagged products: out[a][b] = sum_{t>=a, s>=b} e[t][s] z[t-a][s-b]. */
+static void lagged2_direct(const double *e, const double *z, long H, long W, double *out)
+{
+    for (long a = 0; a < H; ++a)
+        for (long b = 0; b < W; ++b) {
+            double acc = 0.0;
+            for (long t = a; t < H; ++t)
+                for (long s = b; s < W; ++s) acc += e[t * W + s] * z[(t - a) * W + (s - b)];
+            out[a * W + b] = acc;
+        }
+}
+
+/* out[a][b] = sum_{t,s} p[t+a][s+b] q[t][s] for a < H, b < W: the 2-D DFT
+ * of both zero-padded to PH x PW >= 2H x 2W, IDFT(P conj(Q)) / (PH PW).
+ * corr2_direct (p = e, q = h) and lagged2_direct (p = e, q = z) both have
+ * this form. */
+static void corr2_fft(const double *p, const double *q, long H, long W, double *out, fft2_scratch *s)
+{
+    const long PH = s->PH, PW = s->PW;
+    for (long r = 0; r < PH; ++r)
+        for (long c = 0; c < PW; ++c) {
+            const int in = r < H && c < W;
+            s->ur[r * PW + c] = in ? p[r * W + c] : 0.0; s->ui[r * PW + c] = 0.0;
+            s->hr[r * PW + c] = in ? q[r * W + c] : 0.0; s->hi[r * PW + c] = 0.0;
+        }
+    fft2(s->ur, s->ui, s, -1);
+    fft2(s->hr, s->hi, s, -1);
+    for (long k = 0; k < PH * PW; ++k) {
+        const double re = s->ur[k] * s->hr[k] + s->ui[k] * s->hi[k];
+        const double im = s->ui[k] * s->hr[k] - s->ur[k] * s->hi[k];
+        s->ur[k] = re;
+        s->ui[k] = im;
+    }
+    fft2(s->ur, s->ui, s, +1);
+    for (long r = 0; r < H; ++r)
+        for (long c = 0; c < W; ++c) out[r * W + c] = s->ur[r * PW + c] / (double)(PH * PW);
+}
+
+typedef struct {
+    const double *v, *x, *h, *bias, *dy;
+    long B, C, H, W, N;
+    int route;
+    double *dv, *dx, *dh, *dbias;
+    long c0, step; /* channels c0, c0 + step, ... (dh, db summed over b here) */
+    int status;
+} bwd2_job;
+
+static void *backward_2d_worker(void *arg)
+{
+    bwd2_job *j = (bwd2_job *)arg;
+    const long HW = j->H * j->W, N = j->N, C = j->C, BCHW = j->B * C * HW;
+    double *z = malloc(sizeof(double) * N * HW), *c = malloc(sizeof(double) * N * HW);
+    double *g = malloc(sizeof(double) * HW), *e = malloc(sizeof(double) * HW);
+    double *tmp = malloc(sizeof(double) * HW);
+    fft2_scratch s = {0};
+    if (!z || !c || !g || !e || !tmp ||
+        (j->route == ROUTE_FFT &&
+         scratch2_alloc(&s, next_pow2(2 * j->H), next_pow2(2 * j->W)) != ORACLE_OK)) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (long ch = j->c0; ch < C; ch += j->step) {
+        for (long n = 0; n < N; ++n) {
+            memset(j->dh + (n * C + ch) * HW, 0, sizeof(double) * HW);
+            j->dbias[n * C + ch] = 0.0;
+        }
+        for (long b = 0; b < j->B; ++b) {
+            const long img = b * C + ch;
+            /* forward, keeping z_{n-1} and c_n */
+            memcpy(z, j->v + img * HW, sizeof(double) * HW);
+            for (long n = 0; n < N; ++n) {
+                const double *hn = j->h + (n * C + ch) * HW, *xn = j->x + n * BCHW + img * HW;
+                const double bn = j->bias[n * C + ch];
+                double *zn = z + n * HW, *cn = c + n * HW;
+                if (j->route == ROUTE_DIRECT) conv2_direct(hn, zn, j->H, j->W, cn);
+                else conv2_fft(hn, zn, j->H, j->W, cn, &s);
+                for (long t = 0; t < HW; ++t) cn[t] += bn * zn[t];
+                if (n + 1 < N)
+                    for (long t = 0; t < HW; ++t) z[(n + 1) * HW + t] = xn[t] * cn[t];
+            }
+            /* backward */
+            memcpy(g, j->dy + img * HW, sizeof(double) * HW);
+            for (long n = N - 1; n >= 0; --n) {
+                const double *hn = j->h + (n * C + ch) * HW, *xn = j->x + n * BCHW + img * HW;
+                const double bn = j->bias[n * C + ch];
+                const double *zn = z + n * HW, *cn = c + n * HW;
+                double *dxn = j->dx + n * BCHW + img * HW, *dhn = j->dh + (n * C + ch) * HW;
+                for (long t = 0; t < HW; ++t) {
+                    dxn[t] = g[t] * cn[t];
+                    e[t] = g[t] * xn[t];
+                }
+                if (j->route == ROUTE_DIRECT) lagged2_direct(e, zn, j->H, j->W, tmp);
+                else corr2_fft(e, zn, j->H, j->W, tmp, &s);
+                for (long t = 0; t < HW; ++t) dhn[t] += tmp[t];
+                double db = 0.0;
+                for (long t = 0; t < HW; ++t) db += e[t] * zn[t];
+                j->dbias[n * C + ch] += db;
+                if (j->route == ROUTE_DIRECT) corr2_direct(hn, e, j->H, j->W, tmp);
+                else corr2_fft(e, hn, j->H, j->W, tmp, &s);
+                for (long t = 0; t < HW; ++t) g[t] = tmp[t] + bn * e[t];
+            }
+            memcpy(j->dv + img * HW, g, sizeof(double) * HW);
+        }
+    }
+    j->status = ORACLE_OK;
+done:
+    free(z); free(c); free(g); free(e); free(tmp);
+    if (j->route == ROUTE_FFT) scratch2_free(&s);
+    return NULL;
+}
+
+/* Gradients of a scalar loss with dL/dy = dy [B][C][H][W] through the 2-D
+ * recurrence: dv [B][C][H][W], dx [N][B][C][H][W], dh [N][C][H][W] and
+ * dbias [N][C] (both summed over the batch). */
+int oracle_hyena_backward_2d(const double *v, const double *x, const double *h, const double *bias,
+                             const double *dy, long B, long C, long H, long W, long N, int route,
+                             int nthreads, double *dv, double *dx, double *dh, double *dbias)
+{
+    if (!v || !x || !h || !bias || !dy || !dv || !dx || !dh || !dbias || B < 1 || C < 1 || H < 1 ||
+        W < 1 || N < 1 || (route != ROUTE_DIRECT && route != ROUTE_FFT))
+        return ORACLE_EBADARG;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > C) nthreads = (int)C;
+    bwd2_job *jobs = calloc(nthreads, sizeof(bwd2_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        bwd2_job jb = {v, x, h, bias, dy, B, C, H, W, N, route, dv, dx, dh, dbias, k, nthreads, 0};
+        jobs[k] = jb;
+        pthread_create(&tid[k], NULL, backward_2d_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}

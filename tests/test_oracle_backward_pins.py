@@ -93,3 +93,70 @@ def test_backward_linear_in_dy_and_threads_agree():
     g2 = oracle.hyena_backward(v, x, h, b, 2.5 * dy, threads=3)
     for a, c in zip(g1, g2):
         assert rel_err(c, 2.5 * a) < 1e-13
+
+
+# ------------------------------------------------------------------ 2-D
+
+def problem_2d(B, C, H, W, N, seed):
+    r = np.random.default_rng(seed)
+    v = r.standard_normal((B, C, H, W))
+    x = r.standard_normal((N, B, C, H, W))
+    h = r.standard_normal((N, C, H, W)) * np.exp(-np.arange(H) / 3.0)[:, None] * np.exp(-np.arange(W) / 3.0)
+    b = r.standard_normal((N, C))
+    dy = r.standard_normal((B, C, H, W))
+    return v, x, h, b, dy
+
+
+@pytest.mark.parametrize("N", [1, 2])
+def test_backward_2d_matches_finite_differences(N):
+    # loss = sum(dy * y) through the separately pinned 2-D oracle forward
+    v, x, h, b, dy = problem_2d(2, 2, 3, 4, N, seed=20 + N)
+    dv, dx, dh, db = oracle.hyena_backward_2d(v, x, h, b, dy, route="direct")
+
+    def loss(v_, x_, h_, b_):
+        return float(np.sum(dy * oracle.hyena_forward_2d(v_, x_, h_, b_, route="direct")))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name
+
+
+def test_backward_2d_of_one_row_is_the_1d_backward():
+    # a 1 x W grid is a sequence: every gradient equals the pinned 1-D adjoint
+    B, C, W, N = 2, 3, 16, 3
+    v, x, h, b, dy = problem(B, C, W, N, seed=30)
+    got = oracle.hyena_backward_2d(v[:, :, None], x[:, :, :, None], h[:, :, None], b, dy[:, :, None], route="fft")
+    want = oracle.hyena_backward(v, x, h, b, dy, route="direct")
+    for g_, w_, name in zip(got, want, ("dv", "dx", "dh", "db")):
+        assert rel_err(np.squeeze(g_, axis=-2) if g_.ndim > 2 else g_, w_) < 1e-12, name
+
+
+def test_backward_2d_transposed_grid_transposes_every_gradient():
+    # the 2-D convolution commutes with transposing both operands: the
+    # gradients of the transposed problem are the transposed gradients
+    v, x, h, b, dy = problem_2d(1, 2, 4, 8, 2, seed=31)
+    t = lambda a: np.swapaxes(a, -1, -2).copy()
+    got = oracle.hyena_backward_2d(t(v), t(x), t(h), b, t(dy), route="fft")
+    want = oracle.hyena_backward_2d(v, x, h, b, dy, route="direct")
+    for g_, w_, name in zip(got, want, ("dv", "dx", "dh")):
+        assert rel_err(g_, t(w_)) < 1e-12, name
+    assert rel_err(got[3], want[3]) < 1e-12
+
+
+@pytest.mark.parametrize("route", ["direct", "fft"])
+def test_backward_2d_routes_agree_and_db_is_dh_origin(route):
+    v, x, h, b, dy = problem_2d(2, 3, 8, 16, 2, seed=32)
+    got = oracle.hyena_backward_2d(v, x, h, b, dy, route=route)
+    ref = oracle.hyena_backward_2d(v, x, h, b, dy, route="direct")
+    for g_, w_ in zip(got, ref):
+        assert rel_err(g_, w_) < 1e-12
+    assert rel_err(got[3], got[2][:, :, 0, 0]) < 1e-12
