@@ -97,7 +97,9 @@ def alg_bytes_backward(wl: synth.Workload) -> int:
     dx_1..dx_N out (storage type), the spectra H in (complex64), dh and
     dbias out (float32)."""
     io = 2 if wl.io == "bf16" else 4
-    act = wl.B * wl.D * wl.L * io
+    act = wl.positions * io
+    if wl.kind == "2d":     # 2H x W spectrum slots a filter, H x W of dh
+        return (2 * wl.N + 3) * act + wl.N * wl.D * wl.H * wl.W * (16 + 4) + wl.N * wl.D * 4
     return (2 * wl.N + 3) * act + wl.N * wl.D * wl.L * (8 + 4) + wl.N * wl.D * 4
 
 
@@ -508,15 +510,26 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(bb) for a, bb in eev))
 
-    # ---- the backward pass (1-D, L <= 16384): one call per timed repetition
+    # ---- the backward pass (1-D with L <= 16384, and 2-D): one call per
+    # timed repetition
     bwd = None
-    if wl.kind == "1d" and not long_path(wl) and not wl.film and not wl.circular:
+    if (wl.kind == "1d" and not long_path(wl) and not wl.film and not wl.circular) or \
+            (wl.kind == "2d" and not wl.circular):
         dy = to_dev(synth.make_output_grad(wl), io)
-        ws_b = torch.empty(hyena.hyena_fftconv_backward_workspace_size(wl.D, wl.L, wl.N),
-                           device="cuda", dtype=torch.uint8)
+        if wl.kind == "2d":
+            ws_b = torch.empty(hyena.hyena_fftconv2d_backward_workspace_size(wl.B, wl.D, wl.H, wl.W, wl.N),
+                               device="cuda", dtype=torch.uint8)
+            bwd_kernel = "fft2d_bwd_row_kernel+fft2d_bwd_col_kernel (hyena_fftconv2d_gate_backward, all launches)"
 
-        def backward():
-            hyena.hyena_fftconv_gate_backward(v, xs, b, H, dy, workspace=ws_b)
+            def backward():
+                hyena.hyena_fftconv2d_gate_backward(v, xs, b, H, dy, workspace=ws_b)
+        else:
+            ws_b = torch.empty(hyena.hyena_fftconv_backward_workspace_size(wl.D, wl.L, wl.N),
+                               device="cuda", dtype=torch.uint8)
+            bwd_kernel = "backward1d_kernel (hyena_fftconv_gate_backward)"
+
+            def backward():
+                hyena.hyena_fftconv_gate_backward(v, xs, b, H, dy, workspace=ws_b)
 
         for _ in range(3):
             backward()
@@ -529,7 +542,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             bev[i][1].record(stream)
         torch.cuda.synchronize()
         bwd_ms = max_over_ranks(statistics.mean(a.elapsed_time(bb) for a, bb in bev))
-        bwd = {"kernel": "backward1d_kernel (hyena_fftconv_gate_backward)", "ms_per_call": bwd_ms,
+        bwd = {"kernel": bwd_kernel, "ms_per_call": bwd_ms,
                "value": wl.positions * world / (bwd_ms / 1e3), "unit": UNIT,
                "alg_bytes_per_call": alg_bytes_backward(wl),
                "achieved_gbs": alg_bytes_backward(wl) / (bwd_ms / 1e3) / 1e9}

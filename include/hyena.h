@@ -440,6 +440,34 @@ HYENA_API hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, co
                                                                hyena_dtype_t io, void* y, void* workspace,
                                                                size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------- 2-D backward */
+
+/* Bytes of workspace hyena_fftconv2d_gate_backward needs: the accumulated
+ * dh spectra [N][C][2H][W] complex64, and per wave of images the saved
+ * spectra of z_n (N x 2H x W complex), the saved c_n (N x H x W float32)
+ * and the scratch (H x W complex); (size_t)-1 for invalid sizes. */
+HYENA_API size_t hyena_fftconv2d_backward_workspace_size(int B, int C, int H, int W, int N);
+
+/* Gradients of a scalar loss through the 2-D recurrence of
+ * hyena_fftconv2d_gate_forward, given dy = dL/dy [B][C][H][W] (the chain
+ * rule; the pages give no training formulas):
+ *   dv [B][C][H][W] io, dx = HOST array of N device pointers [B][C][H][W]
+ *   io, dh [N][C][H][W] float32 (dL/dh_n, summed over the batch), dbias
+ *   [N][C] float32 (= dh_n[0][0]).
+ * Inputs as the forward with the spectra Hs [N][C][2H][W] given.  H, W
+ * powers of two in [16, 1024].  Alignment: activations, Hs, dh 16 bytes;
+ * bias, dbias 4; workspace 256.  Outputs must not overlap any input, each
+ * other or the workspace.  Per wave of images: the forward again, saving
+ * Z_n and c_n; then per order in reverse, the rows (dx_n, e = g x_n,
+ * forward rows of e) and the columns (dh spectrum += E conj(Z_n); g from
+ * (conj(H_n) + b_n) E); finally dh and db from the accumulated spectra.
+ * Deterministic (no atomics). */
+HYENA_API hyena_status_t hyena_fftconv2d_gate_backward(const void* v, const void* const* x, const float* Hs,
+                                                       const float* bias, const void* dy, int B, int C, int H,
+                                                       int W, int N, hyena_dtype_t io, void* dv,
+                                                       void* const* dx, float* dh, float* dbias,
+                                                       void* workspace, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -4,6 +4,7 @@
 
 #include "k_circular.cuh"
 #include "k_fft2d.cuh"
+#include "k_fft2d_bwd.cuh"
 #include "k_fft3d.cuh"
 #include "launch.cuh"
 
@@ -881,6 +882,111 @@ hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, const void* 
     cudaStream_t st = (cudaStream_t)stream;
     return io == HYENA_BF16 ? dispatch_fft3d_bf16(lm, lh, lz, a, N, scratch, st, false)
                             : dispatch_fft3d_f32(lm, lh, lz, a, N, scratch, st, false);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------- 2-D backward
+
+namespace {
+
+struct Bwd2dLayout {
+    size_t acc, zsave, csave, scratch, total;
+    long wcap;
+};
+
+Bwd2dLayout bwd2d_layout(int B, int C, int H, int W, int N)
+{
+    Bwd2dLayout l;
+    l.wcap = wave_images((long)B * C, H, W);
+    const size_t slots = (size_t)2 * H * W;                  // 2H x W spectrum slots
+    l.acc = 0;
+    l.zsave = l.acc + round_up(sizeof(float2) * (size_t)N * C * slots, 256);
+    l.csave = l.zsave + round_up(sizeof(float2) * (size_t)N * l.wcap * slots, 256);
+    l.scratch = l.csave + round_up(sizeof(float) * (size_t)N * l.wcap * H * W, 256);
+    l.total = l.scratch + round_up(sizeof(float2) * (size_t)l.wcap * H * W, 256);
+    return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hyena_fftconv2d_backward_workspace_size(int B, int C, int H, int W, int N)
+{
+    if (B < 1 || C < 1 || N < 1 || N > HYENA_MAX_ORDER) return (size_t)-1;
+    const int lh = exact_log2(H), lw = exact_log2(W);
+    if (lh < kMinLog2H2d || lh > kMaxLog2H2d || lw < kMinLog2W2d || lw > kMaxLog2W2d) return (size_t)-1;
+    return bwd2d_layout(B, C, H, W, N).total;
+}
+
+hyena_status_t hyena_fftconv2d_gate_backward(const void* v, const void* const* x, const float* Hs,
+                                             const float* bias, const void* dy, int B, int C, int H, int W,
+                                             int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh,
+                                             float* dbias, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!v || !x || !Hs || !bias || !dy || !dv || !dx || !dh || !dbias) return HYENA_ERR_INVALID_ARG;
+    if (B < 1 || C < 1 || N < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
+    if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
+    const int lh = exact_log2(H), lw = exact_log2(W);
+    if (lh < kMinLog2H2d || lh > kMaxLog2H2d || lw < kMinLog2W2d || lw > kMaxLog2W2d)
+        return HYENA_ERR_UNSUPPORTED;
+    if ((long)B * C > (1L << 20) || (long)N * C * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    for (int n = 0; n < N; ++n)
+        if (!x[n] || !dx[n] || !aligned(x[n], 16) || !aligned(dx[n], 16)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(v, 16) || !aligned(dy, 16) || !aligned(dv, 16) || !aligned(Hs, 16) || !aligned(dh, 16) ||
+        !aligned(bias, 4) || !aligned(dbias, 4))
+        return HYENA_ERR_INVALID_ARG;
+    const Bwd2dLayout lay = bwd2d_layout(B, C, H, W, N);
+    if (!workspace || ws_bytes < lay.total || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+
+    // every output against every input, the other outputs and the workspace
+    const size_t act = (size_t)B * C * H * W * io_bytes(io);
+    struct Range { const void* p; size_t n; };
+    Range in[kMaxOrder + 5], out[kMaxOrder + 3];
+    int ni = 0, no = 0;
+    in[ni++] = {v, act};
+    in[ni++] = {dy, act};
+    in[ni++] = {Hs, sizeof(float2) * (size_t)N * C * 2 * H * W};
+    in[ni++] = {bias, sizeof(float) * N * C};
+    in[ni++] = {workspace, lay.total};
+    for (int n = 0; n < N; ++n) in[ni++] = {x[n], act};
+    out[no++] = {dv, act};
+    out[no++] = {dh, sizeof(float) * (size_t)N * C * H * W};
+    out[no++] = {dbias, sizeof(float) * N * C};
+    for (int n = 0; n < N; ++n) out[no++] = {dx[n], act};
+    for (int o = 0; o < no; ++o) {
+        for (int i = 0; i < ni; ++i)
+            if (overlap(out[o].p, out[o].n, in[i].p, in[i].n)) return HYENA_ERR_INVALID_ARG;
+        for (int p = o + 1; p < no; ++p)
+            if (overlap(out[o].p, out[o].n, out[p].p, out[p].n)) return HYENA_ERR_INVALID_ARG;
+    }
+
+    char* ws = static_cast<char*>(workspace);
+    Bwd2dArgs a = {};
+    a.f.v = v;
+    for (int n = 0; n < kMaxOrder; ++n) {
+        a.f.x[n] = n < N ? x[n] : nullptr;
+        a.dx[n] = n < N ? dx[n] : nullptr;
+    }
+    a.f.Hs = reinterpret_cast<const float2*>(Hs);
+    a.f.bias = bias;
+    a.f.S = reinterpret_cast<float2*>(ws + lay.scratch);
+    a.f.B = B;
+    a.f.C = C;
+    a.f.H = H;
+    a.f.W = W;
+    a.dy = dy;
+    a.dv = dv;
+    a.acc = reinterpret_cast<float2*>(ws + lay.acc);
+    a.zsave = reinterpret_cast<float2*>(ws + lay.zsave);
+    a.csave = reinterpret_cast<float*>(ws + lay.csave);
+    a.dh = dh;
+    a.dbias = dbias;
+    a.wcap = (int)lay.wcap;
+    cudaStream_t st = (cudaStream_t)stream;
+    return io == HYENA_BF16 ? dispatch_bwd2d_bf16(lw, lh, a, N, st) : dispatch_bwd2d_f32(lw, lh, a, N, st);
 }
 
 }  // extern "C"

@@ -78,6 +78,9 @@ def _load() -> ctypes.CDLL:
                                           vp, sz, vp], i),
         "hyena_filter_rfft3d": ([vp, i, i, i, i, i, vp, vp], i),
         "hyena_filter_rfft2d_circular": ([vp, i, i, i, i, vp, vp], i),
+        "hyena_fftconv2d_backward_workspace_size": ([i, i, i, i, i], sz),
+        "hyena_fftconv2d_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
+                                           ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_filter_rfft3d_circular": ([vp, i, i, i, i, i, vp, vp], i),
         "hyena_fftconv3d_circular_workspace_size": ([i, i, i, i, i], sz),
         "hyena_fftconv3d_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, i, vp, vp,
@@ -547,4 +550,37 @@ def hyena_fftconv3d_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tenso
         ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+def hyena_fftconv2d_backward_workspace_size(B: int, C: int, H: int, W: int, N: int) -> int:
+    n = LIB.hyena_fftconv2d_backward_workspace_size(B, C, H, W, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv2d_backward_workspace_size", HYENA_ERR_INVALID_ARG, "invalid sizes")
+    return n
+
+
+def hyena_fftconv2d_gate_backward(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                  dy: torch.Tensor, *, workspace=None, stream=None):
+    """Gradients of a loss with dL/dy = dy through the 2-D forward: returns
+    (dv [B][C][H][W], [dx_1..dx_N], dh [N][C][H][W] float32, dbias [N][C]
+    float32); v, x_n, dy float32 or bf16, Hs the packed 2-D spectra."""
+    B, C, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty((N, C, H, W), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, C), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(hyena_fftconv2d_backward_workspace_size(B, C, H, W, N), device=v.device,
+                                dtype=torch.uint8)
+    _check("hyena_fftconv2d_gate_backward", LIB.hyena_fftconv2d_gate_backward(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+        B, C, H, W, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+        ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db
 

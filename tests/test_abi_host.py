@@ -294,3 +294,25 @@ def test_circular_nd_rejects_bad_arguments(lib):
     assert f3(P(0), xs, P(3), P(4), 2, 3, 16, 16, 32, 2, 7, P(5), P(6), need, None) == INVALID  # io
     assert f3(P(0), xs, P(3), P(4), 2, 3, 16, 16, 32, 2, F32, P(5), None, need, None) == WORKSPACE
     assert f3(P(0), xs, P(3), P(4), 2, 3, 16, 16, 32, 17, F32, P(5), P(6), need, None) == UNSUPPORTED
+
+
+def test_backward_2d_rejects_bad_arguments(lib):
+    ws = lib.hyena_fftconv2d_backward_workspace_size
+    n = ws(2, 3, 32, 64, 2)
+    # acc (N C 2H W) + saved spectra and c_n of one wave + scratch
+    assert n >= (2 * 3 * 64 * 64 * 8) + (2 * 6 * 64 * 64 * 8) + (2 * 6 * 32 * 64 * 4) + (6 * 32 * 64 * 8)
+    assert ws(2, 3, 8, 64, 2) == ctypes.c_size_t(-1).value
+    assert ws(2, 3, 32, 64, 17) == ctypes.c_size_t(-1).value
+    f = lib.hyena_fftconv2d_gate_backward
+    xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
+    dxs = (ctypes.c_void_p * 2)(P(8).value, P(9).value)
+    args = lambda **k: [k.get("v", P(0)), xs, k.get("Hs", P(3)), P(4), P(5), 2, 3, 32, 64, 2, k.get("io", F32),
+                        k.get("dv", P(6)), k.get("dxs", dxs), k.get("dh", P(7)), P(10), k.get("wsp", P(11)),
+                        k.get("nb", n), None]
+    assert f(*args(v=None)) == INVALID
+    assert f(*args(Hs=None)) == INVALID
+    assert f(*args(io=9)) == INVALID
+    assert f(*args(nb=n - 256)) == WORKSPACE
+    assert f(*args(dv=P(0))) == INVALID                                    # dv aliases v
+    assert f(*args(dh=P(6))) == INVALID                                    # dh aliases dv
+    assert f(*args(dxs=(ctypes.c_void_p * 2)(P(8).value, P(8).value))) == INVALID   # dx_1 aliases dx_2
