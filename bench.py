@@ -510,11 +510,9 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(bb) for a, bb in eev))
 
-    # ---- the backward pass (1-D with L <= 16384, and 2-D): one call per
-    # timed repetition
+    # ---- the backward pass (1-D and 2-D): one call per timed repetition
     bwd = None
-    if (wl.kind == "1d" and not long_path(wl) and not wl.film and not wl.circular) or \
-            (wl.kind == "2d" and not wl.circular):
+    if (wl.kind == "1d" and not wl.film and not wl.circular) or (wl.kind == "2d" and not wl.circular):
         dy = to_dev(synth.make_output_grad(wl), io)
         if wl.kind == "2d":
             ws_b = torch.empty(hyena.hyena_fftconv2d_backward_workspace_size(wl.B, wl.D, wl.H, wl.W, wl.N),
@@ -526,7 +524,8 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
         else:
             ws_b = torch.empty(hyena.hyena_fftconv_backward_workspace_size(wl.D, wl.L, wl.N),
                                device="cuda", dtype=torch.uint8)
-            bwd_kernel = "backward1d_kernel (hyena_fftconv_gate_backward)"
+            bwd_kernel = ("fourstep_bwd_row_kernel+fourstep_bwd_col_kernel (hyena_fftconv_gate_backward, "
+                          "all launches)" if long_path(wl) else "backward1d_kernel (hyena_fftconv_gate_backward)")
 
             def backward():
                 hyena.hyena_fftconv_gate_backward(v, xs, b, H, dy, workspace=ws_b)

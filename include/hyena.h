@@ -259,13 +259,19 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_noalloc(const void* v, const
  *   dh     [N][D][L] float32 out    summed over the batch
  *   dbias  [N][D] float32 out       summed over the batch
  *   workspace / ws_bytes: device scratch of at least
- *          hyena_fftconv_backward_workspace_size(D, L, N) bytes (20 N D L),
- *          256-byte aligned; nothing in it needs to start at zero.
- * L is a power of two, 16 <= L <= 16384 (HYENA_ERR_UNSUPPORTED above);
- * 1 <= N <= HYENA_MAX_ORDER.  Two launches: a group of threads owns a
- * channel and walks its B sequences (the forward again, then the orders
- * backwards), accumulating the channel's dh spectra, so dh and dbias need
- * no atomics and are deterministic; a second launch inverts those spectra. 
+ *          hyena_fftconv_backward_workspace_size(D, L, N) bytes (20 N D L
+ *          for L <= 16384; above, 8 N D L plus about N * 100 MB + 64 MB
+ *          for the waves), 256-byte aligned; nothing in it needs to start
+ *          at zero.
+ * L is a power of two, 16 <= L <= 2^22; 1 <= N <= HYENA_MAX_ORDER.
+ * L <= 16384: two launches: a group of threads owns a channel and walks its
+ * B sequences (the forward again, then the orders backwards), accumulating
+ * the channel's dh spectra; a second launch inverts those spectra.
+ * L > 16384 (the four-step transform): per wave of sequences the forward
+ * again, saving each order's spectrum and c_n, then per order in reverse a
+ * column launch (dx_n, e = g x_n) and a row launch per channel that
+ * accumulates the dh spectrum and forms g's; finally the spectra inverted.
+ * Both are deterministic (no atomics).
  * Alignment: v, x_n, dy, dv, dx_n, H, dh 16 bytes; bias, dbias 4.  Outputs
  * must not overlap each other, any input or the workspace. */
 HYENA_API size_t hyena_fftconv_backward_workspace_size(int D, int L, int N);

@@ -159,7 +159,7 @@ fft2d_bwd_row_kernel(Bwd2dArgs ba)
 // inverse columns of the accumulated spectra (all 2H rows), scaled by
 // 1/2H, rows y < H back in place.
 template <int LOG2H2, int MODE>
-__global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS, 1)
+__global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS, Fft2dCols<LOG2H2>::MIN_BLOCKS)
 fft2d_bwd_col_kernel(Bwd2dArgs ba)
 {
     grid_dependency_begin();

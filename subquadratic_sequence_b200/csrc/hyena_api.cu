@@ -5,6 +5,7 @@
 #include "k_circular.cuh"
 #include "k_fft2d.cuh"
 #include "k_fft2d_bwd.cuh"
+#include "k_fourstep_bwd.cuh"
 #include "k_fft3d.cuh"
 #include "launch.cuh"
 
@@ -391,8 +392,9 @@ hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* co
 size_t hyena_fftconv_backward_workspace_size(int D, int L, int N)
 {
     int log2m = 0;
-    if (D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2Fused, &log2m) != HYENA_OK)
+    if (D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2, &log2m) != HYENA_OK)
         return (size_t)-1;
+    if (log2m > kMaxLog2Fused) return fourstep_bwd_layout(log2m, D, N).total;
     const size_t spec = sizeof(float2) * (size_t)N * D * L;
     return round_up(spec, 256) * 2 + round_up(spec / 2, 256);   // acc, wz, wc
 }
@@ -408,7 +410,7 @@ hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, 
     if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
     if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
     int log2m = 0;
-    hyena_status_t s = check_len(L, kMaxLog2Fused, &log2m);
+    hyena_status_t s = check_len(L, kMaxLog2, &log2m);
     if (s != HYENA_OK) return s;
     if ((long)B * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
     for (int n = 0; n < N; ++n)
@@ -443,6 +445,32 @@ hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, 
 
     const size_t spec = sizeof(float2) * (size_t)N * D * L;
     char* ws = static_cast<char*>(workspace);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (log2m > kMaxLog2Fused) {
+        // four-step backward (L > 16384)
+        const FourStepBwdLayout lay = fourstep_bwd_layout(log2m, D, N);
+        FourStepBwdArgs b = {};
+        b.f.v = v;
+        for (int n = 0; n < kMaxOrder; ++n) {
+            b.f.x[n] = n < N ? x[n] : nullptr;
+            b.dx[n] = n < N ? dx[n] : nullptr;
+        }
+        b.f.H = reinterpret_cast<const float2*>(H);
+        b.f.bias = bias;
+        b.f.S = reinterpret_cast<float2*>(ws + lay.scratch);
+        b.f.B = B;
+        b.f.D = D;
+        b.dy = dy;
+        b.dv = dv;
+        b.zsave = reinterpret_cast<float2*>(ws + lay.zsave);
+        b.csave = reinterpret_cast<float2*>(ws + lay.csave);
+        b.acc = reinterpret_cast<float2*>(ws + lay.acc);
+        b.dh = dh;
+        b.dbias = dbias;
+        b.wcap = (int)lay.wcap;
+        return io == HYENA_BF16 ? dispatch_fourstep_bwd_bf16(log2m, b, N, st)
+                                : dispatch_fourstep_bwd_f32(log2m, b, N, st);
+    }
     Backward1dArgs a;
     a.v = v;
     a.dy = dy;
@@ -461,7 +489,6 @@ hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, 
     a.B = B;
     a.D = D;
     a.N = N;
-    cudaStream_t st = (cudaStream_t)stream;
     return io == HYENA_BF16 ? dispatch_backward_bf16(log2m, a, st) : dispatch_backward_f32(log2m, a, st);
 }
 

@@ -294,7 +294,7 @@ def hyena_fftconv_gate_backward(v: torch.Tensor, xs, bias: torch.Tensor, H: torc
                                 dy: torch.Tensor, *, workspace=None, stream=None):
     """Gradients of a loss with dL/dy = dy through the order-N forward:
     returns (dv [B][D][L], [dx_1..dx_N], dh [N][D][L] float32, dbias [N][D]
-    float32); v, x_n, dy float32 or bf16, H the packed spectra, L <= 16384."""
+    float32); v, x_n, dy float32 or bf16, H the packed spectra, L <= 2^22."""
     B, D, L = v.shape
     N = len(xs)
     io = io_dtype(v)

@@ -134,7 +134,10 @@ def test_backward_rejects_bad_arguments(lib):
     lib.hyena_fftconv_backward_workspace_size.argtypes = [ctypes.c_int] * 3
     need = lib.hyena_fftconv_backward_workspace_size(3, 64, 2)
     assert need >= 20 * 2 * 3 * 64
-    assert lib.hyena_fftconv_backward_workspace_size(3, 1 << 15, 2) == ctypes.c_size_t(-1).value
+    # four-step lengths: the accumulated spectra plus the waves' saved spectra, c_n and scratch
+    long_need = lib.hyena_fftconv_backward_workspace_size(3, 1 << 15, 2)
+    assert long_need >= 8 * 2 * 3 * (1 << 15) + (64 << 20) and long_need % 256 == 0
+    assert lib.hyena_fftconv_backward_workspace_size(3, 1 << 23, 2) == ctypes.c_size_t(-1).value
     assert lib.hyena_fftconv_backward_workspace_size(0, 64, 2) == ctypes.c_size_t(-1).value
     for k in ("v", "H", "bias", "dy", "dv", "dh", "db"):
         assert bwd(lib, **{k: None}) == INVALID, k
@@ -142,9 +145,10 @@ def test_backward_rejects_bad_arguments(lib):
     assert bwd(lib, dxs=(P(7), None)) == INVALID
     assert bwd(lib, B=0) == INVALID
     assert bwd(lib, io=3) == INVALID
-    # only the single-CTA lengths
-    assert bwd(lib, L=1 << 15) == UNSUPPORTED
+    # lengths up to 2^22 (the four-step path above 16384), powers of two
+    assert bwd(lib, L=1 << 23) == UNSUPPORTED
     assert bwd(lib, L=100) == UNSUPPORTED
+    assert bwd(lib, L=1 << 15, wsb=need) == WORKSPACE          # the four-step workspace is larger
     # workspace: missing, short, misaligned
     assert bwd(lib, ws=None) == WORKSPACE
     assert bwd(lib, wsb=need - 1) == WORKSPACE

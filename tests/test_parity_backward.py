@@ -98,3 +98,33 @@ def test_backward_of_delta_filters_is_the_closed_form(hy):
     gain = (1.0 + inp["b"][0].astype(np.float64))[None, :, None]
     assert rel_max_err(dv, dy * inp["x"][0] * gain) <= 1e-5
     assert rel_max_err(dx[0], dy * gain * inp["v"]) <= 1e-5
+
+
+# ---------------------------------------------------- four-step (L > 16384)
+
+LONG_CASES = [
+    (1, 3, 32768, 2, "f32"), (2, 2, 65536, 2, "f32"), (1, 2, 131072, 1, "bf16"), (2, 1, 262144, 3, "f32"),
+    (3, 4, 1 << 20, 1, "f32"),      # 12 sequences, 8 a wave: channel 2 spans two waves
+    (1, 1, 1 << 22, 1, "f32"),      # the longest supported length
+]
+
+
+@pytest.mark.parametrize("B,D,L,N,io", LONG_CASES)
+def test_backward_fourstep_matches_oracle(hy, B, D, L, N, io):
+    wl, inp = random_problem(B, D, L, N, seed=700 + N, io=io)
+    h32 = filters(wl, seed=L % 1000 + N)
+    dy = synth.make_output_grad(wl)
+    got = run(hy, wl, inp, h32, dy)
+    ref = oracle.hyena_backward(inp["v"], np.stack(inp["x"]), h32, inp["b"], dy)
+    check(got, ref, io, f"B{B} D{D} L{L} N{N} {io}")
+
+
+def test_backward_c3_64k_full_size(hy):
+    """Order-2, B=1, D=256, L=65536, fp32: every output compared."""
+    wl = synth.WORKLOADS["c3_64k"]
+    inp = synth.make_inputs(wl)
+    h32 = filters(wl, seed=3)
+    dy = synth.make_output_grad(wl)
+    got = run(hy, wl, inp, h32, dy)
+    ref = oracle.hyena_backward(inp["v"], np.stack(inp["x"]), h32, inp["b"], dy)
+    check(got, ref, wl.io, "c3_64k")
