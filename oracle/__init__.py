@@ -68,6 +68,7 @@ def _load():
         "oracle_rfft_circ": [dp, l, l, dp, dp],
         "oracle_hyena_forward_circular": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
         "oracle_cconv3": [dp, dp, l, l, l, i, dp],
+        "oracle_filter_gen_3d": [dp, dp, dp, dp, dp, i, i, i, i, i, i, i, d, i, dp],
         "oracle_hyena_backward_2d": [dp, dp, dp, dp, dp, l, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_hyena_forward_circular_nd": [dp, dp, dp, dp, l, l, l, l, l, l, i, dp],
     }
@@ -379,4 +380,19 @@ def hyena_backward_2d(v, x, h, bias, dy, route="fft", threads=None):
                                           _ptr(dv), _ptr(dx), _ptr(dh), _ptr(db))
     _check(rc, "oracle_hyena_backward_2d")
     return dv, dx, dh, db
+
+
+def filter_gen_3d(W1, W2, W3, Wout, alpha, N, C, Z, H, W, n_bands=8, width=64, decay_div=64.0,
+                  threads=None) -> np.ndarray:
+    """Implicit 3-D filters h[N][C][Z][H][W] (float64): the filter network
+    on [tz, ty, tx, (sin, cos)(2 pi k t) per axis], window
+    exp(-alpha_c (iz + iy + ix) / decay_div)."""
+    W1, W2, W3, Wout, alpha = map(_f64, (W1, W2, W3, Wout, alpha))
+    assert W1.shape == (width, 3 + 6 * n_bands) and Wout.shape == (N * C, width)
+    assert alpha.shape == (C,)
+    h = np.empty((N, C, Z, H, W), dtype=np.float64)
+    rc = _load().oracle_filter_gen_3d(_ptr(W1), _ptr(W2), _ptr(W3), _ptr(Wout), _ptr(alpha), N, C, Z, H, W,
+                                      n_bands, width, float(decay_div), threads or default_threads(), _ptr(h))
+    _check(rc, "oracle_filter_gen_3d")
+    return h
 

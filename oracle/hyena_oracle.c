@@ -1493,3 +1493,86 @@ int oracle_hyena_backward_2d(const double *v, const double *x, const double *h, 
     free(jobs); free(tid);
     return st;
 }
+
+/* ------------------------------------------------------------------ */
+/* Implicit 3-D filters: the filter network of the 1-D and 2-D forms on */
+/* positional features of a volume (Native ND Convolution: a global     */
+/* filter on an L1 x ... x LN grid, produced by the implicit filter MLP */
+/* from the position).  Features [tz, ty, tx, (sin, cos)(2 pi k tz),    */
+/* (sin, cos)(2 pi k ty), (sin, cos)(2 pi k tx)], k = 1..K, t = i / n   */
+/* per axis; window exp(-alpha_c (iz + iy + ix) / decay_div), the       */
+/* product of the three axis windows.                                   */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    const double *W1, *W2, *W3, *Wout, *alpha;
+    int N, C, Z, H, W, n_bands, width;
+    double decay_div;
+    double *h;
+    long p0, p1; /* flattened volume positions handled by this worker */
+    int status;
+} fg3_job;
+
+static void *filter_gen_3d_worker(void *arg)
+{
+    fg3_job *j = (fg3_job *)arg;
+    const int K = j->n_bands, n_in = 3 + 6 * K, n_out = j->N * j->C;
+    const long V = (long)j->Z * j->H * j->W;
+    double *phi = malloc(sizeof(double) * n_in);
+    double *a1 = malloc(sizeof(double) * j->width), *a2 = malloc(sizeof(double) * j->width);
+    double *a3 = malloc(sizeof(double) * j->width), *o = malloc(sizeof(double) * n_out);
+    if (!phi || !a1 || !a2 || !a3 || !o) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (long p = j->p0; p < j->p1; ++p) {
+        const long iz = p / ((long)j->H * j->W), iy = (p / j->W) % j->H, ix = p % j->W;
+        const double t[3] = {(double)iz / j->Z, (double)iy / j->H, (double)ix / j->W};
+        for (int a = 0; a < 3; ++a) {
+            phi[a] = t[a];
+            for (int k = 1; k <= K; ++k) {
+                phi[3 + 2 * K * a + 2 * (k - 1)] = sin(2.0 * ORACLE_PI * k * t[a]);
+                phi[3 + 2 * K * a + 2 * (k - 1) + 1] = cos(2.0 * ORACLE_PI * k * t[a]);
+            }
+        }
+        ffn(j->W1, j->W2, j->W3, j->Wout, n_in, j->width, n_out, phi, a1, a2, a3, o);
+        for (int n = 0; n < j->N; ++n)
+            for (int c = 0; c < j->C; ++c) {
+                const double window = exp(-j->alpha[c] * (double)(iz + iy + ix) / j->decay_div);
+                j->h[((long)n * j->C + c) * V + p] = o[n * j->C + c] * window;
+            }
+    }
+    j->status = ORACLE_OK;
+done:
+    free(phi); free(a1); free(a2); free(a3); free(o);
+    return NULL;
+}
+
+/* h[N][C][Z][H][W] from the FFN weights (W1 [width][3+6K]) and alpha[C]. */
+int oracle_filter_gen_3d(const double *W1, const double *W2, const double *W3, const double *Wout,
+                         const double *alpha, int N, int C, int Z, int H, int W, int n_bands, int width,
+                         double decay_div, int nthreads, double *h)
+{
+    if (!W1 || !W2 || !W3 || !Wout || !alpha || !h || N < 1 || C < 1 || Z < 1 || H < 1 || W < 1 ||
+        n_bands < 0 || width < 1 || !(decay_div > 0.0))
+        return ORACLE_EBADARG;
+    const long V = (long)Z * H * W;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > V) nthreads = (int)V;
+    fg3_job *jobs = calloc(nthreads, sizeof(fg3_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        fg3_job jb = {W1, W2, W3, Wout, alpha, N, C, Z, H, W, n_bands, width, decay_div, h,
+                      V * k / nthreads, V * (k + 1) / nthreads, 0};
+        jobs[k] = jb;
+        pthread_create(&tid[k], NULL, filter_gen_3d_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}

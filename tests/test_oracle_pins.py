@@ -421,3 +421,67 @@ def test_forward_3d_delta_filter_and_routes(route):
     h = r.standard_normal((N, C, Z, H, W))
     assert rel_err(oracle.hyena_forward_3d(v, x, h, b, route="fft"),
                    oracle.hyena_forward_3d(v, x, h, b, route="direct")) < 1e-12
+
+
+# --------------------------------------------------------- 3-D filters
+
+def test_filter_gen_3d_closed_form():
+    # K = 2 bands -> features [tz, ty, tx, s1z, c1z, s2z, c2z, s1y, c1y, s2y, c2y, s1x, c1x, s2x, c2x]
+    K, width, N, C, Z, H, W = 2, 6, 2, 2, 4, 8, 16
+    n_in = 3 + 6 * K
+    sel = np.array([0, 1, 2, 6, 8, 13])          # tz, ty, tx, c2z, c1y, s2x
+    coef = np.array([1.1, -0.6, 0.7, 1.9, 0.8, -1.3])
+    perm2 = np.array([3, 2, 0, 1, 5, 4])
+    perm3 = np.array([1, 0, 3, 2, 4, 5])
+    head = np.array([0, 3, 5, 1])
+    W1, W2, W3, Wout = _selector_ffn(n_in, width, N * C, sel, coef, perm2, perm3, head)
+    alpha = np.array([0.3, 1.5])
+    h = oracle.filter_gen_3d(W1, W2, W3, Wout, alpha, N, C, Z, H, W, n_bands=K, width=width)
+    iz, iy, ix = np.meshgrid(np.arange(Z), np.arange(H), np.arange(W), indexing="ij")
+    tz, ty, tx = iz / Z, iy / H, ix / W
+    feats = [tz, ty, tx]
+    for t in (tz, ty, tx):
+        feats += [np.sin(2 * np.pi * t), np.cos(2 * np.pi * t), np.sin(4 * np.pi * t), np.cos(4 * np.pi * t)]
+    a1 = [np.sin(coef[j] * feats[sel[j]]) for j in range(width)]
+    a2 = [np.sin(a1[perm2[j]]) for j in range(width)]
+    a3 = [np.sin(a2[perm3[j]]) for j in range(width)]
+    for n in range(N):
+        for c in range(C):
+            ref = a3[head[n * C + c]] * np.exp(-alpha[c] * (iz + iy + ix) / 64.0)
+            assert np.max(np.abs(h[n, c] - ref)) < 1e-14
+
+
+def test_filter_gen_3d_without_z_features_is_the_2d_filter_times_the_z_window():
+    # W1 columns of the z features zeroed: every plane is the 2-D filter
+    # (the pinned 2-D oracle, same y/x columns) times exp(-alpha iz / 64)
+    r = rng(40)
+    K, width, N, C, Z, H, W = 3, 8, 2, 3, 4, 8, 16
+    W1 = r.standard_normal((width, 3 + 6 * K))
+    W2, W3 = r.standard_normal((width, width)), r.standard_normal((width, width))
+    Wout, alpha = r.standard_normal((N * C, width)), np.linspace(0.3, 1.5, C)
+    zcols = [0] + list(range(3, 3 + 2 * K))
+    W1[:, zcols] = 0.0
+    # the 2-D oracle's columns: [ty, tx, y bands, x bands]
+    W1_2d = W1[:, [1, 2] + list(range(3 + 2 * K, 3 + 6 * K))]
+    h3 = oracle.filter_gen_3d(W1, W2, W3, Wout, alpha, N, C, Z, H, W, n_bands=K, width=width)
+    # cos(0) = 1 in the zeroed z columns contributes nothing, so each plane differs only by the window
+    h2 = oracle.filter_gen_2d(W1_2d, W2, W3, Wout, alpha, N, C, H, W, n_bands=K, width=width)
+    win_z = np.exp(-alpha[None, :, None, None, None] * np.arange(Z)[None, None, :, None, None] / 64.0)
+    assert rel_err(h3, h2[:, :, None] * win_z) < 1e-13
+
+
+def test_filter_gen_3d_axis_permutation():
+    # swapping the roles of y and x (volume transposed, W1 columns swapped)
+    # transposes the filter
+    r = rng(41)
+    K, width, N, C, Z, H, W = 2, 8, 1, 2, 4, 8, 16
+    W1 = r.standard_normal((width, 3 + 6 * K))
+    W2, W3 = r.standard_normal((width, width)), r.standard_normal((width, width))
+    Wout, alpha = r.standard_normal((N * C, width)), np.array([0.4, 1.2])
+    ycols = [1] + list(range(3 + 2 * K, 3 + 4 * K))
+    xcols = [2] + list(range(3 + 4 * K, 3 + 6 * K))
+    W1s = W1.copy()
+    W1s[:, ycols], W1s[:, xcols] = W1[:, xcols], W1[:, ycols]
+    a = oracle.filter_gen_3d(W1, W2, W3, Wout, alpha, N, C, Z, H, W, n_bands=K, width=width)
+    b = oracle.filter_gen_3d(W1s, W2, W3, Wout, alpha, N, C, Z, W, H, n_bands=K, width=width)
+    assert rel_err(b, np.swapaxes(a, -1, -2)) < 1e-13
