@@ -56,7 +56,8 @@ def _describe(wl: synth.Workload) -> dict:
                             f"{wl.Z}x{wl.H}x{wl.W} volumes (padded to {2 * wl.Z}x{2 * wl.H}x{2 * wl.W}), "
                             f"{wl.io} storage, fp32 compute",
                 "N": wl.N, "B": wl.B, "C": wl.D, "Z": wl.Z, "H": wl.H, "W": wl.W, "io": wl.io,
-                "filters": "given (seeded decaying random volumes); their 3-D spectra recomputed every step",
+                "filters": f"implicit FFN over (z/Z, y/H, x/W) (3 sine layers of width {synth.WIDTH}, "
+                           f"{synth.N_BANDS} bands per axis) x separable decay, regenerated every step",
                 "l2": "flushed (256 MB write) before every timed step"}
     if wl.kind == "2d":
         return {"workload": f"{wl.name}: order-{wl.N} Hyena 2-D operator, B={wl.B}, C={wl.D}, "
@@ -141,8 +142,6 @@ def launches_rfft(wl: synth.Workload) -> int:
 
 
 def launches_filter_gen(wl: synth.Workload) -> int:
-    if wl.kind == "3d":
-        return 0
     return 3 if wl.N * wl.D > 64 else 1
 
 
@@ -326,13 +325,13 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     v = to_dev(inp["v"], io)
     xs = [to_dev(x, io) for x in inp["x"]]
     b = to_dev(inp["b"])
-    wkeys = ("h",) if wl.kind == "3d" else ("W1", "W2", "W3", "Wout", "alpha")
+    wkeys = ("W1", "W2", "W3", "Wout", "alpha")
     W = [to_dev(inp[k]) for k in wkeys]
     y = torch.empty_like(v)
     flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
     stream = torch.cuda.current_stream()
     if wl.circular and wl.kind == "3d":
-        h = W[0]
+        h = torch.empty((wl.N, wl.D, wl.Z, wl.H, wl.W), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.N, wl.D, wl.Z, wl.H, wl.W // 2), device="cuda", dtype=torch.complex64)
         ws_fwd = torch.empty(hyena.hyena_fftconv3d_circular_workspace_size(wl.B, wl.D, wl.Z, wl.H, wl.W),
                              device="cuda", dtype=torch.uint8)
@@ -341,6 +340,8 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             hyena.hyena_fftconv3d_gate_forward_circular(v, xs, b, H, out=y, workspace=ws_fwd)
 
         def step():
+            hyena.hyena_filter_gen_3d(*W, wl.N, wl.D, wl.Z, wl.H, wl.W, n_bands=synth.N_BANDS,
+                                      width=synth.WIDTH, decay_div=synth.DECAY_DIV, out=h)
             hyena.hyena_filter_rfft3d_circular(h, out=H)
             forward()
     elif wl.circular and wl.kind == "2d":
@@ -370,7 +371,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             hyena.hyena_filter_rfft_circular(h, out=H)
             forward()
     elif wl.kind == "3d":
-        h = W[0]
+        h = torch.empty((wl.N, wl.D, wl.Z, wl.H, wl.W), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.N, wl.D, 2 * wl.Z, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
         ws_n = hyena.hyena_fftconv3d_workspace_size(wl.B, wl.D, wl.Z, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
         ws_fwd = torch.empty(ws_n, device="cuda", dtype=torch.uint8)
@@ -379,6 +380,8 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             hyena.hyena_fftconv3d_gate_forward(v, xs, b, Hs=H, out=y, workspace=ws_fwd)
 
         def step():
+            hyena.hyena_filter_gen_3d(*W, wl.N, wl.D, wl.Z, wl.H, wl.W, n_bands=synth.N_BANDS,
+                                      width=synth.WIDTH, decay_div=synth.DECAY_DIV, out=h)
             hyena.hyena_filter_rfft3d(h, out=H)
             forward()
     elif wl.kind == "2d":
@@ -590,8 +593,14 @@ def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: 
     v = inp["v"][:, channels].astype(np.float64)
     x = np.stack([xx[:, channels] for xx in inp["x"]]).astype(np.float64)
     bias = inp["b"][:, channels].astype(np.float64)
-    if wl.circular and wl.kind == "3d":
-        oracle.hyena_forward_circular_nd(v, x, inp["h"][:, channels].astype(np.float64), bias, route="fft")
+    if wl.kind == "3d":
+        h = oracle.filter_gen_3d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
+                                 wl.N, len(channels), wl.Z, wl.H, wl.W, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                 decay_div=synth.DECAY_DIV, threads=threads)
+        if wl.circular:
+            oracle.hyena_forward_circular_nd(v, x, h, bias, route="fft")
+        else:
+            oracle.hyena_forward_3d(v, x, h, bias, route="fft")
         return time.perf_counter() - t0
     if wl.circular and wl.kind == "2d":
         h = oracle.filter_gen_2d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
@@ -604,9 +613,6 @@ def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: 
                               wl.N, len(channels), wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
                               decay_div=synth.DECAY_DIV, threads=threads)
         oracle.hyena_forward_circular(v, x, h, bias, route="fft", threads=threads)
-        return time.perf_counter() - t0
-    if wl.kind == "3d":
-        oracle.hyena_forward_3d(v, x, inp["h"][:, channels].astype(np.float64), bias, route="fft")
         return time.perf_counter() - t0
     if wl.kind == "2d":
         h = oracle.filter_gen_2d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
@@ -646,7 +652,7 @@ def one_thread(wl: synth.Workload) -> bool:
 def stages(wl: synth.Workload) -> str:
     circ = "circular " if wl.circular else ""
     if wl.kind == "3d":
-        return f"3-D spectra + order-{wl.N} {circ}forward, one thread"
+        return f"3-D filter generation (all cores) + order-{wl.N} {circ}forward (one thread)"
     if one_thread(wl):
         return f"filter generation (all cores) + order-{wl.N} {circ}forward (one thread)"
     if wl.circular:
@@ -667,7 +673,7 @@ def cpu_baseline(wl: synth.Workload, budget_s: float = 15.0, inp: dict | None = 
         n = n2
         t = oracle_sample(wl, inp, np.sort(rng.choice(wl.D, n, replace=False)), threads)
     positions = wl.B * n * wl.per_channel
-    cores = 1 if wl.kind == "3d" else threads
+    cores = threads
     return {"value": positions / t, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{n} of {wl.D} channels x all {wl.B} batch elements x {extent(wl)} "
                       f"({stages(wl)}, float64 FFT route), {t:.1f} s"}
@@ -695,7 +701,7 @@ def run_reference(args, wl: synth.Workload) -> dict | None:
     value = positions * args.steps / total
     sample = (f"{n} of {wl.D} channels x all {wl.B} batch elements x {extent(wl)} per step "
               f"({stages(wl)}, float64 FFT route)")
-    threads = 1 if wl.kind == "3d" else threads
+
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

@@ -350,6 +350,16 @@ HYENA_API hyena_status_t hyena_fftconv2d_gate_forward_per_sample(const void* v, 
 
 /* ---------------------------------------------------------------- 3-D */
 
+/* Implicit 3-D filters h [N][C][Z][H][W] float32: the filter network of
+ * hyena_ffn_t on per-axis features of the volume,
+ *   phi(iz, iy, ix) = [tz, ty, tx, (sin, cos)(2 pi k tz) for k = 1..n_bands,
+ *                      the same for ty, then for tx],  t = i / n per axis
+ * (W1 is [width][3 + 6 n_bands]), times the separable decay window
+ * exp(-alpha_c (iz + iy + ix) / decay_div).  n_bands <= 10 (else
+ * HYENA_ERR_UNSUPPORTED).  Any Z, H, W >= 1. */
+HYENA_API hyena_status_t hyena_filter_gen_3d(const hyena_ffn_t* ffn, int N, int C, int Z, int H, int W,
+                                             float* h, void* stream);
+
 /* 3-D filter spectra Hs [N][C][2Z][2H][W] complex64, for filters h
  * [N][C][Z][H][W] float32 (offsets 0..Z-1 x 0..H-1 x 0..W-1) zero-padded
  * to 2Z x 2H x 2W ("Native Multi-Dimensional Subquadratic Operators via

@@ -41,8 +41,9 @@ struct FilterGenArgs {
     const float *W1, *W2, *W3, *Wout, *alpha;
     int n_in, width, rows;         // rows = N * D
     int D;                         // channels (alpha index = row % D)
-    int L;                         // 1-D length; 0 for 2-D
-    int Hh, Ww;                    // 2-D grid; 0 for 1-D
+    int L;                         // 1-D length; 0 for 2-D and 3-D
+    int Hh, Ww;                    // 2-D grid (the planes of a 3-D volume); 0 for 1-D
+    int Zz;                        // 3-D volume depth; 0 for 1-D and 2-D (3-D runs the 2-D kernels)
     int n_bands;
     float inv_div;                 // 1 / decay_div
     float* h;                      // [rows][positions] (per sample with FiLM)
@@ -55,6 +56,7 @@ struct FilterGenArgs {
     int film;                      // 1: modulate (any of the three given)
     int gaussian;                  // 1: window exp(-t^2 / (2 sigma^2)), sigma in alpha[]
     float inv_L, inv_H, inv_W;     // 1/L (1-D), 1/H and 1/W (2-D): t = i/L, ty = iy/H, tx = ix/W
+    float inv_Z;                   // 1/Z (3-D): tz = iz/Z
     long sample_stride;            // floats of h per sample (rows * positions)
 };
 
@@ -74,6 +76,18 @@ __device__ __forceinline__ void select_sample(FilterGenArgs& a)
     if (a.gamma) a.gamma += (long)b * 3 * a.width;
     if (a.beta) a.beta += (long)b * 3 * a.width;
 }
+
+// Positions of one filter: L (1-D), H W (2-D) or Z H W (3-D).
+template <bool TWO_D>
+__device__ __forceinline__ long fg_positions(const FilterGenArgs& a)
+{
+    if constexpr (!TWO_D) return (long)a.L;
+    else return (long)(a.Zz ? a.Zz : 1) * a.Hh * a.Ww;
+}
+
+// 3-D feature slots (n_bands <= 10): [tz, ty, tx], then per axis a (z, y,
+// x) and band b = 1..10 the pair (sin, cos) at 3 + 20 a + 2 (b - 1).
+constexpr int kFg3dBands = 10;
 
 constexpr int kFgThreads = 256;     // a 16 x 16 thread grid
 constexpr int kFgTile = 64;         // positions per head / tail / layers tile
@@ -131,6 +145,33 @@ __device__ __forceinline__ void features_tile(const FilterGenArgs& a, long npos,
                 sX[(2 * k) * AS + p] = cs;
             }
         }
+    } else if (a.Zz) {
+        for (int e = tid; e < (1 + 3 * kFg3dBands) * PT; e += kFgThreads) {
+            const int k = e / PT, p = e % PT;
+            const long pos = p0 + p;
+            const int ip = (int)pos, iz = ip / (a.Hh * a.Ww), iyx = ip - iz * (a.Hh * a.Ww);
+            const int iy = iyx / a.Ww, ix = iyx - iy * a.Ww;
+            if (k == 0) {
+                sX[p] = pos < npos ? (float)iz / (float)a.Zz : 0.0f;
+                sX[AS + p] = pos < npos ? (float)iy / (float)a.Hh : 0.0f;
+                sX[2 * AS + p] = pos < npos ? (float)ix / (float)a.Ww : 0.0f;
+            } else {
+                const int axis = (k - 1) / kFg3dBands, band = (k - 1) % kFg3dBands + 1;
+                float sn = 0.0f, cs = 0.0f;
+                if (band <= a.n_bands && pos < npos) {
+                    const int n = axis == 0 ? a.Zz : (axis == 1 ? a.Hh : a.Ww);
+                    const int c = axis == 0 ? iz : (axis == 1 ? iy : ix);
+                    const int qk = (int)(((long)band * c) % n);
+                    sincospif(2.0f * (float)qk / (float)n, &sn, &cs);
+                }
+                const int slot = 3 + 2 * kFg3dBands * axis + 2 * (band - 1);
+                sX[slot * AS + p] = sn;
+                sX[(slot + 1) * AS + p] = cs;
+            }
+        }
+        // slots 63 .. kFfnMaxIn - 1 are never written: their W1 rows are zero
+        for (int e = tid; e < (kFfnMaxIn - 3 - 6 * kFg3dBands) * PT; e += kFgThreads)
+            sX[(3 + 6 * kFg3dBands + e / PT) * AS + e % PT] = 0.0f;
     } else {
         constexpr int XB = 2 + 2 * 16;                  // slot of the first x-band feature
         for (int e = tid; e < 33 * PT; e += kFgThreads) {
@@ -178,6 +219,14 @@ __device__ __forceinline__ void stage_weights(const FilterGenArgs& a, float* sW)
             int src = -1;
             if constexpr (!TWO_D) {
                 src = c < a.n_in ? c : -1;
+            } else if (a.Zz) {
+                // canonical 3-D slot -> W1 column [tz, ty, tx, z bands, y bands, x bands]
+                if (c < 3) {
+                    src = c;
+                } else if (c < 3 + 6 * kFg3dBands) {
+                    const int axis = (c - 3) / (2 * kFg3dBands), rem = (c - 3) % (2 * kFg3dBands);
+                    if (rem < 2 * a.n_bands) src = 3 + 2 * a.n_bands * axis + rem;
+                }
             } else {
                 constexpr int XB = 2 + 2 * 16;
                 if (c < 2 + 2 * a.n_bands) src = c;
@@ -305,12 +354,17 @@ __device__ __forceinline__ float window_u(const FilterGenArgs& a, long pos)
         }
         return (float)pos;
     } else {
-        const int ip = (int)pos, iy = ip / a.Ww, ix = ip - iy * a.Ww;
-        if (a.gaussian) {
-            const float ty = (float)iy * a.inv_H, tx = (float)ix * a.inv_W;
-            return ty * ty + tx * tx;
+        int ip = (int)pos, iz = 0;
+        if (a.Zz) {
+            iz = ip / (a.Hh * a.Ww);
+            ip -= iz * (a.Hh * a.Ww);
         }
-        return (float)(iy + ix);
+        const int iy = ip / a.Ww, ix = ip - iy * a.Ww;
+        if (a.gaussian) {
+            const float tz = (float)iz * a.inv_Z, ty = (float)iy * a.inv_H, tx = (float)ix * a.inv_W;
+            return tz * tz + ty * ty + tx * tx;
+        }
+        return (float)(iz + iy + ix);
     }
 }
 
@@ -459,7 +513,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_layers_kernel(FilterGenArgs
     float* sX = fg_smem + kFgWRegion;
     float* sY = sX + kFfnMaxIn * AS;
     float* sF = sY + kFfnWidth * AS;
-    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long npos = fg_positions<TWO_D>(a);
     const long ntiles = (npos + PT - 1) / PT;
     float* stash = a.h + (long)(a.rows - kFfnWidth) * npos;
     const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
@@ -502,7 +556,7 @@ __global__ void __launch_bounds__(kFgThreads, NG == 1 ? 3 : 2) filter_head_kerne
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][132]: Wout tile, transposed
     float* sA = fg_smem + kFfnWidth * kFgRS;                // [64][64 NG + 4]: a3 tile
-    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long npos = fg_positions<TWO_D>(a);
     const long p0 = (long)blockIdx.x * (64 * NG);
     const int r0 = blockIdx.y * kFgRowTile;
     const int stash_row = a.rows - kFfnWidth;
@@ -524,7 +578,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_tail_kernel(FilterGenArgs a
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][68]: Wout stash rows, transposed
     float* sA = fg_smem + kFfnWidth * kFgUS;                // [64][68]: a3 tile
-    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long npos = fg_positions<TWO_D>(a);
     const long p0 = (long)blockIdx.x * kFgTile;
     const int stash_row = a.rows - kFfnWidth;
     float al[4];
@@ -546,7 +600,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_tail16_kernel(FilterGenArgs
     extern __shared__ __align__(16) float fg_smem[];
     float* sWT = fg_smem;                                   // [64][68]: Wout stash rows, transposed
     float* sA = fg_smem + kFfnWidth * kFgUS;                // [64][20]: a3 tile
-    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long npos = fg_positions<TWO_D>(a);
     const long p0 = (long)blockIdx.x * PT;
     const int stash_row = a.rows - kFfnWidth;
     float* stash = a.h + (long)stash_row * npos;
@@ -599,7 +653,7 @@ __global__ void __launch_bounds__(kFgThreads) filter_gen_kernel(FilterGenArgs a)
     float* sX = fg_smem + kFgWRegion;
     float* sY = sX + kFfnMaxIn * LT::AS;
     float* sF = sY + kFfnWidth * LT::AS;
-    const long npos = TWO_D ? (long)a.Hh * a.Ww : (long)a.L;
+    const long npos = fg_positions<TWO_D>(a);
     const long p0 = (long)blockIdx.x * kFgTile;
     float al[4];
     load_alpha<4>(a, 0, a.rows, al);

@@ -75,11 +75,13 @@ hyena_status_t check_ffn(const hyena_ffn_t* f)
 
 hyena_status_t filter_gen(const hyena_ffn_t* f, int rows, int D, long npos, int L, int Hh,
                           int Ww, bool two_d, float* h, cudaStream_t st,
-                          const hyena_film_t* film = nullptr, int B = 1)
+                          const hyena_film_t* film = nullptr, int B = 1, int Zz = 0)
 {
     FilterGenArgs a = {};
     a.W1 = f->W1; a.W2 = f->W2; a.W3 = f->W3; a.Wout = f->Wout; a.alpha = f->alpha;
-    a.n_in = two_d ? 2 + 4 * f->n_bands : 1 + 2 * f->n_bands;
+    a.n_in = !two_d ? 1 + 2 * f->n_bands : (Zz ? 3 + 6 * f->n_bands : 2 + 4 * f->n_bands);
+    a.Zz = Zz;
+    a.inv_Z = Zz > 0 ? 1.0f / (float)Zz : 0.0f;
     a.width = f->width;
     a.rows = rows;
     a.D = D;
@@ -194,6 +196,19 @@ hyena_status_t hyena_filter_gen_2d(const hyena_ffn_t* ffn, int N, int C, int H, 
         (long)N * C * (long)H * W > (1L << 40))
         return HYENA_ERR_UNSUPPORTED;
     return filter_gen(ffn, N * C, C, (long)H * W, 0, H, W, true, h, (cudaStream_t)stream);
+}
+
+hyena_status_t hyena_filter_gen_3d(const hyena_ffn_t* ffn, int N, int C, int Z, int H, int W, float* h,
+                                   void* stream)
+{
+    hyena_status_t s = check_ffn(ffn);
+    if (s != HYENA_OK) return s;
+    if (!h || N < 1 || C < 1 || Z < 1 || H < 1 || W < 1 || !aligned(h, 4)) return HYENA_ERR_INVALID_ARG;
+    if (ffn->n_bands > kFg3dBands) return HYENA_ERR_UNSUPPORTED;
+    const long npos = (long)Z * H * W;
+    if (npos > (1L << 30) || (long)N * C > 65535L * kFgRowTile || (long)N * C * npos > (1L << 40))
+        return HYENA_ERR_UNSUPPORTED;
+    return filter_gen(ffn, N * C, C, npos, 0, H, W, true, h, (cudaStream_t)stream, nullptr, 1, Z);
 }
 
 size_t hyena_filter_rfft_workspace_size(int N, int D, int L)

@@ -77,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv2d_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
                                           vp, sz, vp], i),
         "hyena_filter_rfft3d": ([vp, i, i, i, i, i, vp, vp], i),
+        "hyena_filter_gen_3d": ([ffn_p, i, i, i, i, i, vp, vp], i),
         "hyena_filter_rfft2d_circular": ([vp, i, i, i, i, vp, vp], i),
         "hyena_fftconv2d_backward_workspace_size": ([i, i, i, i, i], sz),
         "hyena_fftconv2d_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
@@ -583,4 +584,15 @@ def hyena_fftconv2d_gate_backward(v: torch.Tensor, xs, bias: torch.Tensor, Hs: t
         ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return dv, dxs, dh, db
+
+
+def hyena_filter_gen_3d(W1, W2, W3, Wout, alpha, N: int, C: int, Z: int, H: int, W: int, *,
+                        n_bands: int = 8, width: int = 64, decay_div: float = 64.0, out=None, stream=None):
+    """Implicit 3-D filters h [N][C][Z][H][W] float32 (W1 [width][3 + 6 n_bands])."""
+    f = _ffn(W1, W2, W3, Wout, alpha, n_bands, width, decay_div)
+    if out is None:
+        out = torch.empty((N, C, Z, H, W), device=W1.device, dtype=torch.float32)
+    _check("hyena_filter_gen_3d", LIB.hyena_filter_gen_3d(
+        ctypes.byref(f), N, C, Z, H, W, ctypes.c_void_p(_dev(out, torch.float32, "h")), _stream(stream)))
+    return out
 

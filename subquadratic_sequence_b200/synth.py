@@ -95,8 +95,7 @@ WORKLOADS = {
     # c1 with input-dependent filters: a filter set per sample (FiLM-modulated
     # sine layers, multi-frequency first layer, Gaussian window)
     "c1_film": Workload("c1_film", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), film=True),
-    # order-2 3-D operator on 64^3 volumes, B=2, C=32, bf16 storage (the
-    # filters are inputs: seeded decaying random volumes)
+    # order-2 3-D operator on 64^3 volumes, B=2, C=32, bf16 storage
     "c5_3d": Workload("c5_3d", "3d", N=2, B=2, D=32, Z=64, H=64, W=64, io="bf16", seed=_seed(5)),
     # circular mode (periodic boundaries) at the shapes of c1, c4 and c5_3d
     "c1_circ": Workload("c1_circ", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), circular=True),
@@ -146,9 +145,7 @@ def make_inputs(wl: Workload) -> dict:
     v = _activation(rng, shape, wl.io)
     x = [_activation(rng, shape, wl.io) for _ in range(wl.N)]
     b = rng.standard_normal((wl.N, wl.D)).astype(np.float32)
-    if wl.kind == "3d":
-        return dict(v=v, x=x, b=b, h=filters_3d(rng, wl.N, wl.D, wl.Z, wl.H, wl.W))
-    n_in = 1 + 2 * N_BANDS if wl.kind == "1d" else 2 + 4 * N_BANDS
+    n_in = {"1d": 1 + 2 * N_BANDS, "2d": 2 + 4 * N_BANDS, "3d": 3 + 6 * N_BANDS}[wl.kind]
     W1, W2, W3, Wout = _weights(rng, n_in, WIDTH, wl.N * wl.D)
     alpha = np.linspace(0.3, 1.5, wl.D).astype(np.float32)
     out = dict(v=v, x=x, b=b, W1=W1, W2=W2, W3=W3, Wout=Wout, alpha=alpha)
@@ -178,14 +175,3 @@ def make_output_grad(wl: Workload) -> np.ndarray:
     stream (seed + 1) so the forward inputs are unchanged."""
     rng = np.random.default_rng(wl.seed + 1)
     return _activation(rng, wl.shape, wl.io)
-
-
-def filters_3d(rng: np.random.Generator, N: int, C: int, Z: int, H: int, W: int) -> np.ndarray:
-    """Seeded 3-D filters [N][C][Z][H][W] float32: N(0, 1) values under a
-    separable exponential envelope exp(-4 (iz/Z + iy/H + ix/W)), scaled by
-    8 / sqrt(Z H W) (long, decaying, O(1) response)."""
-    h = rng.standard_normal((N, C, Z, H, W), dtype=np.float32)
-    h *= np.exp(-np.arange(Z, dtype=np.float32) / (Z / 4))[:, None, None]
-    h *= np.exp(-np.arange(H, dtype=np.float32) / (H / 4))[:, None]
-    h *= np.exp(-np.arange(W, dtype=np.float32) / (W / 4))
-    return (h * np.float32(8.0 / np.sqrt(Z * H * W))).astype(np.float32)

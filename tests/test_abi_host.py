@@ -320,3 +320,15 @@ def test_backward_2d_rejects_bad_arguments(lib):
     assert f(*args(dv=P(0))) == INVALID                                    # dv aliases v
     assert f(*args(dh=P(6))) == INVALID                                    # dh aliases dv
     assert f(*args(dxs=(ctypes.c_void_p * 2)(P(8).value, P(8).value))) == INVALID   # dx_1 aliases dx_2
+
+
+def test_filter_gen_3d_rejects_bad_arguments(lib):
+    from subquadratic_sequence_b200 import hyena
+    f = lib.hyena_filter_gen_3d
+    ffn = hyena.hyena_ffn_t(P(0).value, P(1).value, P(2).value, P(3).value, P(4).value, 11, 64, 64.0)
+    assert f(ctypes.byref(ffn), 2, 3, 4, 8, 16, P(5), None) == UNSUPPORTED        # n_bands > 10
+    ffn.n_bands = 8
+    assert f(ctypes.byref(ffn), 2, 3, 0, 8, 16, P(5), None) == INVALID           # Z < 1
+    assert f(ctypes.byref(ffn), 2, 3, 4, 8, 16, None, None) == INVALID           # no output
+    ffn.width = 65
+    assert f(ctypes.byref(ffn), 2, 3, 4, 8, 16, P(5), None) == UNSUPPORTED        # width > 64

@@ -160,3 +160,40 @@ def test_forward_3d_largest_volume_shift_filters(hy):
     sh[..., 3:, 5:, 7:] = z1[..., :-3, :-5, :-7]
     ref = x64[1] * (sh + b[1].astype(np.float64)[None, :, None, None, None] * z1)
     assert_close(got, ref, "bf16", "3-D 256^3 shift filters")
+
+
+# ------------------------------------------------- implicit 3-D filters
+
+def ffn_3d(rng, N, C, K, width=64):
+    n_in = 3 + 6 * K
+    W1 = rng.standard_normal((width, n_in)) / np.sqrt(n_in)
+    W2 = rng.standard_normal((width, width)) / np.sqrt(width)
+    W3 = rng.standard_normal((width, width)) / np.sqrt(width)
+    Wout = rng.standard_normal((N * C, width)) / np.sqrt(width)
+    alpha = np.linspace(0.3, 1.5, C)
+    return [w.astype(np.float32) for w in (W1, W2, W3, Wout, alpha)]
+
+
+@pytest.mark.parametrize("N,C,Z,H,W,K", [
+    (2, 3, 4, 8, 16, 8), (1, 2, 16, 16, 16, 10), (2, 40, 8, 8, 8, 8), (2, 8, 64, 64, 64, 8),
+    (1, 3, 3, 5, 7, 2), (3, 30, 16, 32, 16, 0),
+])
+def test_filter_gen_3d_matches_oracle(hy, N, C, Z, H, W, K):
+    rng = np.random.default_rng(Z * 7 + H * 3 + W + K)
+    w = ffn_3d(rng, N, C, K)
+    got = host(hy.hyena_filter_gen_3d(*[dev(a) for a in w], N, C, Z, H, W, n_bands=K))
+    ref = oracle.filter_gen_3d(*w, N, C, Z, H, W, n_bands=K)
+    assert np.max(np.abs(got - ref)) <= 2e-5 * np.max(np.abs(ref))
+
+
+def test_forward_3d_with_generated_filters(hy):
+    # the 3-D step: filters from the network, their spectra, the forward
+    B, C, Z, H, W, N = 2, 3, 16, 16, 32, 2
+    rng = np.random.default_rng(12)
+    w = ffn_3d(rng, N, C, 8)
+    v, x, b, _ = problem_3d(B, C, Z, H, W, N, seed=13)
+    h = hy.hyena_filter_gen_3d(*[dev(a) for a in w], N, C, Z, H, W)
+    y = host(hy.hyena_fftconv3d_gate_forward(dev(v), [dev(xx) for xx in x], dev(b), Hs=hy.hyena_filter_rfft3d(h)))
+    href = oracle.filter_gen_3d(*w, N, C, Z, H, W)
+    ref = oracle.hyena_forward_3d(v.astype(np.float64), np.stack(x).astype(np.float64), href, b.astype(np.float64))
+    assert_close(y, ref, "f32", "3-D generated filters")
