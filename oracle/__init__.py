@@ -69,6 +69,7 @@ def _load():
         "oracle_hyena_forward_circular": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
         "oracle_cconv3": [dp, dp, l, l, l, i, dp],
         "oracle_filter_gen_3d": [dp, dp, dp, dp, dp, i, i, i, i, i, i, i, d, i, dp],
+        "oracle_filter_gen_film_3d": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, i, i, d, i, dp],
         "oracle_hyena_backward_2d": [dp, dp, dp, dp, dp, l, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_hyena_forward_circular_nd": [dp, dp, dp, dp, l, l, l, l, l, l, i, dp],
     }
@@ -395,4 +396,27 @@ def filter_gen_3d(W1, W2, W3, Wout, alpha, N, C, Z, H, W, n_bands=8, width=64, d
                                       n_bands, width, float(decay_div), threads or default_threads(), _ptr(h))
     _check(rc, "oracle_filter_gen_3d")
     return h
+
+
+def filter_gen_film_3d(W1, W2, W3, Wout, omega, gamma, beta, window, gaussian, N, C, Z, H, W, n_bands=8,
+                       width=64, decay_div=64.0, threads=None) -> np.ndarray:
+    """Per-sample 3-D filters h [B][N][C][Z][H][W]: the FiLM-modulated sine
+    layers on the 3-D features; window [C] is alpha (separable exponential
+    decay) or sigma (Gaussian exp(-(tz^2 + ty^2 + tx^2) / (2 sigma^2)))."""
+    W1, W2, W3, Wout, omega, gamma, beta, window = map(_f64, (W1, W2, W3, Wout, omega, gamma, beta, window))
+    B = gamma.shape[0]
+    h = np.empty((B, N, C, Z, H, W))
+    rc = _load().oracle_filter_gen_film_3d(_ptr(W1), _ptr(W2), _ptr(W3), _ptr(Wout), _ptr(omega), _ptr(gamma),
+                                           _ptr(beta), _ptr(window), int(bool(gaussian)), B, N, C, Z, H, W,
+                                           n_bands, width, float(decay_div), threads or default_threads(),
+                                           _ptr(h))
+    _check(rc, "oracle_filter_gen_film_3d")
+    return h
+
+
+def hyena_forward_3d_per_sample(v, x, h, bias, route="fft") -> np.ndarray:
+    """The 3-D forward with a filter set per sample, h [B][N][C][Z][H][W]."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    return np.concatenate([hyena_forward_3d(v[b:b + 1], x[:, b:b + 1], h[b], bias, route)
+                           for b in range(v.shape[0])])
 

@@ -1576,3 +1576,93 @@ int oracle_filter_gen_3d(const double *W1, const double *W2, const double *W3, c
     free(jobs); free(tid);
     return st;
 }
+
+/* Input-dependent 3-D filters: the FiLM-modulated sine layers of
+ * oracle_filter_gen_film on the 3-D features of oracle_filter_gen_3d,
+ * h[B][N][C][Z][H][W]; the window is the separable exponential decay of
+ * oracle_filter_gen_3d (gaussian = 0, win = alpha) or the Gaussian
+ * exp(-(tz^2 + ty^2 + tx^2) / (2 sigma_c^2)) (gaussian = 1, win = sigma). */
+typedef struct {
+    const double *W1, *W2, *W3, *Wout, *omega, *gamma, *beta, *win;
+    int gaussian, B, N, C, Z, H, W, n_bands, width;
+    double decay_div;
+    double *h;
+    long p0, p1;
+    int status;
+} fgf3_job;
+
+static void *filter_gen_film_3d_worker(void *arg)
+{
+    fgf3_job *j = (fgf3_job *)arg;
+    const int K = j->n_bands, n_in = 3 + 6 * K, w = j->width, n_out = j->N * j->C;
+    const long V = (long)j->Z * j->H * j->W;
+    double *phi = malloc(sizeof(double) * n_in);
+    double *a1 = malloc(sizeof(double) * w), *a2 = malloc(sizeof(double) * w);
+    double *a3 = malloc(sizeof(double) * w), *o = malloc(sizeof(double) * n_out);
+    if (!phi || !a1 || !a2 || !a3 || !o) {
+        j->status = ORACLE_ENOMEM;
+        goto done;
+    }
+    for (int b = 0; b < j->B; ++b) {
+        const double *g = j->gamma + (long)b * 3 * w, *be = j->beta + (long)b * 3 * w;
+        for (long p = j->p0; p < j->p1; ++p) {
+            const long iz = p / ((long)j->H * j->W), iy = (p / j->W) % j->H, ix = p % j->W;
+            const double t[3] = {(double)iz / j->Z, (double)iy / j->H, (double)ix / j->W};
+            for (int a = 0; a < 3; ++a) {
+                phi[a] = t[a];
+                for (int k = 1; k <= K; ++k) {
+                    phi[3 + 2 * K * a + 2 * (k - 1)] = sin(2.0 * ORACLE_PI * k * t[a]);
+                    phi[3 + 2 * K * a + 2 * (k - 1) + 1] = cos(2.0 * ORACLE_PI * k * t[a]);
+                }
+            }
+            matvec(j->W1, w, n_in, phi, a1);
+            film_sin(a1, w, j->omega, g, be);
+            matvec(j->W2, w, w, a1, a2);
+            film_sin(a2, w, j->omega + w, g + w, be + w);
+            matvec(j->W3, w, w, a2, a3);
+            film_sin(a3, w, j->omega + 2 * w, g + 2 * w, be + 2 * w);
+            matvec(j->Wout, n_out, w, a3, o);
+            for (int n = 0; n < j->N; ++n)
+                for (int c = 0; c < j->C; ++c) {
+                    const double s = j->win[c];
+                    const double window =
+                        j->gaussian ? exp(-(t[0] * t[0] + t[1] * t[1] + t[2] * t[2]) / (2.0 * s * s))
+                                    : exp(-s * (double)(iz + iy + ix) / j->decay_div);
+                    j->h[(((long)b * j->N + n) * j->C + c) * V + p] = o[n * j->C + c] * window;
+                }
+        }
+    }
+    j->status = ORACLE_OK;
+done:
+    free(phi); free(a1); free(a2); free(a3); free(o);
+    return NULL;
+}
+
+int oracle_filter_gen_film_3d(const double *W1, const double *W2, const double *W3, const double *Wout,
+                              const double *omega, const double *gamma, const double *beta, const double *win,
+                              int gaussian, int B, int N, int C, int Z, int H, int W, int n_bands, int width,
+                              double decay_div, int nthreads, double *h)
+{
+    if (!W1 || !W2 || !W3 || !Wout || !omega || !gamma || !beta || !win || !h || B < 1 || N < 1 || C < 1 ||
+        Z < 1 || H < 1 || W < 1 || n_bands < 0 || width < 1 || !(decay_div > 0.0))
+        return ORACLE_EBADARG;
+    const long V = (long)Z * H * W;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > V) nthreads = (int)V;
+    fgf3_job *jobs = calloc(nthreads, sizeof(fgf3_job));
+    pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
+    if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
+    for (int k = 0; k < nthreads; ++k) {
+        fgf3_job jb = {W1, W2, W3, Wout, omega, gamma, beta, win, gaussian, B, N, C, Z, H, W, n_bands, width,
+                       decay_div, h, V * k / nthreads, V * (k + 1) / nthreads, 0};
+        jobs[k] = jb;
+        pthread_create(&tid[k], NULL, filter_gen_film_3d_worker, &jobs[k]);
+    }
+    int st = ORACLE_OK;
+    for (int k = 0; k < nthreads; ++k) {
+        pthread_join(tid[k], NULL);
+        if (jobs[k].status != ORACLE_OK) st = jobs[k].status;
+    }
+    free(jobs); free(tid);
+    return st;
+}

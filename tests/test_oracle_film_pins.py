@@ -163,3 +163,72 @@ def test_2d_per_sample_forward_with_shared_filters_is_the_forward():
     h, bias = r.standard_normal((N, D, 8, 8)) * 0.3, r.standard_normal((N, D))
     hp = np.broadcast_to(h, (B, N, D, 8, 8))
     assert np.array_equal(oracle.hyena_forward_2d_per_sample(v, x, hp, bias), oracle.hyena_forward_2d(v, x, h, bias))
+
+
+# ------------------------------------------------------------------ 3-D
+
+Z3, H3, W3_ = 4, 6, 8
+
+
+def film3(n, omega, gamma, beta, window, gaussian=False):
+    return oracle.filter_gen_film_3d(n["W1"], n["W2"], n["W3"], n["Wout"], omega, gamma, beta, window,
+                                     gaussian, N, D, Z3, H3, W3_, n_bands=4)
+
+
+def net3(seed=0):
+    r = np.random.default_rng(seed)
+    n_in = 3 + 6 * 4
+    return dict(W1=r.standard_normal((W, n_in)) / np.sqrt(n_in), W2=r.standard_normal((W, W)) / 8,
+                W3=r.standard_normal((W, W)) / 8, Wout=r.standard_normal((N * D, W)) / 8)
+
+
+def test_3d_identity_modulation_is_the_shared_filter():
+    n = net3()
+    B = 2
+    h = film3(n, np.ones((3, W)), np.ones((B, 3, W)), np.zeros((B, 3, W)), ALPHA)
+    ref = oracle.filter_gen_3d(n["W1"], n["W2"], n["W3"], n["Wout"], ALPHA, N, D, Z3, H3, W3_, n_bands=4)
+    for b in range(B):
+        assert np.array_equal(h[b], ref)
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_3d_beta_pi_flips_the_sign(layer):
+    n = net3(1)
+    be = np.zeros((1, 3, W))
+    be[0, layer] = np.pi
+    a = film3(n, np.ones((3, W)), np.ones((1, 3, W)), be, ALPHA)
+    b = film3(n, np.ones((3, W)), np.ones((1, 3, W)), np.zeros((1, 3, W)), ALPHA)
+    assert np.max(np.abs(a + b)) < 1e-12 * np.max(np.abs(b))
+
+
+def test_3d_gaussian_window_ratio():
+    n = net3(2)
+    sigma = np.array([0.1, 0.3, 0.7])
+    r = np.random.default_rng(4)
+    g, be = r.uniform(0.5, 1.5, (1, 3, W)), r.normal(0, 0.3, (1, 3, W))
+    hg = film3(n, np.ones((3, W)), g, be, sigma, gaussian=True)
+    he = film3(n, np.ones((3, W)), g, be, ALPHA)
+    iz, iy, ix = np.meshgrid(np.arange(Z3), np.arange(H3), np.arange(W3_), indexing="ij")
+    t2 = (iz / Z3) ** 2 + (iy / H3) ** 2 + (ix / W3_) ** 2
+    gauss = np.exp(-t2[None] / (2 * sigma[:, None, None, None] ** 2))
+    expo = np.exp(-ALPHA[:, None, None, None] * (iz + iy + ix)[None] / 64.0)
+    np.testing.assert_allclose(hg[0], he[0] * (gauss / expo)[None], rtol=1e-12, atol=1e-300)
+
+
+def test_3d_samples_do_not_mix():
+    n = net3(3)
+    r = np.random.default_rng(5)
+    g, be = r.uniform(0.5, 1.5, (3, 3, W)), r.normal(0, 0.3, (3, 3, W))
+    om = r.uniform(0.5, 2.0, (3, W))
+    h = film3(n, om, g, be, ALPHA)
+    for b in range(3):
+        assert np.array_equal(h[b], film3(n, om, g[b:b + 1], be[b:b + 1], ALPHA)[0])
+
+
+def test_3d_per_sample_forward_with_shared_filters_is_the_forward():
+    r = np.random.default_rng(10)
+    B = 2
+    v, x = r.standard_normal((B, D, 4, 4, 8)), r.standard_normal((N, B, D, 4, 4, 8))
+    h, bias = r.standard_normal((N, D, 4, 4, 8)) * 0.3, r.standard_normal((N, D))
+    hp = np.broadcast_to(h, (B, N, D, 4, 4, 8))
+    assert np.array_equal(oracle.hyena_forward_3d_per_sample(v, x, hp, bias), oracle.hyena_forward_3d(v, x, h, bias))
