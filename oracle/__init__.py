@@ -69,6 +69,7 @@ def _load():
         "oracle_hyena_forward_circular": [dp, dp, dp, dp, l, l, l, l, i, i, dp],
         "oracle_cconv3": [dp, dp, l, l, l, i, dp],
         "oracle_filter_gen_3d": [dp, dp, dp, dp, dp, i, i, i, i, i, i, i, d, i, dp],
+        "oracle_hyena_backward_circular": [dp, dp, dp, dp, dp, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_filter_gen_film_3d": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, i, i, d, i, dp],
         "oracle_hyena_backward_2d": [dp, dp, dp, dp, dp, l, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_hyena_forward_circular_nd": [dp, dp, dp, dp, l, l, l, l, l, l, i, dp],
@@ -233,6 +234,39 @@ def hyena_backward(v, x, h, bias, dy, route="fft", threads=None):
                                        B, D, L, N, _route(route), threads or default_threads(),
                                        _ptr(dv), _ptr(dx), _ptr(dh), _ptr(db))
     _check(rc, "oracle_hyena_backward")
+    return dv, dx, dh, db
+
+
+def hyena_backward_circular(v, x, h, bias, dy, route="fft", threads=None):
+    """Gradients through :func:`hyena_forward_circular` (circular
+    convolutions of length L): (dv, dx, dh [N][D][L], dbias [N][D]), dh and
+    dbias summed over the batch."""
+    v, x, h, bias, dy = map(_f64, (v, x, h, bias, dy))
+    B, D, L = v.shape
+    N = h.shape[0]
+    assert x.shape == (N, B, D, L) and h.shape == (N, D, L) and bias.shape == (N, D)
+    assert dy.shape == v.shape
+    dv, dx, dh, db = np.empty_like(v), np.empty_like(x), np.empty_like(h), np.empty_like(bias)
+    rc = _load().oracle_hyena_backward_circular(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), _ptr(dy),
+                                                B, D, L, N, _route(route), threads or default_threads(),
+                                                _ptr(dv), _ptr(dx), _ptr(dh), _ptr(db))
+    _check(rc, "oracle_hyena_backward_circular")
+    return dv, dx, dh, db
+
+
+def hyena_backward_per_sample(v, x, h, bias, dy, route="fft", threads=None):
+    """The gradients through :func:`hyena_forward_per_sample` (a filter set
+    per sample, h [B][N][D][L]): each sample's adjoint by
+    :func:`hyena_backward` with its own filters.  Returns (dv, dx, dh
+    [B][N][D][L] per sample, dbias [N][D] summed over the samples, as the
+    bias is shared)."""
+    v, x, h, bias, dy = map(_f64, (v, x, h, bias, dy))
+    parts = [hyena_backward(v[b:b + 1], x[:, b:b + 1], h[b], bias, dy[b:b + 1], route, threads)
+             for b in range(v.shape[0])]
+    dv = np.concatenate([p[0] for p in parts])
+    dx = np.concatenate([p[1] for p in parts], axis=1)
+    dh = np.stack([p[2] for p in parts])
+    db = np.sum([p[3] for p in parts], axis=0)
     return dv, dx, dh, db
 
 

@@ -861,6 +861,21 @@ static void corr_fft(const double *a, const double *b, long L, double *out,
     for (long t = 0; t < L; ++t) out[t] = s->ur[t] / (double)P;
 }
 
+/* Circular counterpart of both sums above (length-L circular convolution,
+ * "Handling Boundaries": periodic systems): out[s] = sum_t a[t] b[(t - s)
+ * mod L], s = 0..L-1.  With a = e, b = z it is dh; with a = e, b = h the
+ * adjoint of the circular convolution with respect to its signal.  Its FFT
+ * route is corr_fft with scratch of exactly L points (no padding, so the
+ * product of spectra wraps around). */
+static void ccorr_direct(const double *a, const double *b, long L, double *out)
+{
+    for (long s = 0; s < L; ++s) {
+        double acc = 0.0;
+        for (long t = 0; t < L; ++t) acc += a[t] * b[((t - s) % L + L) % L];
+        out[s] = acc;
+    }
+}
+
 typedef struct {
     const double *v, *x, *h, *bias, *dy;
     long B, D, L, N;
@@ -868,6 +883,7 @@ typedef struct {
     double *dv, *dx, *dh, *dbias;
     long d0, step; /* channels d0, d0 + step, ... (dh, db summed over b here) */
     int status;
+    int circular;  /* 1: the recurrence with circular convolutions of length L */
 } bwd_job;
 
 static void *backward_worker(void *arg)
@@ -880,7 +896,7 @@ static void *backward_worker(void *arg)
     double *tmp = malloc(sizeof(double) * L);
     fft_scratch s = {0};
     if (!z || !c || !g || !e || !tmp ||
-        (j->route == ROUTE_FFT && scratch_alloc(&s, next_pow2(2 * L)) != ORACLE_OK)) {
+        (j->route == ROUTE_FFT && scratch_alloc(&s, j->circular ? L : next_pow2(2 * L)) != ORACLE_OK)) {
         j->status = ORACLE_ENOMEM;
         goto done;
     }
@@ -898,8 +914,13 @@ static void *backward_worker(void *arg)
                 const double *xn = j->x + n * BDL + seq * L;
                 const double bn = j->bias[n * D + d];
                 double *zn = z + n * L, *cn = c + n * L;
-                if (j->route == ROUTE_DIRECT) conv_direct(hn, zn, L, cn);
-                else conv_fft(hn, zn, L, cn, &s);
+                if (j->circular) {
+                    if (j->route == ROUTE_DIRECT) cconv_direct(hn, zn, L, cn);
+                    else cconv_fft(hn, zn, L, cn, &s);
+                } else {
+                    if (j->route == ROUTE_DIRECT) conv_direct(hn, zn, L, cn);
+                    else conv_fft(hn, zn, L, cn, &s);
+                }
                 for (long t = 0; t < L; ++t) cn[t] += bn * zn[t];
                 if (n + 1 < N)
                     for (long t = 0; t < L; ++t) z[(n + 1) * L + t] = xn[t] * cn[t];
@@ -917,14 +938,16 @@ static void *backward_worker(void *arg)
                     dxn[t] = g[t] * cn[t];
                     e[t] = g[t] * xn[t];
                 }
-                if (j->route == ROUTE_DIRECT) lagged_direct(e, zn, L, tmp);
-                else corr_fft(e, zn, L, tmp, &s);
+                if (j->route == ROUTE_FFT) corr_fft(e, zn, L, tmp, &s);
+                else if (j->circular) ccorr_direct(e, zn, L, tmp);
+                else lagged_direct(e, zn, L, tmp);
                 for (long t = 0; t < L; ++t) dhn[t] += tmp[t];
                 double db = 0.0;
                 for (long t = 0; t < L; ++t) db += e[t] * zn[t];
                 j->dbias[n * D + d] += db;
-                if (j->route == ROUTE_DIRECT) corr_direct(hn, e, L, tmp);
-                else corr_fft(e, hn, L, tmp, &s);
+                if (j->route == ROUTE_FFT) corr_fft(e, hn, L, tmp, &s);
+                else if (j->circular) ccorr_direct(e, hn, L, tmp);
+                else corr_direct(hn, e, L, tmp);
                 for (long t = 0; t < L; ++t) g[t] = tmp[t] + bn * e[t];
             }
             memcpy(j->dv + seq * L, g, sizeof(double) * L); /* dv = dz_0 */
@@ -940,10 +963,34 @@ done:
 /* Gradients of a scalar loss with dL/dy = dy [B][D][L]: dv [B][D][L],
  * dx [N][B][D][L], dh [N][D][L] and dbias [N][D] (both summed over the
  * batch).  Inputs as oracle_hyena_forward. */
+static int backward_any(const double *v, const double *x, const double *h, const double *bias,
+                        const double *dy, long B, long D, long L, long N, int route, int nthreads,
+                        int circular, double *dv, double *dx, double *dh, double *dbias);
+
 int oracle_hyena_backward(const double *v, const double *x, const double *h,
                           const double *bias, const double *dy, long B, long D,
                           long L, long N, int route, int nthreads, double *dv,
                           double *dx, double *dh, double *dbias)
+{
+    return backward_any(v, x, h, bias, dy, B, D, L, N, route, nthreads, 0, dv, dx, dh, dbias);
+}
+
+/* The same gradients through the recurrence with circular convolutions of
+ * length L (oracle_hyena_forward_circular): dh_n[s] = sum_b sum_t e[t]
+ * z_{n-1}[(t - s) mod L], dz_{n-1}[u] = sum_t h_n[(t - u) mod L] e[t] +
+ * b_n e[u].  L a power of two for the FFT route. */
+int oracle_hyena_backward_circular(const double *v, const double *x, const double *h,
+                                   const double *bias, const double *dy, long B, long D,
+                                   long L, long N, int route, int nthreads, double *dv,
+                                   double *dx, double *dh, double *dbias)
+{
+    if (route == ROUTE_FFT && !is_pow2(L)) return ORACLE_EBADARG;
+    return backward_any(v, x, h, bias, dy, B, D, L, N, route, nthreads, 1, dv, dx, dh, dbias);
+}
+
+static int backward_any(const double *v, const double *x, const double *h, const double *bias,
+                        const double *dy, long B, long D, long L, long N, int route, int nthreads,
+                        int circular, double *dv, double *dx, double *dh, double *dbias)
 {
     if (!v || !x || !h || !bias || !dy || !dv || !dx || !dh || !dbias || B < 1 ||
         D < 1 || L < 1 || N < 1 || (route != ROUTE_DIRECT && route != ROUTE_FFT))
@@ -954,7 +1001,7 @@ int oracle_hyena_backward(const double *v, const double *x, const double *h,
     pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
     if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
     for (int k = 0; k < nthreads; ++k) {
-        bwd_job j = {v, x, h, bias, dy, B, D, L, N, route, dv, dx, dh, dbias, k, nthreads, 0};
+        bwd_job j = {v, x, h, bias, dy, B, D, L, N, route, dv, dx, dh, dbias, k, nthreads, 0, circular};
         jobs[k] = j;
         pthread_create(&tid[k], NULL, backward_worker, &jobs[k]);
     }

@@ -160,3 +160,92 @@ def test_backward_2d_routes_agree_and_db_is_dh_origin(route):
     for g_, w_ in zip(got, ref):
         assert rel_err(g_, w_) < 1e-12
     assert rel_err(got[3], got[2][:, :, 0, 0]) < 1e-12
+
+
+# ------------------------------------------------- per-sample filters
+
+def test_backward_per_sample_matches_finite_differences():
+    # a filter set per sample: every gradient against a central difference
+    # of the per-sample oracle forward; dh must be per sample (a sum over
+    # the batch, or another sample's filters, fails), dbias summed
+    B, D, L, N = 3, 2, 6, 2
+    r = np.random.default_rng(21)
+    v, x = r.standard_normal((B, D, L)), r.standard_normal((N, B, D, L))
+    h = r.standard_normal((B, N, D, L)) * np.exp(-np.arange(L) / 4.0)
+    b, dy = r.standard_normal((N, D)), r.standard_normal((B, D, L))
+    dv, dx, dh, db = oracle.hyena_backward_per_sample(v, x, h, b, dy, route="direct")
+    assert dh.shape == h.shape and db.shape == b.shape
+
+    def loss(v_, x_, h_, b_):
+        return float(np.sum(dy * oracle.hyena_forward_per_sample(v_, x_, h_, b_, route="direct")))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name
+
+
+def test_backward_per_sample_with_equal_sets_sums_to_the_shared_backward():
+    B, D, L, N = 3, 4, 32, 2
+    v, x, h, b, dy = problem(B, D, L, N, seed=22)
+    dv, dx, dh, db = oracle.hyena_backward(v, x, h, b, dy)
+    pv, px, ph, pb = oracle.hyena_backward_per_sample(v, x, np.broadcast_to(h, (B,) + h.shape), b, dy)
+    assert rel_err(pv, dv) < 1e-13 and rel_err(px, dx) < 1e-13
+    assert rel_err(ph.sum(axis=0), dh) < 1e-12 and rel_err(pb, db) < 1e-12
+    # and each sample's dh is that sample's own shared-filter backward
+    for s in range(B):
+        one = oracle.hyena_backward(v[s:s + 1], x[:, s:s + 1], h, b, dy[s:s + 1])
+        assert rel_err(ph[s], one[2]) < 1e-13
+
+
+# ------------------------------------------------- circular convolution
+
+@pytest.mark.parametrize("N", [1, 2])
+def test_backward_circular_matches_finite_differences(N):
+    v, x, h, b, dy = problem(2, 2, 8, N, seed=30 + N)
+    dv, dx, dh, db = oracle.hyena_backward_circular(v, x, h, b, dy, route="direct")
+
+    def loss(v_, x_, h_, b_):
+        return float(np.sum(dy * oracle.hyena_forward_circular(v_, x_, h_, b_, route="direct")))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name
+
+
+def test_backward_circular_routes_agree_and_db_is_dh_lag0():
+    v, x, h, b, dy = problem(3, 4, 64, 3, seed=33)
+    d = oracle.hyena_backward_circular(v, x, h, b, dy, route="direct")
+    f = oracle.hyena_backward_circular(v, x, h, b, dy, route="fft")
+    for a, c in zip(d, f):
+        assert rel_err(c, a) < 1e-12
+    assert rel_err(d[3], d[2][:, :, 0]) < 1e-13
+
+
+def test_backward_circular_on_zero_padded_sequences_is_the_causal_backward():
+    # length 2L with v, x_n, dy and h_n zero beyond L: no product wraps
+    # around, so every gradient's first L entries are the causal ones
+    B, D, L, N = 2, 3, 16, 2
+    v, x, h, b, dy = problem(B, D, L, N, seed=34)
+    pad = lambda a: np.concatenate([a, np.zeros_like(a)], axis=-1)
+    dv, dx, dh, db = oracle.hyena_backward_circular(pad(v), pad(x), pad(h), b, pad(dy))
+    rv, rx, rh, rb = oracle.hyena_backward(v, x, h, b, dy)
+    assert rel_err(dv[..., :L], rv) < 1e-12 and rel_err(dx[..., :L], rx) < 1e-12
+    assert rel_err(dh[..., :L], rh) < 1e-12 and rel_err(db, rb) < 1e-12
