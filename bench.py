@@ -52,12 +52,18 @@ def describe(wl: synth.Workload) -> dict:
 
 def _describe(wl: synth.Workload) -> dict:
     if wl.kind == "3d":
+        filters = (f"implicit FFN over (z/Z, y/H, x/W) (3 sine layers of width {synth.WIDTH}, "
+                   f"{synth.N_BANDS} bands per axis) x separable decay, regenerated every step")
+        if wl.film:
+            filters = (f"input-dependent: a filter set per sample, the {synth.WIDTH}-wide sine layers over "
+                       f"(z/Z, y/H, x/W) ({synth.N_BANDS} bands per axis) FiLM-modulated per sample, first "
+                       "layer at frequencies 1/2/4/8, Gaussian window; B*N*C filters and spectra "
+                       "regenerated every step")
         return {"workload": f"{wl.name}: order-{wl.N} Hyena 3-D operator, B={wl.B}, C={wl.D}, "
                             f"{wl.Z}x{wl.H}x{wl.W} volumes (padded to {2 * wl.Z}x{2 * wl.H}x{2 * wl.W}), "
                             f"{wl.io} storage, fp32 compute",
                 "N": wl.N, "B": wl.B, "C": wl.D, "Z": wl.Z, "H": wl.H, "W": wl.W, "io": wl.io,
-                "filters": f"implicit FFN over (z/Z, y/H, x/W) (3 sine layers of width {synth.WIDTH}, "
-                           f"{synth.N_BANDS} bands per axis) x separable decay, regenerated every step",
+                "filters": filters,
                 "l2": "flushed (256 MB write) before every timed step"}
     if wl.kind == "2d":
         return {"workload": f"{wl.name}: order-{wl.N} Hyena 2-D operator, B={wl.B}, C={wl.D}, "
@@ -85,11 +91,11 @@ def alg_bytes_forward(wl: synth.Workload) -> int:
     act = (wl.N + 2) * wl.positions * wl.io_bytes
     if wl.circular:                        # spectra of the grid itself: half a slot per position
         return act + wl.N * wl.D * wl.per_channel // 2 * 8
-    if wl.kind == "3d":
-        return act + wl.N * wl.D * 4 * wl.Z * wl.H * wl.W * 8
-    if wl.kind == "2d":
-        return act + wl.N * wl.D * 2 * wl.H * wl.W * 8
     sets = wl.B if wl.film else 1          # filter spectra per sample, or shared by the batch
+    if wl.kind == "3d":
+        return act + sets * wl.N * wl.D * 4 * wl.Z * wl.H * wl.W * 8
+    if wl.kind == "2d":
+        return act + sets * wl.N * wl.D * 2 * wl.H * wl.W * 8
     return act + sets * wl.N * wl.D * wl.L * 8
 
 
@@ -99,6 +105,10 @@ def alg_bytes_backward(wl: synth.Workload) -> int:
     dbias out (float32)."""
     io = 2 if wl.io == "bf16" else 4
     act = wl.positions * io
+    if wl.film:             # spectra in and dh out per sample
+        return (2 * wl.N + 3) * act + wl.B * wl.N * wl.D * wl.L * (8 + 4) + wl.N * wl.D * 4
+    if wl.circular:         # L/2 spectrum slots a filter, L lags of dh
+        return (2 * wl.N + 3) * act + wl.N * wl.D * wl.L * (4 + 4) + wl.N * wl.D * 4
     if wl.kind == "2d":     # 2H x W spectrum slots a filter, H x W of dh
         return (2 * wl.N + 3) * act + wl.N * wl.D * wl.H * wl.W * (16 + 4) + wl.N * wl.D * 4
     return (2 * wl.N + 3) * act + wl.N * wl.D * wl.L * (8 + 4) + wl.N * wl.D * 4
@@ -370,6 +380,23 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
                                    decay_div=synth.DECAY_DIV, out=h)
             hyena.hyena_filter_rfft_circular(h, out=H)
             forward()
+    elif wl.kind == "3d" and wl.film:
+        F = [to_dev(inp[k]) for k in ("omega", "gamma", "beta", "sigma")]
+        h = torch.empty((wl.B, wl.N, wl.D, wl.Z, wl.H, wl.W), device="cuda", dtype=torch.float32)
+        H = torch.empty((wl.B, wl.N, wl.D, 2 * wl.Z, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
+        ws_n = hyena.hyena_fftconv3d_workspace_size(wl.B, wl.D, wl.Z, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
+        ws_fwd = torch.empty(ws_n, device="cuda", dtype=torch.uint8)
+
+        def forward():
+            hyena.hyena_fftconv3d_gate_forward_per_sample(v, xs, b, H, out=y, workspace=ws_fwd)
+
+        def step():
+            hyena.hyena_filter_gen_film_3d(*W, wl.N, wl.D, wl.Z, wl.H, wl.W, B=wl.B, omega=F[0], gamma=F[1],
+                                           beta=F[2], sigma=F[3], n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                           decay_div=synth.DECAY_DIV, out=h)
+            hyena.hyena_filter_rfft3d(h.view(wl.B * wl.N, wl.D, wl.Z, wl.H, wl.W),
+                                      out=H.view(wl.B * wl.N, wl.D, 2 * wl.Z, 2 * wl.H, wl.W))
+            forward()
     elif wl.kind == "3d":
         h = torch.empty((wl.N, wl.D, wl.Z, wl.H, wl.W), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.N, wl.D, 2 * wl.Z, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
@@ -515,9 +542,24 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
 
     # ---- the backward pass (1-D and 2-D): one call per timed repetition
     bwd = None
-    if (wl.kind == "1d" and not wl.film and not wl.circular) or (wl.kind == "2d" and not wl.circular):
+    if ((wl.kind == "1d" and not (wl.film and long_path(wl)))
+            or (wl.kind == "2d" and not wl.circular and not wl.film)):
         dy = to_dev(synth.make_output_grad(wl), io)
-        if wl.kind == "2d":
+        if wl.circular:
+            ws_b = torch.empty(hyena.hyena_fftconv_backward_circular_workspace_size(wl.D, wl.L, wl.N),
+                               device="cuda", dtype=torch.uint8)
+            bwd_kernel = "backward1d_kernel<PAD=false> (hyena_fftconv_gate_backward_circular)"
+
+            def backward():
+                hyena.hyena_fftconv_gate_backward_circular(v, xs, b, H, dy, workspace=ws_b)
+        elif wl.film:
+            ws_b = torch.empty(hyena.hyena_fftconv_backward_per_sample_workspace_size(wl.B, wl.D, wl.L, wl.N),
+                               device="cuda", dtype=torch.uint8)
+            bwd_kernel = "backward1d_kernel<PS> (hyena_fftconv_gate_backward_per_sample)"
+
+            def backward():
+                hyena.hyena_fftconv_gate_backward_per_sample(v, xs, b, H, dy, workspace=ws_b)
+        elif wl.kind == "2d":
             ws_b = torch.empty(hyena.hyena_fftconv2d_backward_workspace_size(wl.B, wl.D, wl.H, wl.W, wl.N),
                                device="cuda", dtype=torch.uint8)
             bwd_kernel = "fft2d_bwd_row_kernel+fft2d_bwd_col_kernel (hyena_fftconv2d_gate_backward, all launches)"
@@ -593,6 +635,13 @@ def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: 
     v = inp["v"][:, channels].astype(np.float64)
     x = np.stack([xx[:, channels] for xx in inp["x"]]).astype(np.float64)
     bias = inp["b"][:, channels].astype(np.float64)
+    if wl.kind == "3d" and wl.film:
+        h = oracle.filter_gen_film_3d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["omega"],
+                                      inp["gamma"], inp["beta"], inp["sigma"][channels], True, wl.N,
+                                      len(channels), wl.Z, wl.H, wl.W, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                      decay_div=synth.DECAY_DIV, threads=threads)
+        oracle.hyena_forward_3d_per_sample(v, x, h, bias, route="fft")
+        return time.perf_counter() - t0
     if wl.kind == "3d":
         h = oracle.filter_gen_3d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],
                                  wl.N, len(channels), wl.Z, wl.H, wl.W, n_bands=synth.N_BANDS, width=synth.WIDTH,

@@ -218,6 +218,27 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, cons
                                                              int D, int L, int N, hyena_dtype_t io,
                                                              void* y, void* stream);
 
+/* The backward pass of the circular recurrence (hyena_fftconv_gate_forward_
+ * circular), for training: the exact adjoint with every convolution
+ * circular of length L, so both sums wrap around:
+ *   dx_n = g * c_n,   e = g * x_n,
+ *   dh_n[d][s] = sum_b sum_t e[t] z_{n-1}[(t - s) mod L]   (all L lags),
+ *   db_n[d] = dh_n[d][0],
+ *   dz_{n-1}[u] = sum_t h_n[(t - u) mod L] e[t] + b_n e[u],   dv = dz_0.
+ * Arguments as hyena_fftconv_gate_backward with H [N][D][L/2] from
+ * hyena_filter_rfft_circular; dh [N][D][L] and dbias [N][D] summed over the
+ * batch; workspace of hyena_fftconv_backward_circular_workspace_size(D, L,
+ * N) bytes (12 N D L), 256-byte aligned.  32 <= L <= 16384, a power of two
+ * (the size function returns (size_t)-1 otherwise).  Two launches,
+ * deterministic, as the L <= 16384 backward. */
+HYENA_API size_t hyena_fftconv_backward_circular_workspace_size(int D, int L, int N);
+HYENA_API hyena_status_t hyena_fftconv_gate_backward_circular(const void* v, const void* const* x,
+                                                              const float* H, const float* bias,
+                                                              const void* dy, int B, int D, int L, int N,
+                                                              hyena_dtype_t io, void* dv, void* const* dx,
+                                                              float* dh, float* dbias, void* workspace,
+                                                              size_t ws_bytes, void* stream);
+
 /* Size of the scratch array built into the library for
  * hyena_fftconv_gate_forward_noalloc (16 MB on every device that loads the
  * library, held until the process exits). */
@@ -281,6 +302,29 @@ HYENA_API hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* 
                                                      hyena_dtype_t io, void* dv, void* const* dx,
                                                      float* dh, float* dbias, void* workspace,
                                                      size_t ws_bytes, void* stream);
+
+/* The backward pass with a spectrum set per sample (input-dependent
+ * filters, see hyena_filter_gen_film and
+ * hyena_fftconv_gate_forward_per_sample), for training: the same adjoint
+ * with sequence (b, d) using sample b's filters, so
+ *   H      [B][N][D][L] packed complex64 (sample b's set at H + b*N*D*L)
+ *   dh     [B][N][D][L] float32 out, per sample (no sum over the batch):
+ *          dh_n[b][d][s] = sum_t e[t] z_{n-1}[t-s] of sequence (b, d)
+ *   dbias  [N][D] float32 out, summed over the batch (the bias is shared)
+ *   workspace: hyena_fftconv_backward_per_sample_workspace_size(B, D, L, N)
+ *          bytes (8 B N D L + 12 N D L), 256-byte aligned.
+ * Everything else as hyena_fftconv_gate_backward.  L <= 16384 (else
+ * HYENA_ERR_UNSUPPORTED; the size function returns (size_t)-1).  Two
+ * launches, deterministic: a group of threads per channel walks its B
+ * sequences, each with its own dh spectrum; the second launch inverts the
+ * B spectra of each (n, d) and sums their lag-0 values into dbias. */
+HYENA_API size_t hyena_fftconv_backward_per_sample_workspace_size(int B, int D, int L, int N);
+HYENA_API hyena_status_t hyena_fftconv_gate_backward_per_sample(const void* v, const void* const* x,
+                                                                const float* H, const float* bias,
+                                                                const void* dy, int B, int D, int L, int N,
+                                                                hyena_dtype_t io, void* dv, void* const* dx,
+                                                                float* dh, float* dbias, void* workspace,
+                                                                size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- 2-D */
 
@@ -360,6 +404,22 @@ HYENA_API hyena_status_t hyena_fftconv2d_gate_forward_per_sample(const void* v, 
 HYENA_API hyena_status_t hyena_filter_gen_3d(const hyena_ffn_t* ffn, int N, int C, int Z, int H, int W,
                                              float* h, void* stream);
 
+/* Input-dependent 3-D filters h [B][N][C][Z][H][W] float32 ("Native
+ * Multi-Dimensional Subquadratic Operators via Input Dependent Long
+ * Convolutions": Input-Dependent Kernels via Registers and FiLM, Kernel
+ * Parameterization, read on 3-D volumes): per sample b the sine layers of
+ * hyena_filter_gen_3d's network are FiLM-modulated as in
+ * hyena_filter_gen_film (film: omega [3][width], gamma and beta
+ * [B][3][width], device pointers, NULL for 1 / 1 / 0).  Window: with
+ * film->sigma [C] the Gaussian exp(-(tz^2 + ty^2 + tx^2) / (2 sigma_c^2)),
+ * t = i / n per axis, else the separable decay of hyena_filter_gen_3d.
+ * n_bands <= 10; B <= 65535.  Their spectra are hyena_filter_rfft3d of the
+ * B*N rows of C filters; the forward is
+ * hyena_fftconv3d_gate_forward_per_sample. */
+HYENA_API hyena_status_t hyena_filter_gen_film_3d(const hyena_ffn_t* ffn, const hyena_film_t* film,
+                                                  int B, int N, int C, int Z, int H, int W, float* h,
+                                                  void* stream);
+
 /* 3-D filter spectra Hs [N][C][2Z][2H][W] complex64, for filters h
  * [N][C][Z][H][W] float32 (offsets 0..Z-1 x 0..H-1 x 0..W-1) zero-padded
  * to 2Z x 2H x 2W ("Native Multi-Dimensional Subquadratic Operators via
@@ -401,6 +461,18 @@ HYENA_API hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void*
                                                       int H, int W, int N, hyena_dtype_t io,
                                                       void* y, void* workspace, size_t ws_bytes,
                                                       void* stream);
+
+/* The 3-D forward with a spectrum set per sample: Hs [B][N][C][2Z][2H][W]
+ * (hyena_filter_rfft3d of per-sample filters, e.g. from
+ * hyena_filter_gen_film_3d), volume (b, c) multiplied by sample b's
+ * spectra of channel c; otherwise as hyena_fftconv3d_gate_forward with the
+ * spectrum given (the same workspace size).  B*N*C*Z*H <= 2^30. */
+HYENA_API hyena_status_t hyena_fftconv3d_gate_forward_per_sample(const void* v, const void* const* x,
+                                                                 const float* Hs, const float* bias,
+                                                                 int B, int C, int Z, int H, int W,
+                                                                 int N, hyena_dtype_t io, void* y,
+                                                                 void* workspace, size_t ws_bytes,
+                                                                 void* stream);
 
 /* ------------------------------------------------------- circular 2-D */
 

@@ -39,38 +39,67 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def _compile(src: str, obj: str, verbose: bool) -> str:
+OBJDIR = os.path.join(PKG, "lib", "_obj")
+
+
+def _obj_paths(src: str) -> tuple[str, str]:
+    base = os.path.join(OBJDIR, os.path.basename(src)[:-3])
+    return base + ".o", base + ".d"
+
+
+def _obj_stale(src: str) -> bool:
+    """An object is rebuilt when it is missing or older than its source, any
+    header its dependency file lists, or this build script."""
+    obj, dep = _obj_paths(src)
+    if not (os.path.exists(obj) and os.path.exists(dep)):
+        return True
+    t = os.path.getmtime(obj)
+    with open(dep) as f:
+        text = f.read().replace("\\\n", " ")
+    paths = text.split(":", 1)[1].split() if ":" in text else []
+    paths += [src, os.path.abspath(__file__)]
+    return any(not os.path.exists(p) or os.path.getmtime(p) > t for p in paths)
+
+
+def _compile(src: str, verbose: bool) -> str:
+    obj, dep = _obj_paths(src)
+    tmp = obj + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-           "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+           "-I", INCLUDE, "-I", CSRC, "-MD", "-MF", dep, "-c", "-o", tmp, src]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{r.stdout}{r.stderr}")
+    os.replace(tmp, obj)
     return r.stdout + r.stderr
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ (one translation unit per kernel
-    family, in parallel) and link them into one shared library, if stale."""
-    if not force and up_to_date():
+    """Compile the .cu files under csrc/ whose objects are stale (one
+    translation unit per kernel family, in parallel; objects and their
+    dependency files kept under lib/_obj) and link them into one shared
+    library, if anything changed."""
+    if not force and not verbose and up_to_date():
         return LIB
     from concurrent.futures import ThreadPoolExecutor
 
-    objdir = os.path.join(PKG, "lib", "_obj")
-    os.makedirs(objdir, exist_ok=True)
+    os.makedirs(OBJDIR, exist_ok=True)
     srcs = sources()
-    objs = [os.path.join(objdir, os.path.basename(s)[:-3] + f".{os.getpid()}.o") for s in srcs]
-    with ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
-        logs = list(ex.map(lambda so: _compile(so[0], so[1], verbose), zip(srcs, objs)))
-    if verbose:
-        print("".join(logs))
-    tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call([nvcc(), *ARCH_FLAGS, "-shared", "-o", tmp, *objs])
-    for o in objs:
-        os.remove(o)
-    os.replace(tmp, LIB)
+    todo = [s for s in srcs if force or verbose or _obj_stale(s)]
+    if todo:
+        with ThreadPoolExecutor(max_workers=min(len(todo), os.cpu_count() or 4)) as ex:
+            logs = list(ex.map(lambda s: _compile(s, verbose), todo))
+        if verbose:
+            print("".join(logs))
+    objs = [_obj_paths(s)[0] for s in srcs]
+    if todo or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([nvcc(), *ARCH_FLAGS, "-shared", "-o", tmp, *objs])
+        os.replace(tmp, LIB)
+    else:
+        os.utime(LIB)
     return LIB
 
 

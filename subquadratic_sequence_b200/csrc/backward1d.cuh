@@ -25,6 +25,16 @@
 // halves the kernel's instruction footprint.  A second launch turns each
 // accumulated spectrum into dh_n (inverse real FFT, first L lags) and
 // db_n = dh_n[0].
+//
+// Per-sample filters (PS, input-dependent filters): sequence (b, d) reads
+// sample b's spectra at H + b H_bstride, and its dh spectrum is its own
+// (acc [B][N][D][L], no sum over the batch), so dh_n is per sample
+// ([B][N][D][L]); the bias is shared, so db_n = sum_b dh_{b,n}[0].
+//
+// Circular mode (PAD = false, "Handling Boundaries": circular convolutions
+// for periodic systems): the same steps on the L-point grid itself (L = 2M
+// reals as M packed points, no padding, nothing cropped), so both sums are
+// circular correlations and dh_n has all L lags.
 #pragma once
 
 #include "fused1d.cuh"
@@ -45,17 +55,20 @@ struct Backward1dArgs {
     float2* wz;                    // workspace [D][N][L]: Z_n in register order
     float2* wc;                    // workspace [D][N][L/2]: c_{n+1} in register order
     int B, D, N;
+    size_t H_bstride;              // per-sample spectra: slots between samples' sets
 };
 
-template <int LOG2M, typename IO>
-__global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS, Fft1d<LOG2M>::MIN_BLOCKS)
+template <int LOG2M, typename IO, bool PS = false, bool PAD = true>
+__global__ void __launch_bounds__(Fft1d<LOG2M, PAD>::THREADS, Fft1d<LOG2M, PAD>::MIN_BLOCKS)
 backward1d_kernel(Backward1dArgs args)
 {
     grid_dependency_begin();
-    using F = Fft1d<LOG2M>;
+    using F = Fft1d<LOG2M, PAD>;
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;
     constexpr int M = F::M, E = F::E, T = F::T, RF = F::P::RF;
+    constexpr int SEQ = F::SEQ;                 // packed pairs per sequence: M/2 (padded), M (circular)
+    constexpr int NIO = PAD ? E / 2 : E;        // io registers per thread
     extern __shared__ __align__(16) float2 smem_dyn[];
 
     const int g = threadIdx.x / T, t = threadIdx.x % T;
@@ -66,9 +79,9 @@ backward1d_kernel(Backward1dArgs args)
     float2* sm = smem_dyn + g * F::SMEM_SEQ;
     float2* stage = smem_dyn + F::G * F::SMEM_SEQ + g * F::STAGE_SEQ;
     float2* wz = args.wz + (size_t)d * N * M;
-    float2* wc = args.wc + (size_t)d * N * (M / 2);
-    // index of io register i among the thread's E/2 io registers
-    auto io_slot = [](int i) { return (i / RF) * (RF / 2) + i % RF; };
+    float2* wc = args.wc + (size_t)d * N * SEQ;
+    // index of io register i among the thread's NIO io registers
+    auto io_slot = [](int i) { return PAD ? (i / RF) * (RF / 2) + i % RF : i; };
     auto pick = [](const void* const* arr, int n) {
         const void* p = arr[0];
 #pragma unroll
@@ -80,8 +93,9 @@ backward1d_kernel(Backward1dArgs args)
     float2 a[E];
     for (int b = 0; b < args.B; ++b) {
         const size_t seq = (size_t)b * D + d;
+        const float2* Hb = PS ? args.H + (size_t)b * args.H_bstride : args.H;
         {
-            const PT* vp = reinterpret_cast<const PT*>(args.v) + seq * (M / 2);
+            const PT* vp = reinterpret_cast<const PT*>(args.v) + seq * SEQ;
             F::for_each_io(t, [&](int i, int m) { a[i] = IOP::load(vp + m); });
         }
         // One step per order, forwards (A) and then backwards (B), through a
@@ -94,13 +108,13 @@ backward1d_kernel(Backward1dArgs args)
             const bool back = s >= N;
             const int n = back ? 2 * N - 1 - s : s;
             const float bias = __ldg(args.bias + n * D + d);
-            const PT* xp = reinterpret_cast<const PT*>(pick(args.x, n)) + seq * (M / 2);
-            float2* wcn = wc + (size_t)n * (M / 2);
+            const PT* xp = reinterpret_cast<const PT*>(pick(args.x, n)) + seq * SEQ;
+            float2* wcn = wc + (size_t)n * SEQ;
             if (back) {
                 PT* dxp = reinterpret_cast<PT*>(const_cast<void*>(pick(reinterpret_cast<const void* const*>(args.dx), n)))
-                          + seq * (M / 2);
+                          + seq * SEQ;
                 // all loads first, then the stores: one latency, not one per value
-                float2 c[E / 2], xv[E / 2];
+                float2 c[NIO], xv[NIO];
                 F::for_each_io(t, [&](int i, int m) {
                     c[io_slot(i)] = wcn[io_slot(i) * T + t];
                     xv[io_slot(i)] = IOP::load(xp + m);
@@ -112,7 +126,7 @@ backward1d_kernel(Backward1dArgs args)
                 });
             }
             if constexpr (!F::H_IN_EXCHANGE)
-                cp_async_row(stage, args.H + ((size_t)n * D + d) * M, M * 8, t, T);
+                cp_async_row(stage, Hb + ((size_t)n * D + d) * M, M * 8, t, T);
             F::forward(a, sm, t);
             if (!back) {
                 if (active)
@@ -122,9 +136,9 @@ backward1d_kernel(Backward1dArgs args)
                     });
             } else if (active) {
                 // dh spectrum: acc[k] (+)= E[k] conj(Z_n[k]) over the 2L-point bins
-                float2* acc = args.acc + ((size_t)n * D + d) * M;
+                float2* acc = args.acc + (((size_t)(PS ? b : 0) * N + n) * D + d) * M;
                 const float2* zr = wz + (size_t)n * M;
-                const bool first = b == 0;
+                const bool first = PS || b == 0;
                 float2 z[E];
                 static_for<E>([&](auto ii) {
                     constexpr int i = decltype(ii)::value;
@@ -152,7 +166,7 @@ backward1d_kernel(Backward1dArgs args)
             }
             const float2* Hs = stage;
             if constexpr (F::H_IN_EXCHANGE) {
-                cp_async_row(sm, args.H + ((size_t)n * D + d) * M, M * 8, t, T);
+                cp_async_row(sm, Hb + ((size_t)n * D + d) * M, M * 8, t, T);
                 Hs = sm;
             }
             cp_async_wait_all();
@@ -162,7 +176,7 @@ backward1d_kernel(Backward1dArgs args)
             F::inverse(a, sm, t);
             if (!back) {
                 // a = c_{n+1}: save it, then z_{n+1} = x_{n+1} c_{n+1}, or g = dy
-                const PT* gp = reinterpret_cast<const PT*>(args.dy) + seq * (M / 2);
+                const PT* gp = reinterpret_cast<const PT*>(args.dy) + seq * SEQ;
                 F::for_each_io(t, [&](int i, int m) {
                     if (active) wcn[io_slot(i) * T + t] = a[i];
                     if (n + 1 < N) {
@@ -175,7 +189,7 @@ backward1d_kernel(Backward1dArgs args)
             }
         }
         if (active) {
-            PT* dvp = reinterpret_cast<PT*>(args.dv) + seq * (M / 2);
+            PT* dvp = reinterpret_cast<PT*>(args.dv) + seq * SEQ;
             F::for_each_io(t, [&](int i, int m) { IOP::store(dvp + m, a[i]); });
         }
     }
@@ -183,13 +197,14 @@ backward1d_kernel(Backward1dArgs args)
 
 // dh_n[d] and db_n[d] from the accumulated spectra: one group per row
 // (n, d): the inverse real FFT of the packed spectrum (scale 1/P), the
-// first L lags, and db = dh[0].
-template <int LOG2M>
-__global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS)
+// first L lags, and db = dh[0].  PS: the group inverts the B per-sample
+// spectra of its row in turn and db is the sum of their lag-0 values.
+template <int LOG2M, bool PS = false, bool PAD = true>
+__global__ void __launch_bounds__(Fft1d<LOG2M, PAD>::THREADS)
 dh_finalize_kernel(Backward1dArgs args)
 {
     grid_dependency_begin();
-    using F = Fft1d<LOG2M>;
+    using F = Fft1d<LOG2M, PAD>;
     constexpr int M = F::M, E = F::E, T = F::T;
     extern __shared__ __align__(16) float2 smem_dyn[];
     const int g = threadIdx.x / T, t = threadIdx.x % T;
@@ -198,8 +213,11 @@ dh_finalize_kernel(Backward1dArgs args)
     const bool active = row_raw < rows;
     const int row = active ? row_raw : rows - 1;
     float2* sm = smem_dyn + g * F::SMEM_SEQ;
-    const float2* acc = args.acc + (size_t)row * M;
     constexpr float s = 1.0f / (2.0f * (float)M);           // 1/P of the inverse DFT
+    float db = 0.0f;
+    for (int b = 0; b < (PS ? args.B : 1); ++b) {
+    const size_t srow = (size_t)b * rows + row;              // [B][N][D] rows (b = 0 when shared)
+    const float2* acc = args.acc + srow * M;
     float2 a[E];
     F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
         float2 z1, z2;
@@ -219,12 +237,18 @@ dh_finalize_kernel(Backward1dArgs args)
     });
     F::inverse(a, sm, t);
     if (active) {
-        float2* dhp = reinterpret_cast<float2*>(args.dh + (size_t)row * M);
+        float2* dhp = reinterpret_cast<float2*>(args.dh) + srow * F::SEQ;   // L = 2 SEQ lags a row
         F::for_each_io(t, [&](int i, int m) {
             dhp[m] = a[i];
-            if (m == 0) args.dbias[row] = a[i].x;             // db_n = dh_n[0]
+            if (m == 0) db += a[i].x;                         // db_n = sum of dh_n[0]
         });
     }
+    __syncthreads();                                          // sm is reused by the next sample
+    }
+    if (active)
+        F::for_each_io(t, [&](int i, int m) {
+            if (m == 0) args.dbias[row] = db;
+        });
 }
 
 }  // namespace hyena

@@ -48,7 +48,9 @@ struct Fft3dZ {
 // it to every volume of that channel in the wave: z transform, multiply,
 // inverse, planes z < Z kept.  kx = 0 is left to the pair CTAs: each takes
 // TC/2 pairs u in [0, H], slot 0 of rows ky = u (column 2j) and 2H - u
-// (column 2j + 1).  MODE 1 (spectra): forward z transform of every slot of
+// (column 2j + 1).  MODE 2: MODE 0 with per-sample spectra, each volume b
+// of the channel loading sample b's column (at Hs + b Hs_bstride) instead.
+// MODE 1 (spectra): forward z transform of every slot of
 // the filters' planes z < Z, all 2Z planes written.  Circular (PAD false):
 // Z-point transforms of all Z planes, H rows a plane, nothing cropped.
 template <int LOG2Z2, int MODE, bool PAD = true>
@@ -124,16 +126,24 @@ fft3d_z_kernel(Fft2dArgs a)
         const int qa = max(a.q0, c * a.B), qb = min(a.q0 + a.nq, (c + 1) * a.B);
         const float bias = __ldg(a.bias + a.n * a.C + c);
         const float2* Hn = a.Hs + ((size_t)a.n * a.C + c) * Z2 * plane;   // [2Z][2H][W]
+        // per-sample spectra (MODE 2): volume q = c B + b takes sample b's set
+        constexpr bool PS = MODE == 2;
+        auto spectra_of = [&](int q) { return PS ? Hn + (size_t)(q - c * a.B) * a.Hs_bstride : Hn; };
         const float s = 1.0f / ((float)Z2 * (float)H2);
         if (!pair_cta) {
-            // the filter column, (H + b) / (2Z 2H), in register order
+            // the filter column, (H + b) / (2Z 2H), in register order; loaded
+            // once for the channel, or per volume with per-sample spectra
             float2 hv[V];
-            static_for<V>([&](auto rr) {
-                constexpr int r = decltype(rr)::value;
-                const float2 h = __ldg(Hn + (size_t)(t + r * (Z2 / V)) * plane + (size_t)ky * W + kx);
-                hv[r] = make_float2((h.x + bias) * s, h.y * s);
-            });
+            auto load_filter = [&](const float2* Hq) {
+                static_for<V>([&](auto rr) {
+                    constexpr int r = decltype(rr)::value;
+                    const float2 h = __ldg(Hq + (size_t)(t + r * (Z2 / V)) * plane + (size_t)ky * W + kx);
+                    hv[r] = make_float2((h.x + bias) * s, h.y * s);
+                });
+            };
+            if constexpr (!PS) load_filter(Hn);
             for (int q = qa; q < qb; ++q) {
+                if constexpr (PS) load_filter(spectra_of(q));
                 float2* colp = a.S + (size_t)(q - a.q0) * a.zp * plane + (size_t)ky * W + kx;
                 load_col(colp);
                 FZ::template run<-1, true, PAD>(buf, reg, t);
@@ -152,6 +162,7 @@ fft3d_z_kernel(Fft2dArgs a)
         } else {
             const int u0 = (int)((blk - (long)nch * reg_per) % npair) * NP;
             for (int q = qa; q < qb; ++q) {
+                const float2* Hq = spectra_of(q);
                 float2* colp = a.S + (size_t)(q - a.q0) * a.zp * plane + (size_t)ky * W;
                 load_col(colp);
                 FZ::template run<-1, true, PAD>(buf, reg, t);
@@ -172,8 +183,8 @@ fft3d_z_kernel(Fft2dArgs a)
                     float2* bB = self ? bA : smem_z + (2 * j + 1) * ZL::STRIDE;
                     const int kz2 = (Z2 - kz) % Z2;
                     const float2 A = bA[pad16(kz)], Bp = bB[pad16(kz2)];
-                    const float2 p1 = __ldg(Hn + (size_t)kz * plane + (size_t)uj * W);
-                    const float2 p2 = __ldg(Hn + (size_t)kz2 * plane + (size_t)u2 * W);
+                    const float2 p1 = __ldg(Hq + (size_t)kz * plane + (size_t)uj * W);
+                    const float2 p2 = __ldg(Hq + (size_t)kz2 * plane + (size_t)u2 * W);
                     // X0 = (A + conj B')/2, XW = (A - conj B')/(2i); the filter likewise
                     const float2 x0 = make_float2(0.5f * (A.x + Bp.x), 0.5f * (A.y - Bp.y));
                     const float2 xw = make_float2(0.5f * (A.y + Bp.y), -0.5f * (A.x - Bp.x));

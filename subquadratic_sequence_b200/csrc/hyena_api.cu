@@ -118,6 +118,14 @@ hyena_status_t forward_impl(const void* v, const void* const* x, const float* h,
 hyena_status_t forward2d_impl(const void* v, const void* const* x, const float* h, const float* Hs,
                               bool per_sample, const float* bias, int B, int C, int H, int W, int N,
                               hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes, void* stream);
+hyena_status_t backward_impl(const void* v, const void* const* x, const float* H, bool per_sample,
+                             bool circular, const float* bias, const void* dy, int B, int D, int L, int N,
+                             hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
+                             void* workspace, size_t ws_bytes, void* stream);
+hyena_status_t forward3d_impl(const void* v, const void* const* x, const float* h, const float* Hs,
+                              bool per_sample, const float* bias, int B, int C, int Z, int H, int W,
+                              int N, hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes,
+                              void* stream);
 
 }  // namespace
 
@@ -209,6 +217,24 @@ hyena_status_t hyena_filter_gen_3d(const hyena_ffn_t* ffn, int N, int C, int Z, 
     if (npos > (1L << 30) || (long)N * C > 65535L * kFgRowTile || (long)N * C * npos > (1L << 40))
         return HYENA_ERR_UNSUPPORTED;
     return filter_gen(ffn, N * C, C, npos, 0, H, W, true, h, (cudaStream_t)stream, nullptr, 1, Z);
+}
+
+hyena_status_t hyena_filter_gen_film_3d(const hyena_ffn_t* ffn, const hyena_film_t* film, int B, int N,
+                                        int C, int Z, int H, int W, float* h, void* stream)
+{
+    hyena_status_t s = check_ffn(ffn);
+    if (s != HYENA_OK) return s;
+    if (!film || !h || B < 1 || N < 1 || C < 1 || Z < 1 || H < 1 || W < 1 || !aligned(h, 4))
+        return HYENA_ERR_INVALID_ARG;
+    const void* p[4] = {film->omega, film->gamma, film->beta, film->sigma};
+    for (const void* q : p)
+        if (q && !aligned(q, 4)) return HYENA_ERR_INVALID_ARG;
+    if (ffn->n_bands > kFg3dBands) return HYENA_ERR_UNSUPPORTED;
+    const long npos = (long)Z * H * W;
+    if (B > 65535 || npos > (1L << 30) || (long)N * C > 65535L * kFgRowTile ||
+        (long)B * N * C * npos > (1L << 40))
+        return HYENA_ERR_UNSUPPORTED;
+    return filter_gen(ffn, N * C, C, npos, 0, H, W, true, h, (cudaStream_t)stream, film, B, Z);
 }
 
 size_t hyena_filter_rfft_workspace_size(int N, int D, int L)
@@ -414,27 +440,88 @@ size_t hyena_fftconv_backward_workspace_size(int D, int L, int N)
     return round_up(spec, 256) * 2 + round_up(spec / 2, 256);   // acc, wz, wc
 }
 
+size_t hyena_fftconv_backward_per_sample_workspace_size(int B, int D, int L, int N)
+{
+    int log2m = 0;
+    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2Fused, &log2m) != HYENA_OK)
+        return (size_t)-1;
+    const size_t spec = sizeof(float2) * (size_t)N * D * L;
+    return round_up(spec * B, 256) + round_up(spec, 256) + round_up(spec / 2, 256);   // acc, wz, wc
+}
+
 hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, const float* H,
                                            const float* bias, const void* dy, int B, int D, int L,
                                            int N, hyena_dtype_t io, void* dv, void* const* dx,
                                            float* dh, float* dbias, void* workspace, size_t ws_bytes,
                                            void* stream)
 {
+    return backward_impl(v, x, H, false, false, bias, dy, B, D, L, N, io, dv, dx, dh, dbias, workspace,
+                         ws_bytes, stream);
+}
+
+size_t hyena_fftconv_backward_circular_workspace_size(int D, int L, int N)
+{
+    const int k = exact_log2(L);
+    if (D < 1 || N < 1 || N > HYENA_MAX_ORDER || k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1)
+        return (size_t)-1;
+    return 3 * round_up(sizeof(float2) * (size_t)N * D * (L / 2), 256);   // acc, wz, wc
+}
+
+hyena_status_t hyena_fftconv_gate_backward_circular(const void* v, const void* const* x, const float* H,
+                                                    const float* bias, const void* dy, int B, int D, int L,
+                                                    int N, hyena_dtype_t io, void* dv, void* const* dx,
+                                                    float* dh, float* dbias, void* workspace,
+                                                    size_t ws_bytes, void* stream)
+{
+    return backward_impl(v, x, H, false, true, bias, dy, B, D, L, N, io, dv, dx, dh, dbias, workspace,
+                         ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv_gate_backward_per_sample(const void* v, const void* const* x, const float* H,
+                                                      const float* bias, const void* dy, int B, int D, int L,
+                                                      int N, hyena_dtype_t io, void* dv, void* const* dx,
+                                                      float* dh, float* dbias, void* workspace,
+                                                      size_t ws_bytes, void* stream)
+{
+    return backward_impl(v, x, H, true, false, bias, dy, B, D, L, N, io, dv, dx, dh, dbias, workspace,
+                         ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// per_sample: a spectrum set per sample (L <= 16384); circular: the
+// circular recurrence (32 <= L <= 16384, spectra of L/2 slots)
+hyena_status_t backward_impl(const void* v, const void* const* x, const float* H, bool per_sample,
+                             bool circular, const float* bias, const void* dy, int B, int D, int L, int N,
+                             hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
+                             void* workspace, size_t ws_bytes, void* stream)
+{
     if (!v || !x || !H || !bias || !dy || !dv || !dx || !dh || !dbias) return HYENA_ERR_INVALID_ARG;
     if (B < 1 || D < 1 || N < 1 || L < 1) return HYENA_ERR_INVALID_ARG;
     if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
     if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
     int log2m = 0;
-    hyena_status_t s = check_len(L, kMaxLog2, &log2m);
-    if (s != HYENA_OK) return s;
-    if ((long)B * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    if (circular) {
+        const int k = exact_log2(L);
+        if (k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1) return HYENA_ERR_UNSUPPORTED;
+        log2m = k - 1;                       // M = L/2 packed points
+    } else {
+        hyena_status_t s = check_len(L, per_sample ? kMaxLog2Fused : kMaxLog2, &log2m);
+        if (s != HYENA_OK) return s;
+    }
+    if ((long)B * D > (1L << 30) || (per_sample && (long)B * N * D > (1L << 30))) return HYENA_ERR_UNSUPPORTED;
     for (int n = 0; n < N; ++n)
         if (!x[n] || !dx[n] || !aligned(x[n], 16) || !aligned(dx[n], 16)) return HYENA_ERR_INVALID_ARG;
     if (!aligned(v, 16) || !aligned(dy, 16) || !aligned(dv, 16) || !aligned(H, 16) || !aligned(dh, 16) ||
         !aligned(bias, 4) || !aligned(dbias, 4))
         return HYENA_ERR_INVALID_ARG;
-    const size_t need = hyena_fftconv_backward_workspace_size(D, L, N);
+    const size_t need = circular ? hyena_fftconv_backward_circular_workspace_size(D, L, N)
+                        : per_sample ? hyena_fftconv_backward_per_sample_workspace_size(B, D, L, N)
+                                     : hyena_fftconv_backward_workspace_size(D, L, N);
     if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+    const size_t sets = per_sample ? (size_t)B : 1;           // spectrum sets and dh sets
 
     // every output against every input, the other outputs and the workspace
     const size_t act = (size_t)B * D * L * io_bytes(io);
@@ -443,12 +530,12 @@ hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, 
     int ni = 0, no = 0;
     in[ni++] = {v, act};
     in[ni++] = {dy, act};
-    in[ni++] = {H, spectrum_bytes(N, D, L)};
+    in[ni++] = {H, spectrum_bytes(N, D, circular ? L / 2 : L) * sets};
     in[ni++] = {bias, sizeof(float) * N * D};
     in[ni++] = {workspace, need};
     for (int n = 0; n < N; ++n) in[ni++] = {x[n], act};
     out[no++] = {dv, act};
-    out[no++] = {dh, sizeof(float) * (size_t)N * D * L};
+    out[no++] = {dh, sizeof(float) * (size_t)N * D * L * sets};
     out[no++] = {dbias, sizeof(float) * N * D};
     for (int n = 0; n < N; ++n) out[no++] = {dx[n], act};
     for (int o = 0; o < no; ++o) {
@@ -458,10 +545,10 @@ hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, 
             if (overlap(out[o].p, out[o].n, out[p].p, out[p].n)) return HYENA_ERR_INVALID_ARG;
     }
 
-    const size_t spec = sizeof(float2) * (size_t)N * D * L;
+    const size_t spec = sizeof(float2) * (size_t)N * D * (circular ? L / 2 : L);   // one spectrum set
     char* ws = static_cast<char*>(workspace);
     cudaStream_t st = (cudaStream_t)stream;
-    if (log2m > kMaxLog2Fused) {
+    if (!circular && log2m > kMaxLog2Fused) {
         // four-step backward (L > 16384)
         const FourStepBwdLayout lay = fourstep_bwd_layout(log2m, D, N);
         FourStepBwdArgs b = {};
@@ -499,13 +586,23 @@ hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, 
     a.dh = dh;
     a.dbias = dbias;
     a.acc = reinterpret_cast<float2*>(ws);
-    a.wz = reinterpret_cast<float2*>(ws + round_up(spec, 256));
-    a.wc = reinterpret_cast<float2*>(ws + 2 * round_up(spec, 256));
+    a.wz = reinterpret_cast<float2*>(ws + round_up(spec * sets, 256));
+    a.wc = reinterpret_cast<float2*>(ws + round_up(spec * sets, 256) + round_up(spec, 256));   // [D][N][SEQ]
     a.B = B;
     a.D = D;
     a.N = N;
+    a.H_bstride = per_sample ? (size_t)N * D * L : 0;
+    if (circular)
+        return io == HYENA_BF16 ? dispatch_backward_circ_bf16(log2m, a, st)
+                                : dispatch_backward_circ_f32(log2m, a, st);
+    if (per_sample)
+        return io == HYENA_BF16 ? dispatch_backward_ps_bf16(log2m, a, st) : dispatch_backward_ps_f32(log2m, a, st);
     return io == HYENA_BF16 ? dispatch_backward_bf16(log2m, a, st) : dispatch_backward_f32(log2m, a, st);
 }
+
+}  // namespace
+
+extern "C" {
 
 // ------------------------------------------------------------------ 2-D
 
@@ -686,13 +783,36 @@ hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void* const* x,
                                             int H, int W, int N, hyena_dtype_t io, void* y,
                                             void* workspace, size_t ws_bytes, void* stream)
 {
+    return forward3d_impl(v, x, h, Hs, false, bias, B, C, Z, H, W, N, io, y, workspace, ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv3d_gate_forward_per_sample(const void* v, const void* const* x, const float* Hs,
+                                                       const float* bias, int B, int C, int Z, int H, int W,
+                                                       int N, hyena_dtype_t io, void* y, void* workspace,
+                                                       size_t ws_bytes, void* stream)
+{
+    if (!Hs) return HYENA_ERR_INVALID_ARG;
+    return forward3d_impl(v, x, nullptr, Hs, true, bias, B, C, Z, H, W, N, io, y, workspace, ws_bytes,
+                          stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+hyena_status_t forward3d_impl(const void* v, const void* const* x, const float* h, const float* Hs,
+                              bool per_sample, const float* bias, int B, int C, int Z, int H, int W,
+                              int N, hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes,
+                              void* stream)
+{
     if (!v || !x || !y || !bias || (!h && !Hs)) return HYENA_ERR_INVALID_ARG;
     if (B < 1 || C < 1 || N < 1 || Z < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
     if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
     if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
     int lz, lh, lw;
     if (!dims3d_ok(Z, H, W, lz, lh, lw)) return HYENA_ERR_UNSUPPORTED;
-    if ((long)B * C > (1L << 20) || (long)N * C * Z * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)B * C > (1L << 20) || (long)N * C * Z * H * (per_sample ? B : 1) > (1L << 30))
+        return HYENA_ERR_UNSUPPORTED;
     for (int n = 0; n < N; ++n)
         if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
     if (!aligned(v, 16) || !aligned(y, 16) || !aligned(bias, 4)) return HYENA_ERR_INVALID_ARG;
@@ -700,7 +820,7 @@ hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void* const* x,
 
     const size_t vol = (size_t)Z * H * W;
     const size_t act = (size_t)B * C * vol * io_bytes(io);
-    const size_t spec = sizeof(float2) * (size_t)N * C * 4 * vol;
+    const size_t spec = sizeof(float2) * (size_t)N * C * 4 * vol * (per_sample ? (size_t)B : 1);
     const size_t filt = sizeof(float) * (size_t)N * C * vol;
     const size_t need = hyena_fftconv3d_workspace_size(B, C, Z, H, W, N, io, Hs != nullptr);
     if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
@@ -736,6 +856,7 @@ hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void* const* x,
     for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
     a.y = y;
     a.Hs = spectrum;
+    a.Hs_bstride = per_sample ? (size_t)N * C * 4 * vol : 0;
     a.bias = bias;
     a.B = B;
     a.C = C;
@@ -747,7 +868,7 @@ hyena_status_t hyena_fftconv3d_gate_forward(const void* v, const void* const* x,
                             : dispatch_fft3d_f32(lw, lh, lz, a, N, scratch, st);
 }
 
-}  // extern "C"
+}  // namespace
 
 // ------------------------------------------------------- circular 2-D
 

@@ -86,5 +86,9 @@ hyena_status_t dispatch_fourstep_rfft(int log2m, const float* h, int rows, float
 hyena_status_t launch_filter_gen(const FilterGenArgs& a, bool two_d, long npos, int B, cudaStream_t st);
 hyena_status_t dispatch_backward_f32(int log2m, const Backward1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_backward_bf16(int log2m, const Backward1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_backward_ps_f32(int log2m, const Backward1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_backward_ps_bf16(int log2m, const Backward1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_backward_circ_f32(int log2m, const Backward1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_backward_circ_bf16(int log2m, const Backward1dArgs& a, cudaStream_t st);
 
 }  // namespace hyena

@@ -65,6 +65,12 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv_gate_forward_noalloc": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp,
                                                 vp], i),
         "hyena_fftconv_backward_workspace_size": ([i, i, i], sz),
+        "hyena_fftconv_backward_per_sample_workspace_size": ([i, i, i, i], sz),
+        "hyena_fftconv_backward_circular_workspace_size": ([i, i, i], sz),
+        "hyena_fftconv_gate_backward_circular": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp,
+                                                  ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
+        "hyena_fftconv_gate_backward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp,
+                                                    ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_fftconv_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp,
                                          ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_filter_rfft_circular": ([vp, i, i, i, vp, vp], i),
@@ -78,6 +84,9 @@ def _load() -> ctypes.CDLL:
                                           vp, sz, vp], i),
         "hyena_filter_rfft3d": ([vp, i, i, i, i, i, vp, vp], i),
         "hyena_filter_gen_3d": ([ffn_p, i, i, i, i, i, vp, vp], i),
+        "hyena_filter_gen_film_3d": ([ffn_p, ctypes.POINTER(hyena_film_t), i, i, i, i, i, i, vp, vp], i),
+        "hyena_fftconv3d_gate_forward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, i, vp,
+                                                     vp, sz, vp], i),
         "hyena_filter_rfft2d_circular": ([vp, i, i, i, i, vp, vp], i),
         "hyena_fftconv2d_backward_workspace_size": ([i, i, i, i, i], sz),
         "hyena_fftconv2d_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
@@ -309,6 +318,74 @@ def hyena_fftconv_gate_backward(v: torch.Tensor, xs, bias: torch.Tensor, H: torc
         workspace = torch.empty(hyena_fftconv_backward_workspace_size(D, L, N), device=v.device,
                                 dtype=torch.uint8)
     _check("hyena_fftconv_gate_backward", LIB.hyena_fftconv_gate_backward(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+        B, D, L, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+        ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db
+
+
+def hyena_fftconv_backward_per_sample_workspace_size(B: int, D: int, L: int, N: int) -> int:
+    n = LIB.hyena_fftconv_backward_per_sample_workspace_size(B, D, L, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv_backward_per_sample_workspace_size", HYENA_ERR_UNSUPPORTED,
+                         "invalid sizes (L <= 16384)")
+    return n
+
+
+def hyena_fftconv_gate_backward_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor,
+                                           dy: torch.Tensor, *, workspace=None, stream=None):
+    """The backward with a spectrum set per sample, H [B][N][D][L]: returns
+    (dv, [dx_1..dx_N], dh [B][N][D][L] per sample, dbias [N][D] summed over
+    the batch); L <= 16384."""
+    B, D, L = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty((B, N, D, L), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, D), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(hyena_fftconv_backward_per_sample_workspace_size(B, D, L, N), device=v.device,
+                                dtype=torch.uint8)
+    _check("hyena_fftconv_gate_backward_per_sample", LIB.hyena_fftconv_gate_backward_per_sample(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+        B, D, L, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+        ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db
+
+
+def hyena_fftconv_backward_circular_workspace_size(D: int, L: int, N: int) -> int:
+    n = LIB.hyena_fftconv_backward_circular_workspace_size(D, L, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv_backward_circular_workspace_size", HYENA_ERR_UNSUPPORTED,
+                         "invalid sizes (32 <= L <= 16384)")
+    return n
+
+
+def hyena_fftconv_gate_backward_circular(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor,
+                                         dy: torch.Tensor, *, workspace=None, stream=None):
+    """The backward of the circular forward (H [N][D][L/2] from
+    hyena_filter_rfft_circular): returns (dv, [dx_1..dx_N], dh [N][D][L],
+    dbias [N][D]), dh and dbias summed over the batch."""
+    B, D, L = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty((N, D, L), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, D), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(hyena_fftconv_backward_circular_workspace_size(D, L, N), device=v.device,
+                                dtype=torch.uint8)
+    _check("hyena_fftconv_gate_backward_circular", LIB.hyena_fftconv_gate_backward_circular(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
         B, D, L, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
@@ -596,3 +673,38 @@ def hyena_filter_gen_3d(W1, W2, W3, Wout, alpha, N: int, C: int, Z: int, H: int,
         ctypes.byref(f), N, C, Z, H, W, ctypes.c_void_p(_dev(out, torch.float32, "h")), _stream(stream)))
     return out
 
+
+def hyena_filter_gen_film_3d(W1, W2, W3, Wout, alpha, N: int, C: int, Z: int, H: int, W: int, *, B: int,
+                             omega=None, gamma=None, beta=None, sigma=None, n_bands: int = 8,
+                             width: int = 64, decay_div: float = 64.0, out=None, stream=None):
+    """Per-sample 3-D filters h [B][N][C][Z][H][W] float32 (FiLM-modulated;
+    the Gaussian window when sigma [C] is given)."""
+    f = _ffn(W1, W2, W3, Wout, alpha, n_bands, width, decay_div)
+    opt = lambda t, name: ctypes.c_void_p(_dev(t, torch.float32, name)) if t is not None else None
+    film = hyena_film_t(opt(omega, "omega"), opt(gamma, "gamma"), opt(beta, "beta"), opt(sigma, "sigma"))
+    if out is None:
+        out = torch.empty((B, N, C, Z, H, W), device=W1.device, dtype=torch.float32)
+    _check("hyena_filter_gen_film_3d", LIB.hyena_filter_gen_film_3d(
+        ctypes.byref(f), ctypes.byref(film), B, N, C, Z, H, W,
+        ctypes.c_void_p(_dev(out, torch.float32, "h")), _stream(stream)))
+    return out
+
+
+def hyena_fftconv3d_gate_forward_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor, *,
+                                            out=None, workspace=None, stream=None):
+    """The 3-D forward with per-sample spectra Hs [B][N][C][2Z][2H][W] complex64."""
+    B, C, Z, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    need = hyena_fftconv3d_workspace_size(B, C, Z, H, W, N, io, True)
+    if workspace is None:
+        workspace = torch.empty(need, device=v.device, dtype=torch.uint8)
+    _check("hyena_fftconv3d_gate_forward_per_sample", LIB.hyena_fftconv3d_gate_forward_per_sample(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, Z, H, W, N, io,
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out

@@ -97,6 +97,9 @@ WORKLOADS = {
     "c1_film": Workload("c1_film", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), film=True),
     # order-2 3-D operator on 64^3 volumes, B=2, C=32, bf16 storage
     "c5_3d": Workload("c5_3d", "3d", N=2, B=2, D=32, Z=64, H=64, W=64, io="bf16", seed=_seed(5)),
+    # c5_3d with input-dependent (per-sample, FiLM-modulated) 3-D filters
+    "c5_3d_film": Workload("c5_3d_film", "3d", N=2, B=2, D=32, Z=64, H=64, W=64, io="bf16", seed=_seed(5),
+                           film=True),
     # circular mode (periodic boundaries) at the shapes of c1, c4 and c5_3d
     "c1_circ": Workload("c1_circ", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), circular=True),
     "c4_circ": Workload("c4_circ", "2d", N=2, B=2, D=128, H=256, W=256, io="f32", seed=_seed(4), circular=True),

@@ -128,3 +128,49 @@ def test_backward_c3_64k_full_size(hy):
     got = run(hy, wl, inp, h32, dy)
     ref = oracle.hyena_backward(inp["v"], np.stack(inp["x"]), h32, inp["b"], dy)
     check(got, ref, wl.io, "c3_64k")
+
+
+# ------------------------------------------------- per-sample filters
+
+PS_CASES = [(2, 3, 64, 2, "f32"), (3, 13, 2048, 2, "f32"), (2, 5, 1024, 3, "bf16"), (2, 2, 16384, 2, "f32"),
+            (1, 1, 16, 1, "f32")]
+
+
+@pytest.mark.parametrize("B,D,L,N,io", PS_CASES)
+def test_backward_per_sample_matches_oracle(hy, B, D, L, N, io):
+    wl, inp = random_problem(B, D, L, N, seed=700 + L + N, io=io)
+    r = np.random.default_rng(L + B)
+    decay = np.exp(-np.arange(L) * np.linspace(0.3, 1.5, D)[:, None] / 64.0)
+    h32 = (r.standard_normal((B, N, D, L)) * 0.2 * decay).astype(np.float32)
+    dy = synth.make_output_grad(wl)
+    H = hy.hyena_filter_rfft(dev(h32.reshape(B * N, D, L))).reshape(B, N, D, L)
+    dv, dxs, dh, db = hy.hyena_fftconv_gate_backward_per_sample(
+        dev(inp["v"], io), [dev(x, io) for x in inp["x"]], dev(inp["b"]), H, dev(dy, io))
+    torch.cuda.synchronize()
+    got = host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+    ref = oracle.hyena_backward_per_sample(inp["v"], np.stack(inp["x"]), h32, inp["b"], dy)
+    check(got, ref, io, f"per-sample B{B} D{D} L{L} N{N} {io}")
+
+
+def test_backward_per_sample_with_equal_sets_is_the_shared_backward(hy):
+    """Every sample given the same spectra: dv and dx equal the shared
+    backward's bit for bit, the per-sample dh sum to its dh."""
+    B, D, L, N = 4, 6, 2048, 2
+    wl, inp = random_problem(B, D, L, N, seed=41, io="bf16")
+    h32 = filters(wl, seed=42)
+    dy = dev(synth.make_output_grad(wl), "bf16")
+    H = hy.hyena_filter_rfft(dev(h32))
+    v, xs, b = dev(inp["v"], "bf16"), [dev(x, "bf16") for x in inp["x"]], dev(inp["b"])
+    dv, dxs, dh, db = hy.hyena_fftconv_gate_backward(v, xs, b, H, dy)
+    pv, pxs, ph, pb = hy.hyena_fftconv_gate_backward_per_sample(
+        v, xs, b, H.unsqueeze(0).expand(B, -1, -1, -1).contiguous(), dy)
+    torch.cuda.synchronize()
+    assert torch.equal(dv, pv) and all(torch.equal(a, c) for a, c in zip(dxs, pxs))
+    assert rel_max_err(host(ph).sum(axis=0), host(dh)) <= 1e-5
+    assert rel_max_err(host(pb), host(db)) <= 1e-5
+
+
+def test_backward_per_sample_rejects_long_sequences(hy):
+    from subquadratic_sequence_b200.hyena import HyenaError
+    with pytest.raises(HyenaError):
+        hy.hyena_fftconv_backward_per_sample_workspace_size(2, 4, 32768, 2)

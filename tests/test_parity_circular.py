@@ -60,3 +60,61 @@ def test_circular_shift_filter_rotates(hy):
     y = hy.hyena_fftconv_gate_forward_circular(dev(v), [dev(np.ones_like(v))], dev(np.zeros((1, D), np.float32)), H)
     torch.cuda.synchronize()
     assert rel_max_err(host(y), np.roll(v, k, axis=-1)) <= 1e-5
+
+
+# ------------------------------------------------------------ backward
+
+def check_backward(got, ref, io, name):
+    dv, dx, dh, db = got
+    rdv, rdx, rdh, rdb = ref
+    assert_close(dv, rdv, io, f"{name} dv")
+    assert_close(dx, rdx, io, f"{name} dx")
+    assert rel_max_err(dh, rdh) <= 1e-4, f"{name} dh {rel_max_err(dh, rdh):.3e}"
+    assert rel_max_err(db, rdb) <= 1e-4, f"{name} db {rel_max_err(db, rdb):.3e}"
+
+
+@pytest.mark.parametrize("B,D,L,N,io", [
+    (1, 1, 32, 1, "f32"), (2, 3, 64, 2, "f32"), (2, 5, 1024, 3, "bf16"), (2, 13, 4096, 2, "f32"),
+    (1, 2, 16384, 2, "f32"), (8, 6, 2048, 2, "bf16"), (3, 2, 256, 16, "f32"),
+])
+def test_backward_circular_matches_oracle(hy, B, D, L, N, io):
+    wl, inp = random_problem(B, D, L, N, seed=900 + L + N, io=io)
+    h = filters(N, D, L, seed=L + 9)
+    dy = np.random.default_rng(L).standard_normal((B, D, L)).astype(np.float32)
+    if io == "bf16":
+        from subquadratic_sequence_b200 import synth
+        dy = synth.bf16_round(dy)
+    H = hy.hyena_filter_rfft_circular(dev(h))
+    dv, dxs, dh, db = hy.hyena_fftconv_gate_backward_circular(
+        dev(inp["v"], io), [dev(x, io) for x in inp["x"]], dev(inp["b"]), H, dev(dy, io))
+    torch.cuda.synchronize()
+    got = host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+    ref = oracle.hyena_backward_circular(inp["v"], np.stack(inp["x"]), h, inp["b"], dy)
+    check_backward(got, ref, io, f"circular backward B{B} D{D} L{L} N{N} {io}")
+
+
+def test_backward_circular_shift_filter_closed_form(hy):
+    # N = 1, h = delta_k, b = 0: y = x roll(v, k), so dv = roll(dy x, -k),
+    # dx = dy roll(v, k), dh[s] = sum_b sum_t dy[t] x[t] v[(t - s) mod L]
+    B, D, L, k = 2, 3, 512, 37
+    r = np.random.default_rng(3)
+    v, x, dy = (r.standard_normal((B, D, L)).astype(np.float32) for _ in range(3))
+    h = np.zeros((1, D, L), np.float32)
+    h[:, :, k] = 1.0
+    H = hy.hyena_filter_rfft_circular(dev(h))
+    dv, dxs, dh, db = hy.hyena_fftconv_gate_backward_circular(
+        dev(v), [dev(x)], dev(np.zeros((1, D), np.float32)), H, dev(dy))
+    torch.cuda.synchronize()
+    e = (dy * x).astype(np.float64)
+    assert rel_max_err(host(dv), np.roll(e, -k, axis=-1)) <= 1e-5
+    assert rel_max_err(host(dxs[0]), dy * np.roll(v, k, axis=-1)) <= 1e-5
+    ref_dh = np.stack([np.sum(e * np.roll(v, s, axis=-1), axis=(0, 2)) for s in range(L)], axis=-1)
+    assert rel_max_err(host(dh)[0], ref_dh) <= 1e-4
+    assert rel_max_err(host(db)[0], ref_dh[:, 0]) <= 1e-4
+
+
+def test_backward_circular_rejects_unsupported_lengths(hy):
+    from subquadratic_sequence_b200.hyena import HyenaError
+    for L in (16, 32768):
+        with pytest.raises(HyenaError):
+            hy.hyena_fftconv_backward_circular_workspace_size(4, L, 2)
