@@ -195,25 +195,36 @@ fourstep_bwd_row_kernel(FourStepBwdArgs ba)
             cp_async_wait_all();
             __syncthreads();
             forward_rows(nullptr);                                // E (rows of e)
+            // the products E conj(Z) replace the staged Z rows, then the
+            // accumulator is read in one sweep and written in another, so
+            // its loads are not each held behind the previous store (every
+            // thread touches only its own pairs: no barrier in between)
             FS::for_each_pair(smem_fb, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2 w) {
                 const float2 e1 = *p1, e2 = *p2, y1 = p1[FB::ZOFF], y2 = p2[FB::ZOFF];
                 float2 z1 = e1, z2 = e2;
                 if (kind == 1) {
                     // slot 0: bins 0 and M, both real
-                    const float2 p = make_float2((e1.x + e1.y) * (y1.x + y1.y), (e1.x - e1.y) * (y1.x - y1.y));
-                    Ar[0] = cadd(Ar[0], p);
+                    p1[FB::ZOFF] = make_float2((e1.x + e1.y) * (y1.x + y1.y), (e1.x - e1.y) * (y1.x - y1.y));
                     const float2 h0 = __ldg(Hr);
                     spectral_pair<M>(z1, z2, make_float2(h0.x, 0.0f), make_float2(h0.y, 0.0f), w, bias);
                 } else {
                     float2 E1, E2, Z1, Z2;
                     real_split(e1, e2, w, E1, E2);
                     real_split(y1, y2, w, Z1, Z2);
-                    Ar[k] = cadd(Ar[k], cmulc(E1, Z1));
-                    if (kind == 0) Ar[M - k] = cadd(Ar[M - k], cmulc(E2, Z2));
+                    p1[FB::ZOFF] = cmulc(E1, Z1);
+                    if (kind == 0) p2[FB::ZOFF] = cmulc(E2, Z2);
                     spectral_pair<M>(z1, z2, cconj(__ldg(Hr + k)), cconj(__ldg(Hr + (M - k))), w, bias);
                 }
                 *p1 = z1;
                 if (kind == 0) *p2 = z2;
+            });
+            FS::for_each_pair(smem_fb, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2) {
+                p1[FB::ZOFF] = cadd(p1[FB::ZOFF], Ar[k]);
+                if (kind == 0) p2[FB::ZOFF] = cadd(p2[FB::ZOFF], Ar[M - k]);
+            });
+            FS::for_each_pair(smem_fb, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2) {
+                Ar[k] = p1[FB::ZOFF];
+                if (kind == 0) Ar[M - k] = p2[FB::ZOFF];
             });
             __syncthreads();
             inverse_rows(Sq);
