@@ -417,6 +417,18 @@ def hyena_backward_2d(v, x, h, bias, dy, route="fft", threads=None):
     return dv, dx, dh, db
 
 
+def hyena_backward_2d_per_sample(v, x, h, bias, dy, route="fft", threads=None):
+    """The gradients through :func:`hyena_forward_2d_per_sample` (a filter
+    set per sample, h [B][N][C][H][W]): each sample's 2-D adjoint with its
+    own filters.  Returns (dv, dx, dh [B][N][C][H][W] per sample, dbias
+    [N][C] summed over the samples)."""
+    v, x, h, bias, dy = map(_f64, (v, x, h, bias, dy))
+    parts = [hyena_backward_2d(v[b:b + 1], x[:, b:b + 1], h[b], bias, dy[b:b + 1], route, threads)
+             for b in range(v.shape[0])]
+    return (np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts], axis=1),
+            np.stack([p[2] for p in parts]), np.sum([p[3] for p in parts], axis=0))
+
+
 def filter_gen_3d(W1, W2, W3, Wout, alpha, N, C, Z, H, W, n_bands=8, width=64, decay_div=64.0,
                   threads=None) -> np.ndarray:
     """Implicit 3-D filters h[N][C][Z][H][W] (float64): the filter network

@@ -249,3 +249,40 @@ def test_backward_circular_on_zero_padded_sequences_is_the_causal_backward():
     rv, rx, rh, rb = oracle.hyena_backward(v, x, h, b, dy)
     assert rel_err(dv[..., :L], rv) < 1e-12 and rel_err(dx[..., :L], rx) < 1e-12
     assert rel_err(dh[..., :L], rh) < 1e-12 and rel_err(db, rb) < 1e-12
+
+
+def test_backward_2d_per_sample_matches_finite_differences():
+    B, C, H, W, N = 2, 2, 3, 4, 2
+    r = np.random.default_rng(40)
+    v, x = r.standard_normal((B, C, H, W)), r.standard_normal((N, B, C, H, W))
+    h = r.standard_normal((B, N, C, H, W)) * 0.5
+    b, dy = r.standard_normal((N, C)), r.standard_normal((B, C, H, W))
+    dv, dx, dh, db = oracle.hyena_backward_2d_per_sample(v, x, h, b, dy, route="direct")
+    assert dh.shape == h.shape and db.shape == b.shape
+
+    def loss(v_, x_, h_, b_):
+        return float(np.sum(dy * oracle.hyena_forward_2d_per_sample(v_, x_, h_, b_, route="direct")))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name
+
+
+def test_backward_2d_per_sample_with_equal_sets_sums_to_the_shared_backward():
+    B, C, H, W, N = 3, 2, 8, 16, 2
+    r = np.random.default_rng(41)
+    v, x = r.standard_normal((B, C, H, W)), r.standard_normal((N, B, C, H, W))
+    h, b, dy = r.standard_normal((N, C, H, W)) * 0.3, r.standard_normal((N, C)), r.standard_normal((B, C, H, W))
+    dv, dx, dh, db = oracle.hyena_backward_2d(v, x, h, b, dy)
+    pv, px, ph, pb = oracle.hyena_backward_2d_per_sample(v, x, np.broadcast_to(h, (B,) + h.shape), b, dy)
+    assert rel_err(pv, dv) < 1e-13 and rel_err(px, dx) < 1e-13
+    assert rel_err(ph.sum(axis=0), dh) < 1e-12 and rel_err(pb, db) < 1e-12
