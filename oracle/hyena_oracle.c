@@ -1439,6 +1439,23 @@ static void corr2_fft(const double *p, const double *q, long H, long W, double *
         for (long c = 0; c < W; ++c) out[r * W + c] = s->ur[r * PW + c] / (double)(PH * PW);
 }
 
+/* Circular counterpart of both 2-D sums (periodic boundaries, "Handling
+ * Boundaries"): out[a][b] = sum_{t,s} p[t][s] q[(t - a) mod H][(s - b) mod
+ * W].  With p = e, q = z it is dh; with p = e, q = h the adjoint of the
+ * circular convolution with respect to its signal.  Its FFT route is
+ * corr2_fft on an H x W scratch (no padding, so the product wraps). */
+static void ccorr2_direct(const double *p, const double *q, long H, long W, double *out)
+{
+    for (long a = 0; a < H; ++a)
+        for (long b = 0; b < W; ++b) {
+            double acc = 0.0;
+            for (long t = 0; t < H; ++t)
+                for (long s = 0; s < W; ++s)
+                    acc += p[t * W + s] * q[((t - a + H) % H) * W + (s - b + W) % W];
+            out[a * W + b] = acc;
+        }
+}
+
 typedef struct {
     const double *v, *x, *h, *bias, *dy;
     long B, C, H, W, N;
@@ -1446,6 +1463,7 @@ typedef struct {
     double *dv, *dx, *dh, *dbias;
     long c0, step; /* channels c0, c0 + step, ... (dh, db summed over b here) */
     int status;
+    int circular;  /* 1: circular convolutions on the H x W grid itself */
 } bwd2_job;
 
 static void *backward_2d_worker(void *arg)
@@ -1458,7 +1476,8 @@ static void *backward_2d_worker(void *arg)
     fft2_scratch s = {0};
     if (!z || !c || !g || !e || !tmp ||
         (j->route == ROUTE_FFT &&
-         scratch2_alloc(&s, next_pow2(2 * j->H), next_pow2(2 * j->W)) != ORACLE_OK)) {
+         scratch2_alloc(&s, j->circular ? j->H : next_pow2(2 * j->H),
+                        j->circular ? j->W : next_pow2(2 * j->W)) != ORACLE_OK)) {
         j->status = ORACLE_ENOMEM;
         goto done;
     }
@@ -1475,8 +1494,14 @@ static void *backward_2d_worker(void *arg)
                 const double *hn = j->h + (n * C + ch) * HW, *xn = j->x + n * BCHW + img * HW;
                 const double bn = j->bias[n * C + ch];
                 double *zn = z + n * HW, *cn = c + n * HW;
-                if (j->route == ROUTE_DIRECT) conv2_direct(hn, zn, j->H, j->W, cn);
-                else conv2_fft(hn, zn, j->H, j->W, cn, &s);
+                if (j->circular) {
+                    if (j->route == ROUTE_DIRECT) cconv3_direct(hn, zn, 1, j->H, j->W, cn);
+                    else conv2_fft(hn, zn, j->H, j->W, cn, &s);   /* H x W scratch: wraps */
+                } else if (j->route == ROUTE_DIRECT) {
+                    conv2_direct(hn, zn, j->H, j->W, cn);
+                } else {
+                    conv2_fft(hn, zn, j->H, j->W, cn, &s);
+                }
                 for (long t = 0; t < HW; ++t) cn[t] += bn * zn[t];
                 if (n + 1 < N)
                     for (long t = 0; t < HW; ++t) z[(n + 1) * HW + t] = xn[t] * cn[t];
@@ -1492,14 +1517,16 @@ static void *backward_2d_worker(void *arg)
                     dxn[t] = g[t] * cn[t];
                     e[t] = g[t] * xn[t];
                 }
-                if (j->route == ROUTE_DIRECT) lagged2_direct(e, zn, j->H, j->W, tmp);
-                else corr2_fft(e, zn, j->H, j->W, tmp, &s);
+                if (j->route == ROUTE_FFT) corr2_fft(e, zn, j->H, j->W, tmp, &s);
+                else if (j->circular) ccorr2_direct(e, zn, j->H, j->W, tmp);
+                else lagged2_direct(e, zn, j->H, j->W, tmp);
                 for (long t = 0; t < HW; ++t) dhn[t] += tmp[t];
                 double db = 0.0;
                 for (long t = 0; t < HW; ++t) db += e[t] * zn[t];
                 j->dbias[n * C + ch] += db;
-                if (j->route == ROUTE_DIRECT) corr2_direct(hn, e, j->H, j->W, tmp);
-                else corr2_fft(e, hn, j->H, j->W, tmp, &s);
+                if (j->route == ROUTE_FFT) corr2_fft(e, hn, j->H, j->W, tmp, &s);
+                else if (j->circular) ccorr2_direct(e, hn, j->H, j->W, tmp);
+                else corr2_direct(hn, e, j->H, j->W, tmp);
                 for (long t = 0; t < HW; ++t) g[t] = tmp[t] + bn * e[t];
             }
             memcpy(j->dv + img * HW, g, sizeof(double) * HW);
@@ -1515,9 +1542,34 @@ done:
 /* Gradients of a scalar loss with dL/dy = dy [B][C][H][W] through the 2-D
  * recurrence: dv [B][C][H][W], dx [N][B][C][H][W], dh [N][C][H][W] and
  * dbias [N][C] (both summed over the batch). */
+static int backward_2d_any(const double *v, const double *x, const double *h, const double *bias,
+                           const double *dy, long B, long C, long H, long W, long N, int route,
+                           int nthreads, int circular, double *dv, double *dx, double *dh, double *dbias);
+
 int oracle_hyena_backward_2d(const double *v, const double *x, const double *h, const double *bias,
                              const double *dy, long B, long C, long H, long W, long N, int route,
                              int nthreads, double *dv, double *dx, double *dh, double *dbias)
+{
+    return backward_2d_any(v, x, h, bias, dy, B, C, H, W, N, route, nthreads, 0, dv, dx, dh, dbias);
+}
+
+/* The same gradients through the 2-D recurrence with circular convolutions
+ * on the H x W grid itself (oracle_hyena_forward_circular_nd with Z = 1):
+ * dh_n[a][b] = sum_b' sum_{t,s} e[t][s] z_{n-1}[(t - a) mod H][(s - b) mod W],
+ * dz_{n-1}[u][w] = sum_{t,s} h_n[(t - u) mod H][(s - w) mod W] e[t][s] +
+ * b_n e[u][w].  H, W powers of two for the FFT route. */
+int oracle_hyena_backward_circular_2d(const double *v, const double *x, const double *h,
+                                      const double *bias, const double *dy, long B, long C, long H,
+                                      long W, long N, int route, int nthreads, double *dv, double *dx,
+                                      double *dh, double *dbias)
+{
+    if (route == ROUTE_FFT && (!is_pow2(H) || !is_pow2(W))) return ORACLE_EBADARG;
+    return backward_2d_any(v, x, h, bias, dy, B, C, H, W, N, route, nthreads, 1, dv, dx, dh, dbias);
+}
+
+static int backward_2d_any(const double *v, const double *x, const double *h, const double *bias,
+                           const double *dy, long B, long C, long H, long W, long N, int route,
+                           int nthreads, int circular, double *dv, double *dx, double *dh, double *dbias)
 {
     if (!v || !x || !h || !bias || !dy || !dv || !dx || !dh || !dbias || B < 1 || C < 1 || H < 1 ||
         W < 1 || N < 1 || (route != ROUTE_DIRECT && route != ROUTE_FFT))
@@ -1528,7 +1580,7 @@ int oracle_hyena_backward_2d(const double *v, const double *x, const double *h, 
     pthread_t *tid = calloc(nthreads, sizeof(pthread_t));
     if (!jobs || !tid) { free(jobs); free(tid); return ORACLE_ENOMEM; }
     for (int k = 0; k < nthreads; ++k) {
-        bwd2_job jb = {v, x, h, bias, dy, B, C, H, W, N, route, dv, dx, dh, dbias, k, nthreads, 0};
+        bwd2_job jb = {v, x, h, bias, dy, B, C, H, W, N, route, dv, dx, dh, dbias, k, nthreads, 0, circular};
         jobs[k] = jb;
         pthread_create(&tid[k], NULL, backward_2d_worker, &jobs[k]);
     }

@@ -286,3 +286,63 @@ def test_backward_2d_per_sample_with_equal_sets_sums_to_the_shared_backward():
     pv, px, ph, pb = oracle.hyena_backward_2d_per_sample(v, x, np.broadcast_to(h, (B,) + h.shape), b, dy)
     assert rel_err(pv, dv) < 1e-13 and rel_err(px, dx) < 1e-13
     assert rel_err(ph.sum(axis=0), dh) < 1e-12 and rel_err(pb, db) < 1e-12
+
+
+# ------------------------------------------------- circular 2-D
+
+@pytest.mark.parametrize("N", [1, 2])
+def test_backward_circular_2d_matches_finite_differences(N):
+    v, x, h, b, dy = problem_2d(2, 2, 4, 4, N, seed=50 + N)
+    dv, dx, dh, db = oracle.hyena_backward_circular_2d(v, x, h, b, dy, route="direct")
+
+    def loss(v_, x_, h_, b_):
+        return float(np.sum(dy * oracle.hyena_forward_circular_nd(v_, x_, h_, b_, route="direct")))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name
+
+
+def test_backward_circular_2d_routes_agree_and_db_is_dh_origin():
+    v, x, h, b, dy = problem_2d(2, 3, 16, 8, 2, seed=53)
+    d = oracle.hyena_backward_circular_2d(v, x, h, b, dy, route="direct")
+    f = oracle.hyena_backward_circular_2d(v, x, h, b, dy, route="fft")
+    for a, c in zip(d, f):
+        assert rel_err(c, a) < 1e-12
+    assert rel_err(d[3], d[2][:, :, 0, 0]) < 1e-13
+
+
+def test_backward_circular_2d_on_zero_padded_grids_is_the_linear_backward():
+    # 2H x 2W grids with v, x_n, dy and h_n zero outside [0, H) x [0, W):
+    # nothing wraps, so the gradients there are the linear 2-D backward's
+    B, C, H, W, N = 2, 2, 4, 8, 2
+    v, x, h, b, dy = problem_2d(B, C, H, W, N, seed=54)
+
+    def pad(a):
+        out = np.zeros(a.shape[:-2] + (2 * H, 2 * W))
+        out[..., :H, :W] = a
+        return out
+    dv, dx, dh, db = oracle.hyena_backward_circular_2d(pad(v), pad(x), pad(h), b, pad(dy))
+    rv, rx, rh, rb = oracle.hyena_backward_2d(v, x, h, b, dy)
+    assert rel_err(dv[..., :H, :W], rv) < 1e-12 and rel_err(dx[..., :H, :W], rx) < 1e-12
+    assert rel_err(dh[..., :H, :W], rh) < 1e-12 and rel_err(db, rb) < 1e-12
+
+
+def test_backward_circular_2d_of_one_row_is_the_circular_1d_backward():
+    # H = 1: the 2-D circular recurrence is the 1-D one along the row
+    B, C, W, N = 2, 3, 16, 2
+    v, x, h, b, dy = problem(B, C, W, N, seed=55)
+    g2 = oracle.hyena_backward_circular_2d(v[:, :, None], x[:, :, :, None], h[:, :, None], b, dy[:, :, None])
+    g1 = oracle.hyena_backward_circular(v, x, h, b, dy)
+    for a, c in zip(g2[:3], g1[:3]):
+        assert rel_err(a[..., 0, :], c) < 1e-12
+    assert rel_err(g2[3], g1[3]) < 1e-12
