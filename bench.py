@@ -107,8 +107,8 @@ def alg_bytes_backward(wl: synth.Workload) -> int:
     act = wl.positions * io
     if wl.film:             # spectra in and dh out per sample
         return (2 * wl.N + 3) * act + wl.B * wl.N * wl.D * wl.L * (8 + 4) + wl.N * wl.D * 4
-    if wl.circular:         # L/2 spectrum slots a filter, L lags of dh
-        return (2 * wl.N + 3) * act + wl.N * wl.D * wl.L * (4 + 4) + wl.N * wl.D * 4
+    if wl.circular:         # half a spectrum slot and one dh value per position
+        return (2 * wl.N + 3) * act + wl.N * wl.D * wl.per_channel * (4 + 4) + wl.N * wl.D * 4
     if wl.kind == "2d":     # 2H x W spectrum slots a filter, H x W of dh
         return (2 * wl.N + 3) * act + wl.N * wl.D * wl.H * wl.W * (16 + 4) + wl.N * wl.D * 4
     return (2 * wl.N + 3) * act + wl.N * wl.D * wl.L * (8 + 4) + wl.N * wl.D * 4
@@ -542,10 +542,18 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
 
     # ---- the backward pass (1-D and 2-D): one call per timed repetition
     bwd = None
-    if ((wl.kind == "1d" and not (wl.film and long_path(wl)))
-            or (wl.kind == "2d" and not wl.circular and not wl.film)):
+    if wl.kind == "1d" or (wl.kind == "2d" and not wl.film):
         dy = to_dev(synth.make_output_grad(wl), io)
-        if wl.circular:
+        if wl.circular and wl.kind == "2d":
+            ws_b = torch.empty(hyena.hyena_fftconv2d_backward_circular_workspace_size(wl.B, wl.D, wl.H, wl.W,
+                                                                                      wl.N),
+                               device="cuda", dtype=torch.uint8)
+            bwd_kernel = ("fft2d_bwd_row_kernel+fft2d_bwd_col_kernel<PAD=false> "
+                          "(hyena_fftconv2d_gate_backward_circular, all launches)")
+
+            def backward():
+                hyena.hyena_fftconv2d_gate_backward_circular(v, xs, b, H, dy, workspace=ws_b)
+        elif wl.circular:
             ws_b = torch.empty(hyena.hyena_fftconv_backward_circular_workspace_size(wl.D, wl.L, wl.N),
                                device="cuda", dtype=torch.uint8)
             bwd_kernel = "backward1d_kernel<PAD=false> (hyena_fftconv_gate_backward_circular)"

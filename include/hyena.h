@@ -312,12 +312,14 @@ HYENA_API hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* 
  *          dh_n[b][d][s] = sum_t e[t] z_{n-1}[t-s] of sequence (b, d)
  *   dbias  [N][D] float32 out, summed over the batch (the bias is shared)
  *   workspace: hyena_fftconv_backward_per_sample_workspace_size(B, D, L, N)
- *          bytes (8 B N D L + 12 N D L), 256-byte aligned.
- * Everything else as hyena_fftconv_gate_backward.  L <= 16384 (else
- * HYENA_ERR_UNSUPPORTED; the size function returns (size_t)-1).  Two
- * launches, deterministic: a group of threads per channel walks its B
- * sequences, each with its own dh spectrum; the second launch inverts the
- * B spectra of each (n, d) and sums their lag-0 values into dbias. */
+ *          bytes (8 B N D L + 12 N D L for L <= 16384; above, the
+ *          four-step backward's with B times the dh spectra), 256-byte
+ *          aligned.
+ * Everything else, L up to 2^22 included, as hyena_fftconv_gate_backward.
+ * Deterministic: each sequence has its own dh spectrum; L <= 16384 takes
+ * two launches (the second inverts the B spectra of each (n, d) and sums
+ * their lag-0 values into dbias), longer L the four-step launches plus one
+ * that sums dbias. */
 HYENA_API size_t hyena_fftconv_backward_per_sample_workspace_size(int B, int D, int L, int N);
 HYENA_API hyena_status_t hyena_fftconv_gate_backward_per_sample(const void* v, const void* const* x,
                                                                 const float* H, const float* bias,
@@ -555,6 +557,45 @@ HYENA_API hyena_status_t hyena_fftconv2d_gate_backward(const void* v, const void
                                                        int W, int N, hyena_dtype_t io, void* dv,
                                                        void* const* dx, float* dh, float* dbias,
                                                        void* workspace, size_t ws_bytes, void* stream);
+
+/* The 2-D backward with a spectrum set per sample (input-dependent filters,
+ * see hyena_filter_gen_film_2d and hyena_fftconv2d_gate_forward_per_sample):
+ * image (b, c) uses sample b's filters, so
+ *   Hs     [B][N][C][2H][W] (sample b's set at Hs + b*N*C*2H*W)
+ *   dh     [B][N][C][H][W] float32 out, per sample (no sum over the batch)
+ *   dbias  [N][C] float32 out, summed over the batch (the bias is shared)
+ *   workspace: hyena_fftconv2d_backward_per_sample_workspace_size(...)
+ *          bytes (B times the dh spectra of the shared backward),
+ *          256-byte aligned.
+ * Everything else as hyena_fftconv2d_gate_backward; deterministic, one
+ * more launch sums dbias over the samples in order. */
+HYENA_API size_t hyena_fftconv2d_backward_per_sample_workspace_size(int B, int C, int H, int W, int N);
+HYENA_API hyena_status_t hyena_fftconv2d_gate_backward_per_sample(const void* v, const void* const* x,
+                                                                  const float* Hs, const float* bias,
+                                                                  const void* dy, int B, int C, int H, int W,
+                                                                  int N, hyena_dtype_t io, void* dv,
+                                                                  void* const* dx, float* dh, float* dbias,
+                                                                  void* workspace, size_t ws_bytes,
+                                                                  void* stream);
+
+/* The backward of the circular 2-D recurrence (hyena_fftconv2d_gate_forward_
+ * circular), for training: the exact adjoint with every 2-D convolution
+ * circular on the H x W grid, so both correlations wrap around:
+ *   dh_n[c][a][b] = sum_b' sum_{t,s} e[t][s] z_{n-1}[(t - a) mod H][(s - b) mod W],
+ *   db_n[c] = dh_n[c][0][0],
+ *   dz_{n-1}[u][w] = sum_{t,s} h_n[(t - u) mod H][(s - w) mod W] e[t][s] + b_n e[u][w].
+ * Arguments as hyena_fftconv2d_gate_backward with Hs [N][C][H][W/2] from
+ * hyena_filter_rfft2d_circular, dh [N][C][H][W] and dbias [N][C] summed
+ * over the batch, and a workspace of
+ * hyena_fftconv2d_backward_circular_workspace_size(...) bytes, 256-byte
+ * aligned.  H a power of two in [16, 1024], W in [32, 1024]. */
+HYENA_API size_t hyena_fftconv2d_backward_circular_workspace_size(int B, int C, int H, int W, int N);
+HYENA_API hyena_status_t hyena_fftconv2d_gate_backward_circular(const void* v, const void* const* x,
+                                                                const float* Hs, const float* bias,
+                                                                const void* dy, int B, int C, int H, int W,
+                                                                int N, hyena_dtype_t io, void* dv,
+                                                                void* const* dx, float* dh, float* dbias,
+                                                                void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

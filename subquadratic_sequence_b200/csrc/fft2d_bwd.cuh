@@ -29,6 +29,11 @@
 // Slot 0 (bins 0 and W of the row transform, packed as one complex
 // number) is separated and re-packed through the pair (ky, 2H - ky) as in
 // the forward column step.
+//
+// Per-sample spectra (f.Hs_bstride != 0, input-dependent filters): image
+// (b, c) reads sample b's spectra and owns its own dh spectrum (acc
+// [B][N][C][2H][W]), so dh is [B][N][C][H][W]; the shared bias's db_n =
+// sum_b dh_{b,n}[0][0] is summed by a last small launch.
 #pragma once
 
 #include "fft2d.cuh"
@@ -42,9 +47,10 @@ struct Bwd2dArgs {
     void* dx[kMaxOrder];           // [B][C][H][W] io each
     float2* zsave;                 // [N][wcap][2H][W] spectra of z_n (the wave's images)
     float* csave;                  // [N][wcap][H][W] c_n
-    float2* acc;                   // [N][C][2H][W] accumulated dh spectra
-    float* dh;                     // [N][C][H][W]
+    float2* acc;                   // [N][C][2H][W] accumulated dh spectra ([B][N][C][2H][W] per sample)
+    float* dh;                     // [N][C][H][W] ([B][N][C][H][W] per sample)
     float* dbias;                  // [N][C]
+    int N;                         // order
     int wcap;                      // images a wave holds
     int first;                     // rows MODE 1: g = dy (the last order), else g from the scratch
     int last;                      // rows MODE 0: the last order (c_n saved, no gate, no forward rows)
@@ -66,13 +72,13 @@ __device__ __forceinline__ T pick_order(T const* arr, int n)
 // the inverse rows of the scratch; dx_n = g c_n; e = g x_n; forward rows of
 // e.  MODE 2: dv = inverse rows of the scratch.  MODE 3: dh rows from the
 // accumulated spectra (rows y < H after the inverse columns), db = dh[0][0].
-template <int LOG2W, typename IO, int MODE>
-__global__ void __launch_bounds__(Fft1d<LOG2W>::THREADS)
+template <int LOG2W, typename IO, int MODE, bool PAD = true>
+__global__ void __launch_bounds__(Fft1d<LOG2W, PAD>::THREADS)
 fft2d_bwd_row_kernel(Bwd2dArgs ba)
 {
     grid_dependency_begin();
     const Fft2dArgs& a = ba.f;
-    using R = Fft2dRows<LOG2W>;
+    using R = Fft2dRows<LOG2W, PAD>;
     using F = typename R::F;
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;
@@ -91,13 +97,13 @@ fft2d_bwd_row_kernel(Bwd2dArgs ba)
 
     if constexpr (MODE == 3) {
         // q: filter row n*C + c of the accumulated spectra [2H][W]
-        const float2* row = ba.acc + ((size_t)q * 2 * a.H + yrow) * W;
+        const float2* row = ba.acc + ((size_t)q * (PAD ? 2 : 1) * a.H + yrow) * W;
         R::unsplit_inverse(arr, sm, row, t);
         if (active) {
             float2* dhp = reinterpret_cast<float2*>(ba.dh + ((size_t)q * a.H + yrow) * 2 * SEQ);
             F::for_each_io(t, [&](int i, int m) {
                 dhp[m] = arr[i];
-                if (yrow == 0 && m == 0) ba.dbias[q] = arr[i].x;       // db_n = dh_n[0][0]
+                if (yrow == 0 && m == 0 && a.Hs_bstride == 0) ba.dbias[q] = arr[i].x;   // db_n = dh_n[0][0]
             });
         }
         return;
@@ -105,7 +111,7 @@ fft2d_bwd_row_kernel(Bwd2dArgs ba)
         const int c = q / a.B, b = q % a.B;
         const size_t img = (size_t)b * a.C + c;
         const size_t off = (img * a.H + yrow) * SEQ;             // value pairs of this grid row
-        float2* row = scratch_row<true>(a, qi, yrow);
+        float2* row = scratch_row<PAD>(a, qi, yrow);
         float2* cs = reinterpret_cast<float2*>(ba.csave) + (((size_t)a.n * ba.wcap + qi) * a.H + yrow) * SEQ;
         const PT* xp = reinterpret_cast<const PT*>(pick_order(a.x, a.n)) + off;
         if constexpr (MODE == 0) {
@@ -128,8 +134,9 @@ fft2d_bwd_row_kernel(Bwd2dArgs ba)
             PT* dxp = reinterpret_cast<PT*>(pick_order(ba.dx, a.n)) + off;
             // all loads first, then the stores: one latency, not one per value
             constexpr int RF = F::P::RF;
-            auto io_slot = [](int i) { return (i / RF) * (RF / 2) + i % RF; };   // io register -> [0, E/2)
-            float2 cv[E / 2], xv[E / 2];
+            constexpr int NIO = PAD ? E / 2 : E;                     // io registers
+            auto io_slot = [](int i) { return PAD ? (i / RF) * (RF / 2) + i % RF : i; };   // -> [0, NIO)
+            float2 cv[NIO], xv[NIO];
             F::for_each_io(t, [&](int i, int m) {
                 cv[io_slot(i)] = cs[m];
                 xv[io_slot(i)] = IOP::load(xp + m);
@@ -158,15 +165,17 @@ fft2d_bwd_row_kernel(Bwd2dArgs ba)
 // by (conj(H_n) + b_n) / 2H, inverse columns, rows y < H back.  MODE 2:
 // inverse columns of the accumulated spectra (all 2H rows), scaled by
 // 1/2H, rows y < H back in place.
-template <int LOG2H2, int MODE>
-__global__ void __launch_bounds__(Fft2dCols<LOG2H2>::THREADS, Fft2dCols<LOG2H2>::MIN_BLOCKS)
+template <int LOG2H2, int MODE, bool PAD = true>
+__global__ void __launch_bounds__(Fft2dCols<LOG2H2, PAD>::THREADS, Fft2dCols<LOG2H2, PAD>::MIN_BLOCKS)
 fft2d_bwd_col_kernel(Bwd2dArgs ba)
 {
     grid_dependency_begin();
     const Fft2dArgs& a = ba.f;
-    using CL = Fft2dCols<LOG2H2>;
+    using CL = Fft2dCols<LOG2H2, PAD>;
     using FC = typename CL::FC;
     constexpr int H2 = CL::H2, TC = CL::TC, HH = H2 / 2, V = FC::V;
+    constexpr int ROWS = PAD ? HH : H2;                 // grid rows in a column
+    constexpr int VL = PAD ? V / 2 : V;                 // registers holding grid rows
     constexpr float s = 1.0f / (float)H2;
     const int W = a.W;
     const int CTAS_PER_ROW = W / TC;
@@ -187,7 +196,7 @@ fft2d_bwd_col_kernel(Bwd2dArgs ba)
         });
         __syncthreads();
         FC::template run<+1, true>(buf, reg, t);
-        static_for<V / 2>([&](auto rr) {
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             col[(size_t)(t + r * (H2 / V)) * W] = make_float2(reg[r].x * s, reg[r].y * s);
         });
@@ -205,18 +214,21 @@ fft2d_bwd_col_kernel(Bwd2dArgs ba)
             qb = min(a.q0 + a.nq, (c + 1) * a.B);
         }
         const float bias = __ldg(a.bias + a.n * a.C + c);
-        const float2* Hc = a.Hs + ((size_t)a.n * a.C + c) * H2 * W + kx;
-        float2* accc = ba.acc + ((size_t)a.n * a.C + c) * H2 * W + kx;
+        const bool ps = a.Hs_bstride != 0;
         for (int q = qa; q < qb; ++q) {
             const int qi = q - a.q0;
-            float2* col = a.S + (size_t)qi * HH * W + kx;
+            // per-sample spectra: sample b's filters and its own dh spectrum
+            const size_t sb = ps ? (size_t)(q % a.B) : 0;
+            const float2* Hc = a.Hs + sb * a.Hs_bstride + ((size_t)a.n * a.C + c) * H2 * W + kx;
+            float2* accc = ba.acc + ((sb * ba.N + a.n) * a.C + c) * H2 * W + kx;
+            float2* col = a.S + (size_t)qi * ROWS * W + kx;
             float2* zc = ba.zsave + ((size_t)a.n * ba.wcap + qi) * H2 * W + kx;
-            static_for<V / 2>([&](auto rr) {
+            static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
                 buf[pad16_at<H2 / V>(t, pt, r)] = col[(size_t)(t + r * (H2 / V)) * W];
             });
             __syncthreads();
-            FC::template run<-1, true, true>(buf, reg, t);
+            FC::template run<-1, true, PAD>(buf, reg, t);
             if constexpr (MODE == 0)
                 static_for<V>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
@@ -232,17 +244,30 @@ fft2d_bwd_col_kernel(Bwd2dArgs ba)
             // (runtime loops over the thread's rows: fully unrolled, the
             // compiler hoists every load and runs out of registers)
             if (kx != 0) {
-#pragma unroll 2
-                for (int r = 0; r < V; ++r) {
-                    const int ky = t + r * (H2 / V);
-                    const int pk = pad16(ky);
-                    const float2 ev = buf[pk];
-                    if constexpr (MODE == 1) {
-                        const float2 zv = zc[(size_t)ky * W];
-                        accc[(size_t)ky * W] = cadd(accc[(size_t)ky * W], cmulc(ev, zv));
-                    }
-                    const float2 hv = __ldg(Hc + (size_t)ky * W);
-                    buf[pk] = cmul(ev, make_float2((hv.x + bias) * s, cj * hv.y * s));
+                // K rows at a time, every load of the group before its stores:
+                // interleaved, each accumulator load would wait for the store
+                // before it
+                constexpr int K = 4;
+                static_assert(V % K == 0, "row groups");
+#pragma unroll 1
+                for (int r0 = 0; r0 < V; r0 += K) {
+                    float2 ev[K], hv[K], zv[K], av[K];
+                    static_for<K>([&](auto jj) {
+                        constexpr int j = decltype(jj)::value;
+                        const int ky = t + (r0 + j) * (H2 / V);
+                        ev[j] = buf[pad16(ky)];
+                        hv[j] = __ldg(Hc + (size_t)ky * W);
+                        if constexpr (MODE == 1) {
+                            zv[j] = zc[(size_t)ky * W];
+                            av[j] = accc[(size_t)ky * W];
+                        }
+                    });
+                    static_for<K>([&](auto jj) {
+                        constexpr int j = decltype(jj)::value;
+                        const int ky = t + (r0 + j) * (H2 / V);
+                        if constexpr (MODE == 1) accc[(size_t)ky * W] = cadd(av[j], cmulc(ev[j], zv[j]));
+                        buf[pad16(ky)] = cmul(ev[j], make_float2((hv[j].x + bias) * s, cj * hv[j].y * s));
+                    });
                 }
             } else {
                 // slot 0 = (bin-0 column) + i (bin-W column): separate both
@@ -276,12 +301,26 @@ fft2d_bwd_col_kernel(Bwd2dArgs ba)
             }
             __syncthreads();
             FC::template run<+1, true>(buf, reg, t);
-            static_for<V / 2>([&](auto rr) {
+            static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
                 col[(size_t)(t + r * (H2 / V)) * W] = reg[r];
             });
         }
     }
+}
+
+// Per-sample spectra: db_n[c] = sum_b dh_{b,n}[c][0][0], one thread per
+// (n, c), the samples in order (deterministic).
+static __global__ void __launch_bounds__(256) db2d_sum_kernel(Bwd2dArgs ba)
+{
+    grid_dependency_begin();
+    const int rows = ba.N * ba.f.C;
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    const size_t plane = (size_t)ba.f.H * ba.f.W;
+    float s = 0.0f;
+    for (int b = 0; b < ba.f.B; ++b) s += ba.dh[((size_t)b * rows + r) * plane];
+    ba.dbias[r] = s;
 }
 
 }  // namespace hyena

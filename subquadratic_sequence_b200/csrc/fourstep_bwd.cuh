@@ -29,6 +29,11 @@
 // After the last wave each accumulated spectrum (packed like the filter
 // spectra) is re-packed, inverse-transformed by rows and columns, and
 // cropped: dh_n, and db_n = dh_n[0].
+//
+// Per-sample spectra (f.H_bstride != 0, input-dependent filters): sequence
+// (b, d) reads sample b's H and owns its own dh spectrum (acc [B][N][D][M]),
+// so dh is [B][N][D][L]; the shared bias's db_n = sum_b dh_{b,n}[0] is
+// summed by a last small launch.
 #pragma once
 
 #include "fourstep.cuh"
@@ -43,8 +48,9 @@ struct FourStepBwdArgs {
     float2* zsave;                 // [N][wcap][M1][RS] row-transformed spectra of z_n, rows in the
                                    // padded shared-memory layout (RS = the row kernel's row stride)
     float2* csave;                 // [N][wcap][M/2] c_n (value pairs)
-    float2* acc;                   // [N][D][M] accumulated dh spectra (packed like H)
-    float* dh;                     // [N][D][L]
+    float2* acc;                   // [N][D][M] accumulated dh spectra (packed like H); [B][N][D][M]
+                                   // with per-sample spectra
+    float* dh;                     // [N][D][L] ([B][N][D][L] with per-sample spectra)
     float* dbias;                  // [N][D]
     int wcap;                      // sequences a wave holds
     int nq;                        // sequences (or filter rows) in this wave
@@ -167,7 +173,7 @@ fourstep_bwd_row_kernel(FourStepBwdArgs ba)
         __syncthreads();
         forward_rows(ba.zsave + ((size_t)a.n * ba.wcap + qi) * M1 * RS);
         const float bias = __ldg(a.bias + a.n * a.D + d);
-        const float2* Hr = a.H + ((size_t)a.n * a.D + d) * M;
+        const float2* Hr = a.H + (size_t)(q % a.B) * a.H_bstride + ((size_t)a.n * a.D + d) * M;
         FS::for_each_pair(smem_fb, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2 w) {
             float2 z1 = *p1, z2 = *p2;
             if (kind == 1) {
@@ -185,10 +191,13 @@ fourstep_bwd_row_kernel(FourStepBwdArgs ba)
         const int d = a.q0 / a.B + unit;
         const int qa = max(a.q0, d * a.B), qb = min(a.q0 + ba.nq, (d + 1) * a.B);
         const float bias = __ldg(a.bias + a.n * a.D + d);
-        const float2* Hr = a.H + ((size_t)a.n * a.D + d) * M;
-        float2* Ar = ba.acc + ((size_t)a.n * a.D + d) * M;
+        const bool ps = a.H_bstride != 0;
         for (int q = qa; q < qb; ++q) {
             const int qi = q - a.q0;
+            // per-sample spectra: sample b's H and its own dh spectrum
+            const size_t sb = ps ? (size_t)(q % a.B) : 0;
+            const float2* Hr = a.H + sb * a.H_bstride + ((size_t)a.n * a.D + d) * M;
+            float2* Ar = ba.acc + ((sb * (a.n_last + 1) + a.n) * a.D + d) * M;
             float2* Sq = a.S + (size_t)qi * M;
             stage_rows(Sq, 0, M2);
             stage_rows(ba.zsave + ((size_t)a.n * ba.wcap + qi) * M1 * RS, FB::ZOFF, RS);
@@ -285,7 +294,7 @@ fourstep_bwd_col_kernel(FourStepBwdArgs ba)
             constexpr int r = decltype(rr)::value;
             dhp[at(r)] = reg[r];
         });
-        if (n2 == 0 && t == 0) ba.dbias[q] = reg[0].x;          // db_n = dh_n[0]
+        if (n2 == 0 && t == 0 && a.H_bstride == 0) ba.dbias[q] = reg[0].x;   // db_n = dh_n[0]
         return;
     } else {
         const size_t cso = ((size_t)a.n * ba.wcap + qi) * (M / 2);
@@ -349,6 +358,20 @@ fourstep_bwd_col_kernel(FourStepBwdArgs ba)
             if constexpr (r < V1 - 1) w = cmul(w, step);
         });
     }
+}
+
+// Per-sample spectra: db_n[d] = sum_b dh_{b,n}[d][0] over dh rows of L
+// floats, one thread per (n, d), the samples in order (deterministic).
+template <int L>
+__global__ void __launch_bounds__(256) dbias_sum_kernel(FourStepBwdArgs ba)
+{
+    grid_dependency_begin();
+    const int rows = (ba.f.n_last + 1) * ba.f.D;
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    float s = 0.0f;
+    for (int b = 0; b < ba.f.B; ++b) s += ba.dh[((size_t)b * rows + r) * L];
+    ba.dbias[r] = s;
 }
 
 }  // namespace hyena

@@ -122,6 +122,11 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
                              bool circular, const float* bias, const void* dy, int B, int D, int L, int N,
                              hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
                              void* workspace, size_t ws_bytes, void* stream);
+hyena_status_t backward2d_impl(const void* v, const void* const* x, const float* Hs, bool per_sample,
+                               bool circular, const float* bias, const void* dy, int B, int C, int H, int W,
+                               int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
+                               void* workspace, size_t ws_bytes, void* stream);
+bool dims2d_circ_ok(int H, int W, int& lh, int& lm);
 hyena_status_t forward3d_impl(const void* v, const void* const* x, const float* h, const float* Hs,
                               bool per_sample, const float* bias, int B, int C, int Z, int H, int W,
                               int N, hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes,
@@ -443,8 +448,9 @@ size_t hyena_fftconv_backward_workspace_size(int D, int L, int N)
 size_t hyena_fftconv_backward_per_sample_workspace_size(int B, int D, int L, int N)
 {
     int log2m = 0;
-    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2Fused, &log2m) != HYENA_OK)
+    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2, &log2m) != HYENA_OK)
         return (size_t)-1;
+    if (log2m > kMaxLog2Fused) return fourstep_bwd_layout(log2m, D, N, B).total;
     const size_t spec = sizeof(float2) * (size_t)N * D * L;
     return round_up(spec * B, 256) + round_up(spec, 256) + round_up(spec / 2, 256);   // acc, wz, wc
 }
@@ -508,7 +514,7 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
         if (k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1) return HYENA_ERR_UNSUPPORTED;
         log2m = k - 1;                       // M = L/2 packed points
     } else {
-        hyena_status_t s = check_len(L, per_sample ? kMaxLog2Fused : kMaxLog2, &log2m);
+        hyena_status_t s = check_len(L, kMaxLog2, &log2m);
         if (s != HYENA_OK) return s;
     }
     if ((long)B * D > (1L << 30) || (per_sample && (long)B * N * D > (1L << 30))) return HYENA_ERR_UNSUPPORTED;
@@ -550,7 +556,7 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
     cudaStream_t st = (cudaStream_t)stream;
     if (!circular && log2m > kMaxLog2Fused) {
         // four-step backward (L > 16384)
-        const FourStepBwdLayout lay = fourstep_bwd_layout(log2m, D, N);
+        const FourStepBwdLayout lay = fourstep_bwd_layout(log2m, D, N, (int)sets);
         FourStepBwdArgs b = {};
         b.f.v = v;
         for (int n = 0; n < kMaxOrder; ++n) {
@@ -558,6 +564,7 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
             b.dx[n] = n < N ? dx[n] : nullptr;
         }
         b.f.H = reinterpret_cast<const float2*>(H);
+        b.f.H_bstride = per_sample ? (size_t)N * D * L : 0;
         b.f.bias = bias;
         b.f.S = reinterpret_cast<float2*>(ws + lay.scratch);
         b.f.B = B;
@@ -1058,16 +1065,19 @@ struct Bwd2dLayout {
     long wcap;
 };
 
-Bwd2dLayout bwd2d_layout(int B, int C, int H, int W, int N)
+// sets: dh spectra per (n, c): B with per-sample spectra, else 1.
+// circular: H x W/2 spectrum slots and scratch rows of W/2 slots
+Bwd2dLayout bwd2d_layout(int B, int C, int H, int W, int N, int sets = 1, bool circular = false)
 {
     Bwd2dLayout l;
-    l.wcap = wave_images((long)B * C, H, W);
-    const size_t slots = (size_t)2 * H * W;                  // 2H x W spectrum slots
+    const int Ws = circular ? W / 2 : W;                      // slots per row
+    l.wcap = wave_images((long)B * C, H, Ws);
+    const size_t slots = (size_t)(circular ? 1 : 2) * H * Ws; // 2H x W (padded) or H x W/2 spectrum slots
     l.acc = 0;
-    l.zsave = l.acc + round_up(sizeof(float2) * (size_t)N * C * slots, 256);
+    l.zsave = l.acc + round_up(sizeof(float2) * (size_t)sets * N * C * slots, 256);
     l.csave = l.zsave + round_up(sizeof(float2) * (size_t)N * l.wcap * slots, 256);
     l.scratch = l.csave + round_up(sizeof(float) * (size_t)N * l.wcap * H * W, 256);
-    l.total = l.scratch + round_up(sizeof(float2) * (size_t)l.wcap * H * W, 256);
+    l.total = l.scratch + round_up(sizeof(float2) * (size_t)l.wcap * H * Ws, 256);
     return l;
 }
 
@@ -1083,25 +1093,81 @@ size_t hyena_fftconv2d_backward_workspace_size(int B, int C, int H, int W, int N
     return bwd2d_layout(B, C, H, W, N).total;
 }
 
+size_t hyena_fftconv2d_backward_per_sample_workspace_size(int B, int C, int H, int W, int N)
+{
+    if (B < 1 || C < 1 || N < 1 || N > HYENA_MAX_ORDER) return (size_t)-1;
+    const int lh = exact_log2(H), lw = exact_log2(W);
+    if (lh < kMinLog2H2d || lh > kMaxLog2H2d || lw < kMinLog2W2d || lw > kMaxLog2W2d) return (size_t)-1;
+    return bwd2d_layout(B, C, H, W, N, B).total;
+}
+
 hyena_status_t hyena_fftconv2d_gate_backward(const void* v, const void* const* x, const float* Hs,
                                              const float* bias, const void* dy, int B, int C, int H, int W,
                                              int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh,
                                              float* dbias, void* workspace, size_t ws_bytes, void* stream)
 {
+    return backward2d_impl(v, x, Hs, false, false, bias, dy, B, C, H, W, N, io, dv, dx, dh, dbias, workspace,
+                           ws_bytes, stream);
+}
+
+size_t hyena_fftconv2d_backward_circular_workspace_size(int B, int C, int H, int W, int N)
+{
+    int lh, lm;
+    if (B < 1 || C < 1 || N < 1 || N > HYENA_MAX_ORDER || !dims2d_circ_ok(H, W, lh, lm)) return (size_t)-1;
+    return bwd2d_layout(B, C, H, W, N, 1, true).total;
+}
+
+hyena_status_t hyena_fftconv2d_gate_backward_circular(const void* v, const void* const* x, const float* Hs,
+                                                      const float* bias, const void* dy, int B, int C, int H,
+                                                      int W, int N, hyena_dtype_t io, void* dv, void* const* dx,
+                                                      float* dh, float* dbias, void* workspace, size_t ws_bytes,
+                                                      void* stream)
+{
+    return backward2d_impl(v, x, Hs, false, true, bias, dy, B, C, H, W, N, io, dv, dx, dh, dbias, workspace,
+                           ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv2d_gate_backward_per_sample(const void* v, const void* const* x, const float* Hs,
+                                                        const float* bias, const void* dy, int B, int C, int H,
+                                                        int W, int N, hyena_dtype_t io, void* dv,
+                                                        void* const* dx, float* dh, float* dbias,
+                                                        void* workspace, size_t ws_bytes, void* stream)
+{
+    return backward2d_impl(v, x, Hs, true, false, bias, dy, B, C, H, W, N, io, dv, dx, dh, dbias, workspace,
+                           ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// per_sample: a spectrum set per sample; circular: the circular recurrence
+// (spectra of H x W/2 slots, hyena_filter_rfft2d_circular)
+hyena_status_t backward2d_impl(const void* v, const void* const* x, const float* Hs, bool per_sample,
+                               bool circular, const float* bias, const void* dy, int B, int C, int H, int W,
+                               int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
+                               void* workspace, size_t ws_bytes, void* stream)
+{
     if (!v || !x || !Hs || !bias || !dy || !dv || !dx || !dh || !dbias) return HYENA_ERR_INVALID_ARG;
     if (B < 1 || C < 1 || N < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
     if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
     if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
-    const int lh = exact_log2(H), lw = exact_log2(W);
-    if (lh < kMinLog2H2d || lh > kMaxLog2H2d || lw < kMinLog2W2d || lw > kMaxLog2W2d)
+    int lh = exact_log2(H), lw = exact_log2(W), lm = 0;
+    if (circular) {
+        if (!dims2d_circ_ok(H, W, lh, lm)) return HYENA_ERR_UNSUPPORTED;
+    } else if (lh < kMinLog2H2d || lh > kMaxLog2H2d || lw < kMinLog2W2d || lw > kMaxLog2W2d) {
         return HYENA_ERR_UNSUPPORTED;
-    if ((long)B * C > (1L << 20) || (long)N * C * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    }
+    const int sets = per_sample ? B : 1;                     // spectrum sets and dh sets
+    const int Ws = circular ? W / 2 : W;                     // spectrum slots per row
+    const int RP = circular ? 1 : 2;                         // spectrum rows per grid row
+    if ((long)B * C > (1L << 20) || (long)sets * N * C * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
     for (int n = 0; n < N; ++n)
         if (!x[n] || !dx[n] || !aligned(x[n], 16) || !aligned(dx[n], 16)) return HYENA_ERR_INVALID_ARG;
     if (!aligned(v, 16) || !aligned(dy, 16) || !aligned(dv, 16) || !aligned(Hs, 16) || !aligned(dh, 16) ||
         !aligned(bias, 4) || !aligned(dbias, 4))
         return HYENA_ERR_INVALID_ARG;
-    const Bwd2dLayout lay = bwd2d_layout(B, C, H, W, N);
+    const Bwd2dLayout lay = bwd2d_layout(B, C, H, W, N, sets, circular);
     if (!workspace || ws_bytes < lay.total || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
 
     // every output against every input, the other outputs and the workspace
@@ -1111,12 +1177,12 @@ hyena_status_t hyena_fftconv2d_gate_backward(const void* v, const void* const* x
     int ni = 0, no = 0;
     in[ni++] = {v, act};
     in[ni++] = {dy, act};
-    in[ni++] = {Hs, sizeof(float2) * (size_t)N * C * 2 * H * W};
+    in[ni++] = {Hs, sizeof(float2) * (size_t)sets * N * C * RP * H * Ws};
     in[ni++] = {bias, sizeof(float) * N * C};
     in[ni++] = {workspace, lay.total};
     for (int n = 0; n < N; ++n) in[ni++] = {x[n], act};
     out[no++] = {dv, act};
-    out[no++] = {dh, sizeof(float) * (size_t)N * C * H * W};
+    out[no++] = {dh, sizeof(float) * (size_t)sets * N * C * H * W};
     out[no++] = {dbias, sizeof(float) * N * C};
     for (int n = 0; n < N; ++n) out[no++] = {dx[n], act};
     for (int o = 0; o < no; ++o) {
@@ -1128,6 +1194,7 @@ hyena_status_t hyena_fftconv2d_gate_backward(const void* v, const void* const* x
 
     char* ws = static_cast<char*>(workspace);
     Bwd2dArgs a = {};
+    a.f.Hs_bstride = per_sample ? (size_t)N * C * RP * H * Ws : 0;
     a.f.v = v;
     for (int n = 0; n < kMaxOrder; ++n) {
         a.f.x[n] = n < N ? x[n] : nullptr;
@@ -1139,7 +1206,7 @@ hyena_status_t hyena_fftconv2d_gate_backward(const void* v, const void* const* x
     a.f.B = B;
     a.f.C = C;
     a.f.H = H;
-    a.f.W = W;
+    a.f.W = Ws;
     a.dy = dy;
     a.dv = dv;
     a.acc = reinterpret_cast<float2*>(ws + lay.acc);
@@ -1149,7 +1216,10 @@ hyena_status_t hyena_fftconv2d_gate_backward(const void* v, const void* const* x
     a.dbias = dbias;
     a.wcap = (int)lay.wcap;
     cudaStream_t st = (cudaStream_t)stream;
+    if (circular)
+        return io == HYENA_BF16 ? dispatch_bwd2d_circ_bf16(lm, lh, a, N, st)
+                                : dispatch_bwd2d_circ_f32(lm, lh, a, N, st);
     return io == HYENA_BF16 ? dispatch_bwd2d_bf16(lw, lh, a, N, st) : dispatch_bwd2d_f32(lw, lh, a, N, st);
 }
 
-}  // extern "C"
+}  // namespace

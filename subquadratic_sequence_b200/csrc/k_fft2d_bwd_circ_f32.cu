@@ -1,0 +1,9 @@
+// 2-D backward pass in circular mode, float32 activations.
+#include "k_fft2d_bwd.cuh"
+
+namespace hyena {
+hyena_status_t dispatch_bwd2d_circ_f32(int log2m, int log2h, const Bwd2dArgs& a, int N, cudaStream_t st)
+{
+    return dispatch_bwd2d_circ<float>(log2m, log2h, a, N, st);
+}
+}  // namespace hyena

@@ -10,22 +10,23 @@ namespace hyena {
 // sequences a wave of the four-step backward holds (the forward's scratch budget)
 inline long bwd_wave_cap(long M) { return wave_seqs(1L << 30, M); }
 
-// Workspace layout of the four-step backward (bytes): acc [N][D][M], zsave
-// [N][wcap][M1][RS], csave [N][wcap][M/2], scratch [wcap][M].
+// Workspace layout of the four-step backward (bytes): acc [sets][N][D][M]
+// (sets = B with per-sample spectra, else 1), zsave [N][wcap][M1][RS],
+// csave [N][wcap][M/2], scratch [wcap][M].
 struct FourStepBwdLayout {
     size_t acc, zsave, csave, scratch, total;
     long wcap;
 };
 
 template <int LM1, int LM2>
-FourStepBwdLayout fourstep_bwd_layout_n(int D, int N)
+FourStepBwdLayout fourstep_bwd_layout_n(int D, int N, int sets)
 {
     using FS = FourStep<LM1, LM2>;
     auto up = [](size_t n) { return (n + 255) / 256 * 256; };
     FourStepBwdLayout l;
     l.wcap = bwd_wave_cap(FS::M);
     l.acc = 0;
-    l.zsave = l.acc + up(sizeof(float2) * (size_t)N * D * FS::M);
+    l.zsave = l.acc + up(sizeof(float2) * (size_t)sets * N * D * FS::M);
     l.csave = l.zsave + up(sizeof(float2) * (size_t)N * l.wcap * FS::M1 * FS::ROW_STRIDE);
     l.scratch = l.csave + up(sizeof(float2) * (size_t)N * l.wcap * (FS::M / 2));
     l.total = l.scratch + up(sizeof(float2) * (size_t)l.wcap * FS::M);
@@ -39,8 +40,9 @@ hyena_status_t run_fourstep_bwd(FourStepBwdArgs a, int N, cudaStream_t st)
     using FB = FourStepBwd<LM1, LM2>;
     FourStepArgs& f = a.f;
     const long nseq = (long)f.B * f.D, per = a.wcap;
+    const long sets = f.H_bstride != 0 ? f.B : 1;             // dh spectra per (n, d)
     f.n_last = N - 1;
-    const cudaError_t e = cudaMemsetAsync(a.acc, 0, sizeof(float2) * (size_t)N * f.D * FS::M, st);
+    const cudaError_t e = cudaMemsetAsync(a.acc, 0, sizeof(float2) * (size_t)sets * N * f.D * FS::M, st);
     if (e != cudaSuccess) return from_cuda(e);
     for (long q0 = 0; q0 < nseq; q0 += per) {
         const unsigned nq = (unsigned)(nseq - q0 < per ? nseq - q0 : per);
@@ -75,8 +77,8 @@ hyena_status_t run_fourstep_bwd(FourStepBwdArgs a, int N, cudaStream_t st)
                        FS::COL_SMEM, st, a);
         if (s != HYENA_OK) return s;
     }
-    // dh_n, db_n from the N*D accumulated spectra, a wave of rows at a time
-    const long rows = (long)N * f.D;
+    // dh_n, db_n from the sets*N*D accumulated spectra, a wave of rows at a time
+    const long rows = sets * N * f.D;
     for (long r0 = 0; r0 < rows; r0 += per) {
         const unsigned nq = (unsigned)(rows - r0 < per ? rows - r0 : per);
         f.q0 = (int)r0;
@@ -87,6 +89,10 @@ hyena_status_t run_fourstep_bwd(FourStepBwdArgs a, int N, cudaStream_t st)
             s = launch(fourstep_bwd_col_kernel<LM1, LM2, IO, 3>, nq * FS::COL_CTAS_PER_SEQ, FS::COL_THREADS,
                        FS::COL_SMEM, st, a);
         if (s != HYENA_OK) return s;
+    }
+    if (f.H_bstride != 0) {          // per-sample: db from the B lag-0 values (any B)
+        const int nd = N * f.D;
+        return launch(dbias_sum_kernel<FS::M>, (unsigned)((nd + 255) / 256), 256, 0, st, a);   // rows of L = M
     }
     return HYENA_OK;
 }
@@ -107,17 +113,17 @@ hyena_status_t dispatch_fourstep_bwd(int log2m, const FourStepBwdArgs& a, int N,
     }
 }
 
-inline FourStepBwdLayout fourstep_bwd_layout(int log2m, int D, int N)
+inline FourStepBwdLayout fourstep_bwd_layout(int log2m, int D, int N, int sets = 1)
 {
     switch (log2m) {
-    case 15: return fourstep_bwd_layout_n<7, 8>(D, N);
-    case 16: return fourstep_bwd_layout_n<8, 8>(D, N);
-    case 17: return fourstep_bwd_layout_n<8, 9>(D, N);
-    case 18: return fourstep_bwd_layout_n<9, 9>(D, N);
-    case 19: return fourstep_bwd_layout_n<9, 10>(D, N);
-    case 20: return fourstep_bwd_layout_n<10, 10>(D, N);
-    case 21: return fourstep_bwd_layout_n<10, 11>(D, N);
-    default: return fourstep_bwd_layout_n<11, 11>(D, N);
+    case 15: return fourstep_bwd_layout_n<7, 8>(D, N, sets);
+    case 16: return fourstep_bwd_layout_n<8, 8>(D, N, sets);
+    case 17: return fourstep_bwd_layout_n<8, 9>(D, N, sets);
+    case 18: return fourstep_bwd_layout_n<9, 9>(D, N, sets);
+    case 19: return fourstep_bwd_layout_n<9, 10>(D, N, sets);
+    case 20: return fourstep_bwd_layout_n<10, 10>(D, N, sets);
+    case 21: return fourstep_bwd_layout_n<10, 11>(D, N, sets);
+    default: return fourstep_bwd_layout_n<11, 11>(D, N, sets);
     }
 }
 

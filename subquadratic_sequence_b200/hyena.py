@@ -89,6 +89,12 @@ def _load() -> ctypes.CDLL:
                                                      vp, sz, vp], i),
         "hyena_filter_rfft2d_circular": ([vp, i, i, i, i, vp, vp], i),
         "hyena_fftconv2d_backward_workspace_size": ([i, i, i, i, i], sz),
+        "hyena_fftconv2d_backward_per_sample_workspace_size": ([i, i, i, i, i], sz),
+        "hyena_fftconv2d_backward_circular_workspace_size": ([i, i, i, i, i], sz),
+        "hyena_fftconv2d_gate_backward_circular": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
+                                                    ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
+        "hyena_fftconv2d_gate_backward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
+                                                      ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_fftconv2d_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, vp,
                                            ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_filter_rfft3d_circular": ([vp, i, i, i, i, i, vp, vp], i),
@@ -330,7 +336,7 @@ def hyena_fftconv_backward_per_sample_workspace_size(B: int, D: int, L: int, N: 
     n = LIB.hyena_fftconv_backward_per_sample_workspace_size(B, D, L, N)
     if n == ctypes.c_size_t(-1).value:
         raise HyenaError("hyena_fftconv_backward_per_sample_workspace_size", HYENA_ERR_UNSUPPORTED,
-                         "invalid sizes (L <= 16384)")
+                         "invalid sizes")
     return n
 
 
@@ -338,7 +344,7 @@ def hyena_fftconv_gate_backward_per_sample(v: torch.Tensor, xs, bias: torch.Tens
                                            dy: torch.Tensor, *, workspace=None, stream=None):
     """The backward with a spectrum set per sample, H [B][N][D][L]: returns
     (dv, [dx_1..dx_N], dh [B][N][D][L] per sample, dbias [N][D] summed over
-    the batch); L <= 16384."""
+    the batch); L up to 2^22."""
     B, D, L = v.shape
     N = len(xs)
     io = io_dtype(v)
@@ -708,3 +714,61 @@ def hyena_fftconv3d_gate_forward_per_sample(v: torch.Tensor, xs, bias: torch.Ten
         ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+def hyena_fftconv2d_gate_backward_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                             dy: torch.Tensor, *, workspace=None, stream=None):
+    """The 2-D backward with per-sample spectra Hs [B][N][C][2H][W]: returns
+    (dv, [dx_1..dx_N], dh [B][N][C][H][W] per sample, dbias [N][C] summed
+    over the batch)."""
+    B, C, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty((B, N, C, H, W), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, C), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        n = LIB.hyena_fftconv2d_backward_per_sample_workspace_size(B, C, H, W, N)
+        if n == ctypes.c_size_t(-1).value:
+            raise HyenaError("hyena_fftconv2d_backward_per_sample_workspace_size", HYENA_ERR_UNSUPPORTED,
+                             "invalid sizes")
+        workspace = torch.empty(n, device=v.device, dtype=torch.uint8)
+    _check("hyena_fftconv2d_gate_backward_per_sample", LIB.hyena_fftconv2d_gate_backward_per_sample(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+        B, C, H, W, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+        ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db
+
+
+def hyena_fftconv2d_gate_backward_circular(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                           dy: torch.Tensor, *, workspace=None, stream=None):
+    """The backward of the circular 2-D forward (Hs [N][C][H][W/2] from
+    hyena_filter_rfft2d_circular): returns (dv, [dx_1..dx_N], dh
+    [N][C][H][W], dbias [N][C]), dh and dbias summed over the batch."""
+    B, C, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty((N, C, H, W), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, C), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        n = LIB.hyena_fftconv2d_backward_circular_workspace_size(B, C, H, W, N)
+        if n == ctypes.c_size_t(-1).value:
+            raise HyenaError("hyena_fftconv2d_backward_circular_workspace_size", HYENA_ERR_UNSUPPORTED,
+                             "invalid sizes")
+        workspace = torch.empty(n, device=v.device, dtype=torch.uint8)
+    _check("hyena_fftconv2d_gate_backward_circular", LIB.hyena_fftconv2d_gate_backward_circular(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+        B, C, H, W, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+        ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db

@@ -133,7 +133,11 @@ def test_backward_c3_64k_full_size(hy):
 # ------------------------------------------------- per-sample filters
 
 PS_CASES = [(2, 3, 64, 2, "f32"), (3, 13, 2048, 2, "f32"), (2, 5, 1024, 3, "bf16"), (2, 2, 16384, 2, "f32"),
-            (1, 1, 16, 1, "f32")]
+            (1, 1, 16, 1, "f32"),
+            # four-step: L = 2^15 (N = 1), 2^16 in bf16, and 2^18, where a wave
+            # holds 32 sequences, so channel 10's three samples straddle two waves
+            (3, 2, 32768, 1, "f32"), (2, 3, 65536, 2, "bf16"), (3, 11, 262144, 1, "f32"),
+            (1, 2, 32768, 2, "f32")]     # one sample: dbias still comes from the per-sample sum
 
 
 @pytest.mark.parametrize("B,D,L,N,io", PS_CASES)
@@ -170,7 +174,8 @@ def test_backward_per_sample_with_equal_sets_is_the_shared_backward(hy):
     assert rel_max_err(host(pb), host(db)) <= 1e-5
 
 
-def test_backward_per_sample_rejects_long_sequences(hy):
+def test_backward_per_sample_rejects_unsupported_lengths(hy):
     from subquadratic_sequence_b200.hyena import HyenaError
-    with pytest.raises(HyenaError):
-        hy.hyena_fftconv_backward_per_sample_workspace_size(2, 4, 32768, 2)
+    for L in (8, 1 << 23, 3000):
+        with pytest.raises(HyenaError):
+            hy.hyena_fftconv_backward_per_sample_workspace_size(2, 4, L, 2)

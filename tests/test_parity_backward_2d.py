@@ -104,3 +104,36 @@ def test_backward_2d_delta_filter_closed_form(hy):
         for c in range(32):
             want_dh[:, a, c] = np.sum(e[:, :, a:, c:] * v[:, :, :16 - a, :32 - c], axis=(0, 2, 3))
     assert rel_max_err(dh[0], want_dh) <= 1e-4
+
+
+# ------------------------------------------------- per-sample filters
+
+@pytest.mark.parametrize("B,C,H,W,N,io", [(2, 3, 32, 64, 2, "f32"), (3, 2, 16, 128, 2, "bf16"),
+                                          (1, 2, 16, 16, 1, "f32"),
+                                          (3, 12, 512, 512, 1, "f32")])   # a channel across two waves
+def test_backward_2d_per_sample_matches_oracle(hy, B, C, H, W, N, io):
+    wl, inp, _, dy = problem(B, C, H, W, N, seed=60 + H, io=io)
+    r = np.random.default_rng(H + W)
+    decay = np.exp(-np.arange(H) / (H / 4))[:, None] * np.exp(-np.arange(W) / (W / 4))
+    h = (r.standard_normal((B, N, C, H, W)) * decay * 8 / np.sqrt(H * W)).astype(np.float32)
+    Hs = hy.hyena_filter_rfft2d(dev(h.reshape(B * N, C, H, W))).reshape(B, N, C, 2 * H, W)
+    dv, dxs, dh, db = hy.hyena_fftconv2d_gate_backward_per_sample(
+        dev(inp["v"], io), [dev(x, io) for x in inp["x"]], dev(inp["b"]), Hs, dev(dy, io))
+    torch.cuda.synchronize()
+    got = host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+    ref = oracle.hyena_backward_2d_per_sample(inp["v"], np.stack(inp["x"]), h, inp["b"], dy)
+    check(got, ref, io, f"2-D per-sample B{B} C{C} {H}x{W} N{N} {io}")
+
+
+def test_backward_2d_per_sample_with_equal_sets_is_the_shared_backward(hy):
+    B, C, H, W, N = 3, 4, 64, 64, 2
+    wl, inp, h, dy = problem(B, C, H, W, N, seed=77, io="f32")
+    Hs = hy.hyena_filter_rfft2d(dev(h))
+    v, xs, b, g = dev(inp["v"]), [dev(x) for x in inp["x"]], dev(inp["b"]), dev(dy)
+    dv, dxs, dh, db = hy.hyena_fftconv2d_gate_backward(v, xs, b, Hs, g)
+    pv, pxs, ph, pb = hy.hyena_fftconv2d_gate_backward_per_sample(
+        v, xs, b, Hs.unsqueeze(0).expand(B, -1, -1, -1, -1).contiguous(), g)
+    torch.cuda.synchronize()
+    assert torch.equal(dv, pv) and all(torch.equal(a, c) for a, c in zip(dxs, pxs))
+    assert rel_max_err(host(ph).sum(axis=0), host(dh)) <= 1e-5
+    assert rel_max_err(host(pb), host(db)) <= 1e-5

@@ -119,6 +119,57 @@ def test_forward_2d_circular_on_padded_grids_is_the_linear_forward(hy):
 
 # ------------------------------------------------------------------ 3-D
 
+def check_backward(got, ref, io, name):
+    dv, dx, dh, db = got
+    rdv, rdx, rdh, rdb = ref
+    assert_close(dv, rdv, io, f"{name} dv")
+    assert_close(dx, rdx, io, f"{name} dx")
+    err_h = np.max(np.abs(dh - rdh)) / np.max(np.abs(rdh))
+    err_b = np.max(np.abs(db - rdb)) / np.max(np.abs(rdb))
+    assert err_h <= 1e-4, f"{name} dh {err_h:.3e}"
+    assert err_b <= 1e-4, f"{name} db {err_b:.3e}"
+
+
+@pytest.mark.parametrize("B,C,H,W,N,io", [
+    (1, 2, 16, 32, 1, "f32"), (2, 3, 32, 64, 2, "f32"), (2, 2, 16, 128, 2, "bf16"), (1, 1, 128, 32, 3, "f32"),
+    (1, 1, 1024, 32, 1, "f32"), (1, 1, 16, 1024, 2, "f32"), (2, 2, 256, 256, 2, "f32"),
+    (3, 22, 512, 512, 1, "f32"),     # 66 images, 64 a wave: channel 21 spans two waves
+])
+def test_backward_2d_circular_matches_oracle(hy, B, C, H, W, N, io):
+    v, x, b, h = problem(B, C, (H, W), N, seed=2 * H + W + N)
+    dy = np.random.default_rng(H * W).standard_normal((B, C, H, W)).astype(np.float32)
+    Hs = hy.hyena_filter_rfft2d_circular(dev(h))
+    dv, dxs, dh, db = hy.hyena_fftconv2d_gate_backward_circular(dev(v, io), [dev(xx, io) for xx in x], dev(b),
+                                                                Hs, dev(dy, io))
+    torch.cuda.synchronize()
+    got = host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+    ref = oracle.hyena_backward_circular_2d(as_io(v, io), np.stack([as_io(xx, io) for xx in x]),
+                                            h.astype(np.float64), b.astype(np.float64), as_io(dy, io))
+    check_backward(got, ref, io, f"circular 2-D backward B{B} C{C} {H}x{W} N{N} {io}")
+
+
+def test_backward_2d_circular_shift_filter_closed_form(hy):
+    # N = 1, h = delta at (k, l), b = 0: y = x roll(v, (k, l)), so
+    # dv = roll(dy x, (-k, -l)), dx = dy roll(v, (k, l)),
+    # db = sum dy x v, dh[a][b] = sum dy x roll(v, (a, b))
+    B, C, H, W, k, l = 2, 2, 32, 64, 5, 30
+    rng = np.random.default_rng(9)
+    v, x, dy = (rng.standard_normal((B, C, H, W)).astype(np.float32) for _ in range(3))
+    h = np.zeros((1, C, H, W), np.float32)
+    h[0, :, k, l] = 1.0
+    dv, dxs, dh, db = hy.hyena_fftconv2d_gate_backward_circular(
+        dev(v), [dev(x)], dev(np.zeros((1, C), np.float32)), hy.hyena_filter_rfft2d_circular(dev(h)), dev(dy))
+    torch.cuda.synchronize()
+    e = dy.astype(np.float64) * x
+    assert_close(host(dv), np.roll(e, (-k, -l), axis=(2, 3)), "f32", "dv")
+    assert_close(host(dxs[0]), dy.astype(np.float64) * np.roll(v, (k, l), axis=(2, 3)), "f32", "dx")
+    for a_, b_ in [(0, 0), (1, 0), (0, 1), (k, l), (H - 1, W - 1), (7, 33)]:
+        ref = np.sum(e * np.roll(v, (a_, b_), axis=(2, 3)), axis=(0, 2, 3))
+        got = host(dh)[0, :, a_, b_]
+        assert np.max(np.abs(got - ref)) <= 1e-4 * np.max(np.abs(host(dh))), (a_, b_)
+    assert np.max(np.abs(host(db)[0] - np.sum(e * v, axis=(0, 2, 3)))) <= 1e-4 * np.max(np.abs(host(dh)))
+
+
 def unpack_circ_3d(P):
     """Packed [..., Z, H, M] -> bins [..., Z, H, M + 1] (M = W/2)."""
     M = P.shape[-1]
