@@ -1291,6 +1291,119 @@ int oracle_hyena_forward_3d(const double *v, const double *x, const double *h, c
 }
 
 /* ------------------------------------------------------------------ */
+/* The backward pass of the 3-D recurrence: the exact adjoint, as in   */
+/* 1-D and 2-D, with 3-D correlations.                                  */
+/* ------------------------------------------------------------------ */
+
+/* out[a][b][c] = sum_{t >= a, s >= b, u >= c} p[t][s][u] q[t-a][s-b][u-c]:
+ * with p = e, q = z it is dh; with p = e, q = h the adjoint of the linear
+ * 3-D convolution with respect to its signal.  The definition, O(V^2). */
+static void lagged3_direct(const double *p, const double *q, long Z, long H, long W, double *out)
+{
+    for (long a = 0; a < Z; ++a)
+        for (long b = 0; b < H; ++b)
+            for (long c = 0; c < W; ++c) {
+                double acc = 0.0;
+                for (long t = a; t < Z; ++t)
+                    for (long s = b; s < H; ++s)
+                        for (long u = c; u < W; ++u)
+                            acc += p[(t * H + s) * W + u] * q[((t - a) * H + (s - b)) * W + (u - c)];
+                out[(a * H + b) * W + c] = acc;
+            }
+}
+
+/* The same through the DFT of both zero-padded to 2Z x 2H x 2W (powers of
+ * two): IDFT(P conj(Q)) / (8 Z H W) at a < Z, b < H, c < W. */
+static int lagged3_fft(const double *p, const double *q, long Z, long H, long W, double *out)
+{
+    const long PZ = 2 * Z, PH = 2 * H, PW = 2 * W, P = PZ * PH * PW;
+    double *pr = calloc(P, sizeof(double)), *pi = calloc(P, sizeof(double));
+    double *qr = calloc(P, sizeof(double)), *qi = calloc(P, sizeof(double));
+    int st = ORACLE_ENOMEM;
+    if (!pr || !pi || !qr || !qi) goto out;
+    for (long z = 0; z < Z; ++z)
+        for (long y = 0; y < H; ++y)
+            for (long x = 0; x < W; ++x) {
+                pr[(z * PH + y) * PW + x] = p[(z * H + y) * W + x];
+                qr[(z * PH + y) * PW + x] = q[(z * H + y) * W + x];
+            }
+    if ((st = fft3(pr, pi, PZ, PH, PW, -1)) != ORACLE_OK) goto out;
+    if ((st = fft3(qr, qi, PZ, PH, PW, -1)) != ORACLE_OK) goto out;
+    for (long k = 0; k < P; ++k) {
+        const double re = pr[k] * qr[k] + pi[k] * qi[k], im = pi[k] * qr[k] - pr[k] * qi[k];
+        pr[k] = re;
+        pi[k] = im;
+    }
+    if ((st = fft3(pr, pi, PZ, PH, PW, +1)) != ORACLE_OK) goto out;
+    for (long z = 0; z < Z; ++z)
+        for (long y = 0; y < H; ++y)
+            for (long x = 0; x < W; ++x) out[(z * H + y) * W + x] = pr[(z * PH + y) * PW + x] / (double)P;
+out:
+    free(pr); free(pi); free(qr); free(qi);
+    return st;
+}
+
+/* Gradients of a scalar loss with dL/dy = dy [B][C][Z][H][W] through the
+ * 3-D recurrence (oracle_hyena_forward_3d): dv, dx [N][B][C][Z][H][W],
+ * dh [N][C][Z][H][W] and dbias [N][C] (both summed over the batch).  With
+ * c_n = h_n (*) z_{n-1} + b_n z_{n-1}, z_n = x_n c_n and g = dL/dz_n:
+ * dx_n = g c_n, e = g x_n, dh_n += lagged3(e, z_{n-1}), db_n += sum e
+ * z_{n-1}, dz_{n-1} = lagged3(e, h_n) + b_n e.  One thread. */
+int oracle_hyena_backward_3d(const double *v, const double *x, const double *h, const double *bias,
+                             const double *dy, long B, long C, long Z, long H, long W, long N, int route,
+                             double *dv, double *dx, double *dh, double *dbias)
+{
+    if (!v || !x || !h || !bias || !dy || !dv || !dx || !dh || !dbias || B < 1 || C < 1 || Z < 1 || H < 1 ||
+        W < 1 || N < 1 || (route != ROUTE_DIRECT && route != ROUTE_FFT))
+        return ORACLE_EBADARG;
+    if (route == ROUTE_FFT && (!is_pow2(Z) || !is_pow2(H) || !is_pow2(W))) return ORACLE_EBADARG;
+    const long V = Z * H * W, BCV = B * C * V;
+    double *z = malloc(sizeof(double) * N * V), *c = malloc(sizeof(double) * N * V);
+    double *g = malloc(sizeof(double) * V), *e = malloc(sizeof(double) * V), *tmp = malloc(sizeof(double) * V);
+    int st = ORACLE_OK;
+    if (!z || !c || !g || !e || !tmp) { st = ORACLE_ENOMEM; goto done; }
+    memset(dh, 0, sizeof(double) * N * C * V);
+    memset(dbias, 0, sizeof(double) * N * C);
+    for (long img = 0; img < B * C && st == ORACLE_OK; ++img) {
+        const long ch = img % C;
+        memcpy(z, v + img * V, sizeof(double) * V);              /* z_0 = v */
+        for (long n = 0; n < N && st == ORACLE_OK; ++n) {
+            const double *hn = h + (n * C + ch) * V, *xn = x + n * BCV + img * V;
+            const double bn = bias[n * C + ch];
+            double *zn = z + n * V, *cn = c + n * V;
+            st = oracle_conv3(hn, zn, Z, H, W, route, cn);
+            for (long t = 0; t < V; ++t) cn[t] += bn * zn[t];
+            if (n + 1 < N)
+                for (long t = 0; t < V; ++t) z[(n + 1) * V + t] = xn[t] * cn[t];
+        }
+        memcpy(g, dy + img * V, sizeof(double) * V);
+        for (long n = N - 1; n >= 0 && st == ORACLE_OK; --n) {
+            const double *hn = h + (n * C + ch) * V, *xn = x + n * BCV + img * V;
+            const double bn = bias[n * C + ch];
+            const double *zn = z + n * V, *cn = c + n * V;
+            double *dxn = dx + n * BCV + img * V, *dhn = dh + (n * C + ch) * V;
+            for (long t = 0; t < V; ++t) {
+                dxn[t] = g[t] * cn[t];
+                e[t] = g[t] * xn[t];
+            }
+            if (route == ROUTE_DIRECT) lagged3_direct(e, zn, Z, H, W, tmp);
+            else st = lagged3_fft(e, zn, Z, H, W, tmp);
+            for (long t = 0; t < V; ++t) dhn[t] += tmp[t];
+            double db = 0.0;
+            for (long t = 0; t < V; ++t) db += e[t] * zn[t];
+            dbias[n * C + ch] += db;
+            if (route == ROUTE_DIRECT) lagged3_direct(e, hn, Z, H, W, tmp);
+            else if (st == ORACLE_OK) st = lagged3_fft(e, hn, Z, H, W, tmp);
+            for (long t = 0; t < V; ++t) g[t] = tmp[t] + bn * e[t];
+        }
+        memcpy(dv + img * V, g, sizeof(double) * V);             /* dv = dz_0 */
+    }
+done:
+    free(z); free(c); free(g); free(e); free(tmp);
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
 /* Circular convolution on 2-D grids and 3-D volumes (Handling          */
 /* Boundaries: circular convolutions for periodic physical systems; a   */
 /* 2-D grid is a volume with Z = 1).                                    */

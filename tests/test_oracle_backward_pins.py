@@ -346,3 +346,64 @@ def test_backward_circular_2d_of_one_row_is_the_circular_1d_backward():
     for a, c in zip(g2[:3], g1[:3]):
         assert rel_err(a[..., 0, :], c) < 1e-12
     assert rel_err(g2[3], g1[3]) < 1e-12
+
+
+# ------------------------------------------------- 3-D
+
+def problem_3d(B, C, Z, H, W, N, seed):
+    r = np.random.default_rng(seed)
+    env = (np.exp(-np.arange(Z) / 3.0)[:, None, None] * np.exp(-np.arange(H) / 3.0)[:, None]
+           * np.exp(-np.arange(W) / 3.0))
+    return (r.standard_normal((B, C, Z, H, W)), r.standard_normal((N, B, C, Z, H, W)),
+            r.standard_normal((N, C, Z, H, W)) * env, r.standard_normal((N, C)),
+            r.standard_normal((B, C, Z, H, W)))
+
+
+@pytest.mark.parametrize("N", [1, 2])
+def test_backward_3d_matches_finite_differences(N):
+    v, x, h, b, dy = problem_3d(2, 2, 2, 3, 3, N, seed=60 + N)
+    dv, dx, dh, db = oracle.hyena_backward_3d(v, x, h, b, dy, route="direct")
+
+    def loss(v_, x_, h_, b_):
+        return float(np.sum(dy * oracle.hyena_forward_3d(v_, x_, h_, b_, route="direct")))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name
+
+
+def test_backward_3d_routes_agree_and_db_is_dh_origin():
+    v, x, h, b, dy = problem_3d(2, 2, 4, 4, 8, 2, seed=63)
+    d = oracle.hyena_backward_3d(v, x, h, b, dy, route="direct")
+    f = oracle.hyena_backward_3d(v, x, h, b, dy, route="fft")
+    for a, c in zip(d, f):
+        assert rel_err(c, a) < 1e-12
+    assert rel_err(d[3], d[2][:, :, 0, 0, 0]) < 1e-13
+
+
+def test_backward_3d_of_one_plane_is_the_2d_backward():
+    v, x, h, b, dy = problem_3d(2, 3, 1, 8, 4, 2, seed=64)
+    g3 = oracle.hyena_backward_3d(v, x, h, b, dy)
+    g2 = oracle.hyena_backward_2d(v[:, :, 0], x[:, :, :, 0], h[:, :, 0], b, dy[:, :, 0])
+    for a, c in zip(g3[:3], g2[:3]):
+        assert rel_err(a[..., 0, :, :], c) < 1e-12
+    assert rel_err(g3[3], g2[3]) < 1e-12
+
+
+def test_backward_3d_axis_permutation_permutes_every_gradient():
+    v, x, h, b, dy = problem_3d(1, 2, 2, 4, 8, 2, seed=65)
+    perm = lambda a: np.swapaxes(a, -1, -3)                 # z <-> x
+    g = oracle.hyena_backward_3d(v, x, h, b, dy)
+    gp = oracle.hyena_backward_3d(perm(v), perm(x), perm(h), b, perm(dy))
+    for a, c in zip(g[:3], gp[:3]):
+        assert rel_err(perm(c), a) < 1e-12
+    assert rel_err(gp[3], g[3]) < 1e-12
