@@ -130,7 +130,7 @@ def launches_forward(wl: synth.Workload) -> int:
             return waves(wl.B * wl.D, wl.per_channel) * (4 * wl.N + 1)
         if wl.kind == "2d":
             return waves(wl.B * wl.D, wl.per_channel // 2) * (1 + 2 * wl.N)
-        return 1
+        return waves(wl.B * wl.D, wl.L // 2) * (1 + 2 * wl.N) if long_path(wl) else 1
     if wl.kind == "3d":
         # per wave: rows, columns, then per order z, inverse columns, rows
         # (and forward columns before every order but the first)
@@ -142,6 +142,8 @@ def launches_forward(wl: synth.Workload) -> int:
 
 def launches_rfft(wl: synth.Workload) -> int:
     if wl.circular:
+        if long_path(wl):
+            return waves(wl.N * wl.D, wl.L // 2) * 2
         return {"1d": 1, "2d": 2, "3d": 3}[wl.kind]
     if wl.kind == "3d":
         return 3
@@ -158,6 +160,8 @@ def launches_filter_gen(wl: synth.Workload) -> int:
 def forward_kernel(wl: synth.Workload) -> str:
     """The timed unit of the roofline: the forward call (one fused kernel,
     or the 2N+1 four-step kernels of each wave)."""
+    if wl.circular and long_path(wl):
+        return "fourstep_row_kernel+fourstep_col_kernel<PAD=false> (hyena_fftconv_gate_forward_circular, all launches)"
     if wl.circular:
         return {"1d": "fused1d_kernel<PAD=false> (hyena_fftconv_gate_forward_circular)",
                 "2d": "fft2d_row_kernel+fft2d_col_kernel<PAD=false> (hyena_fftconv2d_gate_forward_circular, "
@@ -371,14 +375,19 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     elif wl.circular:
         h = torch.empty((wl.N, wl.D, wl.L), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.N, wl.D, wl.L // 2), device="cuda", dtype=torch.complex64)
+        # four-step workspaces (L > 16384), allocated once
+        ws_rfft_n = hyena.LIB.hyena_filter_rfft_circular_workspace_size(wl.N, wl.D, wl.L)
+        ws_fwd_n = hyena.LIB.hyena_fftconv_circular_workspace_size(wl.B, wl.D, wl.L, wl.N)
+        ws_rfft = torch.empty(ws_rfft_n, device="cuda", dtype=torch.uint8) if ws_rfft_n else None
+        ws_fwd = torch.empty(ws_fwd_n, device="cuda", dtype=torch.uint8) if ws_fwd_n else None
 
         def forward():
-            hyena.hyena_fftconv_gate_forward_circular(v, xs, b, H, out=y)
+            hyena.hyena_fftconv_gate_forward_circular(v, xs, b, H, out=y, workspace=ws_fwd)
 
         def step():
             hyena.hyena_filter_gen(*W, wl.N, wl.D, wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
                                    decay_div=synth.DECAY_DIV, out=h)
-            hyena.hyena_filter_rfft_circular(h, out=H)
+            hyena.hyena_filter_rfft_circular(h, out=H, workspace=ws_rfft)
             forward()
     elif wl.kind == "3d" and wl.film:
         F = [to_dev(inp[k]) for k in ("omega", "gamma", "beta", "sigma")]
@@ -542,7 +551,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
 
     # ---- the backward pass (1-D and 2-D): one call per timed repetition
     bwd = None
-    if wl.kind == "1d" or (wl.kind == "2d" and not wl.film):
+    if (wl.kind == "1d" and not (wl.circular and long_path(wl))) or (wl.kind == "2d" and not wl.film):
         dy = to_dev(synth.make_output_grad(wl), io)
         if wl.circular and wl.kind == "2d":
             ws_b = torch.empty(hyena.hyena_fftconv2d_backward_circular_workspace_size(wl.B, wl.D, wl.H, wl.W,

@@ -204,19 +204,27 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_per_sample(const void* v, co
  * for periodic systems, the alternative to zero padding).  The same
  * recurrence with every convolution circular of length L:
  *     (h (*) u)[t] = sum_{s=0..L-1} h[s] u[(t - s) mod L].
- * L is a power of two, 32 <= L <= 16384 (one launch, each sequence on one
- * SM); other L return HYENA_ERR_UNSUPPORTED.
+ * L is a power of two, 32 <= L <= HYENA_MAX_LEN; other L return
+ * HYENA_ERR_UNSUPPORTED.  L <= 16384 runs one launch with each sequence on
+ * one SM and needs no workspace; longer L the four-step transform through
+ * the workspace, 2N + 1 launches per wave of sequences.
  * hyena_filter_rfft_circular: H [N][D][L/2] complex64, the L-point DFT X of
  * each filter without padding, packed like hyena_filter_rfft's spectra:
- * slot 0 = (X[0], X[L/2]) (both real), slot k = X[k] for 1 <= k < L/2.
+ * slot 0 = (X[0], X[L/2]) (both real), slot k = X[k] for 1 <= k < L/2;
+ * workspace of hyena_filter_rfft_circular_workspace_size(N, D, L) bytes.
  * hyena_fftconv_gate_forward_circular: v, x_n, y [B][D][L] io, H as above,
- * bias [N][D]; no workspace.  Alignment: h, H, v, x_n, y 16 bytes; bias 4. */
+ * bias [N][D]; workspace of hyena_fftconv_circular_workspace_size(B, D, L,
+ * N) bytes.  Workspaces are 256-byte aligned, NULL / 0 when the size is 0,
+ * and must not overlap any argument.  Alignment: h, H, v, x_n, y 16 bytes;
+ * bias 4.  The size functions return (size_t)-1 for invalid sizes. */
+HYENA_API size_t hyena_filter_rfft_circular_workspace_size(int N, int D, int L);
 HYENA_API hyena_status_t hyena_filter_rfft_circular(const float* h, int N, int D, int L, float* H,
-                                                    void* stream);
+                                                    void* workspace, size_t ws_bytes, void* stream);
+HYENA_API size_t hyena_fftconv_circular_workspace_size(int B, int D, int L, int N);
 HYENA_API hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* const* x,
-                                                             const float* H, const float* bias, int B,
-                                                             int D, int L, int N, hyena_dtype_t io,
-                                                             void* y, void* stream);
+                                                             const float* H, const float* bias, int B, int D,
+                                                             int L, int N, hyena_dtype_t io, void* y,
+                                                             void* workspace, size_t ws_bytes, void* stream);
 
 /* The backward pass of the circular recurrence (hyena_fftconv_gate_forward_
  * circular), for training: the exact adjoint with every convolution

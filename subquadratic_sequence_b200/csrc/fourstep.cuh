@@ -311,8 +311,11 @@ fourstep_row_kernel(FourStepArgs a)
 
 // Column kernel.  MODE 0: the first order's forward columns from v (or, for
 // the spectrum, from h); MODE 1: inverse columns, gate, next order's forward
-// columns; MODE 2: inverse columns, gate, store y.
-template <int LOG2M1, int LOG2M2, typename IO, int MODE>
+// columns; MODE 2: inverse columns, gate, store y.  PAD false: circular
+// mode ("Handling Boundaries": periodic systems), the M-point transform of
+// the unpadded sequence of 2M reals: every n1 is data and no output is
+// cropped.
+template <int LOG2M1, int LOG2M2, typename IO, int MODE, bool PAD = true>
 __global__ void __launch_bounds__(FourStep<LOG2M1, LOG2M2>::COL_THREADS)
 fourstep_col_kernel(FourStepArgs a)
 {
@@ -321,6 +324,8 @@ fourstep_col_kernel(FourStepArgs a)
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;
     constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, TC = FS::TC, V1 = FS::F1::V;
+    constexpr int VL = PAD ? V1 / 2 : V1;                   // registers holding data (n1 < M1/2, or all)
+    constexpr int SEQ = PAD ? M / 2 : M;                     // value pairs per sequence
     extern __shared__ __align__(16) float2 smem_fs[];
 
     const int qi = blockIdx.x / FS::COL_CTAS_PER_SEQ;
@@ -336,8 +341,8 @@ fourstep_col_kernel(FourStepArgs a)
     float2 reg[V1];
 
     if constexpr (MODE == 0) {
-        const PT* vp = reinterpret_cast<const PT*>(a.v) + seq * (M / 2);
-        static_for<V1 / 2>([&](auto rr) {
+        const PT* vp = reinterpret_cast<const PT*>(a.v) + seq * SEQ;
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             reg[r] = IOP::load(vp + n2 + (size_t)M2 * (t + r * (M1 / V1)));
         });
@@ -350,37 +355,37 @@ fourstep_col_kernel(FourStepArgs a)
         });
         __syncthreads();
         FS::F1::template run<+1, true>(buf, reg, t);
-        // crop (n1 = t + r M1/V1 < M1/2 <=> r < V1/2) and gate
+        // crop (n1 = t + r M1/V1 < M1/2 <=> r < V1/2; circular: none) and gate
         const void* xn = a.x[0];
 #pragma unroll
         for (int i = 1; i < kMaxOrder; ++i)
             if (i == a.n) xn = a.x[i];
-        const PT* xp = reinterpret_cast<const PT*>(xn) + seq * (M / 2);
-        static_for<V1 / 2>([&](auto rr) {
+        const PT* xp = reinterpret_cast<const PT*>(xn) + seq * SEQ;
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             const float2 xv = IOP::load(xp + n2 + (size_t)M2 * (t + r * (M1 / V1)));
             reg[r] = make_float2(reg[r].x * xv.x, reg[r].y * xv.y);
         });
         if constexpr (MODE == 2) {
-            PT* yp = reinterpret_cast<PT*>(a.y) + seq * (M / 2);
-            static_for<V1 / 2>([&](auto rr) {
+            PT* yp = reinterpret_cast<PT*>(a.y) + seq * SEQ;
+            static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
                 IOP::store(yp + n2 + (size_t)M2 * (t + r * (M1 / V1)), reg[r]);
             });
             return;
         }
     }
-    // forward column FFT of z (n1 < M1/2), zero-padded, then the four-step
-    // twiddle exp(-2 pi i n2 k1 / M)
+    // forward column FFT of z (n1 < M1/2, zero-padded; circular: all n1),
+    // then the four-step twiddle exp(-2 pi i n2 k1 / M)
     {
         const int pt = pad16(t);
-        static_for<V1 / 2>([&](auto rr) {
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             buf[pad16_at<M1 / V1>(t, pt, r)] = reg[r];
         });
     }
     __syncthreads();
-    FS::F1::template run<-1, true, true>(buf, reg, t);
+    FS::F1::template run<-1, true, PAD>(buf, reg, t);
     float2 w = expi_pi<-1>(2.0f * (float)((n2 * t) % M) / (float)M);
     const float2 step = expi_pi<-1>(2.0f * (float)((n2 * (M1 / V1)) % M) / (float)M);
     static_for<V1>([&](auto rr) {

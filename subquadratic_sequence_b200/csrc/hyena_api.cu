@@ -5,6 +5,7 @@
 #include "k_circular.cuh"
 #include "k_fft2d.cuh"
 #include "k_fft2d_bwd.cuh"
+#include "k_fourstep.cuh"
 #include "k_fourstep_bwd.cuh"
 #include "k_fft3d.cuh"
 #include "launch.cuh"
@@ -386,15 +387,32 @@ hyena_status_t forward_impl(const void* v, const void* const* x, const float* h,
 
 extern "C" {
 
-hyena_status_t hyena_filter_rfft_circular(const float* h, int N, int D, int L, float* H, void* stream)
+size_t hyena_filter_rfft_circular_workspace_size(int N, int D, int L)
+{
+    const int k = exact_log2(L);
+    if (N < 1 || D < 1 || k < kMinLog2Circ + 1 || k > kMaxLog2) return (size_t)-1;
+    return k - 1 <= kMaxLog2Circ ? 0 : round_up(scratch_bytes((long)N * D, L / 2), 256);
+}
+
+hyena_status_t hyena_filter_rfft_circular(const float* h, int N, int D, int L, float* H, void* workspace,
+                                          size_t ws_bytes, void* stream)
 {
     if (!h || !H || N < 1 || D < 1 || L < 1) return HYENA_ERR_INVALID_ARG;
     const int k = exact_log2(L);
-    if (k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1) return HYENA_ERR_UNSUPPORTED;
+    if (k < kMinLog2Circ + 1 || k > kMaxLog2) return HYENA_ERR_UNSUPPORTED;
     if (!aligned(h, 16) || !aligned(H, 16)) return HYENA_ERR_INVALID_ARG;
     if ((long)N * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
-    if (overlap(h, sizeof(float) * (size_t)N * D * L, H, sizeof(float2) * (size_t)N * D * (L / 2)))
-        return HYENA_ERR_INVALID_ARG;
+    const size_t spec = sizeof(float2) * (size_t)N * D * (L / 2);
+    if (overlap(h, sizeof(float) * (size_t)N * D * L, H, spec)) return HYENA_ERR_INVALID_ARG;
+    if (k - 1 > kMaxLog2Circ) {
+        // four-step (L > 16384): a wave of rows through the workspace
+        const size_t need = hyena_filter_rfft_circular_workspace_size(N, D, L);
+        if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+        if (overlap(workspace, need, h, sizeof(float) * (size_t)N * D * L) || overlap(workspace, need, H, spec))
+            return HYENA_ERR_INVALID_ARG;
+        return dispatch_fourstep_rfft_circ(k - 1, h, N * D, reinterpret_cast<float2*>(H),
+                                           static_cast<float2*>(workspace), (cudaStream_t)stream);
+    }
     Rfft1dArgs ra;
     ra.h = h;
     ra.H = reinterpret_cast<float2*>(H);
@@ -402,26 +420,59 @@ hyena_status_t hyena_filter_rfft_circular(const float* h, int N, int D, int L, f
     return dispatch_rfft_circ(k - 1, ra, (cudaStream_t)stream);
 }
 
+size_t hyena_fftconv_circular_workspace_size(int B, int D, int L, int N)
+{
+    const int k = exact_log2(L);
+    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || k < kMinLog2Circ + 1 || k > kMaxLog2)
+        return (size_t)-1;
+    return k - 1 <= kMaxLog2Circ ? 0 : round_up(scratch_bytes((long)B * D, L / 2), 256);
+}
+
 hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* const* x, const float* H,
                                                    const float* bias, int B, int D, int L, int N,
-                                                   hyena_dtype_t io, void* y, void* stream)
+                                                   hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes,
+                                                   void* stream)
 {
     if (!v || !x || !H || !bias || !y) return HYENA_ERR_INVALID_ARG;
     if (B < 1 || D < 1 || N < 1 || L < 1) return HYENA_ERR_INVALID_ARG;
     if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
     if (N > HYENA_MAX_ORDER || (long)B * D > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
     const int k = exact_log2(L);
-    if (k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1) return HYENA_ERR_UNSUPPORTED;
+    if (k < kMinLog2Circ + 1 || k > kMaxLog2) return HYENA_ERR_UNSUPPORTED;
     for (int n = 0; n < N; ++n)
         if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
     if (!aligned(v, 16) || !aligned(y, 16) || !aligned(H, 16) || !aligned(bias, 4))
         return HYENA_ERR_INVALID_ARG;
     const size_t act = (size_t)B * D * L * io_bytes(io);
-    if (overlap(y, act, v, act) || overlap(y, act, H, sizeof(float2) * (size_t)N * D * (L / 2)) ||
-        overlap(y, act, bias, sizeof(float) * N * D))
+    const size_t spec = sizeof(float2) * (size_t)N * D * (L / 2);
+    if (overlap(y, act, v, act) || overlap(y, act, H, spec) || overlap(y, act, bias, sizeof(float) * N * D))
         return HYENA_ERR_INVALID_ARG;
     for (int n = 0; n < N; ++n)
         if (overlap(y, act, x[n], act)) return HYENA_ERR_INVALID_ARG;
+    const size_t need = hyena_fftconv_circular_workspace_size(B, D, L, N);
+    if (need > 0) {
+        if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+        if (overlap(y, act, workspace, need) || overlap(workspace, need, v, act) ||
+            overlap(workspace, need, H, spec))
+            return HYENA_ERR_INVALID_ARG;
+        for (int n = 0; n < N; ++n)
+            if (overlap(workspace, need, x[n], act)) return HYENA_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    if (k - 1 > kMaxLog2Circ) {
+        // four-step (L > 16384)
+        FourStepArgs a = {};
+        a.v = v;
+        for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
+        a.y = y;
+        a.H = reinterpret_cast<const float2*>(H);
+        a.bias = bias;
+        a.B = B;
+        a.D = D;
+        float2* scratch = static_cast<float2*>(workspace);
+        return io == HYENA_BF16 ? dispatch_fourstep_circ_bf16(k - 1, a, N, scratch, st)
+                                : dispatch_fourstep_circ_f32(k - 1, a, N, scratch, st);
+    }
     Fused1dArgs a = {};
     a.v = v;
     for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
@@ -431,7 +482,6 @@ hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* co
     a.B = B;
     a.D = D;
     a.N = N;
-    cudaStream_t st = (cudaStream_t)stream;
     return io == HYENA_BF16 ? dispatch_fused_circ_bf16(k - 1, a, st) : dispatch_fused_circ_f32(k - 1, a, st);
 }
 

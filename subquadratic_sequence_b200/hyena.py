@@ -73,8 +73,11 @@ def _load() -> ctypes.CDLL:
                                                     ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_fftconv_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp,
                                          ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
-        "hyena_filter_rfft_circular": ([vp, i, i, i, vp, vp], i),
-        "hyena_fftconv_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp], i),
+        "hyena_filter_rfft_circular_workspace_size": ([i, i, i], sz),
+        "hyena_filter_rfft_circular": ([vp, i, i, i, vp, vp, sz, vp], i),
+        "hyena_fftconv_circular_workspace_size": ([i, i, i, i], sz),
+        "hyena_fftconv_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp, sz,
+                                                 vp], i),
         "hyena_filter_rfft2d": ([vp, i, i, i, i, vp, vp], i),
         "hyena_filter_gen_film_2d": ([ffn_p, ctypes.POINTER(hyena_film_t), i, i, i, i, i, vp, vp], i),
         "hyena_fftconv2d_gate_forward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, vp, vp,
@@ -400,30 +403,47 @@ def hyena_fftconv_gate_backward_circular(v: torch.Tensor, xs, bias: torch.Tensor
     return dv, dxs, dh, db
 
 
-def hyena_filter_rfft_circular(h: torch.Tensor, *, out=None, stream=None):
+def _circ_ws(fn, name, args, workspace, device):
+    """The workspace of a circular-mode call: none up to L = 16384, else the
+    caller's or a fresh one of the size the library asks for."""
+    n = fn(*args)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError(name, HYENA_ERR_UNSUPPORTED, "invalid sizes")
+    if n == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(n, device=device, dtype=torch.uint8)
+    return ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
+
+
+def hyena_filter_rfft_circular(h: torch.Tensor, *, out=None, workspace=None, stream=None):
     """Circular-mode spectra H [N][D][L/2] complex64 of filters h [N][D][L]
     (the L-point DFT without padding, packed: slot 0 = (bin 0, bin L/2))."""
     N, D, L = h.shape
     if out is None:
         out = torch.empty((N, D, L // 2), device=h.device, dtype=torch.complex64)
+    wp, wn = _circ_ws(LIB.hyena_filter_rfft_circular_workspace_size, "hyena_filter_rfft_circular_workspace_size",
+                      (N, D, L), workspace, h.device)
     _check("hyena_filter_rfft_circular", LIB.hyena_filter_rfft_circular(
         ctypes.c_void_p(_dev(h, torch.float32, "h")), N, D, L,
-        ctypes.c_void_p(_dev(out, torch.complex64, "H")), _stream(stream)))
+        ctypes.c_void_p(_dev(out, torch.complex64, "H")), wp, wn, _stream(stream)))
     return out
 
 
 def hyena_fftconv_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor, *,
-                                        out=None, stream=None):
+                                        out=None, workspace=None, stream=None):
     """The order-N forward with circular convolutions of length L."""
     B, D, L = v.shape
     N = len(xs)
     xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
     if out is None:
         out = torch.empty_like(v)
+    wp, wn = _circ_ws(LIB.hyena_fftconv_circular_workspace_size, "hyena_fftconv_circular_workspace_size",
+                      (B, D, L, N), workspace, v.device)
     _check("hyena_fftconv_gate_forward_circular", LIB.hyena_fftconv_gate_forward_circular(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io_dtype(v),
-        ctypes.c_void_p(_dev(out, v.dtype, "y")), _stream(stream)))
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), wp, wn, _stream(stream)))
     return out
 
 

@@ -102,6 +102,8 @@ WORKLOADS = {
                            film=True),
     # circular mode (periodic boundaries) at the shapes of c1, c4 and c5_3d
     "c1_circ": Workload("c1_circ", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), circular=True),
+    "c3_64k_circ": Workload("c3_64k_circ", "1d", N=2, B=1, D=256, L=65536, io="f32", seed=_seed(3, 0),
+                            circular=True),
     "c4_circ": Workload("c4_circ", "2d", N=2, B=2, D=128, H=256, W=256, io="f32", seed=_seed(4), circular=True),
     "c5_3d_circ": Workload("c5_3d_circ", "3d", N=2, B=2, D=32, Z=64, H=64, W=64, io="bf16", seed=_seed(5),
                            circular=True),

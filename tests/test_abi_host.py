@@ -167,15 +167,28 @@ def test_backward_rejects_bad_arguments(lib):
 def test_circular_rejects_bad_arguments(lib):
     xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
     f = lib.hyena_fftconv_gate_forward_circular
-    assert f(P(0), xs, P(3), P(4), 2, 3, 16, 2, F32, P(5), None) == UNSUPPORTED   # L < 32
-    assert f(P(0), xs, P(3), P(4), 2, 3, 1 << 15, 2, F32, P(5), None) == UNSUPPORTED
-    assert f(P(0), xs, P(3), P(4), 2, 3, 96, 2, F32, P(5), None) == UNSUPPORTED   # not a power of two
-    assert f(None, xs, P(3), P(4), 2, 3, 64, 2, F32, P(5), None) == INVALID
-    assert f(P(0), xs, P(3), P(4), 2, 3, 64, 2, F32, P(0), None) == INVALID       # y aliases v
+    assert f(P(0), xs, P(3), P(4), 2, 3, 16, 2, F32, P(5), None, 0, None) == UNSUPPORTED   # L < 32
+    assert f(P(0), xs, P(3), P(4), 2, 3, 1 << 23, 2, F32, P(5), None, 0, None) == UNSUPPORTED
+    assert f(P(0), xs, P(3), P(4), 2, 3, 96, 2, F32, P(5), None, 0, None) == UNSUPPORTED   # not a power of two
+    assert f(None, xs, P(3), P(4), 2, 3, 64, 2, F32, P(5), None, 0, None) == INVALID
+    assert f(P(0), xs, P(3), P(4), 2, 3, 64, 2, F32, P(0), None, 0, None) == INVALID       # y aliases v
+    # above 16384 the four-step path needs a workspace
+    assert f(P(0), xs, P(3), P(4), 2, 3, 1 << 15, 2, F32, P(5), None, 0, None) == WORKSPACE
     r = lib.hyena_filter_rfft_circular
-    assert r(P(0), 2, 3, 16, P(1), None) == UNSUPPORTED
-    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + BIG + 8), None) == INVALID
-    assert r(P(0), 2, 3, 64, P(0), None) == INVALID                               # H overlaps h
+    assert r(P(0), 2, 3, 16, P(1), None, 0, None) == UNSUPPORTED
+    assert r(P(0), 2, 3, 64, ctypes.c_void_p(A + BIG + 8), None, 0, None) == INVALID
+    assert r(P(0), 2, 3, 64, P(0), None, 0, None) == INVALID                               # H overlaps h
+    assert r(P(0), 2, 3, 1 << 16, P(1), None, 0, None) == WORKSPACE
+
+
+def test_circular_workspace_sizes(lib):
+    ws = lib.hyena_fftconv_circular_workspace_size
+    rs = lib.hyena_filter_rfft_circular_workspace_size
+    ws.restype = rs.restype = ctypes.c_size_t
+    assert ws(2, 3, 1 << 14, 2) == 0 and rs(2, 3, 1 << 14) == 0
+    assert ws(2, 3, 1 << 16, 2) >= 6 * (1 << 15) * 8 and ws(2, 3, 1 << 16, 2) % 256 == 0
+    assert rs(2, 3, 1 << 16) >= 6 * (1 << 15) * 8
+    assert ws(2, 3, 16, 2) == ctypes.c_size_t(-1).value and rs(2, 3, 1 << 23) == ctypes.c_size_t(-1).value
 
 
 def test_filter_rfft_rejects_bad_arguments(lib):

@@ -118,3 +118,59 @@ def test_backward_circular_rejects_unsupported_lengths(hy):
     for L in (16, 32768):
         with pytest.raises(HyenaError):
             hy.hyena_fftconv_backward_circular_workspace_size(4, L, 2)
+
+
+# ------------------------------------------- long sequences (four-step)
+
+@pytest.mark.parametrize("L", [32768, 65536, 262144])
+def test_rfft_circular_long_matches_oracle(hy, L):
+    h = filters(2, 2, L, L)
+    Hp = hy.hyena_filter_rfft_circular(dev(h)).cpu().numpy().astype(np.complex128)
+    ref = oracle.rfft_circ(h)
+    got = np.empty_like(ref)
+    got[..., 1:L // 2] = Hp[..., 1:]
+    got[..., 0] = Hp[..., 0].real
+    got[..., L // 2] = Hp[..., 0].imag
+    assert rel_max_err(got, ref) <= 2e-5
+
+
+@pytest.mark.parametrize("B,D,L,N,io", [
+    (2, 2, 32768, 2, "f32"), (1, 3, 65536, 3, "bf16"), (2, 2, 1 << 20, 1, "f32"),
+    (3, 11, 262144, 2, "f32"),      # a wave holds 32 sequences: channel 10 spans two waves
+])
+def test_forward_circular_long_matches_oracle(hy, B, D, L, N, io):
+    wl, inp = random_problem(B, D, L, N, seed=950 + N, io=io)
+    h = filters(N, D, L, seed=L + 11)
+    H = hy.hyena_filter_rfft_circular(dev(h))
+    y = hy.hyena_fftconv_gate_forward_circular(dev(inp["v"], io), [dev(x, io) for x in inp["x"]],
+                                               dev(inp["b"]), H)
+    torch.cuda.synchronize()
+    ref = oracle.hyena_forward_circular(inp["v"], np.stack(inp["x"]), h, inp["b"])
+    assert_close(host(y), ref, io, f"circular B{B} D{D} L{L} N{N} {io}")
+
+
+def test_circular_shift_filter_rotates_at_4m(hy):
+    # L = 2^22 (the longest): h = delta_k, b = 0, x = 1 gives y = roll(v, k)
+    B, D, L, k = 1, 2, 1 << 22, 123457
+    v = np.random.default_rng(2).standard_normal((B, D, L)).astype(np.float32)
+    h = np.zeros((1, D, L), np.float32)
+    h[:, :, k] = 1.0
+    H = hy.hyena_filter_rfft_circular(dev(h))
+    y = hy.hyena_fftconv_gate_forward_circular(dev(v), [dev(np.ones_like(v))], dev(np.zeros((1, D), np.float32)), H)
+    torch.cuda.synchronize()
+    assert rel_max_err(host(y), np.roll(v, k, axis=-1)) <= 1e-5
+
+
+def test_circular_long_on_zero_padded_sequences_is_the_linear_forward(hy):
+    # length 2L with v, x_n and h_n zero beyond L: the circular recurrence's
+    # first L outputs are the linear forward's (both through the four-step)
+    B, D, L, N = 2, 3, 32768, 2
+    wl, inp = random_problem(B, D, L, N, seed=77)
+    h = filters(N, D, L, seed=78)
+    pad = lambda a: np.concatenate([a, np.zeros_like(a)], axis=-1)
+    yc = hy.hyena_fftconv_gate_forward_circular(dev(pad(inp["v"])), [dev(pad(x)) for x in inp["x"]],
+                                                dev(inp["b"]), hy.hyena_filter_rfft_circular(dev(pad(h))))
+    yl = hy.hyena_fftconv_gate_forward(dev(inp["v"]), [dev(x) for x in inp["x"]], dev(inp["b"]),
+                                       H=hy.hyena_filter_rfft(dev(h)))
+    torch.cuda.synchronize()
+    assert rel_max_err(host(yc)[..., :L], host(yl).astype(np.float64)) <= 1e-5
