@@ -345,3 +345,64 @@ def test_filter_gen_3d_rejects_bad_arguments(lib):
     assert f(ctypes.byref(ffn), 2, 3, 4, 8, 16, None, None) == INVALID           # no output
     ffn.width = 65
     assert f(ctypes.byref(ffn), 2, 3, 4, 8, 16, P(5), None) == UNSUPPORTED        # width > 64
+
+
+def test_backward_variants_reject_bad_arguments(lib):
+    bad = ctypes.c_size_t(-1).value
+    # per-sample: B dh spectra; any L up to 2^22
+    ps = lib.hyena_fftconv_backward_per_sample_workspace_size
+    assert ps(4, 3, 64, 2) >= 4 * 2 * 3 * 64 * 8 + 12 * 2 * 3 * 64
+    assert ps(4, 3, 1 << 15, 2) > lib.hyena_fftconv_backward_workspace_size(3, 1 << 15, 2)
+    assert ps(4, 3, 1 << 23, 2) == bad and ps(0, 3, 64, 2) == bad
+    # circular: 32 <= L <= 16384
+    cs = lib.hyena_fftconv_backward_circular_workspace_size
+    assert cs(3, 64, 2) >= 12 * 2 * 3 * 64
+    assert cs(3, 16, 2) == bad and cs(3, 1 << 15, 2) == bad and cs(3, 96, 2) == bad
+    xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
+    dxs = (ctypes.c_void_p * 2)(P(7).value, P(8).value)
+    f = lib.hyena_fftconv_gate_backward_circular
+    args = lambda **k: [k.get("v", P(0)), xs, P(3), P(4), P(5), 2, 3, k.get("L", 64), 2, F32, k.get("dv", P(6)),
+                        dxs, k.get("dh", P(9)), P(10), k.get("ws", P(11)), k.get("nb", 1 << 24), None]
+    assert f(*args(L=16)) == UNSUPPORTED
+    assert f(*args(L=1 << 15)) == UNSUPPORTED
+    assert f(*args(v=None)) == INVALID
+    assert f(*args(ws=None)) == WORKSPACE
+    assert f(*args(dv=P(0))) == INVALID                                          # dv aliases v
+    g = lib.hyena_fftconv_gate_backward_per_sample
+    # dh of B N D L floats: an output that starts inside it overlaps
+    pa = lambda **k: [P(0), xs, P(3), P(4), P(5), 2, 3, 64, 2, F32, P(6), dxs, P(9),
+                      k.get("db", P(10)), P(11), 1 << 24, None]
+    assert g(*pa(db=ctypes.c_void_p(A + 9 * BIG + 4 * 2 * 2 * 3 * 64 - 64))) == INVALID
+    # 2-D variants
+    ws2 = lib.hyena_fftconv2d_backward_per_sample_workspace_size
+    wc2 = lib.hyena_fftconv2d_backward_circular_workspace_size
+    assert ws2(3, 2, 32, 64, 2) > lib.hyena_fftconv2d_backward_workspace_size(3, 2, 32, 64, 2)
+    assert wc2(3, 2, 32, 64, 2) < lib.hyena_fftconv2d_backward_workspace_size(3, 2, 32, 64, 2)
+    assert wc2(3, 2, 32, 16, 2) == bad and ws2(3, 2, 8, 64, 2) == bad
+    h2 = lib.hyena_fftconv2d_gate_backward_circular
+    a2 = lambda **k: [P(0), xs, k.get("Hs", P(3)), P(4), P(5), 2, 3, 32, k.get("W", 64), 2, F32, P(6), dxs, P(9),
+                      P(10), P(11), 1 << 26, None]
+    assert h2(*a2(W=16)) == UNSUPPORTED
+    assert h2(*a2(Hs=None)) == INVALID
+
+
+def test_3d_per_sample_entries_reject_bad_arguments(lib):
+    from subquadratic_sequence_b200 import hyena
+    f = lib.hyena_filter_gen_film_3d
+    ffn = hyena.hyena_ffn_t(P(0).value, P(1).value, P(2).value, P(3).value, P(4).value, 8, 64, 64.0)
+    film = hyena.hyena_film_t(None, None, None, None)
+    assert f(ctypes.byref(ffn), None, 2, 2, 3, 4, 8, 16, P(5), None) == INVALID      # no film struct
+    assert f(ctypes.byref(ffn), ctypes.byref(film), 0, 2, 3, 4, 8, 16, P(5), None) == INVALID   # B < 1
+    film.gamma = ctypes.c_void_p(A + 6 * BIG + 2).value
+    assert f(ctypes.byref(ffn), ctypes.byref(film), 2, 2, 3, 4, 8, 16, P(5), None) == INVALID  # misaligned
+    film.gamma = None
+    ffn.n_bands = 11
+    assert f(ctypes.byref(ffn), ctypes.byref(film), 2, 2, 3, 4, 8, 16, P(5), None) == UNSUPPORTED
+    g = lib.hyena_fftconv3d_gate_forward_per_sample
+    xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
+    a = lambda **k: [P(0), xs, k.get("Hs", P(3)), P(4), 2, 3, 16, 16, k.get("W", 16), 2, F32, k.get("y", P(5)),
+                     P(6), 1 << 28, None]
+    assert g(*a(Hs=None)) == INVALID
+    assert g(*a(W=8)) == UNSUPPORTED
+    assert g(*a(y=P(0))) == INVALID                                              # y aliases v
+    assert g(*a(Hs=ctypes.c_void_p(A + 3 * BIG + 8))) == INVALID
