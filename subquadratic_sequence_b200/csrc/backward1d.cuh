@@ -69,6 +69,9 @@ backward1d_kernel(Backward1dArgs args)
     constexpr int M = F::M, E = F::E, T = F::T, RF = F::P::RF;
     constexpr int SEQ = F::SEQ;                 // packed pairs per sequence: M/2 (padded), M (circular)
     constexpr int NIO = PAD ? E / 2 : E;        // io registers per thread
+    // dh-spectrum update in three sweeps (loads batched ahead of stores)
+    // except at M = 16384, where it would spill
+    constexpr bool BATCH_ACC = LOG2M <= 13;
     extern __shared__ __align__(16) float2 smem_dyn[];
 
     const int g = threadIdx.x / T, t = threadIdx.x % T;
@@ -144,33 +147,57 @@ backward1d_kernel(Backward1dArgs args)
                     constexpr int i = decltype(ii)::value;
                     z[i] = zr[i * T + t];
                 });
-                // three sweeps so that the accumulator's loads are all issued
-                // before any of its stores (interleaved, each load would wait
-                // for the stores before it): the products, in place of z;
-                // the partial sums read back; the sums written
-                F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
-                    const float2 e1 = a[i1], e2 = a[i2];
-                    if (kind == 1) {
-                        // slot 0: bins 0 and M, both real
-                        z[i1] = make_float2((e1.x + e1.y) * (z[i1].x + z[i1].y),
-                                            (e1.x - e1.y) * (z[i1].x - z[i1].y));
-                    } else {
-                        float2 E1, E2, Z1, Z2;
-                        split_pair(e1, e2, w, E1, E2);
-                        split_pair(z[i1], z[i2], w, Z1, Z2);
-                        z[i1] = cmulc(E1, Z1);
-                        if (kind == 0) z[i2] = cmulc(E2, Z2);
-                    }
-                });
-                if (!first)
-                    F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2) {
-                        z[i1] = cadd(z[i1], acc[k]);
-                        if (kind == 0) z[i2] = cadd(z[i2], acc[M - k]);
+                if constexpr (BATCH_ACC) {
+                    // three sweeps so that the accumulator's loads are all issued
+                    // before any of its stores (interleaved, each load would wait
+                    // for the stores before it): the products, in place of z;
+                    // the partial sums read back; the sums written
+                    F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
+                        const float2 e1 = a[i1], e2 = a[i2];
+                        if (kind == 1) {
+                            // slot 0: bins 0 and M, both real
+                            z[i1] = make_float2((e1.x + e1.y) * (z[i1].x + z[i1].y),
+                                                (e1.x - e1.y) * (z[i1].x - z[i1].y));
+                        } else {
+                            float2 E1, E2, Z1, Z2;
+                            split_pair(e1, e2, w, E1, E2);
+                            split_pair(z[i1], z[i2], w, Z1, Z2);
+                            z[i1] = cmulc(E1, Z1);
+                            if (kind == 0) z[i2] = cmulc(E2, Z2);
+                        }
                     });
-                F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2) {
-                    acc[k] = z[i1];
-                    if (kind == 0) acc[M - k] = z[i2];
-                });
+                    if (!first)
+                        F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2) {
+                            z[i1] = cadd(z[i1], acc[k]);
+                            if (kind == 0) z[i2] = cadd(z[i2], acc[M - k]);
+                        });
+                    F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2) {
+                        acc[k] = z[i1];
+                        if (kind == 0) acc[M - k] = z[i2];
+                    });
+                } else {
+                    // one read-modify-write per pair (at L = 16384 the kernel
+                    // runs at 128 registers and the sweeps above spill more
+                    // than they save)
+                    F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
+                        const float2 e1 = a[i1], e2 = a[i2];
+                        if (kind == 1) {
+                            const float2 p = make_float2((e1.x + e1.y) * (z[i1].x + z[i1].y),
+                                                         (e1.x - e1.y) * (z[i1].x - z[i1].y));
+                            acc[0] = first ? p : cadd(acc[0], p);
+                        } else {
+                            float2 E1, E2, Z1, Z2;
+                            split_pair(e1, e2, w, E1, E2);
+                            split_pair(z[i1], z[i2], w, Z1, Z2);
+                            const float2 p1 = cmulc(E1, Z1);
+                            acc[k] = first ? p1 : cadd(acc[k], p1);
+                            if (kind == 0) {
+                                const float2 p2 = cmulc(E2, Z2);
+                                acc[M - k] = first ? p2 : cadd(acc[M - k], p2);
+                            }
+                        }
+                    });
+                }
             }
             const float2* Hs = stage;
             if constexpr (F::H_IN_EXCHANGE) {

@@ -126,9 +126,13 @@ fft3d_z_kernel(Fft2dArgs a)
         const int qa = max(a.q0, c * a.B), qb = min(a.q0 + a.nq, (c + 1) * a.B);
         const float bias = __ldg(a.bias + a.n * a.C + c);
         const float2* Hn = a.Hs + ((size_t)a.n * a.C + c) * Z2 * plane;   // [2Z][2H][W]
-        // per-sample spectra (MODE 2): volume q = c B + b takes sample b's set
-        constexpr bool PS = MODE == 2;
-        auto spectra_of = [&](int q) { return PS ? Hn + (size_t)(q - c * a.B) * a.Hs_bstride : Hn; };
+        // per-sample spectra (MODE 2): volume q = c B + b takes sample b's set.
+        // The mode is a template parameter, so the shared kernel carries no
+        // branch; inside MODE 2 the branch stays a run-time one, which measured
+        // faster than the compile-time form (that one lets the compiler move the
+        // next volume's filter loads ahead and spill)
+        const bool ps = MODE == 2 && a.Hs_bstride != 0;
+        auto spectra_of = [&](int q) { return ps ? Hn + (size_t)(q - c * a.B) * a.Hs_bstride : Hn; };
         const float s = 1.0f / ((float)Z2 * (float)H2);
         if (!pair_cta) {
             // the filter column, (H + b) / (2Z 2H), in register order; loaded
@@ -141,9 +145,9 @@ fft3d_z_kernel(Fft2dArgs a)
                     hv[r] = make_float2((h.x + bias) * s, h.y * s);
                 });
             };
-            if constexpr (!PS) load_filter(Hn);
+            if (!ps) load_filter(Hn);
             for (int q = qa; q < qb; ++q) {
-                if constexpr (PS) load_filter(spectra_of(q));
+                if (ps) load_filter(spectra_of(q));
                 float2* colp = a.S + (size_t)(q - a.q0) * a.zp * plane + (size_t)ky * W + kx;
                 load_col(colp);
                 FZ::template run<-1, true, PAD>(buf, reg, t);

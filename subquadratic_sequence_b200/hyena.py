@@ -765,6 +765,21 @@ def hyena_fftconv2d_gate_backward_per_sample(v: torch.Tensor, xs, bias: torch.Te
     return dv, dxs, dh, db
 
 
+def hyena_fftconv2d_backward_circular_workspace_size(B: int, C: int, H: int, W: int, N: int) -> int:
+    n = LIB.hyena_fftconv2d_backward_circular_workspace_size(B, C, H, W, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv2d_backward_circular_workspace_size", HYENA_ERR_UNSUPPORTED, "invalid sizes")
+    return n
+
+
+def hyena_fftconv2d_backward_per_sample_workspace_size(B: int, C: int, H: int, W: int, N: int) -> int:
+    n = LIB.hyena_fftconv2d_backward_per_sample_workspace_size(B, C, H, W, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv2d_backward_per_sample_workspace_size", HYENA_ERR_UNSUPPORTED,
+                         "invalid sizes")
+    return n
+
+
 def hyena_fftconv2d_gate_backward_circular(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
                                            dy: torch.Tensor, *, workspace=None, stream=None):
     """The backward of the circular 2-D forward (Hs [N][C][H][W/2] from
