@@ -226,6 +226,17 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, cons
                                                              int L, int N, hyena_dtype_t io, void* y,
                                                              void* workspace, size_t ws_bytes, void* stream);
 
+/* The circular forward with a spectrum set per sample (input-dependent
+ * filters in circular mode): H [B][N][D][L/2] from hyena_filter_rfft_circular
+ * of the B*N rows of D filters, sequence (b, d) multiplied by sample b's
+ * spectra.  Everything else (sizes, workspace) as
+ * hyena_fftconv_gate_forward_circular. */
+HYENA_API hyena_status_t hyena_fftconv_gate_forward_circular_per_sample(const void* v, const void* const* x,
+                                                                        const float* H, const float* bias, int B,
+                                                                        int D, int L, int N, hyena_dtype_t io,
+                                                                        void* y, void* workspace, size_t ws_bytes,
+                                                                        void* stream);
+
 /* The backward pass of the circular recurrence (hyena_fftconv_gate_forward_
  * circular), for training: the exact adjoint with every convolution
  * circular of length L, so both sums wrap around:
@@ -512,6 +523,16 @@ HYENA_API hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, co
                                                                void* y, void* workspace, size_t ws_bytes,
                                                                void* stream);
 
+/* The circular 2-D forward with a spectrum set per sample: Hs
+ * [B][N][C][H][W/2] (hyena_filter_rfft2d_circular of per-sample filters);
+ * otherwise as hyena_fftconv2d_gate_forward_circular. */
+HYENA_API hyena_status_t hyena_fftconv2d_gate_forward_circular_per_sample(const void* v, const void* const* x,
+                                                                          const float* Hs, const float* bias,
+                                                                          int B, int C, int H, int W, int N,
+                                                                          hyena_dtype_t io, void* y,
+                                                                          void* workspace, size_t ws_bytes,
+                                                                          void* stream);
+
 /* ------------------------------------------------------- circular 3-D */
 
 /* Circular 3-D filter spectra Hs [N][C][Z][H][W/2] complex64 for filters
@@ -537,6 +558,17 @@ HYENA_API hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, co
                                                                int C, int Z, int H, int W, int N,
                                                                hyena_dtype_t io, void* y, void* workspace,
                                                                size_t ws_bytes, void* stream);
+
+/* The circular 3-D forward with a spectrum set per sample: Hs
+ * [B][N][C][Z][H][W/2] (hyena_filter_rfft3d_circular of per-sample filters,
+ * e.g. from hyena_filter_gen_film_3d); otherwise as
+ * hyena_fftconv3d_gate_forward_circular.  B*N*C*Z*H <= 2^30. */
+HYENA_API hyena_status_t hyena_fftconv3d_gate_forward_circular_per_sample(const void* v, const void* const* x,
+                                                                          const float* Hs, const float* bias,
+                                                                          int B, int C, int Z, int H, int W,
+                                                                          int N, hyena_dtype_t io, void* y,
+                                                                          void* workspace, size_t ws_bytes,
+                                                                          void* stream);
 
 /* ------------------------------------------------------- 2-D backward */
 

@@ -501,3 +501,18 @@ def hyena_forward_3d_per_sample(v, x, h, bias, route="fft") -> np.ndarray:
     return np.concatenate([hyena_forward_3d(v[b:b + 1], x[:, b:b + 1], h[b], bias, route)
                            for b in range(v.shape[0])])
 
+
+def hyena_forward_circular_per_sample(v, x, h, bias, route="fft", threads=None) -> np.ndarray:
+    """The circular 1-D forward with a filter set per sample, h [B][N][D][L]:
+    :func:`hyena_forward_circular` applied to each sample with its own filters."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    return np.concatenate([hyena_forward_circular(v[b:b + 1], x[:, b:b + 1], h[b], bias, route, threads)
+                           for b in range(v.shape[0])])
+
+
+def hyena_forward_circular_nd_per_sample(v, x, h, bias, route="fft") -> np.ndarray:
+    """The circular 2-D / 3-D forward with a filter set per sample, h
+    [B][N][C][(Z)][H][W]: :func:`hyena_forward_circular_nd` per sample."""
+    v, x, h, bias = map(_f64, (v, x, h, bias))
+    return np.concatenate([hyena_forward_circular_nd(v[b:b + 1], x[:, b:b + 1], h[b], bias, route)
+                           for b in range(v.shape[0])])

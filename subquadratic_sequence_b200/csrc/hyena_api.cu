@@ -428,7 +428,7 @@ size_t hyena_fftconv_circular_workspace_size(int B, int D, int L, int N)
     return k - 1 <= kMaxLog2Circ ? 0 : round_up(scratch_bytes((long)B * D, L / 2), 256);
 }
 
-hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* const* x, const float* H,
+static hyena_status_t hyena_fftconv_gate_forward_circular_impl(bool per_sample, const void* v, const void* const* x, const float* H,
                                                    const float* bias, int B, int D, int L, int N,
                                                    hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes,
                                                    void* stream)
@@ -444,7 +444,7 @@ hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* co
     if (!aligned(v, 16) || !aligned(y, 16) || !aligned(H, 16) || !aligned(bias, 4))
         return HYENA_ERR_INVALID_ARG;
     const size_t act = (size_t)B * D * L * io_bytes(io);
-    const size_t spec = sizeof(float2) * (size_t)N * D * (L / 2);
+    const size_t spec = sizeof(float2) * (size_t)N * D * (L / 2) * (per_sample ? (size_t)B : 1);
     if (overlap(y, act, v, act) || overlap(y, act, H, spec) || overlap(y, act, bias, sizeof(float) * N * D))
         return HYENA_ERR_INVALID_ARG;
     for (int n = 0; n < N; ++n)
@@ -466,6 +466,7 @@ hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* co
         for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
         a.y = y;
         a.H = reinterpret_cast<const float2*>(H);
+        a.H_bstride = per_sample ? (size_t)N * D * (L / 2) : 0;
         a.bias = bias;
         a.B = B;
         a.D = D;
@@ -478,12 +479,32 @@ hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* co
     for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
     a.y = y;
     a.H = reinterpret_cast<const float2*>(H);
+    a.H_bstride = per_sample ? (size_t)N * D * (L / 2) : 0;
     a.bias = bias;
     a.B = B;
     a.D = D;
     a.N = N;
+    if (per_sample)
+        return io == HYENA_BF16 ? dispatch_fused_circ_ps_bf16(k - 1, a, st) : dispatch_fused_circ_ps_f32(k - 1, a, st);
     return io == HYENA_BF16 ? dispatch_fused_circ_bf16(k - 1, a, st) : dispatch_fused_circ_f32(k - 1, a, st);
 }
+
+hyena_status_t hyena_fftconv_gate_forward_circular(const void* v, const void* const* x, const float* H,
+                                                   const float* bias, int B, int D, int L, int N,
+                                                   hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes,
+                                                   void* stream)
+{
+    return hyena_fftconv_gate_forward_circular_impl(false, v, x, H, bias, B, D, L, N, io, y, workspace, ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv_gate_forward_circular_per_sample(const void* v, const void* const* x, const float* H,
+                                                   const float* bias, int B, int D, int L, int N,
+                                                   hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes,
+                                                   void* stream)
+{
+    return hyena_fftconv_gate_forward_circular_impl(true, v, x, H, bias, B, D, L, N, io, y, workspace, ws_bytes, stream);
+}
+
 
 size_t hyena_fftconv_backward_workspace_size(int D, int L, int N)
 {
@@ -971,7 +992,7 @@ hyena_status_t hyena_filter_rfft2d_circular(const float* h, int N, int C, int H,
     return dispatch_rfft2d_circ(lm, lh, a, (cudaStream_t)stream);
 }
 
-hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, const void* const* x, const float* Hs,
+static hyena_status_t hyena_fftconv2d_gate_forward_circular_impl(bool per_sample, const void* v, const void* const* x, const float* Hs,
                                                      const float* bias, int B, int C, int H, int W, int N,
                                                      hyena_dtype_t io, void* y, void* workspace,
                                                      size_t ws_bytes, void* stream)
@@ -987,7 +1008,7 @@ hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, const void* 
         if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
     if (!aligned(v, 16) || !aligned(y, 16) || !aligned(bias, 4) || !aligned(Hs, 16)) return HYENA_ERR_INVALID_ARG;
     const size_t act = (size_t)B * C * H * W * io_bytes(io);
-    const size_t spec = sizeof(float2) * (size_t)N * C * H * (W / 2);
+    const size_t spec = sizeof(float2) * (size_t)N * C * H * (W / 2) * (per_sample ? (size_t)B : 1);
     const size_t need = hyena_fftconv2d_circular_workspace_size(B, C, H, W);
     if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
     if (overlap(y, act, v, act) || overlap(y, act, bias, sizeof(float) * N * C) || overlap(y, act, Hs, spec) ||
@@ -1000,6 +1021,7 @@ hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, const void* 
     for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
     a.y = y;
     a.Hs = reinterpret_cast<const float2*>(Hs);
+    a.Hs_bstride = per_sample ? (size_t)N * C * H * (W / 2) : 0;
     a.bias = bias;
     a.B = B;
     a.C = C;
@@ -1010,6 +1032,23 @@ hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, const void* 
     return io == HYENA_BF16 ? dispatch_fft2d_circ_bf16(lm, lh, a, N, scratch, st)
                             : dispatch_fft2d_circ_f32(lm, lh, a, N, scratch, st);
 }
+
+hyena_status_t hyena_fftconv2d_gate_forward_circular(const void* v, const void* const* x, const float* Hs,
+                                                     const float* bias, int B, int C, int H, int W, int N,
+                                                     hyena_dtype_t io, void* y, void* workspace,
+                                                     size_t ws_bytes, void* stream)
+{
+    return hyena_fftconv2d_gate_forward_circular_impl(false, v, x, Hs, bias, B, C, H, W, N, io, y, workspace, ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv2d_gate_forward_circular_per_sample(const void* v, const void* const* x, const float* Hs,
+                                                     const float* bias, int B, int C, int H, int W, int N,
+                                                     hyena_dtype_t io, void* y, void* workspace,
+                                                     size_t ws_bytes, void* stream)
+{
+    return hyena_fftconv2d_gate_forward_circular_impl(true, v, x, Hs, bias, B, C, H, W, N, io, y, workspace, ws_bytes, stream);
+}
+
 
 }  // extern "C"
 
@@ -1062,7 +1101,7 @@ hyena_status_t hyena_filter_rfft3d_circular(const float* h, int N, int C, int Z,
     return dispatch_rfft3d(lm, lh, lz, a, (cudaStream_t)stream, false);
 }
 
-hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, const void* const* x, const float* Hs,
+static hyena_status_t hyena_fftconv3d_gate_forward_circular_impl(bool per_sample, const void* v, const void* const* x, const float* Hs,
                                                      const float* bias, int B, int C, int Z, int H, int W,
                                                      int N, hyena_dtype_t io, void* y, void* workspace,
                                                      size_t ws_bytes, void* stream)
@@ -1073,13 +1112,14 @@ hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, const void* 
     if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
     int lz, lh, lm;
     if (!dims3d_circ_ok(Z, H, W, lz, lh, lm)) return HYENA_ERR_UNSUPPORTED;
-    if ((long)B * C > (1L << 20) || (long)N * C * Z * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    if ((long)B * C > (1L << 20) || (long)N * C * Z * H * (per_sample ? B : 1) > (1L << 30))
+        return HYENA_ERR_UNSUPPORTED;
     for (int n = 0; n < N; ++n)
         if (!x[n] || !aligned(x[n], 16)) return HYENA_ERR_INVALID_ARG;
     if (!aligned(v, 16) || !aligned(y, 16) || !aligned(bias, 4) || !aligned(Hs, 16)) return HYENA_ERR_INVALID_ARG;
     const size_t vol = (size_t)Z * H * W;
     const size_t act = (size_t)B * C * vol * io_bytes(io);
-    const size_t spec = sizeof(float2) * (size_t)N * C * (vol / 2);
+    const size_t spec = sizeof(float2) * (size_t)N * C * (vol / 2) * (per_sample ? (size_t)B : 1);
     const size_t need = hyena_fftconv3d_circular_workspace_size(B, C, Z, H, W);
     if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
     if (overlap(y, act, v, act) || overlap(y, act, bias, sizeof(float) * N * C) || overlap(y, act, Hs, spec) ||
@@ -1092,6 +1132,7 @@ hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, const void* 
     for (int n = 0; n < kMaxOrder; ++n) a.x[n] = n < N ? x[n] : nullptr;
     a.y = y;
     a.Hs = reinterpret_cast<const float2*>(Hs);
+    a.Hs_bstride = per_sample ? (size_t)N * C * (vol / 2) : 0;
     a.bias = bias;
     a.B = B;
     a.C = C;
@@ -1103,6 +1144,23 @@ hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, const void* 
     return io == HYENA_BF16 ? dispatch_fft3d_bf16(lm, lh, lz, a, N, scratch, st, false)
                             : dispatch_fft3d_f32(lm, lh, lz, a, N, scratch, st, false);
 }
+
+hyena_status_t hyena_fftconv3d_gate_forward_circular(const void* v, const void* const* x, const float* Hs,
+                                                     const float* bias, int B, int C, int Z, int H, int W,
+                                                     int N, hyena_dtype_t io, void* y, void* workspace,
+                                                     size_t ws_bytes, void* stream)
+{
+    return hyena_fftconv3d_gate_forward_circular_impl(false, v, x, Hs, bias, B, C, Z, H, W, N, io, y, workspace, ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv3d_gate_forward_circular_per_sample(const void* v, const void* const* x, const float* Hs,
+                                                     const float* bias, int B, int C, int Z, int H, int W,
+                                                     int N, hyena_dtype_t io, void* y, void* workspace,
+                                                     size_t ws_bytes, void* stream)
+{
+    return hyena_fftconv3d_gate_forward_circular_impl(true, v, x, Hs, bias, B, C, Z, H, W, N, io, y, workspace, ws_bytes, stream);
+}
+
 
 }  // extern "C"
 

@@ -15,11 +15,9 @@ hyena_status_t launch_z3d_n(int mode, const Fft2dArgs& a, cudaStream_t st)
     // regular CTAs and its pair CTAs
     const long nch = (long)(a.q0 + a.nq - 1) / a.B - a.q0 / a.B + 1;
     const long npair = (H2 / 2 + 1 + ZL::TC / 2 - 1) / (ZL::TC / 2);
-    if constexpr (PAD) {
-        if (a.Hs_bstride != 0)        // a spectrum set per sample
-            return launch(fft3d_z_kernel<LOG2Z2, 2, PAD>, (unsigned)(nch * (reg + npair)), ZL::THREADS, ZL::SMEM,
-                          st, a, false);
-    }
+    if (a.Hs_bstride != 0)            // a spectrum set per sample
+        return launch(fft3d_z_kernel<LOG2Z2, 2, PAD>, (unsigned)(nch * (reg + npair)), ZL::THREADS, ZL::SMEM,
+                      st, a, false);
     return launch(fft3d_z_kernel<LOG2Z2, 0, PAD>, (unsigned)(nch * (reg + npair)), ZL::THREADS, ZL::SMEM, st,
                   a, false);
 }

@@ -78,6 +78,8 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv_circular_workspace_size": ([i, i, i, i], sz),
         "hyena_fftconv_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp, sz,
                                                  vp], i),
+        "hyena_fftconv_gate_forward_circular_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp,
+                                                            sz, vp], i),
         "hyena_filter_rfft2d": ([vp, i, i, i, i, vp, vp], i),
         "hyena_filter_gen_film_2d": ([ffn_p, ctypes.POINTER(hyena_film_t), i, i, i, i, i, vp, vp], i),
         "hyena_fftconv2d_gate_forward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, vp, vp,
@@ -104,9 +106,13 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv3d_circular_workspace_size": ([i, i, i, i, i], sz),
         "hyena_fftconv3d_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, i, vp, vp,
                                                    sz, vp], i),
+        "hyena_fftconv3d_gate_forward_circular_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, i,
+                                                              vp, vp, sz, vp], i),
         "hyena_fftconv2d_circular_workspace_size": ([i, i, i, i], sz),
         "hyena_fftconv2d_gate_forward_circular": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, vp, vp,
                                                    sz, vp], i),
+        "hyena_fftconv2d_gate_forward_circular_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, i, vp,
+                                                              vp, sz, vp], i),
         "hyena_fftconv3d_workspace_size": ([i, i, i, i, i, i, i, i], sz),
         "hyena_fftconv3d_gate_forward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, i,
                                           vp, vp, sz, vp], i),
@@ -431,7 +437,8 @@ def hyena_filter_rfft_circular(h: torch.Tensor, *, out=None, workspace=None, str
 
 
 def hyena_fftconv_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor, *,
-                                        out=None, workspace=None, stream=None):
+                                        out=None, workspace=None, stream=None,
+                                        _name="hyena_fftconv_gate_forward_circular"):
     """The order-N forward with circular convolutions of length L."""
     B, D, L = v.shape
     N = len(xs)
@@ -440,11 +447,18 @@ def hyena_fftconv_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tensor,
         out = torch.empty_like(v)
     wp, wn = _circ_ws(LIB.hyena_fftconv_circular_workspace_size, "hyena_fftconv_circular_workspace_size",
                       (B, D, L, N), workspace, v.device)
-    _check("hyena_fftconv_gate_forward_circular", LIB.hyena_fftconv_gate_forward_circular(
+    _check(_name, getattr(LIB, _name)(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io_dtype(v),
         ctypes.c_void_p(_dev(out, v.dtype, "y")), wp, wn, _stream(stream)))
     return out
+
+
+def hyena_fftconv_gate_forward_circular_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor, *,
+                                                   out=None, workspace=None, stream=None):
+    """The circular forward with per-sample spectra H [B][N][D][L/2]."""
+    return hyena_fftconv_gate_forward_circular(v, xs, bias, H, out=out, workspace=workspace, stream=stream,
+                                               _name="hyena_fftconv_gate_forward_circular_per_sample")
 
 
 def hyena_filter_rfft2d(h: torch.Tensor, *, out=None, stream=None):
@@ -594,7 +608,8 @@ def hyena_fftconv2d_circular_workspace_size(B: int, C: int, H: int, W: int) -> i
 
 
 def hyena_fftconv2d_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor, *,
-                                          out=None, workspace=None, stream=None):
+                                          out=None, workspace=None, stream=None,
+                                          _name="hyena_fftconv2d_gate_forward_circular"):
     """The order-N recurrence with circular 2-D convolutions: v, x_n
     [B][C][H][W] (float32 or bf16), bias [N][C], Hs from
     hyena_filter_rfft2d_circular."""
@@ -607,12 +622,19 @@ def hyena_fftconv2d_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tenso
     if workspace is None:
         workspace = torch.empty(hyena_fftconv2d_circular_workspace_size(B, C, H, W), device=v.device,
                                 dtype=torch.uint8)
-    _check("hyena_fftconv2d_gate_forward_circular", LIB.hyena_fftconv2d_gate_forward_circular(
+    _check(_name, getattr(LIB, _name)(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, H, W, N, io,
         ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+def hyena_fftconv2d_gate_forward_circular_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                                     *, out=None, workspace=None, stream=None):
+    """The circular 2-D forward with per-sample spectra Hs [B][N][C][H][W/2]."""
+    return hyena_fftconv2d_gate_forward_circular(v, xs, bias, Hs, out=out, workspace=workspace, stream=stream,
+                                                  _name="hyena_fftconv2d_gate_forward_circular_per_sample")
 
 
 def hyena_filter_rfft3d_circular(h: torch.Tensor, *, out=None, stream=None):
@@ -635,7 +657,8 @@ def hyena_fftconv3d_circular_workspace_size(B: int, C: int, Z: int, H: int, W: i
 
 
 def hyena_fftconv3d_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor, *,
-                                          out=None, workspace=None, stream=None):
+                                          out=None, workspace=None, stream=None,
+                                          _name="hyena_fftconv3d_gate_forward_circular"):
     """The order-N recurrence with circular 3-D convolutions: v, x_n
     [B][C][Z][H][W] (float32 or bf16), bias [N][C], Hs from
     hyena_filter_rfft3d_circular."""
@@ -648,12 +671,19 @@ def hyena_fftconv3d_gate_forward_circular(v: torch.Tensor, xs, bias: torch.Tenso
     if workspace is None:
         workspace = torch.empty(hyena_fftconv3d_circular_workspace_size(B, C, Z, H, W), device=v.device,
                                 dtype=torch.uint8)
-    _check("hyena_fftconv3d_gate_forward_circular", LIB.hyena_fftconv3d_gate_forward_circular(
+    _check(_name, getattr(LIB, _name)(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, C, Z, H, W, N, io,
         ctypes.c_void_p(_dev(out, v.dtype, "y")), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+def hyena_fftconv3d_gate_forward_circular_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                                     *, out=None, workspace=None, stream=None):
+    """The circular 3-D forward with per-sample spectra Hs [B][N][C][Z][H][W/2]."""
+    return hyena_fftconv3d_gate_forward_circular(v, xs, bias, Hs, out=out, workspace=workspace, stream=stream,
+                                                  _name="hyena_fftconv3d_gate_forward_circular_per_sample")
 
 
 def hyena_fftconv2d_backward_workspace_size(B: int, C: int, H: int, W: int, N: int) -> int:

@@ -140,3 +140,24 @@ def test_circular_nd_routes_agree_and_differ_from_linear():
     d = oracle.hyena_forward_circular_nd(v, x, h, b, route="direct")
     assert rel_err(a, d) < 1e-12
     assert rel_err(a, oracle.hyena_forward_2d(v, x, h, b, route="direct")) > 1e-2
+
+
+def test_circular_per_sample_forward_is_each_sample_with_its_filters():
+    # equal sets give the shared circular forward; each sample's output is
+    # that sample alone through its own filters (1-D, 2-D and 3-D)
+    r = np.random.default_rng(70)
+    B, N, D, L = 3, 2, 2, 16
+    v, x = r.standard_normal((B, D, L)), r.standard_normal((N, B, D, L))
+    h, bias = r.standard_normal((B, N, D, L)) * 0.3, r.standard_normal((N, D))
+    shared = oracle.hyena_forward_circular(v, x, h[0], bias)
+    assert np.array_equal(oracle.hyena_forward_circular_per_sample(v, x, np.broadcast_to(h[0], h.shape), bias),
+                          shared)
+    ps = oracle.hyena_forward_circular_per_sample(v, x, h, bias)
+    for b in range(B):
+        assert np.array_equal(ps[b], oracle.hyena_forward_circular(v[b:b + 1], x[:, b:b + 1], h[b], bias)[0])
+    for grid in ((4, 8), (2, 4, 8)):
+        v, x = r.standard_normal((B, D) + grid), r.standard_normal((N, B, D) + grid)
+        h = r.standard_normal((B, N, D) + grid) * 0.3
+        ps = oracle.hyena_forward_circular_nd_per_sample(v, x, h, bias)
+        for b in range(B):
+            assert np.array_equal(ps[b], oracle.hyena_forward_circular_nd(v[b:b + 1], x[:, b:b + 1], h[b], bias)[0])

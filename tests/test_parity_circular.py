@@ -174,3 +174,29 @@ def test_circular_long_on_zero_padded_sequences_is_the_linear_forward(hy):
                                        H=hy.hyena_filter_rfft(dev(h)))
     torch.cuda.synchronize()
     assert rel_max_err(host(yc)[..., :L], host(yl).astype(np.float64)) <= 1e-5
+
+
+# ------------------------------------- per-sample spectra (input-dependent)
+
+@pytest.mark.parametrize("B,D,L,N,io", [(3, 4, 2048, 2, "f32"), (2, 3, 512, 2, "bf16"), (2, 2, 65536, 2, "f32")])
+def test_forward_circular_per_sample_matches_oracle(hy, B, D, L, N, io):
+    wl, inp = random_problem(B, D, L, N, seed=1100 + L, io=io)
+    h = np.stack([filters(N, D, L, seed=L + 13 + b) for b in range(B)])          # [B][N][D][L]
+    H = hy.hyena_filter_rfft_circular(dev(h.reshape(B * N, D, L))).reshape(B, N, D, L // 2)
+    y = hy.hyena_fftconv_gate_forward_circular_per_sample(dev(inp["v"], io), [dev(x, io) for x in inp["x"]],
+                                                          dev(inp["b"]), H)
+    torch.cuda.synchronize()
+    ref = oracle.hyena_forward_circular_per_sample(inp["v"], np.stack(inp["x"]), h, inp["b"])
+    assert_close(host(y), ref, io, f"circular per-sample B{B} D{D} L{L} N{N} {io}")
+
+
+def test_forward_circular_per_sample_with_equal_sets_is_the_shared_forward(hy):
+    B, D, L, N = 3, 5, 4096, 2
+    wl, inp = random_problem(B, D, L, N, seed=17)
+    H = hy.hyena_filter_rfft_circular(dev(filters(N, D, L, seed=18)))
+    v, xs, b = dev(inp["v"]), [dev(x) for x in inp["x"]], dev(inp["b"])
+    y1 = hy.hyena_fftconv_gate_forward_circular(v, xs, b, H)
+    y2 = hy.hyena_fftconv_gate_forward_circular_per_sample(v, xs, b, H.unsqueeze(0).expand(B, -1, -1, -1)
+                                                           .contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)

@@ -235,3 +235,31 @@ def test_forward_3d_circular_on_padded_volumes_is_the_linear_forward(hy):
     outside = yc.copy()
     outside[..., :Z, :H, :W] = 0.0
     assert np.max(np.abs(outside)) == 0.0
+
+
+# ------------------------------------- per-sample spectra (input-dependent)
+
+@pytest.mark.parametrize("B,C,H,W,N,io", [(2, 3, 32, 64, 2, "f32"), (3, 2, 16, 128, 1, "bf16")])
+def test_forward_2d_circular_per_sample_matches_oracle(hy, B, C, H, W, N, io):
+    v, x, b, _ = problem(B, C, (H, W), N, seed=300 + H)
+    rng = np.random.default_rng(301 + W)
+    h = np.stack([decaying(rng, (N, C, H, W)) for _ in range(B)])                # [B][N][C][H][W]
+    Hs = hy.hyena_filter_rfft2d_circular(dev(h.reshape(B * N, C, H, W))).reshape(B, N, C, H, W // 2)
+    y = host(hy.hyena_fftconv2d_gate_forward_circular_per_sample(dev(v, io), [dev(xx, io) for xx in x], dev(b),
+                                                                 Hs))
+    ref = oracle.hyena_forward_circular_nd_per_sample(as_io(v, io), np.stack([as_io(xx, io) for xx in x]),
+                                                      h.astype(np.float64), b.astype(np.float64))
+    assert_close(y, ref, io, f"circular 2-D per-sample B{B} C{C} {H}x{W} N{N} {io}")
+
+
+@pytest.mark.parametrize("B,C,Z,H,W,N,io", [(2, 2, 16, 16, 32, 2, "f32"), (2, 1, 16, 32, 64, 1, "bf16")])
+def test_forward_3d_circular_per_sample_matches_oracle(hy, B, C, Z, H, W, N, io):
+    v, x, b, _ = problem(B, C, (Z, H, W), N, seed=400 + Z + W)
+    rng = np.random.default_rng(401 + H)
+    h = np.stack([decaying(rng, (N, C, Z, H, W)) for _ in range(B)])             # [B][N][C][Z][H][W]
+    Hs = hy.hyena_filter_rfft3d_circular(dev(h.reshape(B * N, C, Z, H, W))).reshape(B, N, C, Z, H, W // 2)
+    y = host(hy.hyena_fftconv3d_gate_forward_circular_per_sample(dev(v, io), [dev(xx, io) for xx in x], dev(b),
+                                                                 Hs))
+    ref = oracle.hyena_forward_circular_nd_per_sample(as_io(v, io), np.stack([as_io(xx, io) for xx in x]),
+                                                      h.astype(np.float64), b.astype(np.float64))
+    assert_close(y, ref, io, f"circular 3-D per-sample B{B} C{C} {Z}x{H}x{W} N{N} {io}")
