@@ -66,11 +66,16 @@ def _describe(wl: synth.Workload) -> dict:
                 "filters": filters,
                 "l2": "flushed (256 MB write) before every timed step"}
     if wl.kind == "2d":
+        filters = (f"implicit FFN over (y/H, x/W) (3 sine layers of width {synth.WIDTH}, "
+                   f"{synth.N_BANDS} bands per axis) x separable decay, regenerated every step")
+        if wl.film:
+            filters = (f"input-dependent: a filter set per sample, the {synth.WIDTH}-wide sine layers over "
+                       f"(y/H, x/W) ({synth.N_BANDS} bands per axis) FiLM-modulated per sample, first layer at "
+                       "frequencies 1/2/4/8, Gaussian window; B*N*C filters and spectra regenerated every step")
         return {"workload": f"{wl.name}: order-{wl.N} Hyena 2-D operator, B={wl.B}, C={wl.D}, "
                             f"{wl.H}x{wl.W} grid (padded to {2 * wl.H}x{2 * wl.W}), {wl.io} storage, fp32 compute",
                 "N": wl.N, "B": wl.B, "C": wl.D, "H": wl.H, "W": wl.W, "io": wl.io,
-                "filters": f"implicit FFN over (y/H, x/W) (3 sine layers of width {synth.WIDTH}, "
-                           f"{synth.N_BANDS} bands per axis) x separable decay, regenerated every step",
+                "filters": filters,
                 "l2": "flushed (256 MB write) before every timed step"}
     filters = (f"implicit FFN (3 sine layers of width {synth.WIDTH}, {synth.N_BANDS} bands) "
                "x exponential decay, regenerated every step")
@@ -105,6 +110,8 @@ def alg_bytes_backward(wl: synth.Workload) -> int:
     dbias out (float32)."""
     io = 2 if wl.io == "bf16" else 4
     act = wl.positions * io
+    if wl.film and wl.kind == "2d":   # 2H x W spectrum slots and H x W of dh, per sample
+        return (2 * wl.N + 3) * act + wl.B * wl.N * wl.D * wl.H * wl.W * (16 + 4) + wl.N * wl.D * 4
     if wl.film:             # spectra in and dh out per sample
         return (2 * wl.N + 3) * act + wl.B * wl.N * wl.D * wl.L * (8 + 4) + wl.N * wl.D * 4
     if wl.circular:         # half a spectrum slot and one dh value per position
@@ -420,6 +427,23 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
                                       width=synth.WIDTH, decay_div=synth.DECAY_DIV, out=h)
             hyena.hyena_filter_rfft3d(h, out=H)
             forward()
+    elif wl.kind == "2d" and wl.film:
+        F = [to_dev(inp[k]) for k in ("omega", "gamma", "beta", "sigma")]
+        h = torch.empty((wl.B, wl.N, wl.D, wl.H, wl.W), device="cuda", dtype=torch.float32)
+        H = torch.empty((wl.B, wl.N, wl.D, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
+        ws_n = hyena.hyena_fftconv2d_workspace_size(wl.B, wl.D, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
+        ws_fwd = torch.empty(ws_n, device="cuda", dtype=torch.uint8)
+
+        def forward():
+            hyena.hyena_fftconv2d_gate_forward_per_sample(v, xs, b, H, out=y, workspace=ws_fwd)
+
+        def step():
+            hyena.hyena_filter_gen_film_2d(*W, wl.N, wl.D, wl.H, wl.W, B=wl.B, omega=F[0], gamma=F[1], beta=F[2],
+                                           sigma=F[3], n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                           decay_div=synth.DECAY_DIV, out=h)
+            hyena.hyena_filter_rfft2d(h.view(wl.B * wl.N, wl.D, wl.H, wl.W),
+                                      out=H.view(wl.B * wl.N, wl.D, 2 * wl.H, wl.W))
+            forward()
     elif wl.kind == "2d":
         h = torch.empty((wl.N, wl.D, wl.H, wl.W), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.N, wl.D, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
@@ -551,9 +575,18 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
 
     # ---- the backward pass (1-D and 2-D): one call per timed repetition
     bwd = None
-    if (wl.kind == "1d" and not (wl.circular and long_path(wl))) or (wl.kind == "2d" and not wl.film):
+    if (wl.kind == "1d" and not (wl.circular and long_path(wl))) or wl.kind == "2d":
         dy = to_dev(synth.make_output_grad(wl), io)
-        if wl.circular and wl.kind == "2d":
+        if wl.film and wl.kind == "2d":
+            ws_b = torch.empty(hyena.hyena_fftconv2d_backward_per_sample_workspace_size(wl.B, wl.D, wl.H, wl.W,
+                                                                                        wl.N),
+                               device="cuda", dtype=torch.uint8)
+            bwd_kernel = ("fft2d_bwd_row_kernel+fft2d_bwd_col_kernel (hyena_fftconv2d_gate_backward_per_sample, "
+                          "all launches)")
+
+            def backward():
+                hyena.hyena_fftconv2d_gate_backward_per_sample(v, xs, b, H, dy, workspace=ws_b)
+        elif wl.circular and wl.kind == "2d":
             ws_b = torch.empty(hyena.hyena_fftconv2d_backward_circular_workspace_size(wl.B, wl.D, wl.H, wl.W,
                                                                                       wl.N),
                                device="cuda", dtype=torch.uint8)
@@ -679,6 +712,13 @@ def oracle_sample(wl: synth.Workload, inp: dict, channels: np.ndarray, threads: 
                               wl.N, len(channels), wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
                               decay_div=synth.DECAY_DIV, threads=threads)
         oracle.hyena_forward_circular(v, x, h, bias, route="fft", threads=threads)
+        return time.perf_counter() - t0
+    if wl.kind == "2d" and wl.film:
+        h = oracle.filter_gen_film_2d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["omega"],
+                                      inp["gamma"], inp["beta"], inp["sigma"][channels], True, wl.N,
+                                      len(channels), wl.H, wl.W, n_bands=synth.N_BANDS, width=synth.WIDTH,
+                                      decay_div=synth.DECAY_DIV, threads=threads)
+        oracle.hyena_forward_2d_per_sample(v, x, h, bias, route="fft", threads=threads)
         return time.perf_counter() - t0
     if wl.kind == "2d":
         h = oracle.filter_gen_2d(inp["W1"], inp["W2"], inp["W3"], inp["Wout"][rows], inp["alpha"][channels],

@@ -95,6 +95,8 @@ WORKLOADS = {
     # c1 with input-dependent filters: a filter set per sample (FiLM-modulated
     # sine layers, multi-frequency first layer, Gaussian window)
     "c1_film": Workload("c1_film", "1d", N=2, B=8, D=768, L=2048, io="bf16", seed=_seed(1), film=True),
+    # c4 with input-dependent (per-sample, FiLM-modulated) 2-D filters
+    "c4_film": Workload("c4_film", "2d", N=2, B=2, D=128, H=256, W=256, io="f32", seed=_seed(4), film=True),
     # order-2 3-D operator on 64^3 volumes, B=2, C=32, bf16 storage
     "c5_3d": Workload("c5_3d", "3d", N=2, B=2, D=32, Z=64, H=64, W=64, io="bf16", seed=_seed(5)),
     # c5_3d with input-dependent (per-sample, FiLM-modulated) 3-D filters
