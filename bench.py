@@ -575,7 +575,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
 
     # ---- the backward pass (1-D and 2-D): one call per timed repetition
     bwd = None
-    if (wl.kind == "1d" and not (wl.circular and long_path(wl))) or wl.kind == "2d":
+    if wl.kind in ("1d", "2d"):
         dy = to_dev(synth.make_output_grad(wl), io)
         if wl.film and wl.kind == "2d":
             ws_b = torch.empty(hyena.hyena_fftconv2d_backward_per_sample_workspace_size(wl.B, wl.D, wl.H, wl.W,
@@ -598,7 +598,9 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
         elif wl.circular:
             ws_b = torch.empty(hyena.hyena_fftconv_backward_circular_workspace_size(wl.D, wl.L, wl.N),
                                device="cuda", dtype=torch.uint8)
-            bwd_kernel = "backward1d_kernel<PAD=false> (hyena_fftconv_gate_backward_circular)"
+            bwd_kernel = ("fourstep_bwd_row_kernel+fourstep_bwd_col_kernel<PAD=false> "
+                          "(hyena_fftconv_gate_backward_circular, all launches)" if long_path(wl) else
+                          "backward1d_kernel<PAD=false> (hyena_fftconv_gate_backward_circular)")
 
             def backward():
                 hyena.hyena_fftconv_gate_backward_circular(v, xs, b, H, dy, workspace=ws_b)

@@ -247,9 +247,10 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_circular_per_sample(const vo
  * Arguments as hyena_fftconv_gate_backward with H [N][D][L/2] from
  * hyena_filter_rfft_circular; dh [N][D][L] and dbias [N][D] summed over the
  * batch; workspace of hyena_fftconv_backward_circular_workspace_size(D, L,
- * N) bytes (12 N D L), 256-byte aligned.  32 <= L <= 16384, a power of two
- * (the size function returns (size_t)-1 otherwise).  Two launches,
- * deterministic, as the L <= 16384 backward. */
+ * N) bytes (12 N D L up to L = 16384; above, the four-step backward's),
+ * 256-byte aligned.  32 <= L <= HYENA_MAX_LEN, a power of two (the size
+ * function returns (size_t)-1 otherwise).  Deterministic: two launches up
+ * to L = 16384, the four-step launch sequence above. */
 HYENA_API size_t hyena_fftconv_backward_circular_workspace_size(int D, int L, int N);
 HYENA_API hyena_status_t hyena_fftconv_gate_backward_circular(const void* v, const void* const* x,
                                                               const float* H, const float* bias,

@@ -241,13 +241,14 @@ fourstep_bwd_row_kernel(FourStepBwdArgs ba)
     }
 }
 
-// Column kernel of the backward.  Each CTA: TC columns n2 of one sequence
+// Column kernel of the backward (PAD false: circular mode, every n1 is data
+// and nothing is cropped).  Each CTA: TC columns n2 of one sequence
 // (one filter row in MODE 3).  MODE 0 (A): inverse columns, crop: c_n,
 // saved; unless last, gate with x_n and forward columns + twiddle.  MODE 1
 // (B): g = dy (first) or the inverse columns of the scratch; dx_n = g c_n;
 // e = g x_n; forward columns + twiddle.  MODE 2: dv = the inverse columns.
 // MODE 3: dh = the inverse columns of the finalize scratch, db = dh[0].
-template <int LOG2M1, int LOG2M2, typename IO, int MODE>
+template <int LOG2M1, int LOG2M2, typename IO, int MODE, bool PAD = true>
 __global__ void __launch_bounds__(FourStep<LOG2M1, LOG2M2>::COL_THREADS)
 fourstep_bwd_col_kernel(FourStepBwdArgs ba)
 {
@@ -257,6 +258,8 @@ fourstep_bwd_col_kernel(FourStepBwdArgs ba)
     using IOP = IoPair<IO>;
     using PT = typename IOP::T;
     constexpr int M1 = FS::M1, M2 = FS::M2, M = FS::M, TC = FS::TC, V1 = FS::F1::V;
+    constexpr int VL = PAD ? V1 / 2 : V1;                   // registers holding data (circular: all n1)
+    constexpr int SEQ = PAD ? M / 2 : M;                     // value pairs per sequence
     extern __shared__ __align__(16) float2 smem_fc[];
 
     const int qi = blockIdx.x / FS::COL_CTAS_PER_SEQ;
@@ -289,67 +292,67 @@ fourstep_bwd_col_kernel(FourStepBwdArgs ba)
     if constexpr (MODE == 3) {
         // q: filter row n*D + d; dh row of L floats = M/2 value pairs
         inverse_cols();
-        float2* dhp = reinterpret_cast<float2*>(ba.dh) + (size_t)q * (M / 2);
-        static_for<V1 / 2>([&](auto rr) {
+        float2* dhp = reinterpret_cast<float2*>(ba.dh) + (size_t)q * SEQ;
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             dhp[at(r)] = reg[r];
         });
         if (n2 == 0 && t == 0 && a.H_bstride == 0) ba.dbias[q] = reg[0].x;   // db_n = dh_n[0]
         return;
     } else {
-        const size_t cso = ((size_t)a.n * ba.wcap + qi) * (M / 2);
+        const size_t cso = ((size_t)a.n * ba.wcap + qi) * SEQ;
         float2* cs = ba.csave + cso;
-        const PT* xp = reinterpret_cast<const PT*>(pick_fs(a.x, a.n)) + seq * (M / 2);
+        const PT* xp = reinterpret_cast<const PT*>(pick_fs(a.x, a.n)) + seq * SEQ;
         if constexpr (MODE == 0) {
             inverse_cols();                                     // c_n
-            static_for<V1 / 2>([&](auto rr) {
+            static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
                 cs[at(r)] = reg[r];
             });
             if (ba.last) return;
-            static_for<V1 / 2>([&](auto rr) {
+            static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
                 const float2 xv = IOP::load(xp + at(r));
                 reg[r] = make_float2(reg[r].x * xv.x, reg[r].y * xv.y);
             });
         } else if constexpr (MODE == 1) {
             if (ba.first) {
-                const PT* gp = reinterpret_cast<const PT*>(ba.dy) + seq * (M / 2);
-                static_for<V1 / 2>([&](auto rr) {
+                const PT* gp = reinterpret_cast<const PT*>(ba.dy) + seq * SEQ;
+                static_for<VL>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
                     reg[r] = IOP::load(gp + at(r));
                 });
             } else {
                 inverse_cols();                                 // g = dL/dz_{n+1}
             }
-            PT* dxp = reinterpret_cast<PT*>(pick_fs(ba.dx, a.n)) + seq * (M / 2);
-            float2 cv[V1 / 2], xv[V1 / 2];
-            static_for<V1 / 2>([&](auto rr) {
+            PT* dxp = reinterpret_cast<PT*>(pick_fs(ba.dx, a.n)) + seq * SEQ;
+            float2 cv[VL], xv[VL];
+            static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
                 cv[r] = cs[at(r)];
                 xv[r] = IOP::load(xp + at(r));
             });
-            static_for<V1 / 2>([&](auto rr) {
+            static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
                 IOP::store(dxp + at(r), make_float2(reg[r].x * cv[r].x, reg[r].y * cv[r].y));
                 reg[r] = make_float2(reg[r].x * xv[r].x, reg[r].y * xv[r].y);     // e
             });
         } else {
             inverse_cols();                                     // dv = dL/dz_0
-            PT* dvp = reinterpret_cast<PT*>(ba.dv) + seq * (M / 2);
-            static_for<V1 / 2>([&](auto rr) {
+            PT* dvp = reinterpret_cast<PT*>(ba.dv) + seq * SEQ;
+            static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
                 IOP::store(dvp + at(r), reg[r]);
             });
             return;
         }
-        // forward columns (n1 < M1/2, zero-padded) + twiddle exp(-2 pi i n2 k1 / M)
-        static_for<V1 / 2>([&](auto rr) {
+        // forward columns (n1 < M1/2, zero-padded; circular: all n1) + twiddle exp(-2 pi i n2 k1 / M)
+        static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
             buf[pad16_at<M1 / V1>(t, pt, r)] = reg[r];
         });
         __syncthreads();
-        FS::F1::template run<-1, true, true>(buf, reg, t);
+        FS::F1::template run<-1, true, PAD>(buf, reg, t);
         float2 w = expi_pi<-1>(2.0f * (float)((n2 * t) % M) / (float)M);
         const float2 step = expi_pi<-1>(2.0f * (float)((n2 * (M1 / V1)) % M) / (float)M);
         static_for<V1>([&](auto rr) {

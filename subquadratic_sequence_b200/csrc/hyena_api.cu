@@ -539,8 +539,8 @@ hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, 
 size_t hyena_fftconv_backward_circular_workspace_size(int D, int L, int N)
 {
     const int k = exact_log2(L);
-    if (D < 1 || N < 1 || N > HYENA_MAX_ORDER || k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1)
-        return (size_t)-1;
+    if (D < 1 || N < 1 || N > HYENA_MAX_ORDER || k < kMinLog2Circ + 1 || k > kMaxLog2) return (size_t)-1;
+    if (k - 1 > kMaxLog2Circ) return fourstep_bwd_layout(k - 1, D, N, 1, true).total;   // four-step
     return 3 * round_up(sizeof(float2) * (size_t)N * D * (L / 2), 256);   // acc, wz, wc
 }
 
@@ -582,7 +582,7 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
     int log2m = 0;
     if (circular) {
         const int k = exact_log2(L);
-        if (k < kMinLog2Circ + 1 || k > kMaxLog2Circ + 1) return HYENA_ERR_UNSUPPORTED;
+        if (per_sample || k < kMinLog2Circ + 1 || k > kMaxLog2) return HYENA_ERR_UNSUPPORTED;
         log2m = k - 1;                       // M = L/2 packed points
     } else {
         hyena_status_t s = check_len(L, kMaxLog2, &log2m);
@@ -625,9 +625,9 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
     const size_t spec = sizeof(float2) * (size_t)N * D * (circular ? L / 2 : L);   // one spectrum set
     char* ws = static_cast<char*>(workspace);
     cudaStream_t st = (cudaStream_t)stream;
-    if (!circular && log2m > kMaxLog2Fused) {
+    if (circular ? log2m > kMaxLog2Circ : log2m > kMaxLog2Fused) {
         // four-step backward (L > 16384)
-        const FourStepBwdLayout lay = fourstep_bwd_layout(log2m, D, N, (int)sets);
+        const FourStepBwdLayout lay = fourstep_bwd_layout(log2m, D, N, (int)sets, circular);
         FourStepBwdArgs b = {};
         b.f.v = v;
         for (int n = 0; n < kMaxOrder; ++n) {
@@ -648,6 +648,9 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
         b.dh = dh;
         b.dbias = dbias;
         b.wcap = (int)lay.wcap;
+        if (circular)
+            return io == HYENA_BF16 ? dispatch_fourstep_bwd_circ_bf16(log2m, b, N, st)
+                                    : dispatch_fourstep_bwd_circ_f32(log2m, b, N, st);
         return io == HYENA_BF16 ? dispatch_fourstep_bwd_bf16(log2m, b, N, st)
                                 : dispatch_fourstep_bwd_f32(log2m, b, N, st);
     }

@@ -379,7 +379,7 @@ def hyena_fftconv_backward_circular_workspace_size(D: int, L: int, N: int) -> in
     n = LIB.hyena_fftconv_backward_circular_workspace_size(D, L, N)
     if n == ctypes.c_size_t(-1).value:
         raise HyenaError("hyena_fftconv_backward_circular_workspace_size", HYENA_ERR_UNSUPPORTED,
-                         "invalid sizes (32 <= L <= 16384)")
+                         "invalid sizes (32 <= L <= 2^22)")
     return n
 
 

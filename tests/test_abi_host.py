@@ -357,14 +357,16 @@ def test_backward_variants_reject_bad_arguments(lib):
     # circular: 32 <= L <= 16384
     cs = lib.hyena_fftconv_backward_circular_workspace_size
     assert cs(3, 64, 2) >= 12 * 2 * 3 * 64
-    assert cs(3, 16, 2) == bad and cs(3, 1 << 15, 2) == bad and cs(3, 96, 2) == bad
+    assert cs(3, 16, 2) == bad and cs(3, 1 << 23, 2) == bad and cs(3, 96, 2) == bad
+    assert cs(3, 1 << 15, 2) > (64 << 20)                    # the four-step layout above 16384
     xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
     dxs = (ctypes.c_void_p * 2)(P(7).value, P(8).value)
     f = lib.hyena_fftconv_gate_backward_circular
     args = lambda **k: [k.get("v", P(0)), xs, P(3), P(4), P(5), 2, 3, k.get("L", 64), 2, F32, k.get("dv", P(6)),
                         dxs, k.get("dh", P(9)), P(10), k.get("ws", P(11)), k.get("nb", 1 << 24), None]
     assert f(*args(L=16)) == UNSUPPORTED
-    assert f(*args(L=1 << 15)) == UNSUPPORTED
+    assert f(*args(L=1 << 23)) == UNSUPPORTED
+    assert f(*args(L=1 << 15)) == WORKSPACE                                      # four-step: more workspace
     assert f(*args(v=None)) == INVALID
     assert f(*args(ws=None)) == WORKSPACE
     assert f(*args(dv=P(0))) == INVALID                                          # dv aliases v

@@ -113,9 +113,27 @@ def test_backward_circular_shift_filter_closed_form(hy):
     assert rel_max_err(host(db)[0], ref_dh[:, 0]) <= 1e-4
 
 
+@pytest.mark.parametrize("B,D,L,N,io", [(2, 2, 32768, 2, "f32"), (1, 3, 65536, 1, "bf16"),
+                                        (3, 11, 262144, 1, "f32")])   # channel 10 across two waves
+def test_backward_circular_long_matches_oracle(hy, B, D, L, N, io):
+    wl, inp = random_problem(B, D, L, N, seed=1200 + N, io=io)
+    h = filters(N, D, L, seed=L + 19)
+    dy = np.random.default_rng(L + 1).standard_normal((B, D, L)).astype(np.float32)
+    if io == "bf16":
+        from subquadratic_sequence_b200 import synth
+        dy = synth.bf16_round(dy)
+    H = hy.hyena_filter_rfft_circular(dev(h))
+    dv, dxs, dh, db = hy.hyena_fftconv_gate_backward_circular(
+        dev(inp["v"], io), [dev(x, io) for x in inp["x"]], dev(inp["b"]), H, dev(dy, io))
+    torch.cuda.synchronize()
+    got = host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+    ref = oracle.hyena_backward_circular(inp["v"], np.stack(inp["x"]), h, inp["b"], dy)
+    check_backward(got, ref, io, f"circular backward B{B} D{D} L{L} N{N} {io}")
+
+
 def test_backward_circular_rejects_unsupported_lengths(hy):
     from subquadratic_sequence_b200.hyena import HyenaError
-    for L in (16, 32768):
+    for L in (16, 1 << 23):
         with pytest.raises(HyenaError):
             hy.hyena_fftconv_backward_circular_workspace_size(4, L, 2)
 
