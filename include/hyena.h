@@ -259,6 +259,20 @@ HYENA_API hyena_status_t hyena_fftconv_gate_backward_circular(const void* v, con
                                                               float* dh, float* dbias, void* workspace,
                                                               size_t ws_bytes, void* stream);
 
+/* The circular backward with a spectrum set per sample: H [B][N][D][L/2]
+ * (sample b's set at H + b*N*D*L/2), dh [B][N][D][L] per sample, dbias
+ * [N][D] summed over the batch; workspace of
+ * hyena_fftconv_backward_circular_per_sample_workspace_size(B, D, L, N)
+ * bytes.  Everything else as hyena_fftconv_gate_backward_circular. */
+HYENA_API size_t hyena_fftconv_backward_circular_per_sample_workspace_size(int B, int D, int L, int N);
+HYENA_API hyena_status_t hyena_fftconv_gate_backward_circular_per_sample(const void* v, const void* const* x,
+                                                                         const float* H, const float* bias,
+                                                                         const void* dy, int B, int D, int L,
+                                                                         int N, hyena_dtype_t io, void* dv,
+                                                                         void* const* dx, float* dh,
+                                                                         float* dbias, void* workspace,
+                                                                         size_t ws_bytes, void* stream);
+
 /* Size of the scratch array built into the library for
  * hyena_fftconv_gate_forward_noalloc (16 MB on every device that loads the
  * library, held until the process exits). */

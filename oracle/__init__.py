@@ -516,3 +516,14 @@ def hyena_forward_circular_nd_per_sample(v, x, h, bias, route="fft") -> np.ndarr
     v, x, h, bias = map(_f64, (v, x, h, bias))
     return np.concatenate([hyena_forward_circular_nd(v[b:b + 1], x[:, b:b + 1], h[b], bias, route)
                            for b in range(v.shape[0])])
+
+
+def hyena_backward_circular_per_sample(v, x, h, bias, dy, route="fft", threads=None):
+    """The gradients through :func:`hyena_forward_circular_per_sample` (a
+    filter set per sample, h [B][N][D][L]): each sample's circular adjoint
+    with its own filters; dh per sample, dbias summed over the samples."""
+    v, x, h, bias, dy = map(_f64, (v, x, h, bias, dy))
+    parts = [hyena_backward_circular(v[b:b + 1], x[:, b:b + 1], h[b], bias, dy[b:b + 1], route, threads)
+             for b in range(v.shape[0])]
+    return (np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts], axis=1),
+            np.stack([p[2] for p in parts]), np.sum([p[3] for p in parts], axis=0))

@@ -554,6 +554,25 @@ hyena_status_t hyena_fftconv_gate_backward_circular(const void* v, const void* c
                          ws_bytes, stream);
 }
 
+size_t hyena_fftconv_backward_circular_per_sample_workspace_size(int B, int D, int L, int N)
+{
+    const int k = exact_log2(L);
+    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || k < kMinLog2Circ + 1 || k > kMaxLog2) return (size_t)-1;
+    if (k - 1 > kMaxLog2Circ) return fourstep_bwd_layout(k - 1, D, N, B, true).total;   // four-step
+    const size_t spec = sizeof(float2) * (size_t)N * D * (L / 2);
+    return round_up(spec * B, 256) + 2 * round_up(spec, 256);   // acc (per sample), wz, wc
+}
+
+hyena_status_t hyena_fftconv_gate_backward_circular_per_sample(const void* v, const void* const* x,
+                                                               const float* H, const float* bias, const void* dy,
+                                                               int B, int D, int L, int N, hyena_dtype_t io,
+                                                               void* dv, void* const* dx, float* dh, float* dbias,
+                                                               void* workspace, size_t ws_bytes, void* stream)
+{
+    return backward_impl(v, x, H, true, true, bias, dy, B, D, L, N, io, dv, dx, dh, dbias, workspace,
+                         ws_bytes, stream);
+}
+
 hyena_status_t hyena_fftconv_gate_backward_per_sample(const void* v, const void* const* x, const float* H,
                                                       const float* bias, const void* dy, int B, int D, int L,
                                                       int N, hyena_dtype_t io, void* dv, void* const* dx,
@@ -582,7 +601,7 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
     int log2m = 0;
     if (circular) {
         const int k = exact_log2(L);
-        if (per_sample || k < kMinLog2Circ + 1 || k > kMaxLog2) return HYENA_ERR_UNSUPPORTED;
+        if (k < kMinLog2Circ + 1 || k > kMaxLog2) return HYENA_ERR_UNSUPPORTED;
         log2m = k - 1;                       // M = L/2 packed points
     } else {
         hyena_status_t s = check_len(L, kMaxLog2, &log2m);
@@ -594,7 +613,8 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
     if (!aligned(v, 16) || !aligned(dy, 16) || !aligned(dv, 16) || !aligned(H, 16) || !aligned(dh, 16) ||
         !aligned(bias, 4) || !aligned(dbias, 4))
         return HYENA_ERR_INVALID_ARG;
-    const size_t need = circular ? hyena_fftconv_backward_circular_workspace_size(D, L, N)
+    const size_t need = circular ? (per_sample ? hyena_fftconv_backward_circular_per_sample_workspace_size(B, D, L, N)
+                                               : hyena_fftconv_backward_circular_workspace_size(D, L, N))
                         : per_sample ? hyena_fftconv_backward_per_sample_workspace_size(B, D, L, N)
                                      : hyena_fftconv_backward_workspace_size(D, L, N);
     if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
@@ -635,7 +655,7 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
             b.dx[n] = n < N ? dx[n] : nullptr;
         }
         b.f.H = reinterpret_cast<const float2*>(H);
-        b.f.H_bstride = per_sample ? (size_t)N * D * L : 0;
+        b.f.H_bstride = per_sample ? (size_t)N * D * (circular ? L / 2 : L) : 0;
         b.f.bias = bias;
         b.f.S = reinterpret_cast<float2*>(ws + lay.scratch);
         b.f.B = B;
@@ -672,7 +692,10 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
     a.B = B;
     a.D = D;
     a.N = N;
-    a.H_bstride = per_sample ? (size_t)N * D * L : 0;
+    a.H_bstride = per_sample ? (size_t)N * D * (circular ? L / 2 : L) : 0;
+    if (circular && per_sample)
+        return io == HYENA_BF16 ? dispatch_backward_circ_ps_bf16(log2m, a, st)
+                                : dispatch_backward_circ_ps_f32(log2m, a, st);
     if (circular)
         return io == HYENA_BF16 ? dispatch_backward_circ_bf16(log2m, a, st)
                                 : dispatch_backward_circ_f32(log2m, a, st);

@@ -93,7 +93,8 @@ hyena_status_t run_fourstep_bwd(FourStepBwdArgs a, int N, cudaStream_t st)
     }
     if (f.H_bstride != 0) {          // per-sample: db from the B lag-0 values (any B)
         const int nd = N * f.D;
-        return launch(dbias_sum_kernel<FS::M>, (unsigned)((nd + 255) / 256), 256, 0, st, a);   // rows of L = M
+        // dh rows of L floats: L = M (padded), 2M (circular)
+        return launch(dbias_sum_kernel<PAD ? FS::M : 2 * FS::M>, (unsigned)((nd + 255) / 256), 256, 0, st, a);
     }
     return HYENA_OK;
 }

@@ -90,5 +90,7 @@ hyena_status_t dispatch_backward_ps_f32(int log2m, const Backward1dArgs& a, cuda
 hyena_status_t dispatch_backward_ps_bf16(int log2m, const Backward1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_backward_circ_f32(int log2m, const Backward1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_backward_circ_bf16(int log2m, const Backward1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_backward_circ_ps_f32(int log2m, const Backward1dArgs& a, cudaStream_t st);
+hyena_status_t dispatch_backward_circ_ps_bf16(int log2m, const Backward1dArgs& a, cudaStream_t st);
 
 }  // namespace hyena

@@ -67,6 +67,9 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv_backward_workspace_size": ([i, i, i], sz),
         "hyena_fftconv_backward_per_sample_workspace_size": ([i, i, i, i], sz),
         "hyena_fftconv_backward_circular_workspace_size": ([i, i, i], sz),
+        "hyena_fftconv_backward_circular_per_sample_workspace_size": ([i, i, i, i], sz),
+        "hyena_fftconv_gate_backward_circular_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i,
+                                                             vp, ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_fftconv_gate_backward_circular": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp,
                                                   ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
         "hyena_fftconv_gate_backward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, vp,
@@ -401,6 +404,35 @@ def hyena_fftconv_gate_backward_circular(v: torch.Tensor, xs, bias: torch.Tensor
         workspace = torch.empty(hyena_fftconv_backward_circular_workspace_size(D, L, N), device=v.device,
                                 dtype=torch.uint8)
     _check("hyena_fftconv_gate_backward_circular", LIB.hyena_fftconv_gate_backward_circular(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+        B, D, L, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+        ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db
+
+
+def hyena_fftconv_gate_backward_circular_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor,
+                                                    dy: torch.Tensor, *, workspace=None, stream=None):
+    """The circular backward with per-sample spectra H [B][N][D][L/2]:
+    returns (dv, [dx_1..dx_N], dh [B][N][D][L] per sample, dbias [N][D]
+    summed over the batch)."""
+    B, D, L = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty((B, N, D, L), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, D), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        n = LIB.hyena_fftconv_backward_circular_per_sample_workspace_size(B, D, L, N)
+        if n == ctypes.c_size_t(-1).value:
+            raise HyenaError("hyena_fftconv_backward_circular_per_sample_workspace_size", HYENA_ERR_UNSUPPORTED,
+                             "invalid sizes")
+        workspace = torch.empty(n, device=v.device, dtype=torch.uint8)
+    _check("hyena_fftconv_gate_backward_circular_per_sample", LIB.hyena_fftconv_gate_backward_circular_per_sample(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
         B, D, L, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),

@@ -407,3 +407,30 @@ def test_backward_3d_axis_permutation_permutes_every_gradient():
     for a, c in zip(g[:3], gp[:3]):
         assert rel_err(perm(c), a) < 1e-12
     assert rel_err(gp[3], g[3]) < 1e-12
+
+
+def test_backward_circular_per_sample_matches_finite_differences():
+    B, D, L, N = 2, 2, 8, 2
+    r = np.random.default_rng(80)
+    v, x = r.standard_normal((B, D, L)), r.standard_normal((N, B, D, L))
+    h = r.standard_normal((B, N, D, L)) * np.exp(-np.arange(L) / 4.0)
+    b, dy = r.standard_normal((N, D)), r.standard_normal((B, D, L))
+    dv, dx, dh, db = oracle.hyena_backward_circular_per_sample(v, x, h, b, dy, route="direct")
+
+    def loss(v_, x_, h_, b_):
+        y = np.concatenate([oracle.hyena_forward_circular(v_[s:s + 1], x_[:, s:s + 1], h_[s], b_, route="direct")
+                            for s in range(B)])
+        return float(np.sum(dy * y))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name

@@ -218,3 +218,21 @@ def test_forward_circular_per_sample_with_equal_sets_is_the_shared_forward(hy):
                                                            .contiguous())
     torch.cuda.synchronize()
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("B,D,L,N,io", [(3, 5, 2048, 2, "f32"), (2, 3, 512, 2, "bf16"), (2, 2, 65536, 2, "f32"),
+                                        (1, 2, 32768, 1, "f32")])
+def test_backward_circular_per_sample_matches_oracle(hy, B, D, L, N, io):
+    wl, inp = random_problem(B, D, L, N, seed=1300 + L, io=io)
+    h = np.stack([filters(N, D, L, seed=L + 21 + b) for b in range(B)])
+    dy = np.random.default_rng(L + 2).standard_normal((B, D, L)).astype(np.float32)
+    if io == "bf16":
+        from subquadratic_sequence_b200 import synth
+        dy = synth.bf16_round(dy)
+    H = hy.hyena_filter_rfft_circular(dev(h.reshape(B * N, D, L))).reshape(B, N, D, L // 2)
+    dv, dxs, dh, db = hy.hyena_fftconv_gate_backward_circular_per_sample(
+        dev(inp["v"], io), [dev(x, io) for x in inp["x"]], dev(inp["b"]), H, dev(dy, io))
+    torch.cuda.synchronize()
+    got = host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+    ref = oracle.hyena_backward_circular_per_sample(inp["v"], np.stack(inp["x"]), h, inp["b"], dy)
+    check_backward(got, ref, io, f"circular per-sample backward B{B} D{D} L{L} N{N} {io}")
