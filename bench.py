@@ -1,6 +1,6 @@
 """Benchmark of the Hyena FFT-conv + gate path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c1] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3_1m] [--impl reference]
 
 One step = one pass of the whole path over one batch of synthetic input:
 implicit filter generation (hyena_filter_gen), the filter spectra
@@ -12,6 +12,13 @@ every timed step, outside the timed events.  Under torchrun every rank runs
 the same workload on its own GPU (the channel-sequences are independent, so
 the ranks share no data: weak scaling) and rank 0 prints one JSON line with
 the max time over ranks.
+
+The default workload is the largest single-GPU configuration (order 2,
+B=1, D=256, L=2^20, fp32).  The same run times the forward alone on every
+configuration (``per_config``: c0, c1, c2 at 8k and 16k, c3 at 64k, 256k
+and 1M, the 2-D c4) with its fraction of the HBM roofline.  ``e2e`` runs
+the step end to end from pinned host memory (H2D of the inputs, the step,
+D2H of y), pipelined over two buffer sets on three streams.
 
 --impl reference times the float64 CPU oracle on the host cores on a
 bounded sample of the same workload (the reference arm).
@@ -326,31 +333,36 @@ def throughput(positions_per_rank: int, world: int, steps: int, total_ms: float)
     return positions_per_rank * world * steps / (total_ms / 1e3)
 
 
-def run_gpu(args, wl: synth.Workload) -> dict | None:
-    import torch
+class Buffers:
+    """One set of device inputs and output of a step."""
 
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py: no CUDA device (the path has no CPU fallback)")
+    def __init__(self, wl: synth.Workload, inp: dict):
+        import torch
+        io = torch.bfloat16 if wl.io == "bf16" else torch.float32
+
+        def to_dev(a, dtype=torch.float32):
+            return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda().to(dtype)
+
+        self.v = to_dev(inp["v"], io)
+        self.xs = [to_dev(x, io) for x in inp["x"]]
+        self.b = to_dev(inp["b"])
+        self.W = [to_dev(inp[k]) for k in WKEYS]
+        self.F = [to_dev(inp[k]) for k in FILM_KEYS] if wl.film else []
+        self.y = torch.empty_like(self.v)
+
+
+WKEYS = ("W1", "W2", "W3", "Wout", "alpha")
+FILM_KEYS = ("omega", "gamma", "beta", "sigma")
+
+
+def setup_step(wl: synth.Workload, bf: Buffers):
+    """The step (filter generation, spectra, forward) and the forward alone
+    of one workload on one buffer set, with the filters, spectra and
+    workspaces they use allocated once.  Returns (step, forward, H)."""
+    import torch
     from subquadratic_sequence_b200 import hyena
 
-    ranks = Ranks("nccl")
-    world, rank, local = ranks.world, ranks.rank, ranks.local
-    barrier, max_over_ranks = ranks.barrier, ranks.max
-
-    inp = synth.make_inputs(wl)
-    io = torch.bfloat16 if wl.io == "bf16" else torch.float32
-
-    def to_dev(a, dtype=torch.float32):
-        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda().to(dtype)
-
-    v = to_dev(inp["v"], io)
-    xs = [to_dev(x, io) for x in inp["x"]]
-    b = to_dev(inp["b"])
-    wkeys = ("W1", "W2", "W3", "Wout", "alpha")
-    W = [to_dev(inp[k]) for k in wkeys]
-    y = torch.empty_like(v)
-    flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
-    stream = torch.cuda.current_stream()
+    v, xs, b, W, F, y = bf.v, bf.xs, bf.b, bf.W, bf.F, bf.y
     if wl.circular and wl.kind == "3d":
         h = torch.empty((wl.N, wl.D, wl.Z, wl.H, wl.W), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.N, wl.D, wl.Z, wl.H, wl.W // 2), device="cuda", dtype=torch.complex64)
@@ -397,7 +409,6 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             hyena.hyena_filter_rfft_circular(h, out=H, workspace=ws_rfft)
             forward()
     elif wl.kind == "3d" and wl.film:
-        F = [to_dev(inp[k]) for k in ("omega", "gamma", "beta", "sigma")]
         h = torch.empty((wl.B, wl.N, wl.D, wl.Z, wl.H, wl.W), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.B, wl.N, wl.D, 2 * wl.Z, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
         ws_n = hyena.hyena_fftconv3d_workspace_size(wl.B, wl.D, wl.Z, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
@@ -428,7 +439,6 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             hyena.hyena_filter_rfft3d(h, out=H)
             forward()
     elif wl.kind == "2d" and wl.film:
-        F = [to_dev(inp[k]) for k in ("omega", "gamma", "beta", "sigma")]
         h = torch.empty((wl.B, wl.N, wl.D, wl.H, wl.W), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.B, wl.N, wl.D, 2 * wl.H, wl.W), device="cuda", dtype=torch.complex64)
         ws_n = hyena.hyena_fftconv2d_workspace_size(wl.B, wl.D, wl.H, wl.W, wl.N, hyena.io_dtype(v), True)
@@ -459,7 +469,6 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             hyena.hyena_filter_rfft2d(h, out=H)
             forward()
     elif wl.film:
-        F = [to_dev(inp[k]) for k in ("omega", "gamma", "beta", "sigma")]
         h = torch.empty((wl.B, wl.N, wl.D, wl.L), device="cuda", dtype=torch.float32)
         H = torch.empty((wl.B, wl.N, wl.D, wl.L), device="cuda", dtype=torch.complex64)
         ws_rfft_n = hyena.hyena_filter_rfft_workspace_size(wl.B * wl.N, wl.D, wl.L)
@@ -495,6 +504,138 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             hyena.hyena_filter_rfft(h, out=H, workspace=ws_rfft)
             forward()
 
+    return step, forward, H
+
+
+def run_e2e(args, wl: synth.Workload, inp: dict, bufs: "Buffers", step, max_over_ranks):
+    """Milliseconds of args.steps end-to-end steps (pipelined over two
+    buffer sets: H2D, compute and D2H on their own streams), and the H2D and
+    D2H bytes of one step."""
+    import torch
+    io = bufs.v.dtype
+    pin = lambda a, dt=torch.float32: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dt).pin_memory()
+    hin = [pin(inp["v"], io), *[pin(x, io) for x in inp["x"]], pin(inp["b"]),
+           *[pin(inp[k]) for k in WKEYS], *([pin(inp[k]) for k in FILM_KEYS] if wl.film else [])]
+    hout = [torch.empty(bufs.y.shape, dtype=io).pin_memory() for _ in range(2)]
+    sets = [(bufs, step)]
+    bufs2 = Buffers(wl, inp)
+    step2, _, _ = setup_step(wl, bufs2)
+    sets.append((bufs2, step2))
+    dins = [[s.v, *s.xs, s.b, *s.W, *s.F] for s, _ in sets]
+    h2d = sum(t.numel() * t.element_size() for t in hin)
+    d2h = hout[0].numel() * hout[0].element_size()
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+
+    def run(nsteps: int):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        free_in = [None, None]    # compute done with the set's inputs
+        free_out = [None, None]   # D2H done with the set's y
+        torch.cuda.synchronize()
+        start.record(s_cmp)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        last = None
+        for i in range(nsteps):
+            k = i % 2
+            bf, stp = sets[k]
+            with torch.cuda.stream(s_in):
+                if free_in[k] is not None:
+                    s_in.wait_event(free_in[k])
+                for dst, src in zip(dins[k], hin):
+                    dst.copy_(src, non_blocking=True)
+                landed = ev()
+                landed.record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(landed)
+                if free_out[k] is not None:
+                    s_cmp.wait_event(free_out[k])
+                stp()
+                done = ev()
+                done.record(s_cmp)
+                free_in[k] = done
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done)
+                hout[k].copy_(bf.y, non_blocking=True)
+                last = ev()
+                last.record(s_out)
+                free_out[k] = last
+        s_cmp.wait_event(last)
+        end.record(s_cmp)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
+    run(2)                                    # warm the second set and the streams
+    ms = max_over_ranks(run(args.steps))
+    del sets, bufs2, dins
+    return ms, h2d, d2h
+
+
+# the forward of every BASELINE configuration, timed in the same run as the
+# headline line (the parity configurations c0..c4 at their full sizes)
+PER_CONFIG = ("c0", "c1", "c2_8k", "c2_16k", "c3_64k", "c3_256k", "c3_1m", "c4")
+
+
+def per_config_forward(args, headline: synth.Workload, headline_ms: float, flush, gpu_id: str) -> dict:
+    """Forward ms per call (CUDA events on the launching stream, L2 flushed
+    before each call), algorithmic bytes and fraction of the HBM peak for
+    every configuration, with the clocks sampled over the whole loop."""
+    import torch
+    peak, _ = peaks()
+    stream = torch.cuda.current_stream()
+    out = {}
+    with ClockSampler(gpu_id) as clk:
+        for name in PER_CONFIG:
+            wl = synth.WORKLOADS[name]
+            if wl == headline:
+                ms = headline_ms
+            else:
+                bufs = Buffers(wl, synth.make_inputs(wl))
+                step, forward, _ = setup_step(wl, bufs)
+                for _ in range(3):
+                    step()
+                reps = 10 if wl.positions >= (1 << 26) else 20
+                evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(reps)]
+                for a, b in evs:
+                    flush.zero_()
+                    a.record(stream)
+                    forward()
+                    b.record(stream)
+                torch.cuda.synchronize()
+                ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+                del bufs, step, forward
+                torch.cuda.empty_cache()
+            nbytes = alg_bytes_forward(wl)
+            out[name] = {"kernel": forward_kernel(wl), "ms_per_launch": ms, "alg_bytes_per_launch": nbytes,
+                         "achieved_gbs": nbytes / (ms / 1e3) / 1e9, "frac": nbytes / (ms / 1e3) / 1e9 / peak,
+                         "value": wl.positions / (ms / 1e3), "unit": UNIT}
+    out["clocks"] = clk.summary()
+    return out
+
+
+def run_gpu(args, wl: synth.Workload) -> dict | None:
+    import torch
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the path has no CPU fallback)")
+    from subquadratic_sequence_b200 import hyena
+
+    ranks = Ranks("nccl")
+    world, rank, local = ranks.world, ranks.rank, ranks.local
+    barrier, max_over_ranks = ranks.barrier, ranks.max
+
+    inp = synth.make_inputs(wl)
+    io = torch.bfloat16 if wl.io == "bf16" else torch.float32
+
+    def to_dev(a, dtype=torch.float32):
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda().to(dtype)
+
+    bufs = Buffers(wl, inp)
+    v, xs, b, y = bufs.v, bufs.xs, bufs.b, bufs.y
+    flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+    step, forward, H = setup_step(wl, bufs)
     launches_per_step = launches_filter_gen(wl) + launches_rfft(wl) + launches_forward(wl)
 
     # ---- warm-up
@@ -542,36 +683,13 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     torch.cuda.synchronize()
     fwd_ms = max_over_ranks(statistics.mean(a.elapsed_time(bb) for a, bb in fev))
 
-    # ---- end to end through the C ABI with host buffers: H2D of the step's
-    # inputs from pinned memory, the step, D2H of the result
-    hv = torch.from_numpy(np.ascontiguousarray(inp["v"], np.float32)).to(io).pin_memory()
-    hxs = [torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(io).pin_memory() for x in inp["x"]]
-    hb = torch.from_numpy(inp["b"]).pin_memory()
-    hW = [torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory() for k in wkeys]
-    dW = list(W)
-    if wl.film:   # the per-sample control vectors are step inputs as well
-        hW += [torch.from_numpy(np.ascontiguousarray(inp[k])).pin_memory()
-               for k in ("omega", "gamma", "beta", "sigma")]
-        dW += F
-    hy_out = torch.empty(y.shape, dtype=io).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in [hv, *hxs, hb, *hW])
-    d2h = hy_out.numel() * hy_out.element_size()
-    eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        eev[i][0].record(stream)
-        v.copy_(hv, non_blocking=True)
-        for xd, xh in zip(xs, hxs):
-            xd.copy_(xh, non_blocking=True)
-        b.copy_(hb, non_blocking=True)
-        for wd, wh in zip(dW, hW):
-            wd.copy_(wh, non_blocking=True)
-        step()
-        hy_out.copy_(y, non_blocking=True)
-        eev[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(bb) for a, bb in eev))
+    # ---- end to end through the C ABI with host buffers: every step copies
+    # its inputs from pinned host memory (H2D), runs the whole path and reads
+    # its result back (D2H).  Steps run as a pipeline over two buffer sets on
+    # three streams, as a stream of batches would be served: the H2D of step
+    # i+1 and the D2H of step i-1 overlap the compute of step i.  Every copy
+    # and launch lies inside the timed region.
+    e2e_ms, h2d, d2h = run_e2e(args, wl, inp, bufs, step, max_over_ranks)
 
     # ---- the backward pass (1-D and 2-D): one call per timed repetition
     bwd = None
@@ -643,6 +761,10 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
                "alg_bytes_per_call": alg_bytes_backward(wl),
                "achieved_gbs": alg_bytes_backward(wl) / (bwd_ms / 1e3) / 1e9}
 
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = per_config_forward(args, wl, fwd_ms, flush, gpu_id)
+
     ranks.close()
     if rank != 0:
         return None
@@ -670,6 +792,8 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     if bwd is not None:
         bwd["frac"] = bwd["achieved_gbs"] / peak
         line["backward"] = bwd
+    if per_config is not None:
+        line["per_config"] = per_config
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_seconds)
     return line
@@ -824,7 +948,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="c1", choices=list(synth.WORKLOADS))
+    ap.add_argument("--workload", default="c3_1m", choices=list(synth.WORKLOADS))
+    ap.add_argument("--channels", type=int, default=0,
+                    help="run the workload with this many channels instead (small profiling cases)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the forward timing of every configuration")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -832,6 +960,9 @@ def main():
     if args.warmup < 3:
         raise SystemExit("bench.py: at least 3 warm-up steps are required")
     wl = synth.WORKLOADS[args.workload]
+    if args.channels:
+        wl = wl.with_(D=args.channels, name=f"{wl.name}_D{args.channels}")
+        args.no_per_config = True
     line = run_reference(args, wl) if args.impl == "reference" else run_gpu(args, wl)
     if line is not None:
         print(json.dumps(line), flush=True)

@@ -286,8 +286,10 @@ HYENA_API hyena_status_t hyena_fftconv_gate_backward_circular_per_sample(const v
  * Same arguments and results as hyena_fftconv_gate_forward with the cached
  * spectrum H (no h, no workspace).  Sequences longer than 16384 use a
  * scratch array inside the library instead of a workspace:
- *  - its device address is looked up (cudaGetSymbolAddress) on the first
- *    call on each device; make that first call before any stream capture;
+ *  - its device address is looked up (cudaGetSymbolAddress, the caller's
+ *    device current) on every call, so it stays right after
+ *    cudaDeviceReset; the first call on a device loads the library's
+ *    device code there, so make it before any stream capture;
  *  - one sequence's scratch, 8 L bytes, must fit it: L <= 2^21, else
  *    HYENA_ERR_WORKSPACE;
  *  - all calls on a device share it and it keeps the last call's contents

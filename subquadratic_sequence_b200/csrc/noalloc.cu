@@ -13,9 +13,12 @@
 // (16 MB), so every GPU that loads the library holds those 16 MB until the
 // process exits.  In host code the array's name is only a stand-in for the
 // device object: its device address is looked up with cudaGetSymbolAddress,
-// once per device, with that device current, on the first call made on that
-// device, and passed to the kernels.  Make that first call on each device
-// before any stream capture.
+// with the caller's device current, and passed to the kernels.  The lookup
+// runs on every call (a host-side table lookup, no device work), so the
+// address stays right when a context is torn down and made again
+// (cudaDeviceReset), which may load the array at another address.  The
+// first call on a device is the one that loads the library's device code
+// there; make it before any stream capture.
 //
 // Sharing rules: every call on a device uses the same array and leaves the
 // last call's contents in it.  Nothing in it needs to start at zero -- each
@@ -24,8 +27,6 @@
 // different host threads without ordering) race on it: order such calls on
 // one stream or synchronise between them.
 #include <stdint.h>
-
-#include <mutex>
 
 #include "launch.cuh"
 
@@ -39,26 +40,14 @@ namespace {
 constexpr size_t kScratchBytes = HYENA_NOALLOC_SCRATCH_BYTES;
 constexpr long kScratchSlots = (long)(kScratchBytes / sizeof(float2));
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-float2* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (looked up on
-// the first call per device).
+// Device address of the scratch array on the current device, looked up on
+// every call: a cached address would go stale after cudaDeviceReset.
 hyena_status_t scratch_address(float2** out)
 {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return from_cuda(e);
-    if (dev < 0 || dev >= kMaxDevices) return HYENA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return from_cuda(e);
-        g_scratch_addr[dev] = static_cast<float2*>(p);
-    }
-    *out = g_scratch_addr[dev];
+    *out = static_cast<float2*>(p);
     return HYENA_OK;
 }
 

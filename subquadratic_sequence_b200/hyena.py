@@ -299,13 +299,28 @@ def hyena_fftconv_gate_forward_noalloc(v: torch.Tensor, xs, bias: torch.Tensor, 
     B, D, L = v.shape
     N = len(xs)
     io = io_dtype(v)
+    # the C entry point trusts these extents: check them here, and that
+    # every tensor lives on v's device, whose built-in scratch is used
+    if tuple(H.shape) != (N, D, L):
+        raise ValueError(f"H must be [N][D][L] = {(N, D, L)}, got {tuple(H.shape)}")
+    if tuple(bias.shape) != (N, D):
+        raise ValueError(f"bias must be [N][D] = {(N, D)}, got {tuple(bias.shape)}")
+    for i, x in enumerate(xs):
+        if tuple(x.shape) != (B, D, L):
+            raise ValueError(f"x[{i}] must have v's shape {(B, D, L)}, got {tuple(x.shape)}")
+    if out is not None and tuple(out.shape) != (B, D, L):
+        raise ValueError(f"out must have v's shape {(B, D, L)}, got {tuple(out.shape)}")
+    for name, t in [("H", H), ("bias", bias), ("out", out), *[(f"x[{i}]", x) for i, x in enumerate(xs)]]:
+        if t is not None and t.device != v.device:
+            raise ValueError(f"{name} is on {t.device}, v on {v.device}: all must be on one device")
     xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
     if out is None:
         out = torch.empty_like(v)
-    _check("hyena_fftconv_gate_forward_noalloc", LIB.hyena_fftconv_gate_forward_noalloc(
-        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
-        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
-        ctypes.c_void_p(_dev(out, v.dtype, "y")), _stream(stream)))
+    with torch.cuda.device(v.device):
+        _check("hyena_fftconv_gate_forward_noalloc", LIB.hyena_fftconv_gate_forward_noalloc(
+            ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
+            ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
+            ctypes.c_void_p(_dev(out, v.dtype, "y")), _stream(stream)))
     return out
 
 

@@ -408,3 +408,32 @@ def test_3d_per_sample_entries_reject_bad_arguments(lib):
     assert g(*a(W=8)) == UNSUPPORTED
     assert g(*a(y=P(0))) == INVALID                                              # y aliases v
     assert g(*a(Hs=ctypes.c_void_p(A + 3 * BIG + 8))) == INVALID
+
+
+def fwd_noalloc(lib, v=P(0), xs=(P(1), P(2)), H=P(3), bias=P(4), B=2, D=3, L=64, N=None, io=F32,
+                y=P(5)):
+    N = len(xs) if N is None else N
+    arr = (ctypes.c_void_p * max(len(xs), 1))(*[x.value if x is not None else None for x in xs])
+    return lib.hyena_fftconv_gate_forward_noalloc(v, arr, H, bias, B, D, L, N, io, y, None)
+
+
+def test_noalloc_rejects_bad_arguments(lib):
+    assert fwd_noalloc(lib, v=None) == INVALID
+    assert fwd_noalloc(lib, H=None) == INVALID
+    assert fwd_noalloc(lib, y=None) == INVALID
+    assert fwd_noalloc(lib, xs=(P(1), None)) == INVALID
+    assert fwd_noalloc(lib, B=0) == INVALID
+    assert fwd_noalloc(lib, io=3) == INVALID
+    assert fwd_noalloc(lib, L=1000) == UNSUPPORTED
+    assert fwd_noalloc(lib, L=1 << 23) == UNSUPPORTED
+    # one sequence's four-step scratch (8 L bytes) must fit the built-in 16 MB
+    assert fwd_noalloc(lib, L=1 << 22) == WORKSPACE
+    assert fwd_noalloc(lib, v=ctypes.c_void_p(A + 8)) == INVALID
+    assert fwd_noalloc(lib, H=ctypes.c_void_p(A + 3 * BIG + 8)) == INVALID
+    # y overlapping v, an x_n, the spectra or the bias
+    for L in (64, 1 << 16):
+        assert fwd_noalloc(lib, y=P(0), L=L) == INVALID
+        assert fwd_noalloc(lib, y=ctypes.c_void_p(A + 2 * BIG + 256), L=L) == INVALID
+        assert fwd_noalloc(lib, y=ctypes.c_void_p(A + 1 * BIG - 256), L=L) == INVALID
+        assert fwd_noalloc(lib, y=P(3), L=L) == INVALID
+        assert fwd_noalloc(lib, y=ctypes.c_void_p(A + 4 * BIG - 16), L=L) == INVALID

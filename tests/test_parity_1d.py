@@ -206,22 +206,46 @@ def _sampled_full_size(hy, name, n_samples, seed):
     return assert_close(got, np.stack(refs), wl.io, name)
 
 
-def test_c1_full_size_sampled(hy):
-    """Order-2, B=8, D=768, L=2048, bf16 storage: the whole workload on the
-    GPU, 64 seeded (b, d) rows (plus the first and last) from the oracle."""
-    _sampled_full_size(hy, "c1", 64, seed=1)
+def _full_size(hy, name):
+    """The whole workload on the GPU (filter generation, spectra, forward)
+    against the oracle (its own filters, FFT route) on every (b, d) row."""
+    wl = synth.WORKLOADS[name]
+    inp = synth.make_inputs(wl)
+    h = gpu_filters(inp, wl)
+    H = hy.hyena_filter_rfft(h)
+    del h
+    y = hy.hyena_fftconv_gate_forward(dev(inp["v"], wl.io), [dev(x, wl.io) for x in inp["x"]],
+                                      dev(inp["b"]), H=H)
+    torch.cuda.synchronize()
+    del H
+    got = host(y)
+    del y
+    ref = oracle.hyena_forward(inp["v"], np.stack(inp["x"]), oracle_filters(inp, wl), inp["b"], route="fft")
+    return assert_close(got, ref, wl.io, name)
+
+
+def test_c1_full_size(hy):
+    """Order-2, B=8, D=768, L=2048, bf16 storage: all 6144 (b, d) rows."""
+    _full_size(hy, "c1")
 
 
 @pytest.mark.parametrize("name", ["c2_8k", "c2_16k"])
-def test_c2_full_size_sampled(hy, name):
-    """Order-3, B=2, D=768, L=8192 / 16384, fp32."""
-    _sampled_full_size(hy, name, 16, seed=2)
+def test_c2_full_size(hy, name):
+    """Order-3, B=2, D=768, L=8192 / 16384, fp32: all 1536 (b, d) rows."""
+    _full_size(hy, name)
 
 
-@pytest.mark.parametrize("name", ["c3_64k", "c3_256k", "c3_1m"])
-def test_c3_full_size_sampled(hy, name):
-    """Order-2, B=1, D=256, L = 64k / 256k / 1M, fp32: the four-step path."""
-    _sampled_full_size(hy, name, 4 if name != "c3_1m" else 2, seed=3)
+@pytest.mark.parametrize("name", ["c3_64k", "c3_256k"])
+def test_c3_full_size(hy, name):
+    """Order-2, B=1, D=256, L = 64k / 256k, fp32 (the four-step path): all
+    256 rows."""
+    _full_size(hy, name)
+
+
+def test_c3_1m_full_size_sampled(hy):
+    """Order-2, B=1, D=256, L = 1M, fp32: the whole workload on the GPU, 8
+    seeded channels (plus the first and last) from the oracle."""
+    _sampled_full_size(hy, "c3_1m", 8, seed=3)
 
 
 def test_long_forward_from_filters(hy):
