@@ -355,10 +355,12 @@ WKEYS = ("W1", "W2", "W3", "Wout", "alpha")
 FILM_KEYS = ("omega", "gamma", "beta", "sigma")
 
 
-def setup_step(wl: synth.Workload, bf: Buffers):
+def setup_step(wl: synth.Workload, bf: Buffers, spill: bool = False):
     """The step (filter generation, spectra, forward) and the forward alone
     of one workload on one buffer set, with the filters, spectra and
-    workspaces they use allocated once.  Returns (step, forward, H)."""
+    workspaces they use allocated once.  Returns (step, forward, H).
+    spill: the forward that writes z to HBM between orders instead of the
+    fused one (1-D workloads with a spill variant)."""
     import torch
     from subquadratic_sequence_b200 import hyena
 
@@ -495,8 +497,15 @@ def setup_step(wl: synth.Workload, bf: Buffers):
         ws_rfft = torch.empty(ws_rfft_n, device="cuda", dtype=torch.uint8) if ws_rfft_n else None
         ws_fwd = torch.empty(ws_fwd_n, device="cuda", dtype=torch.uint8) if ws_fwd_n else None
 
-        def forward():
-            hyena.hyena_fftconv_gate_forward(v, xs, b, H=H, out=y, workspace=ws_fwd)
+        if spill:     # z spilled to HBM between orders, one launch per order
+            ws_fwd = torch.empty(hyena.hyena_fftconv_spill_workspace_size(wl.B, wl.D, wl.L, wl.N),
+                                 device="cuda", dtype=torch.uint8)
+
+            def forward():
+                hyena.hyena_fftconv_gate_forward_spill(v, xs, b, H, out=y, workspace=ws_fwd)
+        else:
+            def forward():
+                hyena.hyena_fftconv_gate_forward(v, xs, b, H=H, out=y, workspace=ws_fwd)
 
         def step():
             hyena.hyena_filter_gen(*W, wl.N, wl.D, wl.L, n_bands=synth.N_BANDS, width=synth.WIDTH,
@@ -519,7 +528,7 @@ def run_e2e(args, wl: synth.Workload, inp: dict, bufs: "Buffers", step, max_over
     hout = [torch.empty(bufs.y.shape, dtype=io).pin_memory() for _ in range(2)]
     sets = [(bufs, step)]
     bufs2 = Buffers(wl, inp)
-    step2, _, _ = setup_step(wl, bufs2)
+    step2, _, _ = setup_step(wl, bufs2, spill=args.forward == "spill")
     sets.append((bufs2, step2))
     dins = [[s.v, *s.xs, s.b, *s.W, *s.F] for s, _ in sets]
     h2d = sum(t.numel() * t.element_size() for t in hin)
@@ -571,8 +580,14 @@ def run_e2e(args, wl: synth.Workload, inp: dict, bufs: "Buffers", step, max_over
     return ms, h2d, d2h
 
 
-# the forward of every BASELINE configuration, timed in the same run as the
-# headline line (the parity configurations c0..c4 at their full sizes)
+def has_spill(wl: synth.Workload) -> bool:
+    """Workloads with a spill variant to compare against (1-D, shared
+    spectra, padded, L <= 16384, more than one order)."""
+    return wl.kind == "1d" and not wl.film and not wl.circular and wl.L <= 16384 and wl.N > 1
+
+
+# the configurations whose forward is timed in the same run as the headline
+# line (the parity configurations c0..c4 at their full sizes)
 PER_CONFIG = ("c0", "c1", "c2_8k", "c2_16k", "c3_64k", "c3_256k", "c3_1m", "c4")
 
 
@@ -587,29 +602,52 @@ def per_config_forward(args, headline: synth.Workload, headline_ms: float, flush
     with ClockSampler(gpu_id) as clk:
         for name in PER_CONFIG:
             wl = synth.WORKLOADS[name]
-            if wl == headline:
-                ms = headline_ms
-            else:
-                bufs = Buffers(wl, synth.make_inputs(wl))
-                step, forward, _ = setup_step(wl, bufs)
-                for _ in range(3):
-                    step()
-                reps = 10 if wl.positions >= (1 << 26) else 20
+            reps = 10 if wl.positions >= (1 << 26) else 20
+
+            def timed(fn) -> float:
                 evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                        for _ in range(reps)]
                 for a, b in evs:
                     flush.zero_()
                     a.record(stream)
-                    forward()
+                    fn()
                     b.record(stream)
                 torch.cuda.synchronize()
-                ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-                del bufs, step, forward
+                return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+            spill_ms = None
+            if wl == headline:
+                ms = headline_ms
+            else:
+                bufs = Buffers(wl, synth.make_inputs(wl))
+                step, forward, H = setup_step(wl, bufs)
+                for _ in range(3):
+                    step()
+                ms = timed(forward)
+                if has_spill(wl):
+                    # the same forward with z spilled to HBM between orders
+                    from subquadratic_sequence_b200 import hyena
+                    ws = torch.empty(hyena.hyena_fftconv_spill_workspace_size(wl.B, wl.D, wl.L, wl.N),
+                                     device="cuda", dtype=torch.uint8)
+
+                    def spill():
+                        hyena.hyena_fftconv_gate_forward_spill(bufs.v, bufs.xs, bufs.b, H, out=bufs.y,
+                                                               workspace=ws)
+                    spill()
+                    spill_ms = timed(spill)
+                    del ws
+                del bufs, step, forward, H
                 torch.cuda.empty_cache()
             nbytes = alg_bytes_forward(wl)
             out[name] = {"kernel": forward_kernel(wl), "ms_per_launch": ms, "alg_bytes_per_launch": nbytes,
                          "achieved_gbs": nbytes / (ms / 1e3) / 1e9, "frac": nbytes / (ms / 1e3) / 1e9 / peak,
                          "value": wl.positions / (ms / 1e3), "unit": UNIT}
+            if spill_ms is not None:
+                moved = nbytes + 2 * (wl.N - 1) * wl.positions * 4
+                out[name]["spill"] = {
+                    "kernel": "fused1d_order_kernel x N (hyena_fftconv_gate_forward_spill)",
+                    "ms_per_call": spill_ms, "frac": nbytes / (spill_ms / 1e3) / 1e9 / peak,
+                    "bytes_moved_per_call": moved, "fused_speedup": spill_ms / ms}
     out["clocks"] = clk.summary()
     return out
 
@@ -635,8 +673,11 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     v, xs, b, y = bufs.v, bufs.xs, bufs.b, bufs.y
     flush = torch.empty(L2_FLUSH_BYTES, device="cuda", dtype=torch.uint8)
     stream = torch.cuda.current_stream()
-    step, forward, H = setup_step(wl, bufs)
-    launches_per_step = launches_filter_gen(wl) + launches_rfft(wl) + launches_forward(wl)
+    step, forward, H = setup_step(wl, bufs, spill=args.forward == "spill")
+    launches_per_step = (launches_filter_gen(wl) + launches_rfft(wl)
+                         + (wl.N if args.forward == "spill" else launches_forward(wl)))
+    fwd_name = ("fused1d_order_kernel x N (hyena_fftconv_gate_forward_spill)" if args.forward == "spill"
+                else forward_kernel(wl))
 
     # ---- warm-up
     for _ in range(args.warmup):
@@ -777,11 +818,12 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic", "config": describe(wl),
-        "roofline": {"bound": "hbm", "kernel": forward_kernel(wl),
+        "data": "synthetic", "config": {**describe(wl), **({"forward": "spill: z in HBM between orders"}
+                                                            if args.forward == "spill" else {})},
+        "roofline": {"bound": "hbm", "kernel": fwd_name,
                      "achieved": achieved, "peak": peak, "peak_source": peak_kind,
                      "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": ncu_traffic(forward_kernel(wl).split()[0], wl.name),
+                     "traffic": ncu_traffic(fwd_name.split()[0], wl.name),
                      "alg_bytes_per_launch": alg_bytes_forward(wl), "ms_per_launch": fwd_ms},
         "forward_only": {"value": wl.positions * world / (fwd_ms / 1e3), "unit": UNIT},
         "e2e": {"value": positions * args.steps / (e2e_ms / 1e3), "unit": UNIT,
@@ -937,7 +979,8 @@ def run_reference(args, wl: synth.Workload) -> dict | None:
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": describe(wl),
+            "data": "synthetic", "config": {**describe(wl), **({"forward": "spill: z in HBM between orders"}
+                                                            if args.forward == "spill" else {})},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -951,6 +994,8 @@ def main():
     ap.add_argument("--workload", default="c3_1m", choices=list(synth.WORKLOADS))
     ap.add_argument("--channels", type=int, default=0,
                     help="run the workload with this many channels instead (small profiling cases)")
+    ap.add_argument("--forward", default="fused", choices=["fused", "spill"],
+                    help="spill: the forward that writes z to HBM between orders (L <= 16384)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the forward timing of every configuration")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -960,6 +1005,8 @@ def main():
     if args.warmup < 3:
         raise SystemExit("bench.py: at least 3 warm-up steps are required")
     wl = synth.WORKLOADS[args.workload]
+    if args.forward == "spill" and not has_spill(wl):
+        raise SystemExit(f"bench.py: {wl.name} has no spill variant (1-D, shared spectra, L <= 16384, N > 1)")
     if args.channels:
         wl = wl.with_(D=args.channels, name=f"{wl.name}_D{args.channels}")
         args.no_per_config = True

@@ -273,6 +273,32 @@ HYENA_API hyena_status_t hyena_fftconv_gate_backward_circular_per_sample(const v
                                                                          float* dbias, void* workspace,
                                                                          size_t ws_bytes, void* stream);
 
+/* The order-N forward with z spilled to HBM between orders: one launch per
+ * order, each reading z_{n-1} (v for n = 1) and writing z_n (y for n = N)
+ * to global memory in float32, instead of chaining all orders on chip as
+ * hyena_fftconv_gate_forward does for L <= 16384.  The arithmetic of an
+ * order is the same as there (same FFT passes, spectral step and gate), so
+ * the results agree to float32 rounding.  It exists to measure what keeping
+ * the intermediates on chip saves ("Native Multi-Dimensional Subquadratic
+ * Operators via Input Dependent Long Convolutions", Implementation: nSubQ,
+ * Fused Kernels / Memory Efficiency).
+ * Arguments as hyena_fftconv_gate_forward with the cached spectrum H, plus
+ *   workspace / ws_bytes: at least hyena_fftconv_spill_workspace_size(B, D,
+ *          L, N) bytes (B D L float32 for z, 0 for N = 1), 256-byte
+ *          aligned; nothing in it needs to start at zero; it must not
+ *          overlap v, x_n, H, bias or y.
+ * L is a power of two, 16 <= L <= 16384 (HYENA_ERR_UNSUPPORTED beyond);
+ * 1 <= N <= HYENA_MAX_ORDER.  Returns HYENA_ERR_WORKSPACE if the workspace
+ * is missing or too small.  The size function returns (size_t)-1 for
+ * invalid or unsupported sizes. */
+HYENA_API size_t hyena_fftconv_spill_workspace_size(int B, int D, int L, int N);
+HYENA_API hyena_status_t hyena_fftconv_gate_forward_spill(const void* v, const void* const* x,
+                                                         const float* H, const float* bias,
+                                                         int B, int D, int L, int N,
+                                                         hyena_dtype_t io, void* y,
+                                                         void* workspace, size_t ws_bytes,
+                                                         void* stream);
+
 /* Size of the scratch array built into the library for
  * hyena_fftconv_gate_forward_noalloc (16 MB on every device that loads the
  * library, held until the process exits). */

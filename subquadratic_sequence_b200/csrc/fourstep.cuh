@@ -132,7 +132,9 @@ struct FourStep {
     static constexpr size_t ROW_SMEM = sizeof(float2) * ROWS * ROW_STRIDE;
     static constexpr int ROW_CTAS_PER_SEQ = (M1 / 2) / U;
     // column kernel: TC consecutive columns per CTA, column index fastest
-    // across threads so every global access is a TC-element run
+    // across threads so every global access is a TC-element run (8 columns
+    // at M1 = 1024, 64-byte runs, two CTAs per SM: 13 % slower on L = 2^20
+    // than 16 columns with one CTA per SM)
     static constexpr int TC = (512 / F1::T) > 16 ? 16 : ((512 / F1::T) < 4 ? 4 : 512 / F1::T);
     static constexpr int COL_THREADS = TC * F1::T;
     static constexpr int COL_STRIDE = stride_mod16(M1, 16 / TC);
@@ -197,25 +199,33 @@ struct FourStep {
 };
 
 // The real split + bias-folded spectral multiply + inverse re-pack of one
-// bin pair (k, Mtot - k), as in fused1d.cuh (scale 1/(2P) included).
+// bin pair (k, Mtot - k), as in fused1d.cuh, in reduced form.  With
+// z1 = Z[k], z2 = Z[Mtot - k] (the packed transform), w = exp(-i pi k /
+// Mtot) = c + i s, the bias-folded filter bins G1 = (H[k] + b) / (2 Mtot),
+// G2 = (H[Mtot - k] + b) / (2 Mtot), and P = G1 + conj(G2),
+// Q = G1 - conj(G2) (the bias cancels in Q), the inverse transform's
+// inputs are
+//   Z'[k]        = (P + s Q) z1 + i c Q conj(z2),
+//   Z'[Mtot - k] = conj(P - s Q) z2 + i c conj(Q) conj(z1):
+// the split U[k] = ((z1 + conj z2) - i w (z1 - conj z2)) / 2 and its
+// inverse re-pack composed, which leaves real coefficients 2 +- 2s and
+// +-2ic on the products of (H + b) with z1 and conj(z2).
 template <int MTOT>
 __device__ __forceinline__ void spectral_pair(float2& z1, float2& z2, float2 h1, float2 h2,
                                               float2 w, float bias)
 {
-    constexpr float s = 1.0f / (4.0f * (float)MTOT);
-    const float2 bc = cconj(z2);
-    const float2 S = cadd(z1, bc);
-    const float2 Tw = cmul(w, csub(z1, bc));
-    const float2 X1 = make_float2(S.x + Tw.y, S.y - Tw.x);
-    const float2 X2 = make_float2(S.x - Tw.y, -(S.y + Tw.x));
-    const float2 G1 = make_float2((h1.x + bias) * s, h1.y * s);
-    const float2 G2 = make_float2((h2.x + bias) * s, h2.y * s);
-    const float2 Y1 = cmul(X1, G1);
-    const float2 Y2 = cmul(X2, G2);
-    const float2 U = make_float2(Y1.x + Y2.x, Y1.y - Y2.y);
-    const float2 V = cmulc(make_float2(Y1.x - Y2.x, Y1.y + Y2.y), w);
-    z1 = make_float2(U.x - V.y, U.y + V.x);
-    z2 = make_float2(U.x + V.y, V.x - U.y);
+    constexpr float sc = 1.0f / (2.0f * (float)MTOT);
+    const float bias2 = (2.0f * sc) * bias;
+    const float2 P = make_float2(fmaf(sc, h1.x + h2.x, bias2), sc * (h1.y - h2.y));
+    const float2 Q = make_float2(sc * (h1.x - h2.x), sc * (h1.y + h2.y));
+    const float2 A1 = make_float2(fmaf(w.y, Q.x, P.x), fmaf(w.y, Q.y, P.y));     // P + s Q
+    const float2 A2 = make_float2(fmaf(-w.y, Q.x, P.x), fmaf(-w.y, Q.y, P.y));   // P - s Q
+    const float2 C = make_float2(w.x * Q.x, w.x * Q.y);                          // c Q
+    const float2 a = z1, b = z2;
+    z1 = make_float2(fmaf(A1.x, a.x, fmaf(-A1.y, a.y, fmaf(-C.y, b.x, C.x * b.y))),
+                     fmaf(A1.x, a.y, fmaf(A1.y, a.x, fmaf(C.x, b.x, C.y * b.y))));
+    z2 = make_float2(fmaf(A2.x, b.x, fmaf(A2.y, b.y, fmaf(C.x, a.y, C.y * a.x))),
+                     fmaf(A2.x, b.y, fmaf(-A2.y, b.x, fmaf(C.x, a.x, -C.y * a.y))));
 }
 
 // The real split alone: packed spectrum bins k and Mtot - k from Z[k], Z[Mtot - k].

@@ -270,23 +270,25 @@ struct Fft1d {
     // the bias-folded filter spectrum, and the inverse re-pack.
     //   z1 = Z[k], z2 = Z[M-k]; h1 = H[k], h2 = H[M-k]; w = exp(-i pi k/M)
     // returns Z'[k] in z1 and Z'[M-k] in z2 (scale 1/(2P) included).
+    // With G1 = (h1 + b) / (2M), G2 = (h2 + b) / (2M), P = G1 + conj(G2),
+    // Q = G1 - conj(G2) and w = c + i s, the split and the re-pack compose
+    // to  Z'[k] = (P + s Q) z1 + i c Q conj(z2),
+    //     Z'[M-k] = conj(P - s Q) z2 + i c conj(Q) conj(z1).
     static __device__ __forceinline__ void pair(float2& z1, float2& z2, float2 h1, float2 h2,
                                                 float2 w, float bias)
     {
-        constexpr float s = 1.0f / (4.0f * (float)M);   // 1/2 (split) * 1/P (inverse)
-        const float2 bc = cconj(z2);
-        const float2 S = cadd(z1, bc);
-        const float2 Tw = cmul(w, csub(z1, bc));
-        const float2 X1 = make_float2(S.x + Tw.y, S.y - Tw.x);       // S - i T
-        const float2 X2 = make_float2(S.x - Tw.y, -(S.y + Tw.x));    // conj(S + i T)
-        const float2 G1 = make_float2((h1.x + bias) * s, h1.y * s);
-        const float2 G2 = make_float2((h2.x + bias) * s, h2.y * s);
-        const float2 Y1 = cmul(X1, G1);
-        const float2 Y2 = cmul(X2, G2);
-        const float2 U = make_float2(Y1.x + Y2.x, Y1.y - Y2.y);       // Y1 + conj Y2
-        const float2 V = cmulc(make_float2(Y1.x - Y2.x, Y1.y + Y2.y), w);  // conj(w)(Y1 - conj Y2)
-        z1 = make_float2(U.x - V.y, U.y + V.x);                       // U + i V
-        z2 = make_float2(U.x + V.y, V.x - U.y);                       // conj(U - i V)
+        constexpr float sc = 1.0f / (2.0f * (float)M);
+        const float bias2 = (2.0f * sc) * bias;
+        const float2 P = make_float2(fmaf(sc, h1.x + h2.x, bias2), sc * (h1.y - h2.y));
+        const float2 Q = make_float2(sc * (h1.x - h2.x), sc * (h1.y + h2.y));
+        const float2 A1 = make_float2(fmaf(w.y, Q.x, P.x), fmaf(w.y, Q.y, P.y));     // P + s Q
+        const float2 A2 = make_float2(fmaf(-w.y, Q.x, P.x), fmaf(-w.y, Q.y, P.y));   // P - s Q
+        const float2 C = make_float2(w.x * Q.x, w.x * Q.y);                          // c Q
+        const float2 a = z1, b = z2;
+        z1 = make_float2(fmaf(A1.x, a.x, fmaf(-A1.y, a.y, fmaf(-C.y, b.x, C.x * b.y))),
+                         fmaf(A1.x, a.y, fmaf(A1.y, a.x, fmaf(C.x, b.x, C.y * b.y))));
+        z2 = make_float2(fmaf(A2.x, b.x, fmaf(A2.y, b.y, fmaf(C.x, a.y, C.y * a.x))),
+                         fmaf(A2.x, b.y, fmaf(-A2.y, b.x, fmaf(C.x, a.x, -C.y * a.y))));
     }
 
     // Spectral step on the RL folded layout for one order; Hs is the
@@ -495,6 +497,83 @@ fused1d_kernel(Fused1dArgs args)
     if (active) {
         PT* yp = reinterpret_cast<PT*>(args.y) + seq * SEQ;
         F::for_each_io(t, [&](int i, int m) { IOP::store(yp + m, a[i]); });
+    }
+}
+
+// One order of the recurrence per launch, with z in global memory between
+// orders: the counterpart of fused1d_kernel that spills z_n to HBM (float32)
+// instead of chaining the orders on chip.  It exists to measure what the
+// chaining saves ("Native Multi-Dimensional Subquadratic Operators via Input
+// Dependent Long Convolutions", Implementation: nSubQ, Memory Efficiency:
+// intermediates kept on chip).  z_{n-1} is read as ZIN (v's type for the
+// first order, else float), z_n written as ZOUT (y's type for the last
+// order, else float); x_n is IO.  zin and zout may be the same buffer: each
+// sequence is read whole by the CTA that owns it before that CTA writes it.
+struct Fused1dOrderArgs {
+    const void* zin;               // [B][D][L] ZIN
+    const void* x;                 // [B][D][L] IO (x_n)
+    void* zout;                    // [B][D][L] ZOUT
+    const float2* H;               // [D][L] packed spectra of order n
+    const float* bias;             // [D] (b_n)
+    int B, D;
+};
+
+template <int LOG2M, typename IO, typename ZIN, typename ZOUT>
+__global__ void __launch_bounds__(Fft1d<LOG2M>::THREADS, Fft1d<LOG2M>::MIN_BLOCKS)
+fused1d_order_kernel(Fused1dOrderArgs args)
+{
+    grid_dependency_begin();
+    using F = Fft1d<LOG2M>;
+    using XP = IoPair<IO>;
+    constexpr int M = F::M, E = F::E, T = F::T, SEQ = F::SEQ;
+    constexpr int X_BYTES = SEQ * (int)sizeof(typename XP::T);
+    extern __shared__ __align__(16) float2 smem_dyn[];
+
+    const int g = threadIdx.x / T, t = threadIdx.x % T;
+    const int BD = args.B * args.D;
+    const int q_raw = blockIdx.x * F::G + g;
+    const bool active = q_raw < BD;
+    const int q = active ? q_raw : BD - 1;
+    const int d = q / args.B, b = q % args.B;
+    const size_t seq = (size_t)b * args.D + d;
+    float2* sm = smem_dyn + g * F::SMEM_SEQ;
+    float2* stage = smem_dyn + F::G * F::SMEM_SEQ + g * F::STAGE_SEQ;
+    const float2* Hg = args.H + (size_t)d * M;
+    const typename XP::T* xg = reinterpret_cast<const typename XP::T*>(args.x) + seq * SEQ;
+    const float bias = __ldg(args.bias + d);
+
+    if constexpr (!F::H_IN_EXCHANGE) cp_async_row(stage, Hg, M * 8, t, T);
+    float2 a[E];
+    {
+        const typename IoPair<ZIN>::T* zp = reinterpret_cast<const typename IoPair<ZIN>::T*>(args.zin) + seq * SEQ;
+        F::for_each_io(t, [&](int i, int m) { a[i] = IoPair<ZIN>::load(zp + m); });
+    }
+    const float2* Hs;
+    if constexpr (F::H_IN_EXCHANGE) {
+        cp_async_row(stage, xg, X_BYTES, t, T);
+        F::forward(a, sm, t);
+        cp_async_row(sm, Hg, M * 8, t, T);
+        Hs = sm;
+    } else {
+        F::forward(a, sm, t);
+        Hs = stage;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    F::spectral(a, Hs, bias, t);
+    __syncthreads();
+    if constexpr (!F::H_IN_EXCHANGE) cp_async_row(stage, xg, X_BYTES, t, T);
+    F::inverse(a, sm, t);
+    cp_async_wait_all();
+    __syncthreads();
+    const typename XP::T* xs = reinterpret_cast<const typename XP::T*>(stage);
+    F::for_each_io(t, [&](int i, int m) {
+        const float2 xv = XP::load_smem(xs + m);
+        a[i] = make_float2(a[i].x * xv.x, a[i].y * xv.y);
+    });
+    if (active) {
+        typename IoPair<ZOUT>::T* zp = reinterpret_cast<typename IoPair<ZOUT>::T*>(args.zout) + seq * SEQ;
+        F::for_each_io(t, [&](int i, int m) { IoPair<ZOUT>::store(zp + m, a[i]); });
     }
 }
 

@@ -1,0 +1,9 @@
+// Per-order forward with z spilled to HBM, bf16 activations, last order (y bf16).
+#include "k_spill.cuh"
+
+namespace hyena {
+hyena_status_t dispatch_order_bf16_last(int log2m, const Fused1dOrderArgs& a, cudaStream_t st)
+{
+    return dispatch_order<__nv_bfloat16, float, __nv_bfloat16>(log2m, a, st);
+}
+}  // namespace hyena

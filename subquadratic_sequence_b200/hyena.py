@@ -64,6 +64,9 @@ def _load() -> ctypes.CDLL:
                                         sz, vp], i),
         "hyena_fftconv_gate_forward_noalloc": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp,
                                                 vp], i),
+        "hyena_fftconv_spill_workspace_size": ([i, i, i, i], sz),
+        "hyena_fftconv_gate_forward_spill": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp, sz,
+                                              vp], i),
         "hyena_fftconv_backward_workspace_size": ([i, i, i], sz),
         "hyena_fftconv_backward_per_sample_workspace_size": ([i, i, i, i], sz),
         "hyena_fftconv_backward_circular_workspace_size": ([i, i, i], sz),
@@ -286,6 +289,36 @@ def hyena_fftconv_gate_forward(v: torch.Tensor, xs, bias: torch.Tensor, *, H=Non
     wn = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("hyena_fftconv_gate_forward", LIB.hyena_fftconv_gate_forward(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, hp, Hp,
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
+        ctypes.c_void_p(_dev(out, v.dtype, "y")), wp, wn, _stream(stream)))
+    return out
+
+
+def hyena_fftconv_spill_workspace_size(B: int, D: int, L: int, N: int) -> int:
+    n = LIB.hyena_fftconv_spill_workspace_size(B, D, L, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv_spill_workspace_size", HYENA_ERR_UNSUPPORTED, "invalid sizes")
+    return n
+
+
+def hyena_fftconv_gate_forward_spill(v: torch.Tensor, xs, bias: torch.Tensor, H: torch.Tensor, *,
+                                     out=None, workspace=None, stream=None):
+    """The order-N forward with z written to HBM (float32) between orders,
+    one launch per order (L <= 16384): the counterpart of the fused forward,
+    which chains the orders on chip."""
+    B, D, L = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    if out is None:
+        out = torch.empty_like(v)
+    need = hyena_fftconv_spill_workspace_size(B, D, L, N)
+    if need and workspace is None:
+        workspace = torch.empty(need, device=v.device, dtype=torch.uint8)
+    wp = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+    wn = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("hyena_fftconv_gate_forward_spill", LIB.hyena_fftconv_gate_forward_spill(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
         ctypes.c_void_p(_dev(out, v.dtype, "y")), wp, wn, _stream(stream)))
     return out

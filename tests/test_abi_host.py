@@ -437,3 +437,31 @@ def test_noalloc_rejects_bad_arguments(lib):
         assert fwd_noalloc(lib, y=ctypes.c_void_p(A + 1 * BIG - 256), L=L) == INVALID
         assert fwd_noalloc(lib, y=P(3), L=L) == INVALID
         assert fwd_noalloc(lib, y=ctypes.c_void_p(A + 4 * BIG - 16), L=L) == INVALID
+
+
+def fwd_spill(lib, v=P(0), xs=(P(1), P(2)), H=P(3), bias=P(4), B=2, D=3, L=64, N=None, io=F32,
+              y=P(5), ws=P(6), wsb=1 << 20):
+    N = len(xs) if N is None else N
+    arr = (ctypes.c_void_p * max(len(xs), 1))(*[x.value if x is not None else None for x in xs])
+    return lib.hyena_fftconv_gate_forward_spill(v, arr, H, bias, B, D, L, N, io, y, ws, wsb, None)
+
+
+def test_spill_rejects_bad_arguments(lib):
+    bad = ctypes.c_size_t(-1).value
+    assert lib.hyena_fftconv_spill_workspace_size(2, 3, 64, 2) == 2 * 3 * 64 * 4
+    assert lib.hyena_fftconv_spill_workspace_size(2, 3, 64, 1) == 0
+    assert lib.hyena_fftconv_spill_workspace_size(2, 3, 1 << 15, 2) == bad
+    assert lib.hyena_fftconv_spill_workspace_size(2, 3, 100, 2) == bad
+    assert fwd_spill(lib, v=None) == INVALID
+    assert fwd_spill(lib, H=None) == INVALID
+    assert fwd_spill(lib, xs=(P(1), None)) == INVALID
+    assert fwd_spill(lib, io=2) == INVALID
+    assert fwd_spill(lib, L=1 << 15) == UNSUPPORTED      # the spill variant covers the fused lengths
+    assert fwd_spill(lib, L=48) == UNSUPPORTED
+    assert fwd_spill(lib, ws=None) == WORKSPACE
+    assert fwd_spill(lib, wsb=2 * 3 * 64 * 4 - 4) == WORKSPACE
+    assert fwd_spill(lib, ws=ctypes.c_void_p(A + 6 * BIG + 16)) == INVALID   # 256-byte alignment
+    assert fwd_spill(lib, y=P(0)) == INVALID
+    assert fwd_spill(lib, ws=P(5)) == INVALID             # workspace overlapping y
+    assert fwd_spill(lib, ws=P(2)) == INVALID             # workspace overlapping x_2
+    assert fwd_spill(lib, ws=P(3)) == INVALID             # workspace overlapping H
