@@ -986,6 +986,36 @@ def run_reference(args, wl: synth.Workload) -> dict | None:
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_dft32(args) -> dict:
+    """One radix-32 FFT level on the FP32 pipes and on the tensor cores
+    (hyena_dft32_stage): device time per level per point, L2-resident input
+    (each vector is read once and transformed `reps` times)."""
+    import torch
+    from subquadratic_sequence_b200 import hyena
+    count, reps = 148 * 2 * 128 * 4, 64
+    rng = np.random.default_rng(5)
+    x = torch.from_numpy((rng.standard_normal((count, 32)) + 1j * rng.standard_normal((count, 32)))
+                         .astype(np.complex64)).cuda()
+    y = torch.empty_like(x)
+    stream = torch.cuda.current_stream()
+    out = {"experiment": "one radix-32 FFT level: FP32 pipes vs tcgen05 tensor cores (3xTF32)",
+           "vectors": count, "reps": reps, "points_per_level": count * 32}
+    for method, name in ((0, "simt"), (1, "tcgen05_3xtf32")):
+        for _ in range(3):
+            hyena.hyena_dft32_stage(x, reps, method, out=y)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
+        for a, b in evs:
+            a.record(stream)
+            hyena.hyena_dft32_stage(x, reps, method, out=y)
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        out[name] = {"ms_per_call": ms, "ps_per_point_per_level": ms * 1e9 / (count * 32 * reps)}
+    out["simt_speedup"] = out["tcgen05_3xtf32"]["ms_per_call"] / out["simt"]["ms_per_call"]
+    out["device_faults"] = hyena.LIB.hyena_device_fault_count()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -996,6 +1026,8 @@ def main():
                     help="run the workload with this many channels instead (small profiling cases)")
     ap.add_argument("--forward", default="fused", choices=["fused", "spill"],
                     help="spill: the forward that writes z to HBM between orders (L <= 16384)")
+    ap.add_argument("--experiment", choices=["dft32"], default=None,
+                    help="dft32: time one radix-32 FFT level on the FP32 pipes and on the tensor cores")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the forward timing of every configuration")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -1004,6 +1036,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("bench.py: at least 3 warm-up steps are required")
+    if args.experiment == "dft32":
+        print(json.dumps(run_dft32(args)), flush=True)
+        return
     wl = synth.WORKLOADS[args.workload]
     if args.forward == "spill" and not has_spill(wl):
         raise SystemExit(f"bench.py: {wl.name} has no spill variant (1-D, shared spectra, L <= 16384, N > 1)")

@@ -100,6 +100,14 @@ HYENA_API const char* hyena_status_string(hyena_status_t status);
  * none). */
 HYENA_API int hyena_last_cuda_error(void);
 
+/* Number of tensor-core waits in this library's kernels that ran out of
+ * time on the current device since the library was loaded (0 when none,
+ * -1 if the device could not be queried).  Every such wait is bounded
+ * (about two seconds); a kernel whose wait times out records it here,
+ * frees its tensor memory and returns without writing its outputs.  The
+ * query is a device-to-host copy and so waits for the device. */
+HYENA_API int hyena_device_fault_count(void);
+
 /* ---------------------------------------------------------------- 1-D */
 
 /* Implicit filters h [N][D][L] float32 from the filter network (see
@@ -298,6 +306,23 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_spill(const void* v, const v
                                                          hyena_dtype_t io, void* y,
                                                          void* workspace, size_t ws_bytes,
                                                          void* stream);
+
+/* A measurement of one FFT level on the two kinds of arithmetic units, used
+ * to choose between them: count independent 32-point complex DFTs (x and y
+ * [count][32] complex64, 16-byte aligned, not overlapping), each applied
+ * reps times in a row to its previous result with the unitary scale
+ * 1/sqrt(32) (so four applications give x back).  method 0: the FP32 pipes
+ * (in registers, every value through shared memory between repetitions, as
+ * a pass of the shared-memory FFTs exchanges); method 1: the tcgen05 tensor
+ * cores (128 vectors as a 128 x 64 real matrix times the 64 x 64 real form
+ * of the DFT matrix, TF32 with a hi/lo split for float32 accuracy, the
+ * accumulator in tensor memory, read back into shared memory every
+ * repetition).  The pages point at matrix-multiply hardware for FFT
+ * convolutions ("Long Context Language Models ... #690", 7:06); this entry
+ * point measures whether a DFT level on it beats the FFT's own level.
+ * 1 <= count <= 2^30, reps >= 1. */
+HYENA_API hyena_status_t hyena_dft32_stage(const float* x, float* y, long count, int reps, int method,
+                                           void* stream);
 
 /* Size of the scratch array built into the library for
  * hyena_fftconv_gate_forward_noalloc (16 MB on every device that loads the

@@ -6,6 +6,7 @@ import glob
 import os
 import shutil
 import subprocess
+import time
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -64,6 +65,7 @@ def _obj_stale(src: str) -> bool:
 def _compile(src: str, verbose: bool) -> str:
     obj, dep = _obj_paths(src)
     tmp = obj + f".tmp{os.getpid()}"
+    t0 = time.time()
     cmd = [nvcc(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-I", INCLUDE, "-I", CSRC, "-MD", "-MF", dep, "-c", "-o", tmp, src]
@@ -73,6 +75,10 @@ def _compile(src: str, verbose: bool) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{r.stdout}{r.stderr}")
     os.replace(tmp, obj)
+    # date the object (and its dependency list) by when the compile began, so
+    # that a source edited while nvcc ran is still newer than the object
+    os.utime(obj, (t0, t0))
+    os.utime(dep, (t0, t0))
     return r.stdout + r.stderr
 
 

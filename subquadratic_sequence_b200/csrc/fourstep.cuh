@@ -53,6 +53,16 @@ struct SmemFft {
     static constexpr int R0 = V == 32 ? S / 32
                             : (LOG2S % 4 == 0) ? 16 : (1 << (LOG2S % 4));   // first pass radix
 
+    // S = 1024: the first pass (radix 32) writes at a stride of 32 values,
+    // where the padding alone (one float2 per 16) still maps threads j and
+    // j + 8 to the same banks.  Between the two passes logical element i is
+    // therefore kept at pad16(i ^ ((i >> 8) & 1)): threads with bit 3 of j
+    // set swap neighbouring values, which separates the two halves of a
+    // half-warp; the second pass reads consecutive elements, which the swap
+    // keeps within one 16-value line.
+    static constexpr bool SWZ = S == 1024;
+    static_assert(!SWZ || (T == 32 && R0 == 32 && NP == 2), "swizzled exchange layout");
+
     // PADDED_IN: the input sits at buf[pad16(i)] (else at buf[i]).
     // ZERO_HI: inputs S/2 .. S-1 are zero (a zero-padded transform): the
     // first pass neither reads them nor multiplies by them, so the caller
@@ -71,13 +81,22 @@ struct SmemFft {
                 constexpr int c = decltype(cc)::value;
                 const int j = t + c * T;
                 const int pj = pad16(j);
-                static_for<R>([&](auto rr) {
-                    constexpr int r = decltype(rr)::value;
-                    if constexpr (ZERO_HI && p == 0 && r >= R / 2)
-                        a[c * R + r] = make_float2(0.0f, 0.0f);
-                    else
-                        a[c * R + r] = buf[(p == 0 && !PADDED_IN) ? j + r * (S / R) : pad16_at<S / R>(j, pj, r)];
-                });
+                if constexpr (SWZ && p == 1) {
+                    // element j + 32 r sits at pad16((j ^ ((r >> 3) & 1)) + 32 r)
+                    const int pj1 = pad16(j ^ 1);
+                    static_for<R>([&](auto rr) {
+                        constexpr int r = decltype(rr)::value;
+                        a[c * R + r] = buf[((r >> 3) & 1 ? pj1 : pj) + r * 34];
+                    });
+                } else {
+                    static_for<R>([&](auto rr) {
+                        constexpr int r = decltype(rr)::value;
+                        if constexpr (ZERO_HI && p == 0 && r >= R / 2)
+                            a[c * R + r] = make_float2(0.0f, 0.0f);
+                        else
+                            a[c * R + r] = buf[(p == 0 && !PADDED_IN) ? j + r * (S / R) : pad16_at<S / R>(j, pj, r)];
+                    });
+                }
             });
             __syncthreads();
             float dep = zero_after(a[0].x);
@@ -89,7 +108,16 @@ struct SmemFft {
                 if constexpr (p > 0)
                     apply_twiddle_powers<R>(ar, expi_pi<SIGN>(2.0f * (float)jm / (float)(NS * R) + dep));
                 dft<R, SIGN>(ar);
-                if constexpr (!LAST) {
+                if constexpr (!LAST && SWZ) {
+                    // element 32 j + r at pad16(32 j + (r ^ b)), b = bit 3 of j:
+                    // 34 j + r + r / 16, plus b for even r and minus b for odd r
+                    const int b = (j >> 3) & 1;
+                    const int pe = 34 * j + b, po = 34 * j - b;
+                    static_for<R>([&](auto rr) {
+                        constexpr int r = decltype(rr)::value;
+                        buf[(r & 1 ? po : pe) + r + (r >> 4)] = ar[r];
+                    });
+                } else if constexpr (!LAST) {
                     const int base = (j / NS) * NS * R + jm;
                     const int pb = pad16(base);
                     static_for<R>([&](auto rr) {
@@ -258,10 +286,13 @@ fourstep_row_kernel(FourStepArgs a)
     float2* Sq = a.S + (size_t)qi * M;
     const int tid = threadIdx.x;
 
+    // the wave scratch stays in L2 for the next launch; spectra and
+    // activations stream through
+    const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
 #pragma unroll 1
     for (int rr = 0; rr < FS::ROWS; ++rr)
-        cp_async_row(smem_fs + rr * RS, Sq + (size_t)FS::row_of(ublk, rr) * M2, M2 * 8, tid,
-                     FS::ROW_THREADS);
+        cp_async_row_hint(smem_fs + rr * RS, Sq + (size_t)FS::row_of(ublk, rr) * M2, M2 * 8, tid,
+                          FS::ROW_THREADS, keep);
     cp_async_wait_all();
     __syncthreads();
 
@@ -281,12 +312,12 @@ fourstep_row_kernel(FourStepArgs a)
         FS::for_each_pair(smem_fs, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2 w) {
             if (kind == 1) {                                    // bins 0 and M share slot 0
                 const float2 z = *p1;
-                Ho[0] = make_float2(z.x + z.y, z.x - z.y);
+                st_hint(Ho, make_float2(z.x + z.y, z.x - z.y), stream);
             } else {
                 float2 X1, X2;
                 real_split(*p1, *p2, w, X1, X2);
-                Ho[k] = X1;
-                if (kind == 0) Ho[M - k] = X2;
+                st_hint(Ho + k, X1, stream);
+                if (kind == 0) st_hint(Ho + (M - k), X2, stream);
             }
         });
         return;
@@ -296,10 +327,10 @@ fourstep_row_kernel(FourStepArgs a)
         FS::for_each_pair(smem_fs, ublk, tid, [&](int kind, float2* p1, float2* p2, int k, float2 w) {
             float2 z1 = *p1, z2 = *p2;
             if (kind == 1) {                                    // slot 0 holds (bin 0, bin M), both real
-                const float2 h0 = __ldg(Hr);
+                const float2 h0 = ld_hint(Hr, stream);
                 spectral_pair<M>(z1, z2, make_float2(h0.x, 0.0f), make_float2(h0.y, 0.0f), w, bias);
             } else {
-                spectral_pair<M>(z1, z2, __ldg(Hr + k), __ldg(Hr + (M - k)), w, bias);
+                spectral_pair<M>(z1, z2, ld_hint(Hr + k, stream), ld_hint(Hr + (M - k), stream), w, bias);
             }
             *p1 = z1;
             if (kind == 0) *p2 = z2;
@@ -313,7 +344,7 @@ fourstep_row_kernel(FourStepArgs a)
         const float2 step = expi_pi<+1>(2.0f * (float)((k1 * (M2 / V2)) % M) / (float)M);
         static_for<V2>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            Sq[(size_t)k1 * M2 + t + r * (M2 / V2)] = cmul(reg[r], w);
+            st_hint(Sq + (size_t)k1 * M2 + t + r * (M2 / V2), cmul(reg[r], w), keep);
             if constexpr (r < V2 - 1) w = cmul(w, step);
         });
     }
@@ -349,38 +380,40 @@ fourstep_col_kernel(FourStepArgs a)
     const int n2 = c0 + c;
     float2* buf = smem_fs + c * FS::COL_STRIDE;
     float2 reg[V1];
+    // the wave scratch stays in L2 for the next launch; activations stream
+    const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
 
     if constexpr (MODE == 0) {
         const PT* vp = reinterpret_cast<const PT*>(a.v) + seq * SEQ;
         static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            reg[r] = IOP::load(vp + n2 + (size_t)M2 * (t + r * (M1 / V1)));
+            reg[r] = IOP::load_stream(vp + n2 + (size_t)M2 * (t + r * (M1 / V1)), stream);
         });
     } else {
-        const int pt = pad16(t);
-        static_for<V1>([&](auto rr) {
-            constexpr int r = decltype(rr)::value;
-            const int k1 = t + r * (M1 / V1);
-            buf[pad16_at<M1 / V1>(t, pt, r)] = Sq[(size_t)k1 * M2 + n2];
-        });
-        __syncthreads();
-        FS::F1::template run<+1, true>(buf, reg, t);
-        // crop (n1 = t + r M1/V1 < M1/2 <=> r < V1/2; circular: none) and gate
         const void* xn = a.x[0];
 #pragma unroll
         for (int i = 1; i < kMaxOrder; ++i)
             if (i == a.n) xn = a.x[i];
         const PT* xp = reinterpret_cast<const PT*>(xn) + seq * SEQ;
+        const int pt = pad16(t);
+        static_for<V1>([&](auto rr) {
+            constexpr int r = decltype(rr)::value;
+            const int k1 = t + r * (M1 / V1);
+            buf[pad16_at<M1 / V1>(t, pt, r)] = ld_hint_rw(Sq + (size_t)k1 * M2 + n2, keep);
+        });
+        __syncthreads();
+        FS::F1::template run<+1, true>(buf, reg, t);
+        // crop (n1 = t + r M1/V1 < M1/2 <=> r < V1/2; circular: none) and gate
         static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
-            const float2 xv = IOP::load(xp + n2 + (size_t)M2 * (t + r * (M1 / V1)));
+            const float2 xv = IOP::load_stream(xp + n2 + (size_t)M2 * (t + r * (M1 / V1)), stream);
             reg[r] = make_float2(reg[r].x * xv.x, reg[r].y * xv.y);
         });
         if constexpr (MODE == 2) {
             PT* yp = reinterpret_cast<PT*>(a.y) + seq * SEQ;
             static_for<VL>([&](auto rr) {
                 constexpr int r = decltype(rr)::value;
-                IOP::store(yp + n2 + (size_t)M2 * (t + r * (M1 / V1)), reg[r]);
+                IOP::store_stream(yp + n2 + (size_t)M2 * (t + r * (M1 / V1)), reg[r], stream);
             });
             return;
         }
@@ -400,7 +433,7 @@ fourstep_col_kernel(FourStepArgs a)
     const float2 step = expi_pi<-1>(2.0f * (float)((n2 * (M1 / V1)) % M) / (float)M);
     static_for<V1>([&](auto rr) {
         constexpr int r = decltype(rr)::value;
-        Sq[(size_t)(t + r * (M1 / V1)) * M2 + n2] = cmul(reg[r], w);
+        st_hint(Sq + (size_t)(t + r * (M1 / V1)) * M2 + n2, cmul(reg[r], w), keep);
         if constexpr (r < V1 - 1) w = cmul(w, step);
     });
 }

@@ -11,6 +11,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include <type_traits>
 #include <utility>
@@ -218,6 +219,75 @@ __device__ __forceinline__ void grid_dependency_begin()
     asm volatile("griddepcontrol.wait;\n" ::: "memory");
 }
 
+// ------------------------------------------------ L2 eviction priority
+//
+// Data that is read or written once (activations, spectra) streams through
+// L2 with evict-first priority; scratch that a following launch reads again
+// (the four-step wave scratch, the backward's saved spectra) is kept with
+// evict-last priority, so the streams do not push it out to HBM.
+__device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last()
+{
+    uint64_t p;
+    asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// read-only load / store of a float2 (or a bf16 pair) with an L2 policy
+__device__ __forceinline__ float2 ld_hint(const float2* p, uint64_t pol)
+{
+    float2 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;"
+                 : "=f"(v.x), "=f"(v.y) : "l"(p), "l"(pol));
+    return v;
+}
+__device__ __forceinline__ __nv_bfloat162 ld_hint(const __nv_bfloat162* p, uint64_t pol)
+{
+    uint32_t u;
+    asm volatile("ld.global.nc.L2::cache_hint.b32 %0, [%1], %2;" : "=r"(u) : "l"(p), "l"(pol));
+    __nv_bfloat162 v;
+    memcpy(&v, &u, 4);
+    return v;
+}
+// coherent load (the location may have been written earlier in this grid)
+__device__ __forceinline__ float2 ld_hint_rw(const float2* p, uint64_t pol)
+{
+    float2 v;
+    asm volatile("ld.global.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;"
+                 : "=f"(v.x), "=f"(v.y) : "l"(p), "l"(pol) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_hint(float2* p, float2 v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(v.x), "f"(v.y), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_hint(__nv_bfloat162* p, __nv_bfloat162 v, uint64_t pol)
+{
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(u), "l"(pol) : "memory");
+}
+// 16-byte asynchronous global -> shared copy with an L2 policy
+__device__ __forceinline__ void cp_async16_hint(void* smem_dst, const void* gmem_src, uint64_t pol)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem_src),
+                 "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_row_hint(void* smem_dst, const void* gmem_src, int bytes, int t,
+                                                  int nthreads, uint64_t pol)
+{
+    char* d = static_cast<char*>(smem_dst);
+    const char* s = static_cast<const char*>(gmem_src);
+    for (int i = t * 16; i < bytes; i += nthreads * 16) cp_async16_hint(d + i, s + i, pol);
+}
+
 // ---------------------------------------------------------------- I/O
 
 // Storage types of v, x_n and y.  Two consecutive real samples are moved
@@ -228,6 +298,9 @@ template <> struct IoPair<float> {
     static __device__ __forceinline__ float2 load_smem(const T* p) { return *p; }
     static __device__ __forceinline__ float2 load(const T* p) { return __ldg(p); }
     static __device__ __forceinline__ void store(T* p, float2 v) { *p = v; }
+    // the same, streamed with evict-first L2 priority
+    static __device__ __forceinline__ float2 load_stream(const T* p, uint64_t pol) { return ld_hint(p, pol); }
+    static __device__ __forceinline__ void store_stream(T* p, float2 v, uint64_t pol) { st_hint(p, v, pol); }
 };
 template <> struct IoPair<__nv_bfloat16> {
     using T = __nv_bfloat162;
@@ -239,6 +312,14 @@ template <> struct IoPair<__nv_bfloat16> {
     static __device__ __forceinline__ void store(T* p, float2 v)
     {
         *p = __floats2bfloat162_rn(v.x, v.y);  // round to nearest even
+    }
+    static __device__ __forceinline__ float2 load_stream(const T* p, uint64_t pol)
+    {
+        return __bfloat1622float2(ld_hint(p, pol));
+    }
+    static __device__ __forceinline__ void store_stream(T* p, float2 v, uint64_t pol)
+    {
+        st_hint(p, __floats2bfloat162_rn(v.x, v.y), pol);
     }
 };
 

@@ -1,4 +1,5 @@
 // Implicit filter generation launchers (1-D and 2-D).
+#include "filter_head_tc.cuh"
 #include "launch.cuh"
 
 namespace hyena {
@@ -35,8 +36,14 @@ hyena_status_t filter_gen_launches(const FilterGenArgs& a, long npos, int B, cud
     const int head_rows = a.rows - kFfnWidth;
     const unsigned rtiles = (unsigned)((head_rows + kFgRowTile - 1) / kFgRowTile);
     const unsigned ptiles2 = (unsigned)((npos + 127) / 128);
-    // 128-position tiles (8 x 8 outputs per thread) once they fill every SM twice
-    if (s == HYENA_OK && head_rows > 0)
+    if (s == HYENA_OK && head_rows > 0 && a.vec) {
+        // the tensor-core head: 256 rows per CTA, persistent over 128-position tiles
+        const unsigned rt = (unsigned)((head_rows + tch::kN - 1) / tch::kN);
+        const long per = (long)sms / ((long)rt * B);
+        const unsigned px = (unsigned)(ptiles2 < (per < 1 ? 1 : per) ? ptiles2 : (per < 1 ? 1 : per));
+        s = launch(filter_head_tc_kernel<TWO_D>, dim3(px, rt, B), tch::kThreads, tch::kSmem, st, a);
+    } else if (s == HYENA_OK && head_rows > 0)
+        // 128-position tiles (8 x 8 outputs per thread) once they fill every SM twice
         s = (long)ptiles2 * rtiles * B >= 2L * sms
                 ? launch(filter_head_kernel<TWO_D, 2>, dim3(ptiles2, rtiles, B), kFgThreads,
                          fg_head_smem_bytes<2>(), st, a)
@@ -58,3 +65,11 @@ hyena_status_t launch_filter_gen(const FilterGenArgs& a, bool two_d, long npos, 
 }
 
 }  // namespace hyena
+
+extern "C" int hyena_device_fault_count(void)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, hyena::g_tc_fault, sizeof(int)) != cudaSuccess) return -1;
+    const int w = hyena::dft_stage_fault_count();
+    return w < 0 ? -1 : v + w;
+}

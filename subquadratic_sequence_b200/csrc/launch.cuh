@@ -72,6 +72,8 @@ inline long wave_seqs(long nseq, long L)
     return nseq < per ? nseq : per;
 }
 
+// tensor-core waits of hyena_dft32_stage that timed out (-1: query failed)
+int dft_stage_fault_count();
 hyena_status_t dispatch_fused_f32(int log2m, const Fused1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_fused_bf16(int log2m, const Fused1dArgs& a, cudaStream_t st);
 hyena_status_t dispatch_fused_ps_f32(int log2m, const Fused1dArgs& a, cudaStream_t st);

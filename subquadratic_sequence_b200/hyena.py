@@ -65,6 +65,8 @@ def _load() -> ctypes.CDLL:
         "hyena_fftconv_gate_forward_noalloc": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp,
                                                 vp], i),
         "hyena_fftconv_spill_workspace_size": ([i, i, i, i], sz),
+        "hyena_device_fault_count": ([], i),
+        "hyena_dft32_stage": ([vp, vp, ctypes.c_long, i, i, vp], i),
         "hyena_fftconv_gate_forward_spill": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp, sz,
                                               vp], i),
         "hyena_fftconv_backward_workspace_size": ([i, i, i], sz),
@@ -321,6 +323,20 @@ def hyena_fftconv_gate_forward_spill(v: torch.Tensor, xs, bias: torch.Tensor, H:
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
         ctypes.c_void_p(_dev(bias, torch.float32, "bias")), B, D, L, N, io,
         ctypes.c_void_p(_dev(out, v.dtype, "y")), wp, wn, _stream(stream)))
+    return out
+
+
+def hyena_dft32_stage(x: torch.Tensor, reps: int, method: int, *, out=None, stream=None):
+    """x [count][32] complex64: each 32-point DFT (scaled by 1/sqrt(32))
+    applied reps times; method 0 on the FP32 pipes, 1 on the tensor cores."""
+    count = x.shape[0]
+    if tuple(x.shape) != (count, 32):
+        raise ValueError(f"x must be [count][32], got {tuple(x.shape)}")
+    if out is None:
+        out = torch.empty_like(x)
+    _check("hyena_dft32_stage", LIB.hyena_dft32_stage(
+        ctypes.c_void_p(_dev(x, torch.complex64, "x")), ctypes.c_void_p(_dev(out, torch.complex64, "y")),
+        count, reps, method, _stream(stream)))
     return out
 
 

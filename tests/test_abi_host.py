@@ -465,3 +465,14 @@ def test_spill_rejects_bad_arguments(lib):
     assert fwd_spill(lib, ws=P(5)) == INVALID             # workspace overlapping y
     assert fwd_spill(lib, ws=P(2)) == INVALID             # workspace overlapping x_2
     assert fwd_spill(lib, ws=P(3)) == INVALID             # workspace overlapping H
+
+
+def test_dft32_stage_rejects_bad_arguments(lib):
+    f = lib.hyena_dft32_stage
+    assert f(None, P(1), 4, 1, 0, None) == INVALID
+    assert f(P(0), P(1), 0, 1, 0, None) == INVALID
+    assert f(P(0), P(1), 4, 0, 0, None) == INVALID
+    assert f(P(0), P(1), 4, 1, 2, None) == INVALID
+    assert f(ctypes.c_void_p(A + 8), P(1), 4, 1, 0, None) == INVALID
+    assert f(P(0), P(0), 4, 1, 1, None) == INVALID                  # y overlapping x
+    assert f(P(0), P(1), (1 << 30) + 1, 1, 0, None) == UNSUPPORTED

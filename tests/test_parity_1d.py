@@ -56,15 +56,19 @@ def oracle_forward(inp, h, seqs=None, route="fft"):
 
 # ------------------------------------------------------------- filters
 
-# covers the single-launch path (N*D <= 64), the 64- and 128-position head
-# tiles, and lengths that are not a multiple of 4 (scalar h access)
+# covers the single-launch path (N*D <= 64), the tensor-core head (lengths
+# a multiple of 4: 256-row tiles, a last tile of 192 rows, and head rows
+# that are not a multiple of 16), and the SIMT head for lengths that are
+# not a multiple of 4 (scalar h access)
 @pytest.mark.parametrize("N,D,L", [(2, 64, 1024), (2, 768, 2048), (3, 5, 100), (1, 1, 1), (2, 3, 65536),
-                                   (3, 100, 5001), (2, 256, 65536), (2, 256, 65535)])
+                                   (3, 100, 5001), (2, 256, 65536), (2, 256, 65535), (3, 27, 1024),
+                                   (5, 77, 4096), (2, 40, 132)])
 def test_filter_gen_matches_oracle(hy, N, D, L):
     wl, inp = random_problem(1, D, L, N, seed=11 + L)
     got = host(gpu_filters(inp, wl))
     ref = oracle_filters(inp, wl)
     assert rel_max_err(got, ref) <= 2e-5
+    assert hy.LIB.hyena_device_fault_count() == 0
 
 
 @pytest.mark.parametrize("N,C,H,W", [(2, 4, 16, 32), (1, 3, 7, 5), (2, 128, 256, 256), (2, 128, 255, 257)])
