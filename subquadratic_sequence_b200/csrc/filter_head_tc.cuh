@@ -9,7 +9,7 @@
 // CTA keeps up to 256 rows of Wout in shared memory and walks tiles of 128
 // positions: the 128 x 64 tile of a3 (read from the stash rows of h) goes
 // to shared memory, one thread issues the MMAs (M = 128 positions, N = the
-// rows, K = 64 in steps of 8), and the eight warps read the 128 x N fp32
+// rows, K = 64 in steps of 8), and the sixteen warps read the 128 x N fp32
 // accumulator back from tensor memory, apply the window and store h.
 //
 // Float32 accuracy with TF32 products: each operand is split as
@@ -44,7 +44,7 @@ namespace tch {
 constexpr int kM = 128;                 // positions per tile
 constexpr int kN = 256;                 // rows per CTA, at most
 constexpr int kK = kFfnWidth;           // 64 units
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;             // 16 warps: four per accumulator lane group
 constexpr int kTmemCols = 512;        // two accumulators of 256 columns
 constexpr int kBBytes = kN * kK * 4;    // 64 KB per split half
 constexpr int kABytes = kM * kK * 4;    // 32 KB per split half
@@ -113,11 +113,11 @@ __global__ void __launch_bounds__(tch::kThreads, 1) filter_head_tc_kernel(Filter
     const long ntiles = (npos + kM - 1) / kM;
     uint32_t phase = 0;
 
-    // thread (chunk c = e / 128, position m = e % 128, e = tid + 256 i) holds
+    // thread (chunk c = e / 128, position m = e % 128, e = tid + 512 i) holds
     // units 4c..4c+3 of position p0 + m (a warp: 32 consecutive positions);
     // the next tile's values are loaded while this tile's MMAs and
     // epilogue run
-    constexpr int kPer = kM * (kK / 4) / kThreads;           // 8 chunks per thread
+    constexpr int kPer = kM * (kK / 4) / kThreads;           // 4 chunks per thread
     float4 nxt[kPer];
     auto load_tile = [&](long tile) {
         const long p0 = tile * kM;
@@ -193,29 +193,37 @@ __global__ void __launch_bounds__(tch::kThreads, 1) filter_head_tc_kernel(Filter
             load_tile(tile + 2L * gridDim.x);
         }
         fence_after();
-        // epilogue: warp w reads accumulator lanes 32 (w % 4) .. (positions),
-        // column chunks of 16 rows alternating between the two warp halves,
-        // four chunks per wait
+        // epilogue: warp w reads accumulator lanes 32 (w % 4) .. (positions)
+        // and column chunks of 16 rows c = w / 4, w / 4 + 4, ..., two chunks
+        // per wait; the row pointer advances by whole rows
         {
             const int lg = warp & 3;
             const long p = p0 + 32 * lg + lane;
             const float u = window_u<TWO_D>(a, p);
+            const bool inside = p < npos;
             const uint32_t base = tmem + 256 * (it & 1) + ((uint32_t)(32 * lg) << 16);
             for (int c0 = warp >> 2; c0 < N / 16; c0 += 8) {
-                uint32_t v[4][16];
+                uint32_t v[2][16];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    if (c0 + 2 * q < N / 16) tmem_ld16_issue(base + 16 * (c0 + 2 * q), v[q]);
+                for (int q = 0; q < 2; ++q)
+                    if (c0 + 4 * q < N / 16) tmem_ld16_issue(base + 16 * (c0 + 4 * q), v[q]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int c = c0 + 2 * q;
+                for (int q = 0; q < 2; ++q) {
+                    const int c = c0 + 4 * q;
                     if (c >= N / 16) break;
+                    const float4* cw = reinterpret_cast<const float4*>(sC + 16 * c);
+                    float* hp = a.h + (long)(r0 + 16 * c) * npos + p;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int n = 16 * c + j;
-                        if (n < nrows && p < npos)
-                            a.h[(long)(r0 + n) * npos + p] = __uint_as_float(v[q][j]) * exp2f(sC[n] * u);
+                    for (int j4 = 0; j4 < 4; ++j4) {
+                        const float4 k4 = cw[j4];
+                        const float kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const int j = 4 * j4 + jj;
+                            if (inside && 16 * c + j < nrows) *hp = __uint_as_float(v[q][j]) * exp2f(kk[jj] * u);
+                            hp += npos;
+                        }
                     }
                 }
             }

@@ -383,7 +383,25 @@ fourstep_col_kernel(FourStepArgs a)
     // the wave scratch stays in L2 for the next launch; activations stream
     const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
 
-    if constexpr (MODE == 0) {
+    // float32 activations: the first order's columns of v straight into the
+    // padded column buffers, two adjacent columns per 16-byte load
+    constexpr bool VEC0 = MODE == 0 && std::is_same<IO, float>::value;
+    if constexpr (VEC0) {
+        constexpr int ROWS0 = PAD ? M1 / 2 : M1;                 // rows n1 holding data
+        constexpr int RPP = FS::COL_THREADS / (TC / 2);
+        static_assert(ROWS0 % RPP == 0, "column passes");
+        const int cp = tid % (TC / 2), rr0 = tid / (TC / 2);
+        float2* b0 = smem_fs + (2 * cp) * FS::COL_STRIDE;
+        float2* b1 = b0 + FS::COL_STRIDE;
+        const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float2*>(a.v) + seq * SEQ + c0 + 2 * cp);
+        static_for<ROWS0 / RPP>([&](auto ii) {
+            constexpr int i = decltype(ii)::value;
+            const int n1 = rr0 + i * RPP;
+            const float4 v = ld_hint4(src + (size_t)n1 * (M2 / 2), stream);
+            b0[pad16(n1)] = make_float2(v.x, v.y);
+            b1[pad16(n1)] = make_float2(v.z, v.w);
+        });
+    } else if constexpr (MODE == 0) {
         const PT* vp = reinterpret_cast<const PT*>(a.v) + seq * SEQ;
         static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;
@@ -395,12 +413,25 @@ fourstep_col_kernel(FourStepArgs a)
         for (int i = 1; i < kMaxOrder; ++i)
             if (i == a.n) xn = a.x[i];
         const PT* xp = reinterpret_cast<const PT*>(xn) + seq * SEQ;
-        const int pt = pad16(t);
-        static_for<V1>([&](auto rr) {
-            constexpr int r = decltype(rr)::value;
-            const int k1 = t + r * (M1 / V1);
-            buf[pad16_at<M1 / V1>(t, pt, r)] = ld_hint_rw(Sq + (size_t)k1 * M2 + n2, keep);
-        });
+        // the CTA's TC columns of the scratch, two adjacent columns per
+        // 16-byte load (a warp: 4 rows x 128 bytes), scattered into the
+        // padded column buffers
+        static_assert(TC % 2 == 0 && FS::COL_THREADS % (TC / 2) == 0, "column pairs");
+        constexpr int RPP = FS::COL_THREADS / (TC / 2);           // rows per pass
+        static_assert(M1 % RPP == 0, "column passes");
+        {
+            const int cp = tid % (TC / 2), rr0 = tid / (TC / 2);
+            float2* b0 = smem_fs + (2 * cp) * FS::COL_STRIDE;
+            float2* b1 = b0 + FS::COL_STRIDE;
+            const float4* src = reinterpret_cast<const float4*>(Sq + c0 + 2 * cp);
+            static_for<M1 / RPP>([&](auto ii) {
+                constexpr int i = decltype(ii)::value;
+                const int k1 = rr0 + i * RPP;
+                const float4 v = ld_hint_rw4(src + (size_t)k1 * (M2 / 2), keep);
+                b0[pad16(k1)] = make_float2(v.x, v.y);
+                b1[pad16(k1)] = make_float2(v.z, v.w);
+            });
+        }
         __syncthreads();
         FS::F1::template run<+1, true>(buf, reg, t);
         // crop (n1 = t + r M1/V1 < M1/2 <=> r < V1/2; circular: none) and gate
@@ -420,7 +451,7 @@ fourstep_col_kernel(FourStepArgs a)
     }
     // forward column FFT of z (n1 < M1/2, zero-padded; circular: all n1),
     // then the four-step twiddle exp(-2 pi i n2 k1 / M)
-    {
+    if constexpr (!VEC0) {
         const int pt = pad16(t);
         static_for<VL>([&](auto rr) {
             constexpr int r = decltype(rr)::value;

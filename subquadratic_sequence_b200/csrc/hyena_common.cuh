@@ -261,6 +261,23 @@ __device__ __forceinline__ float2 ld_hint_rw(const float2* p, uint64_t pol)
                  : "=f"(v.x), "=f"(v.y) : "l"(p), "l"(pol) : "memory");
     return v;
 }
+__device__ __forceinline__ float4 ld_hint4(const float4* p, uint64_t pol)
+{
+    float4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+__device__ __forceinline__ float4 ld_hint_rw4(const float4* p, uint64_t pol)
+{
+    float4 v;
+    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(pol)
+                 : "memory");
+    return v;
+}
 __device__ __forceinline__ void st_hint(float2* p, float2 v, uint64_t pol)
 {
     asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(v.x), "f"(v.y), "l"(pol)
