@@ -705,6 +705,100 @@ HYENA_API hyena_status_t hyena_fftconv2d_gate_backward_circular(const void* v, c
                                                                 void* const* dx, float* dh, float* dbias,
                                                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* The backward of the circular 2-D recurrence with a spectrum set per
+ * sample (input-dependent filters, hyena_fftconv2d_gate_forward_circular_
+ * per_sample): per sample the circular adjoint above with that sample's
+ * filters, so dh is per sample and only the shared bias's gradient is
+ * summed over the batch:
+ *   dh_{b,n}[c][a][b'] = sum_{t,s} e_b[t][s] z_{b,n-1}[(t - a) mod H][(s - b') mod W],
+ *   db_n[c] = sum_b dh_{b,n}[c][0][0].
+ * Arguments as hyena_fftconv2d_gate_backward_circular with Hs
+ * [B][N][C][H][W/2] (hyena_filter_rfft2d_circular of each sample's
+ * filters), dh [B][N][C][H][W] and a workspace of
+ * hyena_fftconv2d_backward_circular_per_sample_workspace_size(...) bytes
+ * (B times the dh spectra of the shared backward), 256-byte aligned.
+ * Deterministic: one more launch sums dbias over the samples in order. */
+HYENA_API size_t hyena_fftconv2d_backward_circular_per_sample_workspace_size(int B, int C, int H, int W, int N);
+HYENA_API hyena_status_t hyena_fftconv2d_gate_backward_circular_per_sample(
+    const void* v, const void* const* x, const float* Hs, const float* bias, const void* dy, int B, int C,
+    int H, int W, int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
+    void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------- 3-D backward */
+
+/* Bytes of workspace hyena_fftconv3d_gate_backward needs: the accumulated
+ * dh spectra [N][C][2Z][2H][W] complex64, and per wave of volumes the
+ * saved spectra of z_n (N x 2Z x 2H x W complex), the saved c_n (N x Z x H
+ * x W float32) and the scratch (Z x 2H x W complex); (size_t)-1 for
+ * invalid sizes. */
+HYENA_API size_t hyena_fftconv3d_backward_workspace_size(int B, int C, int Z, int H, int W, int N);
+
+/* Gradients of a scalar loss through the 3-D recurrence of
+ * hyena_fftconv3d_gate_forward, given dy = dL/dy [B][C][Z][H][W] (the chain
+ * rule; the pages give no training formulas):
+ *   dv [B][C][Z][H][W] io, dx = HOST array of N device pointers
+ *   [B][C][Z][H][W] io, dh [N][C][Z][H][W] float32 (dL/dh_n, summed over
+ *   the batch), dbias [N][C] float32 (= dh_n[0][0][0]).
+ * Inputs as the forward with the spectra Hs [N][C][2Z][2H][W] given
+ * (hyena_filter_rfft3d).  Z, H, W powers of two in [16, 256].  Alignment:
+ * activations, Hs, dh 16 bytes; bias, dbias 4; workspace 256.  Outputs
+ * must not overlap any input, each other or the workspace.  Per wave of
+ * volumes: the forward again, saving the 3-D spectra Z_n and c_n; then per
+ * order in reverse, the rows (dx_n, e = g x_n, forward rows of e), the
+ * forward columns, the z step (dh spectrum += E conj(Z_n); g from
+ * (conj(H_n) + b_n) E) and the inverse columns; finally dh and db from the
+ * accumulated spectra.  Deterministic (no atomics). */
+HYENA_API hyena_status_t hyena_fftconv3d_gate_backward(const void* v, const void* const* x, const float* Hs,
+                                                       const float* bias, const void* dy, int B, int C, int Z,
+                                                       int H, int W, int N, hyena_dtype_t io, void* dv,
+                                                       void* const* dx, float* dh, float* dbias,
+                                                       void* workspace, size_t ws_bytes, void* stream);
+
+/* The 3-D backward with a spectrum set per sample (input-dependent filters,
+ * hyena_fftconv3d_gate_forward_per_sample): volume (b, c) uses sample b's
+ * filters, so
+ *   Hs     [B][N][C][2Z][2H][W] (sample b's set at Hs + b*N*C*2Z*2H*W)
+ *   dh     [B][N][C][Z][H][W] float32 out, per sample
+ *   dbias  [N][C] float32 out, summed over the batch (the bias is shared)
+ *   workspace: hyena_fftconv3d_backward_per_sample_workspace_size(...)
+ *          bytes (B times the dh spectra of the shared backward).
+ * Everything else as hyena_fftconv3d_gate_backward; deterministic, one
+ * more launch sums dbias over the samples in order. */
+HYENA_API size_t hyena_fftconv3d_backward_per_sample_workspace_size(int B, int C, int Z, int H, int W, int N);
+HYENA_API hyena_status_t hyena_fftconv3d_gate_backward_per_sample(
+    const void* v, const void* const* x, const float* Hs, const float* bias, const void* dy, int B, int C,
+    int Z, int H, int W, int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
+    void* workspace, size_t ws_bytes, void* stream);
+
+/* The backward of the circular 3-D recurrence (hyena_fftconv3d_gate_forward_
+ * circular): the exact adjoint with every 3-D convolution circular on the
+ * Z x H x W grid, so both correlations wrap around:
+ *   dh_n[c][a][p][q] = sum_b sum_{t,s,u} e[t][s][u] z_{n-1}[(t-a) mod Z][(s-p) mod H][(u-q) mod W],
+ *   db_n[c] = dh_n[c][0][0][0],
+ *   dz_{n-1} = the same correlation of e with h_n, plus b_n e.
+ * Arguments as hyena_fftconv3d_gate_backward with Hs [N][C][Z][H][W/2]
+ * from hyena_filter_rfft3d_circular, dh [N][C][Z][H][W] and dbias [N][C]
+ * summed over the batch, and a workspace of
+ * hyena_fftconv3d_backward_circular_workspace_size(...) bytes, 256-byte
+ * aligned.  Z, H powers of two in [16, 256], W in [32, 256]. */
+HYENA_API size_t hyena_fftconv3d_backward_circular_workspace_size(int B, int C, int Z, int H, int W, int N);
+HYENA_API hyena_status_t hyena_fftconv3d_gate_backward_circular(
+    const void* v, const void* const* x, const float* Hs, const float* bias, const void* dy, int B, int C,
+    int Z, int H, int W, int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
+    void* workspace, size_t ws_bytes, void* stream);
+
+/* The circular 3-D backward with a spectrum set per sample: Hs
+ * [B][N][C][Z][H][W/2], dh [B][N][C][Z][H][W] per sample, dbias [N][C]
+ * summed over the batch, workspace
+ * hyena_fftconv3d_backward_circular_per_sample_workspace_size(...) bytes;
+ * otherwise as hyena_fftconv3d_gate_backward_circular. */
+HYENA_API size_t hyena_fftconv3d_backward_circular_per_sample_workspace_size(int B, int C, int Z, int H, int W,
+                                                                            int N);
+HYENA_API hyena_status_t hyena_fftconv3d_gate_backward_circular_per_sample(
+    const void* v, const void* const* x, const float* Hs, const float* bias, const void* dy, int B, int C,
+    int Z, int H, int W, int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh, float* dbias,
+    void* workspace, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -70,6 +70,7 @@ def _load():
         "oracle_cconv3": [dp, dp, l, l, l, i, dp],
         "oracle_filter_gen_3d": [dp, dp, dp, dp, dp, i, i, i, i, i, i, i, d, i, dp],
         "oracle_hyena_backward_3d": [dp, dp, dp, dp, dp, l, l, l, l, l, l, i, dp, dp, dp, dp],
+        "oracle_hyena_backward_circular_3d": [dp, dp, dp, dp, dp, l, l, l, l, l, l, i, dp, dp, dp, dp],
         "oracle_hyena_backward_circular_2d": [dp, dp, dp, dp, dp, l, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_hyena_backward_circular": [dp, dp, dp, dp, dp, l, l, l, l, i, i, dp, dp, dp, dp],
         "oracle_filter_gen_film_3d": [dp, dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i, i, i, i, d, i, dp],
@@ -449,6 +450,23 @@ def hyena_backward_3d(v, x, h, bias, dy, route="fft"):
     rc = _load().oracle_hyena_backward_3d(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), _ptr(dy), B, C, Z, H, W, N,
                                           _route(route), _ptr(dv), _ptr(dx), _ptr(dh), _ptr(db))
     _check(rc, "oracle_hyena_backward_3d")
+    return dv, dx, dh, db
+
+
+def hyena_backward_circular_3d(v, x, h, bias, dy, route="fft"):
+    """Gradients through the 3-D recurrence with circular convolutions on
+    the Z x H x W grid (:func:`hyena_forward_circular_nd` on volumes): (dv,
+    dx, dh [N][C][Z][H][W], dbias [N][C]), dh and dbias summed over the
+    batch."""
+    v, x, h, bias, dy = map(_f64, (v, x, h, bias, dy))
+    B, C, Z, H, W = v.shape
+    N = h.shape[0]
+    assert x.shape == (N, B, C, Z, H, W) and h.shape == (N, C, Z, H, W) and bias.shape == (N, C)
+    assert dy.shape == v.shape
+    dv, dx, dh, db = np.empty_like(v), np.empty_like(x), np.empty_like(h), np.empty_like(bias)
+    rc = _load().oracle_hyena_backward_circular_3d(_ptr(v), _ptr(x), _ptr(h), _ptr(bias), _ptr(dy), B, C, Z, H,
+                                                   W, N, _route(route), _ptr(dv), _ptr(dx), _ptr(dh), _ptr(db))
+    _check(rc, "oracle_hyena_backward_circular_3d")
     return dv, dx, dh, db
 
 

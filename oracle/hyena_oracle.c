@@ -1492,6 +1492,115 @@ int oracle_hyena_forward_circular_nd(const double *v, const double *x, const dou
 }
 
 /* ------------------------------------------------------------------ */
+/* Backward of the circular 3-D recurrence (oracle_hyena_forward_       */
+/* circular_nd): the chain rule with both sums wrapping around.         */
+/* ------------------------------------------------------------------ */
+
+/* out[a][b][c] = sum_{t,s,u} p[t][s][u] q[(t-a) mod Z][(s-b) mod H][(u-c)
+ * mod W].  With p = e, q = z it is dh; with p = e, q = h the adjoint of the
+ * circular 3-D convolution with respect to its signal.  The definition. */
+static void ccorr3_direct(const double *p, const double *q, long Z, long H, long W, double *out)
+{
+    for (long a = 0; a < Z; ++a)
+        for (long b = 0; b < H; ++b)
+            for (long c = 0; c < W; ++c) {
+                double acc = 0.0;
+                for (long t = 0; t < Z; ++t)
+                    for (long s = 0; s < H; ++s)
+                        for (long u = 0; u < W; ++u)
+                            acc += p[(t * H + s) * W + u] *
+                                   q[(((t - a + Z) % Z) * H + (s - b + H) % H) * W + (u - c + W) % W];
+                out[(a * H + b) * W + c] = acc;
+            }
+}
+
+/* The same through the DFT on the Z x H x W grid itself (powers of two, no
+ * padding, so the product wraps): IDFT(P conj(Q)) / (Z H W). */
+static int ccorr3_fft(const double *p, const double *q, long Z, long H, long W, double *out)
+{
+    const long P = Z * H * W;
+    double *pr = malloc(sizeof(double) * P), *pi = calloc(P, sizeof(double));
+    double *qr = malloc(sizeof(double) * P), *qi = calloc(P, sizeof(double));
+    int st = ORACLE_ENOMEM;
+    if (!pr || !pi || !qr || !qi) goto out;
+    memcpy(pr, p, sizeof(double) * P);
+    memcpy(qr, q, sizeof(double) * P);
+    if ((st = fft3(pr, pi, Z, H, W, -1)) != ORACLE_OK) goto out;
+    if ((st = fft3(qr, qi, Z, H, W, -1)) != ORACLE_OK) goto out;
+    for (long k = 0; k < P; ++k) {
+        const double re = pr[k] * qr[k] + pi[k] * qi[k], im = pi[k] * qr[k] - pr[k] * qi[k];
+        pr[k] = re;
+        pi[k] = im;
+    }
+    if ((st = fft3(pr, pi, Z, H, W, +1)) != ORACLE_OK) goto out;
+    for (long k = 0; k < P; ++k) out[k] = pr[k] / (double)P;
+out:
+    free(pr); free(pi); free(qr); free(qi);
+    return st;
+}
+
+/* Gradients of a scalar loss with dL/dy = dy [B][C][Z][H][W] through the
+ * circular 3-D recurrence: dv, dx [N][B][C][Z][H][W], dh [N][C][Z][H][W]
+ * and dbias [N][C] (both summed over the batch).  With c_n = h_n (*) z_{n-1}
+ * + b_n z_{n-1} (circular), z_n = x_n c_n and g = dL/dz_n: dx_n = g c_n,
+ * e = g x_n, dh_n += ccorr3(e, z_{n-1}), db_n += sum e z_{n-1},
+ * dz_{n-1} = ccorr3(e, h_n) + b_n e.  One thread. */
+int oracle_hyena_backward_circular_3d(const double *v, const double *x, const double *h,
+                                      const double *bias, const double *dy, long B, long C, long Z, long H,
+                                      long W, long N, int route, double *dv, double *dx, double *dh,
+                                      double *dbias)
+{
+    if (!v || !x || !h || !bias || !dy || !dv || !dx || !dh || !dbias || B < 1 || C < 1 || Z < 1 || H < 1 ||
+        W < 1 || N < 1 || (route != ROUTE_DIRECT && route != ROUTE_FFT))
+        return ORACLE_EBADARG;
+    if (route == ROUTE_FFT && (!is_pow2(Z) || !is_pow2(H) || !is_pow2(W))) return ORACLE_EBADARG;
+    const long V = Z * H * W, BCV = B * C * V;
+    double *z = malloc(sizeof(double) * N * V), *c = malloc(sizeof(double) * N * V);
+    double *g = malloc(sizeof(double) * V), *e = malloc(sizeof(double) * V), *tmp = malloc(sizeof(double) * V);
+    int st = ORACLE_OK;
+    if (!z || !c || !g || !e || !tmp) { st = ORACLE_ENOMEM; goto done; }
+    memset(dh, 0, sizeof(double) * N * C * V);
+    memset(dbias, 0, sizeof(double) * N * C);
+    for (long img = 0; img < B * C && st == ORACLE_OK; ++img) {
+        const long ch = img % C;
+        memcpy(z, v + img * V, sizeof(double) * V);              /* z_0 = v */
+        for (long n = 0; n < N && st == ORACLE_OK; ++n) {
+            const double *hn = h + (n * C + ch) * V, *xn = x + n * BCV + img * V;
+            const double bn = bias[n * C + ch];
+            double *zn = z + n * V, *cn = c + n * V;
+            st = oracle_cconv3(hn, zn, Z, H, W, route, cn);
+            for (long t = 0; t < V; ++t) cn[t] += bn * zn[t];
+            if (n + 1 < N)
+                for (long t = 0; t < V; ++t) z[(n + 1) * V + t] = xn[t] * cn[t];
+        }
+        memcpy(g, dy + img * V, sizeof(double) * V);
+        for (long n = N - 1; n >= 0 && st == ORACLE_OK; --n) {
+            const double *hn = h + (n * C + ch) * V, *xn = x + n * BCV + img * V;
+            const double bn = bias[n * C + ch];
+            const double *zn = z + n * V, *cn = c + n * V;
+            double *dxn = dx + n * BCV + img * V, *dhn = dh + (n * C + ch) * V;
+            for (long t = 0; t < V; ++t) {
+                dxn[t] = g[t] * cn[t];
+                e[t] = g[t] * xn[t];
+            }
+            if (route == ROUTE_DIRECT) ccorr3_direct(e, zn, Z, H, W, tmp);
+            else st = ccorr3_fft(e, zn, Z, H, W, tmp);
+            for (long t = 0; t < V; ++t) dhn[t] += tmp[t];
+            double db = 0.0;
+            for (long t = 0; t < V; ++t) db += e[t] * zn[t];
+            dbias[n * C + ch] += db;
+            if (route == ROUTE_DIRECT) ccorr3_direct(e, hn, Z, H, W, tmp);
+            else if (st == ORACLE_OK) st = ccorr3_fft(e, hn, Z, H, W, tmp);
+            for (long t = 0; t < V; ++t) g[t] = tmp[t] + bn * e[t];
+        }
+        memcpy(dv + img * V, g, sizeof(double) * V);             /* dv = dz_0 */
+    }
+done:
+    free(z); free(c); free(g); free(e); free(tmp);
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
 /* Backward of the 2-D recurrence (the chain rule, as in 1-D, with the  */
 /* 2-D linear convolution of Native ND Convolution / Handling           */
 /* Boundaries):                                                         */

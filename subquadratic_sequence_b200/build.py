@@ -34,10 +34,16 @@ def _deps() -> list[str]:
 
 
 def up_to_date() -> bool:
+    """The library exists, is newer than every source, header and object, and
+    no object is stale (an object is dated by when its compile began, so a
+    source edited during a build leaves its object stale even though the
+    library was linked later)."""
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _deps())
+    if not all(os.path.getmtime(p) <= t for p in _deps()):
+        return False
+    return not any(_obj_stale(s) for s in sources())
 
 
 OBJDIR = os.path.join(PKG, "lib", "_obj")

@@ -214,10 +214,10 @@ struct Fft2dCols {
 // spectral multiply with the packed 2-D filter spectrum and the bias,
 // inverse column FFTs, rows y < H back to the scratch.  MODE 1: forward
 // column FFTs of each plane (the packed spectra, or 3-D scratch planes),
-// all H2 rows written back; with zp and PAD, plane q of the filter spectra
-// is plane q % zp of filter q / zp at a pitch of 2 zp planes.  MODE 2
-// (3-D): inverse column FFTs of all H2 rows of each plane, rows y < H
-// written back.
+// all H2 rows written back.  MODE 2 (3-D): inverse column FFTs of all H2
+// rows of each plane, rows y < H written back.  In both, with zp and PAD,
+// plane q is plane q % zp of spectrum q / zp at a pitch of 2 zp planes
+// (the filter spectra, the backward's accumulated spectra).
 template <int LOG2H2, int MODE, bool PAD = true>
 __global__ void __launch_bounds__(Fft2dCols<LOG2H2, PAD>::THREADS, Fft2dCols<LOG2H2, PAD>::MIN_BLOCKS)
 fft2d_col_kernel(Fft2dArgs a)
@@ -241,7 +241,7 @@ fft2d_col_kernel(Fft2dArgs a)
     const int kx = kx0 + cc;
     float2* buf = smem_c2 + cc * CL::STRIDE;
     // rows of this image's column kx: scratch [H][W] or planes [2H][W]
-    const size_t pq = (MODE == 1 && a.zp && PAD) ? (size_t)(q / a.zp) * 2 * a.zp + q % a.zp : (size_t)q;
+    const size_t pq = (MODE != 0 && a.zp && PAD) ? (size_t)(q / a.zp) * 2 * a.zp + q % a.zp : (size_t)q;
     float2* col = MODE != 0 ? a.S + pq * H2 * W + kx : a.S + (size_t)qi * ROWS * W + kx;
     float2 reg[V];
     const int pt = pad16(t);

@@ -72,6 +72,7 @@ __device__ __forceinline__ T pick_order(T const* arr, int n)
 // the inverse rows of the scratch; dx_n = g c_n; e = g x_n; forward rows of
 // e.  MODE 2: dv = inverse rows of the scratch.  MODE 3: dh rows from the
 // accumulated spectra (rows y < H after the inverse columns), db = dh[0][0].
+// 3-D volumes (f.zp != 0) are Z planes of Hp rows: f.H = Z Hp rows a volume.
 template <int LOG2W, typename IO, int MODE, bool PAD = true>
 __global__ void __launch_bounds__(Fft1d<LOG2W, PAD>::THREADS)
 fft2d_bwd_row_kernel(Bwd2dArgs ba)
@@ -96,8 +97,16 @@ fft2d_bwd_row_kernel(Bwd2dArgs ba)
     float2 arr[E];
 
     if constexpr (MODE == 3) {
-        // q: filter row n*C + c of the accumulated spectra [2H][W]
-        const float2* row = ba.acc + ((size_t)q * (PAD ? 2 : 1) * a.H + yrow) * W;
+        // q: filter row n*C + c of the accumulated spectra [2H][W] (3-D:
+        // row y of plane z of [2Z][2H][W], yrow = z Hp + y)
+        constexpr int RP = PAD ? 2 : 1;
+        const float2* row;
+        if (a.zp == 0) {
+            row = ba.acc + ((size_t)q * RP * a.H + yrow) * W;
+        } else {
+            const int z = yrow / a.Hp, y = yrow - z * a.Hp;
+            row = ba.acc + (((size_t)q * RP * a.zp + z) * RP * a.Hp + y) * W;
+        }
         R::unsplit_inverse(arr, sm, row, t);
         if (active) {
             float2* dhp = reinterpret_cast<float2*>(ba.dh + ((size_t)q * a.H + yrow) * 2 * SEQ);
@@ -310,14 +319,16 @@ fft2d_bwd_col_kernel(Bwd2dArgs ba)
 }
 
 // Per-sample spectra: db_n[c] = sum_b dh_{b,n}[c][0][0], one thread per
-// (n, c), the samples in order (deterministic).
-static __global__ void __launch_bounds__(256) db2d_sum_kernel(Bwd2dArgs ba)
+// (n, c), the samples in order (deterministic).  A grid of f.H rows holds
+// f.W reals a row (PAD: one real per slot) or 2 f.W (circular: two).
+template <bool PAD>
+__global__ void __launch_bounds__(256) db2d_sum_kernel(Bwd2dArgs ba)
 {
     grid_dependency_begin();
     const int rows = ba.N * ba.f.C;
     const int r = blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= rows) return;
-    const size_t plane = (size_t)ba.f.H * ba.f.W;
+    const size_t plane = (size_t)ba.f.H * (PAD ? 1 : 2) * ba.f.W;
     float s = 0.0f;
     for (int b = 0; b < ba.f.B; ++b) s += ba.dh[((size_t)b * rows + r) * plane];
     ba.dbias[r] = s;

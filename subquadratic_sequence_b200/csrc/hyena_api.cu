@@ -8,6 +8,7 @@
 #include "k_fourstep.cuh"
 #include "k_fourstep_bwd.cuh"
 #include "k_fft3d.cuh"
+#include "k_fft3d_bwd.cuh"
 #include "launch.cuh"
 
 using namespace hyena;
@@ -1251,6 +1252,24 @@ size_t hyena_fftconv2d_backward_circular_workspace_size(int B, int C, int H, int
     return bwd2d_layout(B, C, H, W, N, 1, true).total;
 }
 
+size_t hyena_fftconv2d_backward_circular_per_sample_workspace_size(int B, int C, int H, int W, int N)
+{
+    int lh, lm;
+    if (B < 1 || C < 1 || N < 1 || N > HYENA_MAX_ORDER || !dims2d_circ_ok(H, W, lh, lm)) return (size_t)-1;
+    return bwd2d_layout(B, C, H, W, N, B, true).total;
+}
+
+hyena_status_t hyena_fftconv2d_gate_backward_circular_per_sample(const void* v, const void* const* x,
+                                                                 const float* Hs, const float* bias,
+                                                                 const void* dy, int B, int C, int H, int W,
+                                                                 int N, hyena_dtype_t io, void* dv,
+                                                                 void* const* dx, float* dh, float* dbias,
+                                                                 void* workspace, size_t ws_bytes, void* stream)
+{
+    return backward2d_impl(v, x, Hs, true, true, bias, dy, B, C, H, W, N, io, dv, dx, dh, dbias, workspace,
+                           ws_bytes, stream);
+}
+
 hyena_status_t hyena_fftconv2d_gate_backward_circular(const void* v, const void* const* x, const float* Hs,
                                                       const float* bias, const void* dy, int B, int C, int H,
                                                       int W, int N, hyena_dtype_t io, void* dv, void* const* dx,
@@ -1357,3 +1376,182 @@ hyena_status_t backward2d_impl(const void* v, const void* const* x, const float*
 }
 
 }  // namespace
+
+// ------------------------------------------------------- 3-D backward
+
+namespace {
+
+// sets: dh spectra per (n, c) (B with per-sample spectra, else 1);
+// circular: Z x H x W/2 spectrum slots a volume, else 2Z x 2H x W
+Bwd2dLayout bwd3d_layout(int B, int C, int Z, int H, int W, int N, int sets, bool circular)
+{
+    Bwd2dLayout l;
+    const int Ws = circular ? W / 2 : W;
+    const int RP = circular ? 1 : 2;
+    l.wcap = wave_images_3d((long)B * C, Z, H, Ws, !circular);
+    const size_t slots = (size_t)RP * Z * RP * H * Ws;
+    l.acc = 0;
+    l.zsave = l.acc + round_up(sizeof(float2) * (size_t)sets * N * C * slots, 256);
+    l.csave = l.zsave + round_up(sizeof(float2) * (size_t)N * l.wcap * slots, 256);
+    l.scratch = l.csave + round_up(sizeof(float) * (size_t)N * l.wcap * Z * H * W, 256);
+    l.total = l.scratch + round_up(sizeof(float2) * (size_t)l.wcap * Z * RP * H * Ws, 256);
+    return l;
+}
+
+bool dims3d_bwd_ok(bool circular, int Z, int H, int W, int& lz, int& lh, int& lm)
+{
+    if (circular) return dims3d_circ_ok(Z, H, W, lz, lh, lm);
+    return dims3d_ok(Z, H, W, lz, lh, lm);
+}
+
+size_t bwd3d_workspace(bool circular, int sets, int B, int C, int Z, int H, int W, int N)
+{
+    int lz, lh, lm;
+    if (B < 1 || C < 1 || N < 1 || N > HYENA_MAX_ORDER || !dims3d_bwd_ok(circular, Z, H, W, lz, lh, lm))
+        return (size_t)-1;
+    return bwd3d_layout(B, C, Z, H, W, N, sets, circular).total;
+}
+
+hyena_status_t backward3d_impl(const void* v, const void* const* x, const float* Hs, bool per_sample,
+                               bool circular, const float* bias, const void* dy, int B, int C, int Z, int H,
+                               int W, int N, hyena_dtype_t io, void* dv, void* const* dx, float* dh,
+                               float* dbias, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!v || !x || !Hs || !bias || !dy || !dv || !dx || !dh || !dbias) return HYENA_ERR_INVALID_ARG;
+    if (B < 1 || C < 1 || N < 1 || Z < 1 || H < 1 || W < 1) return HYENA_ERR_INVALID_ARG;
+    if (io != HYENA_F32 && io != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+    if (N > HYENA_MAX_ORDER) return HYENA_ERR_UNSUPPORTED;
+    int lz, lh, lm;
+    if (!dims3d_bwd_ok(circular, Z, H, W, lz, lh, lm)) return HYENA_ERR_UNSUPPORTED;
+    const int sets = per_sample ? B : 1;
+    const int Ws = circular ? W / 2 : W;                     // spectrum slots per row
+    const int RP = circular ? 1 : 2;                         // spectrum planes (rows) per grid plane (row)
+    if ((long)B * C > (1L << 20) || (long)sets * N * C * Z * H > (1L << 30)) return HYENA_ERR_UNSUPPORTED;
+    for (int n = 0; n < N; ++n)
+        if (!x[n] || !dx[n] || !aligned(x[n], 16) || !aligned(dx[n], 16)) return HYENA_ERR_INVALID_ARG;
+    if (!aligned(v, 16) || !aligned(dy, 16) || !aligned(dv, 16) || !aligned(Hs, 16) || !aligned(dh, 16) ||
+        !aligned(bias, 4) || !aligned(dbias, 4))
+        return HYENA_ERR_INVALID_ARG;
+    const Bwd2dLayout lay = bwd3d_layout(B, C, Z, H, W, N, sets, circular);
+    if (!workspace || ws_bytes < lay.total || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
+
+    // every output against every input, the other outputs and the workspace
+    const size_t vol = (size_t)Z * H * W;
+    const size_t spec_vol = (size_t)RP * Z * RP * H * Ws;    // spectrum slots a volume
+    const size_t act = (size_t)B * C * vol * io_bytes(io);
+    struct Range { const void* p; size_t n; };
+    Range in[kMaxOrder + 5], out[kMaxOrder + 3];
+    int ni = 0, no = 0;
+    in[ni++] = {v, act};
+    in[ni++] = {dy, act};
+    in[ni++] = {Hs, sizeof(float2) * (size_t)sets * N * C * spec_vol};
+    in[ni++] = {bias, sizeof(float) * N * C};
+    in[ni++] = {workspace, lay.total};
+    for (int n = 0; n < N; ++n) in[ni++] = {x[n], act};
+    out[no++] = {dv, act};
+    out[no++] = {dh, sizeof(float) * (size_t)sets * N * C * vol};
+    out[no++] = {dbias, sizeof(float) * N * C};
+    for (int n = 0; n < N; ++n) out[no++] = {dx[n], act};
+    for (int o = 0; o < no; ++o) {
+        for (int i = 0; i < ni; ++i)
+            if (overlap(out[o].p, out[o].n, in[i].p, in[i].n)) return HYENA_ERR_INVALID_ARG;
+        for (int p = o + 1; p < no; ++p)
+            if (overlap(out[o].p, out[o].n, out[p].p, out[p].n)) return HYENA_ERR_INVALID_ARG;
+    }
+
+    char* ws = static_cast<char*>(workspace);
+    Bwd2dArgs a = {};
+    a.f.Hs_bstride = per_sample ? (size_t)N * C * spec_vol : 0;
+    a.f.v = v;
+    for (int n = 0; n < kMaxOrder; ++n) {
+        a.f.x[n] = n < N ? x[n] : nullptr;
+        a.dx[n] = n < N ? dx[n] : nullptr;
+    }
+    a.f.Hs = reinterpret_cast<const float2*>(Hs);
+    a.f.bias = bias;
+    a.f.S = reinterpret_cast<float2*>(ws + lay.scratch);
+    a.f.B = B;
+    a.f.C = C;
+    a.f.H = Z * H;
+    a.f.W = Ws;
+    a.f.zp = Z;
+    a.f.Hp = H;
+    a.dy = dy;
+    a.dv = dv;
+    a.acc = reinterpret_cast<float2*>(ws + lay.acc);
+    a.zsave = reinterpret_cast<float2*>(ws + lay.zsave);
+    a.csave = reinterpret_cast<float*>(ws + lay.csave);
+    a.dh = dh;
+    a.dbias = dbias;
+    a.wcap = (int)lay.wcap;
+    cudaStream_t st = (cudaStream_t)stream;
+    return io == HYENA_BF16 ? dispatch_bwd3d_bf16(lm, lh, lz, a, N, st, !circular)
+                            : dispatch_bwd3d_f32(lm, lh, lz, a, N, st, !circular);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hyena_fftconv3d_backward_workspace_size(int B, int C, int Z, int H, int W, int N)
+{
+    return bwd3d_workspace(false, 1, B, C, Z, H, W, N);
+}
+
+size_t hyena_fftconv3d_backward_per_sample_workspace_size(int B, int C, int Z, int H, int W, int N)
+{
+    return bwd3d_workspace(false, B, B, C, Z, H, W, N);
+}
+
+hyena_status_t hyena_fftconv3d_gate_backward(const void* v, const void* const* x, const float* Hs,
+                                             const float* bias, const void* dy, int B, int C, int Z, int H,
+                                             int W, int N, hyena_dtype_t io, void* dv, void* const* dx,
+                                             float* dh, float* dbias, void* workspace, size_t ws_bytes,
+                                             void* stream)
+{
+    return backward3d_impl(v, x, Hs, false, false, bias, dy, B, C, Z, H, W, N, io, dv, dx, dh, dbias, workspace,
+                           ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv3d_gate_backward_per_sample(const void* v, const void* const* x, const float* Hs,
+                                                        const float* bias, const void* dy, int B, int C, int Z,
+                                                        int H, int W, int N, hyena_dtype_t io, void* dv,
+                                                        void* const* dx, float* dh, float* dbias,
+                                                        void* workspace, size_t ws_bytes, void* stream)
+{
+    return backward3d_impl(v, x, Hs, true, false, bias, dy, B, C, Z, H, W, N, io, dv, dx, dh, dbias, workspace,
+                           ws_bytes, stream);
+}
+
+size_t hyena_fftconv3d_backward_circular_workspace_size(int B, int C, int Z, int H, int W, int N)
+{
+    return bwd3d_workspace(true, 1, B, C, Z, H, W, N);
+}
+
+size_t hyena_fftconv3d_backward_circular_per_sample_workspace_size(int B, int C, int Z, int H, int W, int N)
+{
+    return bwd3d_workspace(true, B, B, C, Z, H, W, N);
+}
+
+hyena_status_t hyena_fftconv3d_gate_backward_circular(const void* v, const void* const* x, const float* Hs,
+                                                      const float* bias, const void* dy, int B, int C, int Z,
+                                                      int H, int W, int N, hyena_dtype_t io, void* dv,
+                                                      void* const* dx, float* dh, float* dbias, void* workspace,
+                                                      size_t ws_bytes, void* stream)
+{
+    return backward3d_impl(v, x, Hs, false, true, bias, dy, B, C, Z, H, W, N, io, dv, dx, dh, dbias, workspace,
+                           ws_bytes, stream);
+}
+
+hyena_status_t hyena_fftconv3d_gate_backward_circular_per_sample(const void* v, const void* const* x,
+                                                                 const float* Hs, const float* bias,
+                                                                 const void* dy, int B, int C, int Z, int H,
+                                                                 int W, int N, hyena_dtype_t io, void* dv,
+                                                                 void* const* dx, float* dh, float* dbias,
+                                                                 void* workspace, size_t ws_bytes, void* stream)
+{
+    return backward3d_impl(v, x, Hs, true, true, bias, dy, B, C, Z, H, W, N, io, dv, dx, dh, dbias, workspace,
+                           ws_bytes, stream);
+}
+
+}  // extern "C"

@@ -70,7 +70,7 @@ hyena_status_t run_bwd2d(Bwd2dArgs a, int N, int log2h, cudaStream_t st)
     hyena_status_t s = cols(2);
     if (s == HYENA_OK) s = launch_bwd_rows2d<LOG2W, IO, 3, PAD>(a, st);
     if (s == HYENA_OK && f.Hs_bstride != 0)   // per-sample: db from the B lag-0 values (any B)
-        s = launch(db2d_sum_kernel, (unsigned)((N * f.C + 255) / 256), 256, 0, st, a);
+        s = launch(db2d_sum_kernel<PAD>, (unsigned)((N * f.C + 255) / 256), 256, 0, st, a);
     return s;
 }
 

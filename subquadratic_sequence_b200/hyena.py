@@ -66,6 +66,22 @@ def _load() -> ctypes.CDLL:
                                                 vp], i),
         "hyena_fftconv_spill_workspace_size": ([i, i, i, i], sz),
         "hyena_device_fault_count": ([], i),
+        "hyena_fftconv2d_backward_circular_per_sample_workspace_size": ([i, i, i, i, i], sz),
+        "hyena_fftconv2d_gate_backward_circular_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i,
+                                                               i, vp, ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
+        "hyena_fftconv3d_backward_workspace_size": ([i, i, i, i, i, i], sz),
+        "hyena_fftconv3d_backward_per_sample_workspace_size": ([i, i, i, i, i, i], sz),
+        "hyena_fftconv3d_gate_backward": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, i, vp,
+                                           ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
+        "hyena_fftconv3d_gate_backward_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, i,
+                                                      vp, ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
+        "hyena_fftconv3d_backward_circular_workspace_size": ([i, i, i, i, i, i], sz),
+        "hyena_fftconv3d_backward_circular_per_sample_workspace_size": ([i, i, i, i, i, i], sz),
+        "hyena_fftconv3d_gate_backward_circular": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i, i, i, vp,
+                                                    ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
+        "hyena_fftconv3d_gate_backward_circular_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i,
+                                                               i, i, vp, ctypes.POINTER(vp), vp, vp, vp, sz,
+                                                               vp], i),
         "hyena_dft32_stage": ([vp, vp, ctypes.c_long, i, i, vp], i),
         "hyena_fftconv_gate_forward_spill": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp, sz,
                                               vp], i),
@@ -933,3 +949,127 @@ def hyena_fftconv2d_gate_backward_circular(v: torch.Tensor, xs, bias: torch.Tens
         ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return dv, dxs, dh, db
+
+
+def hyena_fftconv2d_gate_backward_circular_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                                      dy: torch.Tensor, *, workspace=None, stream=None):
+    """The backward of the circular 2-D forward with a spectrum set per
+    sample (Hs [B][N][C][H][W/2]): returns (dv, [dx_1..dx_N], dh
+    [B][N][C][H][W] per sample, dbias [N][C] summed over the batch)."""
+    B, C, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty((B, N, C, H, W), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, C), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        n = LIB.hyena_fftconv2d_backward_circular_per_sample_workspace_size(B, C, H, W, N)
+        if n == ctypes.c_size_t(-1).value:
+            raise HyenaError("hyena_fftconv2d_backward_circular_per_sample_workspace_size", HYENA_ERR_UNSUPPORTED,
+                             "invalid sizes")
+        workspace = torch.empty(n, device=v.device, dtype=torch.uint8)
+    _check("hyena_fftconv2d_gate_backward_circular_per_sample",
+           LIB.hyena_fftconv2d_gate_backward_circular_per_sample(
+               ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
+               ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+               B, C, H, W, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+               ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+               workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db
+
+
+def hyena_fftconv3d_backward_workspace_size(B: int, C: int, Z: int, H: int, W: int, N: int) -> int:
+    n = LIB.hyena_fftconv3d_backward_workspace_size(B, C, Z, H, W, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv3d_backward_workspace_size", HYENA_ERR_INVALID_ARG, "invalid sizes")
+    return n
+
+
+def hyena_fftconv3d_backward_per_sample_workspace_size(B: int, C: int, Z: int, H: int, W: int, N: int) -> int:
+    n = LIB.hyena_fftconv3d_backward_per_sample_workspace_size(B, C, Z, H, W, N)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError("hyena_fftconv3d_backward_per_sample_workspace_size", HYENA_ERR_INVALID_ARG,
+                         "invalid sizes")
+    return n
+
+
+def _ws3d(name: str, *dims) -> int:
+    n = getattr(LIB, name)(*dims)
+    if n == ctypes.c_size_t(-1).value:
+        raise HyenaError(name, HYENA_ERR_INVALID_ARG, "invalid sizes")
+    return n
+
+
+def hyena_fftconv3d_backward_circular_workspace_size(B: int, C: int, Z: int, H: int, W: int, N: int) -> int:
+    return _ws3d("hyena_fftconv3d_backward_circular_workspace_size", B, C, Z, H, W, N)
+
+
+def hyena_fftconv3d_backward_circular_per_sample_workspace_size(B: int, C: int, Z: int, H: int, W: int,
+                                                                N: int) -> int:
+    return _ws3d("hyena_fftconv3d_backward_circular_per_sample_workspace_size", B, C, Z, H, W, N)
+
+
+_BWD3D_WS = {
+    "hyena_fftconv3d_gate_backward": hyena_fftconv3d_backward_workspace_size,
+    "hyena_fftconv3d_gate_backward_per_sample": hyena_fftconv3d_backward_per_sample_workspace_size,
+    "hyena_fftconv3d_gate_backward_circular": hyena_fftconv3d_backward_circular_workspace_size,
+    "hyena_fftconv3d_gate_backward_circular_per_sample": hyena_fftconv3d_backward_circular_per_sample_workspace_size,
+}
+
+
+def _backward3d(name: str, per_sample: bool, v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                dy: torch.Tensor, workspace, stream):
+    if v.dim() != 5 or dy.shape != v.shape:
+        raise HyenaError(name, HYENA_ERR_INVALID_ARG, "v and dy must be [B][C][Z][H][W] of one shape")
+    B, C, Z, H, W = v.shape
+    N = len(xs)
+    io = io_dtype(v)
+    xp = (ctypes.c_void_p * max(N, 1))(*[_dev(x, v.dtype, f"x[{i}]") for i, x in enumerate(xs)])
+    dv = torch.empty_like(v)
+    dxs = [torch.empty_like(v) for _ in range(N)]
+    dxp = (ctypes.c_void_p * max(N, 1))(*[d.data_ptr() for d in dxs])
+    dh = torch.empty(((B,) if per_sample else ()) + (N, C, Z, H, W), device=v.device, dtype=torch.float32)
+    db = torch.empty((N, C), device=v.device, dtype=torch.float32)
+    if workspace is None:
+        workspace = torch.empty(_BWD3D_WS[name](B, C, Z, H, W, N), device=v.device, dtype=torch.uint8)
+    _check(name, getattr(LIB, name)(
+        ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(Hs, torch.complex64, "Hs")),
+        ctypes.c_void_p(_dev(bias, torch.float32, "bias")), ctypes.c_void_p(_dev(dy, v.dtype, "dy")),
+        B, C, Z, H, W, N, io, ctypes.c_void_p(dv.data_ptr()), dxp, ctypes.c_void_p(dh.data_ptr()),
+        ctypes.c_void_p(db.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dv, dxs, dh, db
+
+
+def hyena_fftconv3d_gate_backward(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor, dy: torch.Tensor,
+                                  *, workspace=None, stream=None):
+    """Gradients of a loss with dL/dy = dy through the 3-D forward: returns
+    (dv [B][C][Z][H][W], [dx_1..dx_N], dh [N][C][Z][H][W] float32, dbias
+    [N][C] float32); Hs the packed 3-D spectra [N][C][2Z][2H][W]."""
+    return _backward3d("hyena_fftconv3d_gate_backward", False, v, xs, bias, Hs, dy, workspace, stream)
+
+
+def hyena_fftconv3d_gate_backward_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                             dy: torch.Tensor, *, workspace=None, stream=None):
+    """The 3-D backward with a spectrum set per sample (Hs
+    [B][N][C][2Z][2H][W]): returns (dv, [dx_1..dx_N], dh [B][N][C][Z][H][W]
+    per sample, dbias [N][C] summed over the batch)."""
+    return _backward3d("hyena_fftconv3d_gate_backward_per_sample", True, v, xs, bias, Hs, dy, workspace, stream)
+
+
+def hyena_fftconv3d_gate_backward_circular(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                           dy: torch.Tensor, *, workspace=None, stream=None):
+    """The backward of the circular 3-D forward (Hs [N][C][Z][H][W/2]):
+    returns (dv, [dx_1..dx_N], dh [N][C][Z][H][W], dbias [N][C])."""
+    return _backward3d("hyena_fftconv3d_gate_backward_circular", False, v, xs, bias, Hs, dy, workspace, stream)
+
+
+def hyena_fftconv3d_gate_backward_circular_per_sample(v: torch.Tensor, xs, bias: torch.Tensor, Hs: torch.Tensor,
+                                                      dy: torch.Tensor, *, workspace=None, stream=None):
+    """The circular 3-D backward with a spectrum set per sample (Hs
+    [B][N][C][Z][H][W/2]): dh [B][N][C][Z][H][W] per sample, dbias summed."""
+    return _backward3d("hyena_fftconv3d_gate_backward_circular_per_sample", True, v, xs, bias, Hs, dy, workspace,
+                       stream)

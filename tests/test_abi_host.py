@@ -476,3 +476,63 @@ def test_dft32_stage_rejects_bad_arguments(lib):
     assert f(ctypes.c_void_p(A + 8), P(1), 4, 1, 0, None) == INVALID
     assert f(P(0), P(0), 4, 1, 1, None) == INVALID                  # y overlapping x
     assert f(P(0), P(1), (1 << 30) + 1, 1, 0, None) == UNSUPPORTED
+
+
+def test_backward_2d_circular_per_sample_rejects_bad_arguments(lib):
+    bad = ctypes.c_size_t(-1).value
+    assert lib.hyena_fftconv2d_backward_circular_per_sample_workspace_size(2, 3, 32, 64, 2) != bad
+    assert (lib.hyena_fftconv2d_backward_circular_per_sample_workspace_size(2, 3, 32, 64, 2)
+            > lib.hyena_fftconv2d_backward_circular_workspace_size(2, 3, 32, 64, 2))
+    assert lib.hyena_fftconv2d_backward_circular_per_sample_workspace_size(2, 3, 30, 64, 2) == bad
+    assert lib.hyena_fftconv2d_backward_circular_per_sample_workspace_size(0, 3, 32, 64, 2) == bad
+    xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
+    dxs = (ctypes.c_void_p * 2)(P(7).value, P(8).value)
+    f = lib.hyena_fftconv2d_gate_backward_circular_per_sample
+    assert f(None, xs, P(3), P(4), P(5), 2, 3, 32, 64, 2, F32, P(6), dxs, P(9), P(10), P(11), 1 << 30,
+             None) == INVALID
+    assert f(P(0), xs, P(3), P(4), P(5), 2, 3, 30, 64, 2, F32, P(6), dxs, P(9), P(10), P(11), 1 << 30,
+             None) == UNSUPPORTED
+    assert f(P(0), xs, P(3), P(4), P(5), 2, 3, 32, 64, 2, F32, P(6), dxs, P(9), P(10), P(11), 16,
+             None) == WORKSPACE
+    assert f(P(0), xs, P(3), P(4), P(5), 2, 3, 32, 64, 2, F32, P(0), dxs, P(9), P(10), P(11), 1 << 30,
+             None) == INVALID                        # dv overlapping v
+
+
+def test_backward_3d_rejects_bad_arguments(lib):
+    bad = ctypes.c_size_t(-1).value
+    shared = lib.hyena_fftconv3d_backward_workspace_size(2, 3, 16, 32, 64, 2)
+    per_sample = lib.hyena_fftconv3d_backward_per_sample_workspace_size(2, 3, 16, 32, 64, 2)
+    assert shared != bad and per_sample != bad and per_sample > shared
+    # the accumulated dh spectra alone: N C 2Z 2H W complex64
+    assert shared >= 2 * 3 * (2 * 16) * (2 * 32) * 64 * 8
+    assert lib.hyena_fftconv3d_backward_workspace_size(2, 3, 16, 32, 512, 2) == bad     # W > 256
+    assert lib.hyena_fftconv3d_backward_workspace_size(2, 3, 8, 32, 64, 2) == bad       # Z < 16
+    assert lib.hyena_fftconv3d_backward_workspace_size(2, 3, 16, 32, 64, 17) == bad     # N > 16
+    assert lib.hyena_fftconv3d_backward_per_sample_workspace_size(0, 3, 16, 32, 64, 2) == bad
+    xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
+    dxs = (ctypes.c_void_p * 2)(P(7).value, P(8).value)
+    circ = lib.hyena_fftconv3d_backward_circular_workspace_size(2, 3, 16, 32, 64, 2)
+    circ_ps = lib.hyena_fftconv3d_backward_circular_per_sample_workspace_size(2, 3, 16, 32, 64, 2)
+    assert bad not in (circ, circ_ps) and shared > circ and circ_ps > circ
+    assert lib.hyena_fftconv3d_backward_circular_workspace_size(2, 3, 16, 32, 16, 2) == bad   # W < 32
+    for f in (lib.hyena_fftconv3d_gate_backward, lib.hyena_fftconv3d_gate_backward_per_sample,
+              lib.hyena_fftconv3d_gate_backward_circular, lib.hyena_fftconv3d_gate_backward_circular_per_sample):
+        ok = (P(0), xs, P(3), P(4), P(5), 2, 3, 16, 32, 64, 2, F32, P(6), dxs, P(9), P(10), P(11), 1 << 30, None)
+
+        def call(**kw):
+            a = list(ok)
+            for k, val in kw.items():
+                a[int(k[1:])] = val
+            return f(*a)
+
+        assert call(a0=None) == INVALID                               # v missing
+        assert call(a2=None) == INVALID                               # spectra missing
+        assert call(a7=30) == UNSUPPORTED                             # H not a power of two
+        assert call(a8=512) == UNSUPPORTED                            # W above 256
+        assert call(a10=17) == UNSUPPORTED                            # order above 16
+        assert call(a11=5) == INVALID                                 # no such storage type
+        assert call(a17=16) == WORKSPACE                              # workspace too small
+        assert call(a16=ctypes.c_void_p(A + 11 * BIG + 16)) == WORKSPACE   # workspace misaligned
+        assert call(a12=P(0)) == INVALID                              # dv overlapping v
+        assert call(a14=P(3)) == INVALID                              # dh overlapping the spectra
+        assert call(a12=ctypes.c_void_p(A + 6 * BIG + 4)) == INVALID  # dv misaligned

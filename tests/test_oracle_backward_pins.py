@@ -409,6 +409,64 @@ def test_backward_3d_axis_permutation_permutes_every_gradient():
     assert rel_err(gp[3], g[3]) < 1e-12
 
 
+# ------------------------------------------------- circular 3-D
+
+@pytest.mark.parametrize("N", [1, 2])
+def test_backward_circular_3d_matches_finite_differences(N):
+    v, x, h, b, dy = problem_3d(2, 2, 2, 3, 3, N, seed=90 + N)
+    dv, dx, dh, db = oracle.hyena_backward_circular_3d(v, x, h, b, dy, route="direct")
+
+    def loss(v_, x_, h_, b_):
+        return float(np.sum(dy * oracle.hyena_forward_circular_nd(v_, x_, h_, b_, route="direct")))
+
+    eps = 1e-6
+    for arr, grad, name in ((v, dv, "v"), (x, dx, "x"), (h, dh, "h"), (b, db, "bias")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            orig = arr[idx]
+            arr[idx] = orig + eps
+            lp = loss(v, x, h, b)
+            arr[idx] = orig - eps
+            lm = loss(v, x, h, b)
+            arr[idx] = orig
+            fd[idx] = (lp - lm) / (2 * eps)
+        assert rel_err(grad, fd) < 1e-7, name
+
+
+def test_backward_circular_3d_routes_agree_and_db_is_dh_origin():
+    v, x, h, b, dy = problem_3d(2, 2, 4, 4, 8, 2, seed=93)
+    d = oracle.hyena_backward_circular_3d(v, x, h, b, dy, route="direct")
+    f = oracle.hyena_backward_circular_3d(v, x, h, b, dy, route="fft")
+    for a, c in zip(d, f):
+        assert rel_err(c, a) < 1e-12
+    assert rel_err(d[3], d[2][:, :, 0, 0, 0]) < 1e-13
+
+
+def test_backward_circular_3d_on_zero_padded_volumes_is_the_linear_backward():
+    # 2Z x 2H x 2W volumes with v, x_n, dy and h_n zero outside the Z x H x W
+    # corner: nothing wraps, so the gradients there are the linear 3-D backward's
+    B, C, Z, H, W, N = 2, 2, 2, 4, 4, 2
+    v, x, h, b, dy = problem_3d(B, C, Z, H, W, N, seed=94)
+
+    def pad(a):
+        out = np.zeros(a.shape[:-3] + (2 * Z, 2 * H, 2 * W))
+        out[..., :Z, :H, :W] = a
+        return out
+    dv, dx, dh, db = oracle.hyena_backward_circular_3d(pad(v), pad(x), pad(h), b, pad(dy))
+    rv, rx, rh, rb = oracle.hyena_backward_3d(v, x, h, b, dy)
+    assert rel_err(dv[..., :Z, :H, :W], rv) < 1e-12 and rel_err(dx[..., :Z, :H, :W], rx) < 1e-12
+    assert rel_err(dh[..., :Z, :H, :W], rh) < 1e-12 and rel_err(db, rb) < 1e-12
+
+
+def test_backward_circular_3d_of_one_plane_is_the_circular_2d_backward():
+    v, x, h, b, dy = problem_3d(2, 3, 1, 8, 4, 2, seed=95)
+    g3 = oracle.hyena_backward_circular_3d(v, x, h, b, dy)
+    g2 = oracle.hyena_backward_circular_2d(v[:, :, 0], x[:, :, :, 0], h[:, :, 0], b, dy[:, :, 0])
+    for a, c in zip(g3[:3], g2[:3]):
+        assert rel_err(a[..., 0, :, :], c) < 1e-12
+    assert rel_err(g3[3], g2[3]) < 1e-12
+
+
 def test_backward_circular_per_sample_matches_finite_differences():
     B, D, L, N = 2, 2, 8, 2
     r = np.random.default_rng(80)

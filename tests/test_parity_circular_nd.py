@@ -148,6 +148,48 @@ def test_backward_2d_circular_matches_oracle(hy, B, C, H, W, N, io):
     check_backward(got, ref, io, f"circular 2-D backward B{B} C{C} {H}x{W} N{N} {io}")
 
 
+@pytest.mark.parametrize("B,C,H,W,N,io", [
+    (2, 2, 16, 32, 2, "f32"), (3, 3, 32, 64, 1, "f32"), (2, 2, 64, 128, 2, "bf16"), (2, 1, 256, 256, 3, "f32"),
+    (3, 22, 512, 512, 1, "f32"),     # 66 images, 64 a wave
+])
+def test_backward_2d_circular_per_sample_matches_oracle(hy, B, C, H, W, N, io):
+    """A spectrum set per sample: per sample b, the circular 2-D backward of
+    the oracle with sample b's filters gives dv, dx and dh_b; db is the sum
+    of the samples' db."""
+    v, x, b, _ = problem(B, C, (H, W), N, seed=3 * H + W + N)
+    rng = np.random.default_rng(H + 7 * W)
+    h = np.stack([decaying(rng, (N, C, H, W)) for _ in range(B)])           # [B][N][C][H][W]
+    dy = rng.standard_normal((B, C, H, W)).astype(np.float32)
+    Hs = hy.hyena_filter_rfft2d_circular(dev(h.reshape(B * N, C, H, W))).view(B, N, C, H, W // 2)
+    dv, dxs, dh, db = hy.hyena_fftconv2d_gate_backward_circular_per_sample(
+        dev(v, io), [dev(xx, io) for xx in x], dev(b), Hs, dev(dy, io))
+    torch.cuda.synchronize()
+    got = host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+    parts = [oracle.hyena_backward_circular_2d(as_io(v[i:i + 1], io), np.stack([as_io(xx[i:i + 1], io) for xx in x]),
+                                               h[i].astype(np.float64), b.astype(np.float64), as_io(dy[i:i + 1], io))
+             for i in range(B)]
+    ref = (np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts], axis=1),
+           np.stack([p[2] for p in parts]), np.sum([p[3] for p in parts], axis=0))
+    check_backward(got, ref, io, f"circular 2-D per-sample backward B{B} C{C} {H}x{W} N{N} {io}")
+
+
+def test_backward_2d_circular_per_sample_with_equal_sets_is_the_shared_backward(hy):
+    B, C, H, W, N = 3, 2, 32, 64, 2
+    v, x, b, h = problem(B, C, (H, W), N, seed=31)
+    dy = np.random.default_rng(5).standard_normal((B, C, H, W)).astype(np.float32)
+    H1 = hy.hyena_filter_rfft2d_circular(dev(h))
+    Hb = H1.unsqueeze(0).expand(B, -1, -1, -1, -1).contiguous()
+    args = (dev(v), [dev(xx) for xx in x], dev(b))
+    sdv, sdx, sdh, sdb = hy.hyena_fftconv2d_gate_backward_circular(*args, H1, dev(dy))
+    pdv, pdx, pdh, pdb = hy.hyena_fftconv2d_gate_backward_circular_per_sample(*args, Hb, dev(dy))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(pdv), host(sdv))
+    for a_, b_ in zip(pdx, sdx):
+        assert np.array_equal(host(a_), host(b_))
+    assert np.max(np.abs(host(pdh).sum(axis=0) - host(sdh))) <= 1e-5 * np.max(np.abs(host(sdh)))
+    assert np.max(np.abs(host(pdb) - host(sdb))) <= 1e-5 * np.max(np.abs(host(sdb)))
+
+
 def test_backward_2d_circular_shift_filter_closed_form(hy):
     # N = 1, h = delta at (k, l), b = 0: y = x roll(v, (k, l)), so
     # dv = roll(dy x, (-k, -l)), dx = dy roll(v, (k, l)),
@@ -263,3 +305,84 @@ def test_forward_3d_circular_per_sample_matches_oracle(hy, B, C, Z, H, W, N, io)
     ref = oracle.hyena_forward_circular_nd_per_sample(as_io(v, io), np.stack([as_io(xx, io) for xx in x]),
                                                       h.astype(np.float64), b.astype(np.float64))
     assert_close(y, ref, io, f"circular 3-D per-sample B{B} C{C} {Z}x{H}x{W} N{N} {io}")
+
+
+# ------------------------------------------------- circular 3-D backward
+
+def gpu_backward_3d_circular(hy, v, x, b, h, dy, io, per_sample=False):
+    if per_sample:
+        B, N, C = h.shape[:3]
+        Hs = hy.hyena_filter_rfft3d_circular(dev(h.reshape((B * N,) + h.shape[2:])))
+        Hs = Hs.view((B, N) + tuple(Hs.shape[1:]))
+        fn = hy.hyena_fftconv3d_gate_backward_circular_per_sample
+    else:
+        Hs = hy.hyena_filter_rfft3d_circular(dev(h))
+        fn = hy.hyena_fftconv3d_gate_backward_circular
+    dv, dxs, dh, db = fn(dev(v, io), [dev(xx, io) for xx in x], dev(b), Hs, dev(dy, io))
+    torch.cuda.synchronize()
+    return host(dv), np.stack([host(d) for d in dxs]), host(dh), host(db)
+
+
+@pytest.mark.parametrize("B,C,Z,H,W,N,io", [
+    (1, 2, 16, 16, 32, 2, "f32"), (2, 1, 32, 16, 64, 1, "f32"), (2, 2, 16, 32, 32, 2, "bf16"),
+    (1, 1, 64, 16, 32, 3, "f32"), (2, 2, 16, 256, 64, 1, "f32"), (1, 1, 256, 16, 32, 1, "f32"),
+])
+def test_backward_3d_circular_matches_oracle(hy, B, C, Z, H, W, N, io):
+    v, x, b, h = problem(B, C, (Z, H, W), N, seed=Z + 2 * H + 5 * W + N)
+    dy = np.random.default_rng(Z * W).standard_normal(v.shape).astype(np.float32)
+    got = gpu_backward_3d_circular(hy, v, x, b, h, dy, io)
+    ref = oracle.hyena_backward_circular_3d(as_io(v, io), np.stack([as_io(xx, io) for xx in x]),
+                                            h.astype(np.float64), b.astype(np.float64), as_io(dy, io))
+    check_backward(got, ref, io, f"circular 3-D backward B{B} C{C} {Z}x{H}x{W} N{N} {io}")
+
+
+def test_backward_3d_circular_channel_across_two_waves(hy):
+    """64 x 64 x 256 volumes (4 MB of scratch each, 16 a wave): 18 volumes
+    of 6 channels put channel 5 across the two waves; the oracle on it."""
+    B, C, Z, H, W, N = 3, 6, 64, 64, 256, 1
+    v, x, b, h = problem(B, C, (Z, H, W), N, seed=66)
+    dy = np.random.default_rng(67).standard_normal(v.shape).astype(np.float32)
+    dv, dx, dh, db = gpu_backward_3d_circular(hy, v, x, b, h, dy, "f32")
+    c = 5
+    sl = slice(c, c + 1)
+    ref = oracle.hyena_backward_circular_3d(v[:, sl], np.stack([xx[:, sl] for xx in x]), h[:, sl], b[:, sl],
+                                            dy[:, sl])
+    check_backward((dv[:, sl], dx[:, :, sl], dh[:, sl], db[:, sl]), ref, "f32", "circular 3-D split channel")
+
+
+@pytest.mark.parametrize("B,C,Z,H,W,N,io", [(2, 2, 16, 16, 32, 2, "f32"), (3, 1, 16, 32, 32, 1, "bf16")])
+def test_backward_3d_circular_per_sample_matches_oracle(hy, B, C, Z, H, W, N, io):
+    v, x, b, _ = problem(B, C, (Z, H, W), N, seed=40 + Z + W)
+    rng = np.random.default_rng(Z + H + W)
+    h = np.stack([decaying(rng, (N, C, Z, H, W)) for _ in range(B)])        # [B][N][C][Z][H][W]
+    dy = rng.standard_normal(v.shape).astype(np.float32)
+    got = gpu_backward_3d_circular(hy, v, x, b, h, dy, io, per_sample=True)
+    parts = [oracle.hyena_backward_circular_3d(as_io(v[i:i + 1], io), np.stack([as_io(xx[i:i + 1], io) for xx in x]),
+                                               h[i].astype(np.float64), b.astype(np.float64), as_io(dy[i:i + 1], io))
+             for i in range(B)]
+    ref = (np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts], axis=1),
+           np.stack([p[2] for p in parts]), np.sum([p[3] for p in parts], axis=0))
+    check_backward(got, ref, io, f"circular 3-D per-sample backward B{B} C{C} {Z}x{H}x{W} N{N} {io}")
+
+
+def test_backward_3d_circular_shift_filter_closed_form(hy):
+    # N = 1, h = delta at (k, l, m), b = 0: y = x roll(v, (k, l, m)), so
+    # dv = roll(dy x, -(k, l, m)), dx = dy roll(v, (k, l, m)) and
+    # dh[s] = sum over the batch of dy x roll(v, s)
+    B, C, Z, H, W = 2, 2, 16, 16, 32
+    v, x, _, _ = problem(B, C, (Z, H, W), 1, seed=88)
+    k = (3, 5, 7)
+    h = np.zeros((1, C, Z, H, W), np.float32)
+    h[0, :, k[0], k[1], k[2]] = 1.0
+    b = np.zeros((1, C), np.float32)
+    dy = np.random.default_rng(89).standard_normal(v.shape).astype(np.float32)
+    dv, dx, dh, db = gpu_backward_3d_circular(hy, v, x, b, h, dy, "f32")
+    e = dy.astype(np.float64) * x[0]
+    axes = (2, 3, 4)
+    assert_close(dv, np.roll(e, tuple(-s for s in k), axis=axes), "f32", "shift dv")
+    assert_close(dx[0], dy * np.roll(v.astype(np.float64), k, axis=axes), "f32", "shift dx")
+    for s in [(0, 0, 0), k, (15, 1, 31), (8, 8, 16)]:
+        want = np.sum(e * np.roll(v.astype(np.float64), s, axis=axes), axis=(0, 2, 3, 4))
+        got = dh[0][:, s[0], s[1], s[2]]
+        assert np.max(np.abs(got - want)) <= 1e-4 * np.max(np.abs(dh)), s
+    assert np.max(np.abs(db[0] - dh[0][:, 0, 0, 0])) <= 1e-5 * np.max(np.abs(dh))
