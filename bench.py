@@ -117,7 +117,9 @@ def alg_bytes_backward(wl: synth.Workload) -> int:
     dbias out (float32)."""
     io = 2 if wl.io == "bf16" else 4
     act = wl.positions * io
-    if wl.kind == "3d" and not wl.circular:   # 2Z x 2H x W spectrum slots and Z x H x W of dh a filter
+    if wl.kind == "3d" and wl.circular:       # Z x H x W/2 spectrum slots and Z x H x W of dh a filter
+        return (2 * wl.N + 3) * act + wl.N * wl.D * wl.Z * wl.H * wl.W * (4 + 4) + wl.N * wl.D * 4
+    if wl.kind == "3d":                       # 2Z x 2H x W spectrum slots and Z x H x W of dh a filter
         sets = wl.B if wl.film else 1
         return (2 * wl.N + 3) * act + sets * wl.N * wl.D * wl.Z * wl.H * wl.W * (32 + 4) + wl.N * wl.D * 4
     if wl.film and wl.kind == "2d":   # 2H x W spectrum slots and H x W of dh, per sample
@@ -735,15 +737,17 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
     # and launch lies inside the timed region.
     e2e_ms, h2d, d2h = run_e2e(args, wl, inp, bufs, step, max_over_ranks)
 
-    # ---- the backward pass (1-D, 2-D, padded 3-D): one call per timed repetition
+    # ---- the backward pass: one call per timed repetition
     bwd = None
-    if wl.kind in ("1d", "2d") or (wl.kind == "3d" and not wl.circular):
+    if wl.kind in ("1d", "2d", "3d"):
         dy = to_dev(synth.make_output_grad(wl), io)
         if wl.kind == "3d":
-            size_fn = (hyena.hyena_fftconv3d_backward_per_sample_workspace_size if wl.film
+            size_fn = (hyena.hyena_fftconv3d_backward_circular_workspace_size if wl.circular
+                       else hyena.hyena_fftconv3d_backward_per_sample_workspace_size if wl.film
                        else hyena.hyena_fftconv3d_backward_workspace_size)
             ws_b = torch.empty(size_fn(wl.B, wl.D, wl.Z, wl.H, wl.W, wl.N), device="cuda", dtype=torch.uint8)
-            bwd_fn = (hyena.hyena_fftconv3d_gate_backward_per_sample if wl.film
+            bwd_fn = (hyena.hyena_fftconv3d_gate_backward_circular if wl.circular
+                      else hyena.hyena_fftconv3d_gate_backward_per_sample if wl.film
                       else hyena.hyena_fftconv3d_gate_backward)
             bwd_kernel = ("fft2d_bwd_row_kernel+fft2d_col_kernel+fft3d_bwd_z_kernel (" + bwd_fn.__name__ +
                           ", all launches)")
@@ -769,7 +773,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             def backward():
                 hyena.hyena_fftconv2d_gate_backward_circular(v, xs, b, H, dy, workspace=ws_b)
         elif wl.circular:
-            ws_b = torch.empty(hyena.hyena_fftconv_backward_circular_workspace_size(wl.D, wl.L, wl.N),
+            ws_b = torch.empty(hyena.hyena_fftconv_backward_circular_workspace_size(wl.B, wl.D, wl.L, wl.N),
                                device="cuda", dtype=torch.uint8)
             bwd_kernel = ("fourstep_bwd_row_kernel+fourstep_bwd_col_kernel<PAD=false> "
                           "(hyena_fftconv_gate_backward_circular, all launches)" if long_path(wl) else
@@ -792,7 +796,7 @@ def run_gpu(args, wl: synth.Workload) -> dict | None:
             def backward():
                 hyena.hyena_fftconv2d_gate_backward(v, xs, b, H, dy, workspace=ws_b)
         else:
-            ws_b = torch.empty(hyena.hyena_fftconv_backward_workspace_size(wl.D, wl.L, wl.N),
+            ws_b = torch.empty(hyena.hyena_fftconv_backward_workspace_size(wl.B, wl.D, wl.L, wl.N),
                                device="cuda", dtype=torch.uint8)
             bwd_kernel = ("fourstep_bwd_row_kernel+fourstep_bwd_col_kernel (hyena_fftconv_gate_backward, "
                           "all launches)" if long_path(wl) else "backward1d_kernel (hyena_fftconv_gate_backward)")

@@ -254,12 +254,12 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_circular_per_sample(const vo
  *   dz_{n-1}[u] = sum_t h_n[(t - u) mod L] e[t] + b_n e[u],   dv = dz_0.
  * Arguments as hyena_fftconv_gate_backward with H [N][D][L/2] from
  * hyena_filter_rfft_circular; dh [N][D][L] and dbias [N][D] summed over the
- * batch; workspace of hyena_fftconv_backward_circular_workspace_size(D, L,
- * N) bytes (12 N D L up to L = 16384; above, the four-step backward's),
- * 256-byte aligned.  32 <= L <= HYENA_MAX_LEN, a power of two (the size
+ * batch; workspace of hyena_fftconv_backward_circular_workspace_size(B,
+ * D, L, N) bytes (12 N D L S up to L = 16384, S = min(B, 8) batch slices;
+ * above, the four-step backward's), 256-byte aligned.  32 <= L <= HYENA_MAX_LEN, a power of two (the size
  * function returns (size_t)-1 otherwise).  Deterministic: two launches up
  * to L = 16384, the four-step launch sequence above. */
-HYENA_API size_t hyena_fftconv_backward_circular_workspace_size(int D, int L, int N);
+HYENA_API size_t hyena_fftconv_backward_circular_workspace_size(int B, int D, int L, int N);
 HYENA_API hyena_status_t hyena_fftconv_gate_backward_circular(const void* v, const void* const* x,
                                                               const float* H, const float* bias,
                                                               const void* dy, int B, int D, int L, int N,
@@ -367,14 +367,17 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_noalloc(const void* v, const
  *   dh     [N][D][L] float32 out    summed over the batch
  *   dbias  [N][D] float32 out       summed over the batch
  *   workspace / ws_bytes: device scratch of at least
- *          hyena_fftconv_backward_workspace_size(D, L, N) bytes (20 N D L
- *          for L <= 16384; above, 8 N D L plus about N * 100 MB + 64 MB
- *          for the waves), 256-byte aligned; nothing in it needs to start
- *          at zero.
+ *          hyena_fftconv_backward_workspace_size(B, D, L, N) bytes (20 N D
+ *          L S for L <= 16384, S = min(B, 8) batch slices; above, 8 N D L
+ *          plus about N * 100 MB + 64 MB for the waves), 256-byte aligned;
+ *          nothing in it needs to start at zero.
  * L is a power of two, 16 <= L <= 2^22; 1 <= N <= HYENA_MAX_ORDER.
- * L <= 16384: two launches: a group of threads owns a channel and walks its
- * B sequences (the forward again, then the orders backwards), accumulating
- * the channel's dh spectra; a second launch inverts those spectra.
+ * L <= 16384: two launches: a group of threads owns a channel and a slice
+ * of the batch (the slice count chosen so that the groups fill the SMs in
+ * the fewest rounds) and walks the slice's sequences (the forward again,
+ * then the orders backwards), accumulating the slice's dh spectra; a
+ * second launch sums each channel's slice spectra in order and inverts
+ * the sums.
  * L > 16384 (the four-step transform): per wave of sequences the forward
  * again, saving each order's spectrum and c_n, then per order in reverse a
  * column launch (dx_n, e = g x_n) and a row launch per channel that
@@ -382,7 +385,7 @@ HYENA_API hyena_status_t hyena_fftconv_gate_forward_noalloc(const void* v, const
  * Both are deterministic (no atomics).
  * Alignment: v, x_n, dy, dv, dx_n, H, dh 16 bytes; bias, dbias 4.  Outputs
  * must not overlap each other, any input or the workspace. */
-HYENA_API size_t hyena_fftconv_backward_workspace_size(int D, int L, int N);
+HYENA_API size_t hyena_fftconv_backward_workspace_size(int B, int D, int L, int N);
 HYENA_API hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x,
                                                      const float* H, const float* bias,
                                                      const void* dy, int B, int D, int L, int N,

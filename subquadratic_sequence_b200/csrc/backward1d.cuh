@@ -15,16 +15,19 @@
 //     DFT(dh_n)     = sum_b DFT(e) conj(DFT(z_{n-1}))   (first L lags)
 //
 // One CTA group (T threads, the same FFT machinery and layouts as the fused
-// forward) owns one channel d and walks its B sequences:
+// forward) owns one unit (channel d, slice s of the batch) and walks the
+// slice's sequences; the host picks the number of slices S so that the D S
+// units fill the chip in the fewest rounds:
 //   A. the forward again, saving Z_n = DFT(z_n) and c_{n+1} to the
 //      workspace in register order (each thread reads back what it wrote);
 //   B. for n = N..1: dx_n and e from g; E = DFT(e); accumulate E conj(Z)
-//      into the channel's dh spectrum (only this group touches it, so a
-//      plain read-modify-write); g = inverse of (conj(H_n) + b_n) E.
+//      into the unit's dh spectrum (only this group touches it, so a
+//      plain read-modify-write; the slice's first sequence stores);
+//      g = inverse of (conj(H_n) + b_n) E.
 // Both phases run through one copy of the FFT code (a step loop), which
-// halves the kernel's instruction footprint.  A second launch turns each
-// accumulated spectrum into dh_n (inverse real FFT, first L lags) and
-// db_n = dh_n[0].
+// halves the kernel's instruction footprint.  A second launch sums each
+// channel's S slice spectra in slice order (deterministic), turns the sum
+// into dh_n (inverse real FFT, first L lags) and db_n = dh_n[0].
 //
 // Per-sample filters (PS, input-dependent filters): sequence (b, d) reads
 // sample b's spectra at H + b H_bstride, and its dh spectrum is its own
@@ -51,10 +54,11 @@ struct Backward1dArgs {
     void* dx[kMaxOrder];           // [B][D][L] io each
     float* dh;                     // [N][D][L]
     float* dbias;                  // [N][D]
-    float2* acc;                   // workspace [N][D][L]: accumulated dh spectra (packed)
-    float2* wz;                    // workspace [D][N][L]: Z_n in register order
-    float2* wc;                    // workspace [D][N][L/2]: c_{n+1} in register order
+    float2* acc;                   // workspace [S][N][D][L]: accumulated dh spectra (packed; [B][N][D][L] per sample)
+    float2* wz;                    // workspace [S][D][N][L]: Z_n in register order
+    float2* wc;                    // workspace [S][D][N][L/2]: c_{n+1} in register order
     int B, D, N;
+    int S;                         // batch slices: unit u = s D + d takes samples [s B / S, (s + 1) B / S)
     size_t H_bstride;              // per-sample spectra: slots between samples' sets
 };
 
@@ -75,14 +79,17 @@ backward1d_kernel(Backward1dArgs args)
     extern __shared__ __align__(16) float2 smem_dyn[];
 
     const int g = threadIdx.x / T, t = threadIdx.x % T;
-    const int d_raw = blockIdx.x * F::G + g;
-    const bool active = d_raw < args.D;      // inactive groups compute but write nothing
-    const int d = active ? d_raw : args.D - 1;
     const int D = args.D, N = args.N;
+    const int units = D * args.S;
+    const int u_raw = blockIdx.x * F::G + g;
+    const bool active = u_raw < units;       // inactive groups compute but write nothing
+    const int u = active ? u_raw : units - 1;
+    const int sl = u / D, d = u - sl * D;    // slice, channel
+    const int b0 = (int)((long)sl * args.B / args.S), b1 = (int)((long)(sl + 1) * args.B / args.S);
     float2* sm = smem_dyn + g * F::SMEM_SEQ;
     float2* stage = smem_dyn + F::G * F::SMEM_SEQ + g * F::STAGE_SEQ;
-    float2* wz = args.wz + (size_t)d * N * M;
-    float2* wc = args.wc + (size_t)d * N * SEQ;
+    float2* wz = args.wz + (size_t)u * N * M;
+    float2* wc = args.wc + (size_t)u * N * SEQ;
     // index of io register i among the thread's NIO io registers
     auto io_slot = [](int i) { return PAD ? (i / RF) * (RF / 2) + i % RF : i; };
     auto pick = [](const void* const* arr, int n) {
@@ -94,7 +101,7 @@ backward1d_kernel(Backward1dArgs args)
     };
 
     float2 a[E];
-    for (int b = 0; b < args.B; ++b) {
+    for (int b = b0; b < b1; ++b) {
         const size_t seq = (size_t)b * D + d;
         const float2* Hb = PS ? args.H + (size_t)b * args.H_bstride : args.H;
         {
@@ -139,9 +146,9 @@ backward1d_kernel(Backward1dArgs args)
                     });
             } else if (active) {
                 // dh spectrum: acc[k] (+)= E[k] conj(Z_n[k]) over the 2L-point bins
-                float2* acc = args.acc + (((size_t)(PS ? b : 0) * N + n) * D + d) * M;
+                float2* acc = args.acc + (((size_t)(PS ? b : sl) * N + n) * D + d) * M;
                 const float2* zr = wz + (size_t)n * M;
-                const bool first = PS || b == 0;
+                const bool first = PS || b == b0;
                 float2 z[E];
                 static_for<E>([&](auto ii) {
                     constexpr int i = decltype(ii)::value;
@@ -231,9 +238,10 @@ backward1d_kernel(Backward1dArgs args)
 }
 
 // dh_n[d] and db_n[d] from the accumulated spectra: one group per row
-// (n, d): the inverse real FFT of the packed spectrum (scale 1/P), the
-// first L lags, and db = dh[0].  PS: the group inverts the B per-sample
-// spectra of its row in turn and db is the sum of their lag-0 values.
+// (n, d): the sum of the row's S slice spectra (in slice order), its
+// inverse real FFT (scale 1/P), the first L lags, and db = dh[0].  PS: the
+// group inverts the B per-sample spectra of its row in turn and db is the
+// sum of their lag-0 values.
 template <int LOG2M, bool PS = false, bool PAD = true>
 __global__ void __launch_bounds__(Fft1d<LOG2M, PAD>::THREADS)
 dh_finalize_kernel(Backward1dArgs args)
@@ -253,19 +261,34 @@ dh_finalize_kernel(Backward1dArgs args)
     for (int b = 0; b < (PS ? args.B : 1); ++b) {
     const size_t srow = (size_t)b * rows + row;              // [B][N][D] rows (b = 0 when shared)
     const float2* acc = args.acc + srow * M;
+    const int nsl = PS ? 1 : args.S;                          // slice spectra [S][N][D] summed
+    const size_t sstride = (size_t)rows * M;
+    // the thread's bins (k in a[i1], M - k in a[i2]), summed over the slices
+    // one slice at a time, so that each slice's loads go out together
     float2 a[E];
+    F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2) {
+        a[i1] = acc[k];
+        if (kind == 0) a[i2] = acc[M - k];
+    });
+    for (int q = 1; q < nsl; ++q) {
+        const float2* aq = acc + q * sstride;
+        F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2) {
+            a[i1] = cadd(a[i1], aq[k]);
+            if (kind == 0) a[i2] = cadd(a[i2], aq[M - k]);
+        });
+    }
     F::for_each_pair(t, [&](int i1, int i2, int k, int kind, float2 w) {
         float2 z1, z2;
         if (kind == 1) {
-            const float2 p = acc[0];
+            const float2 p = a[i1];                           // slot 0: bins 0 and M
             unsplit_pair(make_float2(p.x, 0.0f), make_float2(p.y, 0.0f), w, s, z1, z2);
             a[i1] = z1;
         } else if (kind == 2) {
-            const float2 y = acc[k];
+            const float2 y = a[i1];
             unsplit_pair(y, y, w, s, z1, z2);
             a[i1] = z1;
         } else {
-            unsplit_pair(acc[k], acc[M - k], w, s, z1, z2);
+            unsplit_pair(a[i1], a[i2], w, s, z1, z2);
             a[i1] = z1;
             a[i2] = z2;
         }

@@ -114,6 +114,29 @@ size_t spectrum_bytes(long N, long D, long L) { return sizeof(float2) * N * D * 
 
 size_t round_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
 
+// Workspace of the single-CTA backward (L <= 16384): per batch slice (at
+// most min(B, 8) of them) a dh spectrum set acc [S][N][D][M] (per sample:
+// [B][N][D][M]) and the saved Z_n (wz) and c_n (wc) of each unit.  M = L
+// packed slots (L/2 circular); c_n takes half of that (all of it circular).
+struct Bwd1dLayout {
+    size_t acc, wz, wc, total;
+    int slices;
+};
+
+Bwd1dLayout bwd1d_layout(int B, int D, int L, int N, bool per_sample, bool circular)
+{
+    constexpr int kMaxBwdSlices = 8;
+    Bwd1dLayout l;
+    l.slices = B < kMaxBwdSlices ? B : kMaxBwdSlices;
+    const size_t spec = sizeof(float2) * (size_t)N * D * (circular ? L / 2 : L);   // one spectrum set
+    const size_t cset = circular ? spec : spec / 2;
+    l.acc = 0;
+    l.wz = round_up(spec * (per_sample ? (size_t)B : (size_t)l.slices), 256);
+    l.wc = l.wz + round_up(spec * l.slices, 256);
+    l.total = l.wc + round_up(cset * l.slices, 256);
+    return l;
+}
+
 hyena_status_t forward_impl(const void* v, const void* const* x, const float* h, const float* H,
                             bool per_sample, const float* bias, int B, int D, int L, int N,
                             hyena_dtype_t io, void* y, void* workspace, size_t ws_bytes, void* stream);
@@ -507,14 +530,13 @@ hyena_status_t hyena_fftconv_gate_forward_circular_per_sample(const void* v, con
 }
 
 
-size_t hyena_fftconv_backward_workspace_size(int D, int L, int N)
+size_t hyena_fftconv_backward_workspace_size(int B, int D, int L, int N)
 {
     int log2m = 0;
-    if (D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2, &log2m) != HYENA_OK)
+    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2, &log2m) != HYENA_OK)
         return (size_t)-1;
     if (log2m > kMaxLog2Fused) return fourstep_bwd_layout(log2m, D, N).total;
-    const size_t spec = sizeof(float2) * (size_t)N * D * L;
-    return round_up(spec, 256) * 2 + round_up(spec / 2, 256);   // acc, wz, wc
+    return bwd1d_layout(B, D, L, N, false, false).total;
 }
 
 size_t hyena_fftconv_backward_per_sample_workspace_size(int B, int D, int L, int N)
@@ -523,8 +545,7 @@ size_t hyena_fftconv_backward_per_sample_workspace_size(int B, int D, int L, int
     if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || check_len(L, kMaxLog2, &log2m) != HYENA_OK)
         return (size_t)-1;
     if (log2m > kMaxLog2Fused) return fourstep_bwd_layout(log2m, D, N, B).total;
-    const size_t spec = sizeof(float2) * (size_t)N * D * L;
-    return round_up(spec * B, 256) + round_up(spec, 256) + round_up(spec / 2, 256);   // acc, wz, wc
+    return bwd1d_layout(B, D, L, N, true, false).total;
 }
 
 hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, const float* H,
@@ -537,12 +558,13 @@ hyena_status_t hyena_fftconv_gate_backward(const void* v, const void* const* x, 
                          ws_bytes, stream);
 }
 
-size_t hyena_fftconv_backward_circular_workspace_size(int D, int L, int N)
+size_t hyena_fftconv_backward_circular_workspace_size(int B, int D, int L, int N)
 {
     const int k = exact_log2(L);
-    if (D < 1 || N < 1 || N > HYENA_MAX_ORDER || k < kMinLog2Circ + 1 || k > kMaxLog2) return (size_t)-1;
+    if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || k < kMinLog2Circ + 1 || k > kMaxLog2)
+        return (size_t)-1;
     if (k - 1 > kMaxLog2Circ) return fourstep_bwd_layout(k - 1, D, N, 1, true).total;   // four-step
-    return 3 * round_up(sizeof(float2) * (size_t)N * D * (L / 2), 256);   // acc, wz, wc
+    return bwd1d_layout(B, D, L, N, false, true).total;
 }
 
 hyena_status_t hyena_fftconv_gate_backward_circular(const void* v, const void* const* x, const float* H,
@@ -560,8 +582,7 @@ size_t hyena_fftconv_backward_circular_per_sample_workspace_size(int B, int D, i
     const int k = exact_log2(L);
     if (B < 1 || D < 1 || N < 1 || N > HYENA_MAX_ORDER || k < kMinLog2Circ + 1 || k > kMaxLog2) return (size_t)-1;
     if (k - 1 > kMaxLog2Circ) return fourstep_bwd_layout(k - 1, D, N, B, true).total;   // four-step
-    const size_t spec = sizeof(float2) * (size_t)N * D * (L / 2);
-    return round_up(spec * B, 256) + 2 * round_up(spec, 256);   // acc (per sample), wz, wc
+    return bwd1d_layout(B, D, L, N, true, true).total;
 }
 
 hyena_status_t hyena_fftconv_gate_backward_circular_per_sample(const void* v, const void* const* x,
@@ -615,9 +636,9 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
         !aligned(bias, 4) || !aligned(dbias, 4))
         return HYENA_ERR_INVALID_ARG;
     const size_t need = circular ? (per_sample ? hyena_fftconv_backward_circular_per_sample_workspace_size(B, D, L, N)
-                                               : hyena_fftconv_backward_circular_workspace_size(D, L, N))
+                                               : hyena_fftconv_backward_circular_workspace_size(B, D, L, N))
                         : per_sample ? hyena_fftconv_backward_per_sample_workspace_size(B, D, L, N)
-                                     : hyena_fftconv_backward_workspace_size(D, L, N);
+                                     : hyena_fftconv_backward_workspace_size(B, D, L, N);
     if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return HYENA_ERR_WORKSPACE;
     const size_t sets = per_sample ? (size_t)B : 1;           // spectrum sets and dh sets
 
@@ -643,7 +664,6 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
             if (overlap(out[o].p, out[o].n, out[p].p, out[p].n)) return HYENA_ERR_INVALID_ARG;
     }
 
-    const size_t spec = sizeof(float2) * (size_t)N * D * (circular ? L / 2 : L);   // one spectrum set
     char* ws = static_cast<char*>(workspace);
     cudaStream_t st = (cudaStream_t)stream;
     if (circular ? log2m > kMaxLog2Circ : log2m > kMaxLog2Fused) {
@@ -687,12 +707,14 @@ hyena_status_t backward_impl(const void* v, const void* const* x, const float* H
     a.dv = dv;
     a.dh = dh;
     a.dbias = dbias;
-    a.acc = reinterpret_cast<float2*>(ws);
-    a.wz = reinterpret_cast<float2*>(ws + round_up(spec * sets, 256));
-    a.wc = reinterpret_cast<float2*>(ws + round_up(spec * sets, 256) + round_up(spec, 256));   // [D][N][SEQ]
+    const Bwd1dLayout lay = bwd1d_layout(B, D, L, N, per_sample, circular);
+    a.acc = reinterpret_cast<float2*>(ws + lay.acc);
+    a.wz = reinterpret_cast<float2*>(ws + lay.wz);
+    a.wc = reinterpret_cast<float2*>(ws + lay.wc);
     a.B = B;
     a.D = D;
     a.N = N;
+    a.S = lay.slices;                        // the most batch slices the workspace holds
     a.H_bstride = per_sample ? (size_t)N * D * (circular ? L / 2 : L) : 0;
     if (circular && per_sample)
         return io == HYENA_BF16 ? dispatch_backward_circ_ps_bf16(log2m, a, st)

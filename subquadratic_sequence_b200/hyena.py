@@ -85,9 +85,9 @@ def _load() -> ctypes.CDLL:
         "hyena_dft32_stage": ([vp, vp, ctypes.c_long, i, i, vp], i),
         "hyena_fftconv_gate_forward_spill": ([vp, ctypes.POINTER(vp), vp, vp, i, i, i, i, i, vp, vp, sz,
                                               vp], i),
-        "hyena_fftconv_backward_workspace_size": ([i, i, i], sz),
+        "hyena_fftconv_backward_workspace_size": ([i, i, i, i], sz),
         "hyena_fftconv_backward_per_sample_workspace_size": ([i, i, i, i], sz),
-        "hyena_fftconv_backward_circular_workspace_size": ([i, i, i], sz),
+        "hyena_fftconv_backward_circular_workspace_size": ([i, i, i, i], sz),
         "hyena_fftconv_backward_circular_per_sample_workspace_size": ([i, i, i, i], sz),
         "hyena_fftconv_gate_backward_circular_per_sample": ([vp, ctypes.POINTER(vp), vp, vp, vp, i, i, i, i, i,
                                                              vp, ctypes.POINTER(vp), vp, vp, vp, sz, vp], i),
@@ -391,8 +391,8 @@ def hyena_fftconv_gate_forward_noalloc(v: torch.Tensor, xs, bias: torch.Tensor, 
 
 # ------------------------------------------------------------------ 2-D
 
-def hyena_fftconv_backward_workspace_size(D: int, L: int, N: int) -> int:
-    n = LIB.hyena_fftconv_backward_workspace_size(D, L, N)
+def hyena_fftconv_backward_workspace_size(B: int, D: int, L: int, N: int) -> int:
+    n = LIB.hyena_fftconv_backward_workspace_size(B, D, L, N)
     if n == ctypes.c_size_t(-1).value:
         raise HyenaError("hyena_fftconv_backward_workspace_size", HYENA_ERR_INVALID_ARG, "invalid sizes")
     return n
@@ -413,7 +413,7 @@ def hyena_fftconv_gate_backward(v: torch.Tensor, xs, bias: torch.Tensor, H: torc
     dh = torch.empty((N, D, L), device=v.device, dtype=torch.float32)
     db = torch.empty((N, D), device=v.device, dtype=torch.float32)
     if workspace is None:
-        workspace = torch.empty(hyena_fftconv_backward_workspace_size(D, L, N), device=v.device,
+        workspace = torch.empty(hyena_fftconv_backward_workspace_size(B, D, L, N), device=v.device,
                                 dtype=torch.uint8)
     _check("hyena_fftconv_gate_backward", LIB.hyena_fftconv_gate_backward(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),
@@ -458,8 +458,8 @@ def hyena_fftconv_gate_backward_per_sample(v: torch.Tensor, xs, bias: torch.Tens
     return dv, dxs, dh, db
 
 
-def hyena_fftconv_backward_circular_workspace_size(D: int, L: int, N: int) -> int:
-    n = LIB.hyena_fftconv_backward_circular_workspace_size(D, L, N)
+def hyena_fftconv_backward_circular_workspace_size(B: int, D: int, L: int, N: int) -> int:
+    n = LIB.hyena_fftconv_backward_circular_workspace_size(B, D, L, N)
     if n == ctypes.c_size_t(-1).value:
         raise HyenaError("hyena_fftconv_backward_circular_workspace_size", HYENA_ERR_UNSUPPORTED,
                          "invalid sizes (32 <= L <= 2^22)")
@@ -481,7 +481,7 @@ def hyena_fftconv_gate_backward_circular(v: torch.Tensor, xs, bias: torch.Tensor
     dh = torch.empty((N, D, L), device=v.device, dtype=torch.float32)
     db = torch.empty((N, D), device=v.device, dtype=torch.float32)
     if workspace is None:
-        workspace = torch.empty(hyena_fftconv_backward_circular_workspace_size(D, L, N), device=v.device,
+        workspace = torch.empty(hyena_fftconv_backward_circular_workspace_size(B, D, L, N), device=v.device,
                                 dtype=torch.uint8)
     _check("hyena_fftconv_gate_backward_circular", LIB.hyena_fftconv_gate_backward_circular(
         ctypes.c_void_p(_dev(v, v.dtype, "v")), xp, ctypes.c_void_p(_dev(H, torch.complex64, "H")),

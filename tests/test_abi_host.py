@@ -131,14 +131,19 @@ def bwd(lib, v=P(0), xs=(P(1), P(2)), H=P(3), bias=P(4), dy=P(5), B=2, D=3, L=64
 
 def test_backward_rejects_bad_arguments(lib):
     lib.hyena_fftconv_backward_workspace_size.restype = ctypes.c_size_t
-    lib.hyena_fftconv_backward_workspace_size.argtypes = [ctypes.c_int] * 3
-    need = lib.hyena_fftconv_backward_workspace_size(3, 64, 2)
-    assert need >= 20 * 2 * 3 * 64
+    lib.hyena_fftconv_backward_workspace_size.argtypes = [ctypes.c_int] * 4
+    need = lib.hyena_fftconv_backward_workspace_size(2, 3, 64, 2)
+    assert need >= 20 * 2 * 3 * 64 * 2                       # two batch slices
+    # the slices stop at 8: a larger batch needs no more
+    assert (lib.hyena_fftconv_backward_workspace_size(64, 3, 64, 2)
+            == lib.hyena_fftconv_backward_workspace_size(8, 3, 64, 2)
+            > lib.hyena_fftconv_backward_workspace_size(1, 3, 64, 2))
     # four-step lengths: the accumulated spectra plus the waves' saved spectra, c_n and scratch
-    long_need = lib.hyena_fftconv_backward_workspace_size(3, 1 << 15, 2)
+    long_need = lib.hyena_fftconv_backward_workspace_size(2, 3, 1 << 15, 2)
     assert long_need >= 8 * 2 * 3 * (1 << 15) + (64 << 20) and long_need % 256 == 0
-    assert lib.hyena_fftconv_backward_workspace_size(3, 1 << 23, 2) == ctypes.c_size_t(-1).value
-    assert lib.hyena_fftconv_backward_workspace_size(0, 64, 2) == ctypes.c_size_t(-1).value
+    assert lib.hyena_fftconv_backward_workspace_size(2, 3, 1 << 23, 2) == ctypes.c_size_t(-1).value
+    assert lib.hyena_fftconv_backward_workspace_size(2, 0, 64, 2) == ctypes.c_size_t(-1).value
+    assert lib.hyena_fftconv_backward_workspace_size(0, 3, 64, 2) == ctypes.c_size_t(-1).value
     for k in ("v", "H", "bias", "dy", "dv", "dh", "db"):
         assert bwd(lib, **{k: None}) == INVALID, k
     assert bwd(lib, xs=(P(1), None)) == INVALID
@@ -352,13 +357,14 @@ def test_backward_variants_reject_bad_arguments(lib):
     # per-sample: B dh spectra; any L up to 2^22
     ps = lib.hyena_fftconv_backward_per_sample_workspace_size
     assert ps(4, 3, 64, 2) >= 4 * 2 * 3 * 64 * 8 + 12 * 2 * 3 * 64
-    assert ps(4, 3, 1 << 15, 2) > lib.hyena_fftconv_backward_workspace_size(3, 1 << 15, 2)
+    assert ps(4, 3, 1 << 15, 2) > lib.hyena_fftconv_backward_workspace_size(4, 3, 1 << 15, 2)
     assert ps(4, 3, 1 << 23, 2) == bad and ps(0, 3, 64, 2) == bad
     # circular: 32 <= L <= 16384
     cs = lib.hyena_fftconv_backward_circular_workspace_size
-    assert cs(3, 64, 2) >= 12 * 2 * 3 * 64
-    assert cs(3, 16, 2) == bad and cs(3, 1 << 23, 2) == bad and cs(3, 96, 2) == bad
-    assert cs(3, 1 << 15, 2) > (64 << 20)                    # the four-step layout above 16384
+    assert cs(2, 3, 64, 2) >= 12 * 2 * 3 * 64 * 2
+    assert cs(2, 3, 16, 2) == bad and cs(2, 3, 1 << 23, 2) == bad and cs(2, 3, 96, 2) == bad
+    assert cs(0, 3, 64, 2) == bad
+    assert cs(2, 3, 1 << 15, 2) > (64 << 20)                 # the four-step layout above 16384
     xs = (ctypes.c_void_p * 2)(P(1).value, P(2).value)
     dxs = (ctypes.c_void_p * 2)(P(7).value, P(8).value)
     f = lib.hyena_fftconv_gate_backward_circular

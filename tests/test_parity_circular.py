@@ -135,7 +135,7 @@ def test_backward_circular_rejects_unsupported_lengths(hy):
     from subquadratic_sequence_b200.hyena import HyenaError
     for L in (16, 1 << 23):
         with pytest.raises(HyenaError):
-            hy.hyena_fftconv_backward_circular_workspace_size(4, L, 2)
+            hy.hyena_fftconv_backward_circular_workspace_size(2, 4, L, 2)
 
 
 # ------------------------------------------- long sequences (four-step)
