@@ -174,13 +174,27 @@ struct Fft1d {
         __syncthreads();
     }
 
-    // Middle pass: stride NS, radix R, plain column layout j = t + c*T.
-    // Column c's twiddle base is chained on column c-1's result so the
-    // twiddle arithmetic stays next to the data it multiplies.
-    template <int R, int NS, int SIGN>
+    // Exchange layouts.  The first pass writes at a stride of R elements,
+    // so its output is padded (element i at pad16(i)).  A middle pass reads
+    // and writes 16-element runs that start on a multiple of 16, which are
+    // conflict-free in either layout, and writes its output unpadded
+    // (element i at i).  The last pass reads the mirrored column NCOL - u of
+    // each folded unit: 16 consecutive elements starting one past a multiple
+    // of 16, which the padding would split across two 16-element lines (a
+    // two-way bank conflict in every half-warp but the first), and which
+    // are conflict-free unpadded.  So every pass after a middle pass reads
+    // unpadded.
+    static constexpr bool HAS_MID = P::RM1 > 1 || P::RM2 > 1;
+
+    // Middle pass: stride NS, radix R, plain column layout j = t + c*T;
+    // input padded (PLAIN_IN false) or not, output unpadded.  Column c's
+    // twiddle base is chained on column c-1's result so the twiddle
+    // arithmetic stays next to the data it multiplies.
+    template <int R, int NS, int SIGN, bool PLAIN_IN>
     static __device__ __forceinline__ void pass_mid(float2* a, float2* sm, int t)
     {
         if constexpr (R > 1) {
+            static_assert(NS % 16 == 0, "unpadded output: runs of 16 aligned to 16");
             constexpr int C = E / R;
             static_for<C>([&](auto cc) {
                 constexpr int c = decltype(cc)::value;
@@ -188,7 +202,7 @@ struct Fft1d {
                 const int pj = pad16(j);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    a[c * R + r] = sm[pad16_at<M / R>(j, pj, r)];
+                    a[c * R + r] = sm[PLAIN_IN ? j + r * (M / R) : pad16_at<M / R>(j, pj, r)];
                 });
             });
             __syncthreads();
@@ -201,10 +215,9 @@ struct Fft1d {
                 apply_twiddle_powers<R>(ar, expi_pi<SIGN>(2.0f * (float)jm / (float)(NS * R) + dep));
                 dft<R, SIGN>(ar);
                 const int base = (j / NS) * NS * R + jm;
-                const int pb = pad16(base);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    sm[pad16_at<NS>(base, pb, r)] = ar[r];
+                    sm[base + r * NS] = ar[r];
                 });
                 dep = zero_after(ar[R - 1].x);
             });
@@ -212,7 +225,8 @@ struct Fft1d {
         }
     }
 
-    // Last pass (Ns = M/R) into registers in folded layout.
+    // Last pass (Ns = M/R) into registers in folded layout; its input is
+    // unpadded when a middle pass wrote it.
     template <int R, int SIGN, bool HALF_OUT>
     static __device__ __forceinline__ void pass_last(float2* a, const float2* sm, int t)
     {
@@ -225,7 +239,7 @@ struct Fft1d {
                 const int pj = pad16(j[h]);
                 static_for<R>([&](auto rr) {
                     constexpr int r = decltype(rr)::value;
-                    a[(2 * c + h) * R + r] = sm[pad16_at<M / R>(j[h], pj, r)];
+                    a[(2 * c + h) * R + r] = sm[HAS_MID ? j[h] + r * (M / R) : pad16_at<M / R>(j[h], pj, r)];
                 });
             });
         });
@@ -251,8 +265,8 @@ struct Fft1d {
     static __device__ __forceinline__ void forward(float2* a, float2* sm, int t)
     {
         pass_first<P::RF, -1, PAD>(a, sm, t);
-        pass_mid<P::RM1, P::RF, -1>(a, sm, t);
-        pass_mid<P::RM2, P::RF * P::RM1, -1>(a, sm, t);
+        pass_mid<P::RM1, P::RF, -1, false>(a, sm, t);
+        pass_mid<P::RM2, P::RF * P::RM1, -1, (P::RM1 > 1)>(a, sm, t);
         pass_last<P::RL, -1, false>(a, sm, t);
     }
 
@@ -261,8 +275,8 @@ struct Fft1d {
     static __device__ __forceinline__ void inverse(float2* a, float2* sm, int t)
     {
         pass_first<P::RL, +1, false>(a, sm, t);
-        pass_mid<P::RM2, P::RL, +1>(a, sm, t);
-        pass_mid<P::RM1, P::RL * P::RM2, +1>(a, sm, t);
+        pass_mid<P::RM2, P::RL, +1, false>(a, sm, t);
+        pass_mid<P::RM1, P::RL * P::RM2, +1, (P::RM2 > 1)>(a, sm, t);
         pass_last<P::RF, +1, PAD>(a, sm, t);
     }
 
