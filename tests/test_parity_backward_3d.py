@@ -70,6 +70,8 @@ CASES = [
     (1, 2, 16, 16, 16, 2, "f32"), (2, 1, 16, 32, 64, 2, "f32"), (1, 2, 32, 16, 16, 3, "f32"),
     (2, 2, 16, 16, 32, 1, "bf16"), (1, 1, 64, 16, 16, 2, "f32"), (1, 1, 16, 64, 16, 2, "bf16"),
     (2, 1, 16, 16, 128, 1, "f32"), (1, 1, 16, 16, 16, 16, "f32"),
+    # the longest axes (256: 512-point z, column and row transforms)
+    (1, 1, 256, 16, 16, 1, "f32"), (1, 1, 16, 256, 16, 1, "f32"), (1, 1, 16, 16, 256, 2, "bf16"),
 ]
 
 

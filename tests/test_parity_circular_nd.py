@@ -326,6 +326,7 @@ def gpu_backward_3d_circular(hy, v, x, b, h, dy, io, per_sample=False):
 @pytest.mark.parametrize("B,C,Z,H,W,N,io", [
     (1, 2, 16, 16, 32, 2, "f32"), (2, 1, 32, 16, 64, 1, "f32"), (2, 2, 16, 32, 32, 2, "bf16"),
     (1, 1, 64, 16, 32, 3, "f32"), (2, 2, 16, 256, 64, 1, "f32"), (1, 1, 256, 16, 32, 1, "f32"),
+    (1, 1, 16, 16, 256, 2, "bf16"), (1, 1, 256, 256, 32, 1, "f32"),
 ])
 def test_backward_3d_circular_matches_oracle(hy, B, C, Z, H, W, N, io):
     v, x, b, h = problem(B, C, (Z, H, W), N, seed=Z + 2 * H + 5 * W + N)
