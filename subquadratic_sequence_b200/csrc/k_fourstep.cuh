@@ -45,7 +45,7 @@ hyena_status_t dispatch_fourstep(int log2m, const FourStepArgs& a, int N, float2
     case 15: return run_fourstep<7, 8, IO>(a, N, scratch, st);
     case 16: return run_fourstep<8, 8, IO>(a, N, scratch, st);
     case 17: return run_fourstep<8, 9, IO>(a, N, scratch, st);
-    case 18: return run_fourstep<9, 9, IO>(a, N, scratch, st);
+    case 18: return run_fourstep<8, 10, IO>(a, N, scratch, st);
     case 19: return run_fourstep<9, 10, IO>(a, N, scratch, st);
     case 20: return run_fourstep<10, 10, IO>(a, N, scratch, st);
     case 21: return run_fourstep<10, 11, IO>(a, N, scratch, st);

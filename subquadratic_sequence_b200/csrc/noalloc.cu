@@ -97,7 +97,7 @@ hyena_status_t run_long(int log2m, const FourStepArgs& a, int N, float2* scratch
     case 15: return run_waves<7, 8, IO>(a, N, scratch, st);
     case 16: return run_waves<8, 8, IO>(a, N, scratch, st);
     case 17: return run_waves<8, 9, IO>(a, N, scratch, st);
-    case 18: return run_waves<9, 9, IO>(a, N, scratch, st);
+    case 18: return run_waves<8, 10, IO>(a, N, scratch, st);
     case 19: return run_waves<9, 10, IO>(a, N, scratch, st);
     case 20: return run_waves<10, 10, IO>(a, N, scratch, st);
     case 21: return run_waves<10, 11, IO>(a, N, scratch, st);
