@@ -106,7 +106,7 @@ hyena_status_t dispatch_fourstep_bwd(int log2m, const FourStepBwdArgs& a, int N,
     case 15: return run_fourstep_bwd<7, 8, IO>(a, N, st);
     case 16: return run_fourstep_bwd<8, 8, IO>(a, N, st);
     case 17: return run_fourstep_bwd<8, 9, IO>(a, N, st);
-    case 18: return run_fourstep_bwd<9, 9, IO>(a, N, st);
+    case 18: return run_fourstep_bwd<8, 10, IO>(a, N, st);
     case 19: return run_fourstep_bwd<9, 10, IO>(a, N, st);
     case 20: return run_fourstep_bwd<10, 10, IO>(a, N, st);
     case 21: return run_fourstep_bwd<10, 11, IO>(a, N, st);
@@ -122,7 +122,7 @@ inline FourStepBwdLayout fourstep_bwd_layout(int log2m, int D, int N, int sets =
     case 15: return fourstep_bwd_layout_n<7, 8>(D, N, sets, circular);
     case 16: return fourstep_bwd_layout_n<8, 8>(D, N, sets, circular);
     case 17: return fourstep_bwd_layout_n<8, 9>(D, N, sets, circular);
-    case 18: return fourstep_bwd_layout_n<9, 9>(D, N, sets, circular);
+    case 18: return fourstep_bwd_layout_n<8, 10>(D, N, sets, circular);
     case 19: return fourstep_bwd_layout_n<9, 10>(D, N, sets, circular);
     case 20: return fourstep_bwd_layout_n<10, 10>(D, N, sets, circular);
     case 21: return fourstep_bwd_layout_n<10, 11>(D, N, sets, circular);
@@ -139,7 +139,7 @@ hyena_status_t dispatch_fourstep_bwd_circ(int log2m, const FourStepBwdArgs& a, i
     case 15: return run_fourstep_bwd<7, 8, IO, false>(a, N, st);
     case 16: return run_fourstep_bwd<8, 8, IO, false>(a, N, st);
     case 17: return run_fourstep_bwd<8, 9, IO, false>(a, N, st);
-    case 18: return run_fourstep_bwd<9, 9, IO, false>(a, N, st);
+    case 18: return run_fourstep_bwd<8, 10, IO, false>(a, N, st);
     case 19: return run_fourstep_bwd<9, 10, IO, false>(a, N, st);
     case 20: return run_fourstep_bwd<10, 10, IO, false>(a, N, st);
     case 21: return run_fourstep_bwd<10, 11, IO, false>(a, N, st);
